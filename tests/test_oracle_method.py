@@ -1,0 +1,305 @@
+"""Pins of the oracle's CSA2 steps: the pages' figures, closed forms, invariants, brute force.
+
+CPU only.  Brute-force references here are written with plain Python loops so
+that a dropped term, a wrong sign or index, or a transposed operand in the
+oracle's vectorised code fails one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import csa2 as C
+from oracle import formats as F
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(11)
+
+
+def golden():
+    return json.load(open(os.path.join(GOLDEN, "byte_accounting.json")))
+
+
+# ----------------------------------------------------------------- the pages' figures
+def test_layer_schedule_matches_pages():
+    g = golden()["layer_schedule"]
+    modes = [C.layer_mode(i) for i in range(C.NUM_LAYERS)]
+    assert len(modes) == g["num_layers"]
+    assert [i for i, m in enumerate(modes) if m == "swa"] == g["swa_only"]
+    assert [i for i, m in enumerate(modes) if m == "full"] == g["full"]
+    assert [i for i, m in enumerate(modes) if m == "reindex"] == g["reindex"]
+    assert modes.count("reuse") == g["reuse_count"]
+
+
+def test_entries_and_bytes_per_token():
+    g = golden()
+    enc = sum(1.0 / r for l, r in C.FULL_LAYERS.items() if l < 20)
+    dec = sum(1.0 / r for l, r in C.FULL_LAYERS.items() if l >= 20)
+    assert enc == g["entries_per_token"]["encoder"]
+    assert dec == g["entries_per_token"]["decoder"]
+    assert C.entries_per_token() == g["entries_per_token"]["total"]
+    assert C.global_kv_bytes_per_token() == g["global_kv_bytes_per_token"]["v4_1_flash"]
+
+
+def test_global_kv_at_one_million_tokens():
+    g = golden()["global_kv_at_1m_context_gib"]
+    gib = C.global_kv_bytes_per_token() * 2 ** 20 / 2 ** 30
+    assert round(gib, g["printed_digits"]) == g["value"]
+    # "1M" must be 2^20 here: 10^6 tokens would print 0.83
+    assert round(C.global_kv_bytes_per_token() * 1e6 / 2 ** 30, 2) != g["value"]
+
+
+def test_about_a_quarter_of_v4():
+    g = golden()["global_kv_bytes_per_token"]
+    assert 3.9 < g["v4_flash"] / C.global_kv_bytes_per_token() < 4.0
+
+
+# ----------------------------------------------------------------- compressor
+def test_compressor_ratio_one_is_identity():
+    x = RNG.normal(size=(13, 8)).astype(np.float32)
+    np.testing.assert_array_equal(C.compress(x, 1), x)
+
+
+@pytest.mark.parametrize("r", [2, 4])
+def test_compressor_mean_of_identical_rows(r):
+    row = RNG.normal(size=(1, 16)).astype(np.float32)
+    x = np.repeat(row, 3 * r + 1, axis=0)           # ragged tail of one token
+    out = C.compress(x, r)
+    assert out.shape[0] == 3                         # incomplete group makes no entry
+    np.testing.assert_array_equal(out, np.repeat(row, 3, axis=0))
+
+
+def test_compressor_weighted_sum_brute_force():
+    x = RNG.normal(size=(9, 5)).astype(np.float32)
+    w = RNG.uniform(size=9).astype(np.float32)
+    out = C.compress(x, 3, w)
+    for j in range(3):
+        for d in range(5):
+            acc = np.float32(w[3 * j] * x[3 * j, d])
+            for t in (3 * j + 1, 3 * j + 2):
+                acc = np.float32(acc + np.float32(w[t] * x[t, d]))
+            assert out[j, d] == acc
+
+
+def test_prefill_entry_count():
+    # a 262144-token prefix plus an 8192-token chunk at ratio 2
+    assert 262144 // 2 == 131072 and 8192 // 2 == 4096
+
+
+# ----------------------------------------------------------------- indexer
+def brute_scores(q_ix, w, keys):
+    qh = C.quantised_query(q_ix)
+    out = []
+    for k in keys.tolist():
+        s = 0.0
+        for h in range(len(w)):
+            dot = 0.0
+            for i in range(len(k)):
+                dot += float(qh[h][i]) * k[i]
+            s += float(w[h]) * (dot if dot > 0 else 0.0)
+        out.append(s)
+    return np.array(out)
+
+
+def test_indexer_score_brute_force():
+    H, n = 5, 11
+    q = RNG.normal(size=(H, 128)).astype(np.float32)
+    w = RNG.uniform(-0.5, 1, size=H).astype(np.float32)
+    c, s = F.pack_indexer(RNG.normal(size=(n, 128)).astype(np.float32))
+    keys = F.unpack_indexer(c, s)
+    np.testing.assert_allclose(C.indexer_scores(q, w, keys), brute_scores(q, w, keys), rtol=1e-12, atol=1e-12)
+
+
+def test_indexer_query_is_mxfp4_quantised():
+    q = RNG.normal(size=(3, 128)).astype(np.float32)
+    qh = C.quantised_query(q)
+    assert not np.array_equal(qh, q.astype(np.float64))
+    # every per-32 block of q^ is an e2m1 multiple of one power of two
+    for h in range(3):
+        for b in range(4):
+            blk = qh[h, 32 * b:32 * b + 32]
+            e = int(np.ceil(np.log2(np.float32(np.max(np.abs(q[h, 32 * b:32 * b + 32]))) / np.float32(6))))
+            np.testing.assert_array_equal(np.isin(np.abs(blk) / 2.0 ** e, F.E2M1_MAGNITUDES), True)
+
+
+def test_topk_invariant_under_positive_weight_rescale():
+    H, n = 8, 300
+    q = RNG.normal(size=(H, 128)).astype(np.float32)
+    w = RNG.uniform(size=H).astype(np.float32)
+    c, s = F.pack_indexer(RNG.normal(size=(n, 128)).astype(np.float32))
+    keys = F.unpack_indexer(c, s)
+    a = C.topk(C.indexer_scores(q, w, keys), 17)
+    b = C.topk(C.indexer_scores(q, w * np.float32(4), keys), 17)
+    np.testing.assert_array_equal(a, b)
+
+
+# ----------------------------------------------------------------- top-k
+def brute_topk(scores, k, n_valid=None):
+    n = len(scores) if n_valid is None else n_valid
+    cand = [j for j in range(n) if scores[j] != -math.inf]
+    sel = []
+    for i in cand:
+        rank = sum(1 for j in cand if scores[j] > scores[i] or (scores[j] == scores[i] and j < i))
+        if rank < k:
+            sel.append(i)
+    return sorted(sel) + [-1] * (k - len(sel))
+
+
+@pytest.mark.parametrize("case", range(6))
+def test_topk_against_rank_definition(case):
+    rng = np.random.default_rng(100 + case)
+    n = int(rng.integers(1, 60))
+    s = rng.integers(-3, 4, size=n).astype(np.float64)     # many ties
+    s[rng.uniform(size=n) < 0.1] = -math.inf
+    k = int(rng.integers(1, 70))
+    nv = int(rng.integers(0, n + 1))
+    np.testing.assert_array_equal(C.topk(s, k, nv), brute_topk(s, k, nv))
+    np.testing.assert_array_equal(C.topk(s, k), brute_topk(s, k))
+
+
+def test_topk_equals_full_sort():
+    s = RNG.normal(size=5000)
+    want = np.sort(np.argsort(-s, kind="stable")[:512])
+    np.testing.assert_array_equal(C.topk(s, 512), want)
+
+
+# ----------------------------------------------------------------- attention
+def brute_attend(q, keys, tau):
+    H = len(q)
+    o, lse = [], []
+    for h in range(H):
+        logits = [tau * sum(a * b for a, b in zip(q[h], k)) for k in keys]
+        m = max(logits)
+        e = [math.exp(x - m) for x in logits]
+        z = sum(e)
+        o.append([sum(e[j] * keys[j][d] for j in range(len(keys))) / z for d in range(len(q[h]))])
+        lse.append(m + math.log(z))
+    return np.array(o), np.array(lse)
+
+
+def test_attend_brute_force():
+    q = RNG.normal(size=(3, 6))
+    keys = RNG.normal(size=(7, 6))
+    o, lse = C.attend(q, keys, 0.7)
+    bo, bl = brute_attend(q.tolist(), keys.tolist(), 0.7)
+    np.testing.assert_allclose(o, bo, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, bl, rtol=1e-12, atol=1e-12)
+
+
+def test_attend_empty_set():
+    o, lse = C.attend(np.ones((2, 4)), np.zeros((0, 4)), 1.0)
+    assert not o.any() and np.all(lse == -math.inf)
+
+
+def _tiny_cache(n_tokens, ratio, B=1, seed=5):
+    rng = np.random.default_rng(seed)
+    cache = C.Cache(B, n_tokens // ratio + 4, ratio)
+    for b in range(B):
+        kv = rng.normal(size=(n_tokens, 512)).astype(np.float32)
+        ix = rng.normal(size=(n_tokens, 128)).astype(np.float32)
+        cache.num_entries[b] = cache.pack(b, 0, kv, ix)
+    return cache, rng
+
+
+def test_sparse_equals_dense_when_k_covers_everything():
+    cache, rng = _tiny_cache(80, 2)
+    q = rng.normal(size=(4, 512))
+    q_ix = rng.normal(size=(4, 128)).astype(np.float32)
+    w = rng.uniform(size=4).astype(np.float32)
+    pos = 79
+    idx, _, _ = C.full_select(cache, 0, pos, q_ix, w, k=64)
+    assert (idx[:40] == np.arange(40)).all() and (idx[40:] == -1).all()
+    o, lse = C.sparse_attention(cache, 0, q, idx, 0.05)
+    od, ld = C.attend(q, cache.main_values(0, np.arange(40)), 0.05)
+    np.testing.assert_allclose(o, od, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, ld, rtol=1e-12)
+
+
+def test_full_respects_causality():
+    cache, rng = _tiny_cache(100, 2)
+    q_ix = rng.normal(size=(4, 128)).astype(np.float32)
+    w = rng.uniform(size=4).astype(np.float32)
+    for pos in (0, 1, 2, 17, 60):
+        idx, _, _ = C.full_select(cache, 0, pos, q_ix, w, k=8)
+        sel = idx[idx >= 0]
+        assert len(sel) == min(8, (pos + 1) // 2)
+        assert (sel < (pos + 1) // 2).all()
+
+
+def test_reuse_equals_full_and_reindex_invariants():
+    cache, rng = _tiny_cache(600, 1)
+    q = rng.normal(size=(4, 512))
+    q_ix = rng.normal(size=(4, 128)).astype(np.float32)
+    w = rng.uniform(size=4).astype(np.float32)
+    swa_c, swa_s = F.pack_swa(rng.normal(size=(128, 512)).astype(np.float32))
+    pos = 599
+    full = C.decode_layer("full", cache, 0, pos, q, 0.04, (swa_c, swa_s), q_ix=q_ix, w=w, k=32, pool_k=128)
+    reuse = C.decode_layer("reuse", cache, 0, pos, q, 0.04, (swa_c, swa_s), idx=full["idx"])
+    np.testing.assert_array_equal(full["o"], reuse["o"])
+    np.testing.assert_array_equal(full["lse"], reuse["lse"])
+    pool = full["pool"]
+    assert set(full["idx"].tolist()) <= set(pool.tolist())
+    # Reindex with the Full layer's own query re-finds the Full layer's top-k
+    ri, _ = C.reindex_select(cache, 0, pos, q_ix, w, 32, pool)
+    np.testing.assert_array_equal(ri, full["idx"])
+    # Reindex with a fresh query stays inside the pool
+    q2 = rng.normal(size=(4, 128)).astype(np.float32)
+    ri2, _ = C.reindex_select(cache, 0, pos, q2, w, 32, pool)
+    assert set(ri2.tolist()) <= set(pool.tolist())
+    # with the pool = every visible entry, Reindex == Full
+    allpool = np.arange(600)
+    ri3, _ = C.reindex_select(cache, 0, pos, q2, w, 32, allpool)
+    f3, _, _ = C.full_select(cache, 0, pos, q2, w, 32)
+    np.testing.assert_array_equal(ri3, f3)
+
+
+def test_merge_equals_one_softmax_over_union():
+    q = RNG.normal(size=(3, 16))
+    k1 = RNG.normal(size=(5, 16))
+    k2 = RNG.normal(size=(9, 16))
+    o1, l1 = C.attend(q, k1, 0.3)
+    o2, l2 = C.attend(q, k2, 0.3)
+    o, lse = C.merge(o1, l1, o2, l2)
+    ou, lu = C.attend(q, np.concatenate([k1, k2]), 0.3)
+    np.testing.assert_allclose(o, ou, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, lu, rtol=1e-12)
+    ob, lb = C.merge(o2, l2, o1, l1)
+    np.testing.assert_allclose(o, ob, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse, np.log(np.exp(l1) + np.exp(l2)), rtol=1e-12)
+
+
+def test_merge_with_an_empty_side():
+    q = RNG.normal(size=(2, 8))
+    k = RNG.normal(size=(4, 8))
+    o1, l1 = C.attend(q, k, 1.0)
+    oe, le = C.attend(q, np.zeros((0, 8)), 1.0)
+    o, lse = C.merge(o1, l1, oe, le)
+    np.testing.assert_array_equal(o, o1)
+    np.testing.assert_array_equal(lse, l1)
+    o, lse = C.merge(oe, le, oe, le)
+    assert not o.any() and np.all(lse == -math.inf)
+
+
+def test_swa_equals_dense_over_last_window():
+    rng = np.random.default_rng(9)
+    R, W = 160, 128
+    x = rng.normal(size=(400, 512)).astype(np.float32)
+    codes = np.zeros((R, 512), np.uint8)
+    scale = np.zeros(R, np.float32)
+    pos = 377
+    for t in range(pos - R + 1, pos + 1):                # ring holds the last R tokens
+        codes[t % R], scale[t % R] = F.pack_swa(x[t])
+    q = rng.normal(size=(2, 512))
+    o, lse = C.swa_attention(q, pos, codes, scale, W, 0.05)
+    keys = []
+    for t in range(pos - W + 1, pos + 1):
+        c, s = F.pack_swa(x[t])
+        keys.append([float(F.e4m3_decode(np.uint8(v))) * float(s) for v in c.tolist()])
+    bo, bl = brute_attend(q.tolist(), keys, 0.05)
+    np.testing.assert_allclose(o, bo, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(lse, bl, rtol=1e-12)
+    # at the start of a sequence the window is shorter
+    o0, _ = C.swa_attention(q, 0, codes[[0] * R], scale[[0] * R], W, 0.05)
+    np.testing.assert_allclose(o0, np.repeat(F.unpack_swa(codes[:1], scale[:1]), 2, 0), rtol=1e-12)
