@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""CSA2 decode benchmark: query-tokens/s per CSA2 layer on the hierarchical 1M-context workload.
+
+One step = one decode token for each of the 8 sequences through one Full layer
+and four Reindex layers over a 2^20-entry FP4 global KV cache:
+  pack the token's global KV entry (main + indexer) and its SWA entry per layer,
+  Full layer: indexer scan of all 2^20 entries, top-16384 pool + top-512,
+              sparse attention, SWA attention, log-sum-exp merge,
+  each Reindex layer: indexer over the pool, top-512, sparse attention, SWA, merge.
+value = 8 tokens x 5 layers / step time (device-resident inputs, CUDA events).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl csa2|reference]
+Under torchrun each rank runs its own 8 sequences (weak scaling, no collective
+on the data path); timing is the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode query-tokens/s per CSA2 layer at 64K–1M ctx; indexer+gather HBM GB/s vs peak"
+UNIT = "query-tokens/s/layer"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["csa2", "reference"], default="csa2")
+    ap.add_argument("--workload", default="hier1m")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-seqs", type=int, default=1)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.dev = device_index
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(device_index)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- the workload on the GPU
+class Hier1M:
+    """Device state of the hierarchical Full -> Reindex decode workload."""
+
+    LAYERS = 5   # one Full layer, four Reindex layers
+
+    def __init__(self, spec, dev):
+        import compressed_sparse_attention_score_b200 as k
+        from workloads import configs as W
+        self.k, self.spec, self.dev = k, spec, dev
+        B, N = spec.B, spec.entries(0)
+        self.B, self.N = B, N
+        self.cache = k.GlobalKVCache(B, spec.ratio, seq_stride=N)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        zero = torch.zeros(1, dtype=torch.int32, device=dev)
+        for b in range(B):
+            kv, ix = W.token_latents(spec, b, dev)
+            k.csa2_pack_kv(kv[None].contiguous(), ix[None].contiguous(), zero, self.cache.seq_view(b), err=err)
+            del kv, ix
+        self.cache.num_entries.fill_(N)
+        torch.cuda.synchronize()
+        # per-step inputs (device-resident copies; the e2e run refills them from pinned host memory)
+        L = self.LAYERS
+        self.new_kv = torch.empty((B, 1, 512), dtype=torch.bfloat16, device=dev)
+        self.new_ix = torch.empty((B, 1, 128), dtype=torch.bfloat16, device=dev)
+        kv_last, ix_last = [], []
+        for b in range(B):
+            kv, ix = W.token_latents(spec, b, dev, start=N - 1, stop=N)
+            kv_last.append(kv)
+            ix_last.append(ix)
+        self.new_kv.copy_(torch.stack(kv_last))
+        self.new_ix.copy_(torch.stack(ix_last))
+        self.first_entry = torch.full((B,), N - 1, dtype=torch.int32, device=dev)
+        qs = [W.query_tensors(spec, layer, dev) for layer in range(L)]
+        self.q = torch.stack([t[0] for t in qs])          # [L][B][1][64][512]
+        self.q_ix = torch.stack([t[1] for t in qs])       # [L][B][1][64][128]
+        self.w = torch.stack([t[2] for t in qs])          # [L][B][1][64]
+        self.q_pos = qs[0][3]                             # [B][1]
+        self.R = 128
+        self.swa_codes = torch.zeros((L, B, self.R, 512), dtype=torch.uint8, device=dev)
+        self.swa_scale = torch.zeros((L, B, self.R), dtype=torch.float32, device=dev)
+        self.swa_new = torch.empty((L, B, 1, 512), dtype=torch.bfloat16, device=dev)
+        for layer in range(L):
+            x, pos = W.swa_tokens(spec, layer, dev)
+            k.csa2_pack_swa(x, pos, self.swa_codes[layer], self.swa_scale[layer], err=err)
+            self.swa_new[layer].copy_(x[:, -1:, :])
+        self.swa_pos = self.q_pos.contiguous()
+        # outputs and scratch
+        self.o = torch.empty((L, B, 1, 64, 512), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((L, B, 1, 64), dtype=torch.float32, device=dev)
+        self.o_swa = torch.empty((B, 1, 64, 512), dtype=torch.float32, device=dev)
+        self.l_swa = torch.empty((B, 1, 64), dtype=torch.float32, device=dev)
+        self.scores = torch.empty((B, 1, N), dtype=torch.float32, device=dev)
+        self.pool = torch.empty((B, 1, spec.pool_k), dtype=torch.int32, device=dev)
+        self.idx = torch.empty((B, 1, spec.k), dtype=torch.int32, device=dev)
+        self.ws_reindex = torch.empty(k.csa2_workspace_size("reindex", B, 1, N, spec.k, spec.pool_k),
+                                      dtype=torch.uint8, device=dev)
+        self.err = err
+        torch.cuda.synchronize()
+        assert k.csa2_check(err) == 0
+
+    # kernels launched per step, by call: pack_kv 1, pack_swa 1 per layer, index_score 1, top-k 2 (Full) / 1,
+    # sparse attention 1, SWA attention 1, merge 1 per layer
+    def launches_per_step(self):
+        return 1 + self.LAYERS * 1 + (1 + 2) + (self.LAYERS - 1) * 2 + self.LAYERS * 3
+
+    def step(self, scan_events=None):
+        k, s = self.k, self.spec
+        k.csa2_pack_kv(self.new_kv, self.new_ix, self.first_entry, self.cache, err=self.err)
+        for layer in range(self.LAYERS):
+            k.csa2_pack_swa(self.swa_new[layer], self.swa_pos, self.swa_codes[layer], self.swa_scale[layer],
+                            err=self.err)
+            q, q_ix, w = self.q[layer], self.q_ix[layer], self.w[layer]
+            if layer == 0:
+                if scan_events:
+                    scan_events[0].record()
+                k.csa2_index_score(q_ix, w, self.q_pos, self.cache, self.N, scores=self.scores, err=self.err)
+                if scan_events:
+                    scan_events[1].record()
+                k.csa2_topk(self.scores, s.pool_k, idx=self.pool, val=None)
+                k.csa2_topk(self.scores, s.k, idx=self.idx, val=None)
+                o1, l1 = k.csa2_sparse_attn("reuse", q, self.q_pos, self.cache, s.tau, self.N, k=s.k,
+                                            idx_in=self.idx, o=self.o[layer], lse=self.lse[layer], err=self.err)
+            else:
+                o1, l1 = k.csa2_sparse_attn("reindex", q, self.q_pos, self.cache, s.tau, self.N, k=s.k, q_ix=q_ix,
+                                            w=w, pool_k=s.pool_k, pool_io=self.pool, idx_out=self.idx,
+                                            o=self.o[layer], lse=self.lse[layer], ws=self.ws_reindex,
+                                            err=self.err)
+            k.csa2_swa_attn(q, self.q_pos, self.swa_codes[layer], self.swa_scale[layer], s.tau, o=self.o_swa,
+                            lse=self.l_swa, err=self.err)
+            k.csa2_merge(self.o[layer], self.lse[layer], self.o_swa, self.l_swa, o=self.o[layer],
+                         lse=self.lse[layer])
+
+    def host_io(self):
+        """Pinned host copies of one step's inputs and outputs (for the end-to-end run)."""
+        ins = [self.new_kv, self.new_ix, self.q, self.q_ix, self.w, self.swa_new]
+        outs = [self.o, self.lse]
+        h_in = [t.cpu().pin_memory() for t in ins]
+        h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+        return ins, h_in, outs, h_out
+
+    def scan_bytes(self):
+        """Algorithmic bytes of one Full-layer indexer launch: every key read once, one fp32 score written."""
+        return self.B * self.N * (68 + 4) + self.B * 64 * (128 * 2 + 2)
+
+
+def source_sha(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_sources, name):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m = re.search(r"source_sha:\s*([0-9a-f]+)", txt)
+    t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not m or not t or m.group(1) != source_sha(kernel_sources):
+        return None
+    return float(t.group(1))
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- the oracle's time (CPU baseline)
+def oracle_time(spec, n_seqs=1):
+    """Time the oracle, as it stands, on `n_seqs` sequences of one decode step (all five layers)."""
+    import numpy as np
+    from oracle import csa2 as OC
+    from oracle import formats as OF
+    from workloads import configs as W
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    total = 0.0
+    for b in range(n_seqs):
+        kv, ix = W.token_latents(spec, b, "cpu")
+        n = spec.entries(b)
+        c = OC.Cache(1, n, spec.ratio)
+        c.num_entries[0] = n
+        c.ix_codes[0], c.ix_scales[0] = OF.pack_indexer(ix.float().numpy())
+        qs = [W.query_tensors(spec, layer, "cpu") for layer in range(5)]
+        swa = []
+        for layer in range(5):
+            x, pos = W.swa_tokens(spec, layer, "cpu")
+            codes, sc = OF.pack_swa(x[b].float().numpy())
+            ring_c = np.zeros((128, 512), np.uint8)
+            ring_s = np.zeros(128, np.float32)
+            p = pos[b].numpy()
+            ring_c[p % 128], ring_s[p % 128] = codes, sc
+            swa.append((ring_c, ring_s))
+        kvn = kv.float().numpy()
+
+        def run():
+            pos = spec.tokens[b] - 1
+            t0 = time.perf_counter()
+            out = OC.decode_layer("full", c, 0, pos, qs[0][0][b, 0].float().numpy(), spec.tau, swa[0],
+                                  q_ix=qs[0][1][b, 0].float().numpy(), w=qs[0][2][b, 0].float().numpy(),
+                                  k=spec.k, pool_k=spec.pool_k)
+            rows = [out["idx"]]
+            for layer in range(1, 5):
+                r = OC.decode_layer("reindex", c, 0, pos, qs[layer][0][b, 0].float().numpy(), spec.tau,
+                                    swa[layer], q_ix=qs[layer][1][b, 0].float().numpy(),
+                                    w=qs[layer][2][b, 0].float().numpy(), k=spec.k, pool=out["pool"])
+                rows.append(r["idx"])
+            return time.perf_counter() - t0, rows
+
+        # untimed: put the main entries the step will read into the oracle cache
+        _, rows = run()
+        need = np.unique(np.concatenate(rows))
+        need = need[need >= 0]
+        c.kv_codes[0, need], c.kv_scales[0, need] = OF.pack_main(kvn[need])
+        dt, _ = run()
+        total += dt
+    return total, cores
+
+
+# ---------------------------------------------------------------- main
+def run_reference(args, world, rank):
+    from workloads import configs as W
+    if rank != 0:
+        return
+    spec = W.CONFIGS[args.workload]()
+    n = args.cpu_sample_seqs
+    times = []
+    for _ in range(args.warmup + args.steps):
+        dt, cores = oracle_time(spec, n)
+        times.append(dt)
+    t = sum(times[args.warmup:]) / max(1, args.steps)
+    value = n * 5 / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(spec),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{n} of {spec.B} sequences, one decode step through all 5 layers"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(spec):
+    return {"workload": f"{spec.name}: hierarchical Full->Reindex decode, batch {spec.B}, "
+                        f"{spec.entries(0)} entries/seq at ratio {spec.ratio}, 1 Full + 4 Reindex layers",
+            "batch": spec.B, "ctx_entries": spec.entries(0), "ratio": spec.ratio, "top_k": spec.k,
+            "pool_k": spec.pool_k, "heads": 64, "indexer_heads": 64, "swa_window": 128,
+            "layers_per_step": 5, "parallelism": "dp (independent sequences per rank)",
+            "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write, outside step events)"}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    import compressed_sparse_attention_score_b200  # noqa: F401  (fails loudly without the library)
+    from workloads import configs as W
+    dev = torch.device("cuda", torch.cuda.current_device())
+    spec = W.CONFIGS[args.workload](seed=rank)
+    assert spec.name == "hier1m", "bench.py times the hierarchical 1M-context decode workload"
+    wl = Hier1M(spec, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+    assert wl.k.csa2_check(wl.err) == 0
+
+    # ---- device-resident timing
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index)
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        wl.step(scan_events=sev[i])
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    step_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    scan_ms = sum(a.elapsed_time(b) for a, b in sev) / args.steps
+    step_ms = max_over_ranks(step_ms, world)
+    units = world * wl.B * wl.LAYERS
+    value = units / (step_ms * 1e-3)
+
+    # ---- end to end through the C ABI with host buffers
+    ins, h_in, outs, h_out = wl.host_io()
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        eev[i][0].record(stream)
+        for d, h in zip(ins, h_in):
+            d.copy_(h, non_blocking=True)
+        wl.step()
+        for h, d in zip(h_out, outs):
+            h.copy_(d, non_blocking=True)
+        eev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev) / args.steps, world)
+    assert wl.k.csa2_check(wl.err) == 0
+
+    peak, peak_kind = peaks()
+    achieved = wl.scan_bytes() / (scan_ms * 1e-3) / 1e9
+    traffic = profiled_traffic(["compressed_sparse_attention_score_b200/csrc/index_score.cu"],
+                               "index_score_hier1m.md")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded N(0,1) latents and queries)",
+            "config": config_dict(spec),
+            "roofline": {"bound": "hbm", "kernel": "csa2 indexer scan (Full layer)", "achieved": achieved,
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic, "scan_ms": scan_ms,
+                         "entries_scanned_per_s": wl.B * wl.N / (scan_ms * 1e-3)},
+            "e2e": {"value": units / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": wl.launches_per_step() * args.steps,
+            "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        del wl
+        torch.cuda.empty_cache()
+        dt, cores = oracle_time(spec, args.cpu_sample_seqs)
+        line["cpu_baseline"] = {"value": args.cpu_sample_seqs * 5 / dt, "unit": UNIT, "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"{args.cpu_sample_seqs} of {spec.B} sequences, one decode step "
+                                          f"through all 5 layers (Full scan of {spec.entries(0)} keys)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,187 @@
+// The C ABI of the CSA2 library: argument checks, workspace carving, launches.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <string>
+
+#include "../../include/csa2.h"
+#include "kernels.cuh"
+
+#define CSA2_EXPORT extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+thread_local std::string g_last_error;
+
+csa2_status fail(csa2_status s, const char *msg) {
+  g_last_error = msg;
+  return s;
+}
+
+csa2_status launched(const char *what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+    return CSA2_ERR_CUDA;
+  }
+  g_last_error.clear();
+  return CSA2_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+csa2_status check_cache(const csa2_cache *c, int B) {
+  if (!c) return fail(CSA2_ERR_INVALID_ARG, "cache is NULL");
+  if (!c->kv_codes || !c->kv_scales || !c->ix_codes || !c->ix_scales || !c->num_entries)
+    return fail(CSA2_ERR_INVALID_ARG, "cache plane or num_entries is NULL");
+  if (!aligned16(c->kv_codes) || !aligned16(c->ix_codes) || !aligned16(c->kv_scales) || (reinterpret_cast<uintptr_t>(c->ix_scales) & 3))
+    return fail(CSA2_ERR_INVALID_ARG, "cache planes must be 16-byte aligned (ix_scales 4-byte)");
+  if (c->ratio < 1) return fail(CSA2_ERR_INVALID_ARG, "cache ratio must be >= 1");
+  if (c->num_slots < 0 || c->batch < 0) return fail(CSA2_ERR_INVALID_ARG, "negative cache size");
+  if (B > c->batch) return fail(CSA2_ERR_SHAPE, "B exceeds cache batch");
+  if (c->page_table) {
+    if (c->page_size <= 0 || (c->page_size & (c->page_size - 1)) || c->max_pages <= 0)
+      return fail(CSA2_ERR_INVALID_ARG, "paged cache needs a power-of-two page_size and max_pages > 0");
+  } else if (c->seq_stride <= 0) {
+    return fail(CSA2_ERR_INVALID_ARG, "contiguous cache needs seq_stride > 0");
+  }
+  return CSA2_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+CSA2_EXPORT int csa2_version(void) { return 100; }
+
+CSA2_EXPORT const char *csa2_last_error_string(void) { return g_last_error.c_str(); }
+
+CSA2_EXPORT csa2_status csa2_check(const int32_t *err, csa2_stream_t stream) {
+  if (!err) return fail(CSA2_ERR_INVALID_ARG, "err is NULL");
+  int32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, err, sizeof(h), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) {
+    g_last_error = std::string("csa2_check: ") + cudaGetErrorString(e);
+    return CSA2_ERR_CUDA;
+  }
+  return csa2_status(h);
+}
+
+CSA2_EXPORT size_t csa2_workspace_size(csa2_mode mode, int32_t B, int32_t Q, int32_t max_entries, int32_t k,
+                                       int32_t pool_k) {
+  if (B < 0 || Q < 0 || max_entries < 0 || k < 0 || pool_k < 0) return 0;
+  const size_t rows = size_t(B) * Q;
+  switch (mode) {
+    case CSA2_MODE_FULL: return round256(rows * max_entries * 4) + round256(rows * k * 4);
+    case CSA2_MODE_REINDEX: return round256(rows * pool_k * 4) + round256(rows * k * 4);
+    default: return 0;
+  }
+}
+
+CSA2_EXPORT csa2_status csa2_pack_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype, const float *pool_w,
+                                     int32_t B, int32_t T, const int32_t *first_entry, const csa2_cache *cache,
+                                     int32_t *err, csa2_stream_t stream) {
+  if (csa2_status s = check_cache(cache, B)) return s;
+  if (!lat_kv || !lat_ix || !first_entry) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
+  if (dtype != CSA2_F32 && dtype != CSA2_BF16) return fail(CSA2_ERR_INVALID_ARG, "bad dtype");
+  if (B < 0 || T < 0) return fail(CSA2_ERR_INVALID_ARG, "negative size");
+  if (!aligned16(lat_kv) || (reinterpret_cast<uintptr_t>(lat_ix) & 7)) return fail(CSA2_ERR_INVALID_ARG, "latents misaligned");
+  csa2::launch_pack_kv(lat_kv, lat_ix, dtype, pool_w, B, T, first_entry, *cache, err, stream);
+  return launched("csa2_pack_kv");
+}
+
+CSA2_EXPORT csa2_status csa2_pack_swa(const void *x, csa2_dtype dtype, int32_t B, int32_t T, const int32_t *pos,
+                                      uint8_t *swa_codes, float *swa_scale, int32_t R, int32_t *err,
+                                      csa2_stream_t stream) {
+  if (!x || !pos || !swa_codes || !swa_scale) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
+  if (dtype != CSA2_F32 && dtype != CSA2_BF16) return fail(CSA2_ERR_INVALID_ARG, "bad dtype");
+  if (B < 0 || T < 0 || R < 1) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  if (!aligned16(x) || !aligned16(swa_codes)) return fail(CSA2_ERR_INVALID_ARG, "x / swa_codes misaligned");
+  csa2::launch_pack_swa(x, dtype, B, T, pos, swa_codes, swa_scale, R, err, stream);
+  return launched("csa2_pack_swa");
+}
+
+CSA2_EXPORT csa2_status csa2_index_score(const uint16_t *q_ix, const uint16_t *w, int32_t B, int32_t Q,
+                                         const int32_t *q_pos, const int32_t *cand, int32_t P, int32_t max_entries,
+                                         const csa2_cache *cache, float *scores, int32_t *err,
+                                         csa2_stream_t stream) {
+  if (csa2_status s = check_cache(cache, B)) return s;
+  if (!q_ix || !w || !q_pos || !scores) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
+  if (B < 0 || Q < 0 || max_entries < 0 || (cand && P <= 0)) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  if (!aligned16(q_ix)) return fail(CSA2_ERR_INVALID_ARG, "q_ix misaligned");
+  const int n_out = cand ? P : max_entries;
+  if (n_out > 65535 * 128) return fail(CSA2_ERR_UNSUPPORTED, "more than 8388480 entries per row");
+  csa2::launch_index_score_scalar(q_ix, w, B, Q, q_pos, cand, P, n_out, *cache, scores, err, stream);
+  return launched("csa2_index_score");
+}
+
+CSA2_EXPORT csa2_status csa2_topk(const float *scores, const int32_t *n_valid, int32_t R, int32_t N, int32_t k,
+                                  int32_t *idx, float *val, void *ws, size_t ws_bytes, csa2_stream_t stream) {
+  (void)ws, (void)ws_bytes;
+  if (!scores || !idx) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
+  if (R < 0 || N < 0 || k < 1) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  csa2::launch_topk_rows(scores, n_valid, R, N, k, idx, val, nullptr, stream);
+  return launched("csa2_topk");
+}
+
+CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int32_t B, int32_t Q,
+                                         const int32_t *q_pos, float softmax_scale, const uint16_t *q_ix,
+                                         const uint16_t *w, int32_t k, int32_t pool_k, int32_t *pool_io,
+                                         const int32_t *idx_in, int32_t *idx_out, int32_t max_entries,
+                                         const csa2_cache *cache, float *o, float *lse, void *ws, size_t ws_bytes,
+                                         int32_t *err, csa2_stream_t stream) {
+  if (csa2_status s = check_cache(cache, B)) return s;
+  if (!q || !q_pos || !o || !lse) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
+  if (B < 0 || Q < 0 || k < 1 || pool_k < 0 || max_entries < 0) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  const int rows = B * Q;
+  const int32_t *idx = nullptr;
+  if (mode == CSA2_MODE_REUSE) {
+    if (!idx_in) return fail(CSA2_ERR_INVALID_ARG, "REUSE needs idx_in");
+    idx = idx_in;
+  } else if (mode == CSA2_MODE_FULL || mode == CSA2_MODE_REINDEX) {
+    if (!q_ix || !w) return fail(CSA2_ERR_INVALID_ARG, "FULL/REINDEX need q_ix and w");
+    if (!aligned16(q_ix)) return fail(CSA2_ERR_INVALID_ARG, "q_ix misaligned");
+    if (mode == CSA2_MODE_REINDEX && (!pool_io || pool_k < 1)) return fail(CSA2_ERR_INVALID_ARG, "REINDEX needs pool_io and pool_k");
+    if (mode == CSA2_MODE_FULL && pool_k > 0 && !pool_io) return fail(CSA2_ERR_INVALID_ARG, "pool_k > 0 needs pool_io");
+    const size_t need = csa2_workspace_size(mode, B, Q, max_entries, k, pool_k);
+    if (!ws || ws_bytes < need) return fail(CSA2_ERR_INVALID_ARG, "workspace too small");
+    const int n_out = mode == CSA2_MODE_FULL ? max_entries : pool_k;
+    if (n_out > 65535 * 128) return fail(CSA2_ERR_UNSUPPORTED, "more than 8388480 entries per row");
+    float *scores = static_cast<float *>(ws);
+    int32_t *sel = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + round256(size_t(rows) * n_out * 4));
+    if (idx_out) sel = idx_out;
+    if (mode == CSA2_MODE_FULL) {
+      csa2::launch_index_score_scalar(q_ix, w, B, Q, q_pos, nullptr, 0, max_entries, *cache, scores, err, stream);
+      csa2::launch_topk_rows(scores, nullptr, rows, max_entries, k, sel, nullptr, nullptr, stream);
+      if (pool_k > 0) csa2::launch_topk_rows(scores, nullptr, rows, max_entries, pool_k, pool_io, nullptr, nullptr, stream);
+    } else {
+      csa2::launch_index_score_scalar(q_ix, w, B, Q, q_pos, pool_io, pool_k, pool_k, *cache, scores, err, stream);
+      csa2::launch_topk_rows(scores, nullptr, rows, pool_k, k, sel, nullptr, pool_io, stream);
+    }
+    idx = sel;
+  } else {
+    return fail(CSA2_ERR_INVALID_ARG, "bad mode");
+  }
+  csa2::launch_sparse_attn_scalar(q, B, Q, q_pos, softmax_scale, idx, k, *cache, o, lse, err, stream);
+  return launched("csa2_sparse_attn");
+}
+
+CSA2_EXPORT csa2_status csa2_swa_attn(const uint16_t *q, int32_t B, int32_t Q, const int32_t *q_pos,
+                                      const uint8_t *swa_codes, const float *swa_scale, int32_t R, int32_t window,
+                                      float softmax_scale, float *o, float *lse, int32_t *err, csa2_stream_t stream) {
+  if (!q || !q_pos || !swa_codes || !swa_scale || !o || !lse) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
+  if (B < 0 || Q < 0 || window < 1 || R < window) return fail(CSA2_ERR_INVALID_ARG, "need 1 <= window <= R");
+  if (!aligned16(swa_codes)) return fail(CSA2_ERR_INVALID_ARG, "swa_codes misaligned");
+  csa2::launch_swa_attn_scalar(q, B, Q, q_pos, swa_codes, swa_scale, R, window, softmax_scale, o, lse, err, stream);
+  return launched("csa2_swa_attn");
+}
+
+CSA2_EXPORT csa2_status csa2_merge(const float *o1, const float *l1, const float *o2, const float *l2, int64_t rows,
+                                   int32_t D, float *o, float *lse, csa2_stream_t stream) {
+  if (!o1 || !l1 || !o2 || !l2 || !o || !lse) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
+  if (rows < 0 || D < 4 || (D & 3)) return fail(CSA2_ERR_INVALID_ARG, "D must be a positive multiple of 4");
+  if (!aligned16(o1) || !aligned16(o2) || !aligned16(o)) return fail(CSA2_ERR_INVALID_ARG, "o misaligned");
+  csa2::launch_merge(o1, l1, o2, l2, rows, D, o, lse, stream);
+  return launched("csa2_merge");
+}

@@ -1,0 +1,38 @@
+// Host-side launchers of the CSA2 kernels (internal to the library).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/csa2.h"
+
+namespace csa2 {
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+template <typename F>
+inline void set_smem_limit(F *func, size_t bytes) {
+  static bool done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || done[dev]) return;
+  cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+  done[dev] = true;
+}
+
+void launch_pack_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype, const float *pool_w, int B, int T,
+                    const int32_t *first_entry, const csa2_cache &c, int32_t *err, cudaStream_t st);
+void launch_pack_swa(const void *x, csa2_dtype dtype, int B, int T, const int32_t *pos, uint8_t *codes,
+                     float *scale, int R, int32_t *err, cudaStream_t st);
+void launch_index_score_scalar(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
+                               const int32_t *cand, int P, int n_out, const csa2_cache &c, float *scores,
+                               int32_t *err, cudaStream_t st);
+void launch_topk_rows(const float *scores, const int32_t *n_valid, int R, int N, int k, int32_t *idx, float *val,
+                      const int32_t *map, cudaStream_t st);
+void launch_sparse_attn_scalar(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx,
+                               int k, const csa2_cache &c, float *o, float *lse, int32_t *err, cudaStream_t st);
+void launch_swa_attn_scalar(const uint16_t *q, int B, int Q, const int32_t *q_pos, const uint8_t *codes,
+                            const float *scale, int R, int window, float tau, float *o, float *lse, int32_t *err,
+                            cudaStream_t st);
+void launch_merge(const float *o1, const float *l1, const float *o2, const float *l2, int64_t rows, int D_,
+                  float *o, float *lse, cudaStream_t st);
+
+}  // namespace csa2

@@ -1,0 +1,225 @@
+/*
+ * csa2.h -- C ABI of the CSA2 hot path on B200 (sm_100a).
+ *
+ * CSA2 is compressed sparse attention over a global KV cache that several
+ * layers share, stored in four-bit numbers ("DeepSeek-V4.1 模型结构（0）", 延伸解读
+ * "CSA2 共享池：四种层模式如何分工"; "从V4到V4.1 Flash：架构的激进进化", section
+ * "CSA2架构：跨层压缩的创新方案").  Each layer runs in one of three modes:
+ *   Full    -- score every cache entry with the lightning indexer, keep top-k;
+ *   Reindex -- reuse the shared cache, score only a candidate pool with the
+ *              layer's own indexer query, keep top-k inside the pool;
+ *   Reuse   -- reuse the shared cache and the given top-k indices, no indexer.
+ * A 128-token sliding-window (SWA) branch over a per-layer FP8 cache runs beside
+ * it and the two are combined by log-sum-exp.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every pointer argument is a DEVICE pointer owned by the caller unless the
+ *    comment says "host".  The library never allocates or frees memory; calls
+ *    that need scratch take a caller workspace sized by csa2_workspace_size().
+ *  - Every compute call is asynchronous on `stream` (0 = legacy default stream)
+ *    and returns a csa2_status for the host-side checks and the launch itself.
+ *  - Errors found on the device (an index or page outside the cache) never trap:
+ *    the kernel skips the bad access and stores the status code into *err (a
+ *    caller-owned device int32, first error wins), read back by csa2_check().
+ *  - bf16 tensors are passed as `const uint16_t*` (raw bf16 bits).
+ *  - Fixed dimensions: main-KV and query head dim 512, indexer dim 128,
+ *    query heads H = 64, indexer heads H_I = 64.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *csa2_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  CSA2_OK = 0,
+  CSA2_ERR_INVALID_ARG = 1, /* null pointer, bad enum, negative size */
+  CSA2_ERR_SHAPE = 2,       /* sizes inconsistent with each other or the cache */
+  CSA2_ERR_UNSUPPORTED = 3, /* a valid request this build does not implement */
+  CSA2_ERR_CUDA = 4,        /* launch or runtime error (see csa2_last_error_string) */
+  CSA2_ERR_INDEX = 5,       /* device side: an index or page outside the cache */
+  CSA2_ERR_TIMEOUT = 6      /* device side: a bounded wait gave up */
+} csa2_status;
+
+typedef enum { CSA2_MODE_FULL = 0, CSA2_MODE_REINDEX = 1, CSA2_MODE_REUSE = 2 } csa2_mode;
+typedef enum { CSA2_F32 = 0, CSA2_BF16 = 1 } csa2_dtype;
+
+enum {
+  CSA2_MAIN_DIM = 512,        /* values per main-KV entry */
+  CSA2_MAIN_CODE_BYTES = 256, /* two e2m1 codes per byte, element 2i in the low nibble */
+  CSA2_MAIN_SCALE_BYTES = 32, /* one E4M3 scale per block of 16 values */
+  CSA2_IX_DIM = 128,          /* values per indexer key */
+  CSA2_IX_CODE_BYTES = 64,    /* two e2m1 codes per byte */
+  CSA2_IX_SCALE_BYTES = 4,    /* one E8M0 exponent per block of 32 values */
+  CSA2_SWA_DIM = 512,         /* E4M3 codes per SWA token, plus one fp32 scale */
+  CSA2_HEADS = 64,            /* query heads H */
+  CSA2_IX_HEADS = 64          /* indexer heads H_I */
+};
+
+/*
+ * The shared global KV cache ("DeepSeek-V4.1 模型结构（0）", Q&A "890 字节全局 KV
+ * 是怎么算出来的": a main-KV entry is 512 four-bit numbers plus 32 bytes of scale,
+ * 288 bytes; an indexer-K entry is 128 four-bit numbers plus 4 bytes of scale,
+ * 68 bytes).  The four byte planes are kept apart (structure of arrays) so that
+ * every row starts 16-byte aligned; bytes per entry are still 288 + 68.
+ *
+ * Physical slot of entry n of sequence b:
+ *   contiguous (page_table == NULL): b * seq_stride + n, with n < seq_stride;
+ *   paged: page_table[b * max_pages + n / page_size] * page_size + n % page_size.
+ * Row s of a plane starts at plane + s * (row bytes).  num_slots bounds every slot.
+ * ratio is the compression ratio of the layer that wrote the cache: an entry
+ * pools `ratio` tokens, so a query at position p sees entries
+ * n < min(num_entries[b], (p + 1) / ratio).
+ */
+typedef struct {
+  uint8_t *kv_codes;          /* [num_slots][256] */
+  uint8_t *kv_scales;         /* [num_slots][32]  */
+  uint8_t *ix_codes;          /* [num_slots][64]  */
+  uint8_t *ix_scales;         /* [num_slots][4]   */
+  const int32_t *page_table;  /* [batch][max_pages] or NULL (contiguous) */
+  const int32_t *num_entries; /* [batch] entries present per sequence */
+  int64_t num_slots;          /* rows allocated in each plane */
+  int32_t batch;              /* sequences described by this cache */
+  int32_t ratio;              /* tokens per entry, >= 1 */
+  int32_t seq_stride;         /* contiguous layout: slots per sequence */
+  int32_t page_size;          /* paged layout: entries per page (power of two) */
+  int32_t max_pages;          /* paged layout: page-table row length */
+} csa2_cache;
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int csa2_version(void);
+
+/* Text of the last host-side error on this thread ("" if none).  Static storage. */
+const char *csa2_last_error_string(void);
+
+/*
+ * Synchronises `stream`, reads the caller's device error word and returns it as
+ * a csa2_status (CSA2_OK when zero).  Does not clear it.
+ */
+csa2_status csa2_check(const int32_t *err, csa2_stream_t stream);
+
+/*
+ * Bytes of workspace csa2_sparse_attn needs for these sizes (0 for Reuse).
+ * max_entries bounds num_entries[b]; pool_k is the candidate-pool size (0 if none).
+ */
+size_t csa2_workspace_size(csa2_mode mode, int32_t B, int32_t Q, int32_t max_entries,
+                           int32_t k, int32_t pool_k);
+
+/*
+ * Token compressor + packer: writes floor(T / ratio) new entries per sequence.
+ * ("从V4到V4.1 Flash", section 编码器层: about two tokens per main-KV entry in
+ * the encoder; section 解码器层: ratio 1 in the decoder; "DeepSeek-V4.1 模型结构（0）",
+ * Q&A on the 890 bytes: entry formats.)
+ *   lat_kv  [B][T][512] and lat_ix [B][T][128] in `dtype` (fp32 or bf16);
+ *   pool_w  [B][T] fp32 pooling weights, or NULL for fp32(1/ratio);
+ *   entry j of sequence b = sum over t in [j*r, j*r + r) of pool_w * lat, fp32,
+ *   left to right; then per block of 16 an E4M3 scale = RNE(amax / 6) and e2m1
+ *   codes RNE(x / scale); per block of 32 of the indexer key an E8M0 exponent
+ *   ceil(log2(amax / 6)) and e2m1 codes.  A block with a zero scale has zero codes.
+ *   first_entry [B] (device): entry index of the first new entry of sequence b.
+ * Writes the four planes only; the caller updates num_entries.
+ * Device errors: a slot outside the cache -> CSA2_ERR_INDEX in *err, entry skipped.
+ */
+csa2_status csa2_pack_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype,
+                         const float *pool_w, int32_t B, int32_t T, const int32_t *first_entry,
+                         const csa2_cache *cache, int32_t *err, csa2_stream_t stream);
+
+/*
+ * SWA packer: per token an fp32 scale = amax / 448 and 512 E4M3 codes RNE(x / scale)
+ * (saturating), stored in a per-layer ring at slot pos mod R.  ("DeepSeek V4.1 Flash
+ * 深度解析", 本专栏篇目 "FP4 从权重走进 KV 缓存": the sliding-window cache stays FP8;
+ * "从V4到V4.1 Flash", section "SWA 有界重放": the window keeps the last 128 tokens.)
+ *   x [B][T][512] in `dtype`; pos [B][T] absolute positions (device), a negative
+ *   position marks a padding token that is skipped;
+ *   swa_codes [B][R][512] u8; swa_scale [B][R] fp32.
+ * Positions of one sequence's tokens in a call are consecutive, so only the
+ * last R tokens of the call are stored (earlier ones would be overwritten).
+ */
+csa2_status csa2_pack_swa(const void *x, csa2_dtype dtype, int32_t B, int32_t T,
+                          const int32_t *pos, uint8_t *swa_codes, float *swa_scale, int32_t R,
+                          int32_t *err, csa2_stream_t stream);
+
+/*
+ * Lightning-indexer scores ("DeepSeek V4.1 Flash 深度解析", 本专栏篇目 "前代 · CSA":
+ * an FP4 lightning indexer picks top-512; the score formula is the weighted-ReLU
+ * form s_n = sum_h w_h * relu(q^_h . k^_n) with q^ the per-32 E8M0/e2m1
+ * quantisation of the query heads).
+ *   q_ix [B][Q][64][128] bf16; w [B][Q][64] bf16; q_pos [B][Q] positions;
+ *   cand [B][Q][P] entry indices (-1 = none) or NULL to score entries 0..N-1;
+ *   scores [B][Q][N_out] fp32 with N_out = P when cand != NULL else max_entries.
+ * Entries not visible to the query (see csa2_cache) and -1 candidates score -inf.
+ * Device errors: a candidate >= num_entries[b] or a bad page -> CSA2_ERR_INDEX, -inf.
+ */
+csa2_status csa2_index_score(const uint16_t *q_ix, const uint16_t *w, int32_t B, int32_t Q,
+                             const int32_t *q_pos, const int32_t *cand, int32_t P,
+                             int32_t max_entries, const csa2_cache *cache, float *scores,
+                             int32_t *err, csa2_stream_t stream);
+
+/*
+ * Top-k of each row ("DeepSeek-V4.1 模型结构（0）", 延伸解读 CSA2 共享池: top-512;
+ * "从V4到V4.1 Flash", section 解码器层: a candidate pool, then top-512 inside it).
+ *   scores [R][N] fp32; n_valid [R] (device) or NULL = N: candidates are positions
+ *   j < n_valid[r] whose score is not -inf, ordered by score descending, then j
+ *   ascending.  idx [R][k] receives the first k positions in ascending order,
+ *   padded with -1; val [R][k] (optional) their scores (-inf for pads).
+ *   ws may be NULL (this call needs no workspace).
+ */
+csa2_status csa2_topk(const float *scores, const int32_t *n_valid, int32_t R, int32_t N,
+                      int32_t k, int32_t *idx, float *val, void *ws, size_t ws_bytes,
+                      csa2_stream_t stream);
+
+/*
+ * Sparse attention of one CSA2 layer ("从V4到V4.1 Flash", section CSA2架构: the
+ * Full, Reindex and Reuse modes; section 解码器层: the hierarchical pool).
+ *   q [B][Q][64][512] bf16 query heads; q_pos [B][Q]; softmax_scale tau.
+ *   FULL:    q_ix, w (as csa2_index_score) select top-k of all visible entries;
+ *            if pool_k > 0 the top-pool_k entries are written to pool_io [B][Q][pool_k].
+ *   REINDEX: q_ix, w score the entries listed in pool_io [B][Q][pool_k]; top-k of them.
+ *   REUSE:   idx_in [B][Q][k] given entry indices (-1 = none; order free).
+ *   idx_out [B][Q][k] (optional, FULL/REINDEX) receives the chosen entries, ascending.
+ * Per head: logits tau * q . v_j over the chosen entries, v_j the dequantised
+ * 512-d main entry used as key and value; o [B][Q][64][512] fp32 = softmax-weighted
+ * sum, lse [B][Q][64] fp32 natural-log normaliser; no entries -> o = 0, lse = -inf.
+ * ws: csa2_workspace_size(mode, ...) bytes (may be NULL for REUSE).
+ * Device errors: an index outside the visible entries -> CSA2_ERR_INDEX, skipped.
+ */
+csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int32_t B, int32_t Q,
+                             const int32_t *q_pos, float softmax_scale, const uint16_t *q_ix,
+                             const uint16_t *w, int32_t k, int32_t pool_k, int32_t *pool_io,
+                             const int32_t *idx_in, int32_t *idx_out, int32_t max_entries,
+                             const csa2_cache *cache, float *o, float *lse, void *ws,
+                             size_t ws_bytes, int32_t *err, csa2_stream_t stream);
+
+/*
+ * Sliding-window branch ("从V4到V4.1 Flash", sections "CSA2 机制下的全局 KV 共享与局部
+ * 滑动窗口隔离" (per-layer SWA cache) and "SWA 有界重放" (128 tokens)).
+ *   Window of a query at p: positions max(0, p - window + 1) .. p, read from the
+ *   ring written by csa2_pack_swa (slot t mod R, R >= window).  Keys = values =
+ *   E4M3 code * fp32 scale.  Same o / lse as csa2_sparse_attn.
+ */
+csa2_status csa2_swa_attn(const uint16_t *q, int32_t B, int32_t Q, const int32_t *q_pos,
+                          const uint8_t *swa_codes, const float *swa_scale, int32_t R,
+                          int32_t window, float softmax_scale, float *o, float *lse,
+                          int32_t *err, csa2_stream_t stream);
+
+/*
+ * Log-sum-exp merge of the sparse and sliding-window branches ("从V4到V4.1 Flash",
+ * section 移除混合注意力机制: CSA mixed with SWA): m = max(l1, l2),
+ * o = (e^(l1-m) o1 + e^(l2-m) o2) / (e^(l1-m) + e^(l2-m)), lse = m + log(...).
+ *   o1, o2, o [rows][D] fp32; l1, l2, lse [rows].  o may alias o1 or o2 and lse
+ *   may alias l1 or l2.  Both -inf -> o = 0, lse = -inf.
+ */
+csa2_status csa2_merge(const float *o1, const float *l1, const float *o2, const float *l2,
+                       int64_t rows, int32_t D, float *o, float *lse, csa2_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_H */

@@ -1,0 +1,406 @@
+"""GPU parity: every CSA2 step through the C ABI against the CPU oracle, element by element.
+
+Sizes here span several tiles and a ragged tail and still let the oracle finish
+in seconds; test_gpu_full_size.py covers the full configurations by sampling.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import csa2 as OC
+from oracle import formats as OF
+from workloads import configs as W
+from workloads import normal, uniform
+
+from tests.helpers import (K, check_attention, check_topk, fill_main, gpu_cache, oracle_seq, oracle_swa,
+                           to_np)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _err():
+    return torch.zeros(1, dtype=torch.int32, device=DEV)
+
+
+# ------------------------------------------------------------------ packers
+def _planted_latents(B, T, d, seed, dtype):
+    x = normal((B, T, d), seed, "pack", d, device=DEV)
+    x[0, 0, :32] = 0.0                       # zero blocks
+    x[0, 1, :16] *= 1e-5                     # subnormal E4M3 scales
+    x[0, 2, :] *= 1e3                        # saturating E4M3 scales
+    x[min(1, B - 1), 3, 5] = 1e-40           # a subnormal input
+    x[0, 4, :] = 0.25                        # exact e2m1 ties after scaling
+    x[0, 5, :] = torch.tensor([0.75, -1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 0.5] * (d // 8))
+    return x.to(dtype)
+
+
+@pytest.mark.parametrize("ratio", [1, 2, 4])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("weighted", [False, True])
+def test_pack_kv_bit_exact(ratio, dtype, weighted):
+    k = K()
+    B, T = 3, 1001
+    kv = _planted_latents(B, T, 512, 1, dtype)
+    ix = _planted_latents(B, T, 128, 2, dtype)
+    pw = uniform((B, T), 0, "pack_w", device=DEV) if weighted else None
+    n = T // ratio
+    cache = k.GlobalKVCache(B, ratio, seq_stride=n + 5)
+    first = torch.tensor([0, 3, 5], dtype=torch.int32, device=DEV)
+    err = _err()
+    k.csa2_pack_kv(kv, ix, first, cache, pool_w=pw, err=err)
+    assert k.csa2_check(err) == 0
+    for b in range(B):
+        w_np = None if pw is None else to_np(pw[b])
+        ekv = OC.compress(to_np(kv[b]), ratio, w_np)
+        eix = OC.compress(to_np(ix[b]), ratio, w_np)
+        mc, ms = OF.pack_main(ekv)
+        ic, isc = OF.pack_indexer(eix)
+        f = int(first[b])
+        sl = slice(b * (n + 5) + f, b * (n + 5) + f + n)
+        np.testing.assert_array_equal(to_np(cache.kv_codes[sl]), mc)
+        np.testing.assert_array_equal(to_np(cache.kv_scales[sl]), ms)
+        np.testing.assert_array_equal(to_np(cache.ix_codes[sl]), ic)
+        np.testing.assert_array_equal(to_np(cache.ix_scales[sl]), isc)
+
+
+def test_pack_kv_paged_and_out_of_range():
+    k = K()
+    spec = W.scaled(W.mixed64(), [700, 1300, 260], B=3)
+    spec.page_size = 256
+    spec.paged = True
+    table, pages = W.page_layout(spec, DEV)
+    cache = k.GlobalKVCache(3, 1, num_slots=pages * 256, page_table=table, page_size=256)
+    err = _err()
+    for b in range(3):
+        kv, ix = W.token_latents(spec, b, DEV)
+        v = cache.seq_view(b)
+        v.ratio = spec.seq_ratio(b)
+        k.csa2_pack_kv(kv[None].contiguous(), ix[None].contiguous(), torch.zeros(1, dtype=torch.int32, device=DEV),
+                       v, err=err)
+        c = oracle_seq(spec, b, gen_device=DEV)
+        n = spec.entries(b)
+        tb = table[b].cpu().numpy()
+        slots = np.array([tb[e // 256] * 256 + e % 256 for e in range(n)])
+        np.testing.assert_array_equal(to_np(cache.kv_codes)[slots], c.kv_codes[0, :n])
+        np.testing.assert_array_equal(to_np(cache.kv_scales)[slots], c.kv_scales[0, :n])
+        np.testing.assert_array_equal(to_np(cache.ix_codes)[slots], c.ix_codes[0, :n])
+        np.testing.assert_array_equal(to_np(cache.ix_scales)[slots], c.ix_scales[0, :n])
+    assert k.csa2_check(err) == 0
+    # writing past the last page is refused on the device, not faulted
+    kv, ix = W.token_latents(spec, 2, DEV)
+    v = cache.seq_view(2)
+    k.csa2_pack_kv(kv[None, :300].contiguous(), ix[None, :300].contiguous(),
+                   torch.full((1,), 200, dtype=torch.int32, device=DEV), v, err=err)
+    assert k.csa2_check(err) == 5
+
+
+@pytest.mark.parametrize("R,T", [(128, 300), (512, 300), (128, 1)])
+def test_pack_swa_bit_exact(R, T):
+    k = K()
+    B = 2
+    x = _planted_latents(B, T, 512, 3, torch.bfloat16)
+    pos = (torch.arange(T, dtype=torch.int32, device=DEV) + 1000)[None].repeat(B, 1).contiguous()
+    codes = torch.zeros((B, R, 512), dtype=torch.uint8, device=DEV)
+    scale = torch.zeros((B, R), dtype=torch.float32, device=DEV)
+    err = _err()
+    k.csa2_pack_swa(x, pos, codes, scale, err=err)
+    assert k.csa2_check(err) == 0
+    for b in range(B):
+        keep = slice(max(0, T - R), T)
+        oc, osc = oracle_swa(to_np(x[b])[keep], to_np(pos[b])[keep], R)
+        np.testing.assert_array_equal(to_np(codes[b]), oc)
+        np.testing.assert_array_equal(to_np(scale[b]), osc)
+
+
+# ------------------------------------------------------------------ indexer + top-k
+def test_index_score_full_and_candidates():
+    k = K()
+    spec = W.scaled(W.tiny_full(), [3001, 5000], B=2)
+    cache = gpu_cache(spec)
+    q, q_ix, w, q_pos = W.query_tensors(spec, 0, DEV)
+    q_pos[0, 0] = 1999                      # an earlier query sees fewer entries
+    err = _err()
+    s = k.csa2_index_score(q_ix, w, q_pos, cache, spec.max_entries, err=err)
+    assert k.csa2_check(err) == 0
+    for b in range(2):
+        c = oracle_seq(spec, b, main_rows=[], gen_device=DEV)
+        nvis = c.visible(0, int(q_pos[b, 0]))
+        ref = OC.indexer_scores(to_np(q_ix[b, 0]), to_np(w[b, 0]), c.indexer_values(0, np.arange(nvis)))
+        got = to_np(s[b, 0])
+        assert np.all(np.isneginf(got[nvis:]))
+        np.testing.assert_allclose(got[:nvis], ref, rtol=2e-6, atol=2e-6 * np.abs(ref).max())
+    # candidate lists with pads
+    cand = torch.full((2, 1, 700), -1, dtype=torch.int32, device=DEV)
+    cand[:, :, :650] = torch.randint(0, 999, (2, 1, 650), dtype=torch.int32, device=DEV)
+    sc = k.csa2_index_score(q_ix, w, q_pos, cache, spec.max_entries, cand=cand, err=err)
+    assert k.csa2_check(err) == 0
+    full = to_np(s)
+    got = to_np(sc)
+    cn = to_np(cand)
+    for b in range(2):
+        assert np.all(np.isneginf(got[b, 0, 650:]))
+        np.testing.assert_array_equal(got[b, 0, :650], full[b, 0, cn[b, 0, :650]])
+
+
+def test_index_score_rejects_bad_candidates():
+    k = K()
+    spec = W.scaled(W.tiny_full(), [600], B=1)
+    cache = gpu_cache(spec)
+    q, q_ix, w, q_pos = W.query_tensors(spec, 0, DEV)
+    cand = torch.tensor([[[3, 299, 300, -1]]], dtype=torch.int32, device=DEV)
+    err = _err()
+    sc = k.csa2_index_score(q_ix, w, q_pos, cache, spec.max_entries, cand=cand, err=err)
+    assert k.csa2_check(err) == 5
+    got = to_np(sc)[0, 0]
+    assert np.isfinite(got[:2]).all() and np.isneginf(got[2:]).all()
+
+
+@pytest.mark.parametrize("case", ["random", "ties", "short", "neg_inf", "pool"])
+def test_topk_rows(case):
+    k_ = K()
+    g = torch.Generator(device="cpu").manual_seed(7)
+    R, N, k = 5, 9000, 512
+    if case == "random":
+        s = torch.randn((R, N), generator=g)
+    elif case == "ties":
+        s = torch.randint(-4, 5, (R, N), generator=g).float()
+    elif case == "short":
+        N = 300
+        s = torch.randn((R, N), generator=g)
+    elif case == "neg_inf":
+        s = torch.randn((R, N), generator=g)
+        s[torch.rand((R, N), generator=g) < 0.97] = -math.inf
+    else:
+        N, k = 70000, 16384
+        s = torch.randn((R, N), generator=g) * 100
+    n_valid = torch.tensor([N, N - 1, N // 2, 511, 0][:R], dtype=torch.int32)
+    sd = s.to(DEV)
+    idx, val = k_.csa2_topk(sd, k, n_valid=n_valid.to(DEV))
+    idx = to_np(idx)
+    val = to_np(val)
+    for r in range(R):
+        ref = OC.topk(s[r].double().numpy(), k, int(n_valid[r]))
+        np.testing.assert_array_equal(idx[r], ref)      # same fp32 inputs: exact
+        sel = idx[r][idx[r] >= 0]
+        np.testing.assert_array_equal(val[r][: len(sel)], s[r].numpy()[sel])
+        assert np.all(np.isneginf(val[r][len(sel):]))
+
+
+# ------------------------------------------------------------------ attention
+def _swa_state(spec, layer, R=128):
+    """Device SWA ring for one layer plus the oracle's rings (one per sequence)."""
+    k = K()
+    x, pos = W.swa_tokens(spec, layer, DEV)
+    codes = torch.zeros((spec.B, R, 512), dtype=torch.uint8, device=DEV)
+    scale = torch.zeros((spec.B, R), dtype=torch.float32, device=DEV)
+    err = _err()
+    k.csa2_pack_swa(x, pos, codes, scale, err=err)
+    assert k.csa2_check(err) == 0
+    rings = [oracle_swa(to_np(x[b]), to_np(pos[b]), R) for b in range(spec.B)]
+    return codes, scale, rings
+
+
+def test_swa_attention_and_sequence_start():
+    k = K()
+    spec = W.scaled(W.tiny_full(), [4096, 60, 1], B=3)
+    q, _, _, q_pos = W.query_tensors(spec, 0, DEV)
+    codes, scale, rings = _swa_state(spec, 0)
+    o, lse = k.csa2_swa_attn(q, q_pos, codes, scale, spec.tau)
+    for b in range(3):
+        oo, ol = OC.swa_attention(to_np(q[b, 0]), int(q_pos[b, 0]), rings[b][0], rings[b][1], 128, spec.tau)
+        check_attention(to_np(o[b, 0]), to_np(lse[b, 0]), oo, ol, f"swa b={b}")
+
+
+def test_merge_matches_oracle_and_aliases():
+    k = K()
+    rows = 3 * 64
+    o1 = normal((rows, 512), 1, "m1", device=DEV)
+    o2 = normal((rows, 512), 1, "m2", device=DEV)
+    l1 = normal((rows,), 1, "l1", device=DEV) * 3
+    l2 = normal((rows,), 1, "l2", device=DEV) * 3
+    l1[:5] = -math.inf
+    l2[3:7] = -math.inf
+    ref_o, ref_l = OC.merge(to_np(o1), to_np(l1), to_np(o2), to_np(l2))
+    o, lse = k.csa2_merge(o1, l1, o2, l2)
+    check_attention(to_np(o), to_np(lse), ref_o, ref_l, "merge")
+    k.csa2_merge(o1, l1, o2, l2, o=o1, lse=l1)                 # in place
+    check_attention(to_np(o1), to_np(l1), ref_o, ref_l, "merge in place")
+
+
+def _decode_layer_parity(spec, cache, mode, layer, rings, codes, scale, pool=None, pool_k=0, idx_in=None,
+                         oracle_caches=None):
+    """Run one layer on the GPU (sparse + SWA + merge) and compare with the oracle per sequence."""
+    k = K()
+    q, q_ix, w, q_pos = W.query_tensors(spec, layer, DEV)
+    err = _err()
+    idx_out = torch.empty((spec.B, 1, spec.k), dtype=torch.int32, device=DEV)
+    pool_io = pool
+    if mode == "full" and pool_k:
+        pool_io = torch.empty((spec.B, 1, pool_k), dtype=torch.int32, device=DEV)
+    o1, l1 = k.csa2_sparse_attn(mode, q, q_pos, cache, spec.tau, spec.max_entries, k=spec.k, q_ix=q_ix, w=w,
+                                pool_k=pool_k, pool_io=pool_io, idx_in=idx_in, idx_out=idx_out, err=err)
+    o2, l2 = k.csa2_swa_attn(q, q_pos, codes, scale, spec.tau, err=err)
+    o, lse = k.csa2_merge(o1, l1, o2, l2)
+    assert k.csa2_check(err) == 0
+    same_rows = 0
+    ref_pools = np.full((spec.B, 1, max(pool_k, 1)), -1, np.int64)
+    ref_idxs = np.full((spec.B, 1, spec.k), -1, np.int64)
+    for b in range(spec.B):
+        c = oracle_caches[b]
+        pos = int(q_pos[b, 0])
+        qb, qib, wb = to_np(q[b, 0]), to_np(q_ix[b, 0]), to_np(w[b, 0])
+        if mode == "full":
+            ref_idx, ref_pool, scores = OC.full_select(c, 0, pos, qib, wb, spec.k, pool_k)
+            same = check_topk(to_np(idx_out[b, 0]), scores, ref_idx, spec.k, f"full idx b={b}")
+            if pool_k:
+                check_topk(to_np(pool_io[b, 0]), scores, ref_pool, pool_k, f"pool b={b}")
+                ref_pools[b, 0] = ref_pool
+        elif mode == "reindex":
+            ref_idx, pscores = OC.reindex_select(c, 0, pos, qib, wb, spec.k, to_np(pool[b, 0]))
+            pl = to_np(pool[b, 0])
+            gi = to_np(idx_out[b, 0])
+            gpos = np.array([np.searchsorted(pl, v) if v >= 0 else -1 for v in gi])
+            rpos = np.array([np.searchsorted(pl, v) if v >= 0 else -1 for v in ref_idx])
+            same = check_topk(gpos, pscores, rpos, spec.k, f"reindex idx b={b}")
+        else:
+            ref_idx = to_np(idx_in[b, 0])
+            same = True
+        ref_idxs[b, 0] = ref_idx
+        if same:
+            same_rows += 1
+            fill_main(c, spec, b, ref_idx, gen_device=DEV)
+            ref = OC.decode_layer("reuse", c, 0, pos, qb, spec.tau, rings[b], idx=ref_idx)
+            check_attention(to_np(o1[b, 0]), to_np(l1[b, 0]), *ref["sparse"], f"{mode} sparse b={b}")
+            check_attention(to_np(o[b, 0]), to_np(lse[b, 0]), ref["o"], ref["lse"], f"{mode} merged b={b}")
+    assert same_rows >= max(1, spec.B - 1)
+    # the oracle's own selections, for the layers that consume them
+    return (torch.from_numpy(ref_idxs).to(torch.int32).to(DEV),
+            torch.from_numpy(ref_pools).to(torch.int32).to(DEV))
+
+
+def test_full_decode_tiny_config():
+    spec = W.tiny_full()
+    cache = gpu_cache(spec)
+    codes, scale, rings = _swa_state(spec, 0)
+    oc = [oracle_seq(spec, b, main_rows=[], gen_device=DEV) for b in range(spec.B)]
+    _decode_layer_parity(spec, cache, "full", 0, rings, codes, scale, oracle_caches=oc)
+
+
+def test_reuse_decode_scaled():
+    spec = W.scaled(W.reuse64k(), [5000, 4097, 513, 700], B=4)
+    cache = gpu_cache(spec)
+    codes, scale, rings = _swa_state(spec, 0)
+    idx = W.reuse_indices(spec, DEV)
+    idx[2, 0, 500:] = -1                                      # ragged: fewer than k given
+    oc = [oracle_seq(spec, b, main_rows=[], gen_device=DEV) for b in range(spec.B)]
+    _decode_layer_parity(spec, cache, "reuse", 0, rings, codes, scale, idx_in=idx, oracle_caches=oc)
+
+
+def test_reuse_rejects_out_of_range_indices():
+    k = K()
+    spec = W.scaled(W.reuse64k(), [1000], B=1)
+    cache = gpu_cache(spec)
+    q, _, _, q_pos = W.query_tensors(spec, 0, DEV)
+    idx = W.reuse_indices(spec, DEV)
+    idx[0, 0, 7] = 1000                      # == num_entries
+    idx[0, 0, 9] = -7
+    err = _err()
+    o, lse = k.csa2_sparse_attn("reuse", q, q_pos, cache, spec.tau, spec.max_entries, idx_in=idx, err=err)
+    assert k.csa2_check(err) == 5
+    c = oracle_seq(spec, 0, gen_device=DEV)
+    good = to_np(idx[0, 0]).copy()
+    good[[7, 9]] = -1
+    oo, ol = OC.sparse_attention(c, 0, to_np(q[0, 0]), good, spec.tau)
+    check_attention(to_np(o[0, 0]), to_np(lse[0, 0]), oo, ol, "reuse with rejected indices")
+
+
+def test_hierarchical_full_then_reindex_scaled():
+    spec = W.scaled(W.hier1m(), 40000, B=2, pool_k=2048, n_reindex=2)
+    cache = gpu_cache(spec)
+    oc = [oracle_seq(spec, b, main_rows=[], gen_device=DEV) for b in range(spec.B)]
+    codes, scale, rings = _swa_state(spec, 0)
+    # Reindex and Reuse layers consume the oracle's pool and indices on both sides
+    idx_full, pool = _decode_layer_parity(spec, cache, "full", 0, rings, codes, scale, pool_k=spec.pool_k,
+                                          oracle_caches=oc)
+    for layer in (1, 2):
+        codes, scale, rings = _swa_state(spec, layer)
+        _decode_layer_parity(spec, cache, "reindex", layer, rings, codes, scale, pool=pool, pool_k=spec.pool_k,
+                             oracle_caches=oc)
+    # the Reuse layers after it consume the Full layer's indices
+    codes, scale, rings = _swa_state(spec, 5)
+    _decode_layer_parity(spec, cache, "reuse", 5, rings, codes, scale, idx_in=idx_full, oracle_caches=oc)
+
+
+def test_prefill_chunk_scaled():
+    k = K()
+    spec = W.scaled(W.prefill8k(), [2000 + 300], B=1, q_len=300)
+    cache = gpu_cache(spec)
+    q, q_ix, w, q_pos = W.query_tensors(spec, 0, DEV)
+    x, pos = W.swa_tokens(spec, 0, DEV)
+    R = 512
+    codes = torch.zeros((1, R, 512), dtype=torch.uint8, device=DEV)
+    scale = torch.zeros((1, R), dtype=torch.float32, device=DEV)
+    err = _err()
+    k.csa2_pack_swa(x, pos, codes, scale, err=err)
+    idx_out = torch.empty((1, spec.q_len, spec.k), dtype=torch.int32, device=DEV)
+    o1, l1 = k.csa2_sparse_attn("full", q, q_pos, cache, spec.tau, spec.max_entries, q_ix=q_ix, w=w,
+                                idx_out=idx_out, err=err)
+    o2, l2 = k.csa2_swa_attn(q, q_pos, codes, scale, spec.tau, err=err)
+    o, lse = k.csa2_merge(o1, l1, o2, l2)
+    assert k.csa2_check(err) == 0
+    c = oracle_seq(spec, 0, main_rows=[], gen_device=DEV)
+    ring = oracle_swa(to_np(x[0]), to_np(pos[0]), R)
+    rows = [0, 1, 2, 57, 150, 298, 299]
+    for qi in rows:
+        p = int(q_pos[0, qi])
+        ref_idx, _, scores = OC.full_select(c, 0, p, to_np(q_ix[0, qi]), to_np(w[0, qi]), spec.k)
+        assert (ref_idx[ref_idx >= 0] < (p + 1) // 2).all()
+        if check_topk(to_np(idx_out[0, qi]), scores, ref_idx, spec.k, f"prefill q={qi}"):
+            fill_main(c, spec, 0, ref_idx, gen_device=DEV)
+            ref = OC.decode_layer("reuse", c, 0, p, to_np(q[0, qi]), spec.tau, ring, idx=ref_idx)
+            check_attention(to_np(o[0, qi]), to_np(lse[0, qi]), ref["o"], ref["lse"], f"prefill q={qi}")
+
+
+def test_mixed_paged_batch_scaled():
+    k = K()
+    spec = W.scaled(W.mixed64(), [5000, 3000, 1200, 4097, 900, 2600], B=6)
+    table, pages = W.page_layout(spec, DEV)
+    base = k.GlobalKVCache(6, 1, num_slots=pages * 256, page_table=table, page_size=256)
+    err = _err()
+    for b in range(6):
+        kv, ix = W.token_latents(spec, b, DEV)
+        v = base.seq_view(b)
+        v.ratio = spec.seq_ratio(b)
+        k.csa2_pack_kv(kv[None].contiguous(), ix[None].contiguous(), torch.zeros(1, dtype=torch.int32, device=DEV),
+                       v, err=err)
+        base.num_entries[b] = spec.entries(b)
+    full_ids = [b for b in range(6) if spec.seq_mode(b) == "full"]
+    reuse_ids = [b for b in range(6) if spec.seq_mode(b) == "reuse"]
+    q, q_ix, w, q_pos = W.query_tensors(spec, 0, DEV)
+    idx_all = W.reuse_indices(spec, DEV)
+    for ids, mode, ratio in ((full_ids, "full", 2), (reuse_ids, "reuse", 1)):
+        sel = torch.tensor(ids, device=DEV)
+        view = k.GlobalKVCache(len(ids), ratio, num_slots=base.num_slots, page_table=table[sel].contiguous(),
+                               page_size=256, planes=base.planes, num_entries=base.num_entries[sel].contiguous())
+        maxe = max(spec.entries(b) for b in ids)
+        idx_out = torch.empty((len(ids), 1, 512), dtype=torch.int32, device=DEV)
+        o, lse = k.csa2_sparse_attn(mode, q[sel].contiguous(), q_pos[sel].contiguous(), view, spec.tau, maxe,
+                                    q_ix=q_ix[sel].contiguous(), w=w[sel].contiguous(),
+                                    idx_in=idx_all[sel].contiguous() if mode == "reuse" else None,
+                                    idx_out=idx_out if mode == "full" else None, err=err)
+        assert k.csa2_check(err) == 0
+        for j, b in enumerate(ids):
+            c = oracle_seq(spec, b, main_rows=[], gen_device=DEV)
+            p = int(q_pos[b, 0])
+            if mode == "full":
+                ref_idx, _, scores = OC.full_select(c, 0, p, to_np(q_ix[b, 0]), to_np(w[b, 0]), 512)
+                if not check_topk(to_np(idx_out[j, 0]), scores, ref_idx, 512, f"mixed full b={b}"):
+                    continue
+            else:
+                ref_idx = to_np(idx_all[b, 0])
+            fill_main(c, spec, b, ref_idx, gen_device=DEV)
+            oo, ol = OC.sparse_attention(c, 0, to_np(q[b, 0]), ref_idx, spec.tau)
+            check_attention(to_np(o[j, 0]), to_np(lse[j, 0]), oo, ol, f"mixed {mode} b={b}")
