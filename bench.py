@@ -172,7 +172,7 @@ class Hier1M:
         self.l_swa = torch.empty((B, 1, 64), dtype=torch.float32, device=dev)
         self.scores = torch.empty((B, 1, N), dtype=torch.float32, device=dev)
         self.pool = torch.empty((B, 1, spec.pool_k), dtype=torch.int32, device=dev)
-        self.idx = torch.empty((B, 1, spec.k), dtype=torch.int32, device=dev)
+        self.idx = torch.empty((L, B, 1, spec.k), dtype=torch.int32, device=dev)   # per layer
         self.ws_reindex = torch.empty(k.csa2_workspace_size("reindex", B, 1, N, spec.k, spec.pool_k),
                                       dtype=torch.uint8, device=dev)
         self.err = err
@@ -198,12 +198,12 @@ class Hier1M:
                 if scan_events:
                     scan_events[1].record()
                 k.csa2_topk(self.scores, s.pool_k, idx=self.pool, val=None)
-                k.csa2_topk(self.scores, s.k, idx=self.idx, val=None)
+                k.csa2_topk(self.scores, s.k, idx=self.idx[0], val=None)
                 o1, l1 = k.csa2_sparse_attn("reuse", q, self.q_pos, self.cache, s.tau, self.N, k=s.k,
-                                            idx_in=self.idx, o=self.o[layer], lse=self.lse[layer], err=self.err)
+                                            idx_in=self.idx[0], o=self.o[layer], lse=self.lse[layer], err=self.err)
             else:
                 o1, l1 = k.csa2_sparse_attn("reindex", q, self.q_pos, self.cache, s.tau, self.N, k=s.k, q_ix=q_ix,
-                                            w=w, pool_k=s.pool_k, pool_io=self.pool, idx_out=self.idx,
+                                            w=w, pool_k=s.pool_k, pool_io=self.pool, idx_out=self.idx[layer],
                                             o=self.o[layer], lse=self.lse[layer], ws=self.ws_reindex,
                                             err=self.err)
             k.csa2_swa_attn(q, self.q_pos, self.swa_codes[layer], self.swa_scale[layer], s.tau, o=self.o_swa,

@@ -45,8 +45,10 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
 }
 
 // ------------------------------------------------------------------ E4M3
+// Round to nearest even, saturating at +-448; a result of zero is code 0 whatever its sign.
 __device__ __forceinline__ uint32_t e4m3_code(float v) {
-  return uint32_t(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+  const uint32_t c = uint32_t(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+  return (c & 0x7F) ? c : 0u;
 }
 
 // Exact value of an E4M3 code (bias 7; exponent 0 is subnormal with quantum 2^-9).

@@ -28,12 +28,13 @@ def _err():
 # ------------------------------------------------------------------ packers
 def _planted_latents(B, T, d, seed, dtype):
     x = normal((B, T, d), seed, "pack", d, device=DEV)
-    x[0, 0, :32] = 0.0                       # zero blocks
-    x[0, 1, :16] *= 1e-5                     # subnormal E4M3 scales
-    x[0, 2, :] *= 1e3                        # saturating E4M3 scales
-    x[min(1, B - 1), 3, 5] = 1e-40           # a subnormal input
-    x[0, 4, :] = 0.25                        # exact e2m1 ties after scaling
-    x[0, 5, :] = torch.tensor([0.75, -1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 0.5] * (d // 8))
+    t = lambda i: (T - 1 - i) if T > 6 else T - 1  # noqa: E731  (plant near the end: kept by a ring)
+    x[0, t(0), :32] = 0.0                    # zero blocks
+    x[0, t(1), :16] *= 1e-5                  # subnormal E4M3 scales
+    x[0, t(2), :] *= 1e3                     # saturating E4M3 scales
+    x[B - 1, t(3), 5] = 1e-40                # a subnormal input
+    x[0, t(4), :] = 0.25
+    x[0, t(5), :] = torch.tensor([0.75, -1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 0.5] * (d // 8))  # e2m1 ties
     return x.to(dtype)
 
 
