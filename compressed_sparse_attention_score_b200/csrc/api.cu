@@ -111,8 +111,8 @@ CSA2_EXPORT csa2_status csa2_index_score(const uint16_t *q_ix, const uint16_t *w
   if (B < 0 || Q < 0 || max_entries < 0 || (cand && P <= 0)) return fail(CSA2_ERR_INVALID_ARG, "bad size");
   if (!aligned16(q_ix)) return fail(CSA2_ERR_INVALID_ARG, "q_ix misaligned");
   const int n_out = cand ? P : max_entries;
-  if (n_out > 65535 * 128) return fail(CSA2_ERR_UNSUPPORTED, "more than 8388480 entries per row");
-  csa2::launch_index_score_scalar(q_ix, w, B, Q, q_pos, cand, P, n_out, *cache, scores, err, stream);
+  if (size_t(B) * Q > 65535) return fail(CSA2_ERR_UNSUPPORTED, "more than 65535 query rows per call");
+  csa2::launch_index_score_mma(q_ix, w, B, Q, q_pos, cand, P, n_out, *cache, scores, err, stream);
   return launched("csa2_index_score");
 }
 
@@ -147,16 +147,16 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
     const size_t need = csa2_workspace_size(mode, B, Q, max_entries, k, pool_k);
     if (!ws || ws_bytes < need) return fail(CSA2_ERR_INVALID_ARG, "workspace too small");
     const int n_out = mode == CSA2_MODE_FULL ? max_entries : pool_k;
-    if (n_out > 65535 * 128) return fail(CSA2_ERR_UNSUPPORTED, "more than 8388480 entries per row");
+    if (rows > 65535) return fail(CSA2_ERR_UNSUPPORTED, "more than 65535 query rows per call");
     float *scores = static_cast<float *>(ws);
     int32_t *sel = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + round256(size_t(rows) * n_out * 4));
     if (idx_out) sel = idx_out;
     if (mode == CSA2_MODE_FULL) {
-      csa2::launch_index_score_scalar(q_ix, w, B, Q, q_pos, nullptr, 0, max_entries, *cache, scores, err, stream);
+      csa2::launch_index_score_mma(q_ix, w, B, Q, q_pos, nullptr, 0, max_entries, *cache, scores, err, stream);
       csa2::launch_topk_rows(scores, nullptr, rows, max_entries, k, sel, nullptr, nullptr, stream);
       if (pool_k > 0) csa2::launch_topk_rows(scores, nullptr, rows, max_entries, pool_k, pool_io, nullptr, nullptr, stream);
     } else {
-      csa2::launch_index_score_scalar(q_ix, w, B, Q, q_pos, pool_io, pool_k, pool_k, *cache, scores, err, stream);
+      csa2::launch_index_score_mma(q_ix, w, B, Q, q_pos, pool_io, pool_k, pool_k, *cache, scores, err, stream);
       csa2::launch_topk_rows(scores, nullptr, rows, pool_k, k, sel, nullptr, pool_io, stream);
     }
     idx = sel;

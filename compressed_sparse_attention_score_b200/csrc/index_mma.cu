@@ -1,0 +1,297 @@
+// K3 (tensor-core form): lightning-indexer scores with block-scaled FP4 tcgen05 MMA.
+//
+// Scores s_n = sum_h w_h * relu(q^_h . k^_n) are one block-scaled FP4 GEMM per
+// 128-key tile: D[128 keys][64 heads] = K^ (e2m1, E8M0 per 32) x Q^^T, then a
+// weighted ReLU row reduction.  The e2m1 codes and E8M0 exponents of the cache
+// are consumed exactly as stored (kind::mxf4, scale vector 32), so the products
+// are exact and only the fp32 accumulation order differs from a plain sum.
+//
+// CTA = one query row x a contiguous range of key tiles.  Warp roles:
+//   warp 0     producer: cp.async of the tile's 128 x 64 B codes into a 64-byte
+//              swizzled K-major layout and of its 128 scale words into the
+//              32 x 4-word scale-factor atom; multistage ring of IM_STAGES;
+//   warp 1     MMA issuer (one lane): tcgen05.cp of the scale atom to TMEM, two
+//              K=64 MMAs into a double-buffered TMEM accumulator, tcgen05.commit;
+//   warps 2-5  epilogue: tcgen05.ld of the 64 head values of its 32 keys,
+//              weighted ReLU sum, coalesced fp32 score store.
+// The query heads are quantised to MXFP4 in the prologue (same codec as the keys).
+// Every mbarrier wait is time-bounded; on expiry the CTA drains and reports
+// CSA2_ERR_TIMEOUT instead of hanging.
+#include "common.cuh"
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace csa2 {
+using namespace sm100;
+
+namespace {
+constexpr int IM_STAGES = 8;
+constexpr int IM_LAG = 5;              // tiles between issuing a stage's copies and publishing it
+constexpr int IM_TILE = 128;           // keys per tile = MMA M
+constexpr int IM_N = 64;               // indexer heads = MMA N
+constexpr int IM_A_BYTES = IM_TILE * 64;
+constexpr int IM_STAGE_BYTES = 9216;   // 8192 codes + 512 scale atom, padded to 1024
+constexpr int IM_THREADS = 192;
+constexpr uint32_t IM_TMEM_COLS = 256;
+constexpr uint32_t COL_SFA = 128;      // two 4-column scale buffers (per accumulator)
+constexpr uint32_t COL_SFB = 136;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+
+constexpr int SM_STAGES = 0;
+constexpr int SM_B = IM_STAGES * IM_STAGE_BYTES;       // 64 x 64 B query codes
+constexpr int SM_SFB = SM_B + IM_N * 64;                // 512 B scale atom
+constexpr int SM_W = SM_SFB + 512;                      // 64 fp32 head weights
+constexpr int SM_BAR = SM_W + 256;                      // mbarriers
+constexpr int N_BARS = 2 * IM_STAGES + 5;
+constexpr int SM_MISC = SM_BAR + 8 * N_BARS;            // tmem base, abort flag
+constexpr int SM_TOTAL = SM_MISC + 16;
+constexpr size_t IM_SMEM_BYTES = SM_TOTAL + 1024;       // slack for 1024-byte alignment
+}  // namespace
+
+struct IndexMmaArgs {
+  const uint16_t *q_ix;
+  const uint16_t *w;
+  int Q;
+  const int32_t *q_pos;
+  const int32_t *cand;
+  int P;
+  int n_out;
+  csa2_cache c;
+  float *scores;
+  int32_t *err;
+  int chunk;  // tiles per CTA
+};
+
+// Physical slot of the key at score position pos of this row, or -1.
+__device__ __forceinline__ int64_t key_slot(const IndexMmaArgs &a, int row, int b, int nvis, int pos, bool report_bad) {
+  int64_t n = pos;
+  if (a.cand) {
+    if (pos >= a.P) return -1;
+    n = a.cand[int64_t(row) * a.P + pos];
+    if (report_bad && (n < -1 || n >= a.c.num_entries[b])) report(a.err, CSA2_ERR_INDEX);
+  }
+  if (n < 0 || n >= nvis) return -1;
+  const int64_t s = cache_slot(a.c, b, n);
+  if (s < 0 && report_bad) report(a.err, CSA2_ERR_INDEX);
+  return s;
+}
+
+__global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(IndexMmaArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM_BAR);
+  uint64_t *empty = full + IM_STAGES;
+  uint64_t *acc_full = empty + IM_STAGES;
+  uint64_t *acc_empty = acc_full + 2;
+  uint64_t *done = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM_MISC + 4);
+  float *ws = reinterpret_cast<float *>(smem + SM_W);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.y, b = row / a.Q;
+  const int nvis = visible_entries(a.c, b, a.q_pos[row]);
+  const int t_all = (a.n_out + IM_TILE - 1) / IM_TILE;
+  const int t_work = a.cand ? (a.P + IM_TILE - 1) / IM_TILE : (nvis + IM_TILE - 1) / IM_TILE;
+  const int t0 = blockIdx.x * a.chunk;
+  const int t1 = min(t0 + a.chunk, t_all);
+  const int ntiles = max(0, min(t1, t_work) - t0);
+
+  // ---------------------------------------------------------------- prologue
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, IM_TMEM_COLS);
+    tmem_relinquish();
+  } else if (warp == 1 && lane == 0) {
+    for (int s = 0; s < IM_STAGES; ++s) {
+      mbar_init(&full[s], 32);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  } else if (warp >= 2) {
+    // quantise the query heads: thread h < 64 owns head h (4 blocks of 32 values)
+    const int t = threadIdx.x - 64;
+    uint32_t sfword = 0;
+    if (t < IM_N) {
+      const uint16_t *qh = a.q_ix + (int64_t(row) * HI + t) * DI;
+      uint8_t *brow = smem + SM_B + t * 64;
+#pragma unroll 1
+      for (int g = 0; g < 4; ++g) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 u = reinterpret_cast<const uint4 *>(qh + 32 * g)[i];
+          const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            v[8 * i + 2 * j] = __uint_as_float(ww[j] << 16);
+            v[8 * i + 2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
+          }
+        }
+        float am = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+        int ex = -127;
+        uint32_t cw[4] = {0, 0, 0, 0};
+        if (am != 0.f) {
+          ex = e8m0_ceil_exponent(__fdiv_rn(am, 6.0f));
+          const float s = pow2f(ex);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) cw[i >> 3] |= e2m1_code(__fdiv_rn(v[i], s)) << (4 * (i & 7));
+        }
+        // 16 bytes = chunk g of this 64-byte row, at its swizzled position
+        *reinterpret_cast<uint4 *>(brow + ((g ^ ((t >> 1) & 3)) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        sfword |= uint32_t(ex + 127) << (8 * g);
+      }
+      ws[t] = bf16_to_f32(a.w[int64_t(row) * HI + t]);
+    }
+    // scale atom word of row r = t (rows 64..127 unused): lane-row r % 32, column r / 32
+    *reinterpret_cast<uint32_t *>(smem + SM_SFB + (t & 31) * 16 + (t >> 5) * 4) = sfword;
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    const uint32_t stages = smem_u32(smem + SM_STAGES);
+    int i = 0;
+    for (; i < ntiles; ++i) {
+      const int s = i % IM_STAGES;
+      if (!mbar_wait_bounded(&empty[s], ((i / IM_STAGES) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+      const int tile = t0 + i;
+      const uint32_t st = stages + s * IM_STAGE_BYTES;
+#pragma unroll 4
+      for (int j = 0; j < 16; ++j) {  // 512 chunks of 16 bytes
+        const int qd = lane + 32 * j, m = qd >> 2, c = qd & 3;
+        const int64_t slot = key_slot(a, row, b, nvis, tile * IM_TILE + m, c == 0);
+        if (slot >= 0)
+          cp_async_16(st + m * 64 + ((c ^ ((m >> 1) & 3)) << 4), a.c.ix_codes + slot * CSA2_IX_CODE_BYTES + c * 16);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {  // 128 scale words into the 32 x 4-word atom
+        const int m = lane + 32 * j;
+        const int64_t slot = key_slot(a, row, b, nvis, tile * IM_TILE + m, false);
+        if (slot >= 0)
+          cp_async_4(st + IM_A_BYTES + (m & 31) * 16 + (m >> 5) * 4, a.c.ix_scales + slot * CSA2_IX_SCALE_BYTES);
+      }
+      cp_async_commit();
+      if (i >= IM_LAG) {
+        cp_async_wait<IM_LAG>();
+        fence_proxy_async_smem();
+        mbar_arrive(&full[(i - IM_LAG) % IM_STAGES]);
+      }
+    }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    if (i == ntiles)
+      for (int k = max(0, ntiles - IM_LAG); k < ntiles; ++k) mbar_arrive(&full[k % IM_STAGES]);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t stages = smem_u32(smem + SM_STAGES);
+      const uint32_t bq = smem_u32(smem + SM_B);
+      tc_cp_32x128b_warpx4(tmem + COL_SFB, smem_desc(smem_u32(smem + SM_SFB), 16, 128, LAYOUT_SWIZZLE_NONE));
+      const uint64_t b0 = smem_desc(bq, 16, 512, LAYOUT_SWIZZLE_64B);
+      const uint64_t b1 = smem_desc(bq + 32, 16, 512, LAYOUT_SWIZZLE_64B);
+      constexpr uint32_t id0 = idesc_mxf4(IM_TILE, IM_N, 0, 0);
+      constexpr uint32_t id1 = idesc_mxf4(IM_TILE, IM_N, 2, 2);
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % IM_STAGES, acc = i & 1;
+        if (!mbar_wait_bounded(&full[s], (i / IM_STAGES) & 1, abort_flag, WAIT_LIMIT_NS)) break;
+        if (!mbar_wait_bounded(&acc_empty[acc], ((i >> 1) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+        tc_fence_after();
+        const uint32_t st = stages + s * IM_STAGE_BYTES;
+        const uint32_t sfa = tmem + COL_SFA + 4 * acc;
+        tc_cp_32x128b_warpx4(sfa, smem_desc(st + IM_A_BYTES, 16, 128, LAYOUT_SWIZZLE_NONE));
+        const uint32_t d = tmem + acc * IM_N;
+        tc_mma_mxf4(d, smem_desc(st, 16, 512, LAYOUT_SWIZZLE_64B), b0, id0, sfa, tmem + COL_SFB, false);
+        tc_mma_mxf4(d, smem_desc(st + 32, 16, 512, LAYOUT_SWIZZLE_64B), b1, id1, sfa, tmem + COL_SFB, true);
+        tc_commit(&empty[s]);
+        tc_commit(&acc_full[acc]);
+      }
+      tc_commit(done);  // fires once every tcgen05 op of this thread has completed
+      // wait for it even after an abort, so TMEM is never freed under a running MMA
+      const uint64_t t_start = globaltimer();
+      while (!mbar_try_wait(done, 0) && globaltimer() - t_start < WAIT_LIMIT_NS) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q4 = warp & 3;              // TMEM sub-partition of this warp
+    const int m = 32 * q4 + lane;         // key row within the tile
+    const float4 *w4 = reinterpret_cast<const float4 *>(ws);
+    for (int i = 0; i < ntiles; ++i) {
+      const int acc = i & 1;
+      if (!mbar_wait_bounded(&acc_full[acc], (i >> 1) & 1, abort_flag, WAIT_LIMIT_NS)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem + (uint32_t(32 * q4) << 16) + acc * IM_N;
+      uint32_t r0[32], r1[32];
+      tc_ld_32x32b_x32(taddr, r0);
+      tc_ld_32x32b_x32(taddr + 32, r1);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      float sc = 0.f;
+#pragma unroll
+      for (int h4 = 0; h4 < 8; ++h4) {
+        const float4 wv = w4[h4];
+        sc = fmaf(wv.x, fmaxf(__uint_as_float(r0[4 * h4]), 0.f), sc);
+        sc = fmaf(wv.y, fmaxf(__uint_as_float(r0[4 * h4 + 1]), 0.f), sc);
+        sc = fmaf(wv.z, fmaxf(__uint_as_float(r0[4 * h4 + 2]), 0.f), sc);
+        sc = fmaf(wv.w, fmaxf(__uint_as_float(r0[4 * h4 + 3]), 0.f), sc);
+      }
+#pragma unroll
+      for (int h4 = 0; h4 < 8; ++h4) {
+        const float4 wv = w4[8 + h4];
+        sc = fmaf(wv.x, fmaxf(__uint_as_float(r1[4 * h4]), 0.f), sc);
+        sc = fmaf(wv.y, fmaxf(__uint_as_float(r1[4 * h4 + 1]), 0.f), sc);
+        sc = fmaf(wv.z, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f), sc);
+        sc = fmaf(wv.w, fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f), sc);
+      }
+      const int pos = (t0 + i) * IM_TILE + m;
+      if (pos < a.n_out) {
+        const bool ok = key_slot(a, row, b, nvis, pos, false) >= 0;
+        a.scores[int64_t(row) * a.n_out + pos] = ok ? sc : -INFINITY;
+      }
+    }
+    // positions past the visible entries (no key tile was loaded for them)
+    if (!a.cand) {
+      const int lo = max(t0, t_work) * IM_TILE, hi = min(t1 * IM_TILE, a.n_out);
+      for (int pos = lo + threadIdx.x - 64; pos < hi; pos += 128) a.scores[int64_t(row) * a.n_out + pos] = -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, IM_TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) report(a.err, CSA2_ERR_TIMEOUT);
+}
+
+void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
+                            const int32_t *cand, int P, int n_out, const csa2_cache &c, float *scores, int32_t *err,
+                            cudaStream_t st) {
+  const int rows = B * Q;
+  if (n_out == 0 || rows == 0) return;
+  const int t_all = (n_out + IM_TILE - 1) / IM_TILE;
+  const int want = (2 * 148 + rows - 1) / rows;           // about two CTAs per SM in total
+  const int splits = max(1, min(min(want, (t_all + 7) / 8), 65535));
+  const int chunk = (t_all + splits - 1) / splits;
+  IndexMmaArgs a{q_ix, w, Q, q_pos, cand, P, n_out, c, scores, err, chunk};
+  set_smem_limit(index_score_mma_kernel, IM_SMEM_BYTES);
+  index_score_mma_kernel<<<dim3((t_all + chunk - 1) / chunk, rows), IM_THREADS, IM_SMEM_BYTES, st>>>(a);
+}
+
+}  // namespace csa2

@@ -25,6 +25,9 @@ void launch_pack_swa(const void *x, csa2_dtype dtype, int B, int T, const int32_
 void launch_index_score_scalar(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
                                const int32_t *cand, int P, int n_out, const csa2_cache &c, float *scores,
                                int32_t *err, cudaStream_t st);
+void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
+                            const int32_t *cand, int P, int n_out, const csa2_cache &c, float *scores, int32_t *err,
+                            cudaStream_t st);
 void launch_topk_rows(const float *scores, const int32_t *n_valid, int R, int N, int k, int32_t *idx, float *val,
                       const int32_t *map, cudaStream_t st);
 void launch_sparse_attn_scalar(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx,
