@@ -42,6 +42,7 @@ def parse():
     ap.add_argument("--workload", default="hier1m")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seqs", type=int, default=1)
+    ap.add_argument("--batch", type=int, default=0, help="override the sequence count (profiling runs)")
     return ap.parse_args()
 
 
@@ -350,6 +351,8 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     spec = W.CONFIGS[args.workload](seed=rank)
     assert spec.name == "hier1m", "bench.py times the hierarchical 1M-context decode workload"
+    if args.batch:
+        spec = W.scaled(spec, spec.tokens[0], B=args.batch)
     wl = Hier1M(spec, dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
