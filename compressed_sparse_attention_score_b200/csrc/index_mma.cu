@@ -6,10 +6,14 @@
 // are consumed exactly as stored (kind::mxf4, scale vector 32), so the products
 // are exact and only the fp32 accumulation order differs from a plain sum.
 //
-// CTA = one query row x a contiguous range of key tiles.  Warp roles:
-//   warp 0     producer: cp.async of the tile's 128 x 64 B codes into a 64-byte
-//              swizzled K-major layout and of its 128 scale words into the
-//              32 x 4-word scale-factor atom; multistage ring of IM_STAGES;
+// CTA = one query row x a contiguous range of key tiles.  Row m of a tile's A
+// operand holds tile entry e(m) = (m % 32) * 4 + m / 32, so the entries' scale
+// words, copied in their natural order, form the 32 x 4-word scale-factor atom
+// that tcgen05.cp expects (word w = (m % 32) * 4 + m / 32 = e).  Warp roles:
+//   warp 0     producer: for a run of whole 128-entry groups one TMA box of a
+//              4-D tensor map whose outer strides perform the row permutation
+//              (64-byte swizzle) plus one 512-byte bulk copy of the scales;
+//              for candidate lists, cp.async of each listed entry instead;
 //   warp 1     MMA issuer (one lane): tcgen05.cp of the scale atom to TMEM, two
 //              K=64 MMAs into a double-buffered TMEM accumulator, tcgen05.commit;
 //   warps 2-5  epilogue: tcgen05.ld of the 64 head values of its 32 keys,
@@ -17,6 +21,11 @@
 // The query heads are quantised to MXFP4 in the prologue (same codec as the keys).
 // Every mbarrier wait is time-bounded; on expiry the CTA drains and reports
 // CSA2_ERR_TIMEOUT instead of hanging.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
@@ -49,6 +58,7 @@ constexpr size_t IM_SMEM_BYTES = SM_TOTAL + 1024;       // slack for 1024-byte a
 }  // namespace
 
 struct IndexMmaArgs {
+  bool use_tma;
   const uint16_t *q_ix;
   const uint16_t *w;
   int Q;
@@ -76,7 +86,12 @@ __device__ __forceinline__ int64_t key_slot(const IndexMmaArgs &a, int row, int 
   return s;
 }
 
-__global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(IndexMmaArgs a) {
+// A-operand row of tile entry e and the inverse map.
+__device__ __forceinline__ int row_of_entry(int e) { return (e & 3) * 32 + (e >> 2); }
+__device__ __forceinline__ int entry_of_row(int m) { return (m & 31) * 4 + (m >> 5); }
+
+__global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                                        IndexMmaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM_BAR);
@@ -103,7 +118,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(IndexMma
     tmem_relinquish();
   } else if (warp == 1 && lane == 0) {
     for (int s = 0; s < IM_STAGES; ++s) {
-      mbar_init(&full[s], 32);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -162,37 +177,58 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(IndexMma
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     const uint32_t stages = smem_u32(smem + SM_STAGES);
-    int i = 0;
-    for (; i < ntiles; ++i) {
-      const int s = i % IM_STAGES;
-      if (!mbar_wait_bounded(&empty[s], ((i / IM_STAGES) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
-      const int tile = t0 + i;
-      const uint32_t st = stages + s * IM_STAGE_BYTES;
+    if (a.use_tma) {
+      if (lane == 0) {
+        for (int i = 0; i < ntiles; ++i) {
+          const int s = i % IM_STAGES;
+          if (!mbar_wait_bounded(&empty[s], ((i / IM_STAGES) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+          const uint32_t st = stages + s * IM_STAGE_BYTES;
+          const int64_t slot0 = cache_slot(a.c, b, int64_t(t0 + i) * IM_TILE);
+          if (slot0 >= 0 && (slot0 & (IM_TILE - 1)) == 0 && slot0 + IM_TILE <= a.c.num_slots) {
+            mbar_arrive_expect_tx(&full[s], IM_A_BYTES + 512);
+            tma_load_4d(st, &tmap, 0, 0, 0, int(slot0 / IM_TILE), &full[s]);
+            bulk_load(st + IM_A_BYTES, a.c.ix_scales + slot0 * CSA2_IX_SCALE_BYTES, 512, &full[s]);
+          } else {
+            report(a.err, CSA2_ERR_INDEX);  // a visible tile without a valid page: epilogue masks it
+            mbar_arrive(&full[s]);
+          }
+        }
+      }
+    } else {
+      int i = 0;
+      for (; i < ntiles; ++i) {
+        const int s = i % IM_STAGES;
+        if (!mbar_wait_bounded(&empty[s], ((i / IM_STAGES) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+        const int tile = t0 + i;
+        const uint32_t st = stages + s * IM_STAGE_BYTES;
 #pragma unroll 4
-      for (int j = 0; j < 16; ++j) {  // 512 chunks of 16 bytes
-        const int qd = lane + 32 * j, m = qd >> 2, c = qd & 3;
-        const int64_t slot = key_slot(a, row, b, nvis, tile * IM_TILE + m, c == 0);
-        if (slot >= 0)
-          cp_async_16(st + m * 64 + ((c ^ ((m >> 1) & 3)) << 4), a.c.ix_codes + slot * CSA2_IX_CODE_BYTES + c * 16);
-      }
+        for (int j = 0; j < 16; ++j) {  // 512 chunks of 16 bytes
+          const int qd = lane + 32 * j, e = qd >> 2, c = qd & 3, m = row_of_entry(e);
+          const int64_t slot = key_slot(a, row, b, nvis, tile * IM_TILE + e, c == 0);
+          if (slot >= 0)
+            cp_async_16(st + m * 64 + ((c ^ ((m >> 1) & 3)) << 4), a.c.ix_codes + slot * CSA2_IX_CODE_BYTES + c * 16);
+        }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {  // 128 scale words into the 32 x 4-word atom
-        const int m = lane + 32 * j;
-        const int64_t slot = key_slot(a, row, b, nvis, tile * IM_TILE + m, false);
-        if (slot >= 0)
-          cp_async_4(st + IM_A_BYTES + (m & 31) * 16 + (m >> 5) * 4, a.c.ix_scales + slot * CSA2_IX_SCALE_BYTES);
+        for (int j = 0; j < 4; ++j) {  // scale word of entry e at atom word e
+          const int e = lane + 32 * j;
+          const int64_t slot = key_slot(a, row, b, nvis, tile * IM_TILE + e, false);
+          if (slot >= 0) cp_async_4(st + IM_A_BYTES + e * 4, a.c.ix_scales + slot * CSA2_IX_SCALE_BYTES);
+        }
+        cp_async_commit();
+        if (i >= IM_LAG) {
+          cp_async_wait<IM_LAG>();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[(i - IM_LAG) % IM_STAGES]);
+        }
       }
-      cp_async_commit();
-      if (i >= IM_LAG) {
-        cp_async_wait<IM_LAG>();
-        fence_proxy_async_smem();
-        mbar_arrive(&full[(i - IM_LAG) % IM_STAGES]);
-      }
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (i == ntiles && lane == 0)
+        for (int k = max(0, ntiles - IM_LAG); k < ntiles; ++k) mbar_arrive(&full[k % IM_STAGES]);
     }
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    if (i == ntiles)
-      for (int k = max(0, ntiles - IM_LAG); k < ntiles; ++k) mbar_arrive(&full[k % IM_STAGES]);
+    __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -227,7 +263,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(IndexMma
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q4 = warp & 3;              // TMEM sub-partition of this warp
-    const int m = 32 * q4 + lane;         // key row within the tile
+    const int e = entry_of_row(32 * q4 + lane);  // tile entry of this thread's accumulator row
     const float4 *w4 = reinterpret_cast<const float4 *>(ws);
     for (int i = 0; i < ntiles; ++i) {
       const int acc = i & 1;
@@ -258,7 +294,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(IndexMma
         sc = fmaf(wv.z, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f), sc);
         sc = fmaf(wv.w, fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f), sc);
       }
-      const int pos = (t0 + i) * IM_TILE + m;
+      const int pos = (t0 + i) * IM_TILE + e;
       if (pos < a.n_out) {
         const bool ok = key_slot(a, row, b, nvis, pos, false) >= 0;
         a.scores[int64_t(row) * a.n_out + pos] = ok ? sc : -INFINITY;
@@ -280,6 +316,37 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(IndexMma
   if (threadIdx.x == 0 && *abort_flag) report(a.err, CSA2_ERR_TIMEOUT);
 }
 
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 4-D view of the indexer-code plane: (64 bytes, entry / 4 within a 128-entry
+// group [stride 256 B], entry % 4 [stride 64 B], group [stride 8192 B]).  A box
+// of (64, 32, 4, 1) lands entry e of the group at shared-memory row (e%4)*32 + e/4.
+bool make_code_map(CUtensorMap *m, const csa2_cache &c) {
+  auto enc = tensor_map_encoder();
+  if (!enc || (c.num_slots % IM_TILE) != 0 || c.num_slots / IM_TILE > (int64_t(1) << 31)) return false;
+  if ((reinterpret_cast<uintptr_t>(c.ix_scales) & 15) || (reinterpret_cast<uintptr_t>(c.ix_codes) & 15)) return false;
+  if (c.page_table ? (c.page_size % IM_TILE) != 0 : (c.seq_stride % IM_TILE) != 0) return false;
+  const cuuint64_t dims[4] = {64, 32, 4, cuuint64_t(c.num_slots / IM_TILE)};
+  const cuuint64_t strides[3] = {256, 64, uint64_t(IM_TILE) * 64};
+  const cuuint32_t box[4] = {64, 32, 4, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, c.ix_codes, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
 void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
                             const int32_t *cand, int P, int n_out, const csa2_cache &c, float *scores, int32_t *err,
                             cudaStream_t st) {
@@ -289,9 +356,12 @@ void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int 
   const int want = (2 * 148 + rows - 1) / rows;           // about two CTAs per SM in total
   const int splits = max(1, min(min(want, (t_all + 7) / 8), 65535));
   const int chunk = (t_all + splits - 1) / splits;
-  IndexMmaArgs a{q_ix, w, Q, q_pos, cand, P, n_out, c, scores, err, chunk};
+  CUtensorMap tmap;
+  memset(&tmap, 0, sizeof(tmap));
+  const bool use_tma = cand == nullptr && make_code_map(&tmap, c);
+  IndexMmaArgs a{use_tma, q_ix, w, Q, q_pos, cand, P, n_out, c, scores, err, chunk};
   set_smem_limit(index_score_mma_kernel, IM_SMEM_BYTES);
-  index_score_mma_kernel<<<dim3((t_all + chunk - 1) / chunk, rows), IM_THREADS, IM_SMEM_BYTES, st>>>(a);
+  index_score_mma_kernel<<<dim3((t_all + chunk - 1) / chunk, rows), IM_THREADS, IM_SMEM_BYTES, st>>>(tmap, a);
 }
 
 }  // namespace csa2
