@@ -180,10 +180,11 @@ class Hier1M:
         torch.cuda.synchronize()
         assert k.csa2_check(err) == 0
 
-    # kernels launched per step, by call: pack_kv 1, pack_swa 1 per layer, index_score 1, top-k 2 (Full) / 1,
-    # sparse attention 1, SWA attention 1, merge 1 per layer
+    # kernels launched per step, by call: pack_kv 1, pack_swa 1 per layer, index_score 1 and top-k 1 per
+    # Full/Reindex layer (the Full layer's top-512 and pool share one top-k launch), sparse attention 1,
+    # SWA attention 1, merge 1 per layer
     def launches_per_step(self):
-        return 1 + self.LAYERS * 1 + (1 + 2) + (self.LAYERS - 1) * 2 + self.LAYERS * 3
+        return 1 + self.LAYERS * 1 + self.LAYERS * 2 + self.LAYERS * 3
 
     def step(self, scan_events=None):
         k, s = self.k, self.spec
@@ -198,8 +199,7 @@ class Hier1M:
                 k.csa2_index_score(q_ix, w, self.q_pos, self.cache, self.N, scores=self.scores, err=self.err)
                 if scan_events:
                     scan_events[1].record()
-                k.csa2_topk(self.scores, s.pool_k, idx=self.pool, val=None)
-                k.csa2_topk(self.scores, s.k, idx=self.idx[0], val=None)
+                k.csa2_topk(self.scores, s.k, idx=self.idx[0], k2=s.pool_k, idx2=self.pool)
                 o1, l1 = k.csa2_sparse_attn("reuse", q, self.q_pos, self.cache, s.tau, self.N, k=s.k,
                                             idx_in=self.idx[0], o=self.o[layer], lse=self.lse[layer], err=self.err)
             else:

@@ -50,8 +50,8 @@ _SIGS = {
                        c_void_p, c_void_p], ctypes.c_int),
     "csa2_index_score": ([c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_int32, c_int32, _P,
                           c_void_p, c_void_p, c_void_p], ctypes.c_int),
-    "csa2_topk": ([c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_size_t,
-                   c_void_p], ctypes.c_int),
+    "csa2_topk": ([c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_int32, c_void_p,
+                   c_void_p, c_void_p], ctypes.c_int),
     "csa2_sparse_attn": ([ctypes.c_int, c_void_p, c_int32, c_int32, c_void_p, c_float, c_void_p, c_void_p,
                           c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int32, _P, c_void_p, c_void_p,
                           c_void_p, c_size_t, c_void_p, c_void_p], ctypes.c_int),
@@ -185,16 +185,17 @@ def csa2_index_score(q_ix, w, q_pos, cache, max_entries, cand=None, scores=None,
     return scores
 
 
-def csa2_topk(scores, k, n_valid=None, idx=None, val=None, ws=None, stream=None):
+def csa2_topk(scores, k, n_valid=None, idx=None, val=None, k2=0, idx2=None, val2=None, stream=None):
+    """Top-k positions of each row (and optionally a second top-k2 selection in the same pass)."""
     N = scores.shape[-1]
     R = scores.numel() // N if N else 0
     if idx is None:
         idx = torch.empty(scores.shape[:-1] + (k,), dtype=torch.int32, device=scores.device)
-    if val is None:
-        val = torch.empty(scores.shape[:-1] + (k,), dtype=torch.float32, device=scores.device)
-    _ok(_lib.csa2_topk(_ptr(scores), _ptr(n_valid), R, N, k, _ptr(idx), _ptr(val), _ptr(ws),
-                       0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)), "csa2_topk")
-    return idx, val
+    if k2 and idx2 is None:
+        idx2 = torch.empty(scores.shape[:-1] + (k2,), dtype=torch.int32, device=scores.device)
+    _ok(_lib.csa2_topk(_ptr(scores), _ptr(n_valid), R, N, k, _ptr(idx), _ptr(val), k2, _ptr(idx2), _ptr(val2),
+                       _stream(stream)), "csa2_topk")
+    return (idx, val) if not k2 else (idx, val, idx2, val2)
 
 
 def csa2_sparse_attn(mode, q, q_pos, cache, softmax_scale, max_entries, k=512, q_ix=None, w=None, pool_k=0,

@@ -117,11 +117,12 @@ CSA2_EXPORT csa2_status csa2_index_score(const uint16_t *q_ix, const uint16_t *w
 }
 
 CSA2_EXPORT csa2_status csa2_topk(const float *scores, const int32_t *n_valid, int32_t R, int32_t N, int32_t k,
-                                  int32_t *idx, float *val, void *ws, size_t ws_bytes, csa2_stream_t stream) {
-  (void)ws, (void)ws_bytes;
+                                  int32_t *idx, float *val, int32_t k2, int32_t *idx2, float *val2,
+                                  csa2_stream_t stream) {
   if (!scores || !idx) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
-  if (R < 0 || N < 0 || k < 1) return fail(CSA2_ERR_INVALID_ARG, "bad size");
-  csa2::launch_topk_rows(scores, n_valid, R, N, k, idx, val, nullptr, stream);
+  if (R < 0 || N < 0 || k < 1 || k2 < 0 || (k2 > 0 && !idx2)) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  if (int64_t(R) * 16 > INT32_MAX) return fail(CSA2_ERR_UNSUPPORTED, "too many rows");
+  csa2::launch_topk_cluster(scores, n_valid, R, N, k, idx, val, k2, k2 > 0 ? idx2 : nullptr, val2, nullptr, stream);
   return launched("csa2_topk");
 }
 
@@ -153,11 +154,11 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
     if (idx_out) sel = idx_out;
     if (mode == CSA2_MODE_FULL) {
       csa2::launch_index_score_mma(q_ix, w, B, Q, q_pos, nullptr, 0, max_entries, *cache, scores, err, stream);
-      csa2::launch_topk_rows(scores, nullptr, rows, max_entries, k, sel, nullptr, nullptr, stream);
-      if (pool_k > 0) csa2::launch_topk_rows(scores, nullptr, rows, max_entries, pool_k, pool_io, nullptr, nullptr, stream);
+      csa2::launch_topk_cluster(scores, nullptr, rows, max_entries, k, sel, nullptr, pool_k,
+                                pool_k > 0 ? pool_io : nullptr, nullptr, nullptr, stream);
     } else {
       csa2::launch_index_score_mma(q_ix, w, B, Q, q_pos, pool_io, pool_k, pool_k, *cache, scores, err, stream);
-      csa2::launch_topk_rows(scores, nullptr, rows, pool_k, k, sel, nullptr, pool_io, stream);
+      csa2::launch_topk_cluster(scores, nullptr, rows, pool_k, k, sel, nullptr, 0, nullptr, nullptr, pool_io, stream);
     }
     idx = sel;
   } else {

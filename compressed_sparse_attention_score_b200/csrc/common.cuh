@@ -112,4 +112,32 @@ __device__ __forceinline__ float key_score(uint32_t k) {
 }
 constexpr uint32_t KEY_NEG_INF = 0x007FFFFFu;  // score_key(-inf)
 
+// Exclusive block-wide prefix sum of v (blockDim a multiple of 32, at most 1024);
+// *total receives the block sum.  sm must hold 32 ints.  Contains __syncthreads.
+__device__ __forceinline__ int block_exclusive_scan_1024(int v, int *sm, int *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sm[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < nw ? sm[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    sm[lane] = t;
+  }
+  __syncthreads();
+  const int off = (warp ? sm[warp - 1] : 0) + x - v;
+  *total = sm[nw - 1];
+  __syncthreads();
+  return off;
+}
+
 }  // namespace csa2

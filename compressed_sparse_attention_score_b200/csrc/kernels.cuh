@@ -22,14 +22,11 @@ void launch_pack_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype, co
                     const int32_t *first_entry, const csa2_cache &c, int32_t *err, cudaStream_t st);
 void launch_pack_swa(const void *x, csa2_dtype dtype, int B, int T, const int32_t *pos, uint8_t *codes,
                      float *scale, int R, int32_t *err, cudaStream_t st);
-void launch_index_score_scalar(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
-                               const int32_t *cand, int P, int n_out, const csa2_cache &c, float *scores,
-                               int32_t *err, cudaStream_t st);
 void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
                             const int32_t *cand, int P, int n_out, const csa2_cache &c, float *scores, int32_t *err,
                             cudaStream_t st);
-void launch_topk_rows(const float *scores, const int32_t *n_valid, int R, int N, int k, int32_t *idx, float *val,
-                      const int32_t *map, cudaStream_t st);
+void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int N, int k0, int32_t *idx0, float *val0,
+                         int k1, int32_t *idx1, float *val1, const int32_t *map, cudaStream_t st);
 void launch_sparse_attn_scalar(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx,
                                int k, const csa2_cache &c, float *o, float *lse, int32_t *err, cudaStream_t st);
 void launch_swa_attn_scalar(const uint16_t *q, int B, int Q, const int32_t *q_pos, const uint8_t *codes,

@@ -169,10 +169,12 @@ csa2_status csa2_index_score(const uint16_t *q_ix, const uint16_t *w, int32_t B,
  *   j < n_valid[r] whose score is not -inf, ordered by score descending, then j
  *   ascending.  idx [R][k] receives the first k positions in ascending order,
  *   padded with -1; val [R][k] (optional) their scores (-inf for pads).
- *   ws may be NULL (this call needs no workspace).
+ *   A second selection of the same rows (k2 > 0 with idx2 [R][k2], val2 optional),
+ *   e.g. the candidate pool, is computed in the same passes; k2 = 0 for none.
+ *   No workspace is needed.  NaN scores give an unspecified selection.
  */
 csa2_status csa2_topk(const float *scores, const int32_t *n_valid, int32_t R, int32_t N,
-                      int32_t k, int32_t *idx, float *val, void *ws, size_t ws_bytes,
+                      int32_t k, int32_t *idx, float *val, int32_t k2, int32_t *idx2, float *val2,
                       csa2_stream_t stream);
 
 /*

@@ -61,7 +61,7 @@ def test_host_side_argument_checks(lib):
     c = csa2_cache()
     # NULL cache / inputs are rejected before any launch
     assert lib.csa2_pack_kv(None, None, 0, None, 1, 1, None, None, None, None) == 1
-    assert lib.csa2_topk(None, None, 1, 10, 5, None, None, None, 0, None) == 1
+    assert lib.csa2_topk(None, None, 1, 10, 5, None, None, 0, None, None, None) == 1
     assert lib.csa2_merge(None, None, None, None, 1, 512, None, None, None) == 1
     assert b"NULL" in lib.csa2_last_error_string()
     # a cache with planes but no layout

@@ -159,11 +159,11 @@ def test_index_score_rejects_bad_candidates():
     assert np.isfinite(got[:2]).all() and np.isneginf(got[2:]).all()
 
 
-@pytest.mark.parametrize("case", ["random", "ties", "short", "neg_inf", "pool"])
+@pytest.mark.parametrize("case", ["random", "ties", "short", "neg_inf", "pool", "long", "zeros"])
 def test_topk_rows(case):
     k_ = K()
     g = torch.Generator(device="cpu").manual_seed(7)
-    R, N, k = 5, 9000, 512
+    R, N, k, k2 = 5, 9000, 512, 0
     if case == "random":
         s = torch.randn((R, N), generator=g)
     elif case == "ties":
@@ -174,20 +174,32 @@ def test_topk_rows(case):
     elif case == "neg_inf":
         s = torch.randn((R, N), generator=g)
         s[torch.rand((R, N), generator=g) < 0.97] = -math.inf
-    else:
-        N, k = 70000, 16384
+    elif case == "pool":
+        N, k2 = 70000, 16384
         s = torch.randn((R, N), generator=g) * 100
+    elif case == "long":                        # the 2^20-entry rows of a Full scan (16-CTA clusters)
+        R, N, k2 = 3, 1 << 20, 16384
+        s = torch.randn((R, N), generator=g).abs() * 50
+        s[:, ::1000] = s[:, ::1000].round()      # some exact ties
+    else:                                       # most scores equal (a fully-ReLU-zeroed row)
+        N, k2 = 300000, 16384
+        s = torch.zeros((R, N))
+        s[:, 5::97] = torch.randn((R, len(range(5, N, 97))), generator=g)
     n_valid = torch.tensor([N, N - 1, N // 2, 511, 0][:R], dtype=torch.int32)
     sd = s.to(DEV)
-    idx, val = k_.csa2_topk(sd, k, n_valid=n_valid.to(DEV))
-    idx = to_np(idx)
+    val = torch.empty((R, k), dtype=torch.float32, device=DEV)
+    out = k_.csa2_topk(sd, k, n_valid=n_valid.to(DEV), val=val, k2=k2)
+    idx = to_np(out[0])
     val = to_np(val)
     for r in range(R):
-        ref = OC.topk(s[r].double().numpy(), k, int(n_valid[r]))
+        srow = s[r].double().numpy()
+        ref = OC.topk(srow, k, int(n_valid[r]))
         np.testing.assert_array_equal(idx[r], ref)      # same fp32 inputs: exact
         sel = idx[r][idx[r] >= 0]
         np.testing.assert_array_equal(val[r][: len(sel)], s[r].numpy()[sel])
         assert np.all(np.isneginf(val[r][len(sel):]))
+        if k2:
+            np.testing.assert_array_equal(to_np(out[2])[r], OC.topk(srow, k2, int(n_valid[r])))
 
 
 # ------------------------------------------------------------------ attention
