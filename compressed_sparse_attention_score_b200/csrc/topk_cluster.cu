@@ -1,8 +1,9 @@
 // K5 (cluster form): deterministic top-k of long score rows with a thread-block
 // cluster per row.
 //
-// The CS CTAs of a cluster split the row into contiguous chunks (each thread a
-// contiguous sub-range, so index order = (CTA, thread, element)).  Three radix
+// The CS CTAs of a cluster split the row into contiguous chunks, each CTA into 32
+// contiguous warp ranges read with coalesced loads (index order = (CTA, warp,
+// iteration, lane)), so ballots give ordered ranks inside a warp.  Three radix
 // passes (key bits 31..20, 19..8, 7..0) build per-CTA histograms in shared memory
 // that are summed across the cluster through distributed shared memory: each CTA
 // reduces one slice of bins over all peers, then gathers the full sums.  Up to two
@@ -65,25 +66,28 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
                                                                      const int32_t *__restrict__ n_valid, int N,
                                                                      Sel s0, Sel s1, int nsel,
                                                                      const int32_t *__restrict__ map) {
+  constexpr int U = 4;  // loads in flight per lane
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint32_t tk_smem[];
-  uint32_t(*hist)[TK_BINS] = reinterpret_cast<uint32_t(*)[TK_BINS]>(tk_smem);                   // [2][TK_BINS]
+  uint32_t(*hist)[TK_BINS] = reinterpret_cast<uint32_t(*)[TK_BINS]>(tk_smem);                         // [2][bins]
   uint32_t(*red)[TK_BINS / CS] = reinterpret_cast<uint32_t(*)[TK_BINS / CS]>(tk_smem + 2 * TK_BINS);  // [2][slice]
   __shared__ int scan_sm[32];
   __shared__ uint32_t prefix_s[2], rem_s[2];
   __shared__ int all_s[2], bin_s[2];
   __shared__ uint32_t above_s[2];
-  __shared__ int cta_tot[2][2];            // per selection: count above T, count equal to T
+  __shared__ int cta_tot[2][2];  // per selection: count above T, count equal to T
 
   const int r = int(cluster.block_rank());
   const int row = blockIdx.x / CS;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = n_valid ? max(0, min(N, n_valid[row])) : N;
   const float *srow = scores + int64_t(row) * N;
+  // CTA chunk, then one contiguous range per warp; lane l reads elements base + 32 u + l
   const int chunk = (n + CS - 1) / CS;
   const int c0 = min(n, r * chunk), c1 = min(n, c0 + chunk);
-  const int sub = (c1 - c0 + TK_THREADS - 1) / TK_THREADS;
-  const int j0 = min(c1, c0 + tid * sub), j1 = min(c1, j0 + sub);
+  const int wsub = (c1 - c0 + 31) / 32;
+  const int wb = min(c1, c0 + warp * wsub), we = min(c1, wb + wsub);
+  const uint32_t lt_mask = (1u << lane) - 1u;
   const Sel sel[2] = {s0, s1};
 
   if (tid < 2) {
@@ -100,17 +104,28 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
     for (int i = tid; i < 2 * TK_BINS; i += TK_THREADS) (&hist[0][0])[i] = 0;
     __syncthreads();
     const uint32_t pre0 = prefix_s[0], pre1 = prefix_s[1];
-    const int act0 = !all_s[0], act1 = nsel > 1 && !all_s[1];
-    for (int j = j0; j < j1; ++j) {
-      const uint32_t key = score_key(srow[j]);
-      if (key == KEY_NEG_INF) continue;
-      const uint32_t bin = (key >> sh) & mask;
-      if (pass == 0) {
-        atomicAdd(&hist[0][bin], 1u);
-      } else {
-        const uint32_t hi = key >> (sh + width);
-        if (act0 && hi == pre0) atomicAdd(&hist[0][bin], 1u);
-        if (act1 && hi == pre1) atomicAdd(&hist[1][bin], 1u);
+    const bool act0 = !all_s[0], act1 = nsel > 1 && !all_s[1];
+    for (int base = wb; base < we; base += 32 * U) {
+      float v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = base + 32 * u + lane;
+        v[u] = j < we ? srow[j] : -INFINITY;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t key = score_key(v[u]);
+        const bool valid = key != KEY_NEG_INF;
+        const uint32_t bin = (key >> sh) & mask;
+        if (pass == 0) {
+          // one atomic per distinct bin in the warp
+          const uint32_t peers = __match_any_sync(0xffffffffu, valid ? bin : 0xFFFFFFFFu);
+          if (valid && (peers & lt_mask) == 0) atomicAdd(&hist[0][bin], uint32_t(__popc(peers)));
+        } else if (valid) {
+          const uint32_t hi = key >> (sh + width);
+          if (act0 && hi == pre0) atomicAdd(&hist[0][bin], 1u);
+          if (act1 && hi == pre1) atomicAdd(&hist[1][bin], 1u);
+        }
       }
     }
     // ---- cluster-wide sums: reduce my slice over all peers, then gather every slice
@@ -159,27 +174,42 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
     __syncthreads();
   }
 
-  // ---- count, prefix over (cluster, thread), write in ascending position order
+  // ---- per-warp counts of keys above / equal to T (warp-uniform via ballots)
   uint32_t T[2];
-  int need[2], gt_t[2] = {0, 0}, eq_t[2] = {0, 0};
-  for (int s = 0; s < nsel; ++s) {
+  int need[2], gt_w[2] = {0, 0}, eq_w[2] = {0, 0};
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
     T[s] = all_s[s] ? KEY_NEG_INF : prefix_s[s];
     need[s] = all_s[s] ? 0 : int(rem_s[s]);
   }
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t key = score_key(srow[j]);
-    if (key == KEY_NEG_INF) continue;
-    for (int s = 0; s < nsel; ++s) {
-      gt_t[s] += key > T[s];
-      eq_t[s] += key == T[s];
+  for (int base = wb; base < we; base += 32 * U) {
+    float v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = base + 32 * u + lane;
+      v[u] = j < we ? srow[j] : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t key = score_key(v[u]);
+      const bool valid = key != KEY_NEG_INF;
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        if (s >= nsel) break;
+        gt_w[s] += __popc(__ballot_sync(0xffffffffu, valid && key > T[s]));
+        eq_w[s] += __popc(__ballot_sync(0xffffffffu, valid && key == T[s]));
+      }
     }
   }
+  // ---- exclusive prefix over (cluster rank, warp)
   int gt_off[2] = {0, 0}, eq_off[2] = {0, 0};
   for (int s = 0; s < nsel; ++s) {
     int tot;
-    gt_off[s] = block_exclusive_scan_1024(gt_t[s], scan_sm, &tot);
+    gt_off[s] = block_exclusive_scan_1024(lane == 0 ? gt_w[s] : 0, scan_sm, &tot);
+    gt_off[s] = __shfl_sync(0xffffffffu, gt_off[s], 0);
     if (tid == 0) cta_tot[s][0] = tot;
-    eq_off[s] = block_exclusive_scan_1024(eq_t[s], scan_sm, &tot);
+    eq_off[s] = block_exclusive_scan_1024(lane == 0 ? eq_w[s] : 0, scan_sm, &tot);
+    eq_off[s] = __shfl_sync(0xffffffffu, eq_off[s], 0);
     if (tid == 0) cta_tot[s][1] = tot;
   }
   cluster.sync();
@@ -195,28 +225,38 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
     eq_off[s] += eb;
     selected[s] = gall + min(eall, need[s]);
   }
-  cluster.sync();  // all peers read cta_tot before the CTA may exit
+  cluster.sync();  // every peer has read cta_tot before any CTA exits
+
+  // ---- write the chosen positions in ascending order
   for (int s = 0; s < nsel; ++s) {
-    const int k = sel[s].k;
+    const int k = sel[s].k, nd = need[s];
+    const uint32_t Ts = T[s];
     int32_t *orow = sel[s].idx + int64_t(row) * k;
     float *vrow = sel[s].val ? sel[s].val + int64_t(row) * k : nullptr;
     const int32_t *mrow = map ? map + int64_t(row) * N : nullptr;
     int g = gt_off[s], e = eq_off[s];
-    for (int j = j0; j < j1 && (g + min(e, need[s])) < k; ++j) {
-      const float v = srow[j];
-      const uint32_t key = score_key(v);
-      if (key == KEY_NEG_INF) continue;
-      int at = -1;
-      if (key > T[s]) {
-        at = g + min(e, need[s]);
-        ++g;
-      } else if (key == T[s]) {
-        if (e < need[s]) at = g + e;
-        ++e;
+    for (int base = wb; base < we && g + min(e, nd) < k; base += 32 * U) {
+      float v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = base + 32 * u + lane;
+        v[u] = j < we ? srow[j] : -INFINITY;
       }
-      if (at >= 0 && at < k) {
-        orow[at] = mrow ? mrow[j] : j;
-        if (vrow) vrow[at] = v;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t key = score_key(v[u]);
+        const bool valid = key != KEY_NEG_INF;
+        const bool is_gt = valid && key > Ts, is_eq = valid && key == Ts;
+        const uint32_t gm = __ballot_sync(0xffffffffu, is_gt), em = __ballot_sync(0xffffffffu, is_eq);
+        const int gbef = g + __popc(gm & lt_mask), ebef = e + __popc(em & lt_mask);
+        const int at = is_gt ? gbef + min(ebef, nd) : ((is_eq && ebef < nd) ? gbef + ebef : -1);
+        if (at >= 0 && at < k) {
+          const int j = base + 32 * u + lane;
+          orow[at] = mrow ? mrow[j] : j;
+          if (vrow) vrow[at] = v[u];
+        }
+        g += __popc(gm);
+        e += __popc(em);
       }
     }
     if (r == 0)
