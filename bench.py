@@ -169,8 +169,6 @@ class Hier1M:
         # outputs and scratch
         self.o = torch.empty((L, B, 1, 64, 512), dtype=torch.float32, device=dev)
         self.lse = torch.empty((L, B, 1, 64), dtype=torch.float32, device=dev)
-        self.o_swa = torch.empty((B, 1, 64, 512), dtype=torch.float32, device=dev)
-        self.l_swa = torch.empty((B, 1, 64), dtype=torch.float32, device=dev)
         self.scores = torch.empty((B, 1, N), dtype=torch.float32, device=dev)
         self.pool = torch.empty((B, 1, spec.pool_k), dtype=torch.int32, device=dev)
         self.idx = torch.empty((L, B, 1, spec.k), dtype=torch.int32, device=dev)   # per layer
@@ -180,11 +178,11 @@ class Hier1M:
         torch.cuda.synchronize()
         assert k.csa2_check(err) == 0
 
-    # kernels launched per step, by call: pack_kv 1, pack_swa 1 per layer, index_score 1 and top-k 1 per
-    # Full/Reindex layer (the Full layer's top-512 and pool share one top-k launch), sparse attention 1,
-    # SWA attention 1, merge 1 per layer
+    # kernels launched per step, by call: pack_kv 1; per layer pack_swa 1, indexer 1, top-k 1 (the Full layer's
+    # top-512 and pool share one launch) and one attention launch that covers the sparse branch, the SWA
+    # branch and their log-sum-exp merge
     def launches_per_step(self):
-        return 1 + self.LAYERS * 1 + self.LAYERS * 2 + self.LAYERS * 3
+        return 1 + self.LAYERS * 4
 
     def step(self, scan_events=None):
         k, s = self.k, self.spec
@@ -193,6 +191,7 @@ class Hier1M:
             k.csa2_pack_swa(self.swa_new[layer], self.swa_pos, self.swa_codes[layer], self.swa_scale[layer],
                             err=self.err)
             q, q_ix, w = self.q[layer], self.q_ix[layer], self.w[layer]
+            swa = dict(swa_codes=self.swa_codes[layer], swa_scale=self.swa_scale[layer])
             if layer == 0:
                 if scan_events:
                     scan_events[0].record()
@@ -200,17 +199,12 @@ class Hier1M:
                 if scan_events:
                     scan_events[1].record()
                 k.csa2_topk(self.scores, s.k, idx=self.idx[0], k2=s.pool_k, idx2=self.pool)
-                o1, l1 = k.csa2_sparse_attn("reuse", q, self.q_pos, self.cache, s.tau, self.N, k=s.k,
-                                            idx_in=self.idx[0], o=self.o[layer], lse=self.lse[layer], err=self.err)
+                k.csa2_sparse_attn("reuse", q, self.q_pos, self.cache, s.tau, self.N, k=s.k, idx_in=self.idx[0],
+                                   o=self.o[layer], lse=self.lse[layer], err=self.err, **swa)
             else:
-                o1, l1 = k.csa2_sparse_attn("reindex", q, self.q_pos, self.cache, s.tau, self.N, k=s.k, q_ix=q_ix,
-                                            w=w, pool_k=s.pool_k, pool_io=self.pool, idx_out=self.idx[layer],
-                                            o=self.o[layer], lse=self.lse[layer], ws=self.ws_reindex,
-                                            err=self.err)
-            k.csa2_swa_attn(q, self.q_pos, self.swa_codes[layer], self.swa_scale[layer], s.tau, o=self.o_swa,
-                            lse=self.l_swa, err=self.err)
-            k.csa2_merge(self.o[layer], self.lse[layer], self.o_swa, self.l_swa, o=self.o[layer],
-                         lse=self.lse[layer])
+                k.csa2_sparse_attn("reindex", q, self.q_pos, self.cache, s.tau, self.N, k=s.k, q_ix=q_ix, w=w,
+                                   pool_k=s.pool_k, pool_io=self.pool, idx_out=self.idx[layer], o=self.o[layer],
+                                   lse=self.lse[layer], ws=self.ws_reindex, err=self.err, **swa)
 
     def host_io(self):
         """Pinned host copies of one step's inputs and outputs (for the end-to-end run)."""

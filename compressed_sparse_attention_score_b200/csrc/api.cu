@@ -130,12 +130,20 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
                                          const int32_t *q_pos, float softmax_scale, const uint16_t *q_ix,
                                          const uint16_t *w, int32_t k, int32_t pool_k, int32_t *pool_io,
                                          const int32_t *idx_in, int32_t *idx_out, int32_t max_entries,
-                                         const csa2_cache *cache, float *o, float *lse, void *ws, size_t ws_bytes,
+                                         const csa2_cache *cache, const uint8_t *swa_codes, const float *swa_scale,
+                                         int32_t R, int32_t window, float *o, float *lse, void *ws, size_t ws_bytes,
                                          int32_t *err, csa2_stream_t stream) {
   if (csa2_status s = check_cache(cache, B)) return s;
   if (!q || !q_pos || !o || !lse) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (B < 0 || Q < 0 || k < 1 || pool_k < 0 || max_entries < 0) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  if (k > 512) return fail(CSA2_ERR_UNSUPPORTED, "k > 512");
+  if (!aligned16(q)) return fail(CSA2_ERR_INVALID_ARG, "q misaligned");
+  if (swa_codes) {
+    if (!swa_scale || window < 1 || window > 128 || R < window) return fail(CSA2_ERR_INVALID_ARG, "need 1 <= window <= 128, window <= R");
+    if (!aligned16(swa_codes)) return fail(CSA2_ERR_INVALID_ARG, "swa_codes misaligned");
+  }
   const int rows = B * Q;
+  if (rows > 65535 * 16) return fail(CSA2_ERR_UNSUPPORTED, "too many query rows per call");
   const int32_t *idx = nullptr;
   if (mode == CSA2_MODE_REUSE) {
     if (!idx_in) return fail(CSA2_ERR_INVALID_ARG, "REUSE needs idx_in");
@@ -164,7 +172,8 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
   } else {
     return fail(CSA2_ERR_INVALID_ARG, "bad mode");
   }
-  csa2::launch_sparse_attn_scalar(q, B, Q, q_pos, softmax_scale, idx, k, *cache, o, lse, err, stream);
+  csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, idx, k, cache, swa_codes, swa_codes ? swa_scale : nullptr, R,
+                        window, o, lse, err, stream);
   return launched("csa2_sparse_attn");
 }
 
@@ -173,8 +182,11 @@ CSA2_EXPORT csa2_status csa2_swa_attn(const uint16_t *q, int32_t B, int32_t Q, c
                                       float softmax_scale, float *o, float *lse, int32_t *err, csa2_stream_t stream) {
   if (!q || !q_pos || !swa_codes || !swa_scale || !o || !lse) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (B < 0 || Q < 0 || window < 1 || R < window) return fail(CSA2_ERR_INVALID_ARG, "need 1 <= window <= R");
-  if (!aligned16(swa_codes)) return fail(CSA2_ERR_INVALID_ARG, "swa_codes misaligned");
-  csa2::launch_swa_attn_scalar(q, B, Q, q_pos, swa_codes, swa_scale, R, window, softmax_scale, o, lse, err, stream);
+  if (window > 128) return fail(CSA2_ERR_UNSUPPORTED, "window > 128");
+  if (!aligned16(swa_codes) || !aligned16(q)) return fail(CSA2_ERR_INVALID_ARG, "swa_codes / q misaligned");
+  if (B * Q > 65535 * 16) return fail(CSA2_ERR_UNSUPPORTED, "too many query rows per call");
+  csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, nullptr, 0, nullptr, swa_codes, swa_scale, R, window, o, lse,
+                        err, stream);
   return launched("csa2_swa_attn");
 }
 

@@ -1,0 +1,458 @@
+// K6/K7/K8 (tensor-core form): attention of 64 query heads over a row's selected
+// global-KV entries and/or its sliding window, on tcgen05 (kind::f16).
+//
+// CTA = one query row x 32 heads.  Each key's 512-d vector is both key and value.
+// Keys come from two sources that share one softmax (so a CTA given both returns
+// the log-sum-exp merge of the two branches exactly):
+//   sparse  -- listed main-KV entries: e2m1 x E4M3-per-16 dequantised to fp16
+//              (exact: <= 6 significant bits, in fp16 range);
+//   window  -- SWA tokens: E4M3 codes to fp16 (exact); the token's fp32 scale is
+//              folded into the logit multiplier and into P.
+// Phase 1  S^T[key][head] = K Q^T per 128-key tile (M = 128 keys, N = 32 heads,
+//          K = 512 dims in 64-dim chunks, 128-byte swizzled K-major operands),
+//          all tiles resident in TMEM.
+// Phase 2  exact two-pass softmax over every key of the row, read from TMEM
+//          (per-head max / sum by warp reduce-scatter), P^T written to shared
+//          memory in fp16 (MN-major, 64-byte swizzle).
+// Phase 3  O^T[dim][head] = V^T P^T per 128-dim tile (M = 128 dims, N = 32 heads,
+//          K = keys in 16-key steps), V^T chunks MN-major with 128-byte swizzle,
+//          accumulated in TMEM.
+// Phase 4  O / sum and lse = max + log(sum), coalesced fp32 stores.
+// The dequantising threads fill a 4-deep ring of 16 KB operand buffers while the
+// single issuing thread drives the tensor core; every wait is time-bounded.
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace csa2 {
+using namespace sm100;
+
+namespace {
+constexpr int AM_THREADS = 256;
+constexpr int AM_HG = 32;          // heads per CTA = MMA N
+constexpr int AM_TILE = 128;       // keys per S^T tile
+constexpr int AM_MAXKEYS = 640;    // 512 listed entries + 128 window tokens
+constexpr int AM_STAGES = 4;
+constexpr int AM_STAGE = 16384;
+constexpr uint32_t AM_TMEM_COLS = 256;
+constexpr uint64_t AM_WAIT_NS = 2000000000ull;
+
+constexpr int SM_Q = 0;                              // 8 chunks x [32 heads x 128 B]
+constexpr int SM_P = SM_Q + 8 * 4096;                // P^T [640 keys x 64 B]
+constexpr int SM_STG = SM_P + AM_MAXKEYS * 64;       // 4 x 16 KB operand ring
+constexpr int SM_SLOT = SM_STG + AM_STAGES * AM_STAGE;
+constexpr int SM_MU = SM_SLOT + AM_MAXKEYS * 8;      // logit multiplier per key
+constexpr int SM_PV = SM_MU + AM_MAXKEYS * 4;        // P multiplier per key
+constexpr int SM_RED = SM_PV + AM_MAXKEYS * 4;       // [4 warps][32 heads]
+constexpr int SM_HM = SM_RED + 4 * 32 * 4;           // head max [32], head sum [32]
+constexpr int SM_BAR = SM_HM + 2 * 32 * 4;
+constexpr int SM_MISC = SM_BAR + 8 * (AM_STAGES + 1);
+constexpr int SM_TOTAL = SM_MISC + 16;
+constexpr size_t AM_SMEM = SM_TOTAL + 1024;
+}  // namespace
+
+struct AttnArgs {
+  const uint16_t *q;
+  int Q;
+  const int32_t *q_pos;
+  float tau;
+  // sparse source (idx == nullptr: none)
+  const int32_t *idx;
+  int k;
+  csa2_cache c;
+  // window source (codes == nullptr: none)
+  const uint8_t *codes;
+  const float *scale;
+  int R, window;
+  float *o, *lse;
+  int32_t *err;
+};
+
+// Offsets inside the swizzled operand layouts (bytes).
+// K-major, 128-byte rows, 1 KB atoms of 8 rows: 16-byte unit u of row r.
+__device__ __forceinline__ int kmaj128(int r, int u) { return (r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4); }
+// MN-major, 128-byte swizzle: element block (m / 64) at LBO 8192, K-row k: unit u of 8 M-elements.
+__device__ __forceinline__ int mnmaj128(int k, int mblk, int u) {
+  return mblk * 8192 + (k >> 3) * 1024 + (k & 7) * 128 + ((u ^ (k & 7)) << 4);
+}
+// MN-major, 64-byte swizzle (P^T): K-row k (key), unit u of 8 heads.
+__device__ __forceinline__ int mnmaj64(int k, int u) { return (k >> 3) * 512 + (k & 7) * 64 + ((u ^ ((k & 7) >> 1)) << 4); }
+
+// Raw bytes one thread dequantises: 32 consecutive dims of one key.
+struct Raw {
+  uint4 a, b;      // sparse: a = 16 bytes of codes; window: a, b = 32 E4M3 codes
+  uint32_t sc;     // sparse: the two E4M3 block scales (low 16 bits)
+};
+
+__device__ __forceinline__ void load_raw(const AttnArgs &p, const int64_t *slot, int nks, int key, int dim0, Raw &r) {
+  const int64_t s = slot[key];
+  if (s < 0) return;
+  if (key < nks) {
+    r.a = *reinterpret_cast<const uint4 *>(p.c.kv_codes + s * CSA2_MAIN_CODE_BYTES + dim0 / 2);
+    r.sc = *reinterpret_cast<const uint16_t *>(p.c.kv_scales + s * CSA2_MAIN_SCALE_BYTES + dim0 / 16);
+  } else {
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.codes + s * CSA2_SWA_DIM + dim0);
+    r.a = src[0];
+    r.b = src[1];
+  }
+}
+
+// 32 fp16 values (4 x 16 bytes) of one key from its raw bytes; zeros for a masked key.
+__device__ __forceinline__ void dequant32(const Raw &r, bool sparse, bool valid, uint4 (&out)[4]) {
+  if (!valid) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) out[i] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  uint32_t h[16];
+  if (sparse) {
+    const uint32_t s0 = cvt_e4m3x2_f16x2((r.sc & 0xFF) * 0x101u);
+    const uint32_t s1 = cvt_e4m3x2_f16x2(((r.sc >> 8) & 0xFF) * 0x101u);
+    const uint32_t w[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) h[i] = hmul2_u32(cvt_e2m1x2_f16x2((w[i >> 2] >> (8 * (i & 3))) & 0xFF), i < 8 ? s0 : s1);
+  } else {
+    const uint32_t w[8] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) h[i] = cvt_e4m3x2_f16x2((w[i >> 1] >> (16 * (i & 1))) & 0xFFFF);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) out[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+}
+
+// Max or sum over the 32 lanes of each of 32 per-lane values: afterwards lane l
+// holds the reduction of value index l.  31 shuffles (reduce-scatter butterfly).
+template <bool MAX>
+__device__ __forceinline__ float reduce_scatter32(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int width = 16; width >= 1; width >>= 1) {
+    const bool upper = lane & width;
+#pragma unroll
+    for (int i = 0; i < width; ++i) {
+      // keep the half selected by this lane's bit, send the other half
+      const float send = upper ? v[i] : v[i + width];
+      const float keep = upper ? v[i + width] : v[i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, width);
+      v[i] = MAX ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  return v[0];
+}
+
+__global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  int64_t *slot = reinterpret_cast<int64_t *>(smem + SM_SLOT);
+  float *mu = reinterpret_cast<float *>(smem + SM_MU);
+  float *pv = reinterpret_cast<float *>(smem + SM_PV);
+  float *red = reinterpret_cast<float *>(smem + SM_RED);
+  float *hmax = reinterpret_cast<float *>(smem + SM_HM);
+  float *hsum = hmax + 32;
+  uint64_t *mma_done = reinterpret_cast<uint64_t *>(smem + SM_BAR);
+  uint64_t *phase_done = mma_done + AM_STAGES;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM_MISC + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.x, hg = blockIdx.y;
+  const int b = row / p.Q;
+  const int pos = p.q_pos[row];
+
+  // ---------------------------------------------------------------- key list
+  const int nks = p.idx ? p.k : 0;
+  int lo = 0, nkw = 0;
+  if (p.codes && pos >= 0) {
+    lo = max(0, pos - p.window + 1);
+    nkw = pos - lo + 1;
+  }
+  const int nk = nks + nkw;
+  const int ntiles = (nk + AM_TILE - 1) / AM_TILE;
+  const int nvis = p.idx ? visible_entries(p.c, b, pos) : 0;
+  for (int j = tid; j < ntiles * AM_TILE; j += AM_THREADS) {
+    int64_t s = -1;
+    float m = 0.f, pm = 0.f;
+    if (j < nks) {
+      const int n = p.idx[int64_t(row) * p.k + j];
+      if (n != -1) {
+        if (n < -1 || n >= nvis) {
+          report(p.err, CSA2_ERR_INDEX);
+        } else {
+          s = cache_slot(p.c, b, n);
+          if (s < 0) report(p.err, CSA2_ERR_INDEX);
+        }
+      }
+      m = p.tau, pm = 1.f;
+    } else if (j < nk) {
+      s = int64_t(b) * p.R + (lo + (j - nks)) % p.R;
+      const float sc = p.scale[s];
+      m = p.tau * sc, pm = sc;
+    }
+    slot[j] = s;
+    mu[j] = m;
+    pv[j] = pm;
+  }
+  // ---------------------------------------------------------------- Q (bf16 -> fp16, K-major 128B swizzle)
+  {
+    const uint16_t *qrow = p.q + (int64_t(row) * H + hg * AM_HG) * D;
+    for (int it = tid; it < AM_HG * (D / 8); it += AM_THREADS) {
+      const int h = it / (D / 8), u8 = it % (D / 8);  // 8 dims per item
+      const uint4 raw = *reinterpret_cast<const uint4 *>(qrow + h * D + u8 * 8);
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      uint32_t o4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __half2 hv = __floats2half2_rn(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+        o4[i] = *reinterpret_cast<const uint32_t *>(&hv);
+      }
+      const int chunk = u8 / 8, u = u8 % 8;
+      *reinterpret_cast<uint4 *>(smem + SM_Q + chunk * 4096 + kmaj128(h, u)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, AM_TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    for (int i = 0; i < AM_STAGES; ++i) mbar_init(&mma_done[i], 1);
+    mbar_init(phase_done, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t stg = smem_u32(smem + SM_STG);
+  bool aborted = false;
+  int chunk_no = 0;  // operand buffers used so far (ring position)
+
+  // ---------------------------------------------------------------- phase 1: S^T = K Q^T
+  if (ntiles > 0) {
+    const int key_in = tid >> 1, half = tid & 1;  // 2 threads per key, 32 dims each
+    const int nch = ntiles * 8;
+    Raw nxt{};
+    {
+      const int key = key_in;
+      load_raw(p, slot, nks, key, 32 * half, nxt);
+    }
+    for (int i = 0; i < nch && !aborted; ++i, ++chunk_no) {
+      const int t = i >> 3, c = i & 7;
+      const int buf = chunk_no % AM_STAGES;
+      bool ok = true;
+      if (chunk_no >= AM_STAGES)
+        ok = mbar_wait_bounded(&mma_done[buf], ((chunk_no / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS);
+      const Raw cur = nxt;
+      if (i + 1 < nch) {
+        const int key = ((i + 1) >> 3) * AM_TILE + key_in;
+        nxt = Raw{};
+        load_raw(p, slot, nks, key, 64 * ((i + 1) & 7) + 32 * half, nxt);
+      }
+      const int key = t * AM_TILE + key_in;
+      uint4 out[4];
+      dequant32(cur, key < nks, slot[key] >= 0, out);
+      uint8_t *dst = smem + SM_STG + buf * AM_STAGE;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4 *>(dst + kmaj128(key_in, 4 * half + u)) = out[u];
+      fence_proxy_async_smem();
+      if (__syncthreads_or(!ok)) {
+        aborted = true;
+        break;
+      }
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, false, false);
+        const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_Q + c * 4096);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+          tc_mma_f16(tmem + t * AM_HG, smem_desc(a0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B),
+                     smem_desc(b0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B), id, c > 0 || s > 0);
+        tc_commit(&mma_done[buf]);
+      }
+    }
+    if (tid == 0) tc_commit(phase_done);
+  } else if (tid == 0) {
+    tc_commit(phase_done);
+  }
+  {
+    const bool ok = aborted ? false : mbar_wait_bounded(phase_done, 0, abort_flag, AM_WAIT_NS);
+    if (__syncthreads_or(!ok)) aborted = true;
+  }
+  tc_fence_after();
+
+  // ---------------------------------------------------------------- phase 2: softmax over all keys
+  if (!aborted && warp < 4) {
+    float mx[32];
+#pragma unroll
+    for (int h = 0; h < 32; ++h) mx[h] = -INFINITY;
+    for (int t = 0; t < ntiles; ++t) {
+      const int key = t * AM_TILE + 32 * warp + lane;
+      uint32_t r0[16], r1[16];
+      const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + t * AM_HG;
+      tc_ld_32x32b_x16(ta, r0);
+      tc_ld_32x32b_x16(ta + 16, r1);
+      tc_wait_ld();
+      if (slot[key] >= 0) {
+        const float m = mu[key];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+          mx[h] = fmaxf(mx[h], m * __uint_as_float(r0[h]));
+          mx[16 + h] = fmaxf(mx[16 + h], m * __uint_as_float(r1[h]));
+        }
+      }
+    }
+    red[warp * 32 + lane] = reduce_scatter32<true>(mx);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (warp == 0)
+      hmax[lane] = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane]));
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    float m_h[32], sm[32];
+#pragma unroll
+    for (int h = 0; h < 32; ++h) {
+      m_h[h] = hmax[h];
+      sm[h] = 0.f;
+    }
+    for (int t = 0; t < ntiles; ++t) {
+      const int key = t * AM_TILE + 32 * warp + lane;
+      uint32_t r0[16], r1[16];
+      const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + t * AM_HG;
+      tc_ld_32x32b_x16(ta, r0);
+      tc_ld_32x32b_x16(ta + 16, r1);
+      tc_wait_ld();
+      const bool valid = slot[key] >= 0;
+      const float m = mu[key], pm = pv[key];
+      uint32_t ph[16];
+#pragma unroll
+      for (int h = 0; h < 32; h += 2) {
+        const float x0 = m * __uint_as_float(h < 16 ? r0[h] : r1[h - 16]);
+        const float x1 = m * __uint_as_float(h + 1 < 16 ? r0[h + 1] : r1[h - 15]);
+        const float e0 = (valid && m_h[h] != -INFINITY) ? __expf(x0 - m_h[h]) : 0.f;
+        const float e1 = (valid && m_h[h + 1] != -INFINITY) ? __expf(x1 - m_h[h + 1]) : 0.f;
+        sm[h] += e0;
+        sm[h + 1] += e1;
+        const __half2 hp = __floats2half2_rn(e0 * pm, e1 * pm);
+        ph[h >> 1] = *reinterpret_cast<const uint32_t *>(&hp);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<uint4 *>(smem + SM_P + mnmaj64(key, u)) =
+            make_uint4(ph[4 * u], ph[4 * u + 1], ph[4 * u + 2], ph[4 * u + 3]);
+    }
+    red[warp * 32 + lane] = reduce_scatter32<false>(sm);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (warp == 0) hsum[lane] = (red[lane] + red[32 + lane]) + (red[64 + lane] + red[96 + lane]);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  // ---------------------------------------------------------------- phase 3: O^T = V^T P^T
+  const int nkc = (ntiles * AM_TILE) / 64;  // 64-key chunks (masked keys carry P = 0, V = 0)
+  if (!aborted && nkc > 0) {
+    const int key_in = tid >> 2, qd = tid & 3;  // 4 threads per key, 32 dims each
+    const int nch = nkc * 4;
+    Raw nxt{};
+    load_raw(p, slot, nks, key_in, 32 * qd, nxt);
+    for (int i = 0; i < nch && !aborted; ++i, ++chunk_no) {
+      const int jc = i >> 2, d = i & 3;
+      const int buf = chunk_no % AM_STAGES;
+      bool ok = true;
+      if (chunk_no >= AM_STAGES)
+        ok = mbar_wait_bounded(&mma_done[buf], ((chunk_no / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS);
+      const Raw cur = nxt;
+      if (i + 1 < nch) {
+        nxt = Raw{};
+        load_raw(p, slot, nks, ((i + 1) >> 2) * 64 + key_in, 128 * ((i + 1) & 3) + 32 * qd, nxt);
+      }
+      const int key = jc * 64 + key_in;
+      uint4 out[4];
+      dequant32(cur, key < nks, slot[key] >= 0, out);
+      uint8_t *dst = smem + SM_STG + buf * AM_STAGE;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<uint4 *>(dst + mnmaj128(key_in, qd >> 1, 4 * (qd & 1) + u)) = out[u];
+      fence_proxy_async_smem();
+      if (__syncthreads_or(!ok)) {
+        aborted = true;
+        break;
+      }
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, true, true);
+        const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_P);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+          tc_mma_f16(tmem + d * AM_HG, smem_desc(a0 + 2048 * s, 8192, 1024, LAYOUT_SWIZZLE_128B),
+                     smem_desc(b0 + (8 * jc + 2 * s) * 512, 16, 512, LAYOUT_SWIZZLE_64B), id, jc > 0 || s > 0);
+        tc_commit(&mma_done[buf]);
+      }
+    }
+  }
+  if (tid == 0) tc_commit(phase_done);
+  {
+    const bool ok = aborted ? false : mbar_wait_bounded(phase_done, 1, abort_flag, AM_WAIT_NS);
+    if (__syncthreads_or(!ok)) aborted = true;
+  }
+  tc_fence_after();
+
+  // ---------------------------------------------------------------- phase 4: normalise and store
+  if (warp < 4) {
+    float inv[32];
+#pragma unroll
+    for (int h = 0; h < 32; ++h) {
+      const float s = aborted ? 0.f : hsum[h];
+      inv[h] = s > 0.f ? 1.f / s : 0.f;
+    }
+    float *orow = p.o + (int64_t(row) * H + hg * AM_HG) * D;
+    for (int d = 0; d < 4; ++d) {
+      uint32_t r0[16], r1[16];
+      if (!aborted && nkc > 0) {
+        const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + d * AM_HG;
+        tc_ld_32x32b_x16(ta, r0);
+        tc_ld_32x32b_x16(ta + 16, r1);
+        tc_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r0[i] = r1[i] = 0u;
+      }
+      const int dim = 128 * d + 32 * warp + lane;
+#pragma unroll
+      for (int h = 0; h < 16; ++h) {
+        orow[h * D + dim] = __uint_as_float(r0[h]) * inv[h];
+        orow[(16 + h) * D + dim] = __uint_as_float(r1[h]) * inv[16 + h];
+      }
+    }
+    if (warp == 0) {
+      const float s = aborted ? 0.f : hsum[lane];
+      p.lse[int64_t(row) * H + hg * AM_HG + lane] = s > 0.f ? hmax[lane] + logf(s) : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, AM_TMEM_COLS);
+  }
+  if (tid == 0 && aborted) report(p.err, CSA2_ERR_TIMEOUT);
+}
+
+void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
+                     const csa2_cache *c, const uint8_t *codes, const float *scale, int R, int window, float *o,
+                     float *lse, int32_t *err, cudaStream_t st) {
+  if (B * Q == 0) return;
+  AttnArgs a{};
+  a.q = q, a.Q = Q, a.q_pos = q_pos, a.tau = tau;
+  a.idx = idx, a.k = idx ? k : 0;
+  if (c) a.c = *c;
+  a.codes = codes, a.scale = scale, a.R = R, a.window = window;
+  a.o = o, a.lse = lse, a.err = err;
+  set_smem_limit(attn_mma_kernel, AM_SMEM);
+  attn_mma_kernel<<<dim3(B * Q, H / AM_HG), AM_THREADS, AM_SMEM, st>>>(a);
+}
+
+}  // namespace csa2

@@ -27,11 +27,9 @@ void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int 
                             cudaStream_t st);
 void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int N, int k0, int32_t *idx0, float *val0,
                          int k1, int32_t *idx1, float *val1, const int32_t *map, cudaStream_t st);
-void launch_sparse_attn_scalar(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx,
-                               int k, const csa2_cache &c, float *o, float *lse, int32_t *err, cudaStream_t st);
-void launch_swa_attn_scalar(const uint16_t *q, int B, int Q, const int32_t *q_pos, const uint8_t *codes,
-                            const float *scale, int R, int window, float tau, float *o, float *lse, int32_t *err,
-                            cudaStream_t st);
+void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
+                     const csa2_cache *c, const uint8_t *codes, const float *scale, int R, int window, float *o,
+                     float *lse, int32_t *err, cudaStream_t st);
 void launch_merge(const float *o1, const float *l1, const float *o2, const float *l2, int64_t rows, int D_,
                   float *o, float *lse, cudaStream_t st);
 

@@ -186,9 +186,14 @@ csa2_status csa2_topk(const float *scores, const int32_t *n_valid, int32_t R, in
  *   REINDEX: q_ix, w score the entries listed in pool_io [B][Q][pool_k]; top-k of them.
  *   REUSE:   idx_in [B][Q][k] given entry indices (-1 = none; order free).
  *   idx_out [B][Q][k] (optional, FULL/REINDEX) receives the chosen entries, ascending.
+ *   k <= 512.
  * Per head: logits tau * q . v_j over the chosen entries, v_j the dequantised
  * 512-d main entry used as key and value; o [B][Q][64][512] fp32 = softmax-weighted
  * sum, lse [B][Q][64] fp32 natural-log normaliser; no entries -> o = 0, lse = -inf.
+ * Optional sliding-window branch in the same call: when swa_codes != NULL the
+ * window of each query (as csa2_swa_attn: ring [B][R], window <= 128) joins the
+ * same softmax, so o / lse are the log-sum-exp merge of the two branches
+ * (what csa2_merge of the separate results gives).  swa_codes = NULL: none.
  * ws: csa2_workspace_size(mode, ...) bytes (may be NULL for REUSE).
  * Device errors: an index outside the visible entries -> CSA2_ERR_INDEX, skipped.
  */
@@ -196,15 +201,17 @@ csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int32_t B, int32
                              const int32_t *q_pos, float softmax_scale, const uint16_t *q_ix,
                              const uint16_t *w, int32_t k, int32_t pool_k, int32_t *pool_io,
                              const int32_t *idx_in, int32_t *idx_out, int32_t max_entries,
-                             const csa2_cache *cache, float *o, float *lse, void *ws,
-                             size_t ws_bytes, int32_t *err, csa2_stream_t stream);
+                             const csa2_cache *cache, const uint8_t *swa_codes,
+                             const float *swa_scale, int32_t R, int32_t window, float *o,
+                             float *lse, void *ws, size_t ws_bytes, int32_t *err,
+                             csa2_stream_t stream);
 
 /*
  * Sliding-window branch ("从V4到V4.1 Flash", sections "CSA2 机制下的全局 KV 共享与局部
  * 滑动窗口隔离" (per-layer SWA cache) and "SWA 有界重放" (128 tokens)).
  *   Window of a query at p: positions max(0, p - window + 1) .. p, read from the
- *   ring written by csa2_pack_swa (slot t mod R, R >= window).  Keys = values =
- *   E4M3 code * fp32 scale.  Same o / lse as csa2_sparse_attn.
+ *   ring written by csa2_pack_swa (slot t mod R, R >= window, window <= 128).
+ *   Keys = values = E4M3 code * fp32 scale.  Same o / lse as csa2_sparse_attn.
  */
 csa2_status csa2_swa_attn(const uint16_t *q, int32_t B, int32_t Q, const int32_t *q_pos,
                           const uint8_t *swa_codes, const float *swa_scale, int32_t R,

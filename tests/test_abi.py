@@ -78,7 +78,9 @@ def test_host_side_argument_checks(lib):
     assert lib.csa2_swa_attn(addr, 1, 1, addr, addr, addr, 64, 128, 1.0, addr, addr, None, None) == 1
     c.ratio = 1
     assert lib.csa2_sparse_attn(7, addr, 1, 1, addr, 1.0, None, None, 512, 0, None, None, None, 16,
-                                ctypes.byref(c), addr, addr, None, 0, None, None) == 1
+                                ctypes.byref(c), None, None, 0, 0, addr, addr, None, 0, None, None) == 1
+    assert lib.csa2_sparse_attn(2, addr, 1, 1, addr, 1.0, None, None, 1024, 0, None, addr, None, 16,
+                                ctypes.byref(c), None, None, 0, 0, addr, addr, None, 0, None, None) == 3
     assert lib.csa2_sparse_attn(0, addr, 1, 1, addr, 1.0, addr, addr, 512, 0, None, None, None, 16,
-                                ctypes.byref(c), addr, addr, None, 0, None, None) == 1
+                                ctypes.byref(c), None, None, 0, 0, addr, addr, None, 0, None, None) == 1
     assert b"workspace" in lib.csa2_last_error_string()

@@ -244,8 +244,12 @@ def test_merge_matches_oracle_and_aliases():
 
 
 def _decode_layer_parity(spec, cache, mode, layer, rings, codes, scale, pool=None, pool_k=0, idx_in=None,
-                         oracle_caches=None):
-    """Run one layer on the GPU (sparse + SWA + merge) and compare with the oracle per sequence."""
+                         oracle_caches=None, fused=False):
+    """Run one layer on the GPU (sparse + SWA + merge) and compare with the oracle per sequence.
+
+    fused=True passes the SWA ring to csa2_sparse_attn (one softmax over both key sets);
+    otherwise the branches run separately and csa2_merge combines them.
+    """
     k = K()
     q, q_ix, w, q_pos = W.query_tensors(spec, layer, DEV)
     err = _err()
@@ -253,10 +257,16 @@ def _decode_layer_parity(spec, cache, mode, layer, rings, codes, scale, pool=Non
     pool_io = pool
     if mode == "full" and pool_k:
         pool_io = torch.empty((spec.B, 1, pool_k), dtype=torch.int32, device=DEV)
-    o1, l1 = k.csa2_sparse_attn(mode, q, q_pos, cache, spec.tau, spec.max_entries, k=spec.k, q_ix=q_ix, w=w,
-                                pool_k=pool_k, pool_io=pool_io, idx_in=idx_in, idx_out=idx_out, err=err)
-    o2, l2 = k.csa2_swa_attn(q, q_pos, codes, scale, spec.tau, err=err)
-    o, lse = k.csa2_merge(o1, l1, o2, l2)
+    if fused:
+        o, lse = k.csa2_sparse_attn(mode, q, q_pos, cache, spec.tau, spec.max_entries, k=spec.k, q_ix=q_ix, w=w,
+                                    pool_k=pool_k, pool_io=pool_io, idx_in=idx_in, idx_out=idx_out, err=err,
+                                    swa_codes=codes, swa_scale=scale)
+        o1 = l1 = None
+    else:
+        o1, l1 = k.csa2_sparse_attn(mode, q, q_pos, cache, spec.tau, spec.max_entries, k=spec.k, q_ix=q_ix,
+                                    w=w, pool_k=pool_k, pool_io=pool_io, idx_in=idx_in, idx_out=idx_out, err=err)
+        o2, l2 = k.csa2_swa_attn(q, q_pos, codes, scale, spec.tau, err=err)
+        o, lse = k.csa2_merge(o1, l1, o2, l2)
     assert k.csa2_check(err) == 0
     same_rows = 0
     ref_pools = np.full((spec.B, 1, max(pool_k, 1)), -1, np.int64)
@@ -286,7 +296,8 @@ def _decode_layer_parity(spec, cache, mode, layer, rings, codes, scale, pool=Non
             same_rows += 1
             fill_main(c, spec, b, ref_idx, gen_device=DEV)
             ref = OC.decode_layer("reuse", c, 0, pos, qb, spec.tau, rings[b], idx=ref_idx)
-            check_attention(to_np(o1[b, 0]), to_np(l1[b, 0]), *ref["sparse"], f"{mode} sparse b={b}")
+            if o1 is not None:
+                check_attention(to_np(o1[b, 0]), to_np(l1[b, 0]), *ref["sparse"], f"{mode} sparse b={b}")
             check_attention(to_np(o[b, 0]), to_np(lse[b, 0]), ref["o"], ref["lse"], f"{mode} merged b={b}")
     assert same_rows >= max(1, spec.B - 1)
     # the oracle's own selections, for the layers that consume them
@@ -294,12 +305,24 @@ def _decode_layer_parity(spec, cache, mode, layer, rings, codes, scale, pool=Non
             torch.from_numpy(ref_pools).to(torch.int32).to(DEV))
 
 
-def test_full_decode_tiny_config():
+@pytest.mark.parametrize("fused", [False, True])
+def test_full_decode_tiny_config(fused):
     spec = W.tiny_full()
     cache = gpu_cache(spec)
     codes, scale, rings = _swa_state(spec, 0)
     oc = [oracle_seq(spec, b, main_rows=[], gen_device=DEV) for b in range(spec.B)]
-    _decode_layer_parity(spec, cache, "full", 0, rings, codes, scale, oracle_caches=oc)
+    _decode_layer_parity(spec, cache, "full", 0, rings, codes, scale, oracle_caches=oc, fused=fused)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_reuse_decode_scaled_fused_variant(fused):
+    spec = W.scaled(W.reuse64k(), [3000, 600, 9000], B=3)
+    cache = gpu_cache(spec)
+    codes, scale, rings = _swa_state(spec, 1)
+    idx = W.reuse_indices(spec, DEV)
+    idx[1, 0, 100:] = -1
+    oc = [oracle_seq(spec, b, main_rows=[], gen_device=DEV) for b in range(spec.B)]
+    _decode_layer_parity(spec, cache, "reuse", 1, rings, codes, scale, idx_in=idx, oracle_caches=oc, fused=fused)
 
 
 def test_reuse_decode_scaled():
@@ -341,7 +364,7 @@ def test_hierarchical_full_then_reindex_scaled():
     for layer in (1, 2):
         codes, scale, rings = _swa_state(spec, layer)
         _decode_layer_parity(spec, cache, "reindex", layer, rings, codes, scale, pool=pool, pool_k=spec.pool_k,
-                             oracle_caches=oc)
+                             oracle_caches=oc, fused=layer == 2)
     # the Reuse layers after it consume the Full layer's indices
     codes, scale, rings = _swa_state(spec, 5)
     _decode_layer_parity(spec, cache, "reuse", 5, rings, codes, scale, idx_in=idx_full, oracle_caches=oc)
