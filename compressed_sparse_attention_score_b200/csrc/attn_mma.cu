@@ -35,6 +35,7 @@ constexpr int AM_HG = 32;          // heads per CTA = MMA N
 constexpr int AM_TILE = 128;       // keys per S^T tile
 constexpr int AM_MAXKEYS = 640;    // 512 listed entries + 128 window tokens
 constexpr int AM_STAGES = 4;
+constexpr int AM_PF = 4;           // chunks of raw key bytes in flight per thread
 constexpr int AM_STAGE = 16384;
 constexpr uint32_t AM_TMEM_COLS = 256;
 constexpr uint64_t AM_WAIT_NS = 2000000000ull;
@@ -231,46 +232,51 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   int chunk_no = 0;  // operand buffers used so far (ring position)
 
   // ---------------------------------------------------------------- phase 1: S^T = K Q^T
+  // Raw bytes of the next AM_PF chunks are kept in flight in a register ring.
   if (ntiles > 0) {
     const int key_in = tid >> 1, half = tid & 1;  // 2 threads per key, 32 dims each
     const int nch = ntiles * 8;
-    Raw nxt{};
-    {
-      const int key = key_in;
-      load_raw(p, slot, nks, key, 32 * half, nxt);
+    Raw ring[AM_PF];
+#pragma unroll
+    for (int u = 0; u < AM_PF; ++u) {
+      ring[u] = Raw{};
+      if (u < nch) load_raw(p, slot, nks, (u >> 3) * AM_TILE + key_in, 64 * (u & 7) + 32 * half, ring[u]);
     }
-    for (int i = 0; i < nch && !aborted; ++i, ++chunk_no) {
-      const int t = i >> 3, c = i & 7;
-      const int buf = chunk_no % AM_STAGES;
-      bool ok = true;
-      if (chunk_no >= AM_STAGES)
-        ok = mbar_wait_bounded(&mma_done[buf], ((chunk_no / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS);
-      const Raw cur = nxt;
-      if (i + 1 < nch) {
-        const int key = ((i + 1) >> 3) * AM_TILE + key_in;
-        nxt = Raw{};
-        load_raw(p, slot, nks, key, 64 * ((i + 1) & 7) + 32 * half, nxt);
-      }
-      const int key = t * AM_TILE + key_in;
-      uint4 out[4];
-      dequant32(cur, key < nks, slot[key] >= 0, out);
-      uint8_t *dst = smem + SM_STG + buf * AM_STAGE;
+    for (int i0 = 0; i0 < nch && !aborted; i0 += AM_PF) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4 *>(dst + kmaj128(key_in, 4 * half + u)) = out[u];
-      fence_proxy_async_smem();
-      if (__syncthreads_or(!ok)) {
-        aborted = true;
-        break;
-      }
-      if (tid == 0) {
-        tc_fence_after();
-        constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, false, false);
-        const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_Q + c * 4096);
+      for (int u = 0; u < AM_PF; ++u) {
+        const int i = i0 + u;
+        if (i >= nch || aborted) break;
+        const int t = i >> 3, c = i & 7;
+        const int buf = chunk_no % AM_STAGES;
+        bool ok = true;
+        if (chunk_no >= AM_STAGES)
+          ok = mbar_wait_bounded(&mma_done[buf], ((chunk_no / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS);
+        const int key = t * AM_TILE + key_in;
+        uint4 out[4];
+        dequant32(ring[u], key < nks, slot[key] >= 0, out);
+        const int inext = i + AM_PF;
+        ring[u] = Raw{};
+        if (inext < nch) load_raw(p, slot, nks, (inext >> 3) * AM_TILE + key_in, 64 * (inext & 7) + 32 * half, ring[u]);
+        uint8_t *dst = smem + SM_STG + buf * AM_STAGE;
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-          tc_mma_f16(tmem + t * AM_HG, smem_desc(a0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B),
-                     smem_desc(b0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B), id, c > 0 || s > 0);
-        tc_commit(&mma_done[buf]);
+        for (int v = 0; v < 4; ++v) *reinterpret_cast<uint4 *>(dst + kmaj128(key_in, 4 * half + v)) = out[v];
+        fence_proxy_async_smem();
+        if (__syncthreads_or(!ok)) {
+          aborted = true;
+          break;
+        }
+        if (tid == 0) {
+          tc_fence_after();
+          constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, false, false);
+          const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_Q + c * 4096);
+#pragma unroll
+          for (int s = 0; s < 4; ++s)
+            tc_mma_f16(tmem + t * AM_HG, smem_desc(a0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B),
+                       smem_desc(b0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B), id, c > 0 || s > 0);
+          tc_commit(&mma_done[buf]);
+        }
+        ++chunk_no;
       }
     }
     if (tid == 0) tc_commit(phase_done);
@@ -355,40 +361,48 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   if (!aborted && nkc > 0) {
     const int key_in = tid >> 2, qd = tid & 3;  // 4 threads per key, 32 dims each
     const int nch = nkc * 4;
-    Raw nxt{};
-    load_raw(p, slot, nks, key_in, 32 * qd, nxt);
-    for (int i = 0; i < nch && !aborted; ++i, ++chunk_no) {
-      const int jc = i >> 2, d = i & 3;
-      const int buf = chunk_no % AM_STAGES;
-      bool ok = true;
-      if (chunk_no >= AM_STAGES)
-        ok = mbar_wait_bounded(&mma_done[buf], ((chunk_no / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS);
-      const Raw cur = nxt;
-      if (i + 1 < nch) {
-        nxt = Raw{};
-        load_raw(p, slot, nks, ((i + 1) >> 2) * 64 + key_in, 128 * ((i + 1) & 3) + 32 * qd, nxt);
-      }
-      const int key = jc * 64 + key_in;
-      uint4 out[4];
-      dequant32(cur, key < nks, slot[key] >= 0, out);
-      uint8_t *dst = smem + SM_STG + buf * AM_STAGE;
+    Raw ring[AM_PF];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        *reinterpret_cast<uint4 *>(dst + mnmaj128(key_in, qd >> 1, 4 * (qd & 1) + u)) = out[u];
-      fence_proxy_async_smem();
-      if (__syncthreads_or(!ok)) {
-        aborted = true;
-        break;
-      }
-      if (tid == 0) {
-        tc_fence_after();
-        constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, true, true);
-        const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_P);
+    for (int u = 0; u < AM_PF; ++u) {
+      ring[u] = Raw{};
+      if (u < nch) load_raw(p, slot, nks, (u >> 2) * 64 + key_in, 128 * (u & 3) + 32 * qd, ring[u]);
+    }
+    for (int i0 = 0; i0 < nch && !aborted; i0 += AM_PF) {
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-          tc_mma_f16(tmem + d * AM_HG, smem_desc(a0 + 2048 * s, 8192, 1024, LAYOUT_SWIZZLE_128B),
-                     smem_desc(b0 + (8 * jc + 2 * s) * 512, 16, 512, LAYOUT_SWIZZLE_64B), id, jc > 0 || s > 0);
-        tc_commit(&mma_done[buf]);
+      for (int u = 0; u < AM_PF; ++u) {
+        const int i = i0 + u;
+        if (i >= nch || aborted) break;
+        const int jc = i >> 2, d = i & 3;
+        const int buf = chunk_no % AM_STAGES;
+        bool ok = true;
+        if (chunk_no >= AM_STAGES)
+          ok = mbar_wait_bounded(&mma_done[buf], ((chunk_no / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS);
+        const int key = jc * 64 + key_in;
+        uint4 out[4];
+        dequant32(ring[u], key < nks, slot[key] >= 0, out);
+        const int inext = i + AM_PF;
+        ring[u] = Raw{};
+        if (inext < nch) load_raw(p, slot, nks, (inext >> 2) * 64 + key_in, 128 * (inext & 3) + 32 * qd, ring[u]);
+        uint8_t *dst = smem + SM_STG + buf * AM_STAGE;
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<uint4 *>(dst + mnmaj128(key_in, qd >> 1, 4 * (qd & 1) + v)) = out[v];
+        fence_proxy_async_smem();
+        if (__syncthreads_or(!ok)) {
+          aborted = true;
+          break;
+        }
+        if (tid == 0) {
+          tc_fence_after();
+          constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, true, true);
+          const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_P);
+#pragma unroll
+          for (int s = 0; s < 4; ++s)
+            tc_mma_f16(tmem + d * AM_HG, smem_desc(a0 + 2048 * s, 8192, 1024, LAYOUT_SWIZZLE_128B),
+                       smem_desc(b0 + (8 * jc + 2 * s) * 512, 16, 512, LAYOUT_SWIZZLE_64B), id, jc > 0 || s > 0);
+          tc_commit(&mma_done[buf]);
+        }
+        ++chunk_no;
       }
     }
   }

@@ -195,25 +195,32 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
         }
       }
     } else {
+      // Gather path: lane l resolves the slots of tile entries l, l+32, l+64, l+96 once
+      // per tile (coalesced candidate loads, next tile prefetched), then shuffles them
+      // to the lanes that copy each 16-byte chunk.
+      auto resolve = [&](int tile, int64_t (&sl)[4]) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sl[j] = tile < t0 + ntiles ? key_slot(a, row, b, nvis, tile * IM_TILE + lane + 32 * j, true) : -1;
+      };
+      int64_t cur[4], nxt[4];
+      resolve(t0, cur);
       int i = 0;
       for (; i < ntiles; ++i) {
         const int s = i % IM_STAGES;
+        resolve(t0 + i + 1, nxt);
         if (!mbar_wait_bounded(&empty[s], ((i / IM_STAGES) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
-        const int tile = t0 + i;
         const uint32_t st = stages + s * IM_STAGE_BYTES;
-#pragma unroll 4
-        for (int j = 0; j < 16; ++j) {  // 512 chunks of 16 bytes
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {  // 512 chunks of 16 bytes: chunk qd = lane + 32 j
           const int qd = lane + 32 * j, e = qd >> 2, c = qd & 3, m = row_of_entry(e);
-          const int64_t slot = key_slot(a, row, b, nvis, tile * IM_TILE + e, c == 0);
+          // entry e = 8 j + lane / 4 lives in lane e % 32, register j / 4
+          const int64_t slot = __shfl_sync(0xffffffffu, cur[j >> 2], e & 31);
           if (slot >= 0)
             cp_async_16(st + m * 64 + ((c ^ ((m >> 1) & 3)) << 4), a.c.ix_codes + slot * CSA2_IX_CODE_BYTES + c * 16);
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {  // scale word of entry e at atom word e
-          const int e = lane + 32 * j;
-          const int64_t slot = key_slot(a, row, b, nvis, tile * IM_TILE + e, false);
-          if (slot >= 0) cp_async_4(st + IM_A_BYTES + e * 4, a.c.ix_scales + slot * CSA2_IX_SCALE_BYTES);
-        }
+        for (int j = 0; j < 4; ++j)  // scale word of entry e = lane + 32 j at atom word e
+          if (cur[j] >= 0) cp_async_4(st + IM_A_BYTES + (lane + 32 * j) * 4, a.c.ix_scales + cur[j] * CSA2_IX_SCALE_BYTES);
         cp_async_commit();
         if (i >= IM_LAG) {
           cp_async_wait<IM_LAG>();
@@ -221,6 +228,8 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
           __syncwarp();
           if (lane == 0) mbar_arrive(&full[(i - IM_LAG) % IM_STAGES]);
         }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
       }
       cp_async_wait<0>();
       fence_proxy_async_smem();

@@ -31,32 +31,57 @@ struct Sel {
   float *val;
 };
 
-// Highest bin b (scanning down from the top) at which the running count reaches rem:
-// returns b and the count strictly above it.  Uses warp 0; result in *out.
-__device__ void find_bin(const uint32_t *h, int nbins, uint32_t rem, int *out_bin, uint32_t *out_above) {
-  const int lane = threadIdx.x & 31;
-  const int per = nbins / 32;
-  // lane l covers bins [nbins - per*(l+1), nbins - per*l), scanned top-down
-  uint32_t sum = 0;
-  for (int i = 0; i < per; ++i) sum += h[nbins - per * lane - 1 - i];
-  uint32_t incl = sum;
+// Threshold search with the whole CTA: the bin at which the count of keys in bins
+// at or above it first reaches rem (scanning from the top), the count strictly
+// above that bin, and the total.  Thread t owns bins nb-4t-4 .. nb-4t-1.
+__device__ void find_bin_block(const uint32_t *h, int nb, uint32_t rem, int *scan_sm, int *out_bin,
+                               uint32_t *out_above, uint32_t *out_total) {
+  const int t = threadIdx.x;
+  uint32_t c[4] = {0, 0, 0, 0}, sum = 0;
+  if (4 * t < nb) {
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+    for (int i = 0; i < 4; ++i) c[i] = h[nb - 4 * t - 1 - i], sum += c[i];
   }
-  const uint32_t excl = incl - sum;
-  if (excl < rem && incl >= rem) {
+  int total;
+  const uint32_t excl = uint32_t(block_exclusive_scan_1024(int(sum), scan_sm, &total));
+  if (t == 0) *out_total = uint32_t(total);
+  if (excl < rem && excl + sum >= rem) {
     uint32_t cum = excl;
-    for (int i = 0; i < per; ++i) {
-      const int bin = nbins - per * lane - 1 - i;
-      if (cum + h[bin] >= rem) {
-        *out_bin = bin;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (cum + c[i] >= rem) {
+        *out_bin = nb - 4 * t - 1 - i;
         *out_above = cum;
         break;
       }
-      cum += h[bin];
+      cum += c[i];
     }
+  }
+  __syncthreads();
+}
+
+// Sum the per-CTA histograms [nh][nb] across the cluster (each CTA reduces one
+// slice of bins over all peers, then gathers every slice).
+template <int CS>
+__device__ __forceinline__ void cluster_hist_sum(cg::cluster_group &cluster, uint32_t (*hist)[TK_BINS],
+                                                 uint32_t (*red)[TK_BINS / CS], int nh, int nb, int r) {
+  if constexpr (CS > 1) {
+    cluster.sync();
+    const int slice = nb / CS;
+    for (int h = 0; h < nh; ++h)
+      for (int i = threadIdx.x; i < slice; i += TK_THREADS) {
+        uint32_t t = 0;
+#pragma unroll
+        for (int p = 0; p < CS; ++p) t += cluster.map_shared_rank(&hist[h][0], p)[r * slice + i];
+        red[h][i] = t;
+      }
+    cluster.sync();
+    for (int h = 0; h < nh; ++h)
+      for (int i = threadIdx.x; i < nb; i += TK_THREADS)
+        hist[h][i] = cluster.map_shared_rank(&red[h][0], i / slice)[i % slice];
+    cluster.sync();  // peers finished reading my red[] before it is rewritten
+  } else {
+    __syncthreads();
   }
 }
 }  // namespace
@@ -66,7 +91,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
                                                                      const int32_t *__restrict__ n_valid, int N,
                                                                      Sel s0, Sel s1, int nsel,
                                                                      const int32_t *__restrict__ map) {
-  constexpr int U = 4;  // loads in flight per lane
+  constexpr int U = 4;        // loads in flight per lane
+  constexpr int SAMPLE = 16;  // one group of 32 keys in SAMPLE is sampled
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint32_t tk_smem[];
   uint32_t(*hist)[TK_BINS] = reinterpret_cast<uint32_t(*)[TK_BINS]>(tk_smem);                         // [2][bins]
@@ -74,7 +100,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   __shared__ int scan_sm[32];
   __shared__ uint32_t prefix_s[2], rem_s[2];
   __shared__ int all_s[2], bin_s[2];
-  __shared__ uint32_t above_s[2];
+  __shared__ uint32_t above_s[2], total_s[2];
   __shared__ int cta_tot[2][2];  // per selection: count above T, count equal to T
 
   const int r = int(cluster.block_rank());
@@ -89,89 +115,113 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   const int wb = min(c1, c0 + warp * wsub), we = min(c1, wb + wsub);
   const uint32_t lt_mask = (1u << lane) - 1u;
   const Sel sel[2] = {s0, s1};
+  const int kbig = nsel > 1 ? max(s0.k, s1.k) : s0.k;
+
+  auto zero_hist = [&]() {
+    for (int i = tid; i < 2 * TK_BINS; i += TK_THREADS) (&hist[0][0])[i] = 0;
+    __syncthreads();
+  };
+  // warp-aggregated histogram of the 12 top key bits for keys whose bin >= lo_bin
+  auto top_hist = [&](int step, int lo_bin) {
+    for (int base = wb; base < we; base += 32 * U * step) {
+      float v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = base + 32 * u * step + lane;
+        v[u] = j < we ? srow[j] : -INFINITY;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t key = score_key(v[u]);
+        const int bin = int(key >> 20);
+        const bool take = key != KEY_NEG_INF && bin >= lo_bin;
+        const uint32_t peers = __match_any_sync(0xffffffffu, take ? uint32_t(bin) : 0xFFFFFFFFu);
+        if (take && (peers & lt_mask) == 0) atomicAdd(&hist[0][bin], uint32_t(__popc(peers)));
+      }
+    }
+  };
+
+  // ---- sampled lower bound: keys below it cannot reach the larger selection (checked below)
+  zero_hist();
+  top_hist(SAMPLE, 0);
+  cluster_hist_sum<CS>(cluster, hist, red, 1, TK_BINS, r);
+  {
+    const uint32_t target = uint32_t(kbig / SAMPLE) + uint32_t(kbig / (2 * SAMPLE)) + 32;
+    if (tid == 0) bin_s[0] = 0;
+    find_bin_block(hist[0], TK_BINS, target, scan_sm, &bin_s[0], &above_s[0], &total_s[0]);
+  }
+  int lo_bin = total_s[0] >= uint32_t(kbig / SAMPLE) + uint32_t(kbig / (2 * SAMPLE)) + 32 ? bin_s[0] : 0;
 
   if (tid < 2) {
     prefix_s[tid] = 0;
     rem_s[tid] = uint32_t(sel[tid].k);
     all_s[tid] = 0;
   }
-
-  for (int pass = 0; pass < 3; ++pass) {
-    const int width = pass == 2 ? 8 : 12;
-    const int sh = pass == 0 ? 20 : (pass == 1 ? 8 : 0), nb = 1 << width;
-    const uint32_t mask = uint32_t(nb - 1);
-    const int nh = pass == 0 ? 1 : nsel;  // the first pass is shared by both selections
-    for (int i = tid; i < 2 * TK_BINS; i += TK_THREADS) (&hist[0][0])[i] = 0;
+  // ---- pass 0 (top 12 bits) over keys at or above the bound; redo without it if too few
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    zero_hist();
+    top_hist(1, lo_bin);
+    cluster_hist_sum<CS>(cluster, hist, red, 1, TK_BINS, r);
+    find_bin_block(hist[0], TK_BINS, 1u, scan_sm, &bin_s[1], &above_s[1], &total_s[1]);  // only for the total
+    if (total_s[1] >= uint32_t(kbig) || lo_bin == 0) break;
+    lo_bin = 0;
+  }
+  const uint32_t counted = total_s[1];
+  if (nsel > 1) {
+    for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[1][i] = hist[0][i];
+  }
+  __syncthreads();
+  for (int s = 0; s < nsel; ++s) {
+    // with the bound in place fewer than all keys are counted, but then at least kbig are
+    if (lo_bin == 0 && counted <= uint32_t(sel[s].k)) {
+      if (tid == 0) all_s[s] = 1;
+      __syncthreads();
+      continue;
+    }
+    find_bin_block(hist[s], TK_BINS, rem_s[s], scan_sm, &bin_s[s], &above_s[s], &total_s[s]);
+    if (tid == 0) {
+      rem_s[s] -= above_s[s];
+      prefix_s[s] = uint32_t(bin_s[s]);
+    }
     __syncthreads();
+  }
+
+  // ---- passes 1, 2 (bits 19..8, 7..0) over keys matching each selection's prefix
+  for (int pass = 1; pass < 3; ++pass) {
+    const int width = pass == 2 ? 8 : 12;
+    const int sh = pass == 1 ? 8 : 0, nb = 1 << width;
+    const uint32_t mask = uint32_t(nb - 1);
+    zero_hist();
     const uint32_t pre0 = prefix_s[0], pre1 = prefix_s[1];
     const bool act0 = !all_s[0], act1 = nsel > 1 && !all_s[1];
-    for (int base = wb; base < we; base += 32 * U) {
-      float v[U];
+    if (act0 || act1) {
+      for (int base = wb; base < we; base += 32 * U) {
+        float v[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = base + 32 * u + lane;
-        v[u] = j < we ? srow[j] : -INFINITY;
-      }
+        for (int u = 0; u < U; ++u) {
+          const int j = base + 32 * u + lane;
+          v[u] = j < we ? srow[j] : -INFINITY;
+        }
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const uint32_t key = score_key(v[u]);
-        const bool valid = key != KEY_NEG_INF;
-        const uint32_t bin = (key >> sh) & mask;
-        if (pass == 0) {
-          // one atomic per distinct bin in the warp
-          const uint32_t peers = __match_any_sync(0xffffffffu, valid ? bin : 0xFFFFFFFFu);
-          if (valid && (peers & lt_mask) == 0) atomicAdd(&hist[0][bin], uint32_t(__popc(peers)));
-        } else if (valid) {
-          const uint32_t hi = key >> (sh + width);
+        for (int u = 0; u < U; ++u) {
+          const uint32_t key = score_key(v[u]);
+          if (key == KEY_NEG_INF) continue;
+          const uint32_t hi = key >> (sh + width), bin = (key >> sh) & mask;
           if (act0 && hi == pre0) atomicAdd(&hist[0][bin], 1u);
           if (act1 && hi == pre1) atomicAdd(&hist[1][bin], 1u);
         }
       }
     }
-    // ---- cluster-wide sums: reduce my slice over all peers, then gather every slice
-    if constexpr (CS > 1) {
-      cluster.sync();
-      const int slice = nb / CS;
-      for (int h = 0; h < nh; ++h)
-        for (int i = tid; i < slice; i += TK_THREADS) {
-          uint32_t t = 0;
-#pragma unroll
-          for (int p = 0; p < CS; ++p) t += cluster.map_shared_rank(&hist[h][0], p)[r * slice + i];
-          red[h][i] = t;
-        }
-      cluster.sync();
-      for (int h = 0; h < nh; ++h)
-        for (int i = tid; i < nb; i += TK_THREADS) hist[h][i] = cluster.map_shared_rank(&red[h][0], i / slice)[i % slice];
-      cluster.sync();  // peers finished reading my red[] before it is rewritten
-    }
-    if (pass == 0 && nsel > 1) {
-      for (int i = tid; i < nb; i += TK_THREADS) hist[1][i] = hist[0][i];
-    }
-    __syncthreads();
-    // ---- threshold bin per selection
-    if (tid < 32) {
-      for (int s = 0; s < nsel; ++s) {
-        if (all_s[s]) continue;
-        if (pass == 0) {
-          uint32_t tot = 0;
-          for (int i = tid; i < nb; i += 32) tot += hist[s][i];
-#pragma unroll
-          for (int o = 16; o; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-          if (tot <= uint32_t(sel[s].k)) {
-            if (tid == 0) all_s[s] = 1;
-            continue;
-          }
-        }
-        find_bin(hist[s], nb, rem_s[s], &bin_s[s], &above_s[s]);
-        __syncwarp();
-        if (tid == 0) {
-          rem_s[s] -= above_s[s];
-          prefix_s[s] = (prefix_s[s] << width) | uint32_t(bin_s[s]);
-        }
-        __syncwarp();
+    cluster_hist_sum<CS>(cluster, hist, red, nsel, nb, r);
+    for (int s = 0; s < nsel; ++s) {
+      if (all_s[s]) continue;
+      find_bin_block(hist[s], nb, rem_s[s], scan_sm, &bin_s[s], &above_s[s], &total_s[s]);
+      if (tid == 0) {
+        rem_s[s] -= above_s[s];
+        prefix_s[s] = (prefix_s[s] << width) | uint32_t(bin_s[s]);
       }
+      __syncthreads();
     }
-    __syncthreads();
   }
 
   // ---- per-warp counts of keys above / equal to T (warp-uniform via ballots)
