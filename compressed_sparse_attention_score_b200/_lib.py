@@ -59,6 +59,10 @@ _SIGS = {
                        c_void_p, c_void_p, c_void_p, c_void_p], ctypes.c_int),
     "csa2_merge": ([c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p],
                    ctypes.c_int),
+    "csa2_noalloc_scratch_bytes": ([], c_size_t),
+    "csa2_sparse_attn_noalloc": ([ctypes.c_int, c_void_p, c_int32, c_int32, c_void_p, c_float, c_void_p, c_void_p,
+                                  c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int32, _P, c_void_p, c_void_p,
+                                  c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_void_p], ctypes.c_int),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -216,6 +220,24 @@ def csa2_sparse_attn(mode, q, q_pos, cache, softmax_scale, max_entries, k=512, q
                               k, pool_k, _ptr(pool_io), _ptr(idx_in), _ptr(idx_out), max_entries, ctypes.byref(d),
                               _ptr(swa_codes), _ptr(swa_scale), R, window, _ptr(o), _ptr(lse), _ptr(ws),
                               0 if ws is None else ws.numel(), _ptr(err), _stream(stream)), "csa2_sparse_attn")
+    return o, lse
+
+
+def csa2_sparse_attn_noalloc(mode, q, q_pos, cache, softmax_scale, max_entries, k=512, q_ix=None, w=None,
+                             pool_k=0, pool_io=None, idx_in=None, idx_out=None, o=None, lse=None, err=None,
+                             stream=None, swa_codes=None, swa_scale=None, window=128):
+    """csa2_sparse_attn using the library's fixed scratch instead of a workspace (see csa2.h)."""
+    B, Q = q.shape[0], q.shape[1]
+    if o is None:
+        o = torch.empty((B, Q, HEADS, MAIN_DIM), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Q, HEADS), dtype=torch.float32, device=q.device)
+    d = cache.desc()
+    R = 0 if swa_codes is None else swa_codes.shape[1]
+    _ok(_lib.csa2_sparse_attn_noalloc(MODE[mode], _ptr(q), B, Q, _ptr(q_pos), float(softmax_scale), _ptr(q_ix),
+                                      _ptr(w), k, pool_k, _ptr(pool_io), _ptr(idx_in), _ptr(idx_out), max_entries,
+                                      ctypes.byref(d), _ptr(swa_codes), _ptr(swa_scale), R, window, _ptr(o),
+                                      _ptr(lse), _ptr(err), _stream(stream)), "csa2_sparse_attn_noalloc")
     return o, lse
 
 

@@ -52,6 +52,11 @@ size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+namespace csa2 {
+// Lets other translation units of the library set the thread's error text.
+void set_last_error(const char *msg) { g_last_error = msg; }
+}  // namespace csa2
+
 CSA2_EXPORT int csa2_version(void) { return 100; }
 
 CSA2_EXPORT const char *csa2_last_error_string(void) { return g_last_error.c_str(); }

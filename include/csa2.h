@@ -228,6 +228,34 @@ csa2_status csa2_swa_attn(const uint16_t *q, int32_t B, int32_t Q, const int32_t
 csa2_status csa2_merge(const float *o1, const float *l1, const float *o2, const float *l2,
                        int64_t rows, int32_t D, float *o, float *lse, csa2_stream_t stream);
 
+/*
+ * csa2_sparse_attn without a caller workspace.  (The pages have no counterpart:
+ * this is a convenience of this library.)  For callers that cannot allocate
+ * device memory -- e.g. an engine whose pool already holds the whole device, or
+ * a serving loop that forbids cudaMalloc/cudaFree on its hot path because they
+ * synchronise the device.  Same arguments and results as csa2_sparse_attn minus
+ * ws / ws_bytes.  Scratch comes from a fixed array inside the library of
+ * CSA2_NOALLOC_SCRATCH_BYTES (8 MiB; every GPU that loads the library holds it
+ * until the process exits); calls whose csa2_workspace_size exceeds it return
+ * CSA2_ERR_UNSUPPORTED with a message.  It allocates nothing itself.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (make that device current); do this first call before any stream
+ *     capture.
+ *   - All calls on a device share the one array and each call overwrites it
+ *     (no part of it needs to start at zero); calls that overlap on the GPU --
+ *     on different streams, or from different host threads -- race.
+ */
+#define CSA2_NOALLOC_SCRATCH_BYTES (8u << 20)
+size_t csa2_noalloc_scratch_bytes(void);
+csa2_status csa2_sparse_attn_noalloc(csa2_mode mode, const uint16_t *q, int32_t B, int32_t Q,
+                                     const int32_t *q_pos, float softmax_scale,
+                                     const uint16_t *q_ix, const uint16_t *w, int32_t k,
+                                     int32_t pool_k, int32_t *pool_io, const int32_t *idx_in,
+                                     int32_t *idx_out, int32_t max_entries,
+                                     const csa2_cache *cache, const uint8_t *swa_codes,
+                                     const float *swa_scale, int32_t R, int32_t window, float *o,
+                                     float *lse, int32_t *err, csa2_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
