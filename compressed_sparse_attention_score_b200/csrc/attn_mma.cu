@@ -20,11 +20,14 @@
 // Phase 4  O / sum and lse = max + log(sum), coalesced fp32 stores.
 // The dequantising threads fill a 4-deep ring of 16 KB operand buffers while the
 // single issuing thread drives the tensor core; every wait is time-bounded.
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace csa2 {
 using namespace sm100;
@@ -46,8 +49,8 @@ constexpr int SM_STG = SM_P + AM_MAXKEYS * 64;       // 4 x 16 KB operand ring
 constexpr int SM_SLOT = SM_STG + AM_STAGES * AM_STAGE;
 constexpr int SM_MU = SM_SLOT + AM_MAXKEYS * 8;      // logit multiplier per key
 constexpr int SM_PV = SM_MU + AM_MAXKEYS * 4;        // P multiplier per key
-constexpr int SM_RED = SM_PV + AM_MAXKEYS * 4;       // [4 warps][32 heads]
-constexpr int SM_HM = SM_RED + 4 * 32 * 4;           // head max [32], head sum [32]
+constexpr int SM_RED = SM_PV + AM_MAXKEYS * 4;       // [4 warps][32 heads]; [CS][32] weights + [32] sums
+constexpr int SM_HM = SM_RED + 8 * 32 * 4;           // head max [32], head sum [32]
 constexpr int SM_BAR = SM_HM + 2 * 32 * 4;
 constexpr int SM_MISC = SM_BAR + 8 * (AM_STAGES + 1);
 constexpr int SM_TOTAL = SM_MISC + 16;
@@ -87,10 +90,12 @@ struct Raw {
   uint32_t sc;     // sparse: the two E4M3 block scales (low 16 bits)
 };
 
-__device__ __forceinline__ void load_raw(const AttnArgs &p, const int64_t *slot, int nks, int key, int dim0, Raw &r) {
+// key: local key index of this CTA (slot[] is local); global key = key0 + key.
+__device__ __forceinline__ void load_raw(const AttnArgs &p, const int64_t *slot, int nks, int key0, int key, int dim0,
+                                         Raw &r) {
   const int64_t s = slot[key];
   if (s < 0) return;
-  if (key < nks) {
+  if (key0 + key < nks) {
     r.a = *reinterpret_cast<const uint4 *>(p.c.kv_codes + s * CSA2_MAIN_CODE_BYTES + dim0 / 2);
     r.sc = *reinterpret_cast<const uint16_t *>(p.c.kv_scales + s * CSA2_MAIN_SCALE_BYTES + dim0 / 16);
   } else {
@@ -143,6 +148,7 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32]) {
   return v[0];
 }
 
+template <int CS>
 __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -170,9 +176,16 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     nkw = pos - lo + 1;
   }
   const int nk = nks + nkw;
-  const int ntiles = (nk + AM_TILE - 1) / AM_TILE;
+  // this CTA's share of the key tiles (a cluster of CS CTAs splits the row's keys)
+  const int split = CS > 1 ? int(cg::this_cluster().block_rank()) : 0;
+  const int tiles_all = (nk + AM_TILE - 1) / AM_TILE;
+  const int tps = (tiles_all + CS - 1) / CS;
+  const int tile0 = min(tiles_all, split * tps);
+  const int ntiles = min(tiles_all, tile0 + tps) - tile0;
+  const int key0 = tile0 * AM_TILE;  // first key of this CTA; local key j is key key0 + j
   const int nvis = p.idx ? visible_entries(p.c, b, pos) : 0;
-  for (int j = tid; j < ntiles * AM_TILE; j += AM_THREADS) {
+  for (int jl = tid; jl < ntiles * AM_TILE; jl += AM_THREADS) {
+    const int j = key0 + jl;
     int64_t s = -1;
     float m = 0.f, pm = 0.f;
     if (j < nks) {
@@ -191,9 +204,9 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       const float sc = p.scale[s];
       m = p.tau * sc, pm = sc;
     }
-    slot[j] = s;
-    mu[j] = m;
-    pv[j] = pm;
+    slot[jl] = s;
+    mu[jl] = m;
+    pv[jl] = pm;
   }
   // ---------------------------------------------------------------- Q (bf16 -> fp16, K-major 128B swizzle)
   {
@@ -240,7 +253,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
 #pragma unroll
     for (int u = 0; u < AM_PF; ++u) {
       ring[u] = Raw{};
-      if (u < nch) load_raw(p, slot, nks, (u >> 3) * AM_TILE + key_in, 64 * (u & 7) + 32 * half, ring[u]);
+      if (u < nch) load_raw(p, slot, nks, key0, (u >> 3) * AM_TILE + key_in, 64 * (u & 7) + 32 * half, ring[u]);
     }
     for (int i0 = 0; i0 < nch && !aborted; i0 += AM_PF) {
 #pragma unroll
@@ -254,10 +267,10 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
           ok = mbar_wait_bounded(&mma_done[buf], ((chunk_no / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS);
         const int key = t * AM_TILE + key_in;
         uint4 out[4];
-        dequant32(ring[u], key < nks, slot[key] >= 0, out);
+        dequant32(ring[u], key0 + key < nks, slot[key] >= 0, out);
         const int inext = i + AM_PF;
         ring[u] = Raw{};
-        if (inext < nch) load_raw(p, slot, nks, (inext >> 3) * AM_TILE + key_in, 64 * (inext & 7) + 32 * half, ring[u]);
+        if (inext < nch) load_raw(p, slot, nks, key0, (inext >> 3) * AM_TILE + key_in, 64 * (inext & 7) + 32 * half, ring[u]);
         uint8_t *dst = smem + SM_STG + buf * AM_STAGE;
 #pragma unroll
         for (int v = 0; v < 4; ++v) *reinterpret_cast<uint4 *>(dst + kmaj128(key_in, 4 * half + v)) = out[v];
@@ -365,7 +378,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
 #pragma unroll
     for (int u = 0; u < AM_PF; ++u) {
       ring[u] = Raw{};
-      if (u < nch) load_raw(p, slot, nks, (u >> 2) * 64 + key_in, 128 * (u & 3) + 32 * qd, ring[u]);
+      if (u < nch) load_raw(p, slot, nks, key0, (u >> 2) * 64 + key_in, 128 * (u & 3) + 32 * qd, ring[u]);
     }
     for (int i0 = 0; i0 < nch && !aborted; i0 += AM_PF) {
 #pragma unroll
@@ -379,10 +392,10 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
           ok = mbar_wait_bounded(&mma_done[buf], ((chunk_no / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS);
         const int key = jc * 64 + key_in;
         uint4 out[4];
-        dequant32(ring[u], key < nks, slot[key] >= 0, out);
+        dequant32(ring[u], key0 + key < nks, slot[key] >= 0, out);
         const int inext = i + AM_PF;
         ring[u] = Raw{};
-        if (inext < nch) load_raw(p, slot, nks, (inext >> 2) * 64 + key_in, 128 * (inext & 3) + 32 * qd, ring[u]);
+        if (inext < nch) load_raw(p, slot, nks, key0, (inext >> 2) * 64 + key_in, 128 * (inext & 3) + 32 * qd, ring[u]);
         uint8_t *dst = smem + SM_STG + buf * AM_STAGE;
 #pragma unroll
         for (int v = 0; v < 4; ++v)
@@ -414,36 +427,101 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   tc_fence_after();
 
   // ---------------------------------------------------------------- phase 4: normalise and store
-  if (warp < 4) {
-    float inv[32];
+  if constexpr (CS == 1) {
+    if (warp < 4) {
+      float inv[32];
 #pragma unroll
-    for (int h = 0; h < 32; ++h) {
-      const float s = aborted ? 0.f : hsum[h];
-      inv[h] = s > 0.f ? 1.f / s : 0.f;
+      for (int h = 0; h < 32; ++h) {
+        const float s = aborted ? 0.f : hsum[h];
+        inv[h] = s > 0.f ? 1.f / s : 0.f;
+      }
+      float *orow = p.o + (int64_t(row) * H + hg * AM_HG) * D;
+      for (int d = 0; d < 4; ++d) {
+        uint32_t r0[16], r1[16];
+        if (!aborted && nkc > 0) {
+          const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + d * AM_HG;
+          tc_ld_32x32b_x16(ta, r0);
+          tc_ld_32x32b_x16(ta + 16, r1);
+          tc_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r0[i] = r1[i] = 0u;
+        }
+        const int dim = 128 * d + 32 * warp + lane;
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+          orow[h * D + dim] = __uint_as_float(r0[h]) * inv[h];
+          orow[(16 + h) * D + dim] = __uint_as_float(r1[h]) * inv[16 + h];
+        }
+      }
+      if (warp == 0) {
+        const float s = aborted ? 0.f : hsum[lane];
+        p.lse[int64_t(row) * H + hg * AM_HG + lane] = s > 0.f ? hmax[lane] + logf(s) : -INFINITY;
+      }
     }
+  } else {
+    // Partial of this CTA's keys: O_s (relative to its own max m_s) staged in shared
+    // memory as [32 heads][512 dims] fp32 (reusing the P^T / operand space), plus m_s
+    // and l_s.  Then each CTA of the cluster combines one slice of dims over all peers:
+    // o = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s, M = max_s m_s.
+    float *stage = reinterpret_cast<float *>(smem + SM_P);
+    if (warp < 4) {
+      if (aborted) {
+        hsum[lane] = 0.f;
+        hmax[lane] = -INFINITY;
+      }
+      for (int d = 0; d < 4; ++d) {
+        uint32_t r0[16], r1[16];
+        if (!aborted && nkc > 0) {
+          const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + d * AM_HG;
+          tc_ld_32x32b_x16(ta, r0);
+          tc_ld_32x32b_x16(ta + 16, r1);
+          tc_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r0[i] = r1[i] = 0u;
+        }
+        const int dim = 128 * d + 32 * warp + lane;
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+          stage[h * D + dim] = __uint_as_float(r0[h]);
+          stage[(16 + h) * D + dim] = __uint_as_float(r1[h]);
+        }
+      }
+    }
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    float *wts = red;          // [CS][32] combination weights (red is free now)
+    float *lsum = red + CS * 32;
+    if (tid < 32) {
+      float M = -INFINITY;
+      for (int q = 0; q < CS; ++q) M = fmaxf(M, cluster.map_shared_rank(hmax, q)[tid]);
+      float L = 0.f;
+      for (int q = 0; q < CS; ++q) {
+        const float mq = cluster.map_shared_rank(hmax, q)[tid];
+        const float wq = (M == -INFINITY || mq == -INFINITY) ? 0.f : __expf(mq - M);
+        wts[q * 32 + tid] = wq;
+        L += wq * cluster.map_shared_rank(hsum, q)[tid];
+      }
+      lsum[tid] = L;
+      if (split == 0) p.lse[int64_t(row) * H + hg * AM_HG + tid] = L > 0.f ? M + logf(L) : -INFINITY;
+    }
+    __syncthreads();
+    const int per = (D + CS - 1) / CS;
+    const int d0 = min(D, split * per), nd = min(D, d0 + per) - d0;
     float *orow = p.o + (int64_t(row) * H + hg * AM_HG) * D;
-    for (int d = 0; d < 4; ++d) {
-      uint32_t r0[16], r1[16];
-      if (!aborted && nkc > 0) {
-        const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + d * AM_HG;
-        tc_ld_32x32b_x16(ta, r0);
-        tc_ld_32x32b_x16(ta + 16, r1);
-        tc_wait_ld();
-      } else {
+    for (int it = tid; it < 32 * nd; it += AM_THREADS) {
+      const int h = it / nd, dim = d0 + it % nd;
+      float acc = 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) r0[i] = r1[i] = 0u;
+      for (int q = 0; q < CS; ++q) {
+        const float wq = wts[q * 32 + h];
+        if (wq != 0.f) acc += wq * cluster.map_shared_rank(stage, q)[h * D + dim];
       }
-      const int dim = 128 * d + 32 * warp + lane;
-#pragma unroll
-      for (int h = 0; h < 16; ++h) {
-        orow[h * D + dim] = __uint_as_float(r0[h]) * inv[h];
-        orow[(16 + h) * D + dim] = __uint_as_float(r1[h]) * inv[16 + h];
-      }
+      const float L = lsum[h];
+      orow[h * D + dim] = L > 0.f ? acc / L : 0.f;
     }
-    if (warp == 0) {
-      const float s = aborted ? 0.f : hsum[lane];
-      p.lse[int64_t(row) * H + hg * AM_HG + lane] = s > 0.f ? hmax[lane] + logf(s) : -INFINITY;
-    }
+    cluster.sync();  // every peer has finished reading this CTA's stage
   }
 
   tc_fence_before();
@@ -455,18 +533,56 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   if (tid == 0 && aborted) report(p.err, CSA2_ERR_TIMEOUT);
 }
 
+template <int CS>
+static void launch_cs(const AttnArgs &a, int rows, cudaStream_t st) {
+  static bool attr[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr[dev]) {
+    cudaFuncSetAttribute(attn_mma_kernel<CS>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(AM_SMEM));
+    attr[dev] = true;
+  }
+  if constexpr (CS == 1) {
+    attn_mma_kernel<1><<<dim3(rows, H / AM_HG, 1), AM_THREADS, AM_SMEM, st>>>(a);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(rows, H / AM_HG, CS);
+    cfg.blockDim = dim3(AM_THREADS);
+    cfg.dynamicSmemBytes = AM_SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = CS;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, attn_mma_kernel<CS>, a);
+  }
+}
+
+// Few query rows leave most SMs idle: then a cluster of CTAs (one per 128-key tile)
+// splits each row's keys and combines the partials through distributed shared memory.
 void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
                      const csa2_cache *c, const uint8_t *codes, const float *scale, int R, int window, float *o,
                      float *lse, int32_t *err, cudaStream_t st) {
-  if (B * Q == 0) return;
+  const int rows = B * Q;
+  if (rows == 0) return;
   AttnArgs a{};
   a.q = q, a.Q = Q, a.q_pos = q_pos, a.tau = tau;
   a.idx = idx, a.k = idx ? k : 0;
   if (c) a.c = *c;
   a.codes = codes, a.scale = scale, a.R = R, a.window = window;
   a.o = o, a.lse = lse, a.err = err;
-  set_smem_limit(attn_mma_kernel, AM_SMEM);
-  attn_mma_kernel<<<dim3(B * Q, H / AM_HG), AM_THREADS, AM_SMEM, st>>>(a);
+  const int tiles = (a.k + (codes ? window : 0) + AM_TILE - 1) / AM_TILE;
+  const int cs = rows * (H / AM_HG) <= 64 ? max(1, min(tiles, 5)) : 1;
+  switch (cs) {
+    case 2: launch_cs<2>(a, rows, st); break;
+    case 3: launch_cs<3>(a, rows, st); break;
+    case 4: launch_cs<4>(a, rows, st); break;
+    case 5: launch_cs<5>(a, rows, st); break;
+    default: launch_cs<1>(a, rows, st); break;
+  }
 }
 
 }  // namespace csa2
