@@ -3,7 +3,11 @@
 //
 // The CS CTAs of a cluster split the row into contiguous chunks, each CTA into 32
 // contiguous warp ranges read with coalesced loads (index order = (CTA, warp,
-// iteration, lane)), so ballots give ordered ranks inside a warp.  Three radix
+// iteration, lane)), so ballots give ordered ranks inside a warp.  A sample of the
+// keys bounds the larger selection from below; one full pass then histograms the
+// keys above the bound and appends them, in order, to per-warp candidate lists in
+// shared memory, and every later pass walks only those lists (falling back to the
+// scores themselves if the bound was too high or a list overflowed).  Three radix
 // passes (key bits 31..20, 19..8, 7..0) build per-CTA histograms in shared memory
 // that are summed across the cluster through distributed shared memory: each CTA
 // reduces one slice of bins over all peers, then gathers the full sums.  Up to two
@@ -24,6 +28,7 @@ namespace csa2 {
 namespace {
 constexpr int TK_THREADS = 1024;
 constexpr int TK_BINS = 4096;
+constexpr int TK_CAPW = 256;  // candidate-list capacity per warp
 
 struct Sel {
   int k;
@@ -97,11 +102,15 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   extern __shared__ uint32_t tk_smem[];
   uint32_t(*hist)[TK_BINS] = reinterpret_cast<uint32_t(*)[TK_BINS]>(tk_smem);                         // [2][bins]
   uint32_t(*red)[TK_BINS / CS] = reinterpret_cast<uint32_t(*)[TK_BINS / CS]>(tk_smem + 2 * TK_BINS);  // [2][slice]
+  uint32_t(*ckey)[TK_CAPW] =
+      reinterpret_cast<uint32_t(*)[TK_CAPW]>(tk_smem + 2 * TK_BINS + (CS > 1 ? 2 * TK_BINS / CS : 0));  // [32][cap]
+  int32_t(*cidx)[TK_CAPW] = reinterpret_cast<int32_t(*)[TK_CAPW]>(&ckey[32][0]);                        // [32][cap]
   __shared__ int scan_sm[32];
   __shared__ uint32_t prefix_s[2], rem_s[2];
   __shared__ int all_s[2], bin_s[2];
   __shared__ uint32_t above_s[2], total_s[2];
   __shared__ int cta_tot[2][2];  // per selection: count above T, count equal to T
+  __shared__ int overflow_s;
 
   const int r = int(cluster.block_rank());
   const int row = blockIdx.x / CS;
@@ -121,8 +130,11 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
     for (int i = tid; i < 2 * TK_BINS; i += TK_THREADS) (&hist[0][0])[i] = 0;
     __syncthreads();
   };
-  // warp-aggregated histogram of the 12 top key bits for keys whose bin >= lo_bin
-  auto top_hist = [&](int step, int lo_bin) {
+  // One pass over the warp's range: warp-aggregated histogram of the top 12 key bits
+  // for keys whose bin >= lo_bin; with `keep`, those keys are also appended, in index
+  // order, to the warp's candidate list (cnt counts them even past the capacity).
+  int cnt = 0;
+  auto top_pass = [&](int step, int lo_bin, bool keep) {
     for (int base = wb; base < we; base += 32 * U * step) {
       float v[U];
 #pragma unroll
@@ -135,37 +147,82 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
         const uint32_t key = score_key(v[u]);
         const int bin = int(key >> 20);
         const bool take = key != KEY_NEG_INF && bin >= lo_bin;
-        const uint32_t peers = __match_any_sync(0xffffffffu, take ? uint32_t(bin) : 0xFFFFFFFFu);
-        if (take && (peers & lt_mask) == 0) atomicAdd(&hist[0][bin], uint32_t(__popc(peers)));
+        const uint32_t m = __ballot_sync(0xffffffffu, take);
+        if (m) {
+          const uint32_t peers = __match_any_sync(0xffffffffu, take ? uint32_t(bin) : 0xFFFFFFFFu);
+          if (take && (peers & lt_mask) == 0) atomicAdd(&hist[0][bin], uint32_t(__popc(peers)));
+          if (keep) {
+            const int at = cnt + __popc(m & lt_mask);
+            if (take && at < TK_CAPW) {
+              ckey[warp][at] = key;
+              cidx[warp][at] = base + 32 * u * step + lane;
+            }
+            cnt += __popc(m);
+          }
+        }
+      }
+    }
+  };
+  // Visit the warp's keys in index order, 32 per step (lane = position in the step):
+  // from its candidate list (fast) or from the scores themselves.  f(key, index, valid).
+  auto walk = [&](bool fast, auto &&f) {
+    if (fast) {
+      const int m = min(cnt, TK_CAPW);
+      for (int b0 = 0; b0 < m; b0 += 32) {
+        const int i = b0 + lane;
+        const bool v = i < m;
+        f(v ? ckey[warp][i] : KEY_NEG_INF, v ? cidx[warp][i] : 0, v);
+      }
+    } else {
+      for (int base = wb; base < we; base += 32 * U) {
+        float vv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int j = base + 32 * u + lane;
+          vv[u] = j < we ? srow[j] : -INFINITY;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const uint32_t key = score_key(vv[u]);
+          f(key, base + 32 * u + lane, key != KEY_NEG_INF);
+        }
       }
     }
   };
 
   // ---- sampled lower bound: keys below it cannot reach the larger selection (checked below)
+  const uint32_t target = uint32_t(kbig / SAMPLE) + uint32_t(kbig / (2 * SAMPLE)) + 32;
   zero_hist();
-  top_hist(SAMPLE, 0);
+  top_pass(SAMPLE, 0, false);
   cluster_hist_sum<CS>(cluster, hist, red, 1, TK_BINS, r);
-  {
-    const uint32_t target = uint32_t(kbig / SAMPLE) + uint32_t(kbig / (2 * SAMPLE)) + 32;
-    if (tid == 0) bin_s[0] = 0;
-    find_bin_block(hist[0], TK_BINS, target, scan_sm, &bin_s[0], &above_s[0], &total_s[0]);
-  }
-  int lo_bin = total_s[0] >= uint32_t(kbig / SAMPLE) + uint32_t(kbig / (2 * SAMPLE)) + 32 ? bin_s[0] : 0;
+  if (tid == 0) bin_s[0] = 0;
+  find_bin_block(hist[0], TK_BINS, target, scan_sm, &bin_s[0], &above_s[0], &total_s[0]);
+  int lo_bin = total_s[0] >= target ? bin_s[0] : 0;
 
   if (tid < 2) {
     prefix_s[tid] = 0;
     rem_s[tid] = uint32_t(sel[tid].k);
     all_s[tid] = 0;
   }
-  // ---- pass 0 (top 12 bits) over keys at or above the bound; redo without it if too few
-  for (int attempt = 0; attempt < 2; ++attempt) {
-    zero_hist();
-    top_hist(1, lo_bin);
-    cluster_hist_sum<CS>(cluster, hist, red, 1, TK_BINS, r);
-    find_bin_block(hist[0], TK_BINS, 1u, scan_sm, &bin_s[1], &above_s[1], &total_s[1]);  // only for the total
-    if (total_s[1] >= uint32_t(kbig) || lo_bin == 0) break;
+  // ---- pass 0 (top 12 bits) over keys at or above the bound, keeping them as candidates
+  zero_hist();
+  if (tid == 0) overflow_s = 0;
+  __syncthreads();
+  top_pass(1, lo_bin, true);
+  if (lane == 0 && cnt > TK_CAPW) atomicOr(&overflow_s, 1);
+  cluster_hist_sum<CS>(cluster, hist, red, 1, TK_BINS, r);
+  find_bin_block(hist[0], TK_BINS, 1u, scan_sm, &bin_s[1], &above_s[1], &total_s[1]);  // for the total
+  int any_overflow = 0;
+  for (int q = 0; q < CS; ++q) any_overflow |= *cluster.map_shared_rank(&overflow_s, q);
+  bool fast = !any_overflow && (total_s[1] >= uint32_t(kbig) || lo_bin == 0);
+  if (!fast) {  // the bound was too high or a list overflowed: count every key from the scores
     lo_bin = 0;
+    zero_hist();
+    top_pass(1, 0, false);
+    cluster_hist_sum<CS>(cluster, hist, red, 1, TK_BINS, r);
+    find_bin_block(hist[0], TK_BINS, 1u, scan_sm, &bin_s[1], &above_s[1], &total_s[1]);
   }
+  cluster.sync();  // peers have read overflow_s
   const uint32_t counted = total_s[1];
   if (nsel > 1) {
     for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[1][i] = hist[0][i];
@@ -195,22 +252,12 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
     const uint32_t pre0 = prefix_s[0], pre1 = prefix_s[1];
     const bool act0 = !all_s[0], act1 = nsel > 1 && !all_s[1];
     if (act0 || act1) {
-      for (int base = wb; base < we; base += 32 * U) {
-        float v[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int j = base + 32 * u + lane;
-          v[u] = j < we ? srow[j] : -INFINITY;
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const uint32_t key = score_key(v[u]);
-          if (key == KEY_NEG_INF) continue;
-          const uint32_t hi = key >> (sh + width), bin = (key >> sh) & mask;
-          if (act0 && hi == pre0) atomicAdd(&hist[0][bin], 1u);
-          if (act1 && hi == pre1) atomicAdd(&hist[1][bin], 1u);
-        }
-      }
+      walk(fast, [&](uint32_t key, int, bool valid) {
+        if (!valid) return;
+        const uint32_t hi = key >> (sh + width), bin = (key >> sh) & mask;
+        if (act0 && hi == pre0) atomicAdd(&hist[0][bin], 1u);
+        if (act1 && hi == pre1) atomicAdd(&hist[1][bin], 1u);
+      });
     }
     cluster_hist_sum<CS>(cluster, hist, red, nsel, nb, r);
     for (int s = 0; s < nsel; ++s) {
@@ -232,25 +279,14 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
     T[s] = all_s[s] ? KEY_NEG_INF : prefix_s[s];
     need[s] = all_s[s] ? 0 : int(rem_s[s]);
   }
-  for (int base = wb; base < we; base += 32 * U) {
-    float v[U];
+  walk(fast, [&](uint32_t key, int, bool valid) {
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int j = base + 32 * u + lane;
-      v[u] = j < we ? srow[j] : -INFINITY;
+    for (int s = 0; s < 2; ++s) {
+      if (s >= nsel) break;
+      gt_w[s] += __popc(__ballot_sync(0xffffffffu, valid && key > T[s]));
+      eq_w[s] += __popc(__ballot_sync(0xffffffffu, valid && key == T[s]));
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const uint32_t key = score_key(v[u]);
-      const bool valid = key != KEY_NEG_INF;
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        if (s >= nsel) break;
-        gt_w[s] += __popc(__ballot_sync(0xffffffffu, valid && key > T[s]));
-        eq_w[s] += __popc(__ballot_sync(0xffffffffu, valid && key == T[s]));
-      }
-    }
-  }
+  });
   // ---- exclusive prefix over (cluster rank, warp)
   int gt_off[2] = {0, 0}, eq_off[2] = {0, 0};
   for (int s = 0; s < nsel; ++s) {
@@ -285,30 +321,18 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
     float *vrow = sel[s].val ? sel[s].val + int64_t(row) * k : nullptr;
     const int32_t *mrow = map ? map + int64_t(row) * N : nullptr;
     int g = gt_off[s], e = eq_off[s];
-    for (int base = wb; base < we && g + min(e, nd) < k; base += 32 * U) {
-      float v[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = base + 32 * u + lane;
-        v[u] = j < we ? srow[j] : -INFINITY;
+    walk(fast, [&](uint32_t key, int j, bool valid) {
+      const bool is_gt = valid && key > Ts, is_eq = valid && key == Ts;
+      const uint32_t gm = __ballot_sync(0xffffffffu, is_gt), em = __ballot_sync(0xffffffffu, is_eq);
+      const int gbef = g + __popc(gm & lt_mask), ebef = e + __popc(em & lt_mask);
+      const int at = is_gt ? gbef + min(ebef, nd) : ((is_eq && ebef < nd) ? gbef + ebef : -1);
+      if (at >= 0 && at < k) {
+        orow[at] = mrow ? mrow[j] : j;
+        if (vrow) vrow[at] = key_score(key);
       }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const uint32_t key = score_key(v[u]);
-        const bool valid = key != KEY_NEG_INF;
-        const bool is_gt = valid && key > Ts, is_eq = valid && key == Ts;
-        const uint32_t gm = __ballot_sync(0xffffffffu, is_gt), em = __ballot_sync(0xffffffffu, is_eq);
-        const int gbef = g + __popc(gm & lt_mask), ebef = e + __popc(em & lt_mask);
-        const int at = is_gt ? gbef + min(ebef, nd) : ((is_eq && ebef < nd) ? gbef + ebef : -1);
-        if (at >= 0 && at < k) {
-          const int j = base + 32 * u + lane;
-          orow[at] = mrow ? mrow[j] : j;
-          if (vrow) vrow[at] = v[u];
-        }
-        g += __popc(gm);
-        e += __popc(em);
-      }
-    }
+      g += __popc(gm);
+      e += __popc(em);
+    });
     if (r == 0)
       for (int i = selected[s] + tid; i < k; i += TK_THREADS) {
         orow[i] = -1;
@@ -317,7 +341,9 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   }
 }
 
-static size_t tk_smem_bytes(int cs) { return sizeof(uint32_t) * (2 * TK_BINS + (cs > 1 ? 2 * TK_BINS / cs : 0)); }
+static size_t tk_smem_bytes(int cs) {
+  return sizeof(uint32_t) * (2 * TK_BINS + (cs > 1 ? 2 * TK_BINS / cs : 0) + 2 * 32 * TK_CAPW);
+}
 
 template <int CS>
 static cudaError_t launch_cs(const float *scores, const int32_t *n_valid, int R, int N, Sel s0, Sel s1, int nsel,
