@@ -371,7 +371,8 @@ static cudaError_t launch_cs(const float *scores, const int32_t *n_valid, int R,
   return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<CS>, scores, n_valid, N, s0, s1, nsel, map);
 }
 
-// Largest usable cluster for a row length: about 64K scores per CTA, at most 16.
+// Cluster size by row length and count: one CTA per row up to 64K scores or from 148 rows
+// on; otherwise 8 CTAs up to 256K scores and 16 above.
 void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int N, int k0, int32_t *idx0, float *val0,
                          int k1, int32_t *idx1, float *val1, const int32_t *map, cudaStream_t st) {
   if (R == 0) return;
@@ -380,7 +381,7 @@ void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int
   static int cluster16_ok[64] = {};  // 0 unknown, 1 yes, -1 no
   int dev = 0;
   cudaGetDevice(&dev);
-  if (N >= (1 << 18)) {
+  if (N >= (1 << 18) && R < 148) {
     if (dev >= 0 && dev < 64 && cluster16_ok[dev] == 0) {
       cudaFuncSetAttribute(topk_cluster_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       cudaLaunchConfig_t cfg = {};
@@ -407,13 +408,10 @@ void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int
       return;
     }
     launch_cs<8>(scores, n_valid, R, N, s0, s1, nsel, map, st);
-  } else if (N >= (1 << 16)) {
+  } else if (N > (1 << 16) && R < 148) {
     launch_cs<8>(scores, n_valid, R, N, s0, s1, nsel, map, st);
-  } else if (N >= (1 << 14)) {
-    launch_cs<4>(scores, n_valid, R, N, s0, s1, nsel, map, st);
-  } else if (N >= (1 << 12)) {
-    launch_cs<2>(scores, n_valid, R, N, s0, s1, nsel, map, st);
   } else {
+    // rows up to 64K scores, or enough rows to fill the GPU: one CTA per row, no cluster barriers
     launch_cs<1>(scores, n_valid, R, N, s0, s1, nsel, map, st);
   }
 }
