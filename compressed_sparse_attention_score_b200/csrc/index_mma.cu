@@ -35,7 +35,6 @@ using namespace sm100;
 
 namespace {
 constexpr int IM_STAGES = 8;
-constexpr int IM_LAG = 5;              // tiles between issuing a stage's copies and publishing it
 constexpr int IM_TILE = 128;           // keys per tile = MMA M
 constexpr int IM_N = 64;               // indexer heads = MMA N
 constexpr int IM_A_BYTES = IM_TILE * 64;
@@ -72,20 +71,6 @@ struct IndexMmaArgs {
   int chunk;  // tiles per CTA
 };
 
-// Physical slot of the key at score position pos of this row, or -1.
-__device__ __forceinline__ int64_t key_slot(const IndexMmaArgs &a, int row, int b, int nvis, int pos, bool report_bad) {
-  int64_t n = pos;
-  if (a.cand) {
-    if (pos >= a.P) return -1;
-    n = a.cand[int64_t(row) * a.P + pos];
-    if (report_bad && (n < -1 || n >= a.c.num_entries[b])) report(a.err, CSA2_ERR_INDEX);
-  }
-  if (n < 0 || n >= nvis) return -1;
-  const int64_t s = cache_slot(a.c, b, n);
-  if (s < 0 && report_bad) report(a.err, CSA2_ERR_INDEX);
-  return s;
-}
-
 // A-operand row of tile entry e and the inverse map.
 __device__ __forceinline__ int row_of_entry(int e) { return (e & 3) * 32 + (e >> 2); }
 __device__ __forceinline__ int entry_of_row(int m) { return (m & 31) * 4 + (m >> 5); }
@@ -118,7 +103,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     tmem_relinquish();
   } else if (warp == 1 && lane == 0) {
     for (int s = 0; s < IM_STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], a.use_tma ? 1 : 32);  // gather path: one cp.async arrival per producer lane
       mbar_init(&empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -129,44 +114,50 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     *abort_flag = 0;
     mbar_init_fence();
   } else if (warp >= 2) {
-    // quantise the query heads: thread h < 64 owns head h (4 blocks of 32 values)
-    const int t = threadIdx.x - 64;
-    uint32_t sfword = 0;
-    if (t < IM_N) {
-      const uint16_t *qh = a.q_ix + (int64_t(row) * HI + t) * DI;
-      uint8_t *brow = smem + SM_B + t * 64;
+    // quantise the query heads: threads 2h, 2h+1 own blocks {0,1}, {2,3} of head h.
+    // Dividing by the power-of-two scale 2^e is done as the (exactly equal) product
+    // with 2^-e.
+    const int t = threadIdx.x - 64, h = t >> 1, g0 = 2 * (t & 1);
+    const uint16_t *qh = a.q_ix + (int64_t(row) * HI + h) * DI;
+    uint8_t *brow = smem + SM_B + h * 64;
+    uint32_t sfpart = 0;
 #pragma unroll 1
-      for (int g = 0; g < 4; ++g) {
-        float v[32];
+    for (int g = g0; g < g0 + 2; ++g) {
+      float v[32];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 u = reinterpret_cast<const uint4 *>(qh + 32 * g)[i];
-          const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
+      for (int i = 0; i < 4; ++i) {
+        const uint4 u = reinterpret_cast<const uint4 *>(qh + 32 * g)[i];
+        const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            v[8 * i + 2 * j] = __uint_as_float(ww[j] << 16);
-            v[8 * i + 2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
-          }
+        for (int j = 0; j < 4; ++j) {
+          v[8 * i + 2 * j] = __uint_as_float(ww[j] << 16);
+          v[8 * i + 2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
         }
-        float am = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
-        int ex = -127;
-        uint32_t cw[4] = {0, 0, 0, 0};
-        if (am != 0.f) {
-          ex = e8m0_ceil_exponent(__fdiv_rn(am, 6.0f));
-          const float s = pow2f(ex);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) cw[i >> 3] |= e2m1_code(__fdiv_rn(v[i], s)) << (4 * (i & 7));
-        }
-        // 16 bytes = chunk g of this 64-byte row, at its swizzled position
-        *reinterpret_cast<uint4 *>(brow + ((g ^ ((t >> 1) & 3)) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        sfword |= uint32_t(ex + 127) << (8 * g);
       }
-      ws[t] = bf16_to_f32(a.w[int64_t(row) * HI + t]);
+      float am = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+      int ex = -127;
+      uint32_t cw[4] = {0, 0, 0, 0};
+      if (am != 0.f) {
+        ex = e8m0_ceil_exponent(__fdiv_rn(am, 6.0f));
+        const float inv = pow2f(-ex);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) cw[i >> 3] |= e2m1_code(__fmul_rn(v[i], inv)) << (4 * (i & 7));
+      }
+      // 16 bytes = chunk g of this 64-byte row, at its swizzled position
+      *reinterpret_cast<uint4 *>(brow + ((g ^ ((h >> 1) & 3)) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      sfpart |= uint32_t(ex + 127) << (8 * g);
     }
-    // scale atom word of row r = t (rows 64..127 unused): lane-row r % 32, column r / 32
-    *reinterpret_cast<uint32_t *>(smem + SM_SFB + (t & 31) * 16 + (t >> 5) * 4) = sfword;
+    const uint32_t sfword = sfpart | __shfl_xor_sync(0xffffffffu, sfpart, 1);
+    // scale atom word of row r: lane-row r % 32, column r / 32 (rows 64..127 unused, zero)
+    if ((t & 1) == 0) {
+      *reinterpret_cast<uint32_t *>(smem + SM_SFB + (h & 31) * 16 + (h >> 5) * 4) = sfword;
+      ws[h] = bf16_to_f32(a.w[int64_t(row) * HI + h]);
+    } else {
+      const int rz = 64 + h;
+      *reinterpret_cast<uint32_t *>(smem + SM_SFB + (rz & 31) * 16 + (rz >> 5) * 4) = 0u;
+    }
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -195,19 +186,39 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
         }
       }
     } else {
-      // Gather path: lane l resolves the slots of tile entries l, l+32, l+64, l+96 once
-      // per tile (coalesced candidate loads, next tile prefetched), then shuffles them
-      // to the lanes that copy each 16-byte chunk.
-      auto resolve = [&](int tile, int64_t (&sl)[4]) {
+      // Gather path: lane l resolves the slots of tile entries l, l+32, l+64, l+96 (raw
+      // candidate indices are loaded two tiles ahead), the slots are shuffled to the
+      // lanes that copy each 16-byte chunk, and each lane's copies arrive on the stage's
+      // barrier by themselves (cp.async.mbarrier.arrive.noinc).
+      auto load_cand = [&](int tile, int32_t (&cv)[4]) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) sl[j] = tile < t0 + ntiles ? key_slot(a, row, b, nvis, tile * IM_TILE + lane + 32 * j, true) : -1;
+        for (int j = 0; j < 4; ++j) {
+          const int pos = tile * IM_TILE + lane + 32 * j;
+          cv[j] = (tile < t0 + ntiles && pos < a.P) ? a.cand[int64_t(row) * a.P + pos] : -1;
+        }
       };
+      auto resolve = [&](const int32_t (&cv)[4], int64_t (&sl)[4]) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int n = cv[j];
+          if (n < -1 || n >= a.c.num_entries[b]) report(a.err, CSA2_ERR_INDEX);
+          int64_t sv = -1;
+          if (n >= 0 && n < nvis) {
+            sv = cache_slot(a.c, b, n);
+            if (sv < 0) report(a.err, CSA2_ERR_INDEX);
+          }
+          sl[j] = sv;
+        }
+      };
+      int32_t c1[4], c2[4];
       int64_t cur[4], nxt[4];
-      resolve(t0, cur);
-      int i = 0;
-      for (; i < ntiles; ++i) {
+      load_cand(t0, c1);
+      resolve(c1, cur);
+      load_cand(t0 + 1, c1);
+      for (int i = 0; i < ntiles; ++i) {
         const int s = i % IM_STAGES;
-        resolve(t0 + i + 1, nxt);
+        load_cand(t0 + i + 2, c2);
+        resolve(c1, nxt);
         if (!mbar_wait_bounded(&empty[s], ((i / IM_STAGES) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
         const uint32_t st = stages + s * IM_STAGE_BYTES;
 #pragma unroll
@@ -221,21 +232,14 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
 #pragma unroll
         for (int j = 0; j < 4; ++j)  // scale word of entry e = lane + 32 j at atom word e
           if (cur[j] >= 0) cp_async_4(st + IM_A_BYTES + (lane + 32 * j) * 4, a.c.ix_scales + cur[j] * CSA2_IX_SCALE_BYTES);
-        cp_async_commit();
-        if (i >= IM_LAG) {
-          cp_async_wait<IM_LAG>();
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full[(i - IM_LAG) % IM_STAGES]);
-        }
+        cp_async_arrive_noinc(&full[s]);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
+        for (int j = 0; j < 4; ++j) {
+          cur[j] = nxt[j];
+          c1[j] = c2[j];
+        }
       }
       cp_async_wait<0>();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (i == ntiles && lane == 0)
-        for (int k = max(0, ntiles - IM_LAG); k < ntiles; ++k) mbar_arrive(&full[k % IM_STAGES]);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -252,6 +256,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
         const int s = i % IM_STAGES, acc = i & 1;
         if (!mbar_wait_bounded(&full[s], (i / IM_STAGES) & 1, abort_flag, WAIT_LIMIT_NS)) break;
         if (!mbar_wait_bounded(&acc_empty[acc], ((i >> 1) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+        fence_proxy_async_smem();  // cp.async-filled stages (gather path) are read by the tensor core
         tc_fence_after();
         const uint32_t st = stages + s * IM_STAGE_BYTES;
         const uint32_t sfa = tmem + COL_SFA + 4 * acc;
@@ -274,8 +279,17 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     const int q4 = warp & 3;              // TMEM sub-partition of this warp
     const int e = entry_of_row(32 * q4 + lane);  // tile entry of this thread's accumulator row
     const float4 *w4 = reinterpret_cast<const float4 *>(ws);
+    // the entry behind this thread's row, one tile ahead (candidate lists are read from global)
+    auto entry_at = [&](int i) -> int64_t {
+      const int pos = (t0 + i) * IM_TILE + e;
+      if (!a.cand) return pos;
+      return (i < ntiles && pos < a.P) ? a.cand[int64_t(row) * a.P + pos] : -1;
+    };
+    int64_t n_next = entry_at(0);
     for (int i = 0; i < ntiles; ++i) {
       const int acc = i & 1;
+      const int64_t n_cur = n_next;
+      n_next = entry_at(i + 1);
       if (!mbar_wait_bounded(&acc_full[acc], (i >> 1) & 1, abort_flag, WAIT_LIMIT_NS)) break;
       tc_fence_after();
       const uint32_t taddr = tmem + (uint32_t(32 * q4) << 16) + acc * IM_N;
@@ -307,7 +321,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       const float sc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
       const int pos = (t0 + i) * IM_TILE + e;
       if (pos < a.n_out) {
-        const bool ok = key_slot(a, row, b, nvis, pos, false) >= 0;
+        const bool ok = n_cur >= 0 && n_cur < nvis && cache_slot(a.c, b, n_cur) >= 0;
         a.scores[int64_t(row) * a.n_out + pos] = ok ? sc : -INFINITY;
       }
     }
