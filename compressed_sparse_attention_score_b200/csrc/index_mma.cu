@@ -34,15 +34,17 @@ namespace csa2 {
 using namespace sm100;
 
 namespace {
-constexpr int IM_STAGES = 8;
+constexpr int IM_STAGES = 16;
 constexpr int IM_TILE = 128;           // keys per tile = MMA M
 constexpr int IM_N = 64;               // indexer heads = MMA N
 constexpr int IM_A_BYTES = IM_TILE * 64;
 constexpr int IM_STAGE_BYTES = 9216;   // 8192 codes + 512 scale atom, padded to 1024
-constexpr int IM_THREADS = 192;
-constexpr uint32_t IM_TMEM_COLS = 256;
-constexpr uint32_t COL_SFA = 128;      // two 4-column scale buffers (per accumulator)
-constexpr uint32_t COL_SFB = 136;
+constexpr int IM_ACC = 4;              // TMEM accumulators (64 columns each)
+constexpr int IM_EPI_WG = 2;           // epilogue warpgroups, alternating tiles
+constexpr int IM_THREADS = 64 + 128 * IM_EPI_WG;
+constexpr uint32_t IM_TMEM_COLS = 512;
+constexpr uint32_t COL_SFA = IM_ACC * 64;   // one 4-column scale buffer per accumulator
+constexpr uint32_t COL_SFB = COL_SFA + 4 * IM_ACC;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
 constexpr int SM_STAGES = 0;
@@ -50,7 +52,7 @@ constexpr int SM_B = IM_STAGES * IM_STAGE_BYTES;       // 64 x 64 B query codes
 constexpr int SM_SFB = SM_B + IM_N * 64;                // 512 B scale atom
 constexpr int SM_W = SM_SFB + 512;                      // 64 fp32 head weights
 constexpr int SM_BAR = SM_W + 256;                      // mbarriers
-constexpr int N_BARS = 2 * IM_STAGES + 5;
+constexpr int N_BARS = 2 * IM_STAGES + 2 * IM_ACC + 1;
 constexpr int SM_MISC = SM_BAR + 8 * N_BARS;            // tmem base, abort flag
 constexpr int SM_TOTAL = SM_MISC + 16;
 constexpr size_t IM_SMEM_BYTES = SM_TOTAL + 1024;       // slack for 1024-byte alignment
@@ -75,15 +77,15 @@ struct IndexMmaArgs {
 __device__ __forceinline__ int row_of_entry(int e) { return (e & 3) * 32 + (e >> 2); }
 __device__ __forceinline__ int entry_of_row(int m) { return (m & 31) * 4 + (m >> 5); }
 
-__global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __grid_constant__ CUtensorMap tmap,
+__global__ void __launch_bounds__(IM_THREADS, 1) index_score_mma_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                         IndexMmaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM_BAR);
   uint64_t *empty = full + IM_STAGES;
   uint64_t *acc_full = empty + IM_STAGES;
-  uint64_t *acc_empty = acc_full + 2;
-  uint64_t *done = acc_empty + 2;
+  uint64_t *acc_empty = acc_full + IM_ACC;
+  uint64_t *done = acc_empty + IM_ACC;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM_MISC + 4);
   float *ws = reinterpret_cast<float *>(smem + SM_W);
@@ -106,14 +108,14 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       mbar_init(&full[s], a.use_tma ? 1 : 32);  // gather path: one cp.async arrival per producer lane
       mbar_init(&empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < IM_ACC; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
     mbar_init_fence();
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp < 6) {
     // quantise the query heads: threads 2h, 2h+1 own blocks {0,1}, {2,3} of head h.
     // Dividing by the power-of-two scale 2^e is done as the (exactly equal) product
     // with 2^-e.
@@ -190,18 +192,20 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       // candidate indices are loaded two tiles ahead), the slots are shuffled to the
       // lanes that copy each 16-byte chunk, and each lane's copies arrive on the stage's
       // barrier by themselves (cp.async.mbarrier.arrive.noinc).
-      auto load_cand = [&](int tile, int32_t (&cv)[4]) {
+      auto load_cand = [&](int tile, int32_t (&cv)[4]) {  // entry index of each position (-1: none)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int pos = tile * IM_TILE + lane + 32 * j;
-          cv[j] = (tile < t0 + ntiles && pos < a.P) ? a.cand[int64_t(row) * a.P + pos] : -1;
+          if (tile >= t0 + ntiles) cv[j] = -1;
+          else if (!a.cand) cv[j] = pos;
+          else cv[j] = pos < a.P ? a.cand[int64_t(row) * a.P + pos] : -1;
         }
       };
       auto resolve = [&](const int32_t (&cv)[4], int64_t (&sl)[4]) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int n = cv[j];
-          if (n < -1 || n >= a.c.num_entries[b]) report(a.err, CSA2_ERR_INDEX);
+          if (a.cand && (n < -1 || n >= a.c.num_entries[b])) report(a.err, CSA2_ERR_INDEX);
           int64_t sv = -1;
           if (n >= 0 && n < nvis) {
             sv = cache_slot(a.c, b, n);
@@ -253,9 +257,9 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       constexpr uint32_t id0 = idesc_mxf4(IM_TILE, IM_N, 0, 0);
       constexpr uint32_t id1 = idesc_mxf4(IM_TILE, IM_N, 2, 2);
       for (int i = 0; i < ntiles; ++i) {
-        const int s = i % IM_STAGES, acc = i & 1;
+        const int s = i % IM_STAGES, acc = i % IM_ACC;
         if (!mbar_wait_bounded(&full[s], (i / IM_STAGES) & 1, abort_flag, WAIT_LIMIT_NS)) break;
-        if (!mbar_wait_bounded(&acc_empty[acc], ((i >> 1) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+        if (!mbar_wait_bounded(&acc_empty[acc], ((i / IM_ACC) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
         fence_proxy_async_smem();  // cp.async-filled stages (gather path) are read by the tensor core
         tc_fence_after();
         const uint32_t st = stages + s * IM_STAGE_BYTES;
@@ -279,18 +283,20 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     const int q4 = warp & 3;              // TMEM sub-partition of this warp
     const int e = entry_of_row(32 * q4 + lane);  // tile entry of this thread's accumulator row
     const float4 *w4 = reinterpret_cast<const float4 *>(ws);
-    // the entry behind this thread's row, one tile ahead (candidate lists are read from global)
+    // warpgroup wg takes tiles wg, wg + IM_EPI_WG, ...; the entry behind this thread's
+    // row is fetched one of its tiles ahead (candidate lists are read from global)
+    const int wg = (warp - 2) >> 2;
     auto entry_at = [&](int i) -> int64_t {
       const int pos = (t0 + i) * IM_TILE + e;
       if (!a.cand) return pos;
       return (i < ntiles && pos < a.P) ? a.cand[int64_t(row) * a.P + pos] : -1;
     };
-    int64_t n_next = entry_at(0);
-    for (int i = 0; i < ntiles; ++i) {
-      const int acc = i & 1;
+    int64_t n_next = entry_at(wg);
+    for (int i = wg; i < ntiles; i += IM_EPI_WG) {
+      const int acc = i % IM_ACC;
       const int64_t n_cur = n_next;
-      n_next = entry_at(i + 1);
-      if (!mbar_wait_bounded(&acc_full[acc], (i >> 1) & 1, abort_flag, WAIT_LIMIT_NS)) break;
+      n_next = entry_at(i + IM_EPI_WG);
+      if (!mbar_wait_bounded(&acc_full[acc], (i / IM_ACC) & 1, abort_flag, WAIT_LIMIT_NS)) break;
       tc_fence_after();
       const uint32_t taddr = tmem + (uint32_t(32 * q4) << 16) + acc * IM_N;
       uint32_t r0[32], r1[32];
@@ -328,7 +334,8 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     // positions past the visible entries (no key tile was loaded for them)
     if (!a.cand) {
       const int lo = max(t0, t_work) * IM_TILE, hi = min(t1 * IM_TILE, a.n_out);
-      for (int pos = lo + threadIdx.x - 64; pos < hi; pos += 128) a.scores[int64_t(row) * a.n_out + pos] = -INFINITY;
+      for (int pos = lo + threadIdx.x - 64; pos < hi; pos += 128 * IM_EPI_WG)
+        a.scores[int64_t(row) * a.n_out + pos] = -INFINITY;
     }
   }
 
@@ -378,7 +385,7 @@ void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int 
   const int rows = B * Q;
   if (n_out == 0 || rows == 0) return;
   const int t_all = (n_out + IM_TILE - 1) / IM_TILE;
-  const int want = (2 * 148 + rows - 1) / rows;           // about two CTAs per SM in total
+  const int want = (148 + rows - 1) / rows;               // about one CTA per SM in total
   const int splits = max(1, min(min(want, (t_all + 7) / 8), 65535));
   const int chunk = (t_all + splits - 1) / splits;
   CUtensorMap tmap;
