@@ -34,15 +34,15 @@ namespace csa2 {
 using namespace sm100;
 
 namespace {
-constexpr int IM_STAGES = 16;
+constexpr int IM_STAGES = 8;
 constexpr int IM_TILE = 128;           // keys per tile = MMA M
 constexpr int IM_N = 64;               // indexer heads = MMA N
 constexpr int IM_A_BYTES = IM_TILE * 64;
 constexpr int IM_STAGE_BYTES = 9216;   // 8192 codes + 512 scale atom, padded to 1024
-constexpr int IM_ACC = 4;              // TMEM accumulators (64 columns each)
-constexpr int IM_EPI_WG = 2;           // epilogue warpgroups, alternating tiles
+constexpr int IM_ACC = 2;              // TMEM accumulators (64 columns each)
+constexpr int IM_EPI_WG = 1;           // epilogue warpgroups, alternating tiles
 constexpr int IM_THREADS = 64 + 128 * IM_EPI_WG;
-constexpr uint32_t IM_TMEM_COLS = 512;
+constexpr uint32_t IM_TMEM_COLS = 256;
 constexpr uint32_t COL_SFA = IM_ACC * 64;   // one 4-column scale buffer per accumulator
 constexpr uint32_t COL_SFB = COL_SFA + 4 * IM_ACC;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
@@ -77,7 +77,7 @@ struct IndexMmaArgs {
 __device__ __forceinline__ int row_of_entry(int e) { return (e & 3) * 32 + (e >> 2); }
 __device__ __forceinline__ int entry_of_row(int m) { return (m & 31) * 4 + (m >> 5); }
 
-__global__ void __launch_bounds__(IM_THREADS, 1) index_score_mma_kernel(const __grid_constant__ CUtensorMap tmap,
+__global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                         IndexMmaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -385,7 +385,7 @@ void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int 
   const int rows = B * Q;
   if (n_out == 0 || rows == 0) return;
   const int t_all = (n_out + IM_TILE - 1) / IM_TILE;
-  const int want = (148 + rows - 1) / rows;               // about one CTA per SM in total
+  const int want = (2 * 148 + rows - 1) / rows;           // about two CTAs per SM in total
   const int splits = max(1, min(min(want, (t_all + 7) / 8), 65535));
   const int chunk = (t_all + splits - 1) / splits;
   CUtensorMap tmap;
