@@ -3,19 +3,21 @@
 //
 // The CS CTAs of a cluster split the row into contiguous chunks, each CTA into 32
 // contiguous warp ranges read with coalesced loads (index order = (CTA, warp,
-// iteration, lane)), so ballots give ordered ranks inside a warp.  A sample of the
-// keys bounds the larger selection from below; one full pass then histograms the
-// keys above the bound and appends them, in order, to per-warp candidate lists in
-// shared memory, and every later pass walks only those lists (falling back to the
-// scores themselves if the bound was too high or a list overflowed).  Three radix
-// passes (key bits 31..20, 19..8, 7..0) build per-CTA histograms in shared memory
-// that are summed across the cluster through distributed shared memory: each CTA
-// reduces one slice of bins over all peers, then gathers the full sums.  Up to two
-// selections (e.g. top-512 and a 16384-entry pool) are refined in the same passes.
-// The exact k-th key T and the number of ties to take follow; a counting pass and
-// a cluster-wide exclusive prefix give every thread its output offset, and the
-// writing pass emits the chosen positions in ascending order (ties: lower position
-// first), padded with -1.
+// iteration, lane)), so ballots give ordered ranks inside a warp.  The exact k-th
+// key T is found by radix selection on the order-preserving 32-bit keys (bits 31..20,
+// 19..8, 7..0).  Every stage builds its histogram in the CTA's own shared memory,
+// together with a coarse copy (8 bins summed per entry); after one cluster barrier
+// each CTA sums the peers' coarse bins through distributed shared memory, finds the
+// coarse bin that holds the threshold and then sums only the 8 fine bins inside it,
+// so a stage costs one barrier and no CTA ever writes into a histogram a peer reads.
+// A sample of the keys first bounds the larger selection from below; the first full
+// pass counts only keys above the bound and appends them, in index order, to per-warp
+// candidate lists, and the later passes walk the lists (or the scores again if the
+// bound was too high or a list overflowed).  Up to two selections (e.g. top-512 and a
+// 16384-entry pool) are refined in the same passes.  A counting pass and a
+// cluster-wide exclusive prefix (each CTA pushes its totals into every peer) give
+// every thread its output offset, and the writing pass emits the chosen positions in
+// ascending order (ties: lower position first), padded with -1.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -27,8 +29,15 @@ namespace csa2 {
 
 namespace {
 constexpr int TK_THREADS = 1024;
-constexpr int TK_BINS = 4096;
-constexpr int TK_CAPW = 256;  // candidate-list capacity per warp
+constexpr int TK_BINS = 4096;   // 12-bit radix digit
+constexpr int TK_CBINS = 512;   // coarse copy: 8 fine bins per entry
+constexpr int TK_CAPW = 256;    // candidate-list capacity per warp
+// shared-memory words: candidate lists, then sample / pass-0 / pass-1 (x2) / pass-2 (x2)
+// histograms with their coarse copies, then the coarse cluster sums
+constexpr int TK_LIST_WORDS = 2 * 32 * TK_CAPW;
+constexpr int TK_H12_WORDS = TK_BINS + TK_CBINS;
+constexpr int TK_H8_WORDS = 256 + 32;
+constexpr int TK_SMEM_WORDS = TK_LIST_WORDS + 4 * TK_H12_WORDS + 2 * TK_H8_WORDS + TK_CBINS;
 
 struct Sel {
   int k;
@@ -64,31 +73,6 @@ __device__ void find_bin_block(const uint32_t *h, int nb, uint32_t rem, int *sca
   }
   __syncthreads();
 }
-
-// Sum the per-CTA histograms [nh][nb] across the cluster (each CTA reduces one
-// slice of bins over all peers, then gathers every slice).
-template <int CS>
-__device__ __forceinline__ void cluster_hist_sum(cg::cluster_group &cluster, uint32_t (*hist)[TK_BINS],
-                                                 uint32_t (*red)[TK_BINS / CS], int nh, int nb, int r) {
-  if constexpr (CS > 1) {
-    cluster.sync();
-    const int slice = nb / CS;
-    for (int h = 0; h < nh; ++h)
-      for (int i = threadIdx.x; i < slice; i += TK_THREADS) {
-        uint32_t t = 0;
-#pragma unroll
-        for (int p = 0; p < CS; ++p) t += cluster.map_shared_rank(&hist[h][0], p)[r * slice + i];
-        red[h][i] = t;
-      }
-    cluster.sync();
-    for (int h = 0; h < nh; ++h)
-      for (int i = threadIdx.x; i < nb; i += TK_THREADS)
-        hist[h][i] = cluster.map_shared_rank(&red[h][0], i / slice)[i % slice];
-    cluster.sync();  // peers finished reading my red[] before it is rewritten
-  } else {
-    __syncthreads();
-  }
-}
 }  // namespace
 
 template <int CS>
@@ -96,21 +80,23 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
                                                                      const int32_t *__restrict__ n_valid, int N,
                                                                      Sel s0, Sel s1, int nsel,
                                                                      const int32_t *__restrict__ map) {
-  constexpr int U = 4;        // loads in flight per lane
+  constexpr int U = 8;        // loads in flight per lane
   constexpr int SAMPLE = 16;  // one group of 32 keys in SAMPLE is sampled
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint32_t tk_smem[];
-  uint32_t(*hist)[TK_BINS] = reinterpret_cast<uint32_t(*)[TK_BINS]>(tk_smem);                         // [2][bins]
-  uint32_t(*red)[TK_BINS / CS] = reinterpret_cast<uint32_t(*)[TK_BINS / CS]>(tk_smem + 2 * TK_BINS);  // [2][slice]
-  uint32_t(*ckey)[TK_CAPW] =
-      reinterpret_cast<uint32_t(*)[TK_CAPW]>(tk_smem + 2 * TK_BINS + (CS > 1 ? 2 * TK_BINS / CS : 0));  // [32][cap]
-  int32_t(*cidx)[TK_CAPW] = reinterpret_cast<int32_t(*)[TK_CAPW]>(&ckey[32][0]);                        // [32][cap]
+  uint32_t(*ckey)[TK_CAPW] = reinterpret_cast<uint32_t(*)[TK_CAPW]>(tk_smem);        // [32][cap]
+  int32_t(*cidx)[TK_CAPW] = reinterpret_cast<int32_t(*)[TK_CAPW]>(&ckey[32][0]);     // [32][cap]
+  uint32_t *hs = tk_smem + TK_LIST_WORDS;    // sample histogram (later: pass 0 over every key)
+  uint32_t *h0 = hs + TK_H12_WORDS;          // pass 0 over keys above the sampled bound
+  uint32_t *h1 = h0 + TK_H12_WORDS;          // pass 1, one per selection
+  uint32_t *h2 = h1 + 2 * TK_H12_WORDS;      // pass 2, one per selection
+  uint32_t *sumc = h2 + 2 * TK_H8_WORDS;     // coarse bins summed over the cluster
   __shared__ int scan_sm[32];
-  __shared__ uint32_t prefix_s[2], rem_s[2];
-  __shared__ int all_s[2], bin_s[2];
-  __shared__ uint32_t above_s[2], total_s[2];
-  __shared__ int cta_tot[2][2];  // per selection: count above T, count equal to T
+  __shared__ uint32_t fine8[8];
+  __shared__ int cb_s, fbin_s;
+  __shared__ uint32_t cabove_s, ctotal_s, fabove_s;
   __shared__ int overflow_s;
+  __shared__ int tot_all[2][CS][2];  // per selection and CTA: count above T, count equal to T
 
   const int r = int(cluster.block_rank());
   const int row = blockIdx.x / CS;
@@ -126,20 +112,79 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   const Sel sel[2] = {s0, s1};
   const int kbig = nsel > 1 ? max(s0.k, s1.k) : s0.k;
 
-  auto zero_hist = [&]() {
-    for (int i = tid; i < 2 * TK_BINS; i += TK_THREADS) (&hist[0][0])[i] = 0;
+  auto csync = [&]() {
+    if constexpr (CS > 1)
+      cluster.sync();
+    else
+      __syncthreads();
+  };
+  auto peer = [&](const uint32_t *p, int q) -> const uint32_t * {
+    if constexpr (CS > 1)
+      return cluster.map_shared_rank(p, q);
+    else
+      return p;
+  };
+  // coarse[i] = fine[8i] + ... + fine[8i + 7] for this CTA's histogram (after its updates)
+  auto make_coarse = [&](uint32_t *h, int nfine) {
+    __syncthreads();
+    for (int i = tid; i < nfine / 8; i += TK_THREADS) {
+      uint32_t t = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) t += h[8 * i + j];
+      h[nfine + i] = t;
+    }
+  };
+  // After a cluster barrier: sum the coarse bins [lo, nfine/8) of a histogram over the cluster.
+  auto sum_coarse = [&](const uint32_t *h, int nfine, int lo) {
+    const int nc = nfine / 8;
+    for (int b = tid; b < nc; b += TK_THREADS) {
+      uint32_t t = 0;
+      if (b >= lo) {
+#pragma unroll
+        for (int q = 0; q < CS; ++q) t += peer(h + nfine, q)[b];
+      }
+      sumc[b] = t;
+    }
     __syncthreads();
   };
+  // From the coarse sums: the fine bin at which the cluster-wide count from the top first
+  // reaches rem (fbin_s) and the count above it (fabove_s); false if the total (ctotal_s)
+  // stays below rem.  Cluster-uniform, since every CTA sums the same counts.
+  auto select_fine = [&](const uint32_t *h, int nfine, uint32_t rem) -> bool {
+    find_bin_block(sumc, nfine / 8, rem, scan_sm, &cb_s, &cabove_s, &ctotal_s);
+    if (ctotal_s < rem) return false;
+    if (tid < 8) {
+      uint32_t t = 0;
+#pragma unroll
+      for (int q = 0; q < CS; ++q) t += peer(h, q)[8 * cb_s + tid];
+      fine8[tid] = t;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t c = cabove_s;
+      for (int i = 7; i >= 0; --i) {
+        if (c + fine8[i] >= rem) {
+          fbin_s = 8 * cb_s + i;
+          fabove_s = c;
+          break;
+        }
+        c += fine8[i];
+      }
+    }
+    __syncthreads();
+    return true;
+  };
+
   // One pass over the warp's range: warp-aggregated histogram of the top 12 key bits
   // for keys whose bin >= lo_bin; with `keep`, those keys are also appended, in index
   // order, to the warp's candidate list (cnt counts them even past the capacity).
   int cnt = 0;
-  auto top_pass = [&](int step, int lo_bin, bool keep) {
-    for (int base = wb; base < we; base += 32 * U * step) {
+  auto top_pass = [&](int lo_bin, bool keep, uint32_t *hdst) {
+    for (int base = wb; base < we; base += 32 * U) {
       float v[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const int j = base + 32 * u * step + lane;
+        const int j = base + 32 * u + lane;
         v[u] = j < we ? srow[j] : -INFINITY;
       }
 #pragma unroll
@@ -150,12 +195,12 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
         const uint32_t m = __ballot_sync(0xffffffffu, take);
         if (m) {
           const uint32_t peers = __match_any_sync(0xffffffffu, take ? uint32_t(bin) : 0xFFFFFFFFu);
-          if (take && (peers & lt_mask) == 0) atomicAdd(&hist[0][bin], uint32_t(__popc(peers)));
+          if (take && (peers & lt_mask) == 0) atomicAdd(&hdst[bin], uint32_t(__popc(peers)));
           if (keep) {
             const int at = cnt + __popc(m & lt_mask);
             if (take && at < TK_CAPW) {
               ckey[warp][at] = key;
-              cidx[warp][at] = base + 32 * u * step + lane;
+              cidx[warp][at] = base + 32 * u + lane;
             }
             cnt += __popc(m);
           }
@@ -190,84 +235,86 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
     }
   };
 
-  // ---- sampled lower bound: keys below it cannot reach the larger selection (checked below)
-  const uint32_t target = uint32_t(kbig / SAMPLE) + uint32_t(kbig / (2 * SAMPLE)) + 32;
-  zero_hist();
-  top_pass(SAMPLE, 0, false);
-  cluster_hist_sum<CS>(cluster, hist, red, 1, TK_BINS, r);
-  if (tid == 0) bin_s[0] = 0;
-  find_bin_block(hist[0], TK_BINS, target, scan_sm, &bin_s[0], &above_s[0], &total_s[0]);
-  int lo_bin = total_s[0] >= target ? bin_s[0] : 0;
-
-  if (tid < 2) {
-    prefix_s[tid] = 0;
-    rem_s[tid] = uint32_t(sel[tid].k);
-    all_s[tid] = 0;
-  }
-  // ---- pass 0 (top 12 bits) over keys at or above the bound, keeping them as candidates
-  zero_hist();
+  for (int i = tid; i < 4 * TK_H12_WORDS + 2 * TK_H8_WORDS; i += TK_THREADS) hs[i] = 0;
   if (tid == 0) overflow_s = 0;
   __syncthreads();
-  top_pass(1, lo_bin, true);
+
+  // ---- sampled lower bound on the larger selection's threshold (top 12 key bits)
+  const uint32_t target = uint32_t(kbig / SAMPLE) + uint32_t(kbig / (2 * SAMPLE)) + 32;
+  for (int base = wb; base < we; base += 32 * SAMPLE * 4) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = base + 32 * SAMPLE * u + lane;
+      v[u] = j < we ? srow[j] : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t key = score_key(v[u]);
+      const bool take = key != KEY_NEG_INF;
+      const uint32_t peers = __match_any_sync(0xffffffffu, take ? (key >> 20) : 0xFFFFFFFFu);
+      if (take && (peers & lt_mask) == 0) atomicAdd(&hs[key >> 20], uint32_t(__popc(peers)));
+    }
+  }
+  make_coarse(hs, TK_BINS);
+  csync();  // (1)
+  sum_coarse(hs, TK_BINS, 0);
+  int lo_bin = select_fine(hs, TK_BINS, target) ? fbin_s : 0;
+
+  // ---- pass 0 (bits 31..20) over keys at or above the bound, kept as candidates
+  top_pass(lo_bin, true, h0);
   if (lane == 0 && cnt > TK_CAPW) atomicOr(&overflow_s, 1);
-  cluster_hist_sum<CS>(cluster, hist, red, 1, TK_BINS, r);
-  find_bin_block(hist[0], TK_BINS, 1u, scan_sm, &bin_s[1], &above_s[1], &total_s[1]);  // for the total
+  make_coarse(h0, TK_BINS);
+  csync();  // (2)
   int any_overflow = 0;
-  for (int q = 0; q < CS; ++q) any_overflow |= *cluster.map_shared_rank(&overflow_s, q);
-  bool fast = !any_overflow && (total_s[1] >= uint32_t(kbig) || lo_bin == 0);
-  if (!fast) {  // the bound was too high or a list overflowed: count every key from the scores
-    lo_bin = 0;
-    zero_hist();
-    top_pass(1, 0, false);
-    cluster_hist_sum<CS>(cluster, hist, red, 1, TK_BINS, r);
-    find_bin_block(hist[0], TK_BINS, 1u, scan_sm, &bin_s[1], &above_s[1], &total_s[1]);
-  }
-  cluster.sync();  // peers have read overflow_s
-  const uint32_t counted = total_s[1];
-  if (nsel > 1) {
-    for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[1][i] = hist[0][i];
-  }
-  __syncthreads();
-  for (int s = 0; s < nsel; ++s) {
-    // with the bound in place fewer than all keys are counted, but then at least kbig are
-    if (lo_bin == 0 && counted <= uint32_t(sel[s].k)) {
-      if (tid == 0) all_s[s] = 1;
-      __syncthreads();
-      continue;
+#pragma unroll
+  for (int q = 0; q < CS; ++q) any_overflow |= *reinterpret_cast<const int *>(peer(reinterpret_cast<const uint32_t *>(&overflow_s), q));
+  sum_coarse(h0, TK_BINS, lo_bin >> 3);
+  uint32_t prefix[2] = {0, 0}, rem[2] = {0, 0};
+  bool all[2] = {true, true};
+  auto first_digit = [&](const uint32_t *h) {
+    for (int s = 0; s < nsel; ++s) {
+      all[s] = !select_fine(h, TK_BINS, uint32_t(sel[s].k));
+      if (!all[s]) prefix[s] = uint32_t(fbin_s), rem[s] = uint32_t(sel[s].k) - fabove_s;
     }
-    find_bin_block(hist[s], TK_BINS, rem_s[s], scan_sm, &bin_s[s], &above_s[s], &total_s[s]);
-    if (tid == 0) {
-      rem_s[s] -= above_s[s];
-      prefix_s[s] = uint32_t(bin_s[s]);
-    }
+  };
+  first_digit(h0);
+  // the bound is valid when at least kbig keys lie above it (or there was none)
+  const bool fast = !any_overflow && (lo_bin == 0 || ctotal_s >= uint32_t(kbig));
+  if (!fast) {  // count every key from the scores (peers finished reading hs before (2))
+    for (int i = tid; i < TK_H12_WORDS; i += TK_THREADS) hs[i] = 0;
     __syncthreads();
+    top_pass(0, false, hs);
+    make_coarse(hs, TK_BINS);
+    csync();
+    sum_coarse(hs, TK_BINS, 0);
+    first_digit(hs);
   }
 
-  // ---- passes 1, 2 (bits 19..8, 7..0) over keys matching each selection's prefix
+  // ---- pass 1 (bits 19..8) and pass 2 (bits 7..0) over keys matching each prefix
   for (int pass = 1; pass < 3; ++pass) {
-    const int width = pass == 2 ? 8 : 12;
-    const int sh = pass == 1 ? 8 : 0, nb = 1 << width;
-    const uint32_t mask = uint32_t(nb - 1);
-    zero_hist();
-    const uint32_t pre0 = prefix_s[0], pre1 = prefix_s[1];
-    const bool act0 = !all_s[0], act1 = nsel > 1 && !all_s[1];
+    const int width = pass == 1 ? 12 : 8, sh = pass == 1 ? 8 : 0, nfine = 1 << width;
+    const int stride = pass == 1 ? TK_H12_WORDS : TK_H8_WORDS;
+    uint32_t *hp = pass == 1 ? h1 : h2;
+    const uint32_t mask = uint32_t(nfine - 1);
+    const bool act0 = !all[0], act1 = nsel > 1 && !all[1];
     if (act0 || act1) {
       walk(fast, [&](uint32_t key, int, bool valid) {
         if (!valid) return;
         const uint32_t hi = key >> (sh + width), bin = (key >> sh) & mask;
-        if (act0 && hi == pre0) atomicAdd(&hist[0][bin], 1u);
-        if (act1 && hi == pre1) atomicAdd(&hist[1][bin], 1u);
+        if (act0 && hi == prefix[0]) atomicAdd(&hp[bin], 1u);
+        if (act1 && hi == prefix[1]) atomicAdd(&hp[stride + bin], 1u);
       });
     }
-    cluster_hist_sum<CS>(cluster, hist, red, nsel, nb, r);
+    make_coarse(hp, nfine);
+    make_coarse(hp + stride, nfine);
+    csync();  // (3), (4)
     for (int s = 0; s < nsel; ++s) {
-      if (all_s[s]) continue;
-      find_bin_block(hist[s], nb, rem_s[s], scan_sm, &bin_s[s], &above_s[s], &total_s[s]);
-      if (tid == 0) {
-        rem_s[s] -= above_s[s];
-        prefix_s[s] = (prefix_s[s] << width) | uint32_t(bin_s[s]);
-      }
-      __syncthreads();
+      if (all[s]) continue;
+      sum_coarse(hp + s * stride, nfine, 0);
+      select_fine(hp + s * stride, nfine, rem[s]);  // the prefix bin holds at least rem keys
+      prefix[s] = (prefix[s] << width) | uint32_t(fbin_s);
+      rem[s] -= fabove_s;
     }
   }
 
@@ -276,8 +323,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   int need[2], gt_w[2] = {0, 0}, eq_w[2] = {0, 0};
 #pragma unroll
   for (int s = 0; s < 2; ++s) {
-    T[s] = all_s[s] ? KEY_NEG_INF : prefix_s[s];
-    need[s] = all_s[s] ? 0 : int(rem_s[s]);
+    T[s] = all[s] ? KEY_NEG_INF : prefix[s];
+    need[s] = all[s] ? 0 : int(rem[s]);
   }
   walk(fast, [&](uint32_t key, int, bool valid) {
 #pragma unroll
@@ -287,31 +334,32 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
       eq_w[s] += __popc(__ballot_sync(0xffffffffu, valid && key == T[s]));
     }
   });
-  // ---- exclusive prefix over (cluster rank, warp)
+  // ---- exclusive prefix over (cluster rank, warp); each CTA pushes its totals to every peer
   int gt_off[2] = {0, 0}, eq_off[2] = {0, 0};
   for (int s = 0; s < nsel; ++s) {
-    int tot;
-    gt_off[s] = block_exclusive_scan_1024(lane == 0 ? gt_w[s] : 0, scan_sm, &tot);
-    gt_off[s] = __shfl_sync(0xffffffffu, gt_off[s], 0);
-    if (tid == 0) cta_tot[s][0] = tot;
-    eq_off[s] = block_exclusive_scan_1024(lane == 0 ? eq_w[s] : 0, scan_sm, &tot);
-    eq_off[s] = __shfl_sync(0xffffffffu, eq_off[s], 0);
-    if (tid == 0) cta_tot[s][1] = tot;
+    int tg, te;
+    gt_off[s] = __shfl_sync(0xffffffffu, block_exclusive_scan_1024(lane == 0 ? gt_w[s] : 0, scan_sm, &tg), 0);
+    eq_off[s] = __shfl_sync(0xffffffffu, block_exclusive_scan_1024(lane == 0 ? eq_w[s] : 0, scan_sm, &te), 0);
+    if (tid < CS) {
+      int *dst = &tot_all[s][r][0];
+      if constexpr (CS > 1) dst = cluster.map_shared_rank(dst, tid);
+      dst[0] = tg;
+      dst[1] = te;
+    }
   }
-  cluster.sync();
+  csync();  // (5): no shared memory of a peer is touched after this barrier
   int selected[2] = {0, 0};
   for (int s = 0; s < nsel; ++s) {
     int gb = 0, eb = 0, gall = 0, eall = 0;
+#pragma unroll
     for (int p = 0; p < CS; ++p) {
-      const int *pt = cluster.map_shared_rank(&cta_tot[s][0], p);
-      if (p < r) gb += pt[0], eb += pt[1];
-      gall += pt[0], eall += pt[1];
+      if (p < r) gb += tot_all[s][p][0], eb += tot_all[s][p][1];
+      gall += tot_all[s][p][0], eall += tot_all[s][p][1];
     }
     gt_off[s] += gb;
     eq_off[s] += eb;
     selected[s] = gall + min(eall, need[s]);
   }
-  cluster.sync();  // every peer has read cta_tot before any CTA exits
 
   // ---- write the chosen positions in ascending order
   for (int s = 0; s < nsel; ++s) {
@@ -341,9 +389,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   }
 }
 
-static size_t tk_smem_bytes(int cs) {
-  return sizeof(uint32_t) * (2 * TK_BINS + (cs > 1 ? 2 * TK_BINS / cs : 0) + 2 * 32 * TK_CAPW);
-}
+static size_t tk_smem_bytes(int) { return sizeof(uint32_t) * TK_SMEM_WORDS; }
 
 template <int CS>
 static cudaError_t launch_cs(const float *scores, const int32_t *n_valid, int R, int N, Sel s0, Sel s1, int nsel,
