@@ -19,7 +19,7 @@ import json
 import math
 import os
 import re
-import subprocess
+import threading
 import sys
 import time
 
@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seqs", type=int, default=1)
     ap.add_argument("--batch", type=int, default=0, help="override the sequence count (profiling runs)")
+    ap.add_argument("--eager", action="store_true", help="launch every kernel from Python instead of replaying "
+                    "CUDA graphs of the step")
     return ap.parse_args()
 
 
@@ -80,43 +82,55 @@ def barrier(world):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons, read through NVML every 2 ms on a helper thread while the
+    timed region runs (reads only: no clock or other GPU setting is changed)."""
 
-    def __init__(self, device_index):
-        self.proc = None
-        self.dev = device_index
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, dev):
+        self.sm, self.reasons, self.max_mhz, self.thread = [], set(), None, None
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200", "-i", str(device_index)],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                uuid = str(torch.cuda.get_device_properties(dev).uuid)
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(dev.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            return
+        self.nvml, self.h = pynvml, h
+        self.done = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nvml
+        masks = [(name, getattr(nv, attr, 0)) for name, attr in self.REASONS]
+        while True:
+            try:
+                self.sm.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.reasons.update(name for name, m in masks if bits & m)
+            except Exception:
+                return
+            if self.done.wait(0.002):
+                return
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        out, _ = self.proc.communicate(timeout=10)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+        self.done.set()
+        self.thread.join(timeout=5)
+        if not self.sm:
             return None
-        sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        sm = sorted(self.sm)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(sm), "source": "NVML, every 2 ms during the timed steps"}
 
 
 # ---------------------------------------------------------------- the workload on the GPU
@@ -184,27 +198,57 @@ class Hier1M:
     def launches_per_step(self):
         return 1 + self.LAYERS * 4
 
-    def step(self, scan_events=None):
-        k, s = self.k, self.spec
+    # The step in three parts: [pack the new token's entry; pack layer 0's SWA token], [the Full layer's
+    # scan], [its top-k and attention; the four Reindex layers].  The scan stays a separate part so that
+    # CUDA events can time it even when the other two parts are replayed as CUDA graphs.
+    def part_pre(self):
+        k = self.k
         k.csa2_pack_kv(self.new_kv, self.new_ix, self.first_entry, self.cache, err=self.err)
+        k.csa2_pack_swa(self.swa_new[0], self.swa_pos, self.swa_codes[0], self.swa_scale[0], err=self.err)
+
+    def part_scan(self):
+        self.k.csa2_index_score(self.q_ix[0], self.w[0], self.q_pos, self.cache, self.N, scores=self.scores,
+                                err=self.err)
+
+    def part_post(self):
+        k, s = self.k, self.spec
+        k.csa2_topk(self.scores, s.k, idx=self.idx[0], k2=s.pool_k, idx2=self.pool)
         for layer in range(self.LAYERS):
-            k.csa2_pack_swa(self.swa_new[layer], self.swa_pos, self.swa_codes[layer], self.swa_scale[layer],
-                            err=self.err)
+            if layer > 0:
+                k.csa2_pack_swa(self.swa_new[layer], self.swa_pos, self.swa_codes[layer], self.swa_scale[layer],
+                                err=self.err)
             q, q_ix, w = self.q[layer], self.q_ix[layer], self.w[layer]
             swa = dict(swa_codes=self.swa_codes[layer], swa_scale=self.swa_scale[layer])
             if layer == 0:
-                if scan_events:
-                    scan_events[0].record()
-                k.csa2_index_score(q_ix, w, self.q_pos, self.cache, self.N, scores=self.scores, err=self.err)
-                if scan_events:
-                    scan_events[1].record()
-                k.csa2_topk(self.scores, s.k, idx=self.idx[0], k2=s.pool_k, idx2=self.pool)
                 k.csa2_sparse_attn("reuse", q, self.q_pos, self.cache, s.tau, self.N, k=s.k, idx_in=self.idx[0],
                                    o=self.o[layer], lse=self.lse[layer], err=self.err, **swa)
             else:
                 k.csa2_sparse_attn("reindex", q, self.q_pos, self.cache, s.tau, self.N, k=s.k, q_ix=q_ix, w=w,
                                    pool_k=s.pool_k, pool_io=self.pool, idx_out=self.idx[layer], o=self.o[layer],
                                    lse=self.lse[layer], ws=self.ws_reindex, err=self.err, **swa)
+
+    def capture(self):
+        """Record part_pre and part_post as CUDA graphs (after at least one eager step)."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        self.graphs = (torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(self.graphs[0], stream=side):
+                self.part_pre()
+            with torch.cuda.graph(self.graphs[1], stream=side):
+                self.part_post()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+
+    def step(self, scan_events=None, graphs=False):
+        """One decode step: eagerly, or replaying the captured graphs around an eager scan."""
+        self.graphs[0].replay() if graphs else self.part_pre()
+        if scan_events:
+            scan_events[0].record()
+        self.part_scan()
+        if scan_events:
+            scan_events[1].record()
+        self.graphs[1].replay() if graphs else self.part_post()
 
     def host_io(self):
         """Pinned host copies of one step's inputs and outputs (for the end-to-end run)."""
@@ -351,21 +395,24 @@ def main():
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    for _ in range(args.warmup):
-        wl.step()
+    graphs = not args.eager
+    for i in range(args.warmup):
+        wl.step(graphs=graphs and i > 0)
+        if graphs and i == 0:
+            wl.capture()
     torch.cuda.synchronize()
     assert wl.k.csa2_check(wl.err) == 0
 
     # ---- device-resident timing
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    clocks = ClockSampler(dev.index)
+    clocks = ClockSampler(dev)
     barrier(world)
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
-        wl.step(scan_events=sev[i])
+        wl.step(scan_events=sev[i], graphs=graphs)
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -388,7 +435,7 @@ def main():
         eev[i][0].record(stream)
         for d, h in zip(ins, h_in):
             d.copy_(h, non_blocking=True)
-        wl.step()
+        wl.step(graphs=graphs)
         for h, d in zip(h_out, outs):
             h.copy_(d, non_blocking=True)
         eev[i][1].record(stream)
@@ -399,12 +446,13 @@ def main():
 
     peak, peak_kind = peaks()
     achieved = wl.scan_bytes() / (scan_ms * 1e-3) / 1e9
-    traffic = profiled_traffic(["compressed_sparse_attention_score_b200/csrc/index_score.cu"],
+    traffic = profiled_traffic(["compressed_sparse_attention_score_b200/csrc/index_mma.cu"],
                                "index_score_hier1m.md")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded N(0,1) latents and queries)",
-            "config": config_dict(spec),
+            "config": dict(config_dict(spec), launch="eager" if args.eager else
+                           "CUDA graphs of the step around an eagerly launched Full-layer scan"),
             "roofline": {"bound": "hbm", "kernel": "csa2 indexer scan (Full layer)", "achieved": achieved,
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "scan_ms": scan_ms,

@@ -37,7 +37,7 @@ constexpr int TK_CAPW = 256;    // candidate-list capacity per warp
 constexpr int TK_LIST_WORDS = 2 * 32 * TK_CAPW;
 constexpr int TK_H12_WORDS = TK_BINS + TK_CBINS;
 constexpr int TK_H8_WORDS = 256 + 32;
-constexpr int TK_SMEM_WORDS = TK_LIST_WORDS + 4 * TK_H12_WORDS + 2 * TK_H8_WORDS + TK_CBINS;
+constexpr int TK_SMEM_WORDS = TK_LIST_WORDS + 4 * TK_H12_WORDS + 2 * TK_H8_WORDS + 2 * TK_CBINS;
 
 struct Sel {
   int k;
@@ -45,34 +45,6 @@ struct Sel {
   float *val;
 };
 
-// Threshold search with the whole CTA: the bin at which the count of keys in bins
-// at or above it first reaches rem (scanning from the top), the count strictly
-// above that bin, and the total.  Thread t owns bins nb-4t-4 .. nb-4t-1.
-__device__ void find_bin_block(const uint32_t *h, int nb, uint32_t rem, int *scan_sm, int *out_bin,
-                               uint32_t *out_above, uint32_t *out_total) {
-  const int t = threadIdx.x;
-  uint32_t c[4] = {0, 0, 0, 0}, sum = 0;
-  if (4 * t < nb) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) c[i] = h[nb - 4 * t - 1 - i], sum += c[i];
-  }
-  int total;
-  const uint32_t excl = uint32_t(block_exclusive_scan_1024(int(sum), scan_sm, &total));
-  if (t == 0) *out_total = uint32_t(total);
-  if (excl < rem && excl + sum >= rem) {
-    uint32_t cum = excl;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (cum + c[i] >= rem) {
-        *out_bin = nb - 4 * t - 1 - i;
-        *out_above = cum;
-        break;
-      }
-      cum += c[i];
-    }
-  }
-  __syncthreads();
-}
 }  // namespace
 
 template <int CS>
@@ -80,7 +52,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
                                                                      const int32_t *__restrict__ n_valid, int N,
                                                                      Sel s0, Sel s1, int nsel,
                                                                      const int32_t *__restrict__ map) {
-  constexpr int U = 8;        // loads in flight per lane
+  constexpr int U = 8;        // scalar loads in flight per lane
+  constexpr int UV = 4;       // 16-byte loads in flight per lane in the first full pass
   constexpr int SAMPLE = 16;  // one group of 32 keys in SAMPLE is sampled
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint32_t tk_smem[];
@@ -90,12 +63,11 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   uint32_t *h0 = hs + TK_H12_WORDS;          // pass 0 over keys above the sampled bound
   uint32_t *h1 = h0 + TK_H12_WORDS;          // pass 1, one per selection
   uint32_t *h2 = h1 + 2 * TK_H12_WORDS;      // pass 2, one per selection
-  uint32_t *sumc = h2 + 2 * TK_H8_WORDS;     // coarse bins summed over the cluster
-  __shared__ int scan_sm[32];
-  __shared__ uint32_t fine8[8];
-  __shared__ int cb_s, fbin_s;
-  __shared__ uint32_t cabove_s, ctotal_s, fabove_s;
+  uint32_t *sumc = h2 + 2 * TK_H8_WORDS;     // [2][TK_CBINS] coarse bins summed over the cluster
+  __shared__ int sel_bin[2];
+  __shared__ uint32_t sel_above[2], sel_count[2], sel_total[2];
   __shared__ int overflow_s;
+  __shared__ int wc[32][4];          // per warp: keys above / equal to T for both selections
   __shared__ int tot_all[2][CS][2];  // per selection and CTA: count above T, count equal to T
 
   const int r = int(cluster.block_rank());
@@ -103,13 +75,13 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = n_valid ? max(0, min(N, n_valid[row])) : N;
   const float *srow = scores + int64_t(row) * N;
-  // CTA chunk, then one contiguous range per warp; lane l reads elements base + 32 u + l
-  const int chunk = (n + CS - 1) / CS;
+  const bool vec = (N & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
+  // CTA chunk, then one contiguous range per warp, both multiples of 4 elements
+  const int chunk = ((n + CS - 1) / CS + 3) & ~3;
   const int c0 = min(n, r * chunk), c1 = min(n, c0 + chunk);
-  const int wsub = (c1 - c0 + 31) / 32;
+  const int wsub = ((c1 - c0 + 31) / 32 + 3) & ~3;
   const int wb = min(c1, c0 + warp * wsub), we = min(c1, wb + wsub);
   const uint32_t lt_mask = (1u << lane) - 1u;
-  const Sel sel[2] = {s0, s1};
   const int kbig = nsel > 1 ? max(s0.k, s1.k) : s0.k;
 
   auto csync = [&]() {
@@ -134,52 +106,131 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
       h[nfine + i] = t;
     }
   };
-  // After a cluster barrier: sum the coarse bins [lo, nfine/8) of a histogram over the cluster.
-  auto sum_coarse = [&](const uint32_t *h, int nfine, int lo) {
+  // After a cluster barrier: sumc[s][b] = the cluster's sum of coarse bin b >= lo of the
+  // histogram h + s * stride, for each selection s marked active.
+  auto sum_coarse = [&](const uint32_t *h, int stride, int nfine, int lo, bool a0, bool a1) {
     const int nc = nfine / 8;
-    for (int b = tid; b < nc; b += TK_THREADS) {
+    for (int b = tid; b < 2 * nc; b += TK_THREADS) {
+      const int s = b >= nc, c = b - s * nc;
       uint32_t t = 0;
-      if (b >= lo) {
+      if ((s ? a1 : a0) && c >= lo) {
+        const uint32_t *hc = h + s * stride + nfine;
 #pragma unroll
-        for (int q = 0; q < CS; ++q) t += peer(h + nfine, q)[b];
+        for (int q = 0; q < CS; ++q) t += peer(hc, q)[c];
       }
-      sumc[b] = t;
+      sumc[s * TK_CBINS + c] = t;
     }
     __syncthreads();
   };
-  // From the coarse sums: the fine bin at which the cluster-wide count from the top first
-  // reaches rem (fbin_s) and the count above it (fabove_s); false if the total (ctotal_s)
-  // stays below rem.  Cluster-uniform, since every CTA sums the same counts.
-  auto select_fine = [&](const uint32_t *h, int nfine, uint32_t rem) -> bool {
-    find_bin_block(sumc, nfine / 8, rem, scan_sm, &cb_s, &cabove_s, &ctotal_s);
-    if (ctotal_s < rem) return false;
-    if (tid < 8) {
-      uint32_t t = 0;
+  // One warp: the fine bin at which the cluster-wide count from the top first reaches rem,
+  // from the coarse sums sc and the peers' fine bins h (nfine/8 coarse bins, 32 | nfine/8).
+  // Results in slot s: bin, count above it, its own count and the total (bin -1 when the
+  // total stays below rem).  Cluster-uniform, since every CTA sums the same counts.
+  auto warp_select = [&](const uint32_t *sc, const uint32_t *h, int nfine, uint32_t rem, int s) {
+    const int nc = nfine / 8, per = nc / 32;  // lane 0 owns the top per bins
+    uint32_t sum = 0;
+    for (int i = 0; i < per; ++i) sum += sc[nc - 1 - lane * per - i];
+    uint32_t x = sum;
 #pragma unroll
-      for (int q = 0; q < CS; ++q) t += peer(h, q)[8 * cb_s + tid];
-      fine8[tid] = t;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    __syncthreads();
-    if (tid == 0) {
-      uint32_t c = cabove_s;
-      for (int i = 7; i >= 0; --i) {
-        if (c + fine8[i] >= rem) {
-          fbin_s = 8 * cb_s + i;
-          fabove_s = c;
+    const uint32_t total = __shfl_sync(0xffffffffu, x, 31);
+    if (total < rem) {
+      if (lane == 0) sel_bin[s] = -1, sel_total[s] = total;
+      return;
+    }
+    const uint32_t excl = x - sum;
+    const int L = __ffs(__ballot_sync(0xffffffffu, excl < rem && x >= rem)) - 1;
+    int cb = 0;
+    uint32_t cab = 0;
+    if (lane == L) {
+      uint32_t cum = excl;
+      for (int i = 0; i < per; ++i) {
+        const uint32_t v = sc[nc - 1 - L * per - i];
+        if (cum + v >= rem) {
+          cb = nc - 1 - L * per - i;
+          cab = cum;
           break;
         }
-        c += fine8[i];
+        cum += v;
       }
     }
-    __syncthreads();
-    return true;
+    cb = __shfl_sync(0xffffffffu, cb, L);
+    cab = __shfl_sync(0xffffffffu, cab, L);
+    uint32_t f = 0;  // lanes 0..7: fine bins 8cb+7 .. 8cb of the cluster, from the top
+    if (lane < 8) {
+#pragma unroll
+      for (int q = 0; q < CS; ++q) f += peer(h, q)[8 * cb + 7 - lane];
+    }
+    uint32_t fx = f;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, fx, o);
+      if (lane >= o) fx += y;
+    }
+    const int F = __ffs(__ballot_sync(0xffffffffu, lane < 8 && cab + fx - f < rem && cab + fx >= rem)) - 1;
+    if (lane == F) {
+      sel_bin[s] = 8 * cb + 7 - F;
+      sel_above[s] = cab + fx - f;
+      sel_count[s] = f;
+      sel_total[s] = total;
+    }
   };
 
-  // One pass over the warp's range: warp-aggregated histogram of the top 12 key bits
-  // for keys whose bin >= lo_bin; with `keep`, those keys are also appended, in index
-  // order, to the warp's candidate list (cnt counts them even past the capacity).
+  // Full pass over the warp's range keeping keys at or above lo_bin: their top-12-bit
+  // histogram and, in index order, the warp's candidate list.  Four consecutive keys per
+  // lane; stops once the list has overflowed (the caller then counts from the scores).
   int cnt = 0;
-  auto top_pass = [&](int lo_bin, bool keep, uint32_t *hdst) {
+  auto keep_pass = [&](int lo_bin, uint32_t *hdst) {
+    for (int base = wb; base < we && cnt <= TK_CAPW; base += 128 * UV) {
+      float4 v[UV];
+#pragma unroll
+      for (int u = 0; u < UV; ++u) {
+        const int j = base + 128 * u + 4 * lane;
+        if (vec && j + 3 < we) {
+          v[u] = *reinterpret_cast<const float4 *>(srow + j);
+        } else {
+          v[u].x = j < we ? srow[j] : -INFINITY;
+          v[u].y = j + 1 < we ? srow[j + 1] : -INFINITY;
+          v[u].z = j + 2 < we ? srow[j + 2] : -INFINITY;
+          v[u].w = j + 3 < we ? srow[j + 3] : -INFINITY;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < UV; ++u) {
+        const uint32_t kk[4] = {score_key(v[u].x), score_key(v[u].y), score_key(v[u].z), score_key(v[u].w)};
+        bool t[4];
+        int c = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          t[e] = kk[e] != KEY_NEG_INF && int(kk[e] >> 20) >= lo_bin;
+          c += t[e];
+        }
+        if (__ballot_sync(0xffffffffu, c != 0)) {
+          const uint32_t b0 = __ballot_sync(0xffffffffu, c & 1), b1 = __ballot_sync(0xffffffffu, c & 2),
+                         b2 = __ballot_sync(0xffffffffu, c & 4);
+          int at = cnt + __popc(b0 & lt_mask) + 2 * __popc(b1 & lt_mask) + 4 * __popc(b2 & lt_mask);
+          const int j = base + 128 * u + 4 * lane;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (t[e]) {
+              atomicAdd(&hdst[kk[e] >> 20], 1u);
+              if (at < TK_CAPW) {
+                ckey[warp][at] = kk[e];
+                cidx[warp][at] = j + e;
+              }
+              ++at;
+            }
+          }
+          cnt += __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
+        }
+      }
+    }
+  };
+  // Count pass over every key (no lists): warp-aggregated top-12-bit histogram.
+  auto count_pass = [&](uint32_t *hdst) {
     for (int base = wb; base < we; base += 32 * U) {
       float v[U];
 #pragma unroll
@@ -190,21 +241,9 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const uint32_t key = score_key(v[u]);
-        const int bin = int(key >> 20);
-        const bool take = key != KEY_NEG_INF && bin >= lo_bin;
-        const uint32_t m = __ballot_sync(0xffffffffu, take);
-        if (m) {
-          const uint32_t peers = __match_any_sync(0xffffffffu, take ? uint32_t(bin) : 0xFFFFFFFFu);
-          if (take && (peers & lt_mask) == 0) atomicAdd(&hdst[bin], uint32_t(__popc(peers)));
-          if (keep) {
-            const int at = cnt + __popc(m & lt_mask);
-            if (take && at < TK_CAPW) {
-              ckey[warp][at] = key;
-              cidx[warp][at] = base + 32 * u + lane;
-            }
-            cnt += __popc(m);
-          }
-        }
+        const bool take = key != KEY_NEG_INF;
+        const uint32_t peers = __match_any_sync(0xffffffffu, take ? (key >> 20) : 0xFFFFFFFFu);
+        if (take && (peers & lt_mask) == 0) atomicAdd(&hdst[key >> 20], uint32_t(__popc(peers)));
       }
     }
   };
@@ -258,97 +297,126 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   }
   make_coarse(hs, TK_BINS);
   csync();  // (1)
-  sum_coarse(hs, TK_BINS, 0);
-  int lo_bin = select_fine(hs, TK_BINS, target) ? fbin_s : 0;
+  sum_coarse(hs, 0, TK_BINS, 0, true, false);
+  if (warp == 0) warp_select(sumc, hs, TK_BINS, target, 0);
+  __syncthreads();
+  const int lo_bin = sel_bin[0] >= 0 ? sel_bin[0] : 0;
 
   // ---- pass 0 (bits 31..20) over keys at or above the bound, kept as candidates
-  top_pass(lo_bin, true, h0);
+  keep_pass(lo_bin, h0);
   if (lane == 0 && cnt > TK_CAPW) atomicOr(&overflow_s, 1);
   make_coarse(h0, TK_BINS);
   csync();  // (2)
   int any_overflow = 0;
 #pragma unroll
-  for (int q = 0; q < CS; ++q) any_overflow |= *reinterpret_cast<const int *>(peer(reinterpret_cast<const uint32_t *>(&overflow_s), q));
-  sum_coarse(h0, TK_BINS, lo_bin >> 3);
+  for (int q = 0; q < CS; ++q)
+    any_overflow |= int(*peer(reinterpret_cast<const uint32_t *>(&overflow_s), q));
+  // Per selection: radix prefix of T and its width in bits (resolved once the prefix's bin
+  // holds exactly the keys still needed), keys still needed, or "take every key".
   uint32_t prefix[2] = {0, 0}, rem[2] = {0, 0};
+  int width[2] = {0, 0};
   bool all[2] = {true, true};
-  auto first_digit = [&](const uint32_t *h) {
+  auto first_digit = [&](const uint32_t *h, int lo) {
+    sum_coarse(h, 0, TK_BINS, lo, true, false);
+    if (warp < nsel) warp_select(sumc, h, TK_BINS, uint32_t(warp ? s1.k : s0.k), warp);
+    __syncthreads();
     for (int s = 0; s < nsel; ++s) {
-      all[s] = !select_fine(h, TK_BINS, uint32_t(sel[s].k));
-      if (!all[s]) prefix[s] = uint32_t(fbin_s), rem[s] = uint32_t(sel[s].k) - fabove_s;
+      all[s] = sel_bin[s] < 0;
+      if (!all[s]) {
+        prefix[s] = uint32_t(sel_bin[s]);
+        rem[s] = uint32_t(s ? s1.k : s0.k) - sel_above[s];
+        width[s] = 12;
+      }
     }
   };
-  first_digit(h0);
+  first_digit(h0, lo_bin >> 3);
   // the bound is valid when at least kbig keys lie above it (or there was none)
-  const bool fast = !any_overflow && (lo_bin == 0 || ctotal_s >= uint32_t(kbig));
+  const bool fast = !any_overflow && (lo_bin == 0 || sel_total[0] >= uint32_t(kbig));
   if (!fast) {  // count every key from the scores (peers finished reading hs before (2))
     for (int i = tid; i < TK_H12_WORDS; i += TK_THREADS) hs[i] = 0;
     __syncthreads();
-    top_pass(0, false, hs);
+    count_pass(hs);
     make_coarse(hs, TK_BINS);
     csync();
-    sum_coarse(hs, TK_BINS, 0);
-    first_digit(hs);
+    first_digit(hs, 0);
   }
 
-  // ---- pass 1 (bits 19..8) and pass 2 (bits 7..0) over keys matching each prefix
+  // ---- pass 1 (bits 19..8) and pass 2 (bits 7..0) over keys matching each prefix, for
+  // selections whose prefix bin holds more keys than are still needed
   for (int pass = 1; pass < 3; ++pass) {
-    const int width = pass == 1 ? 12 : 8, sh = pass == 1 ? 8 : 0, nfine = 1 << width;
+    const int w = pass == 1 ? 12 : 8, sh = pass == 1 ? 8 : 0, nfine = 1 << w;
     const int stride = pass == 1 ? TK_H12_WORDS : TK_H8_WORDS;
     uint32_t *hp = pass == 1 ? h1 : h2;
     const uint32_t mask = uint32_t(nfine - 1);
-    const bool act0 = !all[0], act1 = nsel > 1 && !all[1];
-    if (act0 || act1) {
-      walk(fast, [&](uint32_t key, int, bool valid) {
-        if (!valid) return;
-        const uint32_t hi = key >> (sh + width), bin = (key >> sh) & mask;
-        if (act0 && hi == prefix[0]) atomicAdd(&hp[bin], 1u);
-        if (act1 && hi == prefix[1]) atomicAdd(&hp[stride + bin], 1u);
-      });
-    }
+    const bool act0 = !all[0] && sel_count[0] != rem[0];
+    const bool act1 = nsel > 1 && !all[1] && sel_count[1] != rem[1];
+    if (!act0 && !act1) break;  // cluster-uniform
+    walk(fast, [&](uint32_t key, int, bool valid) {
+      if (!valid) return;
+      const uint32_t hi = key >> (sh + w), bin = (key >> sh) & mask;
+      if (act0 && hi == prefix[0]) atomicAdd(&hp[bin], 1u);
+      if (act1 && hi == prefix[1]) atomicAdd(&hp[stride + bin], 1u);
+    });
     make_coarse(hp, nfine);
     make_coarse(hp + stride, nfine);
     csync();  // (3), (4)
-    for (int s = 0; s < nsel; ++s) {
-      if (all[s]) continue;
-      sum_coarse(hp + s * stride, nfine, 0);
-      select_fine(hp + s * stride, nfine, rem[s]);  // the prefix bin holds at least rem keys
-      prefix[s] = (prefix[s] << width) | uint32_t(fbin_s);
-      rem[s] -= fabove_s;
-    }
+    sum_coarse(hp, stride, nfine, 0, act0, act1);
+    if ((warp == 0 && act0) || (warp == 1 && act1))
+      warp_select(sumc + warp * TK_CBINS, hp + warp * stride, nfine, rem[warp], warp);
+    __syncthreads();
+    if (act0) prefix[0] = (prefix[0] << w) | uint32_t(sel_bin[0]), rem[0] -= sel_above[0], width[0] += w;
+    if (act1) prefix[1] = (prefix[1] << w) | uint32_t(sel_bin[1]), rem[1] -= sel_above[1], width[1] += w;
   }
 
-  // ---- per-warp counts of keys above / equal to T (warp-uniform via ballots)
+  // ---- per-warp counts of keys above / equal to T (compared on the prefix's bits)
   uint32_t T[2];
-  int need[2], gt_w[2] = {0, 0}, eq_w[2] = {0, 0};
+  int tsh[2], need[2], gt_w[2] = {0, 0}, eq_w[2] = {0, 0};
 #pragma unroll
   for (int s = 0; s < 2; ++s) {
     T[s] = all[s] ? KEY_NEG_INF : prefix[s];
+    tsh[s] = all[s] ? 0 : 32 - width[s];
     need[s] = all[s] ? 0 : int(rem[s]);
   }
   walk(fast, [&](uint32_t key, int, bool valid) {
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
       if (s >= nsel) break;
-      gt_w[s] += __popc(__ballot_sync(0xffffffffu, valid && key > T[s]));
-      eq_w[s] += __popc(__ballot_sync(0xffffffffu, valid && key == T[s]));
+      const uint32_t kh = key >> tsh[s];
+      gt_w[s] += __popc(__ballot_sync(0xffffffffu, valid && kh > T[s]));
+      eq_w[s] += __popc(__ballot_sync(0xffffffffu, valid && kh == T[s]));
     }
   });
   // ---- exclusive prefix over (cluster rank, warp); each CTA pushes its totals to every peer
-  int gt_off[2] = {0, 0}, eq_off[2] = {0, 0};
-  for (int s = 0; s < nsel; ++s) {
-    int tg, te;
-    gt_off[s] = __shfl_sync(0xffffffffu, block_exclusive_scan_1024(lane == 0 ? gt_w[s] : 0, scan_sm, &tg), 0);
-    eq_off[s] = __shfl_sync(0xffffffffu, block_exclusive_scan_1024(lane == 0 ? eq_w[s] : 0, scan_sm, &te), 0);
-    if (tid < CS) {
-      int *dst = &tot_all[s][r][0];
-      if constexpr (CS > 1) dst = cluster.map_shared_rank(dst, tid);
-      dst[0] = tg;
-      dst[1] = te;
+  if (lane == 0) wc[warp][0] = gt_w[0], wc[warp][1] = eq_w[0], wc[warp][2] = gt_w[1], wc[warp][3] = eq_w[1];
+  __syncthreads();
+  if (warp == 0) {
+    int v[4], x[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = x[i] = wc[lane][i];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int y = __shfl_up_sync(0xffffffffu, x[i], o);
+        if (lane >= o) x[i] += y;
+      }
+    int tot[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      wc[lane][i] = x[i] - v[i];
+      tot[i] = __shfl_sync(0xffffffffu, x[i], 31);
+    }
+    if (lane < CS) {
+      for (int s = 0; s < nsel; ++s) {
+        int *dst = &tot_all[s][r][0];
+        if constexpr (CS > 1) dst = cluster.map_shared_rank(dst, lane);
+        dst[0] = tot[2 * s];
+        dst[1] = tot[2 * s + 1];
+      }
     }
   }
   csync();  // (5): no shared memory of a peer is touched after this barrier
-  int selected[2] = {0, 0};
+  int gt_off[2], eq_off[2], selected[2] = {0, 0};
   for (int s = 0; s < nsel; ++s) {
     int gb = 0, eb = 0, gall = 0, eall = 0;
 #pragma unroll
@@ -356,21 +424,23 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
       if (p < r) gb += tot_all[s][p][0], eb += tot_all[s][p][1];
       gall += tot_all[s][p][0], eall += tot_all[s][p][1];
     }
-    gt_off[s] += gb;
-    eq_off[s] += eb;
+    gt_off[s] = wc[warp][2 * s] + gb;
+    eq_off[s] = wc[warp][2 * s + 1] + eb;
     selected[s] = gall + min(eall, need[s]);
   }
 
   // ---- write the chosen positions in ascending order
   for (int s = 0; s < nsel; ++s) {
-    const int k = sel[s].k, nd = need[s];
+    const Sel sl = s ? s1 : s0;
+    const int k = sl.k, nd = need[s], ts = tsh[s];
     const uint32_t Ts = T[s];
-    int32_t *orow = sel[s].idx + int64_t(row) * k;
-    float *vrow = sel[s].val ? sel[s].val + int64_t(row) * k : nullptr;
+    int32_t *orow = sl.idx + int64_t(row) * k;
+    float *vrow = sl.val ? sl.val + int64_t(row) * k : nullptr;
     const int32_t *mrow = map ? map + int64_t(row) * N : nullptr;
     int g = gt_off[s], e = eq_off[s];
     walk(fast, [&](uint32_t key, int j, bool valid) {
-      const bool is_gt = valid && key > Ts, is_eq = valid && key == Ts;
+      const uint32_t kh = key >> ts;
+      const bool is_gt = valid && kh > Ts, is_eq = valid && kh == Ts;
       const uint32_t gm = __ballot_sync(0xffffffffu, is_gt), em = __ballot_sync(0xffffffffu, is_eq);
       const int gbef = g + __popc(gm & lt_mask), ebef = e + __popc(em & lt_mask);
       const int at = is_gt ? gbef + min(ebef, nd) : ((is_eq && ebef < nd) ? gbef + ebef : -1);

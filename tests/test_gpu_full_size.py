@@ -1,6 +1,7 @@
 """GPU parity at the full workload sizes, on sampled sequences / query rows the oracle computes one by one.
 
-hier1m runs exactly the step bench.py times (same calls, same launch configuration).
+hier1m runs exactly the step bench.py times (same calls, same launch configuration, replayed from
+CUDA graphs as the bench does after one eager step).
 """
 import numpy as np
 import pytest
@@ -35,6 +36,17 @@ def test_hier1m_bench_step_sampled():
     wl.step()
     torch.cuda.synchronize()
     assert K().csa2_check(wl.err) == 0
+    eager = [t.clone() for t in (wl.o, wl.lse, wl.idx, wl.pool)]
+    wl.capture()
+    for t in (wl.o, wl.lse):
+        t.fill_(float("nan"))
+    for t in (wl.idx, wl.pool):
+        t.fill_(-7)
+    wl.step(graphs=True)
+    torch.cuda.synchronize()
+    assert K().csa2_check(wl.err) == 0
+    for a, e in zip((wl.o, wl.lse, wl.idx, wl.pool), eager):   # the graphs replay the same kernels
+        assert torch.equal(a, e)
     b = 3
     c = oracle_seq(spec, b, main_rows=[], gen_device=DEV)
     pos = spec.tokens[b] - 1

@@ -159,7 +159,8 @@ def test_index_score_rejects_bad_candidates():
     assert np.isfinite(got[:2]).all() and np.isneginf(got[2:]).all()
 
 
-@pytest.mark.parametrize("case", ["random", "ties", "short", "neg_inf", "pool", "long", "zeros"])
+@pytest.mark.parametrize("case", ["random", "ties", "short", "neg_inf", "pool", "long", "zeros", "odd", "unaligned",
+                                  "long_odd"])
 def test_topk_rows(case):
     k_ = K()
     g = torch.Generator(device="cpu").manual_seed(7)
@@ -181,12 +182,24 @@ def test_topk_rows(case):
         R, N, k2 = 3, 1 << 20, 16384
         s = torch.randn((R, N), generator=g).abs() * 50
         s[:, ::1000] = s[:, ::1000].round()      # some exact ties
+    elif case in ("odd", "unaligned"):          # rows the kernel must read one score at a time
+        N, k2 = (9003, 1024) if case == "odd" else (9000, 1024)
+        s = torch.randn((R, N), generator=g) * 10
+    elif case == "long_odd":
+        R, N, k2 = 2, (1 << 20) - 3, 16384
+        s = torch.randn((R, N), generator=g) * 50
     else:                                       # most scores equal (a fully-ReLU-zeroed row)
         N, k2 = 300000, 16384
         s = torch.zeros((R, N))
         s[:, 5::97] = torch.randn((R, len(range(5, N, 97))), generator=g)
     n_valid = torch.tensor([N, N - 1, N // 2, 511, 0][:R], dtype=torch.int32)
-    sd = s.to(DEV)
+    if case == "unaligned":                     # row base 4 bytes past a 16-byte boundary
+        buf = torch.empty(R * N + 1, dtype=torch.float32, device=DEV)
+        sd = buf[1:].view(R, N)
+        sd.copy_(s)
+        assert sd.data_ptr() % 16 == 4
+    else:
+        sd = s.to(DEV)
     val = torch.empty((R, k), dtype=torch.float32, device=DEV)
     out = k_.csa2_topk(sd, k, n_valid=n_valid.to(DEV), val=val, k2=k2)
     idx = to_np(out[0])
