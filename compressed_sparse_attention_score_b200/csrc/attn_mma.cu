@@ -18,8 +18,12 @@
 //          K = keys in 16-key steps), V^T chunks MN-major with 128-byte swizzle,
 //          accumulated in TMEM.
 // Phase 4  O / sum and lse = max + log(sum), coalesced fp32 stores.
-// The dequantising threads fill a 4-deep ring of 16 KB operand buffers while the
-// single issuing thread drives the tensor core; every wait is time-bounded.
+// A tile's raw key bytes (288 B per listed entry, 512 B per window token) are
+// gathered once into shared memory with asynchronous 16-byte copies, all in flight
+// together; both products dequantise from there, so a CTA whose keys fit one tile
+// reads them from memory once.  The dequantising threads fill a 4-deep ring of
+// 16 KB operand buffers while the single issuing thread drives the tensor core;
+// every wait is time-bounded.
 #include <cooperative_groups.h>
 #include <cuda_fp16.h>
 
@@ -33,26 +37,28 @@ namespace csa2 {
 using namespace sm100;
 
 namespace {
-constexpr int AM_THREADS = 256;
+constexpr int AM_PRODUCERS = 256;               // warps 0-7 dequantise keys
+constexpr int AM_THREADS = AM_PRODUCERS + 32;   // warp 8 drives the tensor core
 constexpr int AM_HG = 32;          // heads per CTA = MMA N
 constexpr int AM_TILE = 128;       // keys per S^T tile
 constexpr int AM_MAXKEYS = 640;    // 512 listed entries + 128 window tokens
 constexpr int AM_STAGES = 4;
-constexpr int AM_PF = 4;           // chunks of raw key bytes in flight per thread
 constexpr int AM_STAGE = 16384;
+constexpr int AM_RAW = 528;        // raw bytes per key in shared memory (512 + 16: conflict-free rows)
 constexpr uint32_t AM_TMEM_COLS = 256;
 constexpr uint64_t AM_WAIT_NS = 2000000000ull;
 
 constexpr int SM_Q = 0;                              // 8 chunks x [32 heads x 128 B]
 constexpr int SM_P = SM_Q + 8 * 4096;                // P^T [640 keys x 64 B]
 constexpr int SM_STG = SM_P + AM_MAXKEYS * 64;       // 4 x 16 KB operand ring
-constexpr int SM_SLOT = SM_STG + AM_STAGES * AM_STAGE;
+constexpr int SM_RAW = SM_STG + AM_STAGES * AM_STAGE;   // one tile of raw keys
+constexpr int SM_SLOT = SM_RAW + AM_TILE * AM_RAW;
 constexpr int SM_MU = SM_SLOT + AM_MAXKEYS * 8;      // logit multiplier per key
 constexpr int SM_PV = SM_MU + AM_MAXKEYS * 4;        // P multiplier per key
 constexpr int SM_RED = SM_PV + AM_MAXKEYS * 4;       // [4 warps][32 heads]; [CS][32] weights + [32] sums
 constexpr int SM_HM = SM_RED + 8 * 32 * 4;           // head max [32], head sum [32]
 constexpr int SM_BAR = SM_HM + 2 * 32 * 4;
-constexpr int SM_MISC = SM_BAR + 8 * (AM_STAGES + 1);
+constexpr int SM_MISC = SM_BAR + 8 * (2 * AM_STAGES + 1);
 constexpr int SM_TOTAL = SM_MISC + 16;
 constexpr size_t AM_SMEM = SM_TOTAL + 1024;
 }  // namespace
@@ -84,29 +90,32 @@ __device__ __forceinline__ int mnmaj128(int k, int mblk, int u) {
 // MN-major, 64-byte swizzle (P^T): K-row k (key), unit u of 8 heads.
 __device__ __forceinline__ int mnmaj64(int k, int u) { return (k >> 3) * 512 + (k & 7) * 64 + ((u ^ ((k & 7) >> 1)) << 4); }
 
-// Raw bytes one thread dequantises: 32 consecutive dims of one key.
-struct Raw {
-  uint4 a, b;      // sparse: a = 16 bytes of codes; window: a, b = 32 E4M3 codes
-  uint32_t sc;     // sparse: the two E4M3 block scales (low 16 bits)
-};
-
-// key: local key index of this CTA (slot[] is local); global key = key0 + key.
-__device__ __forceinline__ void load_raw(const AttnArgs &p, const int64_t *slot, int nks, int key0, int key, int dim0,
-                                         Raw &r) {
-  const int64_t s = slot[key];
-  if (s < 0) return;
-  if (key0 + key < nks) {
-    r.a = *reinterpret_cast<const uint4 *>(p.c.kv_codes + s * CSA2_MAIN_CODE_BYTES + dim0 / 2);
-    r.sc = *reinterpret_cast<const uint16_t *>(p.c.kv_scales + s * CSA2_MAIN_SCALE_BYTES + dim0 / 16);
-  } else {
-    const uint4 *src = reinterpret_cast<const uint4 *>(p.codes + s * CSA2_SWA_DIM + dim0);
-    r.a = src[0];
-    r.b = src[1];
+// Gather the raw bytes of local key tile t into shared memory (asynchronous 16-byte
+// copies by the producer threads, committed as one group): a listed entry's 256 code bytes and 32 scale bytes
+// at offsets 0 and 256 of its row, a window token's 512 codes at offset 0.
+__device__ __forceinline__ void gather_tile(const AttnArgs &p, const int64_t *slot, int nks, int key0, int t,
+                                            uint32_t raw) {
+  for (int i = threadIdx.x; i < AM_TILE * 32; i += AM_PRODUCERS) {
+    const int kt = i & (AM_TILE - 1), piece = i >> 7;  // consecutive threads: consecutive keys
+    const int key = t * AM_TILE + kt;
+    const int64_t s = slot[key];
+    if (s < 0) continue;
+    const uint32_t dst = raw + kt * AM_RAW + piece * 16;
+    if (key0 + key < nks) {
+      if (piece < 16)
+        cp_async_16(dst, p.c.kv_codes + s * CSA2_MAIN_CODE_BYTES + piece * 16);
+      else if (piece < 18)
+        cp_async_16(dst, p.c.kv_scales + s * CSA2_MAIN_SCALE_BYTES + (piece - 16) * 16);
+    } else {
+      cp_async_16(dst, p.codes + s * CSA2_SWA_DIM + piece * 16);
+    }
   }
+  cp_async_commit();
 }
 
-// 32 fp16 values (4 x 16 bytes) of one key from its raw bytes; zeros for a masked key.
-__device__ __forceinline__ void dequant32(const Raw &r, bool sparse, bool valid, uint4 (&out)[4]) {
+// 32 fp16 values (4 x 16 bytes) of dims dim0 .. dim0+31 of one key from its raw row;
+// zeros for a masked key.
+__device__ __forceinline__ void dequant32(const uint8_t *rk, bool sparse, bool valid, int dim0, uint4 (&out)[4]) {
   if (!valid) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) out[i] = make_uint4(0, 0, 0, 0);
@@ -114,13 +123,16 @@ __device__ __forceinline__ void dequant32(const Raw &r, bool sparse, bool valid,
   }
   uint32_t h[16];
   if (sparse) {
-    const uint32_t s0 = cvt_e4m3x2_f16x2((r.sc & 0xFF) * 0x101u);
-    const uint32_t s1 = cvt_e4m3x2_f16x2(((r.sc >> 8) & 0xFF) * 0x101u);
-    const uint32_t w[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
+    const uint4 a = *reinterpret_cast<const uint4 *>(rk + dim0 / 2);
+    const uint32_t sc = *reinterpret_cast<const uint16_t *>(rk + 256 + dim0 / 16);
+    const uint32_t s0 = cvt_e4m3x2_f16x2((sc & 0xFF) * 0x101u);
+    const uint32_t s1 = cvt_e4m3x2_f16x2(((sc >> 8) & 0xFF) * 0x101u);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
     for (int i = 0; i < 16; ++i) h[i] = hmul2_u32(cvt_e2m1x2_f16x2((w[i >> 2] >> (8 * (i & 3))) & 0xFF), i < 8 ? s0 : s1);
   } else {
-    const uint32_t w[8] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w};
+    const uint4 a = *reinterpret_cast<const uint4 *>(rk + dim0), b = *reinterpret_cast<const uint4 *>(rk + dim0 + 16);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int i = 0; i < 16; ++i) h[i] = cvt_e4m3x2_f16x2((w[i >> 1] >> (16 * (i & 1))) & 0xFFFF);
   }
@@ -158,12 +170,14 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   float *red = reinterpret_cast<float *>(smem + SM_RED);
   float *hmax = reinterpret_cast<float *>(smem + SM_HM);
   float *hsum = hmax + 32;
-  uint64_t *mma_done = reinterpret_cast<uint64_t *>(smem + SM_BAR);
-  uint64_t *phase_done = mma_done + AM_STAGES;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM_BAR);  // operand buffer written (256 arrivals)
+  uint64_t *mma_done = full + AM_STAGES;                          // operand buffer consumed (tcgen05.commit)
+  uint64_t *phase_done = mma_done + AM_STAGES;                    // all products of a phase complete
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM_MISC + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool producer = tid < AM_PRODUCERS, issuer = tid == AM_PRODUCERS;
   const int row = blockIdx.x, hg = blockIdx.y;
   const int b = row / p.Q;
   const int pos = p.q_pos[row];
@@ -184,6 +198,17 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   const int ntiles = min(tiles_all, tile0 + tps) - tile0;
   const int key0 = tile0 * AM_TILE;  // first key of this CTA; local key j is key key0 + j
   const int nvis = p.idx ? visible_entries(p.c, b, pos) : 0;
+  // the query block's loads go out first; they are converted once the key list is done
+  constexpr int QU = AM_HG * (D / 8) / AM_PRODUCERS;
+  uint4 qraw[QU];
+  if (producer) {
+    const uint16_t *qrow = p.q + (int64_t(row) * H + hg * AM_HG) * D;
+#pragma unroll
+    for (int u = 0; u < QU; ++u) {
+      const int it = tid + u * AM_PRODUCERS;
+      qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
+    }
+  }
   for (int jl = tid; jl < ntiles * AM_TILE; jl += AM_THREADS) {
     const int j = key0 + jl;
     int64_t s = -1;
@@ -208,32 +233,36 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     mu[jl] = m;
     pv[jl] = pm;
   }
-  // ---------------------------------------------------------------- Q (bf16 -> fp16, K-major 128B swizzle)
-  {
-    const uint16_t *qrow = p.q + (int64_t(row) * H + hg * AM_HG) * D;
-    for (int it = tid; it < AM_HG * (D / 8); it += AM_THREADS) {
-      const int h = it / (D / 8), u8 = it % (D / 8);  // 8 dims per item
-      const uint4 raw = *reinterpret_cast<const uint4 *>(qrow + h * D + u8 * 8);
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  if (warp == AM_PRODUCERS / 32) {
+    tmem_alloc(tmem_slot, AM_TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (issuer) {
+    for (int i = 0; i < AM_STAGES; ++i) {
+      mbar_init(&full[i], AM_PRODUCERS);
+      mbar_init(&mma_done[i], 1);
+    }
+    mbar_init(phase_done, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  __syncthreads();  // key list and barriers ready
+  const uint32_t raw = smem_u32(smem + SM_RAW);
+  if (producer) {
+    if (ntiles > 0) gather_tile(p, slot, nks, key0, 0, raw);
+#pragma unroll
+    for (int u = 0; u < QU; ++u) {
+      const int it = tid + u * AM_PRODUCERS, h = it / (D / 8), u8 = it % (D / 8);
+      const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
       uint32_t o4[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const __half2 hv = __floats2half2_rn(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
         o4[i] = *reinterpret_cast<const uint32_t *>(&hv);
       }
-      const int chunk = u8 / 8, u = u8 % 8;
-      *reinterpret_cast<uint4 *>(smem + SM_Q + chunk * 4096 + kmaj128(h, u)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+      *reinterpret_cast<uint4 *>(smem + SM_Q + (u8 / 8) * 4096 + kmaj128(h, u8 % 8)) =
+          make_uint4(o4[0], o4[1], o4[2], o4[3]);
     }
-  }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, AM_TMEM_COLS);
-    tmem_relinquish();
-  }
-  if (tid == 32) {
-    for (int i = 0; i < AM_STAGES; ++i) mbar_init(&mma_done[i], 1);
-    mbar_init(phase_done, 1);
-    *abort_flag = 0;
-    mbar_init_fence();
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -242,63 +271,78 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   const uint32_t tmem = *tmem_slot;
   const uint32_t stg = smem_u32(smem + SM_STG);
   bool aborted = false;
-  int chunk_no = 0;  // operand buffers used so far (ring position)
+  // Barrier over the producer threads that also ORs their abort state, so that every
+  // producer takes the same branch after it (none may skip a later barrier).
+  auto producers_sync = [&](bool mine) -> bool {
+    uint32_t any;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, 2, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(any)
+        : "r"(uint32_t(mine || *abort_flag)), "n"(AM_PRODUCERS)
+        : "memory");
+    return any != 0;
+  };
+  // Producer side of one operand buffer: wait until the tensor core has consumed what
+  // the buffer held AM_STAGES chunks ago, write it, publish it.  n = chunk number.
+  auto produce = [&](int n, auto &&write) -> bool {
+    const int buf = n % AM_STAGES;
+    if (n >= AM_STAGES && !mbar_wait_bounded(&mma_done[buf], ((n / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS))
+      return false;
+    write(smem + SM_STG + buf * AM_STAGE);
+    fence_proxy_async_smem();
+    mbar_arrive(&full[buf]);
+    return true;
+  };
 
   // ---------------------------------------------------------------- phase 1: S^T = K Q^T
-  // Raw bytes of the next AM_PF chunks are kept in flight in a register ring.
-  if (ntiles > 0) {
-    const int key_in = tid >> 1, half = tid & 1;  // 2 threads per key, 32 dims each
-    const int nch = ntiles * 8;
-    Raw ring[AM_PF];
+  // Producers: per tile, its raw keys in shared memory, then 8 chunks of 64 dims (one key
+  // per thread pair; consecutive threads take consecutive keys, so raw rows are read
+  // conflict-free).  Issuer: one 4-step MMA group per chunk as soon as it is published.
+  const int nch1 = ntiles * 8;
+  if (producer) {
+    const int key_in = tid & (AM_TILE - 1), half = tid >> 7;
+    for (int t = 0; t < ntiles; ++t) {
+      if (t > 0) {
+        aborted = producers_sync(aborted);  // every producer is past its reads of the previous raw tile
+        if (aborted) break;
+        gather_tile(p, slot, nks, key0, t, raw);
+      }
+      cp_async_wait<0>();
+      aborted = producers_sync(aborted);
+      if (aborted) break;
+      const int key = t * AM_TILE + key_in;
+      const bool sparse = key0 + key < nks, valid = slot[key] >= 0;
+      const uint8_t *rk = smem + SM_RAW + key_in * AM_RAW;
+      for (int c = 0; c < 8 && !aborted; ++c) {
+        aborted = !produce(t * 8 + c, [&](uint8_t *dst) {
+          uint4 out[4];
+          dequant32(rk, sparse, valid, 64 * c + 32 * half, out);
 #pragma unroll
-    for (int u = 0; u < AM_PF; ++u) {
-      ring[u] = Raw{};
-      if (u < nch) load_raw(p, slot, nks, key0, (u >> 3) * AM_TILE + key_in, 64 * (u & 7) + 32 * half, ring[u]);
-    }
-    for (int i0 = 0; i0 < nch && !aborted; i0 += AM_PF) {
-#pragma unroll
-      for (int u = 0; u < AM_PF; ++u) {
-        const int i = i0 + u;
-        if (i >= nch || aborted) break;
-        const int t = i >> 3, c = i & 7;
-        const int buf = chunk_no % AM_STAGES;
-        bool ok = true;
-        if (chunk_no >= AM_STAGES)
-          ok = mbar_wait_bounded(&mma_done[buf], ((chunk_no / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS);
-        const int key = t * AM_TILE + key_in;
-        uint4 out[4];
-        dequant32(ring[u], key0 + key < nks, slot[key] >= 0, out);
-        const int inext = i + AM_PF;
-        ring[u] = Raw{};
-        if (inext < nch) load_raw(p, slot, nks, key0, (inext >> 3) * AM_TILE + key_in, 64 * (inext & 7) + 32 * half, ring[u]);
-        uint8_t *dst = smem + SM_STG + buf * AM_STAGE;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) *reinterpret_cast<uint4 *>(dst + kmaj128(key_in, 4 * half + v)) = out[v];
-        fence_proxy_async_smem();
-        if (__syncthreads_or(!ok)) {
-          aborted = true;
-          break;
-        }
-        if (tid == 0) {
-          tc_fence_after();
-          constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, false, false);
-          const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_Q + c * 4096);
-#pragma unroll
-          for (int s = 0; s < 4; ++s)
-            tc_mma_f16(tmem + t * AM_HG, smem_desc(a0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B),
-                       smem_desc(b0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B), id, c > 0 || s > 0);
-          tc_commit(&mma_done[buf]);
-        }
-        ++chunk_no;
+          for (int v = 0; v < 4; ++v) *reinterpret_cast<uint4 *>(dst + kmaj128(key_in, 4 * half + v)) = out[v];
+        });
       }
     }
-    if (tid == 0) tc_commit(phase_done);
-  } else if (tid == 0) {
+  } else if (issuer) {
+    constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, false, false);
+    for (int n = 0; n < nch1; ++n) {
+      const int buf = n % AM_STAGES, t = n >> 3, c = n & 7;
+      if (!mbar_wait_bounded(&full[buf], (n / AM_STAGES) & 1, abort_flag, AM_WAIT_NS)) break;
+      tc_fence_after();
+      const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_Q + c * 4096);
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+        tc_mma_f16(tmem + t * AM_HG, smem_desc(a0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B),
+                   smem_desc(b0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B), id, c > 0 || s > 0);
+      tc_commit(&mma_done[buf]);
+    }
     tc_commit(phase_done);
   }
   {
-    const bool ok = aborted ? false : mbar_wait_bounded(phase_done, 0, abort_flag, AM_WAIT_NS);
-    if (__syncthreads_or(!ok)) aborted = true;
+    const bool ok = mbar_wait_bounded(phase_done, 0, abort_flag, AM_WAIT_NS);
+    if (__syncthreads_or(!ok || aborted)) aborted = true;
   }
   tc_fence_after();
 
@@ -370,59 +414,52 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   tc_fence_after();
 
   // ---------------------------------------------------------------- phase 3: O^T = V^T P^T
+  // Producers: per 64-key chunk, 4 chunks of 128 dims (a CTA with one tile still holds
+  // its raw keys).  Issuer: O^T accumulates over the key chunks.
   const int nkc = (ntiles * AM_TILE) / 64;  // 64-key chunks (masked keys carry P = 0, V = 0)
-  if (!aborted && nkc > 0) {
-    const int key_in = tid >> 2, qd = tid & 3;  // 4 threads per key, 32 dims each
-    const int nch = nkc * 4;
-    Raw ring[AM_PF];
+  if (!aborted && producer) {
+    const int key_in = tid & 63, qd = tid >> 6;  // 4 threads per key, 32 dims each
+    for (int jc = 0; jc < nkc; ++jc) {
+      const int t = jc >> 1;
+      if (ntiles > 1 && (jc & 1) == 0) {
+        aborted = producers_sync(aborted);  // every producer is past its reads of the raw tile
+        if (aborted) break;
+        gather_tile(p, slot, nks, key0, t, raw);
+        cp_async_wait<0>();
+        aborted = producers_sync(aborted);
+        if (aborted) break;
+      }
+      const int key = jc * 64 + key_in;
+      const bool sparse = key0 + key < nks, valid = slot[key] >= 0;
+      const uint8_t *rk = smem + SM_RAW + (key - t * AM_TILE) * AM_RAW;
+      for (int d = 0; d < 4 && !aborted; ++d) {
+        aborted = !produce(nch1 + jc * 4 + d, [&](uint8_t *dst) {
+          uint4 out[4];
+          dequant32(rk, sparse, valid, 128 * d + 32 * qd, out);
 #pragma unroll
-    for (int u = 0; u < AM_PF; ++u) {
-      ring[u] = Raw{};
-      if (u < nch) load_raw(p, slot, nks, key0, (u >> 2) * 64 + key_in, 128 * (u & 3) + 32 * qd, ring[u]);
-    }
-    for (int i0 = 0; i0 < nch && !aborted; i0 += AM_PF) {
-#pragma unroll
-      for (int u = 0; u < AM_PF; ++u) {
-        const int i = i0 + u;
-        if (i >= nch || aborted) break;
-        const int jc = i >> 2, d = i & 3;
-        const int buf = chunk_no % AM_STAGES;
-        bool ok = true;
-        if (chunk_no >= AM_STAGES)
-          ok = mbar_wait_bounded(&mma_done[buf], ((chunk_no / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS);
-        const int key = jc * 64 + key_in;
-        uint4 out[4];
-        dequant32(ring[u], key0 + key < nks, slot[key] >= 0, out);
-        const int inext = i + AM_PF;
-        ring[u] = Raw{};
-        if (inext < nch) load_raw(p, slot, nks, key0, (inext >> 2) * 64 + key_in, 128 * (inext & 3) + 32 * qd, ring[u]);
-        uint8_t *dst = smem + SM_STG + buf * AM_STAGE;
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          *reinterpret_cast<uint4 *>(dst + mnmaj128(key_in, qd >> 1, 4 * (qd & 1) + v)) = out[v];
-        fence_proxy_async_smem();
-        if (__syncthreads_or(!ok)) {
-          aborted = true;
-          break;
-        }
-        if (tid == 0) {
-          tc_fence_after();
-          constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, true, true);
-          const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_P);
-#pragma unroll
-          for (int s = 0; s < 4; ++s)
-            tc_mma_f16(tmem + d * AM_HG, smem_desc(a0 + 2048 * s, 8192, 1024, LAYOUT_SWIZZLE_128B),
-                       smem_desc(b0 + (8 * jc + 2 * s) * 512, 16, 512, LAYOUT_SWIZZLE_64B), id, jc > 0 || s > 0);
-          tc_commit(&mma_done[buf]);
-        }
-        ++chunk_no;
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4 *>(dst + mnmaj128(key_in, qd >> 1, 4 * (qd & 1) + v)) = out[v];
+        });
       }
     }
+  } else if (!aborted && issuer) {
+    constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, true, true);
+    for (int i = 0; i < nkc * 4; ++i) {
+      const int n = nch1 + i, buf = n % AM_STAGES, jc = i >> 2, d = i & 3;
+      if (!mbar_wait_bounded(&full[buf], (n / AM_STAGES) & 1, abort_flag, AM_WAIT_NS)) break;
+      tc_fence_after();
+      const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_P);
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+        tc_mma_f16(tmem + d * AM_HG, smem_desc(a0 + 2048 * s, 8192, 1024, LAYOUT_SWIZZLE_128B),
+                   smem_desc(b0 + (8 * jc + 2 * s) * 512, 16, 512, LAYOUT_SWIZZLE_64B), id, jc > 0 || s > 0);
+      tc_commit(&mma_done[buf]);
+    }
   }
-  if (tid == 0) tc_commit(phase_done);
+  if (issuer) tc_commit(phase_done);
   {
     const bool ok = aborted ? false : mbar_wait_bounded(phase_done, 1, abort_flag, AM_WAIT_NS);
-    if (__syncthreads_or(!ok)) aborted = true;
+    if (__syncthreads_or(!ok || aborted)) aborted = true;
   }
   tc_fence_after();
 
@@ -507,26 +544,46 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       if (split == 0) p.lse[int64_t(row) * H + hg * AM_HG + tid] = L > 0.f ? M + logf(L) : -INFINITY;
     }
     __syncthreads();
-    const int per = (D + CS - 1) / CS;
-    const int d0 = min(D, split * per), nd = min(D, d0 + per) - d0;
+    // this CTA's slice of dims (a multiple of 4), read as float4 from every peer with all
+    // of a thread's loads in flight together
+    const int per = ((D + CS - 1) / CS + 3) & ~3;
+    const int d0 = min(D, split * per), nq = (min(D, d0 + per) - d0) / 4;
     float *orow = p.o + (int64_t(row) * H + hg * AM_HG) * D;
-    for (int it = tid; it < 32 * nd; it += AM_THREADS) {
-      const int h = it / nd, dim = d0 + it % nd;
-      float acc = 0.f;
+    constexpr int CU = 2;  // items per thread per round
+    for (int it0 = tid; it0 < 32 * nq; it0 += CU * AM_THREADS) {
+      float4 x[CU][CS];
 #pragma unroll
-      for (int q = 0; q < CS; ++q) {
-        const float wq = wts[q * 32 + h];
-        if (wq != 0.f) acc += wq * cluster.map_shared_rank(stage, q)[h * D + dim];
+      for (int u = 0; u < CU; ++u) {
+        const int it = min(it0 + u * AM_THREADS, 32 * nq - 1);
+        const int h = it / nq, dim = d0 + 4 * (it % nq);
+#pragma unroll
+        for (int q = 0; q < CS; ++q)
+          x[u][q] = *reinterpret_cast<const float4 *>(cluster.map_shared_rank(stage, q) + h * D + dim);
       }
-      const float L = lsum[h];
-      orow[h * D + dim] = L > 0.f ? acc / L : 0.f;
+#pragma unroll
+      for (int u = 0; u < CU; ++u) {
+        const int it = it0 + u * AM_THREADS;
+        if (it >= 32 * nq) break;
+        const int h = it / nq, dim = d0 + 4 * (it % nq);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < CS; ++q) {
+          const float wq = wts[q * 32 + h];
+          acc.x += wq * x[u][q].x;
+          acc.y += wq * x[u][q].y;
+          acc.z += wq * x[u][q].z;
+          acc.w += wq * x[u][q].w;
+        }
+        const float L = lsum[h], inv = L > 0.f ? 1.f / L : 0.f;
+        *reinterpret_cast<float4 *>(orow + h * D + dim) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      }
     }
     cluster.sync();  // every peer has finished reading this CTA's stage
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == AM_PRODUCERS / 32) {
     tc_fence_after();
     tmem_dealloc(tmem, AM_TMEM_COLS);
   }
