@@ -160,6 +160,94 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32]) {
   return v[0];
 }
 
+// Cluster epilogue of a key-split row.  Partial of this CTA's keys: O_s (relative to
+// its own max m_s) staged in shared memory as [32 heads][512 dims] fp32, plus m_s and
+// l_s.  Then each CTA of the cluster combines one slice of dims over all peers:
+// o = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s, M = max_s m_s.
+template <int CS>
+__device__ __forceinline__ void combine_partials(const AttnArgs &p, uint32_t tmem, bool aborted, bool has_keys,
+                                                 float *stage, float *red, float *hmax, float *hsum, int row, int hg,
+                                                 int split) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (warp < 4) {
+    if (aborted) {
+      hsum[lane] = 0.f;
+      hmax[lane] = -INFINITY;
+    }
+    for (int d = 0; d < 4; ++d) {
+      uint32_t r0[16], r1[16];
+      if (!aborted && has_keys) {
+        const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + d * AM_HG;
+        tc_ld_32x32b_x16(ta, r0);
+        tc_ld_32x32b_x16(ta + 16, r1);
+        tc_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r0[i] = r1[i] = 0u;
+      }
+      const int dim = 128 * d + 32 * warp + lane;
+#pragma unroll
+      for (int h = 0; h < 16; ++h) {
+        stage[h * D + dim] = __uint_as_float(r0[h]);
+        stage[(16 + h) * D + dim] = __uint_as_float(r1[h]);
+      }
+    }
+  }
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();
+  float *wts = red;          // [CS][32] combination weights (red is free now)
+  float *lsum = red + CS * 32;
+  if (tid < 32) {
+    float M = -INFINITY;
+    for (int q = 0; q < CS; ++q) M = fmaxf(M, cluster.map_shared_rank(hmax, q)[tid]);
+    float L = 0.f;
+    for (int q = 0; q < CS; ++q) {
+      const float mq = cluster.map_shared_rank(hmax, q)[tid];
+      const float wq = (M == -INFINITY || mq == -INFINITY) ? 0.f : __expf(mq - M);
+      wts[q * 32 + tid] = wq;
+      L += wq * cluster.map_shared_rank(hsum, q)[tid];
+    }
+    lsum[tid] = L;
+    if (split == 0) p.lse[int64_t(row) * H + hg * AM_HG + tid] = L > 0.f ? M + logf(L) : -INFINITY;
+  }
+  __syncthreads();
+  // this CTA's slice of dims (a multiple of 4), read as float4 from every peer with all
+  // of a thread's loads in flight together
+  const int per = ((D + CS - 1) / CS + 3) & ~3;
+  const int d0 = min(D, split * per), nq = (min(D, d0 + per) - d0) / 4;
+  float *orow = p.o + (int64_t(row) * H + hg * AM_HG) * D;
+  constexpr int CU = 2;  // items per thread per round
+  for (int it0 = tid; it0 < 32 * nq; it0 += CU * AM_THREADS) {
+    float4 x[CU][CS];
+#pragma unroll
+    for (int u = 0; u < CU; ++u) {
+      const int it = min(it0 + u * AM_THREADS, 32 * nq - 1);
+      const int h = it / nq, dim = d0 + 4 * (it % nq);
+#pragma unroll
+      for (int q = 0; q < CS; ++q)
+        x[u][q] = *reinterpret_cast<const float4 *>(cluster.map_shared_rank(stage, q) + h * D + dim);
+    }
+#pragma unroll
+    for (int u = 0; u < CU; ++u) {
+      const int it = it0 + u * AM_THREADS;
+      if (it >= 32 * nq) break;
+      const int h = it / nq, dim = d0 + 4 * (it % nq);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < CS; ++q) {
+        const float wq = wts[q * 32 + h];
+        acc.x += wq * x[u][q].x;
+        acc.y += wq * x[u][q].y;
+        acc.z += wq * x[u][q].z;
+        acc.w += wq * x[u][q].w;
+      }
+      const float L = lsum[h], inv = L > 0.f ? 1.f / L : 0.f;
+      *reinterpret_cast<float4 *>(orow + h * D + dim) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+  }
+  cluster.sync();  // every peer has finished reading this CTA's stage
+}
+
 template <int CS>
 __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   extern __shared__ uint8_t smem_raw[];
@@ -497,88 +585,8 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       }
     }
   } else {
-    // Partial of this CTA's keys: O_s (relative to its own max m_s) staged in shared
-    // memory as [32 heads][512 dims] fp32 (reusing the P^T / operand space), plus m_s
-    // and l_s.  Then each CTA of the cluster combines one slice of dims over all peers:
-    // o = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s, M = max_s m_s.
-    float *stage = reinterpret_cast<float *>(smem + SM_P);
-    if (warp < 4) {
-      if (aborted) {
-        hsum[lane] = 0.f;
-        hmax[lane] = -INFINITY;
-      }
-      for (int d = 0; d < 4; ++d) {
-        uint32_t r0[16], r1[16];
-        if (!aborted && nkc > 0) {
-          const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + d * AM_HG;
-          tc_ld_32x32b_x16(ta, r0);
-          tc_ld_32x32b_x16(ta + 16, r1);
-          tc_wait_ld();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) r0[i] = r1[i] = 0u;
-        }
-        const int dim = 128 * d + 32 * warp + lane;
-#pragma unroll
-        for (int h = 0; h < 16; ++h) {
-          stage[h * D + dim] = __uint_as_float(r0[h]);
-          stage[(16 + h) * D + dim] = __uint_as_float(r1[h]);
-        }
-      }
-    }
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    float *wts = red;          // [CS][32] combination weights (red is free now)
-    float *lsum = red + CS * 32;
-    if (tid < 32) {
-      float M = -INFINITY;
-      for (int q = 0; q < CS; ++q) M = fmaxf(M, cluster.map_shared_rank(hmax, q)[tid]);
-      float L = 0.f;
-      for (int q = 0; q < CS; ++q) {
-        const float mq = cluster.map_shared_rank(hmax, q)[tid];
-        const float wq = (M == -INFINITY || mq == -INFINITY) ? 0.f : __expf(mq - M);
-        wts[q * 32 + tid] = wq;
-        L += wq * cluster.map_shared_rank(hsum, q)[tid];
-      }
-      lsum[tid] = L;
-      if (split == 0) p.lse[int64_t(row) * H + hg * AM_HG + tid] = L > 0.f ? M + logf(L) : -INFINITY;
-    }
-    __syncthreads();
-    // this CTA's slice of dims (a multiple of 4), read as float4 from every peer with all
-    // of a thread's loads in flight together
-    const int per = ((D + CS - 1) / CS + 3) & ~3;
-    const int d0 = min(D, split * per), nq = (min(D, d0 + per) - d0) / 4;
-    float *orow = p.o + (int64_t(row) * H + hg * AM_HG) * D;
-    constexpr int CU = 2;  // items per thread per round
-    for (int it0 = tid; it0 < 32 * nq; it0 += CU * AM_THREADS) {
-      float4 x[CU][CS];
-#pragma unroll
-      for (int u = 0; u < CU; ++u) {
-        const int it = min(it0 + u * AM_THREADS, 32 * nq - 1);
-        const int h = it / nq, dim = d0 + 4 * (it % nq);
-#pragma unroll
-        for (int q = 0; q < CS; ++q)
-          x[u][q] = *reinterpret_cast<const float4 *>(cluster.map_shared_rank(stage, q) + h * D + dim);
-      }
-#pragma unroll
-      for (int u = 0; u < CU; ++u) {
-        const int it = it0 + u * AM_THREADS;
-        if (it >= 32 * nq) break;
-        const int h = it / nq, dim = d0 + 4 * (it % nq);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int q = 0; q < CS; ++q) {
-          const float wq = wts[q * 32 + h];
-          acc.x += wq * x[u][q].x;
-          acc.y += wq * x[u][q].y;
-          acc.z += wq * x[u][q].z;
-          acc.w += wq * x[u][q].w;
-        }
-        const float L = lsum[h], inv = L > 0.f ? 1.f / L : 0.f;
-        *reinterpret_cast<float4 *>(orow + h * D + dim) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      }
-    }
-    cluster.sync();  // every peer has finished reading this CTA's stage
+    combine_partials<CS>(p, tmem, aborted, nkc > 0, reinterpret_cast<float *>(smem + SM_P), red, hmax, hsum, row, hg,
+                         split);
   }
 
   tc_fence_before();
@@ -588,6 +596,303 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     tmem_dealloc(tmem, AM_TMEM_COLS);
   }
   if (tid == 0 && aborted) report(p.err, CSA2_ERR_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------
+// Single-tile form (a cluster of CS CTAs, one 128-key tile each): every key is
+// dequantised once, straight from its loads into a 128 KB fp16 tile laid out as
+// 8 blocks of 64 dims x 128 keys (128-byte swizzle).  The same bytes are the
+// K-major A operand of S^T = K Q^T (one block per 64-dim step) and the MN-major
+// A operand of O^T = V^T P^T (two blocks per 128-dim step, 16 KB apart), so the
+// second product needs no producer work at all.
+namespace {
+constexpr int T_Q = 0;                          // Q (32 KB); P^T once S^T is complete
+constexpr int T_KT = T_Q + 8 * 4096;            // fp16 key tile (128 KB); the partial O afterwards
+constexpr int T_SLOT = T_KT + 8 * 16384;
+constexpr int T_MU = T_SLOT + AM_TILE * 8;
+constexpr int T_PV = T_MU + AM_TILE * 4;
+constexpr int T_RED = T_PV + AM_TILE * 4;
+constexpr int T_HM = T_RED + 8 * 32 * 4;
+constexpr int T_BAR = T_HM + 2 * 32 * 4;        // full[8], qfull, phase_done
+constexpr int T_MISC = T_BAR + 8 * 10;
+constexpr size_t T_SMEM = T_MISC + 16 + 1024;
+}  // namespace
+
+template <int CS>
+__global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  int64_t *slot = reinterpret_cast<int64_t *>(smem + T_SLOT);
+  float *mu = reinterpret_cast<float *>(smem + T_MU);
+  float *pv = reinterpret_cast<float *>(smem + T_PV);
+  float *red = reinterpret_cast<float *>(smem + T_RED);
+  float *hmax = reinterpret_cast<float *>(smem + T_HM);
+  float *hsum = hmax + 32;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + T_BAR);  // 64-dim block b of the tile written (128)
+  uint64_t *qfull = full + 8;                                     // Q written (256)
+  uint64_t *phase_done = qfull + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + T_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + T_MISC + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool producer = tid < AM_PRODUCERS, issuer = tid == AM_PRODUCERS;
+  const int row = blockIdx.x, hg = blockIdx.y;
+  const int split = int(cg::this_cluster().block_rank());
+  const int b = row / p.Q;
+  const int pos = p.q_pos[row];
+  const int nks = p.idx ? p.k : 0;
+  int lo = 0, nkw = 0;
+  if (p.codes && pos >= 0) {
+    lo = max(0, pos - p.window + 1);
+    nkw = pos - lo + 1;
+  }
+  const int nk = nks + nkw;
+  const int key0 = split * AM_TILE;
+
+  // ---------------------------------------------------------------- loads
+  // Producer t: key t % 128, dims 256 (t / 128) .. +255.  The query block's loads go
+  // out first, then the key's index, then its raw bytes, all before any barrier.
+  constexpr int QU = AM_HG * (D / 8) / AM_PRODUCERS;
+  uint4 qraw[QU];
+  uint4 rr[16];  // listed entry: rr[0..7] = 128 code bytes, rr[8] = 16 scale bytes; window: 256 codes
+  const int key_in = tid & (AM_TILE - 1), half = (tid >> 7) & 1;
+  const int j = key0 + key_in;
+  bool sparse = false;
+  int64_t s = -1;
+  if (producer) {
+    const uint16_t *qrow = p.q + (int64_t(row) * H + hg * AM_HG) * D;
+#pragma unroll
+    for (int u = 0; u < QU; ++u) {
+      const int it = tid + u * AM_PRODUCERS;
+      qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
+    }
+    float m = 0.f, pm = 0.f;
+    if (j < nks) {
+      sparse = true;
+      const int n = p.idx[int64_t(row) * p.k + j];
+      if (n != -1) {
+        if (n < -1 || n >= visible_entries(p.c, b, pos)) {
+          if (half == 0) report(p.err, CSA2_ERR_INDEX);
+        } else {
+          s = cache_slot(p.c, b, n);
+          if (s < 0 && half == 0) report(p.err, CSA2_ERR_INDEX);
+        }
+      }
+      m = p.tau, pm = 1.f;
+      if (s >= 0) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.c.kv_codes + s * CSA2_MAIN_CODE_BYTES + half * 128);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) rr[i] = src[i];
+        rr[8] = *reinterpret_cast<const uint4 *>(p.c.kv_scales + s * CSA2_MAIN_SCALE_BYTES + half * 16);
+      }
+    } else if (j < nk) {
+      s = int64_t(b) * p.R + (lo + (j - nks)) % p.R;
+      const float sc = p.scale[s];
+      m = p.tau * sc, pm = sc;
+      const uint4 *src = reinterpret_cast<const uint4 *>(p.codes + s * CSA2_SWA_DIM + half * 256);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) rr[i] = src[i];
+    }
+    if (half == 0) {
+      slot[key_in] = s;
+      mu[key_in] = m;
+      pv[key_in] = pm;
+    }
+  }
+  if (warp == AM_PRODUCERS / 32) {
+    tmem_alloc(tmem_slot, AM_TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (issuer) {
+    for (int i = 0; i < 8; ++i) mbar_init(&full[i], AM_TILE);
+    mbar_init(qfull, AM_PRODUCERS);
+    mbar_init(phase_done, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  tc_fence_before();
+  __syncthreads();  // barriers, key list and TMEM address ready
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool aborted = false;
+
+  // ---------------------------------------------------------------- phase 1: S^T = K Q^T
+  if (producer) {
+#pragma unroll
+    for (int u = 0; u < QU; ++u) {
+      const int it = tid + u * AM_PRODUCERS, h = it / (D / 8), u8 = it % (D / 8);
+      const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
+      uint32_t o4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __half2 hv = __floats2half2_rn(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+        o4[i] = *reinterpret_cast<const uint32_t *>(&hv);
+      }
+      *reinterpret_cast<uint4 *>(smem + T_Q + (u8 / 8) * 4096 + kmaj128(h, u8 % 8)) =
+          make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(qfull);
+    // this thread's four 64-dim blocks of its key, each published as soon as it is written
+    const bool valid = s >= 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int blk = 4 * half + c;
+      uint8_t *dst = smem + T_KT + blk * 16384;
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {  // 32 dims at a time
+        uint32_t h16[16];
+        if (!valid) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) h16[i] = 0u;
+        } else if (sparse) {
+          const uint4 a = rr[2 * c + q2];
+          const uint32_t sw = (&rr[8].x)[c];  // scale bytes of dims 64c .. 64c+63 of this half
+          const uint32_t sc = (sw >> (16 * q2)) & 0xFFFF;
+          const uint32_t s0 = cvt_e4m3x2_f16x2((sc & 0xFF) * 0x101u);
+          const uint32_t s1 = cvt_e4m3x2_f16x2(((sc >> 8) & 0xFF) * 0x101u);
+          const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            h16[i] = hmul2_u32(cvt_e2m1x2_f16x2((w[i >> 2] >> (8 * (i & 3))) & 0xFF), i < 8 ? s0 : s1);
+        } else {
+          const uint4 a = rr[4 * c + 2 * q2], bb = rr[4 * c + 2 * q2 + 1];
+          const uint32_t w[8] = {a.x, a.y, a.z, a.w, bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+          for (int i = 0; i < 16; ++i) h16[i] = cvt_e4m3x2_f16x2((w[i >> 1] >> (16 * (i & 1))) & 0xFFFF);
+        }
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<uint4 *>(dst + kmaj128(key_in, 4 * q2 + v)) =
+              make_uint4(h16[4 * v], h16[4 * v + 1], h16[4 * v + 2], h16[4 * v + 3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&full[blk]);
+    }
+  } else if (issuer) {
+    constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, false, false);
+    bool ok = mbar_wait_bounded(qfull, 0, abort_flag, AM_WAIT_NS);
+    for (int i = 0; i < 8 && ok; ++i) {
+      const int blk = (i & 1) * 4 + (i >> 1);  // both halves' blocks in the order they are written
+      if (!(ok = mbar_wait_bounded(&full[blk], 0, abort_flag, AM_WAIT_NS))) break;
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(smem + T_KT + blk * 16384), b0 = smem_u32(smem + T_Q + blk * 4096);
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4)
+        tc_mma_f16(tmem, smem_desc(a0 + 32 * k4, 16, 1024, LAYOUT_SWIZZLE_128B),
+                   smem_desc(b0 + 32 * k4, 16, 1024, LAYOUT_SWIZZLE_128B), id, i > 0 || k4 > 0);
+    }
+    tc_commit(phase_done);
+  }
+  {
+    const bool ok = mbar_wait_bounded(phase_done, 0, abort_flag, AM_WAIT_NS);
+    if (__syncthreads_or(!ok)) aborted = true;
+  }
+  tc_fence_after();
+
+  // ---------------------------------------------------------------- phase 2: softmax over the tile
+  if (!aborted && warp < 4) {
+    const int key = 32 * warp + lane;
+    uint32_t r0[16], r1[16];
+    const uint32_t ta = tmem + (uint32_t(32 * warp) << 16);
+    tc_ld_32x32b_x16(ta, r0);
+    tc_ld_32x32b_x16(ta + 16, r1);
+    tc_wait_ld();
+    const bool valid = slot[key] >= 0;
+    const float m = mu[key], pm = pv[key];
+    float x[32], mx[32];
+#pragma unroll
+    for (int h = 0; h < 16; ++h) {
+      x[h] = m * __uint_as_float(r0[h]);
+      x[16 + h] = m * __uint_as_float(r1[h]);
+    }
+#pragma unroll
+    for (int h = 0; h < 32; ++h) mx[h] = valid ? x[h] : -INFINITY;
+    red[warp * 32 + lane] = reduce_scatter32<true>(mx);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (warp == 0)
+      hmax[lane] = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane]));
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    float sm[32];
+    uint32_t ph[16];
+#pragma unroll
+    for (int h = 0; h < 32; h += 2) {
+      const float m0 = hmax[h], m1 = hmax[h + 1];
+      const float e0 = (valid && m0 != -INFINITY) ? __expf(x[h] - m0) : 0.f;
+      const float e1 = (valid && m1 != -INFINITY) ? __expf(x[h + 1] - m1) : 0.f;
+      sm[h] = e0;
+      sm[h + 1] = e1;
+      const __half2 hp = __floats2half2_rn(e0 * pm, e1 * pm);
+      ph[h >> 1] = *reinterpret_cast<const uint32_t *>(&hp);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      *reinterpret_cast<uint4 *>(smem + T_Q + mnmaj64(key, u)) =
+          make_uint4(ph[4 * u], ph[4 * u + 1], ph[4 * u + 2], ph[4 * u + 3]);
+    red[warp * 32 + lane] = reduce_scatter32<false>(sm);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (warp == 0) hsum[lane] = (red[lane] + red[32 + lane]) + (red[64 + lane] + red[96 + lane]);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  // ---------------------------------------------------------------- phase 3: O^T = V^T P^T
+  if (!aborted && issuer) {
+    constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, true, true);
+    const uint32_t kt = smem_u32(smem + T_KT), pt = smem_u32(smem + T_Q);
+    for (int d = 0; d < 4; ++d)
+#pragma unroll
+      for (int jc = 0; jc < 2; ++jc)
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4)
+          tc_mma_f16(tmem + d * AM_HG,
+                     smem_desc(kt + (2 * d) * 16384 + jc * 8192 + 2048 * k4, 16384, 1024, LAYOUT_SWIZZLE_128B),
+                     smem_desc(pt + (8 * jc + 2 * k4) * 512, 16, 512, LAYOUT_SWIZZLE_64B), id, jc > 0 || k4 > 0);
+  }
+  if (issuer) tc_commit(phase_done);
+  {
+    const bool ok = aborted ? false : mbar_wait_bounded(phase_done, 1, abort_flag, AM_WAIT_NS);
+    if (__syncthreads_or(!ok)) aborted = true;
+  }
+  tc_fence_after();
+
+  // ---------------------------------------------------------------- phase 4: combine the cluster's partials
+  combine_partials<CS>(p, tmem, aborted, true, reinterpret_cast<float *>(smem + T_KT), red, hmax, hsum, row, hg,
+                       split);
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == AM_PRODUCERS / 32) {
+    tc_fence_after();
+    tmem_dealloc(tmem, AM_TMEM_COLS);
+  }
+  if (tid == 0 && aborted) report(p.err, CSA2_ERR_TIMEOUT);
+}
+
+template <int CS>
+static void launch_tile(const AttnArgs &a, int rows, cudaStream_t st) {
+  static bool attr[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr[dev]) {
+    cudaFuncSetAttribute(attn_tile_kernel<CS>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(T_SMEM));
+    attr[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows, H / AM_HG, CS);
+  cfg.blockDim = dim3(AM_THREADS);
+  cfg.dynamicSmemBytes = T_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = CS;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, attn_tile_kernel<CS>, a);
 }
 
 template <int CS>
@@ -633,6 +938,14 @@ void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, floa
   a.o = o, a.lse = lse, a.err = err;
   const int tiles = (a.k + (codes ? window : 0) + AM_TILE - 1) / AM_TILE;
   const int cs = rows * (H / AM_HG) <= 64 ? max(1, min(tiles, 5)) : 1;
+  if (cs > 1 && cs == tiles) {  // one tile per CTA: the single-dequant form
+    switch (cs) {
+      case 2: launch_tile<2>(a, rows, st); return;
+      case 3: launch_tile<3>(a, rows, st); return;
+      case 4: launch_tile<4>(a, rows, st); return;
+      default: launch_tile<5>(a, rows, st); return;
+    }
+  }
   switch (cs) {
     case 2: launch_cs<2>(a, rows, st); break;
     case 3: launch_cs<3>(a, rows, st); break;

@@ -348,6 +348,19 @@ def test_reuse_decode_scaled():
     _decode_layer_parity(spec, cache, "reuse", 0, rings, codes, scale, idx_in=idx, oracle_caches=oc)
 
 
+@pytest.mark.parametrize("kk,fused", [(128, True), (256, True), (300, True), (384, False), (300, False),
+                                      (512, False)])
+def test_reuse_decode_key_counts(kk, fused):
+    """2 to 5 key tiles per row (one CTA each), tiles that mix listed entries with window tokens."""
+    spec = W.scaled(W.reuse64k(), [6000, 2500, 4096, 777], B=4, k=kk)
+    cache = gpu_cache(spec)
+    codes, scale, rings = _swa_state(spec, 2)
+    idx = W.reuse_indices(spec, DEV)
+    idx[3, 0, kk // 2:] = -1
+    oc = [oracle_seq(spec, b, main_rows=[], gen_device=DEV) for b in range(spec.B)]
+    _decode_layer_parity(spec, cache, "reuse", 2, rings, codes, scale, idx_in=idx, oracle_caches=oc, fused=fused)
+
+
 def test_reuse_rejects_out_of_range_indices():
     k = K()
     spec = W.scaled(W.reuse64k(), [1000], B=1)
