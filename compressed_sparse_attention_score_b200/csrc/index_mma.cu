@@ -15,10 +15,12 @@
 //              (64-byte swizzle) plus one 512-byte bulk copy of the scales;
 //              for candidate lists, cp.async of each listed entry instead;
 //   warp 1     MMA issuer (one lane): tcgen05.cp of the scale atom to TMEM, two
-//              K=64 MMAs into a double-buffered TMEM accumulator, tcgen05.commit;
-//   warps 2-5  epilogue: tcgen05.ld of the 64 head values of its 32 keys,
-//              weighted ReLU sum, coalesced fp32 score store.
-// The query heads are quantised to MXFP4 in the prologue (same codec as the keys).
+//              K=64 MMAs into one of three TMEM accumulators, tcgen05.commit;
+//   warps 2-9  epilogue, two warpgroups taking alternate tiles: tcgen05.ld of
+//              the 64 head values of its 32 keys, weighted ReLU sum, fp32 score
+//              store.
+// The query heads are quantised to MXFP4 in the prologue (warps 2-5; same codec as
+// the keys).
 // Every mbarrier wait is time-bounded; on expiry the CTA drains and reports
 // CSA2_ERR_TIMEOUT instead of hanging.
 #include <cuda.h>
@@ -39,8 +41,8 @@ constexpr int IM_TILE = 128;           // keys per tile = MMA M
 constexpr int IM_N = 64;               // indexer heads = MMA N
 constexpr int IM_A_BYTES = IM_TILE * 64;
 constexpr int IM_STAGE_BYTES = 9216;   // 8192 codes + 512 scale atom, padded to 1024
-constexpr int IM_ACC = 2;              // TMEM accumulators (64 columns each)
-constexpr int IM_EPI_WG = 1;           // epilogue warpgroups, alternating tiles
+constexpr int IM_ACC = 3;              // TMEM accumulators (64 columns each)
+constexpr int IM_EPI_WG = 2;           // epilogue warpgroups, alternating tiles
 constexpr int IM_THREADS = 64 + 128 * IM_EPI_WG;
 constexpr uint32_t IM_TMEM_COLS = 256;
 constexpr uint32_t COL_SFA = IM_ACC * 64;   // one 4-column scale buffer per accumulator
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
         const int s = i % IM_STAGES, acc = i % IM_ACC;
         if (!mbar_wait_bounded(&full[s], (i / IM_STAGES) & 1, abort_flag, WAIT_LIMIT_NS)) break;
         if (!mbar_wait_bounded(&acc_empty[acc], ((i / IM_ACC) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
-        fence_proxy_async_smem();  // cp.async-filled stages (gather path) are read by the tensor core
+        if (!a.use_tma) fence_proxy_async_smem();  // cp.async-filled stages are read by the tensor core
         tc_fence_after();
         const uint32_t st = stages + s * IM_STAGE_BYTES;
         const uint32_t sfa = tmem + COL_SFA + 4 * acc;
