@@ -487,43 +487,51 @@ static cudaError_t launch_cs(const float *scores, const int32_t *n_valid, int R,
   return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<CS>, scores, n_valid, N, s0, s1, nsel, map);
 }
 
+// Clusters of CS CTAs (one per SM) that the device can hold at once, per device.
+template <int CS>
+static int max_active_clusters() {
+  static int cached[64] = {};  // 0 unknown, -1 none
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    if (CS > 8) cudaFuncSetAttribute(topk_cluster_kernel<CS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(topk_cluster_kernel<CS>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(tk_smem_bytes(CS)));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CS);
+    cfg.blockDim = dim3(TK_THREADS);
+    cfg.dynamicSmemBytes = tk_smem_bytes(CS);
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = CS;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    cached[dev] = (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<CS>, &cfg) == cudaSuccess && n > 0) ? n : -1;
+    cudaGetLastError();
+  }
+  return cached[dev];
+}
+
 // Cluster size by row length and count: one CTA per row up to 64K scores or from 148 rows
-// on; otherwise 8 CTAs up to 256K scores and 16 above.
+// on; otherwise the largest of 16, 12 and 8 CTAs whose clusters all fit on the device at
+// once (a cluster needs its CTAs' SMs in one GPC, so fewer large clusters fit than
+// SMs / CS), 8 up to 256K scores.
 void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int N, int k0, int32_t *idx0, float *val0,
                          int k1, int32_t *idx1, float *val1, const int32_t *map, cudaStream_t st) {
   if (R == 0) return;
   const Sel s0{k0, idx0, val0}, s1{k1, idx1, val1};
   const int nsel = (k1 > 0 && idx1) ? 2 : 1;
-  static int cluster16_ok[64] = {};  // 0 unknown, 1 yes, -1 no
-  int dev = 0;
-  cudaGetDevice(&dev);
   if (N >= (1 << 18) && R < 148) {
-    if (dev >= 0 && dev < 64 && cluster16_ok[dev] == 0) {
-      cudaFuncSetAttribute(topk_cluster_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(16);
-      cfg.blockDim = dim3(TK_THREADS);
-      cfg.dynamicSmemBytes = tk_smem_bytes(16);
-      cudaFuncSetAttribute(topk_cluster_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(tk_smem_bytes(16)));
-      cudaLaunchAttribute at[1];
-      at[0].id = cudaLaunchAttributeClusterDimension;
-      at[0].val.clusterDim.x = 16;
-      at[0].val.clusterDim.y = 1;
-      at[0].val.clusterDim.z = 1;
-      cfg.attrs = at;
-      cfg.numAttrs = 1;
-      int nclusters = 0;
-      cluster16_ok[dev] =
-          (cudaOccupancyMaxActiveClusters(&nclusters, topk_cluster_kernel<16>, &cfg) == cudaSuccess && nclusters > 0)
-              ? 1
-              : -1;
-      cudaGetLastError();
-    }
-    if (cluster16_ok[dev] > 0) {
+    if (max_active_clusters<16>() >= R) {
       launch_cs<16>(scores, n_valid, R, N, s0, s1, nsel, map, st);
-      return;
+    } else if (max_active_clusters<12>() >= R) {
+      launch_cs<12>(scores, n_valid, R, N, s0, s1, nsel, map, st);
+    } else {
+      launch_cs<8>(scores, n_valid, R, N, s0, s1, nsel, map, st);
     }
-    launch_cs<8>(scores, n_valid, R, N, s0, s1, nsel, map, st);
   } else if (N > (1 << 16) && R < 148) {
     launch_cs<8>(scores, n_valid, R, N, s0, s1, nsel, map, st);
   } else {

@@ -160,7 +160,7 @@ def test_index_score_rejects_bad_candidates():
 
 
 @pytest.mark.parametrize("case", ["random", "ties", "short", "neg_inf", "pool", "long", "zeros", "odd", "unaligned",
-                                  "long_odd"])
+                                  "long_odd", "long8"])
 def test_topk_rows(case):
     k_ = K()
     g = torch.Generator(device="cpu").manual_seed(7)
@@ -185,6 +185,9 @@ def test_topk_rows(case):
     elif case in ("odd", "unaligned"):          # rows the kernel must read one score at a time
         N, k2 = (9003, 1024) if case == "odd" else (9000, 1024)
         s = torch.randn((R, N), generator=g) * 10
+    elif case == "long8":                       # more 2^20-entry rows than 16-CTA clusters fit at once
+        R, N, k2 = 8, 1 << 20, 16384
+        s = torch.randn((R, N), generator=g) * 30
     elif case == "long_odd":
         R, N, k2 = 2, (1 << 20) - 3, 16384
         s = torch.randn((R, N), generator=g) * 50
@@ -192,7 +195,7 @@ def test_topk_rows(case):
         N, k2 = 300000, 16384
         s = torch.zeros((R, N))
         s[:, 5::97] = torch.randn((R, len(range(5, N, 97))), generator=g)
-    n_valid = torch.tensor([N, N - 1, N // 2, 511, 0][:R], dtype=torch.int32)
+    n_valid = torch.tensor(([N, N - 1, N // 2, 511, 0] + [N - 7 * i for i in range(1, 4)])[:R], dtype=torch.int32)
     if case == "unaligned":                     # row base 4 bytes past a 16-byte boundary
         buf = torch.empty(R * N + 1, dtype=torch.float32, device=DEV)
         sd = buf[1:].view(R, N)
