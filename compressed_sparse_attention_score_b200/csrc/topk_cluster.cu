@@ -229,9 +229,19 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
       }
     }
   };
-  // Count pass over every key (no lists): warp-aggregated top-12-bit histogram.
-  auto count_pass = [&](uint32_t *hdst) {
-    for (int base = wb; base < we; base += 32 * U) {
+  // A single-CTA row of at most TK_LIST_WORDS scores is copied once, as keys, into the
+  // candidate-list space; every pass then reads shared memory instead of the scores.
+  const bool resident = CS == 1 && n <= TK_LIST_WORDS;
+  uint32_t *skeys = tk_smem;
+  // Keys u = 0 .. U-1 of the group starting at base (lane-strided), -inf past the range.
+  auto load_keys = [&](int base, uint32_t (&kk)[U]) {
+    if (resident) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = base + 32 * u + lane;
+        kk[u] = j < we ? skeys[j] : KEY_NEG_INF;
+      }
+    } else {
       float v[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -239,8 +249,17 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
         v[u] = j < we ? srow[j] : -INFINITY;
       }
 #pragma unroll
+      for (int u = 0; u < U; ++u) kk[u] = score_key(v[u]);
+    }
+  };
+  // Count pass over every key (no lists): warp-aggregated top-12-bit histogram.
+  auto count_pass = [&](uint32_t *hdst) {
+    for (int base = wb; base < we; base += 32 * U) {
+      uint32_t kk[U];
+      load_keys(base, kk);
+#pragma unroll
       for (int u = 0; u < U; ++u) {
-        const uint32_t key = score_key(v[u]);
+        const uint32_t key = kk[u];
         const bool take = key != KEY_NEG_INF;
         const uint32_t peers = __match_any_sync(0xffffffffu, take ? (key >> 20) : 0xFFFFFFFFu);
         if (take && (peers & lt_mask) == 0) atomicAdd(&hdst[key >> 20], uint32_t(__popc(peers)));
@@ -248,7 +267,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
     }
   };
   // Visit the warp's keys in index order, 32 per step (lane = position in the step):
-  // from its candidate list (fast) or from the scores themselves.  f(key, index, valid).
+  // from its candidate list (fast) or from all keys (shared memory when the row is
+  // resident, else the scores).  f(key, index, valid).
   auto walk = [&](bool fast, auto &&f) {
     if (fast) {
       const int m = min(cnt, TK_CAPW);
@@ -259,17 +279,10 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
       }
     } else {
       for (int base = wb; base < we; base += 32 * U) {
-        float vv[U];
+        uint32_t kk[U];
+        load_keys(base, kk);
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int j = base + 32 * u + lane;
-          vv[u] = j < we ? srow[j] : -INFINITY;
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const uint32_t key = score_key(vv[u]);
-          f(key, base + 32 * u + lane, key != KEY_NEG_INF);
-        }
+        for (int u = 0; u < U; ++u) f(kk[u], base + 32 * u + lane, kk[u] != KEY_NEG_INF);
       }
     }
   };
@@ -278,6 +291,46 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   if (tid == 0) overflow_s = 0;
   __syncthreads();
 
+  uint32_t prefix[2] = {0, 0}, rem[2] = {0, 0};
+  int width[2] = {0, 0};
+  bool all[2] = {true, true};
+  // Per selection: radix prefix of T and its width in bits (resolved once the prefix's bin
+  // holds exactly the keys still needed), keys still needed, or "take every key".
+  auto first_digit = [&](const uint32_t *h, int lo) {
+    sum_coarse(h, 0, TK_BINS, lo, true, false);
+    if (warp < nsel) warp_select(sumc, h, TK_BINS, uint32_t(warp ? s1.k : s0.k), warp);
+    __syncthreads();
+    for (int s = 0; s < nsel; ++s) {
+      all[s] = sel_bin[s] < 0;
+      if (!all[s]) {
+        prefix[s] = uint32_t(sel_bin[s]);
+        rem[s] = uint32_t(s ? s1.k : s0.k) - sel_above[s];
+        width[s] = 12;
+      }
+    }
+  };
+  bool fast = false;
+  if (resident) {
+    // ---- the whole row into shared memory as keys, then pass 0 over it
+    const float *src = srow;  // one CTA: its range is the whole row
+    if (vec) {
+      for (int i = 4 * tid; i < n; i += 4 * TK_THREADS) {
+        if (i + 3 < n) {
+          const float4 v = *reinterpret_cast<const float4 *>(src + i);
+          *reinterpret_cast<uint4 *>(skeys + i) = make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
+        } else {
+          for (int e = i; e < n; ++e) skeys[e] = score_key(src[e]);
+        }
+      }
+    } else {
+      for (int i = tid; i < n; i += TK_THREADS) skeys[i] = score_key(src[i]);
+    }
+    __syncthreads();
+    count_pass(hs);
+    make_coarse(hs, TK_BINS);
+    __syncthreads();
+    first_digit(hs, 0);
+  } else {
   // ---- sampled lower bound on the larger selection's threshold (top 12 key bits)
   const uint32_t target = uint32_t(kbig / SAMPLE) + uint32_t(kbig / (2 * SAMPLE)) + 32;
   for (int base = wb; base < we; base += 32 * SAMPLE * 4) {
@@ -311,27 +364,9 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
 #pragma unroll
   for (int q = 0; q < CS; ++q)
     any_overflow |= int(*peer(reinterpret_cast<const uint32_t *>(&overflow_s), q));
-  // Per selection: radix prefix of T and its width in bits (resolved once the prefix's bin
-  // holds exactly the keys still needed), keys still needed, or "take every key".
-  uint32_t prefix[2] = {0, 0}, rem[2] = {0, 0};
-  int width[2] = {0, 0};
-  bool all[2] = {true, true};
-  auto first_digit = [&](const uint32_t *h, int lo) {
-    sum_coarse(h, 0, TK_BINS, lo, true, false);
-    if (warp < nsel) warp_select(sumc, h, TK_BINS, uint32_t(warp ? s1.k : s0.k), warp);
-    __syncthreads();
-    for (int s = 0; s < nsel; ++s) {
-      all[s] = sel_bin[s] < 0;
-      if (!all[s]) {
-        prefix[s] = uint32_t(sel_bin[s]);
-        rem[s] = uint32_t(s ? s1.k : s0.k) - sel_above[s];
-        width[s] = 12;
-      }
-    }
-  };
   first_digit(h0, lo_bin >> 3);
   // the bound is valid when at least kbig keys lie above it (or there was none)
-  const bool fast = !any_overflow && (lo_bin == 0 || sel_total[0] >= uint32_t(kbig));
+  fast = !any_overflow && (lo_bin == 0 || sel_total[0] >= uint32_t(kbig));
   if (!fast) {  // count every key from the scores (peers finished reading hs before (2))
     for (int i = tid; i < TK_H12_WORDS; i += TK_THREADS) hs[i] = 0;
     __syncthreads();
@@ -339,6 +374,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
     make_coarse(hs, TK_BINS);
     csync();
     first_digit(hs, 0);
+  }
   }
 
   // ---- pass 1 (bits 19..8) and pass 2 (bits 7..0) over keys matching each prefix, for
