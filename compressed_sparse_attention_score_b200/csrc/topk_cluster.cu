@@ -229,17 +229,17 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
       }
     }
   };
-  // A single-CTA row of at most TK_LIST_WORDS scores is copied once, as keys, into the
+  // A CTA chunk of at most TK_LIST_WORDS scores is copied once, as keys, into the
   // candidate-list space; every pass then reads shared memory instead of the scores.
-  const bool resident = CS == 1 && n <= TK_LIST_WORDS;
-  uint32_t *skeys = tk_smem;
+  const bool resident = chunk <= TK_LIST_WORDS;  // the same in every CTA of the cluster
+  uint32_t *skeys = tk_smem;                      // key of row position j at skeys[j - c0]
   // Keys u = 0 .. U-1 of the group starting at base (lane-strided), -inf past the range.
   auto load_keys = [&](int base, uint32_t (&kk)[U]) {
     if (resident) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int j = base + 32 * u + lane;
-        kk[u] = j < we ? skeys[j] : KEY_NEG_INF;
+        kk[u] = j < we ? skeys[j - c0] : KEY_NEG_INF;
       }
     } else {
       float v[U];
@@ -311,24 +311,24 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   };
   bool fast = false;
   if (resident) {
-    // ---- the whole row into shared memory as keys, then pass 0 over it
-    const float *src = srow;  // one CTA: its range is the whole row
+    // ---- this CTA's chunk into shared memory as keys (c0 is a multiple of 4), then pass 0
     if (vec) {
-      for (int i = 4 * tid; i < n; i += 4 * TK_THREADS) {
-        if (i + 3 < n) {
-          const float4 v = *reinterpret_cast<const float4 *>(src + i);
-          *reinterpret_cast<uint4 *>(skeys + i) = make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
+      for (int i = c0 + 4 * tid; i < c1; i += 4 * TK_THREADS) {
+        if (i + 3 < c1) {
+          const float4 v = *reinterpret_cast<const float4 *>(srow + i);
+          *reinterpret_cast<uint4 *>(skeys + (i - c0)) =
+              make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
         } else {
-          for (int e = i; e < n; ++e) skeys[e] = score_key(src[e]);
+          for (int e = i; e < c1; ++e) skeys[e - c0] = score_key(srow[e]);
         }
       }
     } else {
-      for (int i = tid; i < n; i += TK_THREADS) skeys[i] = score_key(src[i]);
+      for (int i = c0 + tid; i < c1; i += TK_THREADS) skeys[i - c0] = score_key(srow[i]);
     }
     __syncthreads();
     count_pass(hs);
     make_coarse(hs, TK_BINS);
-    __syncthreads();
+    csync();
     first_digit(hs, 0);
   } else {
   // ---- sampled lower bound on the larger selection's threshold (top 12 key bits)
@@ -551,16 +551,18 @@ static int max_active_clusters() {
   return cached[dev];
 }
 
-// Cluster size by row length and count: one CTA per row up to 64K scores or from 148 rows
-// on; otherwise the largest of 16, 12 and 8 CTAs whose clusters all fit on the device at
-// once (a cluster needs its CTAs' SMs in one GPC, so fewer large clusters fit than
-// SMs / CS), 8 up to 256K scores.
+// Cluster size by row length and count.  Rows of at least 2^18 scores: the largest of 16,
+// 12 and 8 CTAs whose clusters all fit on the device at once (a cluster needs its SMs in
+// one GPC, so fewer large clusters fit than SMs / CS).  Shorter rows: about 2048 scores per
+// CTA (then every CTA holds its chunk in shared memory), at most 8 CTAs, as long as all
+// clusters fit at once.  From 148 rows on, or for rows of at most 2048 scores, one CTA per
+// row and no cluster barriers.
 void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int N, int k0, int32_t *idx0, float *val0,
                          int k1, int32_t *idx1, float *val1, const int32_t *map, cudaStream_t st) {
   if (R == 0) return;
   const Sel s0{k0, idx0, val0}, s1{k1, idx1, val1};
   const int nsel = (k1 > 0 && idx1) ? 2 : 1;
-  if (N >= (1 << 18) && R < 148) {
+  if (R < 148 && N >= (1 << 18)) {
     if (max_active_clusters<16>() >= R) {
       launch_cs<16>(scores, n_valid, R, N, s0, s1, nsel, map, st);
     } else if (max_active_clusters<12>() >= R) {
@@ -568,11 +570,18 @@ void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int
     } else {
       launch_cs<8>(scores, n_valid, R, N, s0, s1, nsel, map, st);
     }
-  } else if (N > (1 << 16) && R < 148) {
-    launch_cs<8>(scores, n_valid, R, N, s0, s1, nsel, map, st);
-  } else {
-    // rows up to 64K scores, or enough rows to fill the GPU: one CTA per row, no cluster barriers
-    launch_cs<1>(scores, n_valid, R, N, s0, s1, nsel, map, st);
+    return;
+  }
+  int cs = 1;
+  if (R < 148)
+    while (cs < 8 && cs * 2048 < N && 2 * cs * R <= 148) cs *= 2;
+  if (cs == 8 && max_active_clusters<8>() < R) cs = 4;
+  if (cs == 4 && max_active_clusters<4>() < R) cs = 2;
+  switch (cs) {
+    case 8: launch_cs<8>(scores, n_valid, R, N, s0, s1, nsel, map, st); break;
+    case 4: launch_cs<4>(scores, n_valid, R, N, s0, s1, nsel, map, st); break;
+    case 2: launch_cs<2>(scores, n_valid, R, N, s0, s1, nsel, map, st); break;
+    default: launch_cs<1>(scores, n_valid, R, N, s0, s1, nsel, map, st); break;
   }
 }
 
