@@ -160,7 +160,7 @@ def test_index_score_rejects_bad_candidates():
 
 
 @pytest.mark.parametrize("case", ["random", "ties", "short", "neg_inf", "pool", "long", "zeros", "odd", "unaligned",
-                                  "long_odd", "long8"])
+                                  "long_odd", "long8", "const", "narrow"])
 def test_topk_rows(case):
     k_ = K()
     g = torch.Generator(device="cpu").manual_seed(7)
@@ -185,6 +185,11 @@ def test_topk_rows(case):
     elif case in ("odd", "unaligned"):          # rows the kernel must read one score at a time
         N, k2 = (9003, 1024) if case == "odd" else (9000, 1024)
         s = torch.randn((R, N), generator=g) * 10
+    elif case == "const":                       # every finite score equal: one key, ties by index
+        s = torch.full((R, N), 1.5)
+        s[:, 1::7] = -math.inf
+    elif case == "narrow":                      # scores within 1 % of each other (most key bits shared)
+        s = 1000.0 + torch.rand((R, N), generator=g) * 10.0
     elif case == "long8":                       # more 2^20-entry rows than 16-CTA clusters fit at once
         R, N, k2 = 8, 1 << 20, 16384
         s = torch.randn((R, N), generator=g) * 30
