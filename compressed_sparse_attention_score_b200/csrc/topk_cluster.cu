@@ -53,7 +53,6 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
                                                                      Sel s0, Sel s1, int nsel,
                                                                      const int32_t *__restrict__ map) {
   constexpr int U = 8;        // scalar loads in flight per lane
-  constexpr int UV = 4;       // 16-byte loads in flight per lane in the first full pass
   constexpr int SAMPLE = 16;  // one group of 32 keys in SAMPLE is sampled
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint32_t tk_smem[];
@@ -183,50 +182,49 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   // histogram and, in index order, the warp's candidate list.  Four consecutive keys per
   // lane; stops once the list has overflowed (the caller then counts from the scores).
   int cnt = 0;
+  // Each lane takes 16 consecutive keys of a 512-key group, so that one warp scan of the
+  // lanes' counts places every kept key, in index order, in the warp's list.
   auto keep_pass = [&](int lo_bin, uint32_t *hdst) {
-    for (int base = wb; base < we && cnt <= TK_CAPW; base += 128 * UV) {
-      float4 v[UV];
+    for (int base = wb; base < we && cnt <= TK_CAPW; base += 512) {
+      const int j0 = base + 16 * lane;
+      float f[16];
+      if (vec && j0 + 15 < we) {
 #pragma unroll
-      for (int u = 0; u < UV; ++u) {
-        const int j = base + 128 * u + 4 * lane;
-        if (vec && j + 3 < we) {
-          v[u] = *reinterpret_cast<const float4 *>(srow + j);
-        } else {
-          v[u].x = j < we ? srow[j] : -INFINITY;
-          v[u].y = j + 1 < we ? srow[j + 1] : -INFINITY;
-          v[u].z = j + 2 < we ? srow[j + 2] : -INFINITY;
-          v[u].w = j + 3 < we ? srow[j + 3] : -INFINITY;
+        for (int u = 0; u < 4; ++u) {
+          const float4 v = *reinterpret_cast<const float4 *>(srow + j0 + 4 * u);
+          f[4 * u] = v.x, f[4 * u + 1] = v.y, f[4 * u + 2] = v.z, f[4 * u + 3] = v.w;
         }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) f[e] = j0 + e < we ? srow[j0 + e] : -INFINITY;
       }
+      uint32_t kk[16], tm = 0;
 #pragma unroll
-      for (int u = 0; u < UV; ++u) {
-        const uint32_t kk[4] = {score_key(v[u].x), score_key(v[u].y), score_key(v[u].z), score_key(v[u].w)};
-        bool t[4];
-        int c = 0;
+      for (int e = 0; e < 16; ++e) {
+        kk[e] = score_key(f[e]);
+        if (kk[e] != KEY_NEG_INF && int(kk[e] >> 20) >= lo_bin) tm |= 1u << e;
+      }
+      if (!__any_sync(0xffffffffu, tm != 0)) continue;
+      const int c = __popc(tm);
+      int incl = c;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          t[e] = kk[e] != KEY_NEG_INF && int(kk[e] >> 20) >= lo_bin;
-          c += t[e];
-        }
-        if (__ballot_sync(0xffffffffu, c != 0)) {
-          const uint32_t b0 = __ballot_sync(0xffffffffu, c & 1), b1 = __ballot_sync(0xffffffffu, c & 2),
-                         b2 = __ballot_sync(0xffffffffu, c & 4);
-          int at = cnt + __popc(b0 & lt_mask) + 2 * __popc(b1 & lt_mask) + 4 * __popc(b2 & lt_mask);
-          const int j = base + 128 * u + 4 * lane;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int at = cnt + incl - c;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (t[e]) {
-              atomicAdd(&hdst[kk[e] >> 20], 1u);
-              if (at < TK_CAPW) {
-                ckey[warp][at] = kk[e];
-                cidx[warp][at] = j + e;
-              }
-              ++at;
-            }
+      for (int e = 0; e < 16; ++e) {
+        if (tm & (1u << e)) {
+          atomicAdd(&hdst[kk[e] >> 20], 1u);
+          if (at < TK_CAPW) {
+            ckey[warp][at] = kk[e];
+            cidx[warp][at] = j0 + e;
           }
-          cnt += __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
+          ++at;
         }
       }
+      cnt += __shfl_sync(0xffffffffu, incl, 31);
     }
   };
   // A CTA chunk of at most TK_LIST_WORDS scores is copied once, as keys, into the
@@ -343,9 +341,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const uint32_t key = score_key(v[u]);
-      const bool take = key != KEY_NEG_INF;
-      const uint32_t peers = __match_any_sync(0xffffffffu, take ? (key >> 20) : 0xFFFFFFFFu);
-      if (take && (peers & lt_mask) == 0) atomicAdd(&hs[key >> 20], uint32_t(__popc(peers)));
+      if (key != KEY_NEG_INF) atomicAdd(&hs[key >> 20], 1u);
     }
   }
   make_coarse(hs, TK_BINS);
