@@ -53,7 +53,9 @@ constexpr int SM_STAGES = 0;
 constexpr int SM_B = IM_STAGES * IM_STAGE_BYTES;       // 64 x 64 B query codes
 constexpr int SM_SFB = SM_B + IM_N * 64;                // 512 B scale atom
 constexpr int SM_W = SM_SFB + 512;                      // 64 fp32 head weights
-constexpr int SM_BAR = SM_W + 256;                      // mbarriers
+constexpr int IM_CAND_TILES = 16;                       // candidate lists staged when a CTA has at most this many tiles
+constexpr int SM_CAND = SM_W + 256;                     // [IM_CAND_TILES * 128] candidate entry indices
+constexpr int SM_BAR = SM_CAND + IM_CAND_TILES * IM_TILE * 4;   // mbarriers
 constexpr int N_BARS = 2 * IM_STAGES + 2 * IM_ACC + 1;
 constexpr int SM_MISC = SM_BAR + 8 * N_BARS;            // tmem base, abort flag
 constexpr int SM_TOTAL = SM_MISC + 16;
@@ -95,16 +97,36 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.y, b = row / a.Q;
   const int nvis = visible_entries(a.c, b, a.q_pos[row]);
+  const int n_entries = a.c.num_entries[b];
   const int t_all = (a.n_out + IM_TILE - 1) / IM_TILE;
   const int t_work = a.cand ? (a.P + IM_TILE - 1) / IM_TILE : (nvis + IM_TILE - 1) / IM_TILE;
   const int t0 = blockIdx.x * a.chunk;
   const int t1 = min(t0 + a.chunk, t_all);
   const int ntiles = max(0, min(t1, t_work) - t0);
 
+  // Candidate lists of at most IM_CAND_TILES tiles are copied to shared memory by warp 0
+  // while the other warps run the prologue, so the producer and the epilogue never wait
+  // on a global load of an index.
+  int32_t *cand_s = reinterpret_cast<int32_t *>(smem + SM_CAND);
+  const bool cand_staged = a.cand && ntiles <= IM_CAND_TILES;
+
   // ---------------------------------------------------------------- prologue
   if (warp == 0) {
     tmem_alloc(tmem_slot, IM_TMEM_COLS);
     tmem_relinquish();
+    if (cand_staged) {
+      const int32_t *crow = a.cand + int64_t(row) * a.P;
+      for (int i0 = 0; i0 < ntiles * IM_TILE; i0 += 4 * 32) {
+        int32_t v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int pos = t0 * IM_TILE + i0 + 32 * u + lane;
+          v[u] = pos < a.P ? crow[pos] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) cand_s[i0 + 32 * u + lane] = v[u];
+      }
+    }
   } else if (warp == 1 && lane == 0) {
     for (int s = 0; s < IM_STAGES; ++s) {
       mbar_init(&full[s], a.use_tma ? 1 : 32);  // gather path: one cp.async arrival per producer lane
@@ -200,6 +222,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
           const int pos = tile * IM_TILE + lane + 32 * j;
           if (tile >= t0 + ntiles) cv[j] = -1;
           else if (!a.cand) cv[j] = pos;
+          else if (cand_staged) cv[j] = cand_s[pos - t0 * IM_TILE];
           else cv[j] = pos < a.P ? a.cand[int64_t(row) * a.P + pos] : -1;
         }
       };
@@ -207,7 +230,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int n = cv[j];
-          if (a.cand && (n < -1 || n >= a.c.num_entries[b])) report(a.err, CSA2_ERR_INDEX);
+          if (a.cand && (n < -1 || n >= n_entries)) report(a.err, CSA2_ERR_INDEX);
           int64_t sv = -1;
           if (n >= 0 && n < nvis) {
             sv = cache_slot(a.c, b, n);
@@ -291,7 +314,8 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     auto entry_at = [&](int i) -> int64_t {
       const int pos = (t0 + i) * IM_TILE + e;
       if (!a.cand) return pos;
-      return (i < ntiles && pos < a.P) ? a.cand[int64_t(row) * a.P + pos] : -1;
+      if (i >= ntiles || pos >= a.P) return -1;
+      return cand_staged ? cand_s[pos - t0 * IM_TILE] : a.cand[int64_t(row) * a.P + pos];
     };
     int64_t n_next = entry_at(wg);
     for (int i = wg; i < ntiles; i += IM_EPI_WG) {
