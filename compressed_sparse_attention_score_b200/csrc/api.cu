@@ -87,6 +87,8 @@ CSA2_EXPORT size_t csa2_workspace_size(csa2_mode mode, int32_t B, int32_t Q, int
 CSA2_EXPORT csa2_status csa2_pack_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype, const float *pool_w,
                                      int32_t B, int32_t T, const int32_t *first_entry, const csa2_cache *cache,
                                      int32_t *err, csa2_stream_t stream) {
+  if (B < 0 || T < 0) return fail(CSA2_ERR_INVALID_ARG, "negative size");
+  if (B == 0 || T == 0) return CSA2_OK;
   if (csa2_status s = check_cache(cache, B)) return s;
   if (!lat_kv || !lat_ix || !first_entry) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (dtype != CSA2_F32 && dtype != CSA2_BF16) return fail(CSA2_ERR_INVALID_ARG, "bad dtype");
@@ -99,6 +101,8 @@ CSA2_EXPORT csa2_status csa2_pack_kv(const void *lat_kv, const void *lat_ix, csa
 CSA2_EXPORT csa2_status csa2_pack_swa(const void *x, csa2_dtype dtype, int32_t B, int32_t T, const int32_t *pos,
                                       uint8_t *swa_codes, float *swa_scale, int32_t R, int32_t *err,
                                       csa2_stream_t stream) {
+  if (B < 0 || T < 0 || R < 1) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  if (B == 0 || T == 0) return CSA2_OK;
   if (!x || !pos || !swa_codes || !swa_scale) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (dtype != CSA2_F32 && dtype != CSA2_BF16) return fail(CSA2_ERR_INVALID_ARG, "bad dtype");
   if (B < 0 || T < 0 || R < 1) return fail(CSA2_ERR_INVALID_ARG, "bad size");
@@ -111,6 +115,8 @@ CSA2_EXPORT csa2_status csa2_index_score(const uint16_t *q_ix, const uint16_t *w
                                          const int32_t *q_pos, const int32_t *cand, int32_t P, int32_t max_entries,
                                          const csa2_cache *cache, float *scores, int32_t *err,
                                          csa2_stream_t stream) {
+  if (B < 0 || Q < 0 || max_entries < 0 || (cand && P <= 0)) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  if (B == 0 || Q == 0) return CSA2_OK;
   if (csa2_status s = check_cache(cache, B)) return s;
   if (!q_ix || !w || !q_pos || !scores) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (B < 0 || Q < 0 || max_entries < 0 || (cand && P <= 0)) return fail(CSA2_ERR_INVALID_ARG, "bad size");
@@ -124,6 +130,8 @@ CSA2_EXPORT csa2_status csa2_index_score(const uint16_t *q_ix, const uint16_t *w
 CSA2_EXPORT csa2_status csa2_topk(const float *scores, const int32_t *n_valid, int32_t R, int32_t N, int32_t k,
                                   int32_t *idx, float *val, int32_t k2, int32_t *idx2, float *val2,
                                   csa2_stream_t stream) {
+  if (R < 0 || N < 0 || k < 1 || k2 < 0) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  if (R == 0) return CSA2_OK;
   if (!scores || !idx) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (R < 0 || N < 0 || k < 1 || k2 < 0 || (k2 > 0 && !idx2)) return fail(CSA2_ERR_INVALID_ARG, "bad size");
   if (int64_t(R) * 16 > INT32_MAX) return fail(CSA2_ERR_UNSUPPORTED, "too many rows");
@@ -138,6 +146,8 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
                                          const csa2_cache *cache, const uint8_t *swa_codes, const float *swa_scale,
                                          int32_t R, int32_t window, float *o, float *lse, void *ws, size_t ws_bytes,
                                          int32_t *err, csa2_stream_t stream) {
+  if (B < 0 || Q < 0 || k < 1 || pool_k < 0 || max_entries < 0) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  if (B == 0 || Q == 0) return CSA2_OK;
   if (csa2_status s = check_cache(cache, B)) return s;
   if (!q || !q_pos || !o || !lse) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (B < 0 || Q < 0 || k < 1 || pool_k < 0 || max_entries < 0) return fail(CSA2_ERR_INVALID_ARG, "bad size");
@@ -185,6 +195,8 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
 CSA2_EXPORT csa2_status csa2_swa_attn(const uint16_t *q, int32_t B, int32_t Q, const int32_t *q_pos,
                                       const uint8_t *swa_codes, const float *swa_scale, int32_t R, int32_t window,
                                       float softmax_scale, float *o, float *lse, int32_t *err, csa2_stream_t stream) {
+  if (B < 0 || Q < 0 || window < 1 || R < window) return fail(CSA2_ERR_INVALID_ARG, "need 1 <= window <= R");
+  if (B == 0 || Q == 0) return CSA2_OK;
   if (!q || !q_pos || !swa_codes || !swa_scale || !o || !lse) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (B < 0 || Q < 0 || window < 1 || R < window) return fail(CSA2_ERR_INVALID_ARG, "need 1 <= window <= R");
   if (window > 128) return fail(CSA2_ERR_UNSUPPORTED, "window > 128");
@@ -197,6 +209,8 @@ CSA2_EXPORT csa2_status csa2_swa_attn(const uint16_t *q, int32_t B, int32_t Q, c
 
 CSA2_EXPORT csa2_status csa2_merge(const float *o1, const float *l1, const float *o2, const float *l2, int64_t rows,
                                    int32_t D, float *o, float *lse, csa2_stream_t stream) {
+  if (rows < 0 || D < 4 || (D & 3)) return fail(CSA2_ERR_INVALID_ARG, "D must be a positive multiple of 4");
+  if (rows == 0) return CSA2_OK;
   if (!o1 || !l1 || !o2 || !l2 || !o || !lse) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (rows < 0 || D < 4 || (D & 3)) return fail(CSA2_ERR_INVALID_ARG, "D must be a positive multiple of 4");
   if (!aligned16(o1) || !aligned16(o2) || !aligned16(o)) return fail(CSA2_ERR_INVALID_ARG, "o misaligned");

@@ -22,6 +22,8 @@
  *  - Errors found on the device (an index or page outside the cache) never trap:
  *    the kernel skips the bad access and stores the status code into *err (a
  *    caller-owned device int32, first error wins), read back by csa2_check().
+ *  - A call with no work (a batch, token, row or query count of 0) returns CSA2_OK
+ *    without reading any pointer or launching anything; negative sizes are errors.
  *  - bf16 tensors are passed as `const uint16_t*` (raw bf16 bits).
  *  - Fixed dimensions: main-KV and query head dim 512, indexer dim 128,
  *    query heads H = 64, indexer heads H_I = 64.

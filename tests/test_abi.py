@@ -84,3 +84,18 @@ def test_host_side_argument_checks(lib):
     assert lib.csa2_sparse_attn(0, addr, 1, 1, addr, 1.0, addr, addr, 512, 0, None, None, None, 16,
                                 ctypes.byref(c), None, None, 0, 0, addr, addr, None, 0, None, None) == 1
     assert b"workspace" in lib.csa2_last_error_string()
+
+
+def test_zero_work_calls_are_no_ops(lib):
+    # nothing to do: CSA2_OK without reading any pointer (all NULL here) and without a launch
+    assert lib.csa2_pack_kv(None, None, 0, None, 0, 5, None, None, None, None) == 0
+    assert lib.csa2_pack_swa(None, 0, 3, 0, None, None, None, 128, None, None) == 0
+    assert lib.csa2_index_score(None, None, 0, 1, None, None, 0, 16, None, None, None, None) == 0
+    assert lib.csa2_topk(None, None, 0, 10, 5, None, None, 0, None, None, None) == 0
+    assert lib.csa2_sparse_attn(2, None, 0, 1, None, 1.0, None, None, 512, 0, None, None, None, 16,
+                                None, None, None, 0, 0, None, None, None, 0, None, None) == 0
+    assert lib.csa2_swa_attn(None, 0, 1, None, None, None, 128, 128, 1.0, None, None, None, None) == 0
+    assert lib.csa2_merge(None, None, None, None, 0, 512, None, None, None) == 0
+    # negative sizes are still errors
+    assert lib.csa2_topk(None, None, -1, 10, 5, None, None, 0, None, None, None) == 1
+    assert lib.csa2_merge(None, None, None, None, -1, 512, None, None, None) == 1

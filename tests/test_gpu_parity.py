@@ -248,6 +248,34 @@ def test_swa_attention_and_sequence_start():
         check_attention(to_np(o[b, 0]), to_np(lse[b, 0]), oo, ol, f"swa b={b}")
 
 
+def test_empty_batches_are_no_ops():
+    """Zero sequences, tokens or rows: every entry point returns without touching anything."""
+    k = K()
+    spec = W.scaled(W.tiny_full(), [600], B=1)
+    cache = gpu_cache(spec)
+    q, q_ix, w, q_pos = W.query_tensors(spec, 0, DEV)
+    x, pos = W.swa_tokens(spec, 0, DEV)
+    codes = torch.zeros((1, 128, 512), dtype=torch.uint8, device=DEV)
+    scale = torch.zeros((1, 128), dtype=torch.float32, device=DEV)
+    err = _err()
+    kv, ix = W.token_latents(spec, 0, DEV)
+    k.csa2_pack_kv(kv[None, :0].contiguous(), ix[None, :0].contiguous(), torch.zeros(1, dtype=torch.int32, device=DEV),
+                   cache.seq_view(0), err=err)
+    k.csa2_pack_swa(x[:, :0], pos[:, :0], codes, scale, err=err)
+    assert int(codes.count_nonzero()) == 0 and int(scale.count_nonzero()) == 0
+    sc = k.csa2_index_score(q_ix[:0], w[:0], q_pos[:0], cache, spec.max_entries, err=err)
+    assert sc.numel() == 0
+    idx = k.csa2_topk(torch.empty((0, 1000), device=DEV), 16)[0]
+    assert idx.numel() == 0
+    o, lse = k.csa2_sparse_attn("full", q[:0], q_pos[:0], cache, spec.tau, spec.max_entries, q_ix=q_ix[:0], w=w[:0],
+                                err=err)
+    assert o.numel() == 0 and lse.numel() == 0
+    o2, l2 = k.csa2_swa_attn(q[:0], q_pos[:0], codes, scale, spec.tau, err=err)
+    om, lm = k.csa2_merge(o2, l2, o2, l2)
+    assert om.numel() == 0 and lm.numel() == 0
+    assert k.csa2_check(err) == 0
+
+
 def test_merge_matches_oracle_and_aliases():
     k = K()
     rows = 3 * 64
