@@ -412,7 +412,8 @@ void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int 
   if (n_out == 0 || rows == 0) return;
   const int t_all = (n_out + IM_TILE - 1) / IM_TILE;
   const int want = (2 * 148 + rows - 1) / rows;           // about two CTAs per SM in total
-  const int splits = max(1, min(min(want, (t_all + 7) / 8), 65535));
+  const int min_tiles = cand ? 4 : 8;                     // short candidate lists: spread them wider
+  const int splits = max(1, min(min(want, (t_all + min_tiles - 1) / min_tiles), 65535));
   const int chunk = (t_all + splits - 1) / splits;
   CUtensorMap tmap;
   memset(&tmap, 0, sizeof(tmap));
