@@ -549,9 +549,9 @@ static int max_active_clusters() {
 
 // Cluster size by row length and count.  Rows of at least 2^18 scores: the largest of 16,
 // 12 and 8 CTAs whose clusters all fit on the device at once (a cluster needs its SMs in
-// one GPC, so fewer large clusters fit than SMs / CS).  Shorter rows: about 2048 scores per
+// one GPC, so fewer large clusters fit than SMs / CS).  Shorter rows: about 4096 scores per
 // CTA (then every CTA holds its chunk in shared memory), at most 8 CTAs, as long as all
-// clusters fit at once.  From 148 rows on, or for rows of at most 2048 scores, one CTA per
+// clusters fit at once.  From 148 rows on, or for rows of at most 4096 scores, one CTA per
 // row and no cluster barriers.
 void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int N, int k0, int32_t *idx0, float *val0,
                          int k1, int32_t *idx1, float *val1, const int32_t *map, cudaStream_t st) {
@@ -570,7 +570,7 @@ void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int
   }
   int cs = 1;
   if (R < 148)
-    while (cs < 8 && cs * 2048 < N && 2 * cs * R <= 148) cs *= 2;
+    while (cs < 8 && cs * 4096 < N && 2 * cs * R <= 148) cs *= 2;
   if (cs == 8 && max_active_clusters<8>() < R) cs = 4;
   if (cs == 4 && max_active_clusters<4>() < R) cs = 2;
   switch (cs) {
