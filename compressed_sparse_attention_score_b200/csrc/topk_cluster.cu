@@ -548,7 +548,7 @@ static int max_active_clusters() {
 }
 
 // Cluster size by row length and count.  Rows of at least 2^18 scores: the largest of 16,
-// 12 and 8 CTAs whose clusters all fit on the device at once (a cluster needs its SMs in
+// 12, 10 and 8 CTAs whose clusters all fit on the device at once (a cluster needs its SMs in
 // one GPC, so fewer large clusters fit than SMs / CS).  Shorter rows: about 4096 scores per
 // CTA (then every CTA holds its chunk in shared memory), at most 8 CTAs, as long as all
 // clusters fit at once.  From 148 rows on, or for rows of at most 4096 scores, one CTA per
@@ -563,6 +563,8 @@ void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int
       launch_cs<16>(scores, n_valid, R, N, s0, s1, nsel, map, st);
     } else if (max_active_clusters<12>() >= R) {
       launch_cs<12>(scores, n_valid, R, N, s0, s1, nsel, map, st);
+    } else if (max_active_clusters<10>() >= R) {
+      launch_cs<10>(scores, n_valid, R, N, s0, s1, nsel, map, st);
     } else {
       launch_cs<8>(scores, n_valid, R, N, s0, s1, nsel, map, st);
     }
