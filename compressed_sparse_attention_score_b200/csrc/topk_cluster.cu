@@ -11,10 +11,13 @@
 // coarse bin that holds the threshold and then sums only the 8 fine bins inside it,
 // so a stage costs one barrier and no CTA ever writes into a histogram a peer reads.
 // A sample of the keys first bounds the larger selection from below; the first full
-// pass counts only keys above the bound and appends them, in index order, to per-warp
-// candidate lists, and the later passes walk the lists (or the scores again if the
-// bound was too high or a list overflowed).  Up to two selections (e.g. top-512 and a
-// 16384-entry pool) are refined in the same passes.  A counting pass and a
+// pass (each lane 16 consecutive keys, one warp scan to place them) counts only keys
+// above the bound and appends them, in index order, to per-warp candidate lists, and
+// the later passes walk the lists (or the scores again if the bound was too high or a
+// list overflowed).  A CTA whose chunk fits in shared memory instead copies it there
+// once as keys and every pass reads it there.  Refinement stops as soon as the
+// threshold's prefix bin holds exactly the keys still needed.  Up to two selections
+// (e.g. top-512 and a 16384-entry pool) are refined in the same passes.  A counting pass and a
 // cluster-wide exclusive prefix (each CTA pushes its totals into every peer) give
 // every thread its output offset, and the writing pass emits the chosen positions in
 // ascending order (ties: lower position first), padded with -1.
