@@ -17,7 +17,9 @@
 // Phase 3  O^T[dim][head] = V^T P^T per 128-dim tile (M = 128 dims, N = 32 heads,
 //          K = keys in 16-key steps), V^T chunks MN-major with 128-byte swizzle,
 //          accumulated in TMEM.
-// Phase 4  O / sum and lse = max + log(sum), coalesced fp32 stores.
+// Phase 4  O / sum and lse = max + log(sum), coalesced fp32 stores; when a cluster of
+//          CTAs splits the row's keys, the partials (O, max, sum) are combined over
+//          distributed shared memory, each CTA producing one slice of the 512 dims.
 // A tile's raw key bytes (288 B per listed entry, 512 B per window token) are
 // gathered once into shared memory with asynchronous 16-byte copies, all in flight
 // together; both products dequantise from there, so a CTA whose keys fit one tile
