@@ -160,7 +160,7 @@ def test_index_score_rejects_bad_candidates():
 
 
 @pytest.mark.parametrize("case", ["random", "ties", "short", "neg_inf", "pool", "long", "zeros", "odd", "unaligned",
-                                  "long_odd", "long8", "const", "narrow"])
+                                  "long_odd", "long8", "const", "narrow", "mid"])
 def test_topk_rows(case):
     k_ = K()
     g = torch.Generator(device="cpu").manual_seed(7)
@@ -185,6 +185,9 @@ def test_topk_rows(case):
     elif case in ("odd", "unaligned"):          # rows the kernel must read one score at a time
         N, k2 = (9003, 1024) if case == "odd" else (9000, 1024)
         s = torch.randn((R, N), generator=g) * 10
+    elif case == "mid":                         # 8-CTA clusters whose chunks exceed shared memory
+        N, k2 = 200000, 16384
+        s = torch.randn((R, N), generator=g) * 20
     elif case == "const":                       # every finite score equal: one key, ties by index
         s = torch.full((R, N), 1.5)
         s[:, 1::7] = -math.inf
