@@ -19,7 +19,7 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-MODE = {"full": 0, "reindex": 1, "reuse": 2}
+MODE = {"full": 0, "reindex": 1, "reuse": 2, "dense": 3}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "UNSUPPORTED", 4: "CUDA", 5: "INDEX", 6: "TIMEOUT"}
 

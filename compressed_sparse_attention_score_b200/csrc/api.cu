@@ -50,6 +50,10 @@ csa2_status check_cache(const csa2_cache *c, int B) {
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Dense attention runs over segments of csa2::attn_dense_segment() entries (8192, or 4096 on a
+// device that cannot hold a 16-CTA cluster); the workspace is sized for the smaller.
+constexpr int kDenseMinSegment = 4096;
+
 }  // namespace
 
 namespace csa2 {
@@ -80,6 +84,10 @@ CSA2_EXPORT size_t csa2_workspace_size(csa2_mode mode, int32_t B, int32_t Q, int
   switch (mode) {
     case CSA2_MODE_FULL: return round256(rows * max_entries * 4) + round256(rows * k * 4);
     case CSA2_MODE_REINDEX: return round256(rows * pool_k * 4) + round256(rows * k * 4);
+    case CSA2_MODE_DENSE:  // partial (o, lse) of one key segment beyond the first
+      return max_entries > kDenseMinSegment ? round256(rows * CSA2_HEADS * CSA2_MAIN_DIM * 4) +
+                                                  round256(rows * CSA2_HEADS * 4)
+                                            : 0;
     default: return 0;
   }
 }
@@ -92,7 +100,6 @@ CSA2_EXPORT csa2_status csa2_pack_kv(const void *lat_kv, const void *lat_ix, csa
   if (csa2_status s = check_cache(cache, B)) return s;
   if (!lat_kv || !lat_ix || !first_entry) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (dtype != CSA2_F32 && dtype != CSA2_BF16) return fail(CSA2_ERR_INVALID_ARG, "bad dtype");
-  if (B < 0 || T < 0) return fail(CSA2_ERR_INVALID_ARG, "negative size");
   if (!aligned16(lat_kv) || (reinterpret_cast<uintptr_t>(lat_ix) & 7)) return fail(CSA2_ERR_INVALID_ARG, "latents misaligned");
   csa2::launch_pack_kv(lat_kv, lat_ix, dtype, pool_w, B, T, first_entry, *cache, err, stream);
   return launched("csa2_pack_kv");
@@ -105,7 +112,6 @@ CSA2_EXPORT csa2_status csa2_pack_swa(const void *x, csa2_dtype dtype, int32_t B
   if (B == 0 || T == 0) return CSA2_OK;
   if (!x || !pos || !swa_codes || !swa_scale) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (dtype != CSA2_F32 && dtype != CSA2_BF16) return fail(CSA2_ERR_INVALID_ARG, "bad dtype");
-  if (B < 0 || T < 0 || R < 1) return fail(CSA2_ERR_INVALID_ARG, "bad size");
   if (!aligned16(x) || !aligned16(swa_codes)) return fail(CSA2_ERR_INVALID_ARG, "x / swa_codes misaligned");
   csa2::launch_pack_swa(x, dtype, B, T, pos, swa_codes, swa_scale, R, err, stream);
   return launched("csa2_pack_swa");
@@ -119,7 +125,6 @@ CSA2_EXPORT csa2_status csa2_index_score(const uint16_t *q_ix, const uint16_t *w
   if (B == 0 || Q == 0) return CSA2_OK;
   if (csa2_status s = check_cache(cache, B)) return s;
   if (!q_ix || !w || !q_pos || !scores) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
-  if (B < 0 || Q < 0 || max_entries < 0 || (cand && P <= 0)) return fail(CSA2_ERR_INVALID_ARG, "bad size");
   if (!aligned16(q_ix)) return fail(CSA2_ERR_INVALID_ARG, "q_ix misaligned");
   const int n_out = cand ? P : max_entries;
   if (size_t(B) * Q > 65535) return fail(CSA2_ERR_UNSUPPORTED, "more than 65535 query rows per call");
@@ -133,7 +138,7 @@ CSA2_EXPORT csa2_status csa2_topk(const float *scores, const int32_t *n_valid, i
   if (R < 0 || N < 0 || k < 1 || k2 < 0) return fail(CSA2_ERR_INVALID_ARG, "bad size");
   if (R == 0) return CSA2_OK;
   if (!scores || !idx) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
-  if (R < 0 || N < 0 || k < 1 || k2 < 0 || (k2 > 0 && !idx2)) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  if (k2 > 0 && !idx2) return fail(CSA2_ERR_INVALID_ARG, "k2 > 0 needs idx2");
   if (int64_t(R) * 16 > INT32_MAX) return fail(CSA2_ERR_UNSUPPORTED, "too many rows");
   csa2::launch_topk_cluster(scores, n_valid, R, N, k, idx, val, k2, k2 > 0 ? idx2 : nullptr, val2, nullptr, stream);
   return launched("csa2_topk");
@@ -150,16 +155,34 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
   if (B == 0 || Q == 0) return CSA2_OK;
   if (csa2_status s = check_cache(cache, B)) return s;
   if (!q || !q_pos || !o || !lse) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
-  if (B < 0 || Q < 0 || k < 1 || pool_k < 0 || max_entries < 0) return fail(CSA2_ERR_INVALID_ARG, "bad size");
-  if (k > 512) return fail(CSA2_ERR_UNSUPPORTED, "k > 512");
+  if (k > 512 && mode != CSA2_MODE_DENSE) return fail(CSA2_ERR_UNSUPPORTED, "k > 512");
   if (!aligned16(q)) return fail(CSA2_ERR_INVALID_ARG, "q misaligned");
   if (swa_codes) {
     if (!swa_scale || window < 1 || window > 128 || R < window) return fail(CSA2_ERR_INVALID_ARG, "need 1 <= window <= 128, window <= R");
     if (!aligned16(swa_codes)) return fail(CSA2_ERR_INVALID_ARG, "swa_codes misaligned");
   }
+  if (int64_t(B) * Q > 65535 * 16) return fail(CSA2_ERR_UNSUPPORTED, "too many query rows per call");
   const int rows = B * Q;
-  if (rows > 65535 * 16) return fail(CSA2_ERR_UNSUPPORTED, "too many query rows per call");
   const int32_t *idx = nullptr;
+  if (mode == CSA2_MODE_DENSE) {
+    // every visible entry, in segments of at most `seg` entries; the partials of the segments
+    // after the first go through the workspace and are merged into o / lse in place
+    const int seg = csa2::attn_dense_segment();
+    if (max_entries > seg) {
+      if (!ws || ws_bytes < csa2_workspace_size(mode, B, Q, max_entries, k, pool_k))
+        return fail(CSA2_ERR_INVALID_ARG, "workspace too small");
+    }
+    float *po = static_cast<float *>(ws);
+    float *pl = reinterpret_cast<float *>(static_cast<char *>(ws) + round256(size_t(rows) * CSA2_HEADS * CSA2_MAIN_DIM * 4));
+    for (int s = 0, e0 = 0; s == 0 || e0 < max_entries; ++s, e0 += seg) {
+      const int e1 = e0 + seg < max_entries ? e0 + seg : max_entries;
+      csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, nullptr, 0, true, e0, e1, max_entries, cache,
+                            s == 0 ? swa_codes : nullptr, s == 0 && swa_codes ? swa_scale : nullptr, R, window,
+                            s == 0 ? o : po, s == 0 ? lse : pl, err, stream);
+      if (s > 0) csa2::launch_merge(o, lse, po, pl, int64_t(rows) * CSA2_HEADS, CSA2_MAIN_DIM, o, lse, stream);
+    }
+    return launched("csa2_sparse_attn");
+  }
   if (mode == CSA2_MODE_REUSE) {
     if (!idx_in) return fail(CSA2_ERR_INVALID_ARG, "REUSE needs idx_in");
     idx = idx_in;
@@ -187,8 +210,8 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
   } else {
     return fail(CSA2_ERR_INVALID_ARG, "bad mode");
   }
-  csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, idx, k, cache, swa_codes, swa_codes ? swa_scale : nullptr, R,
-                        window, o, lse, err, stream);
+  csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, idx, k, false, 0, 0, 0, cache, swa_codes,
+                        swa_codes ? swa_scale : nullptr, R, window, o, lse, err, stream);
   return launched("csa2_sparse_attn");
 }
 
@@ -198,12 +221,11 @@ CSA2_EXPORT csa2_status csa2_swa_attn(const uint16_t *q, int32_t B, int32_t Q, c
   if (B < 0 || Q < 0 || window < 1 || R < window) return fail(CSA2_ERR_INVALID_ARG, "need 1 <= window <= R");
   if (B == 0 || Q == 0) return CSA2_OK;
   if (!q || !q_pos || !swa_codes || !swa_scale || !o || !lse) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
-  if (B < 0 || Q < 0 || window < 1 || R < window) return fail(CSA2_ERR_INVALID_ARG, "need 1 <= window <= R");
   if (window > 128) return fail(CSA2_ERR_UNSUPPORTED, "window > 128");
   if (!aligned16(swa_codes) || !aligned16(q)) return fail(CSA2_ERR_INVALID_ARG, "swa_codes / q misaligned");
-  if (B * Q > 65535 * 16) return fail(CSA2_ERR_UNSUPPORTED, "too many query rows per call");
-  csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, nullptr, 0, nullptr, swa_codes, swa_scale, R, window, o, lse,
-                        err, stream);
+  if (int64_t(B) * Q > 65535 * 16) return fail(CSA2_ERR_UNSUPPORTED, "too many query rows per call");
+  csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, nullptr, 0, false, 0, 0, 0, nullptr, swa_codes, swa_scale, R,
+                        window, o, lse, err, stream);
   return launched("csa2_swa_attn");
 }
 
@@ -212,7 +234,6 @@ CSA2_EXPORT csa2_status csa2_merge(const float *o1, const float *l1, const float
   if (rows < 0 || D < 4 || (D & 3)) return fail(CSA2_ERR_INVALID_ARG, "D must be a positive multiple of 4");
   if (rows == 0) return CSA2_OK;
   if (!o1 || !l1 || !o2 || !l2 || !o || !lse) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
-  if (rows < 0 || D < 4 || (D & 3)) return fail(CSA2_ERR_INVALID_ARG, "D must be a positive multiple of 4");
   if (!aligned16(o1) || !aligned16(o2) || !aligned16(o)) return fail(CSA2_ERR_INVALID_ARG, "o misaligned");
   csa2::launch_merge(o1, l1, o2, l2, rows, D, o, lse, stream);
   return launched("csa2_merge");

@@ -4,10 +4,13 @@
 // CTA = one query row x 32 heads.  Each key's 512-d vector is both key and value.
 // Keys come from two sources that share one softmax (so a CTA given both returns
 // the log-sum-exp merge of the two branches exactly):
-//   sparse  -- listed main-KV entries: e2m1 x E4M3-per-16 dequantised to fp16
-//              (exact: <= 6 significant bits, in fp16 range);
+//   sparse  -- listed main-KV entries (or, dense, every visible entry of a range):
+//              e2m1 x E4M3-per-16 dequantised to fp16 (exact: <= 6 significant
+//              bits, in fp16 range);
 //   window  -- SWA tokens: E4M3 codes to fp16 (exact); the token's fp32 scale is
 //              folded into the logit multiplier and into P.
+// The bf16 query heads enter the MMA prescaled by a power of two per head (see
+// store_query_fp16), so they are exact in fp16 whatever their magnitude.
 // Phase 1  S^T[key][head] = K Q^T per 128-key tile (M = 128 keys, N = 32 heads,
 //          K = 512 dims in 64-dim chunks, 128-byte swizzled K-major operands),
 //          all tiles resident in TMEM.
@@ -57,9 +60,12 @@ constexpr int SM_RAW = SM_STG + AM_STAGES * AM_STAGE;   // one tile of raw keys
 constexpr int SM_SLOT = SM_RAW + AM_TILE * AM_RAW;
 constexpr int SM_MU = SM_SLOT + AM_MAXKEYS * 8;      // logit multiplier per key
 constexpr int SM_PV = SM_MU + AM_MAXKEYS * 4;        // P multiplier per key
+constexpr int AM_MAXCS = 16;      // largest cluster splitting one row's keys
+constexpr int AM_QU = AM_HG * (D / 8) / AM_PRODUCERS;   // 16-byte query chunks per producer thread
 constexpr int SM_RED = SM_PV + AM_MAXKEYS * 4;       // [4 warps][32 heads]; [CS][32] weights + [32] sums
-constexpr int SM_HM = SM_RED + 8 * 32 * 4;           // head max [32], head sum [32]
-constexpr int SM_BAR = SM_HM + 2 * 32 * 4;
+constexpr int SM_HM = SM_RED + (AM_MAXCS + 1) * 32 * 4;   // head max [32], head sum [32]
+constexpr int SM_QS = SM_HM + 2 * 32 * 4;            // query prescale: [8 warps][AM_QU] max bits, [32] 2^-s
+constexpr int SM_BAR = SM_QS + (8 * AM_QU + 32) * 4;
 constexpr int SM_MISC = SM_BAR + 8 * (2 * AM_STAGES + 1);
 constexpr int SM_TOTAL = SM_MISC + 16;
 constexpr size_t AM_SMEM = SM_TOTAL + 1024;
@@ -70,9 +76,12 @@ struct AttnArgs {
   int Q;
   const int32_t *q_pos;
   float tau;
-  // sparse source (idx == nullptr: none)
+  // sparse source: the k listed entries idx (idx == nullptr: none), or with dense != 0
+  // every visible entry n in [e0, e1)
   const int32_t *idx;
   int k;
+  int dense, e0, e1;
+  int n_bound;  // dense: entries a query may see (more sets CSA2_ERR_SHAPE)
   csa2_cache c;
   // window source (codes == nullptr: none)
   const uint8_t *codes;
@@ -91,6 +100,57 @@ __device__ __forceinline__ int mnmaj128(int k, int mblk, int u) {
 }
 // MN-major, 64-byte swizzle (P^T): K-row k (key), unit u of 8 heads.
 __device__ __forceinline__ int mnmaj64(int k, int u) { return (k >> 3) * 512 + (k & 7) * 64 + ((u ^ ((k & 7) >> 1)) << 4); }
+
+// Query prescale.  The query heads enter the fp16 MMA multiplied by a power of two 2^s per
+// head that puts the head's largest |q| in [2^14, 2^15): every bf16 value within a factor
+// 2^32 of that maximum is then exact in fp16 (no overflow above 65504, no lost bits in the
+// subnormals), and the logits are multiplied back by 2^-s, which is exact in fp32.
+// Producer thread tid holds query chunks it = tid + 256 u, i.e. head tid / 64 + 4 u, so the
+// two warps 2c, 2c + 1 share the heads c + 4 u.  Each warp publishes the largest |bf16| bit
+// pattern of each of its AM_QU chunks' heads (|x| orders like its bits).
+__device__ __forceinline__ void publish_query_max(const uint4 (&qraw)[AM_QU], uint32_t *qmx) {
+  const int warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int u = 0; u < AM_QU; ++u) {
+    const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
+    uint32_t mb = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mb = max(mb, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+    mb = __reduce_max_sync(0xffffffffu, mb);
+    if ((threadIdx.x & 31) == 0) qmx[warp * AM_QU + u] = mb;
+  }
+}
+// Exponent s of the prescale of a head whose largest |bf16| bit pattern is mb (0 for an all-zero
+// or non-finite head).  floor(log2 max) = E - 127 for the biased exponent E.
+__device__ __forceinline__ int query_prescale_exp(uint32_t mb) {
+  const int E = int(mb >> 7);
+  if (mb == 0 || E >= 255) return 0;
+  return min(126, 141 - max(E, 1));
+}
+__device__ __forceinline__ uint32_t head_max_bits(const uint32_t *qmx, int h) {
+  const int c = h & 3, u = h >> 2;
+  return max(qmx[(2 * c) * AM_QU + u], qmx[(2 * c + 1) * AM_QU + u]);
+}
+// Write this producer's query chunks, prescaled, as fp16 into the K-major 128-byte-swizzled
+// Q operand (8 chunks of 64 dims x 32 heads); thread tid < 32 also stores 2^-s of head tid.
+__device__ __forceinline__ void store_query_fp16(const uint4 (&qraw)[AM_QU], const uint32_t *qmx, float *qinv,
+                                                 uint8_t *qdst) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int u = 0; u < AM_QU; ++u) {
+    const int it = tid + u * AM_PRODUCERS, h = it / (D / 8), u8 = it % (D / 8);
+    const float sc = pow2f(query_prescale_exp(head_max_bits(qmx, h)));
+    const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
+    uint32_t o4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 hv = __floats2half2_rn(__uint_as_float(w[i] << 16) * sc, __uint_as_float(w[i] & 0xFFFF0000u) * sc);
+      o4[i] = *reinterpret_cast<const uint32_t *>(&hv);
+    }
+    *reinterpret_cast<uint4 *>(qdst + (u8 / 8) * 4096 + kmaj128(h, u8 % 8)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+  }
+  if (tid < 32) qinv[tid] = pow2f(-query_prescale_exp(head_max_bits(qmx, tid)));
+}
 
 // Gather the raw bytes of local key tile t into shared memory (asynchronous 16-byte
 // copies by the producer threads, committed as one group): a listed entry's 256 code bytes and 32 scale bytes
@@ -273,7 +333,8 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   const int pos = p.q_pos[row];
 
   // ---------------------------------------------------------------- key list
-  const int nks = p.idx ? p.k : 0;
+  const int nvis = (p.idx || p.dense) ? visible_entries(p.c, b, pos) : 0;
+  const int nks = p.dense ? max(0, min(p.e1, nvis) - p.e0) : (p.idx ? p.k : 0);
   int lo = 0, nkw = 0;
   if (p.codes && pos >= 0) {
     lo = max(0, pos - p.window + 1);
@@ -285,16 +346,19 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   const int tiles_all = (nk + AM_TILE - 1) / AM_TILE;
   const int tps = (tiles_all + CS - 1) / CS;
   const int tile0 = min(tiles_all, split * tps);
-  const int ntiles = min(tiles_all, tile0 + tps) - tile0;
+  // a CTA holds at most AM_MAXKEYS keys (the launcher sizes the cluster for that); keys past
+  // them, or dense entries past the caller's bound, are left out and reported
+  const int ntiles = min(min(tiles_all, tile0 + tps) - tile0, AM_MAXKEYS / AM_TILE);
+  if (tid == 0 && (tps > AM_MAXKEYS / AM_TILE || (p.dense && nvis > p.n_bound))) report(p.err, CSA2_ERR_SHAPE);
   const int key0 = tile0 * AM_TILE;  // first key of this CTA; local key j is key key0 + j
-  const int nvis = p.idx ? visible_entries(p.c, b, pos) : 0;
   // the query block's loads go out first; they are converted once the key list is done
-  constexpr int QU = AM_HG * (D / 8) / AM_PRODUCERS;
-  uint4 qraw[QU];
+  uint32_t *qmx = reinterpret_cast<uint32_t *>(smem + SM_QS);
+  float *qinv = reinterpret_cast<float *>(smem + SM_QS + 8 * AM_QU * 4);
+  uint4 qraw[AM_QU];
   if (producer) {
     const uint16_t *qrow = p.q + (int64_t(row) * H + hg * AM_HG) * D;
 #pragma unroll
-    for (int u = 0; u < QU; ++u) {
+    for (int u = 0; u < AM_QU; ++u) {
       const int it = tid + u * AM_PRODUCERS;
       qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
     }
@@ -304,7 +368,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     int64_t s = -1;
     float m = 0.f, pm = 0.f;
     if (j < nks) {
-      const int n = p.idx[int64_t(row) * p.k + j];
+      const int n = p.dense ? p.e0 + j : p.idx[int64_t(row) * p.k + j];
       if (n != -1) {
         if (n < -1 || n >= nvis) {
           report(p.err, CSA2_ERR_INDEX);
@@ -323,6 +387,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     mu[jl] = m;
     pv[jl] = pm;
   }
+  if (producer) publish_query_max(qraw, qmx);
   if (warp == AM_PRODUCERS / 32) {
     tmem_alloc(tmem_slot, AM_TMEM_COLS);
     tmem_relinquish();
@@ -336,23 +401,11 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     *abort_flag = 0;
     mbar_init_fence();
   }
-  __syncthreads();  // key list and barriers ready
+  __syncthreads();  // key list, query maxima and barriers ready
   const uint32_t raw = smem_u32(smem + SM_RAW);
   if (producer) {
     if (ntiles > 0) gather_tile(p, slot, nks, key0, 0, raw);
-#pragma unroll
-    for (int u = 0; u < QU; ++u) {
-      const int it = tid + u * AM_PRODUCERS, h = it / (D / 8), u8 = it % (D / 8);
-      const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
-      uint32_t o4[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const __half2 hv = __floats2half2_rn(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-        o4[i] = *reinterpret_cast<const uint32_t *>(&hv);
-      }
-      *reinterpret_cast<uint4 *>(smem + SM_Q + (u8 / 8) * 4096 + kmaj128(h, u8 % 8)) =
-          make_uint4(o4[0], o4[1], o4[2], o4[3]);
-    }
+    store_query_fp16(qraw, qmx, qinv, smem + SM_Q);
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -459,8 +512,8 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     }
     red[warp * 32 + lane] = reduce_scatter32<true>(mx);
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (warp == 0)
-      hmax[lane] = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane]));
+    if (warp == 0)  // the maxima of the prescaled logits, scaled back by 2^-s (exact)
+      hmax[lane] = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane])) * qinv[lane];
     asm volatile("bar.sync 1, 128;" ::: "memory");
     float m_h[32], sm[32];
 #pragma unroll
@@ -480,8 +533,8 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       uint32_t ph[16];
 #pragma unroll
       for (int h = 0; h < 32; h += 2) {
-        const float x0 = m * __uint_as_float(h < 16 ? r0[h] : r1[h - 16]);
-        const float x1 = m * __uint_as_float(h + 1 < 16 ? r0[h + 1] : r1[h - 15]);
+        const float x0 = (m * __uint_as_float(h < 16 ? r0[h] : r1[h - 16])) * qinv[h];
+        const float x1 = (m * __uint_as_float(h + 1 < 16 ? r0[h + 1] : r1[h - 15])) * qinv[h + 1];
         const float e0 = (valid && m_h[h] != -INFINITY) ? __expf(x0 - m_h[h]) : 0.f;
         const float e1 = (valid && m_h[h + 1] != -INFINITY) ? __expf(x1 - m_h[h + 1]) : 0.f;
         sm[h] += e0;
@@ -615,7 +668,8 @@ constexpr int T_MU = T_SLOT + AM_TILE * 8;
 constexpr int T_PV = T_MU + AM_TILE * 4;
 constexpr int T_RED = T_PV + AM_TILE * 4;
 constexpr int T_HM = T_RED + 8 * 32 * 4;
-constexpr int T_BAR = T_HM + 2 * 32 * 4;        // full[8], qfull, phase_done
+constexpr int T_QS = T_HM + 2 * 32 * 4;         // query prescale (as SM_QS)
+constexpr int T_BAR = T_QS + (8 * AM_QU + 32) * 4;   // full[8], qfull, phase_done
 constexpr int T_MISC = T_BAR + 8 * 10;
 constexpr size_t T_SMEM = T_MISC + 16 + 1024;
 }  // namespace
@@ -642,7 +696,8 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   const int split = int(cg::this_cluster().block_rank());
   const int b = row / p.Q;
   const int pos = p.q_pos[row];
-  const int nks = p.idx ? p.k : 0;
+  const int nvis = (p.idx || p.dense) ? visible_entries(p.c, b, pos) : 0;
+  const int nks = p.dense ? max(0, min(p.e1, nvis) - p.e0) : (p.idx ? p.k : 0);
   int lo = 0, nkw = 0;
   if (p.codes && pos >= 0) {
     lo = max(0, pos - p.window + 1);
@@ -650,12 +705,14 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   }
   const int nk = nks + nkw;
   const int key0 = split * AM_TILE;
+  if (tid == 0 && p.dense && nvis > p.n_bound) report(p.err, CSA2_ERR_SHAPE);
+  uint32_t *qmx = reinterpret_cast<uint32_t *>(smem + T_QS);
+  float *qinv = reinterpret_cast<float *>(smem + T_QS + 8 * AM_QU * 4);
 
   // ---------------------------------------------------------------- loads
   // Producer t: key t % 128, dims 256 (t / 128) .. +255.  The query block's loads go
   // out first, then the key's index, then its raw bytes, all before any barrier.
-  constexpr int QU = AM_HG * (D / 8) / AM_PRODUCERS;
-  uint4 qraw[QU];
+  uint4 qraw[AM_QU];
   uint4 rr[16];  // listed entry: rr[0..7] = 128 code bytes, rr[8] = 16 scale bytes; window: 256 codes
   const int key_in = tid & (AM_TILE - 1), half = (tid >> 7) & 1;
   const int j = key0 + key_in;
@@ -664,16 +721,16 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   if (producer) {
     const uint16_t *qrow = p.q + (int64_t(row) * H + hg * AM_HG) * D;
 #pragma unroll
-    for (int u = 0; u < QU; ++u) {
+    for (int u = 0; u < AM_QU; ++u) {
       const int it = tid + u * AM_PRODUCERS;
       qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
     }
     float m = 0.f, pm = 0.f;
     if (j < nks) {
       sparse = true;
-      const int n = p.idx[int64_t(row) * p.k + j];
+      const int n = p.dense ? p.e0 + j : p.idx[int64_t(row) * p.k + j];
       if (n != -1) {
-        if (n < -1 || n >= visible_entries(p.c, b, pos)) {
+        if (n < -1 || n >= nvis) {
           if (half == 0) report(p.err, CSA2_ERR_INDEX);
         } else {
           s = cache_slot(p.c, b, n);
@@ -700,6 +757,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
       mu[key_in] = m;
       pv[key_in] = pm;
     }
+    publish_query_max(qraw, qmx);  // after the key loads are out
   }
   if (warp == AM_PRODUCERS / 32) {
     tmem_alloc(tmem_slot, AM_TMEM_COLS);
@@ -713,26 +771,14 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
     mbar_init_fence();
   }
   tc_fence_before();
-  __syncthreads();  // barriers, key list and TMEM address ready
+  __syncthreads();  // barriers, key list, query maxima and TMEM address ready
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   bool aborted = false;
 
   // ---------------------------------------------------------------- phase 1: S^T = K Q^T
   if (producer) {
-#pragma unroll
-    for (int u = 0; u < QU; ++u) {
-      const int it = tid + u * AM_PRODUCERS, h = it / (D / 8), u8 = it % (D / 8);
-      const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
-      uint32_t o4[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const __half2 hv = __floats2half2_rn(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-        o4[i] = *reinterpret_cast<const uint32_t *>(&hv);
-      }
-      *reinterpret_cast<uint4 *>(smem + T_Q + (u8 / 8) * 4096 + kmaj128(h, u8 % 8)) =
-          make_uint4(o4[0], o4[1], o4[2], o4[3]);
-    }
+    store_query_fp16(qraw, qmx, qinv, smem + T_Q);
     fence_proxy_async_smem();
     mbar_arrive(qfull);
     // this thread's four 64-dim blocks of its key, each published as soon as it is written
@@ -804,9 +850,9 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
     const float m = mu[key], pm = pv[key];
     float x[32], mx[32];
 #pragma unroll
-    for (int h = 0; h < 16; ++h) {
-      x[h] = m * __uint_as_float(r0[h]);
-      x[16 + h] = m * __uint_as_float(r1[h]);
+    for (int h = 0; h < 16; ++h) {  // prescaled logits scaled back by 2^-s (exact)
+      x[h] = (m * __uint_as_float(r0[h])) * qinv[h];
+      x[16 + h] = (m * __uint_as_float(r1[h])) * qinv[16 + h];
     }
 #pragma unroll
     for (int h = 0; h < 32; ++h) mx[h] = valid ? x[h] : -INFINITY;
@@ -903,6 +949,7 @@ static void launch_cs(const AttnArgs &a, int rows, cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr[dev]) {
+    if (CS > 8) cudaFuncSetAttribute(attn_mma_kernel<CS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     cudaFuncSetAttribute(attn_mma_kernel<CS>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(AM_SMEM));
     attr[dev] = true;
   }
@@ -925,21 +972,56 @@ static void launch_cs(const AttnArgs &a, int rows, cudaStream_t st) {
   }
 }
 
+// Clusters of CS attention CTAs the device can hold at once (0: none), per device.
+template <int CS>
+static int attn_clusters_fit() {
+  static int cached[64] = {};  // 0 unknown, -1 none
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    if (CS > 8) cudaFuncSetAttribute(attn_mma_kernel<CS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(attn_mma_kernel<CS>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(AM_SMEM));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, CS);
+    cfg.blockDim = dim3(AM_THREADS);
+    cfg.dynamicSmemBytes = AM_SMEM;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = CS;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    cached[dev] = (cudaOccupancyMaxActiveClusters(&n, attn_mma_kernel<CS>, &cfg) == cudaSuccess && n > 0) ? n : -1;
+    cudaGetLastError();
+  }
+  return cached[dev] > 0 ? cached[dev] : 0;
+}
+
+int attn_dense_segment() { return attn_clusters_fit<16>() > 0 ? 8192 : 4096; }
+
 // Few query rows leave most SMs idle: then a cluster of CTAs (one per 128-key tile)
 // splits each row's keys and combines the partials through distributed shared memory.
+// A CTA holds at most 5 tiles (640 keys), so longer key sets (dense segments) always use
+// clusters of up to 16 CTAs.
 void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
-                     const csa2_cache *c, const uint8_t *codes, const float *scale, int R, int window, float *o,
-                     float *lse, int32_t *err, cudaStream_t st) {
+                     bool dense, int e0, int e1, int n_bound, const csa2_cache *c, const uint8_t *codes,
+                     const float *scale,
+                     int R, int window, float *o, float *lse, int32_t *err, cudaStream_t st) {
   const int rows = B * Q;
   if (rows == 0) return;
   AttnArgs a{};
   a.q = q, a.Q = Q, a.q_pos = q_pos, a.tau = tau;
-  a.idx = idx, a.k = idx ? k : 0;
+  a.idx = dense ? nullptr : idx, a.k = (idx && !dense) ? k : 0;
+  a.dense = dense ? 1 : 0, a.e0 = e0, a.e1 = e1, a.n_bound = n_bound;
   if (c) a.c = *c;
   a.codes = codes, a.scale = scale, a.R = R, a.window = window;
   a.o = o, a.lse = lse, a.err = err;
-  const int tiles = (a.k + (codes ? window : 0) + AM_TILE - 1) / AM_TILE;
-  const int cs = rows * (H / AM_HG) <= 64 ? max(1, min(tiles, 5)) : 1;
+  const int nkeys = (dense ? max(0, e1 - e0) : a.k) + (codes ? window : 0);
+  const int tiles = (nkeys + AM_TILE - 1) / AM_TILE;
+  int cs = rows * (H / AM_HG) <= 64 ? max(1, min(tiles, 5)) : 1;
   if (cs > 1 && cs == tiles) {  // one tile per CTA: the single-dequant form
     switch (cs) {
       case 2: launch_tile<2>(a, rows, st); return;
@@ -948,11 +1030,16 @@ void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, floa
       default: launch_tile<5>(a, rows, st); return;
     }
   }
+  cs = max(cs, (tiles + 4) / 5);
+  if (cs > 5) cs = cs <= 8 ? 8 : (cs <= 12 ? 12 : 16);
   switch (cs) {
     case 2: launch_cs<2>(a, rows, st); break;
     case 3: launch_cs<3>(a, rows, st); break;
     case 4: launch_cs<4>(a, rows, st); break;
     case 5: launch_cs<5>(a, rows, st); break;
+    case 8: launch_cs<8>(a, rows, st); break;
+    case 12: launch_cs<12>(a, rows, st); break;
+    case 16: launch_cs<16>(a, rows, st); break;
     default: launch_cs<1>(a, rows, st); break;
   }
 }

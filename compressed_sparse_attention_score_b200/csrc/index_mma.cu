@@ -103,6 +103,8 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
   const int t0 = blockIdx.x * a.chunk;
   const int t1 = min(t0 + a.chunk, t_all);
   const int ntiles = max(0, min(t1, t_work) - t0);
+  // a full scan whose output row is shorter than the visible entries would drop the tail
+  if (!a.cand && nvis > a.n_out && blockIdx.x == 0 && threadIdx.x == 0) report(a.err, CSA2_ERR_SHAPE);
 
   // Candidate lists of at most IM_CAND_TILES tiles are copied to shared memory by warp 0
   // while the other warps run the prologue, so the producer and the epilogue never wait
@@ -411,7 +413,7 @@ void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int 
   const int rows = B * Q;
   if (n_out == 0 || rows == 0) return;
   const int t_all = (n_out + IM_TILE - 1) / IM_TILE;
-  const int want = (2 * 148 + rows - 1) / rows;           // about two CTAs per SM in total
+  const int want = (2 * sm_count() + rows - 1) / rows;   // about two CTAs per SM in total
   const int min_tiles = cand ? 4 : 8;                     // short candidate lists: spread them wider
   const int splits = max(1, min(min(want, (t_all + min_tiles - 1) / min_tiles), 65535));
   const int chunk = (t_all + splits - 1) / splits;

@@ -18,6 +18,23 @@ inline void set_smem_limit(F *func, size_t bytes) {
   done[dev] = true;
 }
 
+// Streaming multiprocessors of the current device (queried once per device).
+inline int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 void launch_pack_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype, const float *pool_w, int B, int T,
                     const int32_t *first_entry, const csa2_cache &c, int32_t *err, cudaStream_t st);
 void launch_pack_swa(const void *x, csa2_dtype dtype, int B, int T, const int32_t *pos, uint8_t *codes,
@@ -28,8 +45,11 @@ void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int 
 void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int N, int k0, int32_t *idx0, float *val0,
                          int k1, int32_t *idx1, float *val1, const int32_t *map, cudaStream_t st);
 void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
-                     const csa2_cache *c, const uint8_t *codes, const float *scale, int R, int window, float *o,
-                     float *lse, int32_t *err, cudaStream_t st);
+                     bool dense, int e0, int e1, int n_bound, const csa2_cache *c, const uint8_t *codes,
+                     const float *scale,
+                     int R, int window, float *o, float *lse, int32_t *err, cudaStream_t st);
+// Entries per dense-attention launch (one cluster of at most 16 CTAs x 640 keys per row).
+int attn_dense_segment();
 void launch_merge(const float *o1, const float *l1, const float *o2, const float *l2, int64_t rows, int D_,
                   float *o, float *lse, cudaStream_t st);
 

@@ -4,10 +4,11 @@
 
 namespace csa2 {
 
-// One warp per row; lanes stride over the row in float4 units.
-__global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ o1, const float *__restrict__ l1,
-                                                    const float *__restrict__ o2, const float *__restrict__ l2,
-                                                    int64_t rows, int D_, float *o, float *lse) {
+// One warp per row; lanes stride over the row in float4 units.  o may alias o1 or o2 and
+// lse may alias l1 or l2 (each element is read before it is written, by the same thread), so
+// none of the pointers is declared __restrict__.
+__global__ void __launch_bounds__(256) merge_kernel(const float *o1, const float *l1, const float *o2,
+                                                    const float *l2, int64_t rows, int D_, float *o, float *lse) {
   const int lane = threadIdx.x & 31;
   const int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= rows) return;

@@ -554,14 +554,15 @@ static int max_active_clusters() {
 // 12, 10 and 8 CTAs whose clusters all fit on the device at once (a cluster needs its SMs in
 // one GPC, so fewer large clusters fit than SMs / CS).  Shorter rows: about 4096 scores per
 // CTA (then every CTA holds its chunk in shared memory), at most 8 CTAs, as long as all
-// clusters fit at once.  From 148 rows on, or for rows of at most 4096 scores, one CTA per
-// row and no cluster barriers.
+// clusters fit at once.  From one row per SM on, or for rows of at most 4096 scores, one CTA
+// per row and no cluster barriers.
 void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int N, int k0, int32_t *idx0, float *val0,
                          int k1, int32_t *idx1, float *val1, const int32_t *map, cudaStream_t st) {
   if (R == 0) return;
   const Sel s0{k0, idx0, val0}, s1{k1, idx1, val1};
   const int nsel = (k1 > 0 && idx1) ? 2 : 1;
-  if (R < 148 && N >= (1 << 18)) {
+  const int sms = sm_count();
+  if (R < sms && N >= (1 << 18)) {
     if (max_active_clusters<16>() >= R) {
       launch_cs<16>(scores, n_valid, R, N, s0, s1, nsel, map, st);
     } else if (max_active_clusters<12>() >= R) {
@@ -574,8 +575,8 @@ void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int
     return;
   }
   int cs = 1;
-  if (R < 148)
-    while (cs < 8 && cs * 4096 < N && 2 * cs * R <= 148) cs *= 2;
+  if (R < sms)
+    while (cs < 8 && cs * 4096 < N && 2 * cs * R <= sms) cs *= 2;
   if (cs == 8 && max_active_clusters<8>() < R) cs = 4;
   if (cs == 4 && max_active_clusters<4>() < R) cs = 2;
   switch (cs) {

@@ -50,7 +50,15 @@ typedef enum {
   CSA2_ERR_TIMEOUT = 6      /* device side: a bounded wait gave up */
 } csa2_status;
 
-typedef enum { CSA2_MODE_FULL = 0, CSA2_MODE_REINDEX = 1, CSA2_MODE_REUSE = 2 } csa2_mode;
+/* CSA2_MODE_DENSE attends every visible entry (no indexer, no indices): the
+ * predecessor's heavily compressed attention ("DeepSeek V4.1 Flash 深度解析",
+ * 本专栏篇目 "前代 · HCA": 128-fold compression, then dense attention). */
+typedef enum {
+  CSA2_MODE_FULL = 0,
+  CSA2_MODE_REINDEX = 1,
+  CSA2_MODE_REUSE = 2,
+  CSA2_MODE_DENSE = 3
+} csa2_mode;
 typedef enum { CSA2_F32 = 0, CSA2_BF16 = 1 } csa2_dtype;
 
 enum {
@@ -108,8 +116,9 @@ const char *csa2_last_error_string(void);
 csa2_status csa2_check(const int32_t *err, csa2_stream_t stream);
 
 /*
- * Bytes of workspace csa2_sparse_attn needs for these sizes (0 for Reuse).
- * max_entries bounds num_entries[b]; pool_k is the candidate-pool size (0 if none).
+ * Bytes of workspace csa2_sparse_attn needs for these sizes (0 for Reuse, and for
+ * Dense up to 4096 entries).  max_entries bounds num_entries[b]; pool_k is the
+ * candidate-pool size (0 if none).
  */
 size_t csa2_workspace_size(csa2_mode mode, int32_t B, int32_t Q, int32_t max_entries,
                            int32_t k, int32_t pool_k);
@@ -157,7 +166,9 @@ csa2_status csa2_pack_swa(const void *x, csa2_dtype dtype, int32_t B, int32_t T,
  *   cand [B][Q][P] entry indices (-1 = none) or NULL to score entries 0..N-1;
  *   scores [B][Q][N_out] fp32 with N_out = P when cand != NULL else max_entries.
  * Entries not visible to the query (see csa2_cache) and -1 candidates score -inf.
- * Device errors: a candidate >= num_entries[b] or a bad page -> CSA2_ERR_INDEX, -inf.
+ * Device errors: a candidate >= num_entries[b] or a bad page -> CSA2_ERR_INDEX, -inf;
+ * without candidates, a query that sees more than max_entries entries ->
+ * CSA2_ERR_SHAPE (only its first max_entries entries are scored).
  */
 csa2_status csa2_index_score(const uint16_t *q_ix, const uint16_t *w, int32_t B, int32_t Q,
                              const int32_t *q_pos, const int32_t *cand, int32_t P,
@@ -187,8 +198,14 @@ csa2_status csa2_topk(const float *scores, const int32_t *n_valid, int32_t R, in
  *            if pool_k > 0 the top-pool_k entries are written to pool_io [B][Q][pool_k].
  *   REINDEX: q_ix, w score the entries listed in pool_io [B][Q][pool_k]; top-k of them.
  *   REUSE:   idx_in [B][Q][k] given entry indices (-1 = none; order free).
+ *   DENSE:   every visible entry (q_ix, w, k, pool and indices unused); the caches of
+ *            the predecessor's 128-fold compressed layers are read this way.  Any
+ *            number of entries: beyond one segment of 4096 or 8192 entries the
+ *            segments' partial results are merged through the workspace.
  *   idx_out [B][Q][k] (optional, FULL/REINDEX) receives the chosen entries, ascending.
- *   k <= 512.
+ *   k <= 512 (FULL, REINDEX, REUSE).
+ * The bf16 query enters the tensor cores scaled by a power of two per head, so every
+ * value within a factor 2^32 of its head's largest is used exactly.
  * Per head: logits tau * q . v_j over the chosen entries, v_j the dequantised
  * 512-d main entry used as key and value; o [B][Q][64][512] fp32 = softmax-weighted
  * sum, lse [B][Q][64] fp32 natural-log normaliser; no entries -> o = 0, lse = -inf.
@@ -197,7 +214,9 @@ csa2_status csa2_topk(const float *scores, const int32_t *n_valid, int32_t R, in
  * same softmax, so o / lse are the log-sum-exp merge of the two branches
  * (what csa2_merge of the separate results gives).  swa_codes = NULL: none.
  * ws: csa2_workspace_size(mode, ...) bytes (may be NULL for REUSE).
- * Device errors: an index outside the visible entries -> CSA2_ERR_INDEX, skipped.
+ * Device errors: an index outside the visible entries -> CSA2_ERR_INDEX, skipped;
+ * FULL or DENSE with a query that sees more than max_entries entries -> CSA2_ERR_SHAPE
+ * (max_entries must bound the visible entries; the tail is left out).
  */
 csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int32_t B, int32_t Q,
                              const int32_t *q_pos, float softmax_scale, const uint16_t *q_ix,
@@ -240,9 +259,10 @@ csa2_status csa2_merge(const float *o1, const float *l1, const float *o2, const 
  * CSA2_NOALLOC_SCRATCH_BYTES (8 MiB; every GPU that loads the library holds it
  * until the process exits); calls whose csa2_workspace_size exceeds it return
  * CSA2_ERR_UNSUPPORTED with a message.  It allocates nothing itself.
- *   - The first call on a device looks up the array's device address on that
- *     device (make that device current); do this first call before any stream
- *     capture.
+ *   - Every call looks up the array's device address on the current device (the
+ *     lookup loads the library's module on a device's first call, so make that
+ *     first call before any stream capture); nothing is cached, so the entry
+ *     point stays valid after a device reset.
  *   - All calls on a device share the one array and each call overwrites it
  *     (no part of it needs to start at zero); calls that overlap on the GPU --
  *     on different streams, or from different host threads -- race.

@@ -136,5 +136,25 @@ def check_topk(gpu_idx, scores, oracle_idx, k, what=""):
     return False
 
 
+def gpu_attend_given(q, q_pos, cache, tau, max_entries, idx, swa=None, fused=False):
+    """GPU attention (Reuse mode) of the query rows q [B][Q][64][512] over the given entry lists
+    idx [B][Q][k] (e.g. the oracle's selection where the GPU's differs at a near-tie).  With
+    swa = (codes, scale) the sliding-window branch is merged: in the same call when fused, else
+    by csa2_swa_attn + csa2_merge.  Returns (o, lse)."""
+    k = K()
+    err = torch.zeros(1, dtype=torch.int32, device=q.device)
+    idx = torch.as_tensor(np.asarray(idx), dtype=torch.int32).to(q.device).contiguous()
+    if swa is not None and fused:
+        o, lse = k.csa2_sparse_attn("reuse", q, q_pos, cache, tau, max_entries, k=idx.shape[-1], idx_in=idx, err=err,
+                                    swa_codes=swa[0], swa_scale=swa[1])
+    else:
+        o, lse = k.csa2_sparse_attn("reuse", q, q_pos, cache, tau, max_entries, k=idx.shape[-1], idx_in=idx, err=err)
+        if swa is not None:
+            o2, l2 = k.csa2_swa_attn(q, q_pos, swa[0], swa[1], tau, err=err)
+            o, lse = k.csa2_merge(o, lse, o2, l2)
+    assert k.csa2_check(err) == 0
+    return o, lse
+
+
 def to_np(t):
     return t.detach().float().cpu().numpy() if t.dtype in (torch.bfloat16, torch.float16) else t.detach().cpu().numpy()

@@ -14,8 +14,8 @@ from oracle import formats as OF
 from workloads import configs as W
 from workloads import normal, uniform
 
-from tests.helpers import (K, check_attention, check_topk, fill_main, gpu_cache, oracle_seq, oracle_swa,
-                           to_np)
+from tests.helpers import (K, check_attention, check_topk, fill_main, gpu_attend_given, gpu_cache, oracle_seq,
+                           oracle_swa, to_np)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -295,12 +295,30 @@ def test_merge_matches_oracle_and_aliases():
     check_attention(to_np(o1), to_np(l1), ref_o, ref_l, "merge in place")
 
 
+def _run_layer(k, mode, spec, cache, q, q_ix, w, q_pos, codes, scale, fused, pool_k=0, pool_io=None, idx_in=None,
+               idx_out=None, err=None):
+    """One layer on the GPU: fused (the SWA ring joins csa2_sparse_attn's softmax) or three calls."""
+    if fused:
+        o, lse = k.csa2_sparse_attn(mode, q, q_pos, cache, spec.tau, spec.max_entries, k=spec.k, q_ix=q_ix, w=w,
+                                    pool_k=pool_k, pool_io=pool_io, idx_in=idx_in, idx_out=idx_out, err=err,
+                                    swa_codes=codes, swa_scale=scale)
+        return o, lse, None, None
+    o1, l1 = k.csa2_sparse_attn(mode, q, q_pos, cache, spec.tau, spec.max_entries, k=spec.k, q_ix=q_ix, w=w,
+                                pool_k=pool_k, pool_io=pool_io, idx_in=idx_in, idx_out=idx_out, err=err)
+    o2, l2 = k.csa2_swa_attn(q, q_pos, codes, scale, spec.tau, err=err)
+    o, lse = k.csa2_merge(o1, l1, o2, l2)
+    return o, lse, o1, l1
+
+
 def _decode_layer_parity(spec, cache, mode, layer, rings, codes, scale, pool=None, pool_k=0, idx_in=None,
                          oracle_caches=None, fused=False):
     """Run one layer on the GPU (sparse + SWA + merge) and compare with the oracle per sequence.
 
     fused=True passes the SWA ring to csa2_sparse_attn (one softmax over both key sets);
-    otherwise the branches run separately and csa2_merge combines them.
+    otherwise the branches run separately and csa2_merge combines them.  Every sequence's
+    attention is compared: where the GPU's selection legitimately differs from the oracle's at
+    a near-tie (check_topk), the GPU layer is run again in Reuse mode on the oracle's indices
+    and that output is compared instead.
     """
     k = K()
     q, q_ix, w, q_pos = W.query_tensors(spec, layer, DEV)
@@ -309,27 +327,19 @@ def _decode_layer_parity(spec, cache, mode, layer, rings, codes, scale, pool=Non
     pool_io = pool
     if mode == "full" and pool_k:
         pool_io = torch.empty((spec.B, 1, pool_k), dtype=torch.int32, device=DEV)
-    if fused:
-        o, lse = k.csa2_sparse_attn(mode, q, q_pos, cache, spec.tau, spec.max_entries, k=spec.k, q_ix=q_ix, w=w,
-                                    pool_k=pool_k, pool_io=pool_io, idx_in=idx_in, idx_out=idx_out, err=err,
-                                    swa_codes=codes, swa_scale=scale)
-        o1 = l1 = None
-    else:
-        o1, l1 = k.csa2_sparse_attn(mode, q, q_pos, cache, spec.tau, spec.max_entries, k=spec.k, q_ix=q_ix,
-                                    w=w, pool_k=pool_k, pool_io=pool_io, idx_in=idx_in, idx_out=idx_out, err=err)
-        o2, l2 = k.csa2_swa_attn(q, q_pos, codes, scale, spec.tau, err=err)
-        o, lse = k.csa2_merge(o1, l1, o2, l2)
+    o, lse, o1, l1 = _run_layer(k, mode, spec, cache, q, q_ix, w, q_pos, codes, scale, fused, pool_k=pool_k,
+                                pool_io=pool_io, idx_in=idx_in, idx_out=idx_out, err=err)
     assert k.csa2_check(err) == 0
-    same_rows = 0
     ref_pools = np.full((spec.B, 1, max(pool_k, 1)), -1, np.int64)
     ref_idxs = np.full((spec.B, 1, spec.k), -1, np.int64)
+    same = []
     for b in range(spec.B):
         c = oracle_caches[b]
         pos = int(q_pos[b, 0])
-        qb, qib, wb = to_np(q[b, 0]), to_np(q_ix[b, 0]), to_np(w[b, 0])
+        qib, wb = to_np(q_ix[b, 0]), to_np(w[b, 0])
         if mode == "full":
             ref_idx, ref_pool, scores = OC.full_select(c, 0, pos, qib, wb, spec.k, pool_k)
-            same = check_topk(to_np(idx_out[b, 0]), scores, ref_idx, spec.k, f"full idx b={b}")
+            same.append(check_topk(to_np(idx_out[b, 0]), scores, ref_idx, spec.k, f"full idx b={b}"))
             if pool_k:
                 check_topk(to_np(pool_io[b, 0]), scores, ref_pool, pool_k, f"pool b={b}")
                 ref_pools[b, 0] = ref_pool
@@ -339,22 +349,30 @@ def _decode_layer_parity(spec, cache, mode, layer, rings, codes, scale, pool=Non
             gi = to_np(idx_out[b, 0])
             gpos = np.array([np.searchsorted(pl, v) if v >= 0 else -1 for v in gi])
             rpos = np.array([np.searchsorted(pl, v) if v >= 0 else -1 for v in ref_idx])
-            same = check_topk(gpos, pscores, rpos, spec.k, f"reindex idx b={b}")
+            same.append(check_topk(gpos, pscores, rpos, spec.k, f"reindex idx b={b}"))
         else:
             ref_idx = to_np(idx_in[b, 0])
-            same = True
+            same.append(True)
         ref_idxs[b, 0] = ref_idx
-        if same:
-            same_rows += 1
-            fill_main(c, spec, b, ref_idx, gen_device=DEV)
-            ref = OC.decode_layer("reuse", c, 0, pos, qb, spec.tau, rings[b], idx=ref_idx)
-            if o1 is not None:
-                check_attention(to_np(o1[b, 0]), to_np(l1[b, 0]), *ref["sparse"], f"{mode} sparse b={b}")
-            check_attention(to_np(o[b, 0]), to_np(lse[b, 0]), ref["o"], ref["lse"], f"{mode} merged b={b}")
-    assert same_rows >= max(1, spec.B - 1)
+    ref_idx_t = torch.from_numpy(ref_idxs).to(torch.int32).to(DEV)
+    if not all(same):   # near-tie selections: the GPU attends the oracle's entries instead
+        o_r, lse_r, o1_r, l1_r = _run_layer(k, "reuse", spec, cache, q, q_ix, w, q_pos, codes, scale, fused,
+                                            idx_in=ref_idx_t, err=err)
+        assert k.csa2_check(err) == 0
+    compared = 0
+    for b in range(spec.B):
+        src = (o, lse, o1, l1) if same[b] else (o_r, lse_r, o1_r, l1_r)
+        c = oracle_caches[b]
+        fill_main(c, spec, b, ref_idxs[b, 0], gen_device=DEV)
+        ref = OC.decode_layer("reuse", c, 0, int(q_pos[b, 0]), to_np(q[b, 0]), spec.tau, rings[b],
+                              idx=ref_idxs[b, 0])
+        if src[2] is not None:
+            check_attention(to_np(src[2][b, 0]), to_np(src[3][b, 0]), *ref["sparse"], f"{mode} sparse b={b}")
+        check_attention(to_np(src[0][b, 0]), to_np(src[1][b, 0]), ref["o"], ref["lse"], f"{mode} merged b={b}")
+        compared += 1
+    assert compared == spec.B
     # the oracle's own selections, for the layers that consume them
-    return (torch.from_numpy(ref_idxs).to(torch.int32).to(DEV),
-            torch.from_numpy(ref_pools).to(torch.int32).to(DEV))
+    return ref_idx_t, torch.from_numpy(ref_pools).to(torch.int32).to(DEV)
 
 
 @pytest.mark.parametrize("fused", [False, True])
@@ -455,14 +473,21 @@ def test_prefill_chunk_scaled():
     c = oracle_seq(spec, 0, main_rows=[], gen_device=DEV)
     ring = oracle_swa(to_np(x[0]), to_np(pos[0]), R)
     rows = [0, 1, 2, 57, 150, 298, 299]
+    compared = 0
     for qi in rows:
         p = int(q_pos[0, qi])
         ref_idx, _, scores = OC.full_select(c, 0, p, to_np(q_ix[0, qi]), to_np(w[0, qi]), spec.k)
         assert (ref_idx[ref_idx >= 0] < (p + 1) // 2).all()
-        if check_topk(to_np(idx_out[0, qi]), scores, ref_idx, spec.k, f"prefill q={qi}"):
-            fill_main(c, spec, 0, ref_idx, gen_device=DEV)
-            ref = OC.decode_layer("reuse", c, 0, p, to_np(q[0, qi]), spec.tau, ring, idx=ref_idx)
-            check_attention(to_np(o[0, qi]), to_np(lse[0, qi]), ref["o"], ref["lse"], f"prefill q={qi}")
+        go, gl = o[0, qi], lse[0, qi]
+        if not check_topk(to_np(idx_out[0, qi]), scores, ref_idx, spec.k, f"prefill q={qi}"):
+            go, gl = gpu_attend_given(q[:, qi:qi + 1].contiguous(), q_pos[:, qi:qi + 1].contiguous(), cache,
+                                      spec.tau, spec.max_entries, ref_idx[None, None], swa=(codes, scale))
+            go, gl = go[0, 0], gl[0, 0]
+        fill_main(c, spec, 0, ref_idx, gen_device=DEV)
+        ref = OC.decode_layer("reuse", c, 0, p, to_np(q[0, qi]), spec.tau, ring, idx=ref_idx)
+        check_attention(to_np(go), to_np(gl), ref["o"], ref["lse"], f"prefill q={qi}")
+        compared += 1
+    assert compared == len(rows)
 
 
 def test_mixed_paged_batch_scaled():
@@ -493,15 +518,130 @@ def test_mixed_paged_batch_scaled():
                                     idx_in=idx_all[sel].contiguous() if mode == "reuse" else None,
                                     idx_out=idx_out if mode == "full" else None, err=err)
         assert k.csa2_check(err) == 0
+        compared = 0
         for j, b in enumerate(ids):
             c = oracle_seq(spec, b, main_rows=[], gen_device=DEV)
             p = int(q_pos[b, 0])
+            go, gl = o[j, 0], lse[j, 0]
             if mode == "full":
                 ref_idx, _, scores = OC.full_select(c, 0, p, to_np(q_ix[b, 0]), to_np(w[b, 0]), 512)
                 if not check_topk(to_np(idx_out[j, 0]), scores, ref_idx, 512, f"mixed full b={b}"):
-                    continue
+                    one = k.GlobalKVCache(1, ratio, num_slots=base.num_slots, page_table=table[b:b + 1].contiguous(),
+                                          page_size=256, planes=base.planes,
+                                          num_entries=base.num_entries[b:b + 1].contiguous())
+                    go, gl = gpu_attend_given(q[b:b + 1].contiguous(), q_pos[b:b + 1].contiguous(), one, spec.tau,
+                                              maxe, ref_idx[None, None])
+                    go, gl = go[0, 0], gl[0, 0]
             else:
                 ref_idx = to_np(idx_all[b, 0])
             fill_main(c, spec, b, ref_idx, gen_device=DEV)
             oo, ol = OC.sparse_attention(c, 0, to_np(q[b, 0]), ref_idx, spec.tau)
-            check_attention(to_np(o[j, 0]), to_np(lse[j, 0]), oo, ol, f"mixed {mode} b={b}")
+            check_attention(to_np(go), to_np(gl), oo, ol, f"mixed {mode} b={b}")
+            compared += 1
+        assert compared == len(ids)
+
+
+# ------------------------------------------------------------------ predecessor variants and dense attention
+def test_full_decode_ratio4():
+    """The predecessor's CSA: 4 tokens per entry, lightning indexer, top-512 (Full mode at r = 4)."""
+    spec = W.scaled(W.tiny_full(), [8192, 6001], B=2, ratio=4)
+    cache = gpu_cache(spec)
+    codes, scale, rings = _swa_state(spec, 0)
+    oc = [oracle_seq(spec, b, main_rows=[], gen_device=DEV) for b in range(spec.B)]
+    assert [int(c.num_entries[0]) for c in oc] == [2048, 1500]
+    _decode_layer_parity(spec, cache, "full", 0, rings, codes, scale, oracle_caches=oc, fused=True)
+
+
+def _dense_parity(spec, cache, fused, tau=None):
+    k = K()
+    tau = spec.tau if tau is None else tau
+    q, _, _, q_pos = W.query_tensors(spec, 0, DEV)
+    codes, scale, rings = _swa_state(spec, 0)
+    err = _err()
+    if fused:
+        o, lse = k.csa2_sparse_attn("dense", q, q_pos, cache, tau, spec.max_entries, err=err, swa_codes=codes,
+                                    swa_scale=scale)
+    else:
+        o, lse = k.csa2_sparse_attn("dense", q, q_pos, cache, tau, spec.max_entries, err=err)
+    assert k.csa2_check(err) == 0
+    for b in range(spec.B):
+        c = oracle_seq(spec, b, gen_device=DEV)
+        pos = int(q_pos[b, 0])
+        every = np.arange(c.visible(0, pos))
+        if fused:
+            ref = OC.decode_layer("reuse", c, 0, pos, to_np(q[b, 0]), tau, rings[b], idx=every)
+            check_attention(to_np(o[b, 0]), to_np(lse[b, 0]), ref["o"], ref["lse"], f"dense+swa b={b}")
+        else:
+            oo, ol = OC.sparse_attention(c, 0, to_np(q[b, 0]), every, tau)
+            check_attention(to_np(o[b, 0]), to_np(lse[b, 0]), oo, ol, f"dense b={b}")
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_dense_attention_hca_ratio128(fused):
+    """The predecessor's HCA: 128 tokens per entry, then attention over every entry."""
+    spec = W.scaled(W.tiny_full(), [128 * 700, 128 * 333 + 77, 128 * 3], B=3, ratio=128)
+    cache = gpu_cache(spec)
+    _dense_parity(spec, cache, fused)
+
+
+def test_dense_attention_over_many_entries():
+    """9000 and 5000 entries: more keys than one cluster holds at 4096 per segment, and (at 8192
+    per segment) a second segment merged through the workspace."""
+    spec = W.scaled(W.reuse64k(), [9000, 5000], B=2)
+    cache = gpu_cache(spec)
+    _dense_parity(spec, cache, fused=True)
+
+
+def test_dense_attention_many_rows():
+    """Enough rows that each row runs on one CTA (no key-split cluster) when its keys fit."""
+    spec = W.scaled(W.reuse64k(), [300 + 7 * i for i in range(40)], B=40)
+    cache = gpu_cache(spec)
+    _dense_parity(spec, cache, fused=True)
+
+
+def test_dense_and_full_report_a_short_max_entries():
+    """A query that sees more entries than max_entries sets CSA2_ERR_SHAPE instead of silently
+    leaving the tail out."""
+    k = K()
+    spec = W.scaled(W.tiny_full(), [3000], B=1)
+    cache = gpu_cache(spec)
+    q, q_ix, w, q_pos = W.query_tensors(spec, 0, DEV)
+    for mode in ("full", "dense"):
+        err = _err()
+        k.csa2_sparse_attn(mode, q, q_pos, cache, spec.tau, 1000, q_ix=q_ix, w=w, err=err)
+        assert k.csa2_check(err) == 2, mode
+
+
+# ------------------------------------------------------------------ query magnitudes
+@pytest.mark.parametrize("B", [3, 40])
+@pytest.mark.parametrize("case", ["large", "small", "mixed"])
+def test_query_magnitudes_are_exact(case, B):
+    """bf16 queries far outside fp16 range (1e5) or deep in its subnormals (1e-6) attend as exactly
+    as N(0,1) ones: the per-head power-of-two prescale keeps every value.  B = 3 runs the one-tile
+    cluster kernel, B = 40 the several-tile kernel."""
+    k = K()
+    spec = W.scaled(W.reuse64k(), [4000 + 37 * b for b in range(B)], B=B)
+    cache = gpu_cache(spec)
+    q, _, _, q_pos = W.query_tensors(spec, 0, DEV)
+    g = q.float()
+    if case == "large":
+        g, tau = g * 1e5, 1e-5
+    elif case == "small":
+        g, tau = g * 1e-6, 1e6
+    else:  # one head mixes both magnitudes; others stay N(0,1)/sqrt(512)
+        g[:, :, 5, :256] *= 1e5
+        g[:, :, 5, 256:] *= 1e-6
+        g[:, :, 9] *= 1e5
+        tau = 1e-5
+    q = g.to(torch.bfloat16).contiguous()
+    idx = W.reuse_indices(spec, DEV)
+    codes, scale, rings = _swa_state(spec, 0)
+    err = _err()
+    o, lse = k.csa2_sparse_attn("reuse", q, q_pos, cache, tau, spec.max_entries, idx_in=idx, err=err,
+                                swa_codes=codes, swa_scale=scale)
+    assert k.csa2_check(err) == 0
+    assert torch.isfinite(o).all()
+    for b in range(0, B, max(1, B // 5)):
+        c = oracle_seq(spec, b, main_rows=to_np(idx[b, 0]), gen_device=DEV)
+        ref = OC.decode_layer("reuse", c, 0, int(q_pos[b, 0]), to_np(q[b, 0]), tau, rings[b], idx=to_np(idx[b, 0]))
+        check_attention(to_np(o[b, 0]), to_np(lse[b, 0]), ref["o"], ref["lse"], f"{case} b={b}")

@@ -303,3 +303,60 @@ def test_swa_equals_dense_over_last_window():
     # at the start of a sequence the window is shorter
     o0, _ = C.swa_attention(q, 0, codes[[0] * R], scale[[0] * R], W, 0.05)
     np.testing.assert_allclose(o0, np.repeat(F.unpack_swa(codes[:1], scale[:1]), 2, 0), rtol=1e-12)
+
+
+# ----------------------------------------------------------------- one whole layer
+def _brute_window_keys(codes, scale, pos, window):
+    """Dequantised SWA tokens of positions max(0, pos - window + 1) .. pos, element by element."""
+    R = codes.shape[0]
+    keys = []
+    for t in range(max(0, pos - window + 1), pos + 1):
+        s = float(scale[t % R])
+        keys.append([float(F.e4m3_decode(np.uint8(c))) * s for c in codes[t % R].tolist()])
+    return keys
+
+
+@pytest.mark.parametrize("mode", ["full", "reindex", "reuse"])
+def test_decode_layer_is_one_softmax_over_entries_and_window(mode):
+    """A layer's output is one softmax over its listed entries and its window tokens together.
+
+    The listed entries are re-derived by brute force (scores by loops, rank definition), the
+    window by position arithmetic, and the attention by plain loops, so that a layer that drops
+    a branch, passes a wrong window or merges with wrong weights fails here.
+    """
+    rng = np.random.default_rng(21)
+    cache, _ = _tiny_cache(40, 1, seed=23)
+    n = int(cache.num_entries[0])
+    H, W, R, pos, k, tau = 3, 5, 8, 37, 6, 0.05
+    q = rng.normal(size=(H, 512))
+    q_ix = rng.normal(size=(4, 128)).astype(np.float32)
+    w = rng.uniform(size=4).astype(np.float32)
+    x = rng.normal(size=(R, 512)).astype(np.float32)
+    codes = np.zeros((R, 512), np.uint8)
+    scale = np.zeros(R, np.float32)
+    for t in range(pos - R + 1, pos + 1):
+        codes[t % R], scale[t % R] = F.pack_swa(x[t % R])
+    vis = min(n, pos + 1)
+    keys_ix = F.unpack_indexer(cache.ix_codes[0, :vis], cache.ix_scales[0, :vis])
+    s_all = brute_scores(q_ix, w, keys_ix)
+    if mode == "full":
+        out = C.decode_layer("full", cache, 0, pos, q, tau, (codes, scale), window=W, q_ix=q_ix, w=w, k=k)
+        want = brute_topk(list(s_all), k)
+    elif mode == "reindex":
+        pool = np.array([3, 7, 11, 12, 19, 25, 30, 31, 36, -1], np.int64)
+        out = C.decode_layer("reindex", cache, 0, pos, q, tau, (codes, scale), window=W, q_ix=q_ix, w=w,
+                             k=k, pool=pool)
+        ps = [s_all[p] if p >= 0 else -math.inf for p in pool.tolist()]
+        want = [int(pool[j]) if j >= 0 else -1 for j in brute_topk(ps, k)]
+    else:
+        idx = np.array([2, 9, -1, 33, 14], np.int64)
+        out = C.decode_layer("reuse", cache, 0, pos, q, tau, (codes, scale), window=W, idx=idx)
+        want = idx.tolist()
+    np.testing.assert_array_equal(np.asarray(out["idx"]), want)
+    listed = [j for j in want if j >= 0]
+    main = F.unpack_main(cache.kv_codes[0, listed], cache.kv_scales[0, listed]).tolist()
+    keys = main + _brute_window_keys(codes, scale, pos, W)
+    assert len(keys) == len(listed) + W
+    bo, bl = brute_attend(q.tolist(), keys, tau)
+    np.testing.assert_allclose(out["o"], bo, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(out["lse"], bl, rtol=1e-12)

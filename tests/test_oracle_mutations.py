@@ -105,3 +105,23 @@ def test_swa_window_off_by_one_is_caught(monkeypatch):
         return C.attend(q, F.unpack_swa(codes[slots], scale[slots]), tau)
     monkeypatch.setattr(C, "swa_attention", bad)
     _fails(TM.test_swa_equals_dense_over_last_window)
+
+
+def test_layer_without_its_window_branch_is_caught(monkeypatch):
+    orig = C.swa_attention
+    monkeypatch.setattr(C, "swa_attention",
+                        lambda q, pos, codes, scale, window, tau: C.attend(q, np.zeros((0, 512)), tau))
+    _fails(TM.test_decode_layer_is_one_softmax_over_entries_and_window, "reuse")
+    monkeypatch.setattr(C, "swa_attention", orig)
+
+
+def test_layer_with_the_default_window_is_caught(monkeypatch):
+    orig = C.swa_attention
+    monkeypatch.setattr(C, "swa_attention",
+                        lambda q, pos, codes, scale, window, tau: orig(q, pos, codes, scale, 128, tau))
+    _fails(TM.test_decode_layer_is_one_softmax_over_entries_and_window, "full")
+
+
+def test_layer_that_skips_its_listed_entries_is_caught(monkeypatch):
+    monkeypatch.setattr(C, "sparse_attention", lambda cache, b, q, idx, tau: C.attend(q, np.zeros((0, 512)), tau))
+    _fails(TM.test_decode_layer_is_one_softmax_over_entries_and_window, "reindex")
