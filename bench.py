@@ -82,7 +82,7 @@ def barrier(world):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """SM clock and clock-event reasons, read through NVML every 2 ms on a helper thread while the
+    """SM clock and clock-event reasons, read through NVML every 0.5 ms on a helper thread while the
     timed region runs (reads only: no clock or other GPU setting is changed)."""
 
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
@@ -118,7 +118,7 @@ class ClockSampler:
                 self.reasons.update(name for name, m in masks if bits & m)
             except Exception:
                 return
-            if self.done.wait(0.002):
+            if self.done.wait(0.0005):
                 return
 
     def stop(self):
@@ -130,7 +130,7 @@ class ClockSampler:
             return None
         sm = sorted(self.sm)
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                "samples": len(sm), "source": "NVML, every 2 ms during the timed steps"}
+                "samples": len(sm), "source": "NVML, every 0.5 ms during the timed steps"}
 
 
 # ---------------------------------------------------------------- the workload on the GPU
@@ -258,9 +258,137 @@ class Hier1M:
         h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
         return ins, h_in, outs, h_out
 
+    def attention(self, layer):
+        """The attention launch of one layer alone (its entries as given indices, its window fused)."""
+        self.k.csa2_sparse_attn("reuse", self.q[layer], self.q_pos, self.cache, self.spec.tau, self.N, k=self.spec.k,
+                                idx_in=self.idx[layer], o=self.o[layer], lse=self.lse[layer], err=self.err,
+                                swa_codes=self.swa_codes[layer], swa_scale=self.swa_scale[layer])
+
+    def gather_bytes(self):
+        """Bytes one attention launch must move: per sequence its 512 listed main entries (288 B), its 128
+        window tokens (516 B), its bf16 query heads (64 KB) and fp32 output heads (128 KB + lse)."""
+        return self.B * (self.spec.k * 288 + 128 * 516 + 64 * 512 * 2 + 64 * 512 * 4 + 64 * 4)
+
     def scan_bytes(self):
-        """Algorithmic bytes of one Full-layer indexer launch: every key read once, one fp32 score written."""
-        return self.B * self.N * (68 + 4) + self.B * 64 * (128 * 2 + 2)
+        """Algorithmic bytes of one Full-layer indexer launch: every 68-byte indexer key read once.
+
+        The fp32 score row (4 B per entry) is an artefact of handing the scores to a separate top-k
+        launch, not of the method, so it counts as traffic, not as algorithmic bytes."""
+        return self.B * self.N * 68
+
+
+class Model40:
+    """Device state of one decode token through the pages' 40-layer stack (csa2_decode_step).
+
+    Four caches, one per Full layer (the encoder's three at ratio 2, the decoder's at ratio 1),
+    hold every token before this step's, so the step itself appends the token to each of them
+    (at ratio 2 the token before it waits in the staging rows); every layer's SWA ring holds the
+    127 tokens before it and the step packs this token's.
+    """
+
+    R = 128
+
+    def __init__(self, spec, dev):
+        import compressed_sparse_attention_score_b200 as k
+        from workloads import configs as W
+        self.k, self.spec, self.dev = k, spec, dev
+        self.plan, self.ratios = k.csa2_plan_v41()
+        L, B, T = len(self.plan), spec.B, spec.tokens[0]
+        assert all(t == T for t in spec.tokens), "one position for every sequence"
+        self.L, self.B, self.T, self.pos_ = L, B, T, T - 1
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.err = err
+        zero = torch.zeros(1, dtype=torch.int32, device=dev)
+        nc = len(self.ratios)
+        rmax = max(self.ratios)
+        self.pos = torch.full((B,), T - 1, dtype=torch.int32, device=dev)
+        self.new_kv = torch.empty((nc, B, 512), dtype=torch.bfloat16, device=dev)
+        self.new_ix = torch.empty((nc, B, 128), dtype=torch.bfloat16, device=dev)
+        self.kv_stage = torch.zeros((nc, B, rmax, 640), dtype=torch.float32, device=dev)
+        self.caches, self.max_entries, self.cache_specs = [], [], []
+        for c, r in enumerate(self.ratios):
+            cs = W.cache_spec(spec, c, r, shares_queries=c == nc - 1)
+            n = T // r
+            cache = k.GlobalKVCache(B, r, seq_stride=(n + 127) // 128 * 128)
+            p0 = (T - 1) // r * r                       # first token of this step's group
+            for b in range(B):
+                kv, ix = W.token_latents(cs, b, dev)
+                k.csa2_pack_kv(kv[None, :p0].contiguous(), ix[None, :p0].contiguous(), zero, cache.seq_view(b),
+                               err=err)
+                self.new_kv[c, b].copy_(kv[T - 1])
+                self.new_ix[c, b].copy_(ix[T - 1])
+                for t in range(p0, T - 1):              # the group's earlier tokens wait in staging
+                    view = cache.seq_view(b)
+                    view.num_entries.fill_(p0 // r)
+                    k.csa2_append_kv(kv[t:t + 1].contiguous(), ix[t:t + 1].contiguous(),
+                                     torch.full((1,), t, dtype=torch.int32, device=dev), view,
+                                     stage=self.kv_stage[c, b:b + 1], err=err)
+                del kv, ix
+            cache.num_entries.fill_(p0 // r)
+            self.caches.append(cache)
+            self.max_entries.append(n)
+            self.cache_specs.append(cs)
+        qs = [W.query_tensors(spec, layer, dev) for layer in range(L)]
+        self.q = torch.stack([t[0][:, 0] for t in qs]).contiguous()        # [L][B][64][512]
+        self.q_ix = torch.stack([t[1][:, 0] for t in qs]).contiguous()     # [L][B][64][128]
+        self.w = torch.stack([t[2][:, 0] for t in qs]).contiguous()        # [L][B][64]
+        self.swa_codes = torch.zeros((L, B, self.R, 512), dtype=torch.uint8, device=dev)
+        self.swa_scale = torch.zeros((L, B, self.R), dtype=torch.float32, device=dev)
+        self.swa_x = torch.empty((L, B, 512), dtype=torch.bfloat16, device=dev)
+        for layer in range(L):
+            x, p = W.swa_tokens(spec, layer, dev)
+            k.csa2_pack_swa(x[:, :-1].contiguous(), p[:, :-1].contiguous(), self.swa_codes[layer],
+                            self.swa_scale[layer], err=err)
+            self.swa_x[layer].copy_(x[:, -1])
+        self.idx = torch.full((L, B, spec.k), -1, dtype=torch.int32, device=dev)
+        self.pool = torch.full((nc, B, spec.pool_k), -1, dtype=torch.int32, device=dev)
+        self.o = torch.empty((L, B, 64, 512), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((L, B, 64), dtype=torch.float32, device=dev)
+        self.dstep = k.DecodeStep(self.plan, self.caches, self.max_entries, self.pos, spec.tau, spec.k, spec.pool_k,
+                                  self.q, self.swa_x, self.swa_codes, self.swa_scale, self.idx, self.o, self.lse,
+                                  q_ix=self.q_ix, w=self.w, pool=self.pool, new_kv=self.new_kv, new_ix=self.new_ix,
+                                  kv_stage=self.kv_stage, window=128)
+        self.ws = torch.empty(max(1, self.dstep.workspace_size()), dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+        assert k.csa2_check(err) == 0
+
+    def step(self, graphs=False):
+        if graphs:
+            self.graph.replay()
+        else:
+            self.dstep.run(self.ws, err=self.err)
+
+    def capture(self):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(self.graph, stream=side):
+                self.dstep.run(self.ws, err=self.err, stream=side)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+
+    def launches_per_step(self):
+        """Kernels of one step: one append per cache, per Full or Reindex layer an indexer scan and a
+        top-k, and per layer one attention launch (which also packs the layer's window token)."""
+        sel = sum(1 for m, _, _ in self.plan if m in (0, 1))
+        return len(self.ratios) + 2 * sel + len(self.plan)
+
+    def reindex_recall(self):
+        """Per Reindex layer: the share of its top-k (searched inside the decoder pool) that an exact
+        top-k over the whole decoder cache with the same indexer query also picks."""
+        k, out = self.k, {}
+        c = self.plan[next(i for i, p in enumerate(self.plan) if p[0] == 1)][2]
+        for layer, (m, _, _) in enumerate(self.plan):
+            if m != 1:
+                continue
+            s = k.csa2_index_score(self.q_ix[layer][:, None].contiguous(), self.w[layer][:, None].contiguous(),
+                                   self.pos[:, None].contiguous(), self.caches[c], self.max_entries[c], err=self.err)
+            exact = k.csa2_topk(s, self.spec.k)[0][:, 0]
+            got = self.idx[layer]
+            hit = [len(set(got[b].tolist()) & set(exact[b].tolist()) - {-1}) / self.spec.k for b in range(self.B)]
+            out[layer] = sum(hit) / len(hit)
+        return out
 
 
 def source_sha(paths):
@@ -378,6 +506,209 @@ def config_dict(spec):
             "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write, outside step events)"}
 
 
+class OneLayer:
+    """Device state of one CSA2 layer call over one of the other configurations, for their own lines:
+    tiny_full (Full decode, 2048 entries), reuse64k (Reuse decode, 32 x 65536 entries), mixed64 (paged,
+    32 Full sequences at ratio 2 and 32 Reuse sequences at ratio 1, two calls) and prefill8k (Full mode
+    for 8192 causal query tokens).  Every call runs the sliding-window branch and the merge in the same
+    launch as the sparse attention."""
+
+    def __init__(self, spec, dev):
+        import compressed_sparse_attention_score_b200 as k
+        from workloads import configs as W
+        self.k, self.spec, self.dev, self.W = k, spec, dev, W
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        zero = torch.zeros(1, dtype=torch.int32, device=dev)
+        B = spec.B
+        self.q, self.q_ix, self.w, self.q_pos = W.query_tensors(spec, 0, dev)
+        if spec.paged:
+            table, pages = W.page_layout(spec, dev)
+            self.base = k.GlobalKVCache(B, 1, num_slots=pages * spec.page_size, page_table=table,
+                                        page_size=spec.page_size)
+        else:
+            self.base = k.GlobalKVCache(B, spec.ratio, seq_stride=(spec.max_entries + 127) // 128 * 128)
+        for b in range(B):
+            kv, ix = W.token_latents(spec, b, dev)
+            v = self.base.seq_view(b)
+            v.ratio = spec.seq_ratio(b)
+            k.csa2_pack_kv(kv[None].contiguous(), ix[None].contiguous(), zero, v, err=self.err)
+            self.base.num_entries[b] = spec.entries(b)
+            del kv, ix
+        x, pos = W.swa_tokens(spec, 0, dev)
+        self.R = 128 if spec.q_len == 1 else spec.q_len + 128
+        self.codes = torch.zeros((B, self.R, 512), dtype=torch.uint8, device=dev)
+        self.scale = torch.zeros((B, self.R), dtype=torch.float32, device=dev)
+        k.csa2_pack_swa(x, pos, self.codes, self.scale, err=self.err)
+        self.calls = []   # (mode, rows tensor index or None, view, max_entries, idx_in)
+        if spec.name == "mixed64":
+            for mode, ratio in (("full", 2), ("reuse", 1)):
+                ids = [b for b in range(B) if spec.seq_mode(b) == mode]
+                sel = torch.tensor(ids, device=dev)
+                view = k.GlobalKVCache(len(ids), ratio, num_slots=self.base.num_slots,
+                                       page_table=self.base.page_table[sel].contiguous(), page_size=spec.page_size,
+                                       planes=self.base.planes, num_entries=self.base.num_entries[sel].contiguous())
+                idx = W.reuse_indices(spec, dev)[sel].contiguous() if mode == "reuse" else None
+                self.calls.append((mode, sel, view, max(spec.entries(b) for b in ids), idx))
+        else:
+            idx = W.reuse_indices(spec, dev) if spec.mode == "reuse" else None
+            self.calls.append((spec.mode if spec.mode != "prefill" else "full", None, self.base, spec.max_entries, idx))
+        self.io = []
+        for mode, sel, view, me, idx in self.calls:
+            take = (lambda t: t) if sel is None else (lambda t, s=sel: t[s].contiguous())
+            rows = take(self.q)
+            o = torch.empty(rows.shape[:2] + (64, 512), dtype=torch.float32, device=dev)
+            lse = torch.empty(rows.shape[:2] + (64,), dtype=torch.float32, device=dev)
+            nbytes = k.csa2_workspace_size(mode, rows.shape[0], rows.shape[1], me, spec.k)
+            ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev) if nbytes else None
+            self.io.append((rows, take(self.q_ix), take(self.w), take(self.q_pos), take(self.codes),
+                            take(self.scale), o, lse, ws))
+        torch.cuda.synchronize()
+        assert k.csa2_check(self.err) == 0
+
+    def step(self, graphs=False):
+        if graphs:
+            self.graph.replay()
+            return
+        for (mode, _, view, me, idx), (q, q_ix, w, q_pos, codes, scale, o, lse, ws) in zip(self.calls, self.io):
+            self.k.csa2_sparse_attn(mode, q, q_pos, view, self.spec.tau, me, k=self.spec.k, q_ix=q_ix, w=w,
+                                    idx_in=idx, o=o, lse=lse, ws=ws, err=self.err, swa_codes=codes, swa_scale=scale)
+
+    def capture(self):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(self.graph, stream=side):
+                self.step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+
+    def query_rows(self):
+        return self.spec.B * self.spec.q_len
+
+    def launches_per_step(self):
+        return sum(3 if mode == "full" else 1 for mode, *_ in self.calls)
+
+    def gather_bytes(self):
+        """Bytes the attention must move per step: per query row its listed main entries (288 B each),
+        its window tokens (516 B each), its bf16 query (64 KB) and fp32 output (128 KB + lse)."""
+        rows = self.query_rows()
+        return rows * (self.spec.k * 288 + 128 * 516 + 64 * 512 * 2 + 64 * 512 * 4 + 64 * 4)
+
+    def scan_pairs(self):
+        """(query, entry) pairs the indexer scores per step (Full calls)."""
+        n = 0
+        for (mode, sel, view, me, _), (q, *_rest) in zip(self.calls, self.io):
+            if mode != "full":
+                continue
+            ids = range(self.spec.B) if sel is None else sel.tolist()
+            for b in ids:
+                r = self.spec.seq_ratio(b)
+                n += sum(min(self.spec.entries(b), (p + 1) // r) for p in self.spec.query_pos(b))
+        return n
+
+
+def run_one_layer(args, spec, dev, world, rank):
+    """Own JSON line of one of the other configurations: query-tokens/s of one CSA2 layer call."""
+    wl = OneLayer(spec, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    graphs = not args.eager
+    for i in range(args.warmup):
+        wl.step(graphs=graphs and i > 0)
+        if graphs and i == 0:
+            wl.capture()
+    torch.cuda.synchronize()
+    assert wl.k.csa2_check(wl.err) == 0
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(dev)
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        wl.step(graphs=graphs)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps, world)
+    assert wl.k.csa2_check(wl.err) == 0
+    peak, peak_kind = peaks()
+    rows = wl.query_rows()
+    pairs = wl.scan_pairs()
+    line = {"metric": f"{spec.name}: query-tokens/s of one CSA2 layer (sparse + SWA + merge)",
+            "value": world * rows / (step_ms * 1e-3), "unit": "query-tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": spec.name, "batch": spec.B, "query_tokens": rows, "top_k": spec.k,
+                       "modes": sorted({m for m, *_ in wl.calls}),
+                       "launch": "eager" if args.eager else "CUDA graph of the layer's calls",
+                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write, outside step events)"},
+            "gather": {"bytes_per_step": wl.gather_bytes(),
+                       "GBps_whole_step": wl.gather_bytes() / (step_ms * 1e-3) / 1e9, "peak": peak,
+                       "peak_kind": peak_kind},
+            "gpu_launches": wl.launches_per_step() * args.steps, "clocks": clk}
+    if pairs:
+        line["indexer"] = {"pairs_per_step": pairs, "fp4_tflop_per_step": pairs * 64 * 128 * 2 / 1e12,
+                           "fp4_tflops_whole_step": pairs * 64 * 128 * 2 / (step_ms * 1e-3) / 1e12}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_model40(args, spec, dev, world, rank):
+    """One decode token of each sequence through the pages' 40-layer stack, one csa2_decode_step per
+    step, replayed from a CUDA graph; its own JSON line (whole-model decode per token)."""
+    wl = Model40(spec, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    graphs = not args.eager
+    for i in range(args.warmup):
+        wl.step(graphs=graphs and i > 0)
+        if graphs and i == 0:
+            wl.capture()
+    torch.cuda.synchronize()
+    assert wl.k.csa2_check(wl.err) == 0
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(dev)
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        wl.step(graphs=graphs)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps, world)
+    assert wl.k.csa2_check(wl.err) == 0
+    recall = wl.reindex_recall()
+    csa2_layers = sum(1 for m, _, _ in wl.plan if m != wl.k.LAYER_SWA)
+    scanned = sum(wl.B * wl.max_entries[c] for c in range(len(wl.ratios)))
+    line = {"metric": "decode tokens/s through the 40-layer CSA2 stack (one csa2_decode_step per token)",
+            "value": world * wl.B / (step_ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded N(0,1) latents, planted 2% cluster)",
+            "config": {"workload": f"{spec.name}: batch {spec.B}, {spec.tokens[0]} tokens/seq, 40 layers "
+                                   f"(2 SWA-only, 4 Full, 4 Reindex, 30 Reuse), caches at ratios {wl.ratios}",
+                       "batch": spec.B, "ctx_tokens": spec.tokens[0], "top_k": spec.k, "pool_k": spec.pool_k,
+                       "launch": "eager" if args.eager else "CUDA graph of csa2_decode_step",
+                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write, outside step events)"},
+            "query_tokens_per_s_per_csa2_layer": world * wl.B * csa2_layers / (step_ms * 1e-3),
+            "full_scan_entries_per_step": scanned,
+            "reindex_recall": {str(k): v for k, v in recall.items()},
+            "gpu_launches": wl.launches_per_step() * args.steps, "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
@@ -388,9 +719,15 @@ def main():
     from workloads import configs as W
     dev = torch.device("cuda", torch.cuda.current_device())
     spec = W.CONFIGS[args.workload](seed=rank)
-    assert spec.name == "hier1m", "bench.py times the hierarchical 1M-context decode workload"
     if args.batch:
         spec = W.scaled(spec, spec.tokens[0], B=args.batch)
+    if spec.name == "model40":
+        run_model40(args, spec, dev, world, rank)
+        return
+    if spec.name in ("tiny_full", "reuse64k", "mixed64", "prefill8k"):
+        run_one_layer(args, spec, dev, world, rank)
+        return
+    assert spec.name == "hier1m", "bench.py times the hierarchical 1M-context decode workload"
     wl = Hier1M(spec, dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -442,9 +779,38 @@ def main():
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev) / args.steps, world)
+    # the same end-to-end steps with every call made through the C ABI from Python (no graph replay)
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        eev[i][0].record(stream)
+        for d, h in zip(ins, h_in):
+            d.copy_(h, non_blocking=True)
+        wl.step(graphs=False)
+        for h, d in zip(h_out, outs):
+            h.copy_(d, non_blocking=True)
+        eev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_eager_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eev) / args.steps, world)
+    # the gather: a Reindex layer's attention launch (512 listed entries + 128 window tokens per row)
+    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        gev[i][0].record(stream)
+        wl.attention(1)
+        gev[i][1].record(stream)
+    torch.cuda.synchronize()
+    gather_ms = sum(a.elapsed_time(b) for a, b in gev) / args.steps
     assert wl.k.csa2_check(wl.err) == 0
 
     peak, peak_kind = peaks()
+    gather_gbs = wl.gather_bytes() / (gather_ms * 1e-3) / 1e9
+    gather = {"kernel": "csa2 sparse attention + SWA + merge (one layer, one launch)",
+              "bytes_per_launch": wl.gather_bytes(), "achieved": gather_gbs, "peak": peak, "peak_kind": peak_kind,
+              "unit": "GB/s", "frac": gather_gbs / peak, "launch_us": gather_ms * 1e3,
+              "timing": "isolated launches, L2 flushed before each"}
     achieved = wl.scan_bytes() / (scan_ms * 1e-3) / 1e9
     traffic = profiled_traffic(["compressed_sparse_attention_score_b200/csrc/index_mma.cu"],
                                "index_score_hier1m.md")
@@ -457,8 +823,12 @@ def main():
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "scan_ms": scan_ms,
                          "entries_scanned_per_s": wl.B * wl.N / (scan_ms * 1e-3)},
+            "gather": gather,
             "e2e": {"value": units / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "e2e_eager": {"value": units / (e2e_eager_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                          "d2h_bytes_per_step": d2h, "ms_per_step": e2e_eager_ms,
+                          "launch": "every call through the C ABI from Python, no graph replay"},
             "gpu_launches": wl.launches_per_step() * args.steps,
             "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

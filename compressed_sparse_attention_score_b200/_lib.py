@@ -38,7 +38,22 @@ class csa2_cache(ctypes.Structure):
                 ("seq_stride", c_int32), ("page_size", c_int32), ("max_pages", c_int32)]
 
 
+class csa2_layer_plan(ctypes.Structure):
+    _fields_ = [("mode", c_int32), ("source", c_int32), ("cache", c_int32)]
+
+
+class csa2_decode_args(ctypes.Structure):
+    _fields_ = [("n_layers", c_int32), ("plan", c_void_p), ("n_caches", c_int32), ("caches", c_void_p),
+                ("max_entries", c_void_p), ("B", c_int32), ("pos", c_void_p), ("softmax_scale", c_float),
+                ("k", c_int32), ("pool_k", c_int32), ("q", c_void_p), ("q_ix", c_void_p), ("w", c_void_p),
+                ("new_kv", c_void_p), ("new_ix", c_void_p), ("kv_stage", c_void_p), ("swa_x", c_void_p),
+                ("swa_codes", c_void_p), ("swa_scale", c_void_p), ("R", c_int32), ("window", c_int32),
+                ("idx", c_void_p), ("pool", c_void_p), ("o", c_void_p), ("lse", c_void_p)]
+
+
+LAYER_SWA = 4
 _P = ctypes.POINTER(csa2_cache)
+_PD = ctypes.POINTER(csa2_decode_args)
 _SIGS = {
     "csa2_version": ([], ctypes.c_int),
     "csa2_last_error_string": ([], ctypes.c_char_p),
@@ -63,6 +78,13 @@ _SIGS = {
     "csa2_sparse_attn_noalloc": ([ctypes.c_int, c_void_p, c_int32, c_int32, c_void_p, c_float, c_void_p, c_void_p,
                                   c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int32, _P, c_void_p, c_void_p,
                                   c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_void_p], ctypes.c_int),
+    "csa2_append_kv": ([c_void_p, c_void_p, ctypes.c_int, c_int32, c_void_p, c_void_p, _P, c_void_p, c_void_p],
+                       ctypes.c_int),
+    "csa2_plan_v41": ([c_void_p, c_int32, c_void_p], c_int32),
+    "csa2_pack_kv_gated": ([c_void_p, c_void_p, ctypes.c_int, c_void_p, c_void_p, c_int32, c_int32, c_void_p, _P,
+                           c_void_p, c_void_p], ctypes.c_int),
+    "csa2_decode_workspace_size": ([_PD], c_size_t),
+    "csa2_decode_step": ([_PD, c_void_p, c_size_t, c_void_p, c_void_p], ctypes.c_int),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -264,3 +286,64 @@ def csa2_merge(o1, l1, o2, l2, o=None, lse=None, stream=None):
     _ok(_lib.csa2_merge(_ptr(o1), _ptr(l1), _ptr(o2), _ptr(l2), rows, D, _ptr(o), _ptr(lse), _stream(stream)),
         "csa2_merge")
     return o, lse
+
+
+def csa2_append_kv(lat_kv, lat_ix, pos, cache, stage=None, err=None, stream=None):
+    """Append one token per sequence (lat_kv [B][512], lat_ix [B][128]) at positions pos [B]."""
+    B = lat_kv.shape[0]
+    assert lat_kv.shape[-1] == MAIN_DIM and lat_ix.shape[-1] == IX_DIM and lat_ix.dtype == lat_kv.dtype
+    d = cache.desc()
+    _ok(_lib.csa2_append_kv(_ptr(lat_kv), _ptr(lat_ix), DTYPE[lat_kv.dtype], B, _ptr(pos), _ptr(stage),
+                            ctypes.byref(d), _ptr(err), _stream(stream)), "csa2_append_kv")
+
+
+def csa2_pack_kv_gated(lat_kv, lat_ix, gate_kv, gate_ix, first_entry, cache, err=None, stream=None):
+    """csa2_pack_kv with per-channel softmax gates over each entry's tokens (gate_* fp32, shaped like lat_*)."""
+    B, T = lat_kv.shape[0], lat_kv.shape[1]
+    assert gate_kv.shape == lat_kv.shape and gate_ix.shape == lat_ix.shape and gate_kv.dtype == torch.float32
+    d = cache.desc()
+    _ok(_lib.csa2_pack_kv_gated(_ptr(lat_kv), _ptr(lat_ix), DTYPE[lat_kv.dtype], _ptr(gate_kv), _ptr(gate_ix), B, T,
+                                _ptr(first_entry), ctypes.byref(d), _ptr(err), _stream(stream)),
+        "csa2_pack_kv_gated")
+
+
+def csa2_plan_v41():
+    """The pages' 40-layer plan: ([(mode, source, cache)] * 40, ratios of its 4 caches)."""
+    n = _lib.csa2_plan_v41(None, 0, None)
+    plan = (csa2_layer_plan * n)()
+    ratios = (c_int32 * 4)()
+    assert _lib.csa2_plan_v41(plan, n, ratios) == n
+    return [(p.mode, p.source, p.cache) for p in plan], list(ratios)
+
+
+class DecodeStep:
+    """Descriptor of csa2_decode_step over caller-owned device tensors (marshalling only).
+
+    plan: [(mode, source, cache)] per layer (mode: a MODE value or LAYER_SWA); caches: GlobalKVCache
+    per cache id; max_entries: per cache.  Tensors are layer-major as csa2.h describes.
+    """
+
+    def __init__(self, plan, caches, max_entries, pos, softmax_scale, k, pool_k, q, swa_x, swa_codes, swa_scale,
+                 idx, o, lse, q_ix=None, w=None, pool=None, new_kv=None, new_ix=None, kv_stage=None, window=128):
+        L, nc = len(plan), len(caches)
+        self._plan = (csa2_layer_plan * L)(*[csa2_layer_plan(*p) for p in plan])
+        self._caches = (csa2_cache * max(nc, 1))(*[c.desc() for c in caches])
+        self._maxe = (c_int32 * max(nc, 1))(*max_entries)
+        self._keep = (caches, pos, q, swa_x, swa_codes, swa_scale, idx, o, lse, q_ix, w, pool, new_kv, new_ix, kv_stage)
+        a = csa2_decode_args()
+        a.n_layers, a.plan = L, ctypes.addressof(self._plan)
+        a.n_caches, a.caches, a.max_entries = nc, ctypes.addressof(self._caches), ctypes.addressof(self._maxe)
+        a.B, a.pos, a.softmax_scale, a.k, a.pool_k = q.shape[1], _ptr(pos), float(softmax_scale), k, pool_k
+        a.q, a.q_ix, a.w = _ptr(q), _ptr(q_ix), _ptr(w)
+        a.new_kv, a.new_ix, a.kv_stage = _ptr(new_kv), _ptr(new_ix), _ptr(kv_stage)
+        a.swa_x, a.swa_codes, a.swa_scale = _ptr(swa_x), _ptr(swa_codes), _ptr(swa_scale)
+        a.R, a.window = swa_codes.shape[2], window
+        a.idx, a.pool, a.o, a.lse = _ptr(idx), _ptr(pool), _ptr(o), _ptr(lse)
+        self.args = a
+
+    def workspace_size(self):
+        return _lib.csa2_decode_workspace_size(ctypes.byref(self.args))
+
+    def run(self, ws, err=None, stream=None):
+        _ok(_lib.csa2_decode_step(ctypes.byref(self.args), _ptr(ws), 0 if ws is None else ws.numel(), _ptr(err),
+                                  _stream(stream)), "csa2_decode_step")

@@ -101,8 +101,23 @@ CSA2_EXPORT csa2_status csa2_pack_kv(const void *lat_kv, const void *lat_ix, csa
   if (!lat_kv || !lat_ix || !first_entry) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (dtype != CSA2_F32 && dtype != CSA2_BF16) return fail(CSA2_ERR_INVALID_ARG, "bad dtype");
   if (!aligned16(lat_kv) || (reinterpret_cast<uintptr_t>(lat_ix) & 7)) return fail(CSA2_ERR_INVALID_ARG, "latents misaligned");
-  csa2::launch_pack_kv(lat_kv, lat_ix, dtype, pool_w, B, T, first_entry, *cache, err, stream);
+  csa2::launch_pack_kv(lat_kv, lat_ix, dtype, pool_w, nullptr, nullptr, B, T, first_entry, *cache, err, stream);
   return launched("csa2_pack_kv");
+}
+
+CSA2_EXPORT csa2_status csa2_pack_kv_gated(const void *lat_kv, const void *lat_ix, csa2_dtype dtype,
+                                           const float *gate_kv, const float *gate_ix, int32_t B, int32_t T,
+                                           const int32_t *first_entry, const csa2_cache *cache, int32_t *err,
+                                           csa2_stream_t stream) {
+  if (B < 0 || T < 0) return fail(CSA2_ERR_INVALID_ARG, "negative size");
+  if (B == 0 || T == 0) return CSA2_OK;
+  if (csa2_status s = check_cache(cache, B)) return s;
+  if (!lat_kv || !lat_ix || !gate_kv || !gate_ix || !first_entry) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
+  if (dtype != CSA2_F32 && dtype != CSA2_BF16) return fail(CSA2_ERR_INVALID_ARG, "bad dtype");
+  if (!aligned16(lat_kv) || (reinterpret_cast<uintptr_t>(lat_ix) & 7) || !aligned16(gate_kv) || !aligned16(gate_ix))
+    return fail(CSA2_ERR_INVALID_ARG, "latents or gates misaligned");
+  csa2::launch_pack_kv(lat_kv, lat_ix, dtype, nullptr, gate_kv, gate_ix, B, T, first_entry, *cache, err, stream);
+  return launched("csa2_pack_kv_gated");
 }
 
 CSA2_EXPORT csa2_status csa2_pack_swa(const void *x, csa2_dtype dtype, int32_t B, int32_t T, const int32_t *pos,
@@ -113,7 +128,7 @@ CSA2_EXPORT csa2_status csa2_pack_swa(const void *x, csa2_dtype dtype, int32_t B
   if (!x || !pos || !swa_codes || !swa_scale) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
   if (dtype != CSA2_F32 && dtype != CSA2_BF16) return fail(CSA2_ERR_INVALID_ARG, "bad dtype");
   if (!aligned16(x) || !aligned16(swa_codes)) return fail(CSA2_ERR_INVALID_ARG, "x / swa_codes misaligned");
-  csa2::launch_pack_swa(x, dtype, B, T, pos, swa_codes, swa_scale, R, err, stream);
+  csa2::launch_pack_swa(x, dtype, B, T, pos, B, swa_codes, swa_scale, R, err, stream);
   return launched("csa2_pack_swa");
 }
 

@@ -65,7 +65,8 @@ constexpr int AM_QU = AM_HG * (D / 8) / AM_PRODUCERS;   // 16-byte query chunks 
 constexpr int SM_RED = SM_PV + AM_MAXKEYS * 4;       // [4 warps][32 heads]; [CS][32] weights + [32] sums
 constexpr int SM_HM = SM_RED + (AM_MAXCS + 1) * 32 * 4;   // head max [32], head sum [32]
 constexpr int SM_QS = SM_HM + 2 * 32 * 4;            // query prescale: [8 warps][AM_QU] max bits, [32] 2^-s
-constexpr int SM_BAR = SM_QS + (8 * AM_QU + 32) * 4;
+constexpr int SM_NEW = SM_QS + (8 * AM_QU + 32) * 4; // this step's window token: 512 codes, scale, [4] maxima
+constexpr int SM_BAR = SM_NEW + 512 + 32;
 constexpr int SM_MISC = SM_BAR + 8 * (2 * AM_STAGES + 1);
 constexpr int SM_TOTAL = SM_MISC + 16;
 constexpr size_t AM_SMEM = SM_TOTAL + 1024;
@@ -83,10 +84,12 @@ struct AttnArgs {
   int dense, e0, e1;
   int n_bound;  // dense: entries a query may see (more sets CSA2_ERR_SHAPE)
   csa2_cache c;
-  // window source (codes == nullptr: none)
+  // window source (codes == nullptr: none); with swa_new [rows][512] bf16, this step's token of
+  // each row is quantised in the launch, used as the window's last key and stored in the ring
   const uint8_t *codes;
   const float *scale;
   int R, window;
+  const uint16_t *swa_new;
   float *o, *lse;
   int32_t *err;
 };
@@ -154,25 +157,67 @@ __device__ __forceinline__ void store_query_fp16(const uint4 (&qraw)[AM_QU], con
 
 // Gather the raw bytes of local key tile t into shared memory (asynchronous 16-byte
 // copies by the producer threads, committed as one group): a listed entry's 256 code bytes and 32 scale bytes
-// at offsets 0 and 256 of its row, a window token's 512 codes at offset 0.
-__device__ __forceinline__ void gather_tile(const AttnArgs &p, const int64_t *slot, int nks, int key0, int t,
-                                            uint32_t raw) {
+// at offsets 0 and 256 of its row, a window token's 512 codes at offset 0.  With new_codes, the
+// row's last key (this step's own window token, nk - 1) is copied from there instead.
+__device__ __forceinline__ void gather_tile(const AttnArgs &p, const int64_t *slot, int nks, int nk, int key0, int t,
+                                            uint8_t *raw, const uint8_t *new_codes) {
+  const uint32_t raw_s = smem_u32(raw);
   for (int i = threadIdx.x; i < AM_TILE * 32; i += AM_PRODUCERS) {
     const int kt = i & (AM_TILE - 1), piece = i >> 7;  // consecutive threads: consecutive keys
     const int key = t * AM_TILE + kt;
     const int64_t s = slot[key];
     if (s < 0) continue;
-    const uint32_t dst = raw + kt * AM_RAW + piece * 16;
+    const uint32_t dst = raw_s + kt * AM_RAW + piece * 16;
     if (key0 + key < nks) {
       if (piece < 16)
         cp_async_16(dst, p.c.kv_codes + s * CSA2_MAIN_CODE_BYTES + piece * 16);
       else if (piece < 18)
         cp_async_16(dst, p.c.kv_scales + s * CSA2_MAIN_SCALE_BYTES + (piece - 16) * 16);
+    } else if (new_codes && key0 + key == nk - 1) {
+      *reinterpret_cast<uint4 *>(raw + kt * AM_RAW + piece * 16) =
+          *reinterpret_cast<const uint4 *>(new_codes + piece * 16);
     } else {
       cp_async_16(dst, p.codes + s * CSA2_SWA_DIM + piece * 16);
     }
   }
   cp_async_commit();
+}
+
+// This step's own window token of the CTA's query row, quantised exactly as pack_swa_kernel does
+// (fp32 scale = amax / 448, E4M3 codes, a zero result code 0): its 512 codes go to new_codes
+// (shared), its scale to *new_scale (shared); the CTA given `store` also writes both to the ring
+// slot of position pos, which no CTA of this launch reads (window slots are distinct mod R).
+// Called by every thread of the CTA; contains two __syncthreads.
+__device__ __forceinline__ void quantise_new_token(const AttnArgs &p, int row, int ring, int pos, bool store,
+                                                   uint8_t *new_codes, float *new_scale, float *red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+  float am = 0.f;
+  if (tid < 128) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p.swa_new + int64_t(row) * CSA2_SWA_DIM + 4 * tid);
+    v[0] = __uint_as_float(u.x << 16), v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(u.y << 16), v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    if (lane == 0) red[warp] = am;
+  }
+  __syncthreads();
+  const float s = __fdiv_rn(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])), 448.0f);
+  if (tid < 128) {
+    uint32_t w = 0;
+    if (s != 0.f) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w |= e4m3_code(__fdiv_rn(v[i], s)) << (8 * i);
+    }
+    reinterpret_cast<uint32_t *>(new_codes)[tid] = w;
+    const int64_t slot = int64_t(ring) * p.R + pos % p.R;
+    // the ring is the caller's writable per-layer SWA cache (given as const for the reading calls)
+    if (store) reinterpret_cast<uint32_t *>(const_cast<uint8_t *>(p.codes) + slot * CSA2_SWA_DIM)[tid] = w;
+    if (store && tid == 0) const_cast<float *>(p.scale)[slot] = s;
+    if (tid == 0) *new_scale = s;
+  }
+  __syncthreads();
 }
 
 // 32 fp16 values (4 x 16 bytes) of dims dim0 .. dim0+31 of one key from its raw row;
@@ -328,8 +373,8 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool producer = tid < AM_PRODUCERS, issuer = tid == AM_PRODUCERS;
-  const int row = blockIdx.x, hg = blockIdx.y;
-  const int b = row / p.Q;
+  const int row = blockIdx.x, hg = blockIdx.y;   // query row; its sequence b owns SWA ring b
+  const int lrow = row, b = row / p.Q, ring = b;
   const int pos = p.q_pos[row];
 
   // ---------------------------------------------------------------- key list
@@ -363,12 +408,17 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
     }
   }
+  // this step's own window token (the row's last key), quantised here and stored by one CTA
+  const bool own_token = p.swa_new && nkw > 0;
+  uint8_t *new_codes = own_token ? smem + SM_NEW : nullptr;
+  float *new_scale = reinterpret_cast<float *>(smem + SM_NEW + 512);
+  if (own_token) quantise_new_token(p, row, ring, pos, split == 0 && hg == 0, smem + SM_NEW, new_scale, new_scale + 4);
   for (int jl = tid; jl < ntiles * AM_TILE; jl += AM_THREADS) {
     const int j = key0 + jl;
     int64_t s = -1;
     float m = 0.f, pm = 0.f;
     if (j < nks) {
-      const int n = p.dense ? p.e0 + j : p.idx[int64_t(row) * p.k + j];
+      const int n = p.dense ? p.e0 + j : p.idx[int64_t(lrow) * p.k + j];
       if (n != -1) {
         if (n < -1 || n >= nvis) {
           report(p.err, CSA2_ERR_INDEX);
@@ -379,8 +429,8 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       }
       m = p.tau, pm = 1.f;
     } else if (j < nk) {
-      s = int64_t(b) * p.R + (lo + (j - nks)) % p.R;
-      const float sc = p.scale[s];
+      s = int64_t(ring) * p.R + (lo + (j - nks)) % p.R;
+      const float sc = (own_token && j == nk - 1) ? *new_scale : p.scale[s];
       m = p.tau * sc, pm = sc;
     }
     slot[jl] = s;
@@ -402,9 +452,9 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     mbar_init_fence();
   }
   __syncthreads();  // key list, query maxima and barriers ready
-  const uint32_t raw = smem_u32(smem + SM_RAW);
+  uint8_t *raw = smem + SM_RAW;
   if (producer) {
-    if (ntiles > 0) gather_tile(p, slot, nks, key0, 0, raw);
+    if (ntiles > 0) gather_tile(p, slot, nks, nk, key0, 0, raw, new_codes);
     store_query_fp16(qraw, qmx, qinv, smem + SM_Q);
   }
   fence_proxy_async_smem();
@@ -451,7 +501,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       if (t > 0) {
         aborted = producers_sync(aborted);  // every producer is past its reads of the previous raw tile
         if (aborted) break;
-        gather_tile(p, slot, nks, key0, t, raw);
+        gather_tile(p, slot, nks, nk, key0, t, raw, new_codes);
       }
       cp_async_wait<0>();
       aborted = producers_sync(aborted);
@@ -567,7 +617,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       if (ntiles > 1 && (jc & 1) == 0) {
         aborted = producers_sync(aborted);  // every producer is past its reads of the raw tile
         if (aborted) break;
-        gather_tile(p, slot, nks, key0, t, raw);
+        gather_tile(p, slot, nks, nk, key0, t, raw, new_codes);
         cp_async_wait<0>();
         aborted = producers_sync(aborted);
         if (aborted) break;
@@ -669,7 +719,8 @@ constexpr int T_PV = T_MU + AM_TILE * 4;
 constexpr int T_RED = T_PV + AM_TILE * 4;
 constexpr int T_HM = T_RED + 8 * 32 * 4;
 constexpr int T_QS = T_HM + 2 * 32 * 4;         // query prescale (as SM_QS)
-constexpr int T_BAR = T_QS + (8 * AM_QU + 32) * 4;   // full[8], qfull, phase_done
+constexpr int T_NEW = T_QS + (8 * AM_QU + 32) * 4;   // this step's window token (as SM_NEW)
+constexpr int T_BAR = T_NEW + 512 + 32;         // full[8], qfull, phase_done
 constexpr int T_MISC = T_BAR + 8 * 10;
 constexpr size_t T_SMEM = T_MISC + 16 + 1024;
 }  // namespace
@@ -694,7 +745,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   const bool producer = tid < AM_PRODUCERS, issuer = tid == AM_PRODUCERS;
   const int row = blockIdx.x, hg = blockIdx.y;
   const int split = int(cg::this_cluster().block_rank());
-  const int b = row / p.Q;
+  const int lrow = row, b = row / p.Q, ring = b;   // the row's sequence b owns SWA ring b
   const int pos = p.q_pos[row];
   const int nvis = (p.idx || p.dense) ? visible_entries(p.c, b, pos) : 0;
   const int nks = p.dense ? max(0, min(p.e1, nvis) - p.e0) : (p.idx ? p.k : 0);
@@ -708,6 +759,11 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   if (tid == 0 && p.dense && nvis > p.n_bound) report(p.err, CSA2_ERR_SHAPE);
   uint32_t *qmx = reinterpret_cast<uint32_t *>(smem + T_QS);
   float *qinv = reinterpret_cast<float *>(smem + T_QS + 8 * AM_QU * 4);
+  // this step's own window token (the row's last key), quantised here and stored by one CTA
+  const bool own_token = p.swa_new && nkw > 0;
+  const uint8_t *new_codes = smem + T_NEW;
+  float *new_scale = reinterpret_cast<float *>(smem + T_NEW + 512);
+  if (own_token) quantise_new_token(p, row, ring, pos, split == 0 && hg == 0, smem + T_NEW, new_scale, new_scale + 4);
 
   // ---------------------------------------------------------------- loads
   // Producer t: key t % 128, dims 256 (t / 128) .. +255.  The query block's loads go
@@ -728,7 +784,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
     float m = 0.f, pm = 0.f;
     if (j < nks) {
       sparse = true;
-      const int n = p.dense ? p.e0 + j : p.idx[int64_t(row) * p.k + j];
+      const int n = p.dense ? p.e0 + j : p.idx[int64_t(lrow) * p.k + j];
       if (n != -1) {
         if (n < -1 || n >= nvis) {
           if (half == 0) report(p.err, CSA2_ERR_INDEX);
@@ -745,10 +801,11 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
         rr[8] = *reinterpret_cast<const uint4 *>(p.c.kv_scales + s * CSA2_MAIN_SCALE_BYTES + half * 16);
       }
     } else if (j < nk) {
-      s = int64_t(b) * p.R + (lo + (j - nks)) % p.R;
-      const float sc = p.scale[s];
+      s = int64_t(ring) * p.R + (lo + (j - nks)) % p.R;
+      const bool own = own_token && j == nk - 1;
+      const float sc = own ? *new_scale : p.scale[s];
       m = p.tau * sc, pm = sc;
-      const uint4 *src = reinterpret_cast<const uint4 *>(p.codes + s * CSA2_SWA_DIM + half * 256);
+      const uint4 *src = reinterpret_cast<const uint4 *>((own ? new_codes : p.codes + s * CSA2_SWA_DIM) + half * 256);
 #pragma unroll
       for (int i = 0; i < 16; ++i) rr[i] = src[i];
     }
@@ -1003,13 +1060,13 @@ static int attn_clusters_fit() {
 int attn_dense_segment() { return attn_clusters_fit<16>() > 0 ? 8192 : 4096; }
 
 // Few query rows leave most SMs idle: then a cluster of CTAs (one per 128-key tile)
-// splits each row's keys and combines the partials through distributed shared memory.
-// A CTA holds at most 5 tiles (640 keys), so longer key sets (dense segments) always use
-// clusters of up to 16 CTAs.
+// splits each row's keys and combines the partials through distributed shared memory, as
+// long as all the rows' tiles fit in about two CTAs per SM.  A CTA holds at most 5 tiles
+// (640 keys), so longer key sets (dense segments) always use clusters of up to 16 CTAs.
 void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
                      bool dense, int e0, int e1, int n_bound, const csa2_cache *c, const uint8_t *codes,
-                     const float *scale,
-                     int R, int window, float *o, float *lse, int32_t *err, cudaStream_t st) {
+                     const float *scale, int R, int window, float *o, float *lse, int32_t *err, cudaStream_t st,
+                     const uint16_t *swa_new) {
   const int rows = B * Q;
   if (rows == 0) return;
   AttnArgs a{};
@@ -1017,11 +1074,11 @@ void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, floa
   a.idx = dense ? nullptr : idx, a.k = (idx && !dense) ? k : 0;
   a.dense = dense ? 1 : 0, a.e0 = e0, a.e1 = e1, a.n_bound = n_bound;
   if (c) a.c = *c;
-  a.codes = codes, a.scale = scale, a.R = R, a.window = window;
+  a.codes = codes, a.scale = scale, a.R = R, a.window = window, a.swa_new = codes ? swa_new : nullptr;
   a.o = o, a.lse = lse, a.err = err;
   const int nkeys = (dense ? max(0, e1 - e0) : a.k) + (codes ? window : 0);
   const int tiles = (nkeys + AM_TILE - 1) / AM_TILE;
-  int cs = rows * (H / AM_HG) <= 64 ? max(1, min(tiles, 5)) : 1;
+  int cs = int64_t(rows) * (H / AM_HG) * tiles <= 2 * sm_count() ? max(1, min(tiles, 5)) : 1;
   if (cs > 1 && cs == tiles) {  // one tile per CTA: the single-dequant form
     switch (cs) {
       case 2: launch_tile<2>(a, rows, st); return;

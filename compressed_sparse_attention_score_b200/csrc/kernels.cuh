@@ -35,19 +35,26 @@ inline int sm_count() {
   return cached[dev];
 }
 
-void launch_pack_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype, const float *pool_w, int B, int T,
-                    const int32_t *first_entry, const csa2_cache &c, int32_t *err, cudaStream_t st);
-void launch_pack_swa(const void *x, csa2_dtype dtype, int B, int T, const int32_t *pos, uint8_t *codes,
-                     float *scale, int R, int32_t *err, cudaStream_t st);
+void launch_pack_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype, const float *pool_w,
+                    const float *gate_kv, const float *gate_ix, int B, int T, const int32_t *first_entry,
+                    const csa2_cache &c, int32_t *err, cudaStream_t st);
+void launch_pack_swa(const void *x, csa2_dtype dtype, int B, int T, const int32_t *pos, int pos_rows,
+                     uint8_t *codes, float *scale, int R, int32_t *err, cudaStream_t st);
+// stage_stride: floats from one sequence's staging rows to the next (at least ratio * 640).
+void launch_append_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype, int B, const int32_t *pos,
+                      float *stage, int64_t stage_stride, const csa2_cache &c, int32_t *num_entries, int32_t *err,
+                      cudaStream_t st);
 void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
                             const int32_t *cand, int P, int n_out, const csa2_cache &c, float *scores, int32_t *err,
                             cudaStream_t st);
 void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int N, int k0, int32_t *idx0, float *val0,
                          int k1, int32_t *idx1, float *val1, const int32_t *map, cudaStream_t st);
+// swa_new [B*Q][512] bf16 (decode): each row's own window token, quantised inside the launch,
+// used as the window's last key and stored in the ring (codes / scale must then be writable).
 void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
                      bool dense, int e0, int e1, int n_bound, const csa2_cache *c, const uint8_t *codes,
-                     const float *scale,
-                     int R, int window, float *o, float *lse, int32_t *err, cudaStream_t st);
+                     const float *scale, int R, int window, float *o, float *lse, int32_t *err, cudaStream_t st,
+                     const uint16_t *swa_new = nullptr);
 // Entries per dense-attention launch (one cluster of at most 16 CTAs x 640 keys per row).
 int attn_dense_segment();
 void launch_merge(const float *o1, const float *l1, const float *o2, const float *l2, int64_t rows, int D_,

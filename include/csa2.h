@@ -143,6 +143,24 @@ csa2_status csa2_pack_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtyp
                          const csa2_cache *cache, int32_t *err, csa2_stream_t stream);
 
 /*
+ * csa2_pack_kv with a learned (gated) pooling: the encoder pools about two tokens
+ * per entry ("从V4到V4.1 Flash", section 编码器层) by a rule the pages do not give;
+ * this call reads it as a gated sum.  For each channel d of entry j,
+ *   x_d = sum over t in the group of softmax_t(g_t,d) * lat_t,d,
+ * the softmax taken over the group's r tokens: m = max g, e_t = exp(g_t,d - m),
+ * weights e_t / (sum of e, left to right), products summed left to right, every step
+ * one fp32 operation and exp evaluated by a fixed fp32 sequence (2^f by its degree-7
+ * Taylor polynomial after n = rint(x log2 e)), so the codes do not depend on a math
+ * library.  Then quantised as csa2_pack_kv.
+ *   gate_kv [B][T][512], gate_ix [B][T][128] fp32 gate logits (computed by the model);
+ *   the other arguments as csa2_pack_kv.  Equal logits give csa2_pack_kv's mean.
+ */
+csa2_status csa2_pack_kv_gated(const void *lat_kv, const void *lat_ix, csa2_dtype dtype,
+                               const float *gate_kv, const float *gate_ix, int32_t B, int32_t T,
+                               const int32_t *first_entry, const csa2_cache *cache, int32_t *err,
+                               csa2_stream_t stream);
+
+/*
  * SWA packer: per token an fp32 scale = amax / 448 and 512 E4M3 codes RNE(x / scale)
  * (saturating), stored in a per-layer ring at slot pos mod R.  ("DeepSeek V4.1 Flash
  * 深度解析", 本专栏篇目 "FP4 从权重走进 KV 缓存": the sliding-window cache stays FP8;
@@ -248,6 +266,97 @@ csa2_status csa2_swa_attn(const uint16_t *q, int32_t B, int32_t Q, const int32_t
  */
 csa2_status csa2_merge(const float *o1, const float *l1, const float *o2, const float *l2,
                        int64_t rows, int32_t D, float *o, float *lse, csa2_stream_t stream);
+
+/*
+ * Decode-time append of one token per sequence to a cache written at ratio r
+ * ("从V4到V4.1 Flash", section 编码器层: the encoder pools about two tokens per entry;
+ * section 解码器层: the decoder keeps ratio 1).  The token at position pos[b] is kept,
+ * in fp32, in row pos % r of the sequence's staging buffer; when it completes a group
+ * of r tokens, the group is pooled and packed exactly as csa2_pack_kv does (fp32, left
+ * to right, weight fp32(1/r)) into entry pos / r, and cache->num_entries[b] is raised
+ * to pos / r + 1 (this call writes num_entries on the device).
+ *   lat_kv [B][512], lat_ix [B][128] in `dtype`; pos [B] (negative: skip the row);
+ *   stage [B][r][640] fp32 (512 main then 128 indexer values), may be NULL when r = 1;
+ *   it carries the incomplete group from call to call.
+ * Device errors: an entry outside the cache -> CSA2_ERR_INDEX, skipped.
+ */
+csa2_status csa2_append_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype, int32_t B,
+                           const int32_t *pos, float *stage, const csa2_cache *cache, int32_t *err,
+                           csa2_stream_t stream);
+
+/*
+ * Multi-layer decode: one token per sequence through a stack of layers.
+ * ("DeepSeek-V4.1 模型结构（0）", Q&A "DeepSeek-V4.1-Flash 的 40 层具体如何排布？": layers
+ * 0-1 use only the sliding window, 2 / 8 / 14 / 20 are Full, 24 / 28 / 32 / 36 Reindex,
+ * the other 30 Reuse; 延伸解读 "CSA2 共享池": only the Full layers produce global KV;
+ * "从V4到V4.1 Flash", 解码器层: the decoder's first layer keeps a candidate pool that the
+ * later layers search.)
+ * A layer's plan: its mode (a csa2_mode or CSA2_LAYER_SWA), the earlier layer it takes
+ * its entries from (Reuse) or whose pool it searches (Reindex, a Full layer), and the
+ * global cache it reads (Full: the one it writes).
+ */
+#define CSA2_LAYER_SWA 4
+typedef struct {
+  int32_t mode;
+  int32_t source; /* -1 unless Reuse or Reindex */
+  int32_t cache;  /* index into the step's caches, -1 for CSA2_LAYER_SWA */
+} csa2_layer_plan;
+
+/*
+ * The pages' 40-layer plan into plan[0..39] (host) and, if cache_ratio (host [4]) is
+ * given, its caches' ratios: caches 0-2 are written by the encoder's Full layers 2, 8, 14
+ * at ratio 2, cache 3 by the decoder's Full layer 20 at ratio 1, whose pool the Reindex
+ * layers search; every Reuse layer takes the nearest earlier Full or Reindex layer's
+ * entries.  Returns 40 (and writes nothing when max_layers < 40).
+ */
+int32_t csa2_plan_v41(csa2_layer_plan *plan, int32_t max_layers, int32_t *cache_ratio);
+
+/*
+ * One decode step.  Host fields: n_layers, plan, n_caches, caches, max_entries and the
+ * sizes; every other pointer is device memory, layer-major.  For each layer l:
+ *   q [L][B][64][512], q_ix [L][B][64][128], w [L][B][64] bf16 (q_ix / w are read only
+ *   for Full and Reindex layers); swa_x [L][B][512] bf16, this token's hidden state for
+ *   the layer's ring swa_codes [L][B][R][512] / swa_scale [L][B][R] (quantised as
+ *   csa2_pack_swa does and stored by the layer's attention launch);
+ *   idx [L][B][k]: Full and Reindex layers write the entries they chose (a Reuse layer
+ *   attends its source's row); o [L][B][64][512], lse [L][B][64] fp32 as csa2_sparse_attn
+ *   with the window merged.
+ * Caches: new_kv [n_caches][B][512] and new_ix [n_caches][B][128] bf16 are this token's
+ * latents per cache (NULL: no append), appended as csa2_append_kv does before the first
+ * layer that reads the cache, with staging kv_stage [n_caches][B][rmax][640] fp32 (rmax =
+ * the largest ratio); pool [n_caches][B][pool_k] holds the pool of the cache's Full layer
+ * when a Reindex layer searches it.  max_entries [n_caches] (host) bounds each cache's
+ * entries after the append.
+ * The layers run in order, each with its own launches (a Full layer: indexer scan, top-k,
+ * attention; Reindex the same over the pool; Reuse and window-only layers: one attention
+ * launch), on `stream` without synchronising or allocating (capturable in a CUDA graph).
+ * Dense layers hold at most one segment (4096 entries).
+ */
+typedef struct {
+  int32_t n_layers;
+  const csa2_layer_plan *plan;
+  int32_t n_caches;
+  const csa2_cache *caches;
+  const int32_t *max_entries;
+  int32_t B;
+  const int32_t *pos; /* [B] position of this step's token */
+  float softmax_scale;
+  int32_t k, pool_k;
+  const uint16_t *q, *q_ix, *w;
+  const uint16_t *new_kv, *new_ix;
+  float *kv_stage;
+  const uint16_t *swa_x;
+  uint8_t *swa_codes;
+  float *swa_scale;
+  int32_t R, window;
+  int32_t *idx, *pool;
+  float *o, *lse;
+} csa2_decode_args;
+
+/* Workspace bytes csa2_decode_step needs (the largest layer's fp32 scores). */
+size_t csa2_decode_workspace_size(const csa2_decode_args *args);
+csa2_status csa2_decode_step(const csa2_decode_args *args, void *ws, size_t ws_bytes, int32_t *err,
+                             csa2_stream_t stream);
 
 /*
  * csa2_sparse_attn without a caller workspace.  (The pages have no counterpart:

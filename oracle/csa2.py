@@ -80,6 +80,56 @@ def compress(lat, ratio, pool_w=None):
     return out
 
 
+# Reading for a learned ("gated") compressor: [PRISM] 编码器层 says only that the encoder pools
+# about two tokens into an entry; the rule is a learned weighting the pages do not give.  Read
+# as a gated sum: per channel, the r tokens of a group are weighted by the softmax (over those
+# r tokens) of gate logits that the model computes and the caller supplies.  Every step is an
+# fp32 operation in a fixed order, exp included, so that the quantised codes are one answer.
+LOG2E_F32 = np.float32(1.4426950408889634)
+EXP2_TAYLOR_F32 = [np.float32(math.log(2) ** i / math.factorial(i)) for i in range(8)]
+
+
+def exp_fp32(x):
+    """exp(x) from fp32 operations: t = x log2(e), n = rint(t), f = t - n, 2^f = e^(f ln 2) by its
+    Taylor polynomial of degree 7 (Horner, each product and sum rounded), times 2^n (0 below
+    2^-126, inf above 2^127)."""
+    x = np.asarray(x, np.float32)
+    t = (x * LOG2E_F32).astype(np.float32)
+    n = np.rint(t).astype(np.float32)
+    f = (t - n).astype(np.float32)
+    p = np.full(x.shape, EXP2_TAYLOR_F32[7], np.float32)
+    for c in EXP2_TAYLOR_F32[6::-1]:
+        p = (p * f).astype(np.float32)
+        p = (p + c).astype(np.float32)
+    ni = n.astype(np.int64)
+    scale = np.ldexp(np.ones(x.shape, np.float32), np.clip(ni, -126, 127)).astype(np.float32)
+    out = (p * scale).astype(np.float32)
+    out = np.where(ni < -126, np.float32(0), out)
+    return np.where(ni > 127, np.float32(np.inf), out).astype(np.float32)
+
+
+def compress_gated(lat, gate, ratio):
+    """[T, d] latents and [T, d] gate logits -> [floor(T / r), d] entries: per channel the softmax
+    of the group's logits (max subtracted, exp_fp32, sum left to right, fp32 division) weights the
+    group's latents, summed left to right."""
+    lat = np.asarray(lat, dtype=np.float32)
+    gate = np.asarray(gate, dtype=np.float32)
+    n = lat.shape[0] // ratio
+    out = np.empty((n,) + lat.shape[1:], dtype=np.float32)
+    for j in range(n):
+        g = gate[j * ratio:(j + 1) * ratio]
+        e = exp_fp32((g - g.max(axis=0)).astype(np.float32))
+        den = e[0]
+        for t in range(1, ratio):
+            den = (den + e[t]).astype(np.float32)
+        acc = None
+        for t in range(ratio):
+            term = ((e[t] / den).astype(np.float32) * lat[j * ratio + t]).astype(np.float32)
+            acc = term if acc is None else (acc + term).astype(np.float32)
+        out[j] = acc
+    return out
+
+
 class Cache:
     """Logical per-sequence global KV planes (the oracle ignores physical paging)."""
 
@@ -235,4 +285,44 @@ def decode_layer(mode, cache, b, pos, q, tau, swa, window=128, q_ix=None, w=None
     out["idx"] = np.asarray(idx)
     out["sparse"] = (o1, l1)
     out["swa"] = (o2, l2)
+    return out
+
+
+# --------------------------------------------------------------------------- the layer stack
+# [XHH] Q&A "40 层具体如何排布" gives each layer's mode; 延伸解读 "CSA2 共享池": only the Full
+# layers produce global KV and the layers after them reuse it (Reuse also reuses the indices of
+# the nearest layer that selected them).  [PRISM] 解码器层: the decoder's first layer (the last
+# Full layer) keeps the candidate pool that the Reindex layers search.
+def pool_layer():
+    return max(FULL_LAYERS)
+
+
+def decode_model(caches, b, pos, layers, tau, k=512, pool_k=16384, window=128):
+    """One decode token of sequence b at position pos through the NUM_LAYERS layers.
+
+    caches: {Full layer -> Cache} (each Full layer's own global KV, written at its ratio);
+    layers[l]: dict with q [H, 512], swa = (codes [R, 512], scale [R]) and, for Full and Reindex
+    layers, q_ix [H_I, 128] and w [H_I].  Returns per layer the decode_layer dict plus "head"
+    (the layer whose entries it attends, or None for the sliding-window-only layers).
+    """
+    out = []
+    head, head_cache = None, None
+    for l in range(NUM_LAYERS):
+        mode, L = layer_mode(l), layers[l]
+        if mode == "swa":
+            o, lse = swa_attention(L["q"], pos, L["swa"][0], L["swa"][1], window, tau)
+            out.append({"o": o, "lse": lse, "idx": None, "pool": None, "head": None})
+            continue
+        if mode == "full":
+            head, head_cache = l, caches[l]
+            r = decode_layer("full", head_cache, b, pos, L["q"], tau, L["swa"], window, q_ix=L["q_ix"], w=L["w"],
+                             k=k, pool_k=pool_k if l == pool_layer() else 0)
+        elif mode == "reindex":
+            head, head_cache = l, caches[pool_layer()]
+            r = decode_layer("reindex", head_cache, b, pos, L["q"], tau, L["swa"], window, q_ix=L["q_ix"],
+                             w=L["w"], k=k, pool=out[pool_layer()]["pool"])
+        else:
+            r = decode_layer("reuse", head_cache, b, pos, L["q"], tau, L["swa"], window, idx=out[head]["idx"])
+        r["head"] = head
+        out.append(r)
     return out

@@ -645,3 +645,63 @@ def test_query_magnitudes_are_exact(case, B):
         c = oracle_seq(spec, b, main_rows=to_np(idx[b, 0]), gen_device=DEV)
         ref = OC.decode_layer("reuse", c, 0, int(q_pos[b, 0]), to_np(q[b, 0]), tau, rings[b], idx=to_np(idx[b, 0]))
         check_attention(to_np(o[b, 0]), to_np(lse[b, 0]), ref["o"], ref["lse"], f"{case} b={b}")
+
+
+# ------------------------------------------------------------------ gated compressor and decode-time append
+@pytest.mark.parametrize("ratio", [1, 2, 4, 128])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_pack_kv_gated_bit_exact(ratio, dtype):
+    k = K()
+    B, T = 2, 128 * 3 + 5 if ratio == 128 else 601
+    kv = _planted_latents(B, T, 512, 5, dtype)
+    ix = _planted_latents(B, T, 128, 6, dtype)
+    gkv = normal((B, T, 512), 0, "gate_kv", device=DEV) * 4
+    gix = normal((B, T, 128), 0, "gate_ix", device=DEV) * 4
+    gkv[0, : 2 * ratio] = 0.5                      # equal logits: the plain mean
+    gix[1, :ratio, :7] = 90.0                      # one dominant logit per channel
+    n = T // ratio
+    cache = k.GlobalKVCache(B, ratio, seq_stride=n + 3)
+    first = torch.tensor([0, 3], dtype=torch.int32, device=DEV)
+    err = _err()
+    k.csa2_pack_kv_gated(kv, ix, gkv, gix, first, cache, err=err)
+    assert k.csa2_check(err) == 0
+    for b in range(B):
+        mc, ms = OF.pack_main(OC.compress_gated(to_np(kv[b]), to_np(gkv[b]), ratio))
+        ic, isc = OF.pack_indexer(OC.compress_gated(to_np(ix[b]), to_np(gix[b]), ratio))
+        f = int(first[b])
+        sl = slice(b * (n + 3) + f, b * (n + 3) + f + n)
+        np.testing.assert_array_equal(to_np(cache.kv_codes[sl]), mc)
+        np.testing.assert_array_equal(to_np(cache.kv_scales[sl]), ms)
+        np.testing.assert_array_equal(to_np(cache.ix_codes[sl]), ic)
+        np.testing.assert_array_equal(to_np(cache.ix_scales[sl]), isc)
+
+
+@pytest.mark.parametrize("ratio", [1, 2, 4])
+def test_append_kv_token_by_token_equals_pack_kv(ratio):
+    """Appending tokens one decode step at a time (staging the incomplete group) writes the same
+    bytes and entry counts as packing the whole run at once, and as the oracle."""
+    k = K()
+    B, T = 2, 4 * 7 + 3
+    kv = _planted_latents(B, T, 512, 7, torch.bfloat16)
+    ix = _planted_latents(B, T, 128, 8, torch.bfloat16)
+    n = T // ratio
+    cache = k.GlobalKVCache(B, ratio, seq_stride=n + 1)
+    stage = torch.zeros((B, ratio, 640), dtype=torch.float32, device=DEV)
+    err = _err()
+    for t in range(T):
+        pos = torch.full((B,), t, dtype=torch.int32, device=DEV)
+        k.csa2_append_kv(kv[:, t].contiguous(), ix[:, t].contiguous(), pos, cache, stage=stage, err=err)
+        if t == T // 2:   # padding rows (negative positions) leave every sequence alone
+            k.csa2_append_kv(kv[:, 0].contiguous() * 7, ix[:, 0].contiguous() * 7,
+                             torch.full((B,), -1, dtype=torch.int32, device=DEV), cache, stage=stage, err=err)
+    assert k.csa2_check(err) == 0
+    assert to_np(cache.num_entries).tolist() == [n, n]
+    for b in range(B):
+        ekv, eix = OC.compress(to_np(kv[b]), ratio), OC.compress(to_np(ix[b]), ratio)
+        mc, ms = OF.pack_main(ekv)
+        ic, isc = OF.pack_indexer(eix)
+        sl = slice(b * (n + 1), b * (n + 1) + n)
+        np.testing.assert_array_equal(to_np(cache.kv_codes[sl]), mc)
+        np.testing.assert_array_equal(to_np(cache.kv_scales[sl]), ms)
+        np.testing.assert_array_equal(to_np(cache.ix_codes[sl]), ic)
+        np.testing.assert_array_equal(to_np(cache.ix_scales[sl]), isc)

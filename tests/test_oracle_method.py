@@ -83,6 +83,44 @@ def test_compressor_weighted_sum_brute_force():
             assert out[j, d] == acc
 
 
+def test_fixed_exp_against_the_exponential():
+    """exp_fp32 is exp within its rounding bound (argument reduction in fp32: about 2^-23 (1 + |x|)),
+    exactly 1 at 0, 0 below the fp32 normal range."""
+    rng = np.random.default_rng(3)
+    x = np.concatenate([-np.abs(rng.normal(size=50000)) * 30, -rng.uniform(0, 1, 50000), [0.0, -1e-30]])
+    x = x.astype(np.float32)
+    e = C.exp_fp32(x)
+    ref = np.exp(x.astype(np.float64))
+    ok = ref > 2.0 ** -126
+    assert np.all(np.abs(e[ok] - ref[ok]) <= 1.5e-7 * (1 + np.abs(x[ok])) * ref[ok])
+    assert C.exp_fp32(np.float32(0)) == 1.0 and C.exp_fp32(np.float32(-200)) == 0.0
+    assert C.exp_fp32(np.float32(-1e-30)) == 1.0
+
+
+def test_gated_compressor_reductions():
+    """Equal logits give the plain mean (compress, bit for bit); one dominant logit per channel picks
+    that token's latent exactly; weights of a group sum to one."""
+    rng = np.random.default_rng(4)
+    for r in (1, 2, 4):
+        x = rng.normal(size=(5 * r + r - 1, 24)).astype(np.float32)   # a ragged tail makes no entry
+        g = np.full_like(x, 0.7)
+        np.testing.assert_array_equal(C.compress_gated(x, g, r), C.compress(x, r))
+        pick = rng.integers(0, r, size=24)
+        g = np.zeros_like(x)
+        for j in range(5):
+            g[j * r + pick, np.arange(24)] = 200.0
+        want = np.stack([x[j * r + pick, np.arange(24)] for j in range(5)])
+        np.testing.assert_array_equal(C.compress_gated(x, g, r), want)
+    # general logits: a convex combination, per channel, of the group's tokens
+    x = rng.normal(size=(12, 8)).astype(np.float32)
+    g = rng.normal(size=(12, 8)).astype(np.float32) * 3
+    out = C.compress_gated(x, g, 3)
+    for j in range(4):
+        w = np.exp(g[3 * j:3 * j + 3].astype(np.float64))
+        w /= w.sum(axis=0)
+        np.testing.assert_allclose(out[j], (w * x[3 * j:3 * j + 3]).sum(axis=0), rtol=1e-5, atol=1e-6)
+
+
 def test_prefill_entry_count():
     # a 262144-token prefix plus an 8192-token chunk at ratio 2
     assert 262144 // 2 == 131072 and 8192 // 2 == 4096
@@ -360,3 +398,89 @@ def test_decode_layer_is_one_softmax_over_entries_and_window(mode):
     bo, bl = brute_attend(q.tolist(), keys, tau)
     np.testing.assert_allclose(out["o"], bo, rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(out["lse"], bl, rtol=1e-12)
+
+
+# ----------------------------------------------------------------- the 40-layer stack
+def _tiny_model(seed=31, T=120, H=2, HI=3, R=8):
+    """Four small caches (one per Full layer, at its ratio) and per-layer inputs at position T - 1."""
+    rng = np.random.default_rng(seed)
+    caches = {}
+    for layer, r in C.FULL_LAYERS.items():
+        cache = C.Cache(1, T // r + 2, r)
+        kv = rng.normal(size=(T, 512)).astype(np.float32)
+        ix = rng.normal(size=(T, 128)).astype(np.float32)
+        cache.num_entries[0] = cache.pack(0, 0, kv, ix)
+        caches[layer] = cache
+    pos = T - 1
+    layers = []
+    for _ in range(C.NUM_LAYERS):
+        codes, scale = np.zeros((R, 512), np.uint8), np.zeros(R, np.float32)
+        for t in range(pos - R + 1, pos + 1):
+            codes[t % R], scale[t % R] = F.pack_swa(rng.normal(size=512).astype(np.float32))
+        layers.append({"q": rng.normal(size=(H, 512)), "q_ix": rng.normal(size=(HI, 128)).astype(np.float32),
+                       "w": rng.uniform(size=HI).astype(np.float32), "swa": (codes, scale)})
+    return caches, pos, layers
+
+
+def test_decode_model_follows_the_layer_schedule():
+    """Every layer of the stack against brute force: the window-only layers, each Full layer's
+    own selection over its own cache, the pool of the decoder's Full layer, each Reindex layer's
+    selection inside that pool, and every layer's output as one softmax over the entries of the
+    nearest earlier selecting layer (from that layer's cache) plus its window."""
+    caches, pos, layers = _tiny_model()
+    k, pool_k, W, tau = 6, 20, 5, 0.05
+    out = C.decode_model(caches, 0, pos, layers, tau, k=k, pool_k=pool_k, window=W)
+    assert len(out) == C.NUM_LAYERS == 40
+    brute_s = {}
+    head = None
+    for layer in range(C.NUM_LAYERS):
+        L, m = layers[layer], C.layer_mode(layer)
+        win = _brute_window_keys(L["swa"][0], L["swa"][1], pos, W)
+        if m == "swa":
+            bo, bl = brute_attend(L["q"].tolist(), win, tau)
+            np.testing.assert_allclose(out[layer]["o"], bo, rtol=1e-11, atol=1e-12)
+            continue
+        if m == "full":
+            cache = caches[layer]
+            vis = cache.visible(0, pos)
+            keys = F.unpack_indexer(cache.ix_codes[0, :vis], cache.ix_scales[0, :vis])
+            s = list(brute_scores(L["q_ix"], L["w"], keys))
+            np.testing.assert_array_equal(out[layer]["idx"], brute_topk(s, k))
+            if layer == 20:
+                np.testing.assert_array_equal(out[layer]["pool"], brute_topk(s, pool_k))
+            head, head_cache = layer, cache
+        elif m == "reindex":
+            cache = caches[20]
+            pool = out[20]["pool"]
+            keys = F.unpack_indexer(cache.ix_codes[0, pool], cache.ix_scales[0, pool])
+            s = list(brute_scores(L["q_ix"], L["w"], keys))
+            want = [int(pool[j]) if j >= 0 else -1 for j in brute_topk(s, k)]
+            np.testing.assert_array_equal(out[layer]["idx"], want)
+            head, head_cache = layer, cache
+        assert out[layer]["head"] == head
+        listed = [j for j in out[head]["idx"].tolist() if j >= 0]
+        main = F.unpack_main(head_cache.kv_codes[0, listed], head_cache.kv_scales[0, listed]).tolist()
+        bo, bl = brute_attend(L["q"].tolist(), main + win, tau)
+        np.testing.assert_allclose(out[layer]["o"], bo, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(out[layer]["lse"], bl, rtol=1e-12)
+        brute_s[layer] = True
+    assert len(brute_s) == 38                       # every CSA2 layer checked
+
+
+def test_library_plan_is_the_pages_schedule():
+    """csa2_plan_v41 (host code of the library, no GPU) against the oracle's schedule."""
+    from compressed_sparse_attention_score_b200 import build
+    build.build()
+    import compressed_sparse_attention_score_b200 as K
+    plan, ratios = K.csa2_plan_v41()
+    names = {0: "full", 1: "reindex", 2: "reuse", K.LAYER_SWA: "swa"}
+    assert [names[m] for m, _, _ in plan] == [C.layer_mode(i) for i in range(C.NUM_LAYERS)]
+    full = sorted(C.FULL_LAYERS)
+    assert [plan[f][2] for f in full] == [0, 1, 2, 3]
+    assert ratios == [C.FULL_LAYERS[f] for f in full]
+    for i, (m, src, cache) in enumerate(plan):
+        if names[m] == "reuse":          # the nearest earlier Full or Reindex layer
+            want = max(j for j in range(i) if C.layer_mode(j) in ("full", "reindex"))
+            assert src == want and cache == plan[want][2]
+        if names[m] == "reindex":
+            assert src == C.pool_layer() and cache == plan[C.pool_layer()][2]

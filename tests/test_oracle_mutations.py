@@ -122,6 +122,41 @@ def test_layer_with_the_default_window_is_caught(monkeypatch):
     _fails(TM.test_decode_layer_is_one_softmax_over_entries_and_window, "full")
 
 
+def test_gate_softmax_over_channels_is_caught(monkeypatch):
+    def over_channels(lat, gate, ratio):
+        lat, gate = np.asarray(lat, np.float32), np.asarray(gate, np.float32)
+        n = lat.shape[0] // ratio
+        out = np.empty((n,) + lat.shape[1:], np.float32)
+        for j in range(n):
+            g = gate[j * ratio:(j + 1) * ratio]
+            e = C.exp_fp32((g - g.max(axis=1, keepdims=True)).astype(np.float32))
+            w = (e / e.sum(axis=1, keepdims=True)).astype(np.float32)
+            out[j] = (w * lat[j * ratio:(j + 1) * ratio]).sum(axis=0).astype(np.float32)
+        return out
+    monkeypatch.setattr(C, "compress_gated", over_channels)
+    _fails(TM.test_gated_compressor_reductions)
+
+
+def test_stack_reusing_the_wrong_layer_is_caught(monkeypatch):
+    orig = C.decode_layer
+
+    def first_full(mode, cache, b, pos, q, tau, swa, window=128, **kw):
+        if mode == "reuse" and "idx" in kw:   # every Reuse layer takes layer 2's entries instead
+            kw["idx"] = first_full.layer2
+        r = orig(mode, cache, b, pos, q, tau, swa, window, **kw)
+        if mode == "full" and not hasattr(first_full, "layer2"):
+            first_full.layer2 = r["idx"]
+        return r
+    monkeypatch.setattr(C, "decode_layer", first_full)
+    _fails(TM.test_decode_model_follows_the_layer_schedule)
+
+
+def test_stack_without_the_decoder_pool_is_caught(monkeypatch):
+    monkeypatch.setattr(C, "pool_layer", lambda: 2)
+    with pytest.raises((AssertionError, TypeError, IndexError)):
+        TM.test_decode_model_follows_the_layer_schedule()
+
+
 def test_layer_that_skips_its_listed_entries_is_caught(monkeypatch):
     monkeypatch.setattr(C, "sparse_attention", lambda cache, b, q, idx, tau: C.attend(q, np.zeros((0, 512)), tau))
     _fails(TM.test_decode_layer_is_one_softmax_over_entries_and_window, "reindex")

@@ -88,8 +88,23 @@ def mixed64(seed=0):
                 lat_dtype=torch.bfloat16, seed=seed)
 
 
+def model40(seed=0):
+    """One decode token of 8 sequences at 2^20 tokens through the pages' 40-layer stack: four caches
+    (three encoder caches at ratio 2, the decoder's at ratio 1, 16384-entry pool), each with the
+    planted 2 % indexer cluster of hier1m."""
+    return Spec("model40", 8, [1 << 20] * 8, 1, "model", pool_k=16384, cluster_frac=0.02,
+                lat_dtype=torch.bfloat16, seed=seed)
+
+
 CONFIGS = {"tiny_full": tiny_full, "reuse64k": reuse64k, "hier1m": hier1m, "prefill8k": prefill8k,
-           "mixed64": mixed64}
+           "mixed64": mixed64, "model40": model40}
+
+
+def cache_spec(spec, cache, ratio, shares_queries=False):
+    """The latent recipe of one of a layer stack's caches (its own draws, its own ratio).  The cache
+    that shares_queries keeps the stack's own draws, so its planted cluster is the one the
+    indexer queries of query_tensors lean towards."""
+    return replace(spec, name=spec.name if shares_queries else f"{spec.name}-cache{cache}", ratio=ratio)
 
 
 def scaled(spec, tokens, B=None, **kw):
