@@ -1059,10 +1059,10 @@ static int attn_clusters_fit() {
 
 int attn_dense_segment() { return attn_clusters_fit<16>() > 0 ? 8192 : 4096; }
 
-// Few query rows leave most SMs idle: then a cluster of CTAs (one per 128-key tile)
-// splits each row's keys and combines the partials through distributed shared memory, as
-// long as all the rows' tiles fit in about two CTAs per SM.  A CTA holds at most 5 tiles
-// (640 keys), so longer key sets (dense segments) always use clusters of up to 16 CTAs.
+// Up to 64 query rows: a cluster of CTAs (one per 128-key tile) splits each row's keys and
+// combines the partials through distributed shared memory (a few waves of one-tile CTAs finish
+// sooner than one wave of CTAs that take every tile of a row in turn).  A CTA holds at most 5
+// tiles (640 keys), so longer key sets (dense segments) always use clusters of up to 16 CTAs.
 void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
                      bool dense, int e0, int e1, int n_bound, const csa2_cache *c, const uint8_t *codes,
                      const float *scale, int R, int window, float *o, float *lse, int32_t *err, cudaStream_t st,
@@ -1078,7 +1078,7 @@ void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, floa
   a.o = o, a.lse = lse, a.err = err;
   const int nkeys = (dense ? max(0, e1 - e0) : a.k) + (codes ? window : 0);
   const int tiles = (nkeys + AM_TILE - 1) / AM_TILE;
-  int cs = int64_t(rows) * (H / AM_HG) * tiles <= 2 * sm_count() ? max(1, min(tiles, 5)) : 1;
+  int cs = rows * (H / AM_HG) <= 128 ? max(1, min(tiles, 5)) : 1;
   if (cs > 1 && cs == tiles) {  // one tile per CTA: the single-dequant form
     switch (cs) {
       case 2: launch_tile<2>(a, rows, st); return;

@@ -6,10 +6,10 @@
 // are consumed exactly as stored (kind::mxf4, scale vector 32), so the products
 // are exact and only the fp32 accumulation order differs from a plain sum.
 //
-// CTA = one query row x a set of key tiles.  Row m of a tile's A operand holds tile
-// entry e(m) = (m % 32) * 4 + m / 32, so the entries' scale words, copied in their
-// natural order, form the 32 x 4-word scale-factor atom that tcgen05.cp expects
-// (word w = (m % 32) * 4 + m / 32 = e).  Warp roles:
+// CTA = one query row x a contiguous range of key tiles.  Row m of a tile's A
+// operand holds tile entry e(m) = (m % 32) * 4 + m / 32, so the entries' scale
+// words, copied in their natural order, form the 32 x 4-word scale-factor atom
+// that tcgen05.cp expects (word w = (m % 32) * 4 + m / 32 = e).  Warp roles:
 //   warp 0     producer: for a run of whole 128-entry groups one TMA box of a
 //              4-D tensor map whose outer strides perform the row permutation
 //              (64-byte swizzle) plus one 512-byte bulk copy of the scales;
@@ -19,13 +19,6 @@
 //   warps 2-9  epilogue, two warpgroups taking alternate tiles: tcgen05.ld of
 //              the 64 head values of its 32 keys, weighted ReLU sum, fp32 score
 //              store.
-// Tile schedule: candidate lists and long batches give each CTA one contiguous run
-// of tiles.  Full scans of a few rows (decode) are scheduled dynamically: the CTAs of
-// a row take chunks of IM_CHUNK tiles from the row's counter until the row is done, so
-// CTAs that stream faster take more chunks and the scan ends evenly.  The producer
-// takes each chunk and publishes it to the other roles through a ring of chunk slots
-// with one mbarrier each; the counters live in a static device array, one set per
-// launch slot, and the launch's last CTA clears its set for the next launch.
 // The query heads are quantised to MXFP4 in the prologue (warps 2-5; same codec as
 // the keys).
 // Every mbarrier wait is time-bounded; on expiry the CTA drains and reports
@@ -33,7 +26,6 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <atomic>
 #include <cstring>
 
 #include "common.cuh"
@@ -57,30 +49,18 @@ constexpr uint32_t COL_SFA = IM_ACC * 64;   // one 4-column scale buffer per acc
 constexpr uint32_t COL_SFB = COL_SFA + 4 * IM_ACC;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
-// Dynamic schedule: chunks of IM_CHUNK tiles, published through IM_INFO chunk slots.  The
-// producer runs at most IM_STAGES + IM_ACC tiles ahead of the slowest epilogue, far less than
-// the ring, so a slot is never reused before every role has read it.
-constexpr int IM_CHUNK = 4;
-constexpr int IM_INFO = 16;
-constexpr int IM_DYN_SLOTS = 64;       // launch slots of row counters
-constexpr int IM_DYN_ROWS = 64;        // rows a dynamic launch may have
-
 constexpr int SM_STAGES = 0;
 constexpr int SM_B = IM_STAGES * IM_STAGE_BYTES;       // 64 x 64 B query codes
 constexpr int SM_SFB = SM_B + IM_N * 64;                // 512 B scale atom
 constexpr int SM_W = SM_SFB + 512;                      // 64 fp32 head weights
 constexpr int IM_CAND_TILES = 16;                       // candidate lists staged when a CTA has at most this many tiles
 constexpr int SM_CAND = SM_W + 256;                     // [IM_CAND_TILES * 128] candidate entry indices
-constexpr int SM_INFO = SM_CAND + IM_CAND_TILES * IM_TILE * 4;  // [IM_INFO] chunk of each slot (-1: done)
-constexpr int SM_BAR = SM_INFO + IM_INFO * 4;           // mbarriers
-constexpr int N_BARS = 2 * IM_STAGES + 2 * IM_ACC + 1 + IM_INFO;
+constexpr int SM_BAR = SM_CAND + IM_CAND_TILES * IM_TILE * 4;   // mbarriers
+constexpr int N_BARS = 2 * IM_STAGES + 2 * IM_ACC + 1;
 constexpr int SM_MISC = SM_BAR + 8 * N_BARS;            // tmem base, abort flag
 constexpr int SM_TOTAL = SM_MISC + 16;
 constexpr size_t IM_SMEM_BYTES = SM_TOTAL + 1024;       // slack for 1024-byte alignment
 }  // namespace
-
-// Per launch slot: one chunk counter per row, then the count of CTAs that have finished.
-static __device__ uint32_t g_scan_ctr[IM_DYN_SLOTS][IM_DYN_ROWS + 1];
 
 struct IndexMmaArgs {
   bool use_tma;
@@ -94,8 +74,7 @@ struct IndexMmaArgs {
   csa2_cache c;
   float *scores;
   int32_t *err;
-  int chunk;     // static schedule: tiles per CTA
-  int dyn_slot;  // dynamic schedule: launch slot of the row counters (-1: static)
+  int chunk;  // tiles per CTA
 };
 
 // A-operand row of tile entry e and the inverse map.
@@ -111,8 +90,6 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
   uint64_t *acc_full = empty + IM_STAGES;
   uint64_t *acc_empty = acc_full + IM_ACC;
   uint64_t *done = acc_empty + IM_ACC;
-  uint64_t *info_full = done + 1;
-  int32_t *info = reinterpret_cast<int32_t *>(smem + SM_INFO);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM_MISC + 4);
   float *ws = reinterpret_cast<float *>(smem + SM_W);
@@ -122,12 +99,10 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
   const int nvis = visible_entries(a.c, b, a.q_pos[row]);
   const int n_entries = a.c.num_entries[b];
   const int t_all = (a.n_out + IM_TILE - 1) / IM_TILE;
-  const int t_work = a.cand ? (a.P + IM_TILE - 1) / IM_TILE : min((nvis + IM_TILE - 1) / IM_TILE, t_all);
-  const bool dyn = a.dyn_slot >= 0;
-  const int t0 = dyn ? 0 : blockIdx.x * a.chunk;
-  const int t1 = dyn ? 0 : min(t0 + a.chunk, t_all);
-  const int ntiles = dyn ? 0 : max(0, min(t1, t_work) - t0);
-  uint32_t *row_ctr = dyn ? &g_scan_ctr[a.dyn_slot][row] : nullptr;
+  const int t_work = a.cand ? (a.P + IM_TILE - 1) / IM_TILE : (nvis + IM_TILE - 1) / IM_TILE;
+  const int t0 = blockIdx.x * a.chunk;
+  const int t1 = min(t0 + a.chunk, t_all);
+  const int ntiles = max(0, min(t1, t_work) - t0);
   // a full scan whose output row is shorter than the visible entries would drop the tail
   if (!a.cand && nvis > a.n_out && blockIdx.x == 0 && threadIdx.x == 0) report(a.err, CSA2_ERR_SHAPE);
 
@@ -164,7 +139,6 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       mbar_init(&acc_empty[i], 4);
     }
     mbar_init(done, 1);
-    for (int i = 0; i < IM_INFO; ++i) mbar_init(&info_full[i], 1);
     *abort_flag = 0;
     mbar_init_fence();
   } else if (warp >= 2 && warp < 6) {
@@ -219,56 +193,23 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Chunk k of this CTA's schedule: first tile and tile count, false once there is none.
-  // Static: one chunk, the CTA's run.  Dynamic: the producer takes the chunk from the row's
-  // counter and publishes it in slot k % IM_INFO; the other roles wait for it there.
-  auto take_chunk = [&](int k, int &first, int &count) -> bool {
-    const int c = int(atomicAdd(row_ctr, 1u));
-    const bool ok = c * IM_CHUNK < t_work;
-    info[k % IM_INFO] = ok ? c : -1;
-    mbar_arrive(&info_full[k % IM_INFO]);
-    first = c * IM_CHUNK;
-    count = ok ? min(IM_CHUNK, t_work - first) : 0;
-    return ok;
-  };
-  auto read_chunk = [&](int k, int &first, int &count) -> bool {
-    if (!dyn) {
-      first = t0, count = ntiles;
-      return k == 0 && ntiles > 0;
-    }
-    if (!mbar_wait_bounded(&info_full[k % IM_INFO], (k / IM_INFO) & 1, abort_flag, WAIT_LIMIT_NS)) return false;
-    const int c = info[k % IM_INFO];
-    first = c * IM_CHUNK;
-    count = c >= 0 ? min(IM_CHUNK, t_work - first) : 0;
-    return c >= 0;
-  };
-
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     const uint32_t stages = smem_u32(smem + SM_STAGES);
     if (a.use_tma) {
       if (lane == 0) {
-        int i = 0;  // tiles loaded so far by this CTA
-        bool go = true;
-        for (int k = 0; go; ++k) {
-          int first, count;
-          if (!(dyn ? take_chunk(k, first, count) : read_chunk(k, first, count))) break;
-          for (int tt = 0; tt < count; ++tt, ++i) {
-            const int s = i % IM_STAGES;
-            if (!mbar_wait_bounded(&empty[s], ((i / IM_STAGES) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) {
-              go = false;
-              break;
-            }
-            const uint32_t st = stages + s * IM_STAGE_BYTES;
-            const int64_t slot0 = cache_slot(a.c, b, int64_t(first + tt) * IM_TILE);
-            if (slot0 >= 0 && (slot0 & (IM_TILE - 1)) == 0 && slot0 + IM_TILE <= a.c.num_slots) {
-              mbar_arrive_expect_tx(&full[s], IM_A_BYTES + 512);
-              tma_load_4d(st, &tmap, 0, 0, 0, int(slot0 / IM_TILE), &full[s]);
-              bulk_load(st + IM_A_BYTES, a.c.ix_scales + slot0 * CSA2_IX_SCALE_BYTES, 512, &full[s]);
-            } else {
-              report(a.err, CSA2_ERR_INDEX);  // a visible tile without a valid page: epilogue masks it
-              mbar_arrive(&full[s]);
-            }
+        for (int i = 0; i < ntiles; ++i) {
+          const int s = i % IM_STAGES;
+          if (!mbar_wait_bounded(&empty[s], ((i / IM_STAGES) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+          const uint32_t st = stages + s * IM_STAGE_BYTES;
+          const int64_t slot0 = cache_slot(a.c, b, int64_t(t0 + i) * IM_TILE);
+          if (slot0 >= 0 && (slot0 & (IM_TILE - 1)) == 0 && slot0 + IM_TILE <= a.c.num_slots) {
+            mbar_arrive_expect_tx(&full[s], IM_A_BYTES + 512);
+            tma_load_4d(st, &tmap, 0, 0, 0, int(slot0 / IM_TILE), &full[s]);
+            bulk_load(st + IM_A_BYTES, a.c.ix_scales + slot0 * CSA2_IX_SCALE_BYTES, 512, &full[s]);
+          } else {
+            report(a.err, CSA2_ERR_INDEX);  // a visible tile without a valid page: epilogue masks it
+            mbar_arrive(&full[s]);
           }
         }
       }
@@ -342,29 +283,20 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       const uint64_t b1 = smem_desc(bq + 32, 16, 512, LAYOUT_SWIZZLE_64B);
       constexpr uint32_t id0 = idesc_mxf4(IM_TILE, IM_N, 0, 0);
       constexpr uint32_t id1 = idesc_mxf4(IM_TILE, IM_N, 2, 2);
-      int i = 0;
-      bool go = true;
-      for (int k = 0; go; ++k) {
-        int first, count;
-        if (!read_chunk(k, first, count)) break;
-        for (int tt = 0; tt < count; ++tt, ++i) {
-          const int s = i % IM_STAGES, acc = i % IM_ACC;
-          if (!mbar_wait_bounded(&full[s], (i / IM_STAGES) & 1, abort_flag, WAIT_LIMIT_NS) ||
-              !mbar_wait_bounded(&acc_empty[acc], ((i / IM_ACC) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) {
-            go = false;
-            break;
-          }
-          if (!a.use_tma) fence_proxy_async_smem();  // cp.async-filled stages are read by the tensor core
-          tc_fence_after();
-          const uint32_t st = stages + s * IM_STAGE_BYTES;
-          const uint32_t sfa = tmem + COL_SFA + 4 * acc;
-          tc_cp_32x128b_warpx4(sfa, smem_desc(st + IM_A_BYTES, 16, 128, LAYOUT_SWIZZLE_NONE));
-          const uint32_t d = tmem + acc * IM_N;
-          tc_mma_mxf4(d, smem_desc(st, 16, 512, LAYOUT_SWIZZLE_64B), b0, id0, sfa, tmem + COL_SFB, false);
-          tc_mma_mxf4(d, smem_desc(st + 32, 16, 512, LAYOUT_SWIZZLE_64B), b1, id1, sfa, tmem + COL_SFB, true);
-          tc_commit(&empty[s]);
-          tc_commit(&acc_full[acc]);
-        }
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % IM_STAGES, acc = i % IM_ACC;
+        if (!mbar_wait_bounded(&full[s], (i / IM_STAGES) & 1, abort_flag, WAIT_LIMIT_NS)) break;
+        if (!mbar_wait_bounded(&acc_empty[acc], ((i / IM_ACC) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+        if (!a.use_tma) fence_proxy_async_smem();  // cp.async-filled stages are read by the tensor core
+        tc_fence_after();
+        const uint32_t st = stages + s * IM_STAGE_BYTES;
+        const uint32_t sfa = tmem + COL_SFA + 4 * acc;
+        tc_cp_32x128b_warpx4(sfa, smem_desc(st + IM_A_BYTES, 16, 128, LAYOUT_SWIZZLE_NONE));
+        const uint32_t d = tmem + acc * IM_N;
+        tc_mma_mxf4(d, smem_desc(st, 16, 512, LAYOUT_SWIZZLE_64B), b0, id0, sfa, tmem + COL_SFB, false);
+        tc_mma_mxf4(d, smem_desc(st + 32, 16, 512, LAYOUT_SWIZZLE_64B), b1, id1, sfa, tmem + COL_SFB, true);
+        tc_commit(&empty[s]);
+        tc_commit(&acc_full[acc]);
       }
       tc_commit(done);  // fires once every tcgen05 op of this thread has completed
       // wait for it even after an abort, so TMEM is never freed under a running MMA
@@ -378,13 +310,21 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     const int q4 = warp & 3;              // TMEM sub-partition of this warp
     const int e = entry_of_row(32 * q4 + lane);  // tile entry of this thread's accumulator row
     const float4 *w4 = reinterpret_cast<const float4 *>(ws);
-    // warpgroup wg takes this CTA's tiles wg, wg + IM_EPI_WG, ...
+    // warpgroup wg takes tiles wg, wg + IM_EPI_WG, ...; the entry behind this thread's
+    // row is fetched one of its tiles ahead (candidate lists are read from global)
     const int wg = (warp - 2) >> 2;
-    // Score of the key behind this thread's row of the accumulator of CTA tile i (global tile
-    // `tile`, entry n_cur: -1 for none); false if the wait gave up.
-    auto epi_tile = [&](int i, int tile, int64_t n_cur) -> bool {
+    auto entry_at = [&](int i) -> int64_t {
+      const int pos = (t0 + i) * IM_TILE + e;
+      if (!a.cand) return pos;
+      if (i >= ntiles || pos >= a.P) return -1;
+      return cand_staged ? cand_s[pos - t0 * IM_TILE] : a.cand[int64_t(row) * a.P + pos];
+    };
+    int64_t n_next = entry_at(wg);
+    for (int i = wg; i < ntiles; i += IM_EPI_WG) {
       const int acc = i % IM_ACC;
-      if (!mbar_wait_bounded(&acc_full[acc], (i / IM_ACC) & 1, abort_flag, WAIT_LIMIT_NS)) return false;
+      const int64_t n_cur = n_next;
+      n_next = entry_at(i + IM_EPI_WG);
+      if (!mbar_wait_bounded(&acc_full[acc], (i / IM_ACC) & 1, abort_flag, WAIT_LIMIT_NS)) break;
       tc_fence_after();
       const uint32_t taddr = tmem + (uint32_t(32 * q4) << 16) + acc * IM_N;
       uint32_t r0[32], r1[32];
@@ -413,52 +353,15 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
         part[(4 * h4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f), part[(4 * h4 + 3) & 7]);
       }
       const float sc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-      const int pos = tile * IM_TILE + e;
+      const int pos = (t0 + i) * IM_TILE + e;
       if (pos < a.n_out) {
         const bool ok = n_cur >= 0 && n_cur < nvis && cache_slot(a.c, b, n_cur) >= 0;
         a.scores[int64_t(row) * a.n_out + pos] = ok ? sc : -INFINITY;
       }
-      return true;
-    };
-    if (dyn) {
-      int i = 0;
-      bool go = true;
-      for (int k = 0; go; ++k) {
-        int first, count;
-        if (!read_chunk(k, first, count)) break;
-        for (int tt = 0; tt < count; ++tt, ++i)
-          if (i % IM_EPI_WG == wg && !epi_tile(i, first + tt, int64_t(first + tt) * IM_TILE + e)) {
-            go = false;
-            break;
-          }
-      }
-    } else {
-      // the entry behind this thread's row is fetched one of its tiles ahead (candidate
-      // lists are read from global memory unless staged)
-      auto entry_at = [&](int i) -> int64_t {
-        const int pos = (t0 + i) * IM_TILE + e;
-        if (!a.cand) return pos;
-        if (i >= ntiles || pos >= a.P) return -1;
-        return cand_staged ? cand_s[pos - t0 * IM_TILE] : a.cand[int64_t(row) * a.P + pos];
-      };
-      int64_t n_next = entry_at(wg);
-      for (int i = wg; i < ntiles; i += IM_EPI_WG) {
-        const int64_t n_cur = n_next;
-        n_next = entry_at(i + IM_EPI_WG);
-        if (!epi_tile(i, t0 + i, n_cur)) break;
-      }
     }
-    // positions past the visible entries (no key tile was loaded for them): the CTA's own
-    // run, or with the dynamic schedule the CTA's share of the row's tail
+    // positions past the visible entries (no key tile was loaded for them)
     if (!a.cand) {
-      int lo, hi;
-      if (dyn) {
-        const int tail0 = min(a.n_out, t_work * IM_TILE);
-        const int per = (a.n_out - tail0 + int(gridDim.x) - 1) / int(gridDim.x);
-        lo = min(a.n_out, tail0 + int(blockIdx.x) * per), hi = min(a.n_out, lo + per);
-      } else {
-        lo = max(t0, t_work) * IM_TILE, hi = min(t1 * IM_TILE, a.n_out);
-      }
+      const int lo = max(t0, t_work) * IM_TILE, hi = min(t1 * IM_TILE, a.n_out);
       for (int pos = lo + threadIdx.x - 64; pos < hi; pos += 128 * IM_EPI_WG)
         a.scores[int64_t(row) * a.n_out + pos] = -INFINITY;
     }
@@ -470,21 +373,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     tc_fence_after();
     tmem_dealloc(tmem, IM_TMEM_COLS);
   }
-  if (threadIdx.x == 0) {
-    if (*abort_flag) report(a.err, CSA2_ERR_TIMEOUT);
-    if (dyn) {
-      // every chunk this CTA will take has been taken; the launch's last CTA clears the
-      // slot's counters for the next launch that uses it
-      __threadfence();
-      const uint32_t total = gridDim.x * gridDim.y;
-      uint32_t *ctr = g_scan_ctr[a.dyn_slot];
-      if (atomicAdd(&ctr[IM_DYN_ROWS], 1u) == total - 1) {
-        for (int r = 0; r < int(gridDim.y); ++r) ctr[r] = 0;
-        ctr[IM_DYN_ROWS] = 0;
-        __threadfence();
-      }
-    }
-  }
+  if (threadIdx.x == 0 && *abort_flag) report(a.err, CSA2_ERR_TIMEOUT);
 }
 
 namespace {
@@ -516,10 +405,6 @@ bool make_code_map(CUtensorMap *m, const csa2_cache &c) {
              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-// Launch slots of the dynamic schedule, taken round-robin so that launches in flight at
-// the same time on different streams use different counters.
-std::atomic<uint32_t> g_next_dyn_slot{0};
 }  // namespace
 
 void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
@@ -535,12 +420,9 @@ void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int 
   CUtensorMap tmap;
   memset(&tmap, 0, sizeof(tmap));
   const bool use_tma = cand == nullptr && make_code_map(&tmap, c);
-  // full scans of up to IM_DYN_ROWS rows take their tiles dynamically
-  const int dyn_slot = (use_tma && rows <= IM_DYN_ROWS) ? int(g_next_dyn_slot++ % IM_DYN_SLOTS) : -1;
-  IndexMmaArgs a{use_tma, q_ix, w, Q, q_pos, cand, P, n_out, c, scores, err, chunk, dyn_slot};
+  IndexMmaArgs a{use_tma, q_ix, w, Q, q_pos, cand, P, n_out, c, scores, err, chunk};
   set_smem_limit(index_score_mma_kernel, IM_SMEM_BYTES);
-  const int gx = dyn_slot >= 0 ? splits : (t_all + chunk - 1) / chunk;
-  index_score_mma_kernel<<<dim3(gx, rows), IM_THREADS, IM_SMEM_BYTES, st>>>(tmap, a);
+  index_score_mma_kernel<<<dim3((t_all + chunk - 1) / chunk, rows), IM_THREADS, IM_SMEM_BYTES, st>>>(tmap, a);
 }
 
 }  // namespace csa2
