@@ -419,6 +419,16 @@ def peaks():
     return 6650.0, "fallback"
 
 
+def tensor_peaks():
+    """(dense bf16 TFLOP/s as a burst, kind): the measured cuBLAS figure, else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 # ---------------------------------------------------------------- the oracle's time (CPU baseline)
 def oracle_time(spec, n_seqs=1):
     """Time the oracle, as it stands, on `n_seqs` sequences of one decode step (all five layers)."""
@@ -583,6 +593,20 @@ class OneLayer:
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
 
+    def prefill_select(self):
+        """The prefill chunk's fused indexer + top-k alone (csa2_index_topk)."""
+        q, q_ix, w, q_pos = self.io[0][:4]
+        self.sel = self.k.csa2_index_topk(q_ix, w, q_pos, self.base, self.spec.max_entries, k=self.spec.k,
+                                          idx=getattr(self, "sel", None), err=self.err)
+
+    def prefill_attend(self):
+        """The prefill chunk's attention over that selection (with its window), alone."""
+        q, q_ix, w, q_pos, codes, scale, o, lse, _ = self.io[0]
+        if getattr(self, "sel", None) is None:
+            self.prefill_select()
+        self.k.csa2_sparse_attn("reuse", q, q_pos, self.base, self.spec.tau, self.spec.max_entries, k=self.spec.k,
+                                idx_in=self.sel, o=o, lse=lse, err=self.err, swa_codes=codes, swa_scale=scale)
+
     def query_rows(self):
         return self.spec.B * self.spec.q_len
 
@@ -652,6 +676,32 @@ def run_one_layer(args, spec, dev, world, rank):
     if pairs:
         line["indexer"] = {"pairs_per_step": pairs, "fp4_tflop_per_step": pairs * 64 * 128 * 2 / 1e12,
                            "fp4_tflops_whole_step": pairs * 64 * 128 * 2 / (step_ms * 1e-3) / 1e12}
+    if spec.mode == "prefill":
+        # the two halves of the layer alone: the fused indexer + top-k, then the attention on its selection
+        bf16, kind = tensor_peaks()
+        parts = {}
+        for name, fn in (("indexer", wl.prefill_select), ("attention", wl.prefill_attend)):
+            pev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush.zero_()
+                pev[i][0].record(stream)
+                fn()
+                pev[i][1].record(stream)
+            torch.cuda.synchronize()
+            parts[name] = sum(a.elapsed_time(b) for a, b in pev) / args.steps
+        assert wl.k.csa2_check(wl.err) == 0
+        fp4 = pairs * 64 * 128 * 2 / (parts["indexer"] * 1e-3) / 1e12
+        attn_flop = rows * 64 * (spec.k + 128) * 512 * 4
+        bf = attn_flop / (parts["attention"] * 1e-3) / 1e12
+        line["indexer_roofline"] = {"bound": "tensor", "kernel": "csa2 fused prefill indexer + top-k (FP4 MMA)",
+                                    "achieved": fp4, "peak": 4 * bf16, "unit": "TFLOP/s", "frac": fp4 / (4 * bf16),
+                                    "peak_kind": f"4 x {kind} dense bf16 (the nominal fp4 : bf16 ratio)",
+                                    "ms": parts["indexer"]}
+        line["attention_roofline"] = {"bound": "tensor", "kernel": "csa2 sparse attention + SWA + merge (kind::f16)",
+                                      "achieved": bf, "peak": bf16, "unit": "TFLOP/s", "frac": bf / bf16,
+                                      "peak_kind": f"{kind} dense bf16", "ms": parts["attention"],
+                                      "flop_per_step": attn_flop}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -7,8 +7,8 @@ CPU fallback.  (`python -m compressed_sparse_attention_score_b200.build` builds 
 """
 _NAMES = ("EXPORTED", "MODE", "GlobalKVCache", "csa2_cache", "csa2_check", "csa2_index_score", "csa2_merge",
           "csa2_pack_kv", "csa2_pack_swa", "csa2_sparse_attn", "csa2_sparse_attn_noalloc", "csa2_swa_attn",
-          "csa2_topk", "csa2_version", "csa2_workspace_size", "raw", "LIB_PATH", "csa2_append_kv", "csa2_plan_v41", "csa2_pack_kv_gated",
-          "DecodeStep", "LAYER_SWA")
+          "csa2_topk", "csa2_version", "csa2_workspace_size", "raw", "LIB_PATH", "csa2_append_kv", "csa2_plan_v41",
+          "csa2_pack_kv_gated", "csa2_index_topk", "DecodeStep", "LAYER_SWA")
 
 
 def __getattr__(name):

@@ -81,6 +81,8 @@ _SIGS = {
     "csa2_append_kv": ([c_void_p, c_void_p, ctypes.c_int, c_int32, c_void_p, c_void_p, _P, c_void_p, c_void_p],
                        ctypes.c_int),
     "csa2_plan_v41": ([c_void_p, c_int32, c_void_p], c_int32),
+    "csa2_index_topk": ([c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_int32, c_int32, _P, c_void_p, c_void_p,
+                         c_void_p], ctypes.c_int),
     "csa2_pack_kv_gated": ([c_void_p, c_void_p, ctypes.c_int, c_void_p, c_void_p, c_int32, c_int32, c_void_p, _P,
                            c_void_p, c_void_p], ctypes.c_int),
     "csa2_decode_workspace_size": ([_PD], c_size_t),
@@ -295,6 +297,17 @@ def csa2_append_kv(lat_kv, lat_ix, pos, cache, stage=None, err=None, stream=None
     d = cache.desc()
     _ok(_lib.csa2_append_kv(_ptr(lat_kv), _ptr(lat_ix), DTYPE[lat_kv.dtype], B, _ptr(pos), _ptr(stage),
                             ctypes.byref(d), _ptr(err), _stream(stream)), "csa2_append_kv")
+
+
+def csa2_index_topk(q_ix, w, q_pos, cache, max_entries, k=512, idx=None, err=None, stream=None):
+    """Full-mode selection of every query row (fused indexer + top-k, no scores kept): idx [B][Q][k]."""
+    B, Q = q_ix.shape[0], q_ix.shape[1]
+    if idx is None:
+        idx = torch.empty((B, Q, k), dtype=torch.int32, device=q_ix.device)
+    d = cache.desc()
+    _ok(_lib.csa2_index_topk(_ptr(q_ix), _ptr(w), B, Q, _ptr(q_pos), k, max_entries, ctypes.byref(d), _ptr(idx),
+                             _ptr(err), _stream(stream)), "csa2_index_topk")
+    return idx
 
 
 def csa2_pack_kv_gated(lat_kv, lat_ix, gate_kv, gate_ix, first_entry, cache, err=None, stream=None):

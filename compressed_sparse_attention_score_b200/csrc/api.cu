@@ -54,6 +54,12 @@ size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 // device that cannot hold a 16-CTA cluster); the workspace is sized for the smaller.
 constexpr int kDenseMinSegment = 4096;
 
+// Full mode with this many query rows or more (a prefill chunk) and no pool selects with the
+// fused prefill indexer: each CTA serves 3 query tokens over every key tile they see, so there
+// must be enough of them to fill the device; the scores are never materialised.
+constexpr int64_t kFusedPrefillRows = 1024;
+bool fused_prefill(int64_t rows, int32_t pool_k) { return rows >= kFusedPrefillRows && pool_k == 0; }
+
 }  // namespace
 
 namespace csa2 {
@@ -82,7 +88,8 @@ CSA2_EXPORT size_t csa2_workspace_size(csa2_mode mode, int32_t B, int32_t Q, int
   if (B < 0 || Q < 0 || max_entries < 0 || k < 0 || pool_k < 0) return 0;
   const size_t rows = size_t(B) * Q;
   switch (mode) {
-    case CSA2_MODE_FULL: return round256(rows * max_entries * 4) + round256(rows * k * 4);
+    case CSA2_MODE_FULL:
+      return (fused_prefill(int64_t(rows), pool_k) ? 0 : round256(rows * max_entries * 4)) + round256(rows * k * 4);
     case CSA2_MODE_REINDEX: return round256(rows * pool_k * 4) + round256(rows * k * 4);
     case CSA2_MODE_DENSE:  // partial (o, lse) of one key segment beyond the first
       return max_entries > kDenseMinSegment ? round256(rows * CSA2_HEADS * CSA2_MAIN_DIM * 4) +
@@ -147,6 +154,20 @@ CSA2_EXPORT csa2_status csa2_index_score(const uint16_t *q_ix, const uint16_t *w
   return launched("csa2_index_score");
 }
 
+CSA2_EXPORT csa2_status csa2_index_topk(const uint16_t *q_ix, const uint16_t *w, int32_t B, int32_t Q,
+                                        const int32_t *q_pos, int32_t k, int32_t max_entries,
+                                        const csa2_cache *cache, int32_t *idx, int32_t *err, csa2_stream_t stream) {
+  if (B < 0 || Q < 0 || max_entries < 0 || k < 1) return fail(CSA2_ERR_INVALID_ARG, "bad size");
+  if (B == 0 || Q == 0) return CSA2_OK;
+  if (csa2_status s = check_cache(cache, B)) return s;
+  if (!q_ix || !w || !q_pos || !idx) return fail(CSA2_ERR_INVALID_ARG, "NULL input");
+  if (k > 512) return fail(CSA2_ERR_UNSUPPORTED, "k > 512");
+  if (!aligned16(q_ix)) return fail(CSA2_ERR_INVALID_ARG, "q_ix misaligned");
+  if (B > 65535) return fail(CSA2_ERR_UNSUPPORTED, "more than 65535 sequences per call");
+  csa2::launch_prefill_index(q_ix, w, B, Q, q_pos, k, max_entries, *cache, idx, err, stream);
+  return launched("csa2_index_topk");
+}
+
 CSA2_EXPORT csa2_status csa2_topk(const float *scores, const int32_t *n_valid, int32_t R, int32_t N, int32_t k,
                                   int32_t *idx, float *val, int32_t k2, int32_t *idx2, float *val2,
                                   csa2_stream_t stream) {
@@ -208,6 +229,14 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
     if (mode == CSA2_MODE_FULL && pool_k > 0 && !pool_io) return fail(CSA2_ERR_INVALID_ARG, "pool_k > 0 needs pool_io");
     const size_t need = csa2_workspace_size(mode, B, Q, max_entries, k, pool_k);
     if (!ws || ws_bytes < need) return fail(CSA2_ERR_INVALID_ARG, "workspace too small");
+    if (mode == CSA2_MODE_FULL && fused_prefill(rows, pool_k)) {
+      // a prefill chunk: fused indexer + causal top-k, no score matrix
+      int32_t *sel = idx_out ? idx_out : static_cast<int32_t *>(ws);
+      csa2::launch_prefill_index(q_ix, w, B, Q, q_pos, k, max_entries, *cache, sel, err, stream);
+      csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, sel, k, false, 0, 0, 0, cache, swa_codes,
+                            swa_codes ? swa_scale : nullptr, R, window, o, lse, err, stream);
+      return launched("csa2_sparse_attn");
+    }
     const int n_out = mode == CSA2_MODE_FULL ? max_entries : pool_k;
     if (rows > 65535) return fail(CSA2_ERR_UNSUPPORTED, "more than 65535 query rows per call");
     float *scores = static_cast<float *>(ws);

@@ -389,10 +389,12 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+}  // namespace
+
 // 4-D view of the indexer-code plane: (64 bytes, entry / 4 within a 128-entry
 // group [stride 256 B], entry % 4 [stride 64 B], group [stride 8192 B]).  A box
 // of (64, 32, 4, 1) lands entry e of the group at shared-memory row (e%4)*32 + e/4.
-bool make_code_map(CUtensorMap *m, const csa2_cache &c) {
+bool make_index_code_map(CUtensorMap *m, const csa2_cache &c) {
   auto enc = tensor_map_encoder();
   if (!enc || (c.num_slots % IM_TILE) != 0 || c.num_slots / IM_TILE > (int64_t(1) << 31)) return false;
   if ((reinterpret_cast<uintptr_t>(c.ix_scales) & 15) || (reinterpret_cast<uintptr_t>(c.ix_codes) & 15)) return false;
@@ -405,7 +407,6 @@ bool make_code_map(CUtensorMap *m, const csa2_cache &c) {
              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-}  // namespace
 
 void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
                             const int32_t *cand, int P, int n_out, const csa2_cache &c, float *scores, int32_t *err,
@@ -419,7 +420,7 @@ void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int 
   const int chunk = (t_all + splits - 1) / splits;
   CUtensorMap tmap;
   memset(&tmap, 0, sizeof(tmap));
-  const bool use_tma = cand == nullptr && make_code_map(&tmap, c);
+  const bool use_tma = cand == nullptr && make_index_code_map(&tmap, c);
   IndexMmaArgs a{use_tma, q_ix, w, Q, q_pos, cand, P, n_out, c, scores, err, chunk};
   set_smem_limit(index_score_mma_kernel, IM_SMEM_BYTES);
   index_score_mma_kernel<<<dim3((t_all + chunk - 1) / chunk, rows), IM_THREADS, IM_SMEM_BYTES, st>>>(tmap, a);

@@ -1,5 +1,6 @@
 // Host-side launchers of the CSA2 kernels (internal to the library).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -47,6 +48,12 @@ void launch_append_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype, 
 void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
                             const int32_t *cand, int P, int n_out, const csa2_cache &c, float *scores, int32_t *err,
                             cudaStream_t st);
+// Tensor map of a cache's indexer codes as 128-entry groups (false: the layout does not allow one).
+bool make_index_code_map(CUtensorMap *m, const csa2_cache &c);
+// Fused prefill indexer + causal top-k (k <= 512): idx [B][Q][k], ascending, -1 padded.
+// Entries beyond max_entries are left out and set CSA2_ERR_SHAPE (as the unfused Full path).
+void launch_prefill_index(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos, int k,
+                          int max_entries, const csa2_cache &c, int32_t *idx, int32_t *err, cudaStream_t st);
 void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int N, int k0, int32_t *idx0, float *val0,
                          int k1, int32_t *idx1, float *val1, const int32_t *map, cudaStream_t st);
 // swa_new [B*Q][512] bf16 (decode): each row's own window token, quantised inside the launch,

@@ -1,0 +1,500 @@
+// K4: the prefill indexer with its causal top-k fused in (no score matrix).
+//
+// CTA = PF_Q consecutive query tokens of one sequence x every key tile any of them sees.
+// A 128-entry key tile is loaded once (one TMA box of the codes plus the scale words, or
+// cp.async gathers for caches a tensor map cannot describe) and serves all PF_Q queries: per
+// query two K=64 block-scaled FP4 MMAs (tcgen05 kind::mxf4, N = 64 heads) into the query's
+// accumulator; two sets of accumulators alternate between tiles.  Warp roles:
+//   warp 0     producer;
+//   warp 1     MMA issuer (one lane);
+//   warps 2-9  two epilogue warpgroups on alternate tiles: for each query the weighted-ReLU
+//              score of its 128 keys (the decode kernel's arithmetic, so both give the same
+//              fp32 score); keys the query cannot see are dropped, keys above the query's
+//              running threshold are appended to its candidate list in shared memory.
+// After every pair of tiles the two warpgroups meet; a query whose list could overflow during
+// the next pair is cut back to its best k candidates (radix selection on the scores'
+// order-preserving keys), and its threshold becomes the k-th key: a later key equal to it has
+// a higher entry index and loses the tie.  At the end each query keeps its best k (score
+// descending, entry ascending), written in ascending entry order and padded with -1 -- the
+// selection csa2_topk makes from materialised scores.
+// Every mbarrier wait is time-bounded; on expiry the CTA drains and reports CSA2_ERR_TIMEOUT.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace csa2 {
+using namespace sm100;
+
+namespace {
+constexpr int PF_Q = 3;                 // query tokens per CTA
+constexpr int PF_STAGES = 8;
+constexpr int PF_TILE = 128;            // keys per tile = MMA M
+constexpr int PF_N = 64;                // indexer heads = MMA N
+constexpr int PF_A_BYTES = PF_TILE * 64;
+constexpr int PF_STAGE_BYTES = 9216;    // 8192 codes + 512 scale atom, padded to 1024
+constexpr int PF_EPI = 256;             // epilogue threads (two warpgroups)
+constexpr int PF_THREADS = 64 + PF_EPI;
+constexpr int PF_CAP = 4096;            // candidate list per query
+constexpr int PF_KMAX = 512;
+constexpr uint32_t PF_TMEM_COLS = 512;
+constexpr uint32_t PF_COL_SFA = 2 * PF_Q * 64;         // after the two accumulator sets
+constexpr uint32_t PF_COL_SFB = PF_COL_SFA + 8;
+constexpr uint64_t PF_WAIT_NS = 2000000000ull;
+
+constexpr int PS_STAGES = 0;
+constexpr int PS_B = PF_STAGES * PF_STAGE_BYTES;          // PF_Q x [64 heads x 64 B] query codes
+constexpr int PS_SFB = PS_B + PF_Q * 4096;                // PF_Q x 512 B scale atoms
+constexpr int PS_W = PS_SFB + PF_Q * 512;                 // PF_Q x 64 fp32 head weights
+constexpr int PS_CKEY = PS_W + PF_Q * 256;                // PF_Q x PF_CAP keys
+constexpr int PS_CENT = PS_CKEY + PF_Q * PF_CAP * 4;      // PF_Q x PF_CAP entries
+constexpr int PS_SCR = PS_CENT + PF_Q * PF_CAP * 4;       // cut scratch: PF_KMAX keys, PF_KMAX entries
+constexpr int PS_HIST = PS_SCR + PF_KMAX * 8;             // 256-bin histogram
+constexpr int PS_SEL = PS_HIST + 256 * 4;                 // selection state (16 words)
+constexpr int PS_QS = PS_SEL + 64;                        // per query: count, threshold, visible entries
+constexpr int PS_BAR = PS_QS + 4 * PF_Q * 4;
+constexpr int PF_NBARS = 2 * PF_STAGES + 4 + 1;
+constexpr int PS_MISC = PS_BAR + 8 * PF_NBARS;
+constexpr int PS_TOTAL = PS_MISC + 16;
+constexpr size_t PF_SMEM = PS_TOTAL + 1024;
+}  // namespace
+
+struct PrefillArgs {
+  bool use_tma;
+  const uint16_t *q_ix;
+  const uint16_t *w;
+  int Q;
+  const int32_t *q_pos;
+  int k;
+  int max_entries;  // entries a query may see (more: left out, CSA2_ERR_SHAPE)
+  csa2_cache c;
+  int32_t *idx;  // [B][Q][k]
+  int32_t *err;
+};
+
+namespace {
+__device__ __forceinline__ int pf_row_of_entry(int e) { return (e & 3) * 32 + (e >> 2); }
+__device__ __forceinline__ int pf_entry_of_row(int m) { return (m & 31) * 4 + (m >> 5); }
+
+// Named barrier of the PF_EPI epilogue threads.
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(PF_EPI) : "memory"); }
+
+// The k-th largest key T of list keys[0..n) (n > k) and how many of the keys equal to T belong
+// to the best k (need_eq), by radix selection on 8-bit digits from the top; also whether every
+// key equal to T is kept (all_eq).  Called by the PF_EPI epilogue threads (t = their index).
+__device__ void kth_key(const uint32_t *keys, int n, int k, uint32_t *hist, uint32_t *sel, int t, uint32_t &T,
+                        int &need_eq, bool &all_eq) {
+  uint32_t prefix = 0;
+  int need = k, bin_count = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    hist[t] = 0;  // PF_EPI == 256 bins
+    epi_sync();
+    const uint32_t himask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+    for (int i = t; i < n; i += PF_EPI) {
+      const uint32_t key = keys[i];
+      if ((key & himask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    epi_sync();
+    if (t < 32) {  // one warp finds the digit at which the count from the top reaches `need`
+      uint32_t c8[8], s = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s += (c8[j] = hist[255 - (8 * t + j)]);
+      uint32_t x = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (t >= o) x += y;
+      }
+      const uint32_t excl = x - s;
+      const int L = __ffs(__ballot_sync(0xffffffffu, excl < uint32_t(need) && x >= uint32_t(need))) - 1;
+      if (t == L) {
+        uint32_t cum = excl;
+#pragma unroll 1
+        for (int j = 0; j < 8; ++j) {
+          if (cum + c8[j] >= uint32_t(need)) {
+            sel[0] = uint32_t(255 - (8 * t + j));
+            sel[1] = uint32_t(need) - cum;
+            sel[2] = c8[j];
+            break;
+          }
+          cum += c8[j];
+        }
+      }
+    }
+    epi_sync();
+    prefix |= sel[0] << shift;
+    need = int(sel[1]);
+    bin_count = int(sel[2]);
+    epi_sync();  // sel and hist are rewritten by the next digit
+  }
+  T = prefix;
+  need_eq = need;
+  all_eq = bin_count == need;
+}
+
+// Cut a query's list (keys, ents, *cnt entries) back to its best k (key descending, entry
+// ascending) through the scratch and return the k-th key, the list's new threshold.  Ties on
+// that key are resolved by counting, for each, the tied keys with smaller entries (only when
+// not all of them are kept).  Called by the PF_EPI epilogue threads; contains epi_sync().
+__device__ uint32_t cut_to_k(uint32_t *keys, int32_t *ents, int *cnt, int k, uint32_t *scr_key, int32_t *scr_ent,
+                             uint32_t *hist, uint32_t *sel, int t) {
+  const int n = *cnt;
+  uint32_t T;
+  int need_eq;
+  bool all_eq;
+  kth_key(keys, n, k, hist, sel, t, T, need_eq, all_eq);
+  if (t == 0) sel[3] = 0;
+  epi_sync();
+  for (int i = t; i < n; i += PF_EPI) {
+    const uint32_t key = keys[i];
+    bool keep = key > T;
+    if (key == T) {
+      if (all_eq) {
+        keep = true;
+      } else {
+        const int e = ents[i];
+        int before = 0;
+        for (int j = 0; j < n; ++j) before += (keys[j] == T && ents[j] < e);
+        keep = before < need_eq;
+      }
+    }
+    if (keep) {
+      const int s = int(atomicAdd(&sel[3], 1u));
+      scr_key[s] = key;
+      scr_ent[s] = ents[i];
+    }
+  }
+  epi_sync();
+  for (int i = t; i < k; i += PF_EPI) {
+    keys[i] = scr_key[i];
+    ents[i] = scr_ent[i];
+  }
+  if (t == 0) *cnt = k;
+  epi_sync();
+  return T;
+}
+}  // namespace
+
+__global__ void __launch_bounds__(PF_THREADS, 1) prefill_index_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                                      PrefillArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + PS_BAR);
+  uint64_t *empty = full + PF_STAGES;
+  uint64_t *acc_full = empty + PF_STAGES;
+  uint64_t *acc_empty = acc_full + 2;
+  uint64_t *done = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + PS_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + PS_MISC + 4);
+  float *ws = reinterpret_cast<float *>(smem + PS_W);
+  uint32_t *ckey = reinterpret_cast<uint32_t *>(smem + PS_CKEY);
+  int32_t *cent = reinterpret_cast<int32_t *>(smem + PS_CENT);
+  uint32_t *hist = reinterpret_cast<uint32_t *>(smem + PS_HIST);
+  uint32_t *sel = reinterpret_cast<uint32_t *>(smem + PS_SEL);
+  int *qcnt = reinterpret_cast<int *>(smem + PS_QS);
+  uint32_t *qthr = reinterpret_cast<uint32_t *>(smem + PS_QS + PF_Q * 4);
+  int *qvis = reinterpret_cast<int *>(smem + PS_QS + 2 * PF_Q * 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y, q0 = blockIdx.x * PF_Q;
+  const int nq = min(PF_Q, a.Q - q0);  // query tokens of this CTA
+  int nvis_max = 0;
+  int nvis[PF_Q];
+#pragma unroll
+  for (int qi = 0; qi < PF_Q; ++qi) {
+    nvis[qi] = qi < nq ? visible_entries(a.c, b, a.q_pos[int64_t(b) * a.Q + q0 + qi]) : 0;
+    if (nvis[qi] > a.max_entries) {
+      if (threadIdx.x == 0) report(a.err, CSA2_ERR_SHAPE);
+      nvis[qi] = a.max_entries;
+    }
+    nvis_max = max(nvis_max, nvis[qi]);
+  }
+  const int ntiles = (nvis_max + PF_TILE - 1) / PF_TILE;
+
+  // ---------------------------------------------------------------- prologue
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, PF_TMEM_COLS);
+    tmem_relinquish();
+  } else if (warp == 1 && lane == 0) {
+    for (int s = 0; s < PF_STAGES; ++s) {
+      mbar_init(&full[s], a.use_tma ? 1 : 32);  // gather path: one cp.async arrival per producer lane
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  } else if (warp >= 2) {
+    // quantise the query heads (MXFP4, as the decode kernel): item (qi, h, pair of 32-blocks)
+    const int t = threadIdx.x - 64;
+    for (int item = t; item < PF_Q * 128; item += PF_EPI) {
+      const int qi = item >> 7, h = (item >> 1) & 63, g0 = 2 * (item & 1);
+      uint8_t *brow = smem + PS_B + qi * 4096 + h * 64;
+      uint32_t sfpart = 0;
+      const uint16_t *qh = a.q_ix + ((int64_t(b) * a.Q + q0 + min(qi, nq - 1)) * HI + h) * DI;
+#pragma unroll 1
+      for (int g = g0; g < g0 + 2; ++g) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 u = reinterpret_cast<const uint4 *>(qh + 32 * g)[i];
+          const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            v[8 * i + 2 * j] = __uint_as_float(ww[j] << 16);
+            v[8 * i + 2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
+          }
+        }
+        float am = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+        int ex = -127;
+        uint32_t cw[4] = {0, 0, 0, 0};
+        if (am != 0.f) {
+          ex = e8m0_ceil_exponent(__fdiv_rn(am, 6.0f));
+          const float inv = pow2f(-ex);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) cw[i >> 3] |= e2m1_code(__fmul_rn(v[i], inv)) << (4 * (i & 7));
+        }
+        *reinterpret_cast<uint4 *>(brow + ((g ^ ((h >> 1) & 3)) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        sfpart |= uint32_t(ex + 127) << (8 * g);
+      }
+      const uint32_t sfword = sfpart | __shfl_xor_sync(0xffffffffu, sfpart, 1);
+      uint8_t *sfb = smem + PS_SFB + qi * 512;
+      if ((item & 1) == 0) {
+        *reinterpret_cast<uint32_t *>(sfb + (h & 31) * 16 + (h >> 5) * 4) = sfword;
+        ws[qi * 64 + h] = bf16_to_f32(a.w[(int64_t(b) * a.Q + q0 + min(qi, nq - 1)) * HI + h]);
+      } else {
+        const int rz = 64 + h;
+        *reinterpret_cast<uint32_t *>(sfb + (rz & 31) * 16 + (rz >> 5) * 4) = 0u;
+      }
+    }
+    if (t < PF_Q) {
+      qcnt[t] = 0;
+      qthr[t] = KEY_NEG_INF;  // keep every finite score until the first cut
+      qvis[t] = nvis[t];
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    const uint32_t stages = smem_u32(smem + PS_STAGES);
+    if (a.use_tma) {
+      if (lane == 0) {
+        for (int i = 0; i < ntiles; ++i) {
+          const int s = i % PF_STAGES;
+          if (!mbar_wait_bounded(&empty[s], ((i / PF_STAGES) & 1) ^ 1, abort_flag, PF_WAIT_NS)) break;
+          const uint32_t st = stages + s * PF_STAGE_BYTES;
+          const int64_t slot0 = cache_slot(a.c, b, int64_t(i) * PF_TILE);
+          if (slot0 >= 0 && (slot0 & (PF_TILE - 1)) == 0 && slot0 + PF_TILE <= a.c.num_slots) {
+            mbar_arrive_expect_tx(&full[s], PF_A_BYTES + 512);
+            tma_load_4d(st, &tmap, 0, 0, 0, int(slot0 / PF_TILE), &full[s]);
+            bulk_load(st + PF_A_BYTES, a.c.ix_scales + slot0 * CSA2_IX_SCALE_BYTES, 512, &full[s]);
+          } else {
+            report(a.err, CSA2_ERR_INDEX);  // a visible tile without a valid page: the epilogue drops it
+            mbar_arrive(&full[s]);
+          }
+        }
+      }
+    } else {
+      // gather: lane l copies the 16-byte pieces of entries l, l + 32, l + 64, l + 96
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % PF_STAGES;
+        if (!mbar_wait_bounded(&empty[s], ((i / PF_STAGES) & 1) ^ 1, abort_flag, PF_WAIT_NS)) break;
+        const uint32_t st = stages + s * PF_STAGE_BYTES;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = lane + 32 * j, n = i * PF_TILE + e, m = pf_row_of_entry(e);
+          const int64_t slot = n < nvis_max ? cache_slot(a.c, b, n) : -1;
+          if (slot >= 0) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              cp_async_16(st + m * 64 + ((c ^ ((m >> 1) & 3)) << 4), a.c.ix_codes + slot * CSA2_IX_CODE_BYTES + c * 16);
+            cp_async_4(st + PF_A_BYTES + e * 4, a.c.ix_scales + slot * CSA2_IX_SCALE_BYTES);
+          } else if (n < nvis_max) {
+            report(a.err, CSA2_ERR_INDEX);
+          }
+        }
+        cp_async_arrive_noinc(&full[s]);
+      }
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t stages = smem_u32(smem + PS_STAGES);
+      uint64_t bd0[PF_Q], bd1[PF_Q];
+#pragma unroll
+      for (int qi = 0; qi < PF_Q; ++qi) {
+        const uint32_t bq = smem_u32(smem + PS_B + qi * 4096);
+        tc_cp_32x128b_warpx4(tmem + PF_COL_SFB + 4 * qi,
+                             smem_desc(smem_u32(smem + PS_SFB + qi * 512), 16, 128, LAYOUT_SWIZZLE_NONE));
+        bd0[qi] = smem_desc(bq, 16, 512, LAYOUT_SWIZZLE_64B);
+        bd1[qi] = smem_desc(bq + 32, 16, 512, LAYOUT_SWIZZLE_64B);
+      }
+      constexpr uint32_t id0 = idesc_mxf4(PF_TILE, PF_N, 0, 0);
+      constexpr uint32_t id1 = idesc_mxf4(PF_TILE, PF_N, 2, 2);
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % PF_STAGES, buf = i & 1;
+        if (!mbar_wait_bounded(&full[s], (i / PF_STAGES) & 1, abort_flag, PF_WAIT_NS)) break;
+        if (!mbar_wait_bounded(&acc_empty[buf], ((i >> 1) & 1) ^ 1, abort_flag, PF_WAIT_NS)) break;
+        if (!a.use_tma) fence_proxy_async_smem();  // cp.async-filled stages are read by the tensor core
+        tc_fence_after();
+        const uint32_t st = stages + s * PF_STAGE_BYTES;
+        const uint32_t sfa = tmem + PF_COL_SFA + 4 * buf;
+        tc_cp_32x128b_warpx4(sfa, smem_desc(st + PF_A_BYTES, 16, 128, LAYOUT_SWIZZLE_NONE));
+        const uint64_t a0 = smem_desc(st, 16, 512, LAYOUT_SWIZZLE_64B);
+        const uint64_t a1 = smem_desc(st + 32, 16, 512, LAYOUT_SWIZZLE_64B);
+#pragma unroll
+        for (int qi = 0; qi < PF_Q; ++qi) {
+          const uint32_t d = tmem + (buf * PF_Q + qi) * PF_N;
+          tc_mma_mxf4(d, a0, bd0[qi], id0, sfa, tmem + PF_COL_SFB + 4 * qi, false);
+          tc_mma_mxf4(d, a1, bd1[qi], id1, sfa, tmem + PF_COL_SFB + 4 * qi, true);
+        }
+        tc_commit(&empty[s]);
+        tc_commit(&acc_full[buf]);
+      }
+      tc_commit(done);
+      const uint64_t t_start = globaltimer();
+      while (!mbar_try_wait(done, 0) && globaltimer() - t_start < PF_WAIT_NS) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int t = threadIdx.x - 64;
+    const int q4 = warp & 3, wg = (warp - 2) >> 2;
+    const int e = pf_entry_of_row(32 * q4 + lane);  // tile entry of this thread's accumulator row
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    uint32_t *scr_key = reinterpret_cast<uint32_t *>(smem + PS_SCR);
+    int32_t *scr_ent = reinterpret_cast<int32_t *>(smem + PS_SCR + PF_KMAX * 4);
+    bool ok = true;
+    const int rounds = (ntiles + 1) / 2;
+    for (int r = 0; r < rounds; ++r) {
+      const int i = 2 * r + wg;  // this warpgroup's tile of the round (accumulator set wg)
+      if (i < ntiles && ok) {
+        if (!mbar_wait_bounded(&acc_full[wg], (i >> 1) & 1, abort_flag, PF_WAIT_NS)) {
+          ok = false;
+        } else {
+          tc_fence_after();
+          float sc[PF_Q];
+#pragma unroll
+          for (int qi = 0; qi < PF_Q; ++qi) {
+            const uint32_t taddr = tmem + (uint32_t(32 * q4) << 16) + (wg * PF_Q + qi) * PF_N;
+            uint32_t r0[32], r1[32];
+            tc_ld_32x32b_x32(taddr, r0);
+            tc_ld_32x32b_x32(taddr + 32, r1);
+            tc_wait_ld();
+            const float4 *w4 = reinterpret_cast<const float4 *>(ws + qi * 64);
+            float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int h4 = 0; h4 < 8; ++h4) {
+              const float4 wv = w4[h4];
+              part[(4 * h4) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(r0[4 * h4]), 0.f), part[(4 * h4) & 7]);
+              part[(4 * h4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(r0[4 * h4 + 1]), 0.f), part[(4 * h4 + 1) & 7]);
+              part[(4 * h4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(r0[4 * h4 + 2]), 0.f), part[(4 * h4 + 2) & 7]);
+              part[(4 * h4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(r0[4 * h4 + 3]), 0.f), part[(4 * h4 + 3) & 7]);
+            }
+#pragma unroll
+            for (int h4 = 0; h4 < 8; ++h4) {
+              const float4 wv = w4[8 + h4];
+              part[(4 * h4) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(r1[4 * h4]), 0.f), part[(4 * h4) & 7]);
+              part[(4 * h4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(r1[4 * h4 + 1]), 0.f), part[(4 * h4 + 1) & 7]);
+              part[(4 * h4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f), part[(4 * h4 + 2) & 7]);
+              part[(4 * h4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f), part[(4 * h4 + 3) & 7]);
+            }
+            sc[qi] = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[wg]);
+          // append the keys above each query's threshold (one atomic per warp and query); an
+          // entry without a valid page is never a candidate (its error is already reported)
+          const int n = i * PF_TILE + e;
+          const bool live = n < nvis_max && cache_slot(a.c, b, n) >= 0;
+#pragma unroll
+          for (int qi = 0; qi < PF_Q; ++qi) {
+            const uint32_t key = score_key(sc[qi]);
+            const bool pass = live && n < qvis[qi] && key > qthr[qi];
+            const uint32_t m = __ballot_sync(0xffffffffu, pass);
+            if (m) {
+              int base = 0;
+              if (lane == 0) base = atomicAdd(&qcnt[qi], __popc(m));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              if (pass) {
+                const int at = base + __popc(m & lt_mask);
+                ckey[qi * PF_CAP + at] = key;
+                cent[qi * PF_CAP + at] = n;
+              }
+            }
+          }
+        }
+      }
+      epi_sync();  // both tiles of the round are in the lists
+      int cnt[PF_Q];
+#pragma unroll
+      for (int qi = 0; qi < PF_Q; ++qi) cnt[qi] = qcnt[qi];
+      epi_sync();  // every thread holds the counts before the next round appends to them
+#pragma unroll 1
+      for (int qi = 0; qi < PF_Q; ++qi) {
+        if (cnt[qi] > PF_CAP - 2 * PF_TILE) {  // the next round could overflow: cut to the best k
+          const uint32_t T = cut_to_k(ckey + qi * PF_CAP, cent + qi * PF_CAP, &qcnt[qi], a.k, scr_key, scr_ent,
+                                      hist, sel, t);
+          if (t == 0) qthr[qi] = T;
+          epi_sync();
+        }
+      }
+    }
+    // final: each query's best k, in ascending entry order, -1 padded
+#pragma unroll 1
+    for (int qi = 0; qi < nq; ++qi) {
+      if (qcnt[qi] > a.k) {
+        cut_to_k(ckey + qi * PF_CAP, cent + qi * PF_CAP, &qcnt[qi], a.k, scr_key, scr_ent, hist, sel, t);
+      }
+      const int m = qcnt[qi];
+      int32_t *orow = a.idx + (int64_t(b) * a.Q + q0 + qi) * a.k;
+      for (int j = t; j < m; j += PF_EPI) {
+        const int ej = cent[qi * PF_CAP + j];
+        int rank = 0;
+        for (int l = 0; l < m; ++l) rank += cent[qi * PF_CAP + l] < ej;
+        orow[rank] = ej;
+      }
+      for (int j = m + t; j < a.k; j += PF_EPI) orow[j] = -1;
+      epi_sync();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, PF_TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) report(a.err, CSA2_ERR_TIMEOUT);
+}
+
+void launch_prefill_index(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos, int k,
+                          int max_entries, const csa2_cache &c, int32_t *idx, int32_t *err, cudaStream_t st) {
+  if (B == 0 || Q == 0) return;
+  CUtensorMap tmap;
+  memset(&tmap, 0, sizeof(tmap));
+  const bool use_tma = make_index_code_map(&tmap, c);
+  PrefillArgs a{use_tma, q_ix, w, Q, q_pos, k, max_entries, c, idx, err};
+  set_smem_limit(prefill_index_kernel, PF_SMEM);
+  prefill_index_kernel<<<dim3((Q + PF_Q - 1) / PF_Q, B), PF_THREADS, PF_SMEM, st>>>(tmap, a);
+}
+
+}  // namespace csa2

@@ -118,7 +118,9 @@ csa2_status csa2_check(const int32_t *err, csa2_stream_t stream);
 /*
  * Bytes of workspace csa2_sparse_attn needs for these sizes (0 for Reuse, and for
  * Dense up to 4096 entries).  max_entries bounds num_entries[b]; pool_k is the
- * candidate-pool size (0 if none).
+ * candidate-pool size (0 if none).  Full mode with B * Q >= 1024 query rows and no
+ * pool (a prefill chunk) selects without materialising scores and needs only the
+ * B * Q * k selection.
  */
 size_t csa2_workspace_size(csa2_mode mode, int32_t B, int32_t Q, int32_t max_entries,
                            int32_t k, int32_t pool_k);
@@ -209,11 +211,34 @@ csa2_status csa2_topk(const float *scores, const int32_t *n_valid, int32_t R, in
                       csa2_stream_t stream);
 
 /*
+ * The Full-mode selection of a chunk of query tokens without materialising scores
+ * ("DeepSeek V4.1 Flash 深度解析", 序: prefill compute, HBM and SSD capacity are the
+ * bottlenecks; "从V4到V4.1 Flash", 编码器层: prefill runs the encoder's CSA2 layers over
+ * the whole prompt).  For every query: the scores of csa2_index_score over the entries
+ * it sees, then the top-k of csa2_topk -- the same selection, bit for bit.  Three
+ * query tokens share each key tile loaded; each keeps a running top-k on chip.
+ *   q_ix [B][Q][64][128], w [B][Q][64] bf16; q_pos [B][Q]; idx [B][Q][k] int32,
+ *   ascending entries, -1 padded; k <= 512.  No workspace.
+ * Efficient for hundreds of query tokens or more (a prefill chunk); decode rows are
+ * better served by csa2_index_score + csa2_topk, which spread one row over the GPU.
+ * Device errors: a query that sees more than max_entries entries -> CSA2_ERR_SHAPE
+ * (only the first max_entries are scored); a bad page -> CSA2_ERR_INDEX.
+ */
+csa2_status csa2_index_topk(const uint16_t *q_ix, const uint16_t *w, int32_t B, int32_t Q,
+                            const int32_t *q_pos, int32_t k, int32_t max_entries,
+                            const csa2_cache *cache, int32_t *idx, int32_t *err,
+                            csa2_stream_t stream);
+
+/*
  * Sparse attention of one CSA2 layer ("从V4到V4.1 Flash", section CSA2架构: the
  * Full, Reindex and Reuse modes; section 解码器层: the hierarchical pool).
  *   q [B][Q][64][512] bf16 query heads; q_pos [B][Q]; softmax_scale tau.
  *   FULL:    q_ix, w (as csa2_index_score) select top-k of all visible entries;
  *            if pool_k > 0 the top-pool_k entries are written to pool_io [B][Q][pool_k].
+ *            With B * Q >= 1024 rows and pool_k = 0 (prefill) the indexer scores three
+ *            query tokens per key tile and keeps each one's running top-k on chip
+ *            ("DeepSeek V4.1 Flash 深度解析", 序: prefill compute is the bottleneck);
+ *            the selection is the same as scoring and csa2_topk would give.
  *   REINDEX: q_ix, w score the entries listed in pool_io [B][Q][pool_k]; top-k of them.
  *   REUSE:   idx_in [B][Q][k] given entry indices (-1 = none; order free).
  *   DENSE:   every visible entry (q_ix, w, k, pool and indices unused); the caches of

@@ -647,6 +647,67 @@ def test_query_magnitudes_are_exact(case, B):
         check_attention(to_np(o[b, 0]), to_np(lse[b, 0]), ref["o"], ref["lse"], f"{case} b={b}")
 
 
+# ------------------------------------------------------------------ fused prefill indexer
+@pytest.mark.parametrize("tma", [False, True])
+def test_prefill_fused_selection(tma):
+    """A prefill chunk of 1100 query tokens (Full mode, no pool) selects with the fused indexer:
+    every row's top-512 must equal the unfused path's (materialised scores + csa2_topk) bit for
+    bit, the same fp32 score arithmetic feeding the same exact selection; sampled rows against
+    the oracle too.  tma: a cache layout the tensor map can describe, or the gathering path."""
+    k = K()
+    spec = W.scaled(W.prefill8k(), [6000 + 1100], B=1, q_len=1100)
+    if tma:
+        cache = k.GlobalKVCache(1, spec.ratio, seq_stride=(spec.max_entries + 127) // 128 * 128)
+        kv, ix = W.token_latents(spec, 0, DEV)
+        k.csa2_pack_kv(kv[None].contiguous(), ix[None].contiguous(), torch.zeros(1, dtype=torch.int32, device=DEV),
+                       cache, err=_err())
+        cache.num_entries[0] = spec.entries(0)
+    else:
+        cache = gpu_cache(spec)
+    q, q_ix, w, q_pos = W.query_tensors(spec, 0, DEV)
+    err = _err()
+    assert k.csa2_workspace_size("full", 1, spec.q_len, spec.max_entries, spec.k) == spec.q_len * spec.k * 4
+    idx = torch.empty((1, spec.q_len, spec.k), dtype=torch.int32, device=DEV)
+    k.csa2_sparse_attn("full", q, q_pos, cache, spec.tau, spec.max_entries, q_ix=q_ix, w=w, idx_out=idx, err=err)
+    scores = k.csa2_index_score(q_ix, w, q_pos, cache, spec.max_entries, err=err)
+    ref = k.csa2_topk(scores, spec.k)[0]
+    assert k.csa2_check(err) == 0
+    assert torch.equal(idx, ref), f"{int((idx != ref).any(-1).sum())} rows differ"
+    c = oracle_seq(spec, 0, main_rows=[], gen_device=DEV)
+    for qi in (0, 1, 2, 511, 512, 1097, 1098, 1099):
+        p = int(q_pos[0, qi])
+        ref_idx, _, s = OC.full_select(c, 0, p, to_np(q_ix[0, qi]), to_np(w[0, qi]), spec.k)
+        check_topk(to_np(idx[0, qi]), s, ref_idx, spec.k, f"fused prefill q={qi}")
+
+
+def test_prefill_fused_ties_and_short_rows():
+    """Rows of one repeated score (every key ties: the lowest entries win), rows that see fewer
+    entries than k (all of them, -1 padded) and a chunk whose length is not a multiple of the
+    CTA's three query tokens."""
+    k = K()
+    spec = W.scaled(W.prefill8k(), [2 * 700 + 1025], B=1, q_len=1025)
+    cache = gpu_cache(spec)
+    q, q_ix, w, q_pos = W.query_tensors(spec, 0, DEV)
+    q_ix = q_ix.clone()
+    q_ix[0, :400] = 0.0            # every score 0: ties everywhere
+    q_pos = q_pos.clone()
+    q_pos[0, 400:420] = torch.arange(20, device=DEV, dtype=torch.int32) * 50   # early positions: few entries
+    err = _err()
+    idx = torch.empty((1, spec.q_len, spec.k), dtype=torch.int32, device=DEV)
+    k.csa2_sparse_attn("full", q, q_pos, cache, spec.tau, spec.max_entries, q_ix=q_ix, w=w, idx_out=idx, err=err)
+    scores = k.csa2_index_score(q_ix, w, q_pos, cache, spec.max_entries, err=err)
+    ref = k.csa2_topk(scores, spec.k)[0]
+    assert k.csa2_check(err) == 0
+    assert torch.equal(idx, ref), f"{int((idx != ref).any(-1).sum())} rows differ"
+    assert torch.equal(idx[0, 0], torch.arange(512, dtype=torch.int32, device=DEV))   # ties: lowest entries
+    for qi in range(400, 420):
+        nvis = min(spec.entries(0), (int(q_pos[0, qi]) + 1) // 2)
+        want = list(range(min(nvis, 512))) if nvis <= 512 else None
+        if want is not None:
+            got = to_np(idx[0, qi])
+            assert got[:nvis].tolist() == want and (got[nvis:] == -1).all()
+
+
 # ------------------------------------------------------------------ gated compressor and decode-time append
 @pytest.mark.parametrize("ratio", [1, 2, 4, 128])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
