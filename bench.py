@@ -192,11 +192,11 @@ class Hier1M:
         torch.cuda.synchronize()
         assert k.csa2_check(err) == 0
 
-    # kernels launched per step, by call: pack_kv 1; per layer pack_swa 1, indexer 1, top-k 1 (the Full layer's
-    # top-512 and pool share one launch) and one attention launch that covers the sparse branch, the SWA
-    # branch and their log-sum-exp merge
+    # kernels launched per step, by call: pack_kv 1; per layer pack_swa 1 and one attention launch that covers
+    # the sparse branch, the SWA branch and their log-sum-exp merge; the Full layer's indexer scan 1 and top-k 1
+    # (its top-512 and pool share one launch); per Reindex layer one launch that scores the pool and selects
     def launches_per_step(self):
-        return 1 + self.LAYERS * 4
+        return 1 + 4 + (self.LAYERS - 1) * 3
 
     # The step in three parts: [pack the new token's entry; pack layer 0's SWA token], [the Full layer's
     # scan], [its top-k and attention; the four Reindex layers].  The scan stays a separate part so that
@@ -369,10 +369,12 @@ class Model40:
         torch.cuda.synchronize()
 
     def launches_per_step(self):
-        """Kernels of one step: one append per cache, per Full or Reindex layer an indexer scan and a
-        top-k, and per layer one attention launch (which also packs the layer's window token)."""
-        sel = sum(1 for m, _, _ in self.plan if m in (0, 1))
-        return len(self.ratios) + 2 * sel + len(self.plan)
+        """Kernels of one step: one append per cache, per Full layer an indexer scan and a top-k, per
+        Reindex layer one launch that scores its pool and selects, and per layer one attention launch
+        (which also packs the layer's window token)."""
+        full = sum(1 for m, _, _ in self.plan if m == 0)
+        reindex = sum(1 for m, _, _ in self.plan if m == 1)
+        return len(self.ratios) + 2 * full + reindex + len(self.plan)
 
     def reindex_recall(self):
         """Per Reindex layer: the share of its top-k (searched inside the decoder pool) that an exact
@@ -611,7 +613,13 @@ class OneLayer:
         return self.spec.B * self.spec.q_len
 
     def launches_per_step(self):
-        return sum(3 if mode == "full" else 1 for mode, *_ in self.calls)
+        """Full: indexer scan, top-k and attention, or for a prefill chunk (1024 rows or more) the fused
+        indexer + top-k and attention; Reuse: attention."""
+        n = 0
+        for (mode, *_), io in zip(self.calls, self.io):
+            rows = io[0].shape[0] * io[0].shape[1]
+            n += (2 if rows >= 1024 else 3) if mode == "full" else 1
+        return n
 
     def gather_bytes(self):
         """Bytes the attention must move per step: per query row its listed main entries (288 B each),

@@ -90,7 +90,8 @@ CSA2_EXPORT size_t csa2_workspace_size(csa2_mode mode, int32_t B, int32_t Q, int
   switch (mode) {
     case CSA2_MODE_FULL:
       return (fused_prefill(int64_t(rows), pool_k) ? 0 : round256(rows * max_entries * 4)) + round256(rows * k * 4);
-    case CSA2_MODE_REINDEX: return round256(rows * pool_k * 4) + round256(rows * k * 4);
+    case CSA2_MODE_REINDEX:  // pools of at most REINDEX_SELECT_MAX: scores never leave the chip
+      return (pool_k <= csa2::REINDEX_SELECT_MAX ? 0 : round256(rows * pool_k * 4)) + round256(rows * k * 4);
     case CSA2_MODE_DENSE:  // partial (o, lse) of one key segment beyond the first
       return max_entries > kDenseMinSegment ? round256(rows * CSA2_HEADS * CSA2_MAIN_DIM * 4) +
                                                   round256(rows * CSA2_HEADS * 4)
@@ -239,13 +240,17 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
     }
     const int n_out = mode == CSA2_MODE_FULL ? max_entries : pool_k;
     if (rows > 65535) return fail(CSA2_ERR_UNSUPPORTED, "more than 65535 query rows per call");
+    const bool fused_select = mode == CSA2_MODE_REINDEX && pool_k <= csa2::REINDEX_SELECT_MAX;
     float *scores = static_cast<float *>(ws);
-    int32_t *sel = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + round256(size_t(rows) * n_out * 4));
+    int32_t *sel = reinterpret_cast<int32_t *>(static_cast<char *>(ws) +
+                                               (fused_select ? 0 : round256(size_t(rows) * n_out * 4)));
     if (idx_out) sel = idx_out;
     if (mode == CSA2_MODE_FULL) {
       csa2::launch_index_score_mma(q_ix, w, B, Q, q_pos, nullptr, 0, max_entries, *cache, scores, err, stream);
       csa2::launch_topk_cluster(scores, nullptr, rows, max_entries, k, sel, nullptr, pool_k,
                                 pool_k > 0 ? pool_io : nullptr, nullptr, nullptr, stream);
+    } else if (fused_select) {
+      csa2::launch_reindex_select(q_ix, w, B, Q, q_pos, pool_io, pool_k, k, *cache, sel, err, stream);
     } else {
       csa2::launch_index_score_mma(q_ix, w, B, Q, q_pos, pool_io, pool_k, pool_k, *cache, scores, err, stream);
       csa2::launch_topk_cluster(scores, nullptr, rows, pool_k, k, sel, nullptr, 0, nullptr, nullptr, pool_io, stream);

@@ -70,7 +70,7 @@ size_t scores_bytes(const csa2_decode_args &a) {
   for (int l = 0; l < a.n_layers; ++l) {
     const int m = a.plan[l].mode;
     if (m == CSA2_MODE_FULL) n = std::max(n, size_t(a.max_entries[a.plan[l].cache]));
-    if (m == CSA2_MODE_REINDEX) n = std::max(n, size_t(a.pool_k));
+    if (m == CSA2_MODE_REINDEX && a.pool_k > csa2::REINDEX_SELECT_MAX) n = std::max(n, size_t(a.pool_k));
   }
   return round256(size_t(a.B) * n * 4);
 }
@@ -131,7 +131,8 @@ CSA2_EXPORT csa2_status csa2_decode_step(const csa2_decode_args *a, void *ws, si
   }
   if (need_ix && (!a->q_ix || !a->w)) return fail(CSA2_ERR_INVALID_ARG, "Full/Reindex layers need q_ix and w");
   if (need_pool && (!a->pool || a->pool_k < a->k)) return fail(CSA2_ERR_INVALID_ARG, "Reindex needs pool, pool_k >= k");
-  if (need_ix && (!ws || ws_bytes < scores_bytes(*a))) return fail(CSA2_ERR_INVALID_ARG, "workspace too small");
+  const size_t need_ws = scores_bytes(*a);
+  if (need_ws > 0 && (!ws || ws_bytes < need_ws)) return fail(CSA2_ERR_INVALID_ARG, "workspace too small");
   int rmax = 1;
   for (int c = 0; c < a->n_caches; ++c) rmax = std::max(rmax, int(a->caches[c].ratio));
   if (a->new_kv && (!a->new_ix || (rmax > 1 && !a->kv_stage)))
@@ -168,6 +169,8 @@ CSA2_EXPORT csa2_status csa2_decode_step(const csa2_decode_args *a, void *ws, si
         csa2::launch_index_score_mma(qix, w, B, 1, a->pos, nullptr, 0, me, cc, scores, err, st);
         csa2::launch_topk_cluster(scores, nullptr, B, me, a->k, idx_l, nullptr, pool ? a->pool_k : 0,
                                   pool ? pool_c : nullptr, nullptr, nullptr, st);
+      } else if (a->pool_k <= csa2::REINDEX_SELECT_MAX) {
+        csa2::launch_reindex_select(qix, w, B, 1, a->pos, pool_c, a->pool_k, a->k, cc, idx_l, err, st);
       } else {
         csa2::launch_index_score_mma(qix, w, B, 1, a->pos, pool_c, a->pool_k, a->pool_k, cc, scores, err, st);
         csa2::launch_topk_cluster(scores, nullptr, B, a->pool_k, a->k, idx_l, nullptr, 0, nullptr, nullptr, pool_c,

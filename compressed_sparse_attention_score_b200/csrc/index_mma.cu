@@ -23,6 +23,7 @@
 // the keys).
 // Every mbarrier wait is time-bounded; on expiry the CTA drains and reports
 // CSA2_ERR_TIMEOUT instead of hanging.
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -34,6 +35,7 @@
 
 namespace csa2 {
 using namespace sm100;
+namespace cg = cooperative_groups;
 
 namespace {
 constexpr int IM_STAGES = 8;
@@ -60,6 +62,16 @@ constexpr int N_BARS = 2 * IM_STAGES + 2 * IM_ACC + 1;
 constexpr int SM_MISC = SM_BAR + 8 * N_BARS;            // tmem base, abort flag
 constexpr int SM_TOTAL = SM_MISC + 16;
 constexpr size_t IM_SMEM_BYTES = SM_TOTAL + 1024;       // slack for 1024-byte alignment
+// Fused Reindex selection: each CTA keeps its candidates' keys; only digit histograms and
+// counts cross the cluster.
+constexpr int IM_SEL_MAX = REINDEX_SELECT_MAX;          // candidates per row
+constexpr int SM_KEYS = SM_TOTAL;                       // [IM_CAND_TILES * 128] this CTA's keys
+constexpr int SM_HL = SM_KEYS + IM_CAND_TILES * IM_TILE * 4;   // local 256-bin histogram
+constexpr int SM_HG = SM_HL + 256 * 4;                  // [2][256] cluster-wide histograms (peers add here)
+constexpr int SM_CG = SM_HG + 2 * 256 * 4;              // [16][2] every CTA's counts above / equal
+constexpr int SM_SELW = SM_CG + 16 * 2 * 4;             // selection state (4 words)
+constexpr int SM_WCNT = SM_SELW + 16;                   // per warp: keys above / equal to the threshold
+constexpr size_t IM_SEL_SMEM_BYTES = SM_WCNT + 2 * (IM_THREADS / 32) * 4 + 1024;
 }  // namespace
 
 struct IndexMmaArgs {
@@ -75,14 +87,141 @@ struct IndexMmaArgs {
   float *scores;
   int32_t *err;
   int chunk;  // tiles per CTA
+  int k;         // fused selection: top-k of the candidates ...
+  int32_t *sel;  // ... written here [rows][k] (entries, ascending; -1 pads)
 };
 
 // A-operand row of tile entry e and the inverse map.
 __device__ __forceinline__ int row_of_entry(int e) { return (e & 3) * 32 + (e >> 2); }
 __device__ __forceinline__ int entry_of_row(int m) { return (m & 31) * 4 + (m >> 5); }
 
-__global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __grid_constant__ CUtensorMap tmap,
-                                                                        IndexMmaArgs a) {
+// Top-k of one row's candidates spread over the CS CTAs of a cluster (CTA r holds positions
+// [pos0, pos0 + nl) of the row: keys kl, entries el), score descending and position ascending
+// among equal scores, -inf keys never chosen; written as the chosen candidates' entries in
+// position order, -1 padded -- the selection csa2_topk makes of the same scores with the
+// candidate list as its map.  The threshold key comes from a radix selection on 8-bit digits
+// from the top: per digit every CTA histograms its own keys and adds the histogram into every
+// peer's, one cluster barrier, and every CTA finds the same threshold digit; it stops early once
+// the threshold bin holds exactly the keys still needed.  A last exchange of per-CTA counts
+// places each CTA's chosen entries.  Called by every thread of every CTA of the cluster.
+__device__ __forceinline__ void select_cluster(const uint32_t *kl, const int32_t *el, int nl, int k, int32_t *orow,
+                                               uint32_t *hl, uint32_t *hg, int *cg_, uint32_t *selw, int *wcnt) {
+  constexpr int NW = IM_THREADS / 32;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int cs = int(cluster.num_blocks()), rank = int(cluster.block_rank());
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  uint32_t prefix = 0;
+  int need = k, width = 0;
+  bool all = false;
+  for (int pass = 0, shift = 24; shift >= 0; ++pass, shift -= 8) {
+    uint32_t *hcur = hg + (pass & 1) * 256;
+    if (t < 256) hl[t] = 0;
+    __syncthreads();
+    const uint32_t himask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+    for (int i = t; i - lane < nl; i += IM_THREADS) {  // lanes with the same bin add once
+      const uint32_t key = i < nl ? kl[i] : KEY_NEG_INF;
+      const bool act = key != KEY_NEG_INF && (key & himask) == prefix;
+      const uint32_t am = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t bin = (key >> shift) & 255u, peers = __match_any_sync(am, bin);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hl[bin], uint32_t(__popc(peers)));
+      }
+    }
+    __syncthreads();
+    for (int j = t; j < 256 * cs; j += IM_THREADS) {  // into every CTA's copy, this one's included
+      const uint32_t c = hl[j & 255];
+      if (c) atomicAdd(cluster.map_shared_rank(hcur + (j & 255), j >> 8), c);
+    }
+    if (t < 256) hg[((pass + 1) & 1) * 256 + t] = 0;  // the next digit's copy: read last before the previous barrier
+    cluster.sync();
+    if (warp == 0) {  // the digit at which the count from the top reaches `need`
+      uint32_t c8[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) sum += (c8[j] = hcur[255 - (8 * lane + j)]);
+      uint32_t x = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      const uint32_t excl = x - sum, total = __shfl_sync(0xffffffffu, x, 31);
+      if (total <= uint32_t(need)) {  // first digit only: at most k valid keys, all chosen
+        if (lane == 0) selw[0] = 0xFFFFFFFFu;
+      } else {
+        const int L = __ffs(__ballot_sync(0xffffffffu, excl < uint32_t(need) && x >= uint32_t(need))) - 1;
+        if (lane == L) {
+          uint32_t cum = excl;
+#pragma unroll 1
+          for (int j = 0; j < 8; ++j) {
+            if (cum + c8[j] >= uint32_t(need)) {
+              selw[0] = uint32_t(255 - (8 * lane + j));
+              selw[1] = uint32_t(need) - cum;
+              selw[2] = c8[j];
+              break;
+            }
+            cum += c8[j];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (selw[0] == 0xFFFFFFFFu) {
+      all = true;
+      break;
+    }
+    prefix |= selw[0] << shift;
+    need = int(selw[1]);
+    width = 32 - shift;
+    if (int(selw[2]) == need) break;  // every key of the threshold bin is chosen
+  }
+  // keys above / equal to the threshold T, compared on the top `width` bits
+  const int sh = 32 - width;
+  const uint32_t T = all ? 0u : prefix >> sh;
+  const int seg = ((nl + NW * 32 - 1) / (NW * 32)) * 32, j0 = warp * seg, j1 = min(nl, j0 + seg);
+  int gt = 0, eq = 0;
+  for (int j = j0 + lane; j - lane < j1; j += 32) {
+    const uint32_t key = j < j1 ? kl[j] : KEY_NEG_INF;
+    const bool valid = key != KEY_NEG_INF;
+    gt += __popc(__ballot_sync(0xffffffffu, valid && (all || (key >> sh) > T)));
+    eq += __popc(__ballot_sync(0xffffffffu, valid && !all && (key >> sh) == T));
+  }
+  if (lane == 0) wcnt[2 * warp] = gt, wcnt[2 * warp + 1] = eq;
+  __syncthreads();
+  if (t < cs) {  // this CTA's totals into every CTA's table
+    int g = 0, e = 0;
+    for (int w2 = 0; w2 < NW; ++w2) g += wcnt[2 * w2], e += wcnt[2 * w2 + 1];
+    int *dst = cluster.map_shared_rank(cg_ + 2 * rank, t);
+    dst[0] = g;
+    dst[1] = e;
+  }
+  cluster.sync();  // no shared memory of a peer is touched after this barrier
+  int g = 0, e = 0, gall = 0, eall = 0;
+  for (int r = 0; r < cs; ++r) {
+    if (r < rank) g += cg_[2 * r], e += cg_[2 * r + 1];
+    gall += cg_[2 * r];
+    eall += cg_[2 * r + 1];
+  }
+  for (int w2 = 0; w2 < warp; ++w2) g += wcnt[2 * w2], e += wcnt[2 * w2 + 1];
+  const int nd = all ? 0 : need;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int j = j0 + lane; j - lane < j1; j += 32) {
+    const uint32_t key = j < j1 ? kl[j] : KEY_NEG_INF;
+    const bool valid = key != KEY_NEG_INF;
+    const bool is_gt = valid && (all || (key >> sh) > T), is_eq = valid && !all && (key >> sh) == T;
+    const uint32_t gm = __ballot_sync(0xffffffffu, is_gt), em = __ballot_sync(0xffffffffu, is_eq);
+    const int gbef = g + __popc(gm & lt_mask), ebef = e + __popc(em & lt_mask);
+    const int at = is_gt ? gbef + min(ebef, nd) : ((is_eq && ebef < nd) ? gbef + ebef : -1);
+    if (at >= 0 && at < k) orow[at] = el[j];
+    g += __popc(gm);
+    e += __popc(em);
+  }
+  if (rank == 0)
+    for (int i = gall + min(eall, nd) + t; i < k; i += IM_THREADS) orow[i] = -1;
+}
+
+template <bool SEL>
+__global__ void __launch_bounds__(IM_THREADS, SEL ? 1 : 2) index_score_mma_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                                                 IndexMmaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM_BAR);
@@ -116,18 +255,17 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
   if (warp == 0) {
     tmem_alloc(tmem_slot, IM_TMEM_COLS);
     tmem_relinquish();
-    if (cand_staged) {
+    if (cand_staged) {  // every index copy in flight at once (asynchronous copies), then one wait
       const int32_t *crow = a.cand + int64_t(row) * a.P;
-      for (int i0 = 0; i0 < ntiles * IM_TILE; i0 += 4 * 32) {
-        int32_t v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int pos = t0 * IM_TILE + i0 + 32 * u + lane;
-          v[u] = pos < a.P ? crow[pos] : -1;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) cand_s[i0 + 32 * u + lane] = v[u];
+      for (int i = lane; i < ntiles * IM_TILE; i += 32) {
+        const int pos = t0 * IM_TILE + i;
+        if (pos < a.P)
+          cp_async_4(smem_u32(cand_s + i), crow + pos);
+        else
+          cand_s[i] = -1;
       }
+      cp_async_commit();
+      cp_async_wait<0>();
     }
   } else if (warp == 1 && lane == 0) {
     for (int s = 0; s < IM_STAGES; ++s) {
@@ -179,6 +317,8 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     }
     const uint32_t sfword = sfpart | __shfl_xor_sync(0xffffffffu, sfpart, 1);
     // scale atom word of row r: lane-row r % 32, column r / 32 (rows 64..127 unused, zero)
+    if constexpr (SEL)
+      for (int j = t; j < 512; j += 128) reinterpret_cast<uint32_t *>(smem + SM_HG)[j] = 0;
     if ((t & 1) == 0) {
       *reinterpret_cast<uint32_t *>(smem + SM_SFB + (h & 31) * 16 + (h >> 5) * 4) = sfword;
       ws[h] = bf16_to_f32(a.w[int64_t(row) * HI + h]);
@@ -192,6 +332,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if constexpr (SEL) cluster_arrive();  // this CTA has started and zeroed its histograms (waited on before the selection)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
@@ -313,6 +454,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     // warpgroup wg takes tiles wg, wg + IM_EPI_WG, ...; the entry behind this thread's
     // row is fetched one of its tiles ahead (candidate lists are read from global)
     const int wg = (warp - 2) >> 2;
+    uint32_t *keys_l = reinterpret_cast<uint32_t *>(smem + SM_KEYS);  // fused selection: this CTA's keys
     auto entry_at = [&](int i) -> int64_t {
       const int pos = (t0 + i) * IM_TILE + e;
       if (!a.cand) return pos;
@@ -324,7 +466,9 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       const int acc = i % IM_ACC;
       const int64_t n_cur = n_next;
       n_next = entry_at(i + IM_EPI_WG);
-      if (!mbar_wait_bounded(&acc_full[acc], (i / IM_ACC) & 1, abort_flag, WAIT_LIMIT_NS)) break;
+      // the whole warp takes tcgen05.ld or none of it does
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&acc_full[acc], (i / IM_ACC) & 1, abort_flag, WAIT_LIMIT_NS)))
+        break;
       tc_fence_after();
       const uint32_t taddr = tmem + (uint32_t(32 * q4) << 16) + acc * IM_N;
       uint32_t r0[32], r1[32];
@@ -356,7 +500,10 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       const int pos = (t0 + i) * IM_TILE + e;
       if (pos < a.n_out) {
         const bool ok = n_cur >= 0 && n_cur < nvis && cache_slot(a.c, b, n_cur) >= 0;
-        a.scores[int64_t(row) * a.n_out + pos] = ok ? sc : -INFINITY;
+        if constexpr (SEL)
+          keys_l[pos - t0 * IM_TILE] = score_key(ok ? sc : -INFINITY);
+        else
+          a.scores[int64_t(row) * a.n_out + pos] = ok ? sc : -INFINITY;
       }
     }
     // positions past the visible entries (no key tile was loaded for them)
@@ -374,6 +521,13 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     tmem_dealloc(tmem, IM_TMEM_COLS);
   }
   if (threadIdx.x == 0 && *abort_flag) report(a.err, CSA2_ERR_TIMEOUT);
+  if constexpr (SEL) {
+    cluster_wait();
+    select_cluster(reinterpret_cast<const uint32_t *>(smem + SM_KEYS), cand_s, max(0, min(a.P - t0 * IM_TILE, ntiles * IM_TILE)),
+                   a.k, a.sel + int64_t(row) * a.k, reinterpret_cast<uint32_t *>(smem + SM_HL),
+                   reinterpret_cast<uint32_t *>(smem + SM_HG), reinterpret_cast<int *>(smem + SM_CG),
+                   reinterpret_cast<uint32_t *>(smem + SM_SELW), reinterpret_cast<int *>(smem + SM_WCNT));
+  }
 }
 
 namespace {
@@ -422,8 +576,86 @@ void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int 
   memset(&tmap, 0, sizeof(tmap));
   const bool use_tma = cand == nullptr && make_index_code_map(&tmap, c);
   IndexMmaArgs a{use_tma, q_ix, w, Q, q_pos, cand, P, n_out, c, scores, err, chunk};
-  set_smem_limit(index_score_mma_kernel, IM_SMEM_BYTES);
-  index_score_mma_kernel<<<dim3((t_all + chunk - 1) / chunk, rows), IM_THREADS, IM_SMEM_BYTES, st>>>(tmap, a);
+  set_smem_limit(index_score_mma_kernel<false>, IM_SMEM_BYTES);
+  index_score_mma_kernel<false><<<dim3((t_all + chunk - 1) / chunk, rows), IM_THREADS, IM_SMEM_BYTES, st>>>(tmap, a);
+}
+
+namespace {
+// One-time attributes of the fused-selection kernel for a cluster of CS CTAs, and how many
+// such clusters the device holds at once (0: none).
+template <int CS>
+int select_clusters() {
+  static int cached[64] = {};  // 0 unknown, -1 none
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    if (CS > 8) cudaFuncSetAttribute(index_score_mma_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaFuncSetAttribute(index_score_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         int(IM_SEL_SMEM_BYTES));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CS);
+    cfg.blockDim = dim3(IM_THREADS);
+    cfg.dynamicSmemBytes = IM_SEL_SMEM_BYTES;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = CS;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    cached[dev] =
+        (cudaOccupancyMaxActiveClusters(&n, index_score_mma_kernel<true>, &cfg) == cudaSuccess && n > 0) ? n : -1;
+    cudaGetLastError();
+  }
+  return cached[dev] > 0 ? cached[dev] : 0;
+}
+
+int select_clusters(int cs) {
+  switch (cs) {
+    case 16: return select_clusters<16>();
+    case 8: return select_clusters<8>();
+    case 4: return select_clusters<4>();
+    case 2: return select_clusters<2>();
+    default: return select_clusters<1>();
+  }
+}
+}  // namespace
+
+// Cluster size: at most IM_CAND_TILES tiles per CTA (8 CTAs for a pool of 16384), up to 16 CTAs
+// of about 8 tiles while the rows' clusters fill at most half the SMs (every CTA quantises the
+// row's query again, so many rows take fewer, longer CTAs), and only as large as lets every
+// row's cluster run at once.
+void launch_reindex_select(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
+                           const int32_t *cand, int P, int k, const csa2_cache &c, int32_t *sel, int32_t *err,
+                           cudaStream_t st) {
+  const int rows = B * Q;
+  if (rows == 0 || P == 0) return;
+  const int t_all = (P + IM_TILE - 1) / IM_TILE;
+  int cs_min = 1;  // every CTA's keys and candidate indices fit its shared memory
+  while (cs_min * IM_CAND_TILES < t_all) cs_min *= 2;
+  int cs = cs_min;
+  while (cs < 16 && cs * 8 < t_all && 2 * cs * rows <= sm_count()) cs *= 2;
+  while (cs > cs_min && select_clusters(cs) < min(rows, sm_count() / cs)) cs /= 2;
+  select_clusters(cs);  // sets the kernel's attributes
+  const int chunk = (t_all + cs - 1) / cs;
+  CUtensorMap tmap;
+  memset(&tmap, 0, sizeof(tmap));
+  IndexMmaArgs a{false, q_ix, w, Q, q_pos, cand, P, P, c, nullptr, err, chunk, k, sel};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, rows);
+  cfg.blockDim = dim3(IM_THREADS);
+  cfg.dynamicSmemBytes = IM_SEL_SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = cs;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, index_score_mma_kernel<true>, tmap, a);
 }
 
 }  // namespace csa2

@@ -48,6 +48,14 @@ void launch_append_kv(const void *lat_kv, const void *lat_ix, csa2_dtype dtype, 
 void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
                             const int32_t *cand, int P, int n_out, const csa2_cache &c, float *scores, int32_t *err,
                             cudaStream_t st);
+// Fused Reindex selection: scores of a candidate list of P <= REINDEX_SELECT_MAX entries and
+// their top-k (k <= 512) in one launch, sel [B*Q][k] = the chosen candidates' entries in
+// candidate order (ascending for an ascending list), -1 padded -- what launch_index_score_mma
+// followed by launch_topk_cluster with the list as map returns.
+constexpr int REINDEX_SELECT_MAX = 16384;
+void launch_reindex_select(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
+                           const int32_t *cand, int P, int k, const csa2_cache &c, int32_t *sel, int32_t *err,
+                           cudaStream_t st);
 // Tensor map of a cache's indexer codes as 128-entry groups (false: the layout does not allow one).
 bool make_index_code_map(CUtensorMap *m, const csa2_cache &c);
 // Fused prefill indexer + causal top-k (k <= 512): idx [B][Q][k], ascending, -1 padded.

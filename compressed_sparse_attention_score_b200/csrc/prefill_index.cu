@@ -5,18 +5,17 @@
 // cp.async gathers for caches a tensor map cannot describe) and serves all PF_Q queries: per
 // query two K=64 block-scaled FP4 MMAs (tcgen05 kind::mxf4, N = 64 heads) into the query's
 // accumulator; two sets of accumulators alternate between tiles.  Warp roles:
-//   warp 0     producer;
-//   warp 1     MMA issuer (one lane);
-//   warps 2-9  two epilogue warpgroups on alternate tiles: for each query the weighted-ReLU
-//              score of its 128 keys (the decode kernel's arithmetic, so both give the same
-//              fp32 score); keys the query cannot see are dropped, keys above the query's
-//              running threshold are appended to its candidate list in shared memory.
-// After every pair of tiles the two warpgroups meet; a query whose list could overflow during
-// the next pair is cut back to its best k candidates (radix selection on the scores'
-// order-preserving keys), and its threshold becomes the k-th key: a later key equal to it has
-// a higher entry index and loses the tie.  At the end each query keeps its best k (score
-// descending, entry ascending), written in ascending entry order and padded with -1 -- the
-// selection csa2_topk makes from materialised scores.
+//   warp 0       producer;
+//   warp 1       MMA issuer (one lane);
+//   warps 2-13   one epilogue warpgroup per query: the weighted-ReLU score of each of its 128
+//                keys per tile (the decode kernel's arithmetic, so both give the same fp32
+//                score); keys the query cannot see are dropped, keys above the query's running
+//                threshold are appended to its candidate list in shared memory.
+// A list that could overflow on the next tile is cut back to its best k candidates (radix
+// selection on the scores' order-preserving keys), and its threshold becomes the k-th key: a
+// later key equal to it has a higher entry index and loses the tie.  At the end each query keeps
+// its best k (score descending, entry ascending), written in ascending entry order and padded
+// with -1 -- the selection csa2_topk makes from materialised scores.
 // Every mbarrier wait is time-bounded; on expiry the CTA drains and reports CSA2_ERR_TIMEOUT.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -31,20 +30,22 @@ namespace csa2 {
 using namespace sm100;
 
 namespace {
-constexpr int PF_Q = 3;                 // query tokens per CTA
+constexpr int PF_Q = 3;                 // query tokens per CTA = epilogue warpgroups
 constexpr int PF_STAGES = 8;
 constexpr int PF_TILE = 128;            // keys per tile = MMA M
 constexpr int PF_N = 64;                // indexer heads = MMA N
 constexpr int PF_A_BYTES = PF_TILE * 64;
 constexpr int PF_STAGE_BYTES = 9216;    // 8192 codes + 512 scale atom, padded to 1024
-constexpr int PF_EPI = 256;             // epilogue threads (two warpgroups)
-constexpr int PF_THREADS = 64 + PF_EPI;
+constexpr int PF_WG = 128;              // threads per epilogue warpgroup
+constexpr int PF_THREADS = 64 + PF_Q * PF_WG;
 constexpr int PF_CAP = 4096;            // candidate list per query
 constexpr int PF_KMAX = 512;
 constexpr uint32_t PF_TMEM_COLS = 512;
-constexpr uint32_t PF_COL_SFA = 2 * PF_Q * 64;         // after the two accumulator sets
-constexpr uint32_t PF_COL_SFB = PF_COL_SFA + 8;
+constexpr int PF_ACC = 2;               // accumulator sets (tiles in flight between MMA and epilogue)
+constexpr uint32_t PF_COL_SFA = PF_ACC * PF_Q * 64;    // after the accumulator sets
+constexpr uint32_t PF_COL_SFB = PF_COL_SFA + 4 * PF_ACC;
 constexpr uint64_t PF_WAIT_NS = 2000000000ull;
+static_assert(PF_COL_SFB + 4 * PF_Q <= PF_TMEM_COLS, "accumulators and scale atoms exceed the TMEM allocation");
 
 constexpr int PS_STAGES = 0;
 constexpr int PS_B = PF_STAGES * PF_STAGE_BYTES;          // PF_Q x [64 heads x 64 B] query codes
@@ -52,12 +53,12 @@ constexpr int PS_SFB = PS_B + PF_Q * 4096;                // PF_Q x 512 B scale 
 constexpr int PS_W = PS_SFB + PF_Q * 512;                 // PF_Q x 64 fp32 head weights
 constexpr int PS_CKEY = PS_W + PF_Q * 256;                // PF_Q x PF_CAP keys
 constexpr int PS_CENT = PS_CKEY + PF_Q * PF_CAP * 4;      // PF_Q x PF_CAP entries
-constexpr int PS_SCR = PS_CENT + PF_Q * PF_CAP * 4;       // cut scratch: PF_KMAX keys, PF_KMAX entries
-constexpr int PS_HIST = PS_SCR + PF_KMAX * 8;             // 256-bin histogram
-constexpr int PS_SEL = PS_HIST + 256 * 4;                 // selection state (16 words)
-constexpr int PS_QS = PS_SEL + 64;                        // per query: count, threshold, visible entries
-constexpr int PS_BAR = PS_QS + 4 * PF_Q * 4;
-constexpr int PF_NBARS = 2 * PF_STAGES + 4 + 1;
+constexpr int PS_SCR = PS_CENT + PF_Q * PF_CAP * 4;       // PF_Q x cut scratch: PF_KMAX keys, PF_KMAX entries
+constexpr int PS_HIST = PS_SCR + PF_Q * PF_KMAX * 8;      // PF_Q x 256-bin histogram
+constexpr int PS_SEL = PS_HIST + PF_Q * 256 * 4;          // PF_Q x selection state (4 words)
+constexpr int PS_TCNT = PS_SEL + PF_Q * 16;               // PF_Q x 3 per-tile append counters
+constexpr int PS_BAR = PS_TCNT + 64;
+constexpr int PF_NBARS = 2 * PF_STAGES + 2 * PF_ACC + 1;
 constexpr int PS_MISC = PS_BAR + 8 * PF_NBARS;
 constexpr int PS_TOTAL = PS_MISC + 16;
 constexpr size_t PF_SMEM = PS_TOTAL + 1024;
@@ -80,25 +81,43 @@ namespace {
 __device__ __forceinline__ int pf_row_of_entry(int e) { return (e & 3) * 32 + (e >> 2); }
 __device__ __forceinline__ int pf_entry_of_row(int m) { return (m & 31) * 4 + (m >> 5); }
 
-// Named barrier of the PF_EPI epilogue threads.
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(PF_EPI) : "memory"); }
+// Named barrier of one epilogue warpgroup (ids 1 .. PF_Q).
+__device__ __forceinline__ void wg_sync(int g) { asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "n"(PF_WG) : "memory"); }
+
+// c0 += a0 * b0 and c1 += a1 * b1, each one fp32 fused multiply-add rounded to nearest (the
+// packed form of two fmaf, bit for bit).
+__device__ __forceinline__ void fma2(float &c0, float &c1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\tmov.b64 pc, {%0, %1};\n\t"
+      "fma.rn.f32x2 pc, pa, pb, pc;\n\tmov.b64 {%0, %1}, pc;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
 
 // The k-th largest key T of list keys[0..n) (n > k) and how many of the keys equal to T belong
 // to the best k (need_eq), by radix selection on 8-bit digits from the top; also whether every
-// key equal to T is kept (all_eq).  Called by the PF_EPI epilogue threads (t = their index).
-__device__ void kth_key(const uint32_t *keys, int n, int k, uint32_t *hist, uint32_t *sel, int t, uint32_t &T,
+// key equal to T is kept (all_eq).  Called by the PF_WG threads of warpgroup g (t = their index).
+__device__ void kth_key(const uint32_t *keys, int n, int k, uint32_t *hist, uint32_t *sel, int t, int g, uint32_t &T,
                         int &need_eq, bool &all_eq) {
   uint32_t prefix = 0;
   int need = k, bin_count = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    hist[t] = 0;  // PF_EPI == 256 bins
-    epi_sync();
+    hist[t] = 0;
+    hist[t + PF_WG] = 0;
+    wg_sync(g);
     const uint32_t himask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
-    for (int i = t; i < n; i += PF_EPI) {
-      const uint32_t key = keys[i];
-      if ((key & himask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    // scores crowd into few bins: lanes with the same bin add once (warp-aggregated)
+    const int lane = t & 31;
+    for (int i = t; i - lane < n; i += PF_WG) {
+      const uint32_t key = i < n ? keys[i] : 0u;
+      const bool act = i < n && (key & himask) == prefix;
+      const uint32_t am = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t bin = (key >> shift) & 255u, peers = __match_any_sync(am, bin);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], uint32_t(__popc(peers)));
+      }
     }
-    epi_sync();
+    wg_sync(g);
     if (t < 32) {  // one warp finds the digit at which the count from the top reaches `need`
       uint32_t c8[8], s = 0;
 #pragma unroll
@@ -125,34 +144,34 @@ __device__ void kth_key(const uint32_t *keys, int n, int k, uint32_t *hist, uint
         }
       }
     }
-    epi_sync();
+    wg_sync(g);
     prefix |= sel[0] << shift;
     need = int(sel[1]);
     bin_count = int(sel[2]);
-    epi_sync();  // sel and hist are rewritten by the next digit
+    wg_sync(g);  // sel and hist are rewritten by the next digit
   }
   T = prefix;
   need_eq = need;
   all_eq = bin_count == need;
 }
 
-// Cut a query's list (keys, ents, *cnt entries) back to its best k (key descending, entry
+// Cut a query's list (keys, ents; n > k entries) back to its best k (key descending, entry
 // ascending) through the scratch and return the k-th key, the list's new threshold.  Ties on
 // that key are resolved by counting, for each, the tied keys with smaller entries (only when
-// not all of them are kept).  Called by the PF_EPI epilogue threads; contains epi_sync().
-__device__ uint32_t cut_to_k(uint32_t *keys, int32_t *ents, int *cnt, int k, uint32_t *scr_key, int32_t *scr_ent,
-                             uint32_t *hist, uint32_t *sel, int t) {
-  const int n = *cnt;
+// not all of them are kept).  Called by the PF_WG threads of warpgroup g; contains wg_sync.
+__device__ uint32_t cut_to_k(uint32_t *keys, int32_t *ents, int n, int k, uint32_t *scr_key, int32_t *scr_ent,
+                             uint32_t *hist, uint32_t *sel, int t, int g) {
   uint32_t T;
   int need_eq;
   bool all_eq;
-  kth_key(keys, n, k, hist, sel, t, T, need_eq, all_eq);
+  kth_key(keys, n, k, hist, sel, t, g, T, need_eq, all_eq);
   if (t == 0) sel[3] = 0;
-  epi_sync();
-  for (int i = t; i < n; i += PF_EPI) {
-    const uint32_t key = keys[i];
-    bool keep = key > T;
-    if (key == T) {
+  wg_sync(g);
+  const int lane = t & 31;
+  for (int i = t; i - lane < n; i += PF_WG) {
+    const uint32_t key = i < n ? keys[i] : 0u;
+    bool keep = i < n && key > T;
+    if (i < n && key == T) {
       if (all_eq) {
         keep = true;
       } else {
@@ -162,19 +181,22 @@ __device__ uint32_t cut_to_k(uint32_t *keys, int32_t *ents, int *cnt, int k, uin
         keep = before < need_eq;
       }
     }
+    const uint32_t km = __ballot_sync(0xffffffffu, keep);
+    uint32_t base = 0;
+    if (lane == 0 && km) base = atomicAdd(&sel[3], uint32_t(__popc(km)));
+    base = __shfl_sync(0xffffffffu, base, 0);
     if (keep) {
-      const int s = int(atomicAdd(&sel[3], 1u));
+      const int s = int(base) + __popc(km & ((1u << lane) - 1u));
       scr_key[s] = key;
       scr_ent[s] = ents[i];
     }
   }
-  epi_sync();
-  for (int i = t; i < k; i += PF_EPI) {
+  wg_sync(g);
+  for (int i = t; i < k; i += PF_WG) {
     keys[i] = scr_key[i];
     ents[i] = scr_ent[i];
   }
-  if (t == 0) *cnt = k;
-  epi_sync();
+  wg_sync(g);
   return T;
 }
 }  // namespace
@@ -186,18 +208,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_index_kernel(const __gr
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + PS_BAR);
   uint64_t *empty = full + PF_STAGES;
   uint64_t *acc_full = empty + PF_STAGES;
-  uint64_t *acc_empty = acc_full + 2;
-  uint64_t *done = acc_empty + 2;
+  uint64_t *acc_empty = acc_full + PF_ACC;
+  uint64_t *done = acc_empty + PF_ACC;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + PS_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + PS_MISC + 4);
   float *ws = reinterpret_cast<float *>(smem + PS_W);
-  uint32_t *ckey = reinterpret_cast<uint32_t *>(smem + PS_CKEY);
-  int32_t *cent = reinterpret_cast<int32_t *>(smem + PS_CENT);
-  uint32_t *hist = reinterpret_cast<uint32_t *>(smem + PS_HIST);
-  uint32_t *sel = reinterpret_cast<uint32_t *>(smem + PS_SEL);
-  int *qcnt = reinterpret_cast<int *>(smem + PS_QS);
-  uint32_t *qthr = reinterpret_cast<uint32_t *>(smem + PS_QS + PF_Q * 4);
-  int *qvis = reinterpret_cast<int *>(smem + PS_QS + 2 * PF_Q * 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y, q0 = blockIdx.x * PF_Q;
@@ -224,9 +239,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_index_kernel(const __gr
       mbar_init(&full[s], a.use_tma ? 1 : 32);  // gather path: one cp.async arrival per producer lane
       mbar_init(&empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < PF_ACC; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
+      mbar_init(&acc_empty[i], PF_Q * 4);  // every epilogue warp
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -234,7 +249,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_index_kernel(const __gr
   } else if (warp >= 2) {
     // quantise the query heads (MXFP4, as the decode kernel): item (qi, h, pair of 32-blocks)
     const int t = threadIdx.x - 64;
-    for (int item = t; item < PF_Q * 128; item += PF_EPI) {
+    for (int item = t; item < PF_Q * 128; item += PF_Q * PF_WG) {
       const int qi = item >> 7, h = (item >> 1) & 63, g0 = 2 * (item & 1);
       uint8_t *brow = smem + PS_B + qi * 4096 + h * 64;
       uint32_t sfpart = 0;
@@ -276,11 +291,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_index_kernel(const __gr
         *reinterpret_cast<uint32_t *>(sfb + (rz & 31) * 16 + (rz >> 5) * 4) = 0u;
       }
     }
-    if (t < PF_Q) {
-      qcnt[t] = 0;
-      qthr[t] = KEY_NEG_INF;  // keep every finite score until the first cut
-      qvis[t] = nvis[t];
-    }
+    if (t < PF_Q * 3) reinterpret_cast<uint32_t *>(smem + PS_TCNT)[t] = 0;
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -348,9 +359,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_index_kernel(const __gr
       constexpr uint32_t id0 = idesc_mxf4(PF_TILE, PF_N, 0, 0);
       constexpr uint32_t id1 = idesc_mxf4(PF_TILE, PF_N, 2, 2);
       for (int i = 0; i < ntiles; ++i) {
-        const int s = i % PF_STAGES, buf = i & 1;
+        const int s = i % PF_STAGES, buf = i % PF_ACC;
         if (!mbar_wait_bounded(&full[s], (i / PF_STAGES) & 1, abort_flag, PF_WAIT_NS)) break;
-        if (!mbar_wait_bounded(&acc_empty[buf], ((i >> 1) & 1) ^ 1, abort_flag, PF_WAIT_NS)) break;
+        if (!mbar_wait_bounded(&acc_empty[buf], ((i / PF_ACC) & 1) ^ 1, abort_flag, PF_WAIT_NS)) break;
         if (!a.use_tma) fence_proxy_async_smem();  // cp.async-filled stages are read by the tensor core
         tc_fence_after();
         const uint32_t st = stages + s * PF_STAGE_BYTES;
@@ -375,105 +386,105 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_index_kernel(const __gr
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int t = threadIdx.x - 64;
-    const int q4 = warp & 3, wg = (warp - 2) >> 2;
+    // Warpgroup g scores query g of every tile and keeps its candidate list; the warpgroups
+    // never wait for one another.  Per tile the warps append with one shared-memory atomic on
+    // the tile's counter (counters rotate over three tiles, so one is zeroed while another is
+    // read and a third filled), then meet once; every thread adds the tile's count to its own
+    // copy of the list length, so cut decisions are uniform without a second barrier.
+    const int g = (warp - 2) >> 2, t = threadIdx.x - 64 - PF_WG * g;
+    const int q4 = warp & 3;
     const int e = pf_entry_of_row(32 * q4 + lane);  // tile entry of this thread's accumulator row
     const uint32_t lt_mask = (1u << lane) - 1u;
-    uint32_t *scr_key = reinterpret_cast<uint32_t *>(smem + PS_SCR);
-    int32_t *scr_ent = reinterpret_cast<int32_t *>(smem + PS_SCR + PF_KMAX * 4);
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem + PS_CKEY) + g * PF_CAP;
+    int32_t *ents = reinterpret_cast<int32_t *>(smem + PS_CENT) + g * PF_CAP;
+    uint32_t *scr_key = reinterpret_cast<uint32_t *>(smem + PS_SCR + g * PF_KMAX * 8);
+    int32_t *scr_ent = reinterpret_cast<int32_t *>(smem + PS_SCR + g * PF_KMAX * 8 + PF_KMAX * 4);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem + PS_HIST) + g * 256;
+    uint32_t *sel = reinterpret_cast<uint32_t *>(smem + PS_SEL) + g * 4;
+    uint32_t *tcnt = reinterpret_cast<uint32_t *>(smem + PS_TCNT) + g * 3;
+    const float4 *w4 = reinterpret_cast<const float4 *>(ws + g * 64);
+    int qv = 0;  // entries this query sees (0 past the chunk's end)
+#pragma unroll
+    for (int qi = 0; qi < PF_Q; ++qi)
+      if (qi == g) qv = nvis[qi];
+    int cnt = 0;                    // list length (the same in every thread of the warpgroup)
+    uint32_t thr = KEY_NEG_INF;     // keys must exceed this to enter the list
     bool ok = true;
-    const int rounds = (ntiles + 1) / 2;
-    for (int r = 0; r < rounds; ++r) {
-      const int i = 2 * r + wg;  // this warpgroup's tile of the round (accumulator set wg)
-      if (i < ntiles && ok) {
-        if (!mbar_wait_bounded(&acc_full[wg], (i >> 1) & 1, abort_flag, PF_WAIT_NS)) {
-          ok = false;
-        } else {
-          tc_fence_after();
-          float sc[PF_Q];
+    for (int i = 0; i < ntiles; ++i) {
+      const int buf = i % PF_ACC;
+      if (ok && !mbar_wait_bounded(&acc_full[buf], (i / PF_ACC) & 1, abort_flag, PF_WAIT_NS)) ok = false;
+      ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld is taken by the whole warp or not at all
+      float sc = 0.f;
+      if (ok) {
+        tc_fence_after();
+        const uint32_t taddr = tmem + (uint32_t(32 * q4) << 16) + (buf * PF_Q + g) * PF_N;
+        uint32_t r0[32], r1[32];
+        tc_ld_32x32b_x32(taddr, r0);
+        tc_ld_32x32b_x32(taddr + 32, r1);
+        tc_wait_ld();
+        tc_fence_before();
+        // heads h -> partial h % 8 in head order (the decode kernel's order, so the same score)
+        float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int qi = 0; qi < PF_Q; ++qi) {
-            const uint32_t taddr = tmem + (uint32_t(32 * q4) << 16) + (wg * PF_Q + qi) * PF_N;
-            uint32_t r0[32], r1[32];
-            tc_ld_32x32b_x32(taddr, r0);
-            tc_ld_32x32b_x32(taddr + 32, r1);
-            tc_wait_ld();
-            const float4 *w4 = reinterpret_cast<const float4 *>(ws + qi * 64);
-            float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int h4 = 0; h4 < 8; ++h4) {
+          const float4 wv = w4[h4];
+          const int j = (4 * h4) & 7;
+          fma2(part[j], part[j + 1], wv.x, wv.y, fmaxf(__uint_as_float(r0[4 * h4]), 0.f),
+               fmaxf(__uint_as_float(r0[4 * h4 + 1]), 0.f));
+          fma2(part[j + 2], part[j + 3], wv.z, wv.w, fmaxf(__uint_as_float(r0[4 * h4 + 2]), 0.f),
+               fmaxf(__uint_as_float(r0[4 * h4 + 3]), 0.f));
+        }
 #pragma unroll
-            for (int h4 = 0; h4 < 8; ++h4) {
-              const float4 wv = w4[h4];
-              part[(4 * h4) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(r0[4 * h4]), 0.f), part[(4 * h4) & 7]);
-              part[(4 * h4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(r0[4 * h4 + 1]), 0.f), part[(4 * h4 + 1) & 7]);
-              part[(4 * h4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(r0[4 * h4 + 2]), 0.f), part[(4 * h4 + 2) & 7]);
-              part[(4 * h4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(r0[4 * h4 + 3]), 0.f), part[(4 * h4 + 3) & 7]);
-            }
-#pragma unroll
-            for (int h4 = 0; h4 < 8; ++h4) {
-              const float4 wv = w4[8 + h4];
-              part[(4 * h4) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(r1[4 * h4]), 0.f), part[(4 * h4) & 7]);
-              part[(4 * h4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(r1[4 * h4 + 1]), 0.f), part[(4 * h4 + 1) & 7]);
-              part[(4 * h4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f), part[(4 * h4 + 2) & 7]);
-              part[(4 * h4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f), part[(4 * h4 + 3) & 7]);
-            }
-            sc[qi] = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[wg]);
-          // append the keys above each query's threshold (one atomic per warp and query); an
-          // entry without a valid page is never a candidate (its error is already reported)
-          const int n = i * PF_TILE + e;
-          const bool live = n < nvis_max && cache_slot(a.c, b, n) >= 0;
-#pragma unroll
-          for (int qi = 0; qi < PF_Q; ++qi) {
-            const uint32_t key = score_key(sc[qi]);
-            const bool pass = live && n < qvis[qi] && key > qthr[qi];
-            const uint32_t m = __ballot_sync(0xffffffffu, pass);
-            if (m) {
-              int base = 0;
-              if (lane == 0) base = atomicAdd(&qcnt[qi], __popc(m));
-              base = __shfl_sync(0xffffffffu, base, 0);
-              if (pass) {
-                const int at = base + __popc(m & lt_mask);
-                ckey[qi * PF_CAP + at] = key;
-                cent[qi * PF_CAP + at] = n;
-              }
-            }
-          }
+        for (int h4 = 0; h4 < 8; ++h4) {
+          const float4 wv = w4[8 + h4];
+          const int j = (4 * h4) & 7;
+          fma2(part[j], part[j + 1], wv.x, wv.y, fmaxf(__uint_as_float(r1[4 * h4]), 0.f),
+               fmaxf(__uint_as_float(r1[4 * h4 + 1]), 0.f));
+          fma2(part[j + 2], part[j + 3], wv.z, wv.w, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f),
+               fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f));
+        }
+        sc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      // append the keys above the threshold; an entry without a valid page is never a
+      // candidate (its error is already reported)
+      const int n = i * PF_TILE + e;
+      const uint32_t key = score_key(sc);
+      const bool pass = ok && n < qv && key > thr && cache_slot(a.c, b, n) >= 0;
+      const uint32_t m = __ballot_sync(0xffffffffu, pass);
+      if (m) {
+        uint32_t base = 0;
+        if (lane == 0) base = atomicAdd(&tcnt[i % 3], uint32_t(__popc(m)));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (pass) {
+          const int at = cnt + int(base) + __popc(m & lt_mask);
+          keys[at] = key;
+          ents[at] = n;
         }
       }
-      epi_sync();  // both tiles of the round are in the lists
-      int cnt[PF_Q];
-#pragma unroll
-      for (int qi = 0; qi < PF_Q; ++qi) cnt[qi] = qcnt[qi];
-      epi_sync();  // every thread holds the counts before the next round appends to them
-#pragma unroll 1
-      for (int qi = 0; qi < PF_Q; ++qi) {
-        if (cnt[qi] > PF_CAP - 2 * PF_TILE) {  // the next round could overflow: cut to the best k
-          const uint32_t T = cut_to_k(ckey + qi * PF_CAP, cent + qi * PF_CAP, &qcnt[qi], a.k, scr_key, scr_ent,
-                                      hist, sel, t);
-          if (t == 0) qthr[qi] = T;
-          epi_sync();
-        }
+      if (t == 0) tcnt[(i + 1) % 3] = 0;  // last read after tile i - 2's barrier, next filled after this one
+      wg_sync(g);
+      cnt += int(tcnt[i % 3]);
+      if (cnt > PF_CAP - PF_TILE) {  // the next tile could overflow: cut to the best k
+        thr = cut_to_k(keys, ents, cnt, a.k, scr_key, scr_ent, hist, sel, t, g);
+        cnt = a.k;
       }
     }
-    // final: each query's best k, in ascending entry order, -1 padded
-#pragma unroll 1
-    for (int qi = 0; qi < nq; ++qi) {
-      if (qcnt[qi] > a.k) {
-        cut_to_k(ckey + qi * PF_CAP, cent + qi * PF_CAP, &qcnt[qi], a.k, scr_key, scr_ent, hist, sel, t);
+    // final: the query's best k, in ascending entry order, -1 padded
+    if (g < nq) {
+      if (cnt > a.k) {
+        cut_to_k(keys, ents, cnt, a.k, scr_key, scr_ent, hist, sel, t, g);
+        cnt = a.k;
       }
-      const int m = qcnt[qi];
-      int32_t *orow = a.idx + (int64_t(b) * a.Q + q0 + qi) * a.k;
-      for (int j = t; j < m; j += PF_EPI) {
-        const int ej = cent[qi * PF_CAP + j];
+      int32_t *orow = a.idx + (int64_t(b) * a.Q + q0 + g) * a.k;
+      for (int j = t; j < cnt; j += PF_WG) {
+        const int ej = ents[j];
         int rank = 0;
-        for (int l = 0; l < m; ++l) rank += cent[qi * PF_CAP + l] < ej;
+        for (int l = 0; l < cnt; ++l) rank += ents[l] < ej;
         orow[rank] = ej;
       }
-      for (int j = m + t; j < a.k; j += PF_EPI) orow[j] = -1;
-      epi_sync();
+      for (int j = cnt + t; j < a.k; j += PF_WG) orow[j] = -1;
     }
   }
 

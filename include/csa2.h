@@ -119,8 +119,8 @@ csa2_status csa2_check(const int32_t *err, csa2_stream_t stream);
  * Bytes of workspace csa2_sparse_attn needs for these sizes (0 for Reuse, and for
  * Dense up to 4096 entries).  max_entries bounds num_entries[b]; pool_k is the
  * candidate-pool size (0 if none).  Full mode with B * Q >= 1024 query rows and no
- * pool (a prefill chunk) selects without materialising scores and needs only the
- * B * Q * k selection.
+ * pool (a prefill chunk), and Reindex over a pool of at most 16384 candidates, select
+ * without materialising scores and need only the B * Q * k selection.
  */
 size_t csa2_workspace_size(csa2_mode mode, int32_t B, int32_t Q, int32_t max_entries,
                            int32_t k, int32_t pool_k);
@@ -239,7 +239,10 @@ csa2_status csa2_index_topk(const uint16_t *q_ix, const uint16_t *w, int32_t B, 
  *            query tokens per key tile and keeps each one's running top-k on chip
  *            ("DeepSeek V4.1 Flash 深度解析", 序: prefill compute is the bottleneck);
  *            the selection is the same as scoring and csa2_topk would give.
- *   REINDEX: q_ix, w score the entries listed in pool_io [B][Q][pool_k]; top-k of them.
+ *   REINDEX: q_ix, w score the entries listed in pool_io [B][Q][pool_k]; top-k of them
+ *            (ties: the earlier candidate).  Pools of at most 16384: one launch per row
+ *            group, each row's scores gathered in one CTA's shared memory and selected
+ *            there (the same selection as scoring and csa2_topk with the pool as map).
  *   REUSE:   idx_in [B][Q][k] given entry indices (-1 = none; order free).
  *   DENSE:   every visible entry (q_ix, w, k, pool and indices unused); the caches of
  *            the predecessor's 128-fold compressed layers are read this way.  Any
@@ -378,7 +381,8 @@ typedef struct {
   float *o, *lse;
 } csa2_decode_args;
 
-/* Workspace bytes csa2_decode_step needs (the largest layer's fp32 scores). */
+/* Workspace bytes csa2_decode_step needs: the largest Full layer's fp32 scores (and a
+ * Reindex layer's, for pools above 16384); 0 when no layer needs any (ws may be NULL). */
 size_t csa2_decode_workspace_size(const csa2_decode_args *args);
 csa2_status csa2_decode_step(const csa2_decode_args *args, void *ws, size_t ws_bytes, int32_t *err,
                              csa2_stream_t stream);

@@ -53,7 +53,9 @@ def test_workspace_size(lib):
     assert ws(2, 32, 1, 65536, 512, 0) == 0                           # Reuse needs none
     full = ws(0, 8, 1, 1 << 20, 512, 16384)
     assert full >= 8 * (1 << 20) * 4 + 8 * 512 * 4
-    assert ws(1, 8, 1, 1 << 20, 512, 16384) >= 8 * 16384 * 4
+    assert ws(1, 8, 1, 1 << 20, 512, 16384) == 8 * 512 * 4               # Reindex of a 16384 pool: selection only
+    assert ws(1, 8, 1, 1 << 20, 512, 16385) >= 8 * 16385 * 4 + 8 * 512 * 4   # larger pools: scores too
+    assert ws(0, 1024, 1, 1 << 17, 512, 0) == 1024 * 512 * 4             # prefill chunk: selection only
 
 
 def test_host_side_argument_checks(lib):

@@ -708,6 +708,46 @@ def test_prefill_fused_ties_and_short_rows():
             assert got[:nvis].tolist() == want and (got[nvis:] == -1).all()
 
 
+# ------------------------------------------------------------------ fused Reindex selection
+@pytest.mark.parametrize("B,P,tokens", [(8, 16384, 2 * 20000), (3, 5000, 2 * 9000), (4, 3000, 2 * 4000),
+                                        (300, 700, 2 * 1500), (2, 400, 2 * 1000)])
+def test_reindex_fused_selection(B, P, tokens):
+    """Reindex over a pool of at most 16384 candidates scores and selects in one launch (each
+    row's keys in one CTA's shared memory).  Its choice must equal the unfused path's bit for
+    bit: csa2_index_score over the pool, csa2_topk of those scores, mapped through the pool.
+    Pools are ascending with -1 pads and entries the query cannot see; some rows score every
+    candidate 0 (all tied: the earliest candidates win); P = 400 < k pads the selection; B = 300
+    rows run one CTA per row."""
+    k = K()
+    spec = W.scaled(W.tiny_full(), [tokens] * B, B=B)
+    cache = gpu_cache(spec)
+    q, q_ix, w, q_pos = W.query_tensors(spec, 0, DEV)
+    q_ix = q_ix.clone()
+    q_ix[0] = 0.0                                   # every score of row 0 ties
+    n = spec.entries(0)
+    g = torch.Generator(device="cpu").manual_seed(1234 + P)
+    pool = torch.full((B, 1, P), -1, dtype=torch.int32)
+    for b in range(B):
+        m = P - (b % 3) * 7                          # a few -1 pads at the end of some rows
+        pool[b, 0, :m] = torch.randperm(n, generator=g)[:m].sort().values.to(torch.int32)
+    pool = pool.to(DEV)
+    q_pos = q_pos.clone()
+    q_pos[1, 0] = tokens - 700                      # an earlier query: candidates it cannot see
+    err = _err()
+    assert k.csa2_workspace_size("reindex", B, 1, spec.max_entries, spec.k, P) == (B * spec.k * 4 + 255) // 256 * 256
+    idx = torch.empty((B, 1, spec.k), dtype=torch.int32, device=DEV)
+    k.csa2_sparse_attn("reindex", q, q_pos, cache, spec.tau, spec.max_entries, q_ix=q_ix, w=w, pool_k=P,
+                       pool_io=pool, idx_out=idx, err=err)
+    scores = k.csa2_index_score(q_ix, w, q_pos, cache, spec.max_entries, cand=pool, err=err)
+    pos = k.csa2_topk(scores, spec.k)[0]
+    ref = torch.where(pos >= 0, pool.gather(-1, pos.clamp(min=0).long()), torch.full_like(pos, -1))
+    assert k.csa2_check(err) == 0
+    assert torch.equal(idx, ref), f"{int((idx != ref).any(-1).sum())} of {B} rows differ"
+    assert torch.equal(idx[0, 0, :min(P, spec.k)], pool[0, 0, :min(P, spec.k)])   # all tied: earliest win
+    if P < spec.k:
+        assert (idx[:, :, P:] == -1).all()
+
+
 # ------------------------------------------------------------------ gated compressor and decode-time append
 @pytest.mark.parametrize("ratio", [1, 2, 4, 128])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
