@@ -47,17 +47,15 @@ constexpr int AM_THREADS = AM_PRODUCERS + 32;   // warp 8 drives the tensor core
 constexpr int AM_HG = 32;          // heads per CTA = MMA N
 constexpr int AM_TILE = 128;       // keys per S^T tile
 constexpr int AM_MAXKEYS = 640;    // 512 listed entries + 128 window tokens
-constexpr int AM_STAGES = 4;
-constexpr int AM_STAGE = 16384;
-constexpr int AM_RAW = 528;        // raw bytes per key in shared memory (512 + 16: conflict-free rows)
+constexpr int AM_BLOCKS = 8;       // 64-dim blocks of a key tile = operand buffers (one tile)
+constexpr int AM_STAGE = 16384;    // one block: 128 keys x 64 dims fp16
 constexpr uint32_t AM_TMEM_COLS = 256;
 constexpr uint64_t AM_WAIT_NS = 2000000000ull;
 
 constexpr int SM_Q = 0;                              // 8 chunks x [32 heads x 128 B]
 constexpr int SM_P = SM_Q + 8 * 4096;                // P^T [640 keys x 64 B]
-constexpr int SM_STG = SM_P + AM_MAXKEYS * 64;       // 4 x 16 KB operand ring
-constexpr int SM_RAW = SM_STG + AM_STAGES * AM_STAGE;   // one tile of raw keys
-constexpr int SM_SLOT = SM_RAW + AM_TILE * AM_RAW;
+constexpr int SM_STG = SM_P + AM_MAXKEYS * 64;       // one key tile: 8 x 16 KB blocks
+constexpr int SM_SLOT = SM_STG + AM_BLOCKS * AM_STAGE;
 constexpr int SM_MU = SM_SLOT + AM_MAXKEYS * 8;      // logit multiplier per key
 constexpr int SM_PV = SM_MU + AM_MAXKEYS * 4;        // P multiplier per key
 constexpr int AM_MAXCS = 16;      // largest cluster splitting one row's keys
@@ -67,7 +65,7 @@ constexpr int SM_HM = SM_RED + (AM_MAXCS + 1) * 32 * 4;   // head max [32], head
 constexpr int SM_QS = SM_HM + 2 * 32 * 4;            // query prescale: [8 warps][AM_QU] max bits, [32] 2^-s
 constexpr int SM_NEW = SM_QS + (8 * AM_QU + 32) * 4; // this step's window token: 512 codes, scale, [4] maxima
 constexpr int SM_BAR = SM_NEW + 512 + 32;
-constexpr int SM_MISC = SM_BAR + 8 * (2 * AM_STAGES + 1);
+constexpr int SM_MISC = SM_BAR + 8 * (2 * AM_BLOCKS + 1);
 constexpr int SM_TOTAL = SM_MISC + 16;
 constexpr size_t AM_SMEM = SM_TOTAL + 1024;
 }  // namespace
@@ -155,32 +153,60 @@ __device__ __forceinline__ void store_query_fp16(const uint4 (&qraw)[AM_QU], con
   if (tid < 32) qinv[tid] = pow2f(-query_prescale_exp(head_max_bits(qmx, tid)));
 }
 
-// Gather the raw bytes of local key tile t into shared memory (asynchronous 16-byte
-// copies by the producer threads, committed as one group): a listed entry's 256 code bytes and 32 scale bytes
-// at offsets 0 and 256 of its row, a window token's 512 codes at offset 0.  With new_codes, the
-// row's last key (this step's own window token, nk - 1) is copied from there instead.
-__device__ __forceinline__ void gather_tile(const AttnArgs &p, const int64_t *slot, int nks, int nk, int key0, int t,
-                                            uint8_t *raw, const uint8_t *new_codes) {
-  const uint32_t raw_s = smem_u32(raw);
-  for (int i = threadIdx.x; i < AM_TILE * 32; i += AM_PRODUCERS) {
-    const int kt = i & (AM_TILE - 1), piece = i >> 7;  // consecutive threads: consecutive keys
-    const int key = t * AM_TILE + kt;
-    const int64_t s = slot[key];
-    if (s < 0) continue;
-    const uint32_t dst = raw_s + kt * AM_RAW + piece * 16;
-    if (key0 + key < nks) {
-      if (piece < 16)
-        cp_async_16(dst, p.c.kv_codes + s * CSA2_MAIN_CODE_BYTES + piece * 16);
-      else if (piece < 18)
-        cp_async_16(dst, p.c.kv_scales + s * CSA2_MAIN_SCALE_BYTES + (piece - 16) * 16);
-    } else if (new_codes && key0 + key == nk - 1) {
-      *reinterpret_cast<uint4 *>(raw + kt * AM_RAW + piece * 16) =
-          *reinterpret_cast<const uint4 *>(new_codes + piece * 16);
-    } else {
-      cp_async_16(dst, p.codes + s * CSA2_SWA_DIM + piece * 16);
-    }
+// Raw bytes of one half of a key (dims 256 half .. +255) into registers: a listed entry's
+// 128 code bytes (rr[0..7]) and 16 scale bytes (rr[8]) from slot s of the cache, a window
+// token's 256 code bytes (rr[0..15]) from slot s of the ring, or from own_codes (this step's
+// token, quantised in the launch).  Nothing for a masked key (s < 0).
+// Pieces [I0, I1) only (of 9 for a listed entry, 16 for a window token), so that a caller can
+// load the first 9 of the next key ahead and the rest of a window token later.
+template <int I0 = 0, int I1 = 16, int N>
+__device__ __forceinline__ void load_key_half(const AttnArgs &p, int64_t s, bool sparse, const uint8_t *own_codes,
+                                              int half, uint4 (&rr)[N]) {
+  static_assert(I1 <= N, "register set too small");
+  if (s < 0) return;
+  if (sparse) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.c.kv_codes + s * CSA2_MAIN_CODE_BYTES + half * 128);
+#pragma unroll
+    for (int i = I0; i < (I1 < 8 ? I1 : 8); ++i) rr[i] = src[i];
+    if (I0 <= 8 && I1 > 8) rr[8] = *reinterpret_cast<const uint4 *>(p.c.kv_scales + s * CSA2_MAIN_SCALE_BYTES + half * 16);
+  } else {
+    const uint4 *src = reinterpret_cast<const uint4 *>((own_codes ? own_codes : p.codes + s * CSA2_SWA_DIM) + half * 256);
+#pragma unroll
+    for (int i = I0; i < I1; ++i) rr[i] = src[i];
   }
-  cp_async_commit();
+}
+
+// Block c (dims 256 half + 64 c .. +63) of a key half held in registers, dequantised to fp16
+// (exact) into row key_in of a K-major 128-byte-swizzled 128-key block; zeros for a masked key.
+__device__ __forceinline__ void dequant_block(const uint4 (&rr)[16], bool sparse, bool valid, int c, int key_in,
+                                              uint8_t *dst) {
+#pragma unroll
+  for (int q2 = 0; q2 < 2; ++q2) {  // 32 dims at a time
+    uint32_t h16[16];
+    if (!valid) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) h16[i] = 0u;
+    } else if (sparse) {
+      const uint4 a = rr[2 * c + q2];
+      const uint32_t sw = (&rr[8].x)[c];  // scale bytes of dims 64c .. 64c+63 of this half
+      const uint32_t sc = (sw >> (16 * q2)) & 0xFFFF;
+      const uint32_t s0 = cvt_e4m3x2_f16x2((sc & 0xFF) * 0x101u);
+      const uint32_t s1 = cvt_e4m3x2_f16x2(((sc >> 8) & 0xFF) * 0x101u);
+      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        h16[i] = hmul2_u32(cvt_e2m1x2_f16x2((w[i >> 2] >> (8 * (i & 3))) & 0xFF), i < 8 ? s0 : s1);
+    } else {
+      const uint4 a = rr[4 * c + 2 * q2], bb = rr[4 * c + 2 * q2 + 1];
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) h16[i] = cvt_e4m3x2_f16x2((w[i >> 1] >> (16 * (i & 1))) & 0xFFFF);
+    }
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      *reinterpret_cast<uint4 *>(dst + kmaj128(key_in, 4 * q2 + v)) =
+          make_uint4(h16[4 * v], h16[4 * v + 1], h16[4 * v + 2], h16[4 * v + 3]);
+  }
 }
 
 // This step's own window token of the CTA's query row, quantised exactly as pack_swa_kernel does
@@ -218,33 +244,6 @@ __device__ __forceinline__ void quantise_new_token(const AttnArgs &p, int row, i
     if (tid == 0) *new_scale = s;
   }
   __syncthreads();
-}
-
-// 32 fp16 values (4 x 16 bytes) of dims dim0 .. dim0+31 of one key from its raw row;
-// zeros for a masked key.
-__device__ __forceinline__ void dequant32(const uint8_t *rk, bool sparse, bool valid, int dim0, uint4 (&out)[4]) {
-  if (!valid) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) out[i] = make_uint4(0, 0, 0, 0);
-    return;
-  }
-  uint32_t h[16];
-  if (sparse) {
-    const uint4 a = *reinterpret_cast<const uint4 *>(rk + dim0 / 2);
-    const uint32_t sc = *reinterpret_cast<const uint16_t *>(rk + 256 + dim0 / 16);
-    const uint32_t s0 = cvt_e4m3x2_f16x2((sc & 0xFF) * 0x101u);
-    const uint32_t s1 = cvt_e4m3x2_f16x2(((sc >> 8) & 0xFF) * 0x101u);
-    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-    for (int i = 0; i < 16; ++i) h[i] = hmul2_u32(cvt_e2m1x2_f16x2((w[i >> 2] >> (8 * (i & 3))) & 0xFF), i < 8 ? s0 : s1);
-  } else {
-    const uint4 a = *reinterpret_cast<const uint4 *>(rk + dim0), b = *reinterpret_cast<const uint4 *>(rk + dim0 + 16);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 16; ++i) h[i] = cvt_e4m3x2_f16x2((w[i >> 1] >> (16 * (i & 1))) & 0xFFFF);
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) out[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
 }
 
 // Max or sum over the 32 lanes of each of 32 per-lane values: afterwards lane l
@@ -365,9 +364,9 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   float *red = reinterpret_cast<float *>(smem + SM_RED);
   float *hmax = reinterpret_cast<float *>(smem + SM_HM);
   float *hsum = hmax + 32;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM_BAR);  // operand buffer written (256 arrivals)
-  uint64_t *mma_done = full + AM_STAGES;                          // operand buffer consumed (tcgen05.commit)
-  uint64_t *phase_done = mma_done + AM_STAGES;                    // all products of a phase complete
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM_BAR);  // block written (128 arrivals)
+  uint64_t *mma_done = full + AM_BLOCKS;                          // block consumed (tcgen05.commit)
+  uint64_t *phase_done = mma_done + AM_BLOCKS;                    // all products of a phase complete
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM_MISC + 4);
 
@@ -443,8 +442,8 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     tmem_relinquish();
   }
   if (issuer) {
-    for (int i = 0; i < AM_STAGES; ++i) {
-      mbar_init(&full[i], AM_PRODUCERS);
+    for (int i = 0; i < AM_BLOCKS; ++i) {
+      mbar_init(&full[i], AM_TILE);
       mbar_init(&mma_done[i], 1);
     }
     mbar_init(phase_done, 1);
@@ -452,11 +451,16 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     mbar_init_fence();
   }
   __syncthreads();  // key list, query maxima and barriers ready
-  uint8_t *raw = smem + SM_RAW;
-  if (producer) {
-    if (ntiles > 0) gather_tile(p, slot, nks, nk, key0, 0, raw, new_codes);
-    store_query_fp16(qraw, qmx, qinv, smem + SM_Q);
-  }
+  // Producer (key_in, half) owns dims 256 half .. +255 of key key_in of every tile: blocks
+  // 4 half .. 4 half + 3, dequantised from the key half's raw bytes loaded into registers.
+  const int key_in = tid & (AM_TILE - 1), half = (tid >> 7) & 1;
+  uint4 cur[16];
+  auto load_tile = [&](int t) {
+    const int jl = t * AM_TILE + key_in;
+    const bool own = own_token && key0 + jl == nk - 1;
+    load_key_half(p, slot[jl], key0 + jl < nks, own ? new_codes : nullptr, half, cur);
+  };
+  if (producer) store_query_fp16(qraw, qmx, qinv, smem + SM_Q);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -464,72 +468,50 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   const uint32_t tmem = *tmem_slot;
   const uint32_t stg = smem_u32(smem + SM_STG);
   bool aborted = false;
-  // Barrier over the producer threads that also ORs their abort state, so that every
-  // producer takes the same branch after it (none may skip a later barrier).
-  auto producers_sync = [&](bool mine) -> bool {
-    uint32_t any;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, 2, %2, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(any)
-        : "r"(uint32_t(mine || *abort_flag)), "n"(AM_PRODUCERS)
-        : "memory");
-    return any != 0;
+  // Write tile t's four blocks of this producer (use u of the block buffers): wait until the
+  // tensor core has consumed use u - 1, dequantise, publish.
+  auto produce_tile = [&](int t, const uint4 (&rr)[16], int u) -> bool {
+    const int jl = t * AM_TILE + key_in;
+    const bool sparse = key0 + jl < nks, valid = slot[jl] >= 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int blk = 4 * half + c;
+      if (u > 0 && !mbar_wait_bounded(&mma_done[blk], (u - 1) & 1, abort_flag, AM_WAIT_NS)) return false;
+      dequant_block(rr, sparse, valid, c, key_in, smem + SM_STG + blk * AM_STAGE);
+      fence_proxy_async_smem();
+      mbar_arrive(&full[blk]);
+    }
+    return true;
   };
-  // Producer side of one operand buffer: wait until the tensor core has consumed what
-  // the buffer held AM_STAGES chunks ago, write it, publish it.  n = chunk number.
-  auto produce = [&](int n, auto &&write) -> bool {
-    const int buf = n % AM_STAGES;
-    if (n >= AM_STAGES && !mbar_wait_bounded(&mma_done[buf], ((n / AM_STAGES) - 1) & 1, abort_flag, AM_WAIT_NS))
-      return false;
-    write(smem + SM_STG + buf * AM_STAGE);
-    fence_proxy_async_smem();
-    mbar_arrive(&full[buf]);
+  // Every tile in turn (uses u0 + t).
+  auto produce_all = [&](int u0) -> bool {
+    for (int t = 0; t < ntiles; ++t) {
+      load_tile(t);
+      if (!produce_tile(t, cur, u0 + t)) return false;
+    }
     return true;
   };
 
   // ---------------------------------------------------------------- phase 1: S^T = K Q^T
-  // Producers: per tile, its raw keys in shared memory, then 8 chunks of 64 dims (one key
-  // per thread pair; consecutive threads take consecutive keys, so raw rows are read
-  // conflict-free).  Issuer: one 4-step MMA group per chunk as soon as it is published.
-  const int nch1 = ntiles * 8;
+  // Issuer: per tile, one 4-step MMA group per block as soon as it is published (the two
+  // halves' blocks in the order they are written).
   if (producer) {
-    const int key_in = tid & (AM_TILE - 1), half = tid >> 7;
-    for (int t = 0; t < ntiles; ++t) {
-      if (t > 0) {
-        aborted = producers_sync(aborted);  // every producer is past its reads of the previous raw tile
-        if (aborted) break;
-        gather_tile(p, slot, nks, nk, key0, t, raw, new_codes);
-      }
-      cp_async_wait<0>();
-      aborted = producers_sync(aborted);
-      if (aborted) break;
-      const int key = t * AM_TILE + key_in;
-      const bool sparse = key0 + key < nks, valid = slot[key] >= 0;
-      const uint8_t *rk = smem + SM_RAW + key_in * AM_RAW;
-      for (int c = 0; c < 8 && !aborted; ++c) {
-        aborted = !produce(t * 8 + c, [&](uint8_t *dst) {
-          uint4 out[4];
-          dequant32(rk, sparse, valid, 64 * c + 32 * half, out);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) *reinterpret_cast<uint4 *>(dst + kmaj128(key_in, 4 * half + v)) = out[v];
-        });
-      }
-    }
+    aborted = !produce_all(0);
   } else if (issuer) {
     constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, false, false);
-    for (int n = 0; n < nch1; ++n) {
-      const int buf = n % AM_STAGES, t = n >> 3, c = n & 7;
-      if (!mbar_wait_bounded(&full[buf], (n / AM_STAGES) & 1, abort_flag, AM_WAIT_NS)) break;
-      tc_fence_after();
-      const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_Q + c * 4096);
+    bool ok = true;
+    for (int t = 0; t < ntiles && ok; ++t) {
+      for (int i = 0; i < AM_BLOCKS; ++i) {
+        const int blk = (i & 1) * 4 + (i >> 1);
+        if (!(ok = mbar_wait_bounded(&full[blk], t & 1, abort_flag, AM_WAIT_NS))) break;
+        tc_fence_after();
+        const uint32_t a0 = stg + blk * AM_STAGE, b0 = smem_u32(smem + SM_Q + blk * 4096);
 #pragma unroll
-      for (int s = 0; s < 4; ++s)
-        tc_mma_f16(tmem + t * AM_HG, smem_desc(a0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B),
-                   smem_desc(b0 + 32 * s, 16, 1024, LAYOUT_SWIZZLE_128B), id, c > 0 || s > 0);
-      tc_commit(&mma_done[buf]);
+        for (int k4 = 0; k4 < 4; ++k4)
+          tc_mma_f16(tmem + t * AM_HG, smem_desc(a0 + 32 * k4, 16, 1024, LAYOUT_SWIZZLE_128B),
+                     smem_desc(b0 + 32 * k4, 16, 1024, LAYOUT_SWIZZLE_128B), id, i > 0 || k4 > 0);
+        tc_commit(&mma_done[blk]);
+      }
     }
     tc_commit(phase_done);
   }
@@ -565,12 +547,10 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     if (warp == 0)  // the maxima of the prescaled logits, scaled back by 2^-s (exact)
       hmax[lane] = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane])) * qinv[lane];
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    float m_h[32], sm[32];
+    float sm[32];  // the head maxima are read from shared memory (a broadcast) as needed
 #pragma unroll
-    for (int h = 0; h < 32; ++h) {
-      m_h[h] = hmax[h];
-      sm[h] = 0.f;
-    }
+    for (int h = 0; h < 32; ++h) sm[h] = 0.f;
+    const float *m_h = hmax;
     for (int t = 0; t < ntiles; ++t) {
       const int key = t * AM_TILE + 32 * warp + lane;
       uint32_t r0[16], r1[16];
@@ -607,46 +587,36 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   tc_fence_after();
 
   // ---------------------------------------------------------------- phase 3: O^T = V^T P^T
-  // Producers: per 64-key chunk, 4 chunks of 128 dims (a CTA with one tile still holds
-  // its raw keys).  Issuer: O^T accumulates over the key chunks.
-  const int nkc = (ntiles * AM_TILE) / 64;  // 64-key chunks (masked keys carry P = 0, V = 0)
+  // The same blocks serve as the MN-major V^T operand (two blocks = 128 dims, 16 KB apart).
+  // A CTA with one tile still holds it from phase 1; otherwise every tile is dequantised again
+  // (uses ntiles + t).  Issuer: O^T accumulates over the tiles' 64-key halves.
+  const int nkc = ntiles * 2;  // 64-key chunks (masked keys carry P = 0, V = 0)
   if (!aborted && producer) {
-    const int key_in = tid & 63, qd = tid >> 6;  // 4 threads per key, 32 dims each
-    for (int jc = 0; jc < nkc; ++jc) {
-      const int t = jc >> 1;
-      if (ntiles > 1 && (jc & 1) == 0) {
-        aborted = producers_sync(aborted);  // every producer is past its reads of the raw tile
-        if (aborted) break;
-        gather_tile(p, slot, nks, nk, key0, t, raw, new_codes);
-        cp_async_wait<0>();
-        aborted = producers_sync(aborted);
-        if (aborted) break;
-      }
-      const int key = jc * 64 + key_in;
-      const bool sparse = key0 + key < nks, valid = slot[key] >= 0;
-      const uint8_t *rk = smem + SM_RAW + (key - t * AM_TILE) * AM_RAW;
-      for (int d = 0; d < 4 && !aborted; ++d) {
-        aborted = !produce(nch1 + jc * 4 + d, [&](uint8_t *dst) {
-          uint4 out[4];
-          dequant32(rk, sparse, valid, 128 * d + 32 * qd, out);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            *reinterpret_cast<uint4 *>(dst + mnmaj128(key_in, qd >> 1, 4 * (qd & 1) + v)) = out[v];
-        });
-      }
-    }
+    if (ntiles > 1) aborted = !produce_all(ntiles);
   } else if (!aborted && issuer) {
     constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, true, true);
-    for (int i = 0; i < nkc * 4; ++i) {
-      const int n = nch1 + i, buf = n % AM_STAGES, jc = i >> 2, d = i & 3;
-      if (!mbar_wait_bounded(&full[buf], (n / AM_STAGES) & 1, abort_flag, AM_WAIT_NS)) break;
-      tc_fence_after();
-      const uint32_t a0 = stg + buf * AM_STAGE, b0 = smem_u32(smem + SM_P);
+    const uint32_t pt = smem_u32(smem + SM_P);
+    bool ok = true;
+    for (int t = 0; t < ntiles && ok; ++t) {
+      const int u = ntiles + t;
+      for (int dd = 0; dd < 4; ++dd) {
+        const int d = (dd & 1) * 2 + (dd >> 1);  // blocks (0,1), (4,5), (2,3), (6,7): the order they are written
+        if (ntiles > 1) {
+          if (!(ok = mbar_wait_bounded(&full[2 * d], u & 1, abort_flag, AM_WAIT_NS))) break;
+          if (!(ok = mbar_wait_bounded(&full[2 * d + 1], u & 1, abort_flag, AM_WAIT_NS))) break;
+        }
+        tc_fence_after();
 #pragma unroll
-      for (int s = 0; s < 4; ++s)
-        tc_mma_f16(tmem + d * AM_HG, smem_desc(a0 + 2048 * s, 8192, 1024, LAYOUT_SWIZZLE_128B),
-                   smem_desc(b0 + (8 * jc + 2 * s) * 512, 16, 512, LAYOUT_SWIZZLE_64B), id, jc > 0 || s > 0);
-      tc_commit(&mma_done[buf]);
+        for (int jc = 0; jc < 2; ++jc)
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4)
+            tc_mma_f16(tmem + d * AM_HG,
+                       smem_desc(stg + (2 * d) * AM_STAGE + jc * 8192 + 2048 * k4, 16384, 1024, LAYOUT_SWIZZLE_128B),
+                       smem_desc(pt + (8 * (2 * t + jc) + 2 * k4) * 512, 16, 512, LAYOUT_SWIZZLE_64B), id,
+                       t > 0 || jc > 0 || k4 > 0);
+        tc_commit(&mma_done[2 * d]);
+        tc_commit(&mma_done[2 * d + 1]);
+      }
     }
   }
   if (issuer) tc_commit(phase_done);
@@ -794,20 +764,13 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
         }
       }
       m = p.tau, pm = 1.f;
-      if (s >= 0) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.c.kv_codes + s * CSA2_MAIN_CODE_BYTES + half * 128);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) rr[i] = src[i];
-        rr[8] = *reinterpret_cast<const uint4 *>(p.c.kv_scales + s * CSA2_MAIN_SCALE_BYTES + half * 16);
-      }
+      load_key_half(p, s, true, nullptr, half, rr);
     } else if (j < nk) {
       s = int64_t(ring) * p.R + (lo + (j - nks)) % p.R;
       const bool own = own_token && j == nk - 1;
       const float sc = own ? *new_scale : p.scale[s];
       m = p.tau * sc, pm = sc;
-      const uint4 *src = reinterpret_cast<const uint4 *>((own ? new_codes : p.codes + s * CSA2_SWA_DIM) + half * 256);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) rr[i] = src[i];
+      load_key_half(p, s, false, own ? new_codes : nullptr, half, rr);
     }
     if (half == 0) {
       slot[key_in] = s;
@@ -843,34 +806,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int blk = 4 * half + c;
-      uint8_t *dst = smem + T_KT + blk * 16384;
-#pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {  // 32 dims at a time
-        uint32_t h16[16];
-        if (!valid) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) h16[i] = 0u;
-        } else if (sparse) {
-          const uint4 a = rr[2 * c + q2];
-          const uint32_t sw = (&rr[8].x)[c];  // scale bytes of dims 64c .. 64c+63 of this half
-          const uint32_t sc = (sw >> (16 * q2)) & 0xFFFF;
-          const uint32_t s0 = cvt_e4m3x2_f16x2((sc & 0xFF) * 0x101u);
-          const uint32_t s1 = cvt_e4m3x2_f16x2(((sc >> 8) & 0xFF) * 0x101u);
-          const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            h16[i] = hmul2_u32(cvt_e2m1x2_f16x2((w[i >> 2] >> (8 * (i & 3))) & 0xFF), i < 8 ? s0 : s1);
-        } else {
-          const uint4 a = rr[4 * c + 2 * q2], bb = rr[4 * c + 2 * q2 + 1];
-          const uint32_t w[8] = {a.x, a.y, a.z, a.w, bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-          for (int i = 0; i < 16; ++i) h16[i] = cvt_e4m3x2_f16x2((w[i >> 1] >> (16 * (i & 1))) & 0xFFFF);
-        }
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          *reinterpret_cast<uint4 *>(dst + kmaj128(key_in, 4 * q2 + v)) =
-              make_uint4(h16[4 * v], h16[4 * v + 1], h16[4 * v + 2], h16[4 * v + 3]);
-      }
+      dequant_block(rr, sparse, valid, c, key_in, smem + T_KT + blk * 16384);
       fence_proxy_async_smem();
       mbar_arrive(&full[blk]);
     }
