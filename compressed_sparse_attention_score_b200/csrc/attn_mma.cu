@@ -412,29 +412,48 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   uint8_t *new_codes = own_token ? smem + SM_NEW : nullptr;
   float *new_scale = reinterpret_cast<float *>(smem + SM_NEW + 512);
   if (own_token) quantise_new_token(p, row, ring, pos, split == 0 && hg == 0, smem + SM_NEW, new_scale, new_scale + 4);
-  for (int jl = tid; jl < ntiles * AM_TILE; jl += AM_THREADS) {
-    const int j = key0 + jl;
-    int64_t s = -1;
-    float m = 0.f, pm = 0.f;
-    if (j < nks) {
-      const int n = p.dense ? p.e0 + j : p.idx[int64_t(lrow) * p.k + j];
-      if (n != -1) {
-        if (n < -1 || n >= nvis) {
-          report(p.err, CSA2_ERR_INDEX);
-        } else {
-          s = cache_slot(p.c, b, n);
-          if (s < 0) report(p.err, CSA2_ERR_INDEX);
-        }
-      }
-      m = p.tau, pm = 1.f;
-    } else if (j < nk) {
-      s = int64_t(ring) * p.R + (lo + (j - nks)) % p.R;
-      const float sc = (own_token && j == nk - 1) ? *new_scale : p.scale[s];
-      m = p.tau * sc, pm = sc;
+  // The list's index loads go out together (at most three keys per thread), then the slots,
+  // then the window tokens' scales.
+  constexpr int KPT = (AM_MAXKEYS + AM_THREADS - 1) / AM_THREADS;
+  {
+    int nidx[KPT];
+#pragma unroll
+    for (int r = 0; r < KPT; ++r) {
+      const int jl = tid + r * AM_THREADS, j = key0 + jl;
+      nidx[r] = (jl < ntiles * AM_TILE && j < nks) ? (p.dense ? p.e0 + j : p.idx[int64_t(lrow) * p.k + j]) : -1;
     }
-    slot[jl] = s;
-    mu[jl] = m;
-    pv[jl] = pm;
+    int64_t sl[KPT];
+    float sc[KPT];
+#pragma unroll
+    for (int r = 0; r < KPT; ++r) {
+      const int jl = tid + r * AM_THREADS, j = key0 + jl;
+      sl[r] = -1;
+      sc[r] = 1.f;
+      if (jl >= ntiles * AM_TILE) continue;
+      if (j < nks) {
+        const int n = nidx[r];
+        if (n != -1) {
+          if (n < -1 || n >= nvis) {
+            report(p.err, CSA2_ERR_INDEX);
+          } else {
+            sl[r] = cache_slot(p.c, b, n);
+            if (sl[r] < 0) report(p.err, CSA2_ERR_INDEX);
+          }
+        }
+      } else if (j < nk) {
+        sl[r] = int64_t(ring) * p.R + (lo + (j - nks)) % p.R;
+        sc[r] = (own_token && j == nk - 1) ? *new_scale : p.scale[sl[r]];
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < KPT; ++r) {
+      const int jl = tid + r * AM_THREADS, j = key0 + jl;
+      if (jl >= ntiles * AM_TILE) continue;
+      const bool win = j >= nks && j < nk;
+      slot[jl] = sl[r];
+      mu[jl] = j < nks ? p.tau : (win ? p.tau * sc[r] : 0.f);
+      pv[jl] = j < nks ? 1.f : (win ? sc[r] : 0.f);
+    }
   }
   if (producer) publish_query_max(qraw, qmx);
   if (warp == AM_PRODUCERS / 32) {
