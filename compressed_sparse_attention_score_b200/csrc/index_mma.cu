@@ -220,7 +220,7 @@ __device__ __forceinline__ void select_cluster(const uint32_t *kl, const int32_t
 }
 
 template <bool SEL>
-__global__ void __launch_bounds__(IM_THREADS, SEL ? 1 : 2) index_score_mma_kernel(const __grid_constant__ CUtensorMap tmap,
+__global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                                  IndexMmaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -624,9 +624,9 @@ int select_clusters(int cs) {
 }  // namespace
 
 // Cluster size: at most IM_CAND_TILES tiles per CTA (8 CTAs for a pool of 16384), up to 16 CTAs
-// of about 8 tiles while the rows' clusters fill at most half the SMs (every CTA quantises the
-// row's query again, so many rows take fewer, longer CTAs), and only as large as lets every
-// row's cluster run at once.
+// of about 8 tiles while the rows' CTAs fit two per SM (every CTA quantises the row's query
+// again, so many rows take fewer, longer CTAs), and only as large as lets every row's cluster
+// run at once.
 void launch_reindex_select(const uint16_t *q_ix, const uint16_t *w, int B, int Q, const int32_t *q_pos,
                            const int32_t *cand, int P, int k, const csa2_cache &c, int32_t *sel, int32_t *err,
                            cudaStream_t st) {
@@ -636,7 +636,7 @@ void launch_reindex_select(const uint16_t *q_ix, const uint16_t *w, int B, int Q
   int cs_min = 1;  // every CTA's keys and candidate indices fit its shared memory
   while (cs_min * IM_CAND_TILES < t_all) cs_min *= 2;
   int cs = cs_min;
-  while (cs < 16 && cs * 8 < t_all && 2 * cs * rows <= sm_count()) cs *= 2;
+  while (cs < 16 && cs * 8 < t_all && 2 * cs * rows <= 2 * sm_count()) cs *= 2;
   while (cs > cs_min && select_clusters(cs) < min(rows, sm_count() / cs)) cs /= 2;
   select_clusters(cs);  // sets the kernel's attributes
   const int chunk = (t_all + cs - 1) / cs;
