@@ -72,6 +72,8 @@ constexpr int SM_CG = SM_HG + 2 * 256 * 4;              // [16][2] every CTA's c
 constexpr int SM_SELW = SM_CG + 16 * 2 * 4;             // selection state (4 words)
 constexpr int SM_WCNT = SM_SELW + 16;                   // per warp: keys above / equal to the threshold
 constexpr size_t IM_SEL_SMEM_BYTES = SM_WCNT + 2 * (IM_THREADS / 32) * 4 + 1024;
+static_assert((IM_SEL_MAX + IM_TILE - 1) / IM_TILE <= 16 * IM_CAND_TILES,
+              "a pool of IM_SEL_MAX candidates must fit 16 CTAs of IM_CAND_TILES tiles (the count table holds 16)");
 }  // namespace
 
 struct IndexMmaArgs {

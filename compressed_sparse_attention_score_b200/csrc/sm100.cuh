@@ -25,12 +25,12 @@ __device__ __forceinline__ void mbar_init_fence() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-// Split cluster barrier (every thread of every CTA of the cluster, warp-converged): arrive
-// (release: this thread's earlier writes become visible), then wait (acquire).  Used to know
-// that every CTA of the cluster has started, and initialised what peers will write into,
-// before its shared memory is written remotely.
-__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.aligned;" ::: "memory"); }
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+// Split cluster barrier (every thread of every CTA of the cluster): arrive (release: this
+// thread's earlier writes become visible), then wait (acquire).  Used to know that every CTA of
+// the cluster has started, and initialised what peers will write into, before its shared memory
+// is written remotely.  The non-.aligned forms: a warp need not be converged at either.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait;" ::: "memory"); }
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
