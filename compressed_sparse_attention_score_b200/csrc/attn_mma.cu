@@ -266,20 +266,29 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32]) {
   return v[0];
 }
 
-// Cluster epilogue of a key-split row.  Partial of this CTA's keys: O_s (relative to
-// its own max m_s) staged in shared memory as [32 heads][512 dims] fp32, plus m_s and
-// l_s.  Then each CTA of the cluster combines one slice of dims over all peers:
-// o = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s, M = max_s m_s.
+// Cluster epilogue of a key-split row.  Partial of this CTA's keys: O_s (relative to its own
+// max m_s) in TMEM, plus m_s and l_s.  CTA q owns dims [q PER, q PER + PER); every CTA pushes
+// each owner its slice of O_s and every owner its (m_s, l_s), straight from TMEM into the
+// owners' receive buffers (remote stores, nothing waits on them), then one cluster barrier, and
+// each owner combines its slice locally: o = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s,
+// M = max_s m_s.  The receive buffer (recv: CS x 32 x PER floats, then CS x 64 statistics) is
+// the CTA's key-tile memory, so a first barrier (split: arrive when this CTA's products are
+// complete, wait before the first push) keeps peers from writing into a tile still being read.
 template <int CS>
 __device__ __forceinline__ void combine_partials(const AttnArgs &p, uint32_t tmem, bool aborted, bool has_keys,
-                                                 float *stage, float *red, float *hmax, float *hsum, int row, int hg,
+                                                 float *recv, float *red, float *hmax, float *hsum, int row, int hg,
                                                  int split) {
+  constexpr int PER = ((D + CS - 1) / CS + 3) & ~3;  // dims per owner, a multiple of 4
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  float *stats = recv + CS * 32 * PER;  // [source][max 32 | sum 32]
+  cg::cluster_group cluster = cg::this_cluster();
+  if (warp < 4 && aborted) {
+    hsum[lane] = 0.f;
+    hmax[lane] = -INFINITY;
+  }
+  cluster_arrive();  // this CTA's tensor-core products are complete
+  bool waited = false;
   if (warp < 4) {
-    if (aborted) {
-      hsum[lane] = 0.f;
-      hmax[lane] = -INFINITY;
-    }
     for (int d = 0; d < 4; ++d) {
       uint32_t r0[16], r1[16];
       if (!aborted && has_keys) {
@@ -291,67 +300,66 @@ __device__ __forceinline__ void combine_partials(const AttnArgs &p, uint32_t tme
 #pragma unroll
         for (int i = 0; i < 16; ++i) r0[i] = r1[i] = 0u;
       }
-      const int dim = 128 * d + 32 * warp + lane;
+      if (!waited) {
+        cluster_wait();  // every peer's tile memory is free
+        waited = true;
+      }
+      const int dim = 128 * d + 32 * warp + lane, q = dim / PER;
+      float *dst = cluster.map_shared_rank(recv + split * 32 * PER + (dim - q * PER), q);
 #pragma unroll
       for (int h = 0; h < 16; ++h) {
-        stage[h * D + dim] = __uint_as_float(r0[h]);
-        stage[(16 + h) * D + dim] = __uint_as_float(r1[h]);
+        dst[h * PER] = __uint_as_float(r0[h]);
+        dst[(16 + h) * PER] = __uint_as_float(r1[h]);
       }
     }
+    if (warp == 0) {
+      const float m = hmax[lane], l = hsum[lane];
+#pragma unroll
+      for (int q = 0; q < CS; ++q) {
+        float *st = cluster.map_shared_rank(stats + split * 64, q);
+        st[lane] = m;
+        st[32 + lane] = l;
+      }
+    }
+  } else {
+    cluster_wait();
   }
-  cg::cluster_group cluster = cg::this_cluster();
-  cluster.sync();
-  float *wts = red;          // [CS][32] combination weights (red is free now)
+  cluster.sync();  // every slice and statistic has arrived; no peer's memory is touched after this
+  float *wts = red;  // [CS][32] combination weights
   float *lsum = red + CS * 32;
   if (tid < 32) {
     float M = -INFINITY;
-    for (int q = 0; q < CS; ++q) M = fmaxf(M, cluster.map_shared_rank(hmax, q)[tid]);
+#pragma unroll
+    for (int q = 0; q < CS; ++q) M = fmaxf(M, stats[q * 64 + tid]);
     float L = 0.f;
+#pragma unroll
     for (int q = 0; q < CS; ++q) {
-      const float mq = cluster.map_shared_rank(hmax, q)[tid];
+      const float mq = stats[q * 64 + tid];
       const float wq = (M == -INFINITY || mq == -INFINITY) ? 0.f : __expf(mq - M);
       wts[q * 32 + tid] = wq;
-      L += wq * cluster.map_shared_rank(hsum, q)[tid];
+      L += wq * stats[q * 64 + 32 + tid];
     }
     lsum[tid] = L;
     if (split == 0) p.lse[int64_t(row) * H + hg * AM_HG + tid] = L > 0.f ? M + logf(L) : -INFINITY;
   }
   __syncthreads();
-  // this CTA's slice of dims (a multiple of 4), read as float4 from every peer with all
-  // of a thread's loads in flight together
-  const int per = ((D + CS - 1) / CS + 3) & ~3;
-  const int d0 = min(D, split * per), nq = (min(D, d0 + per) - d0) / 4;
+  const int d0 = min(D, split * PER), nq = (min(D, d0 + PER) - d0) / 4;
   float *orow = p.o + (int64_t(row) * H + hg * AM_HG) * D;
-  constexpr int CU = 2;  // items per thread per round
-  for (int it0 = tid; it0 < 32 * nq; it0 += CU * AM_THREADS) {
-    float4 x[CU][CS];
+  for (int it = tid; it < 32 * nq; it += AM_THREADS) {
+    const int h = it / nq, dl = 4 * (it % nq);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int u = 0; u < CU; ++u) {
-      const int it = min(it0 + u * AM_THREADS, 32 * nq - 1);
-      const int h = it / nq, dim = d0 + 4 * (it % nq);
-#pragma unroll
-      for (int q = 0; q < CS; ++q)
-        x[u][q] = *reinterpret_cast<const float4 *>(cluster.map_shared_rank(stage, q) + h * D + dim);
+    for (int q = 0; q < CS; ++q) {
+      const float wq = wts[q * 32 + h];
+      const float4 x = *reinterpret_cast<const float4 *>(recv + (q * 32 + h) * PER + dl);
+      acc.x += wq * x.x;
+      acc.y += wq * x.y;
+      acc.z += wq * x.z;
+      acc.w += wq * x.w;
     }
-#pragma unroll
-    for (int u = 0; u < CU; ++u) {
-      const int it = it0 + u * AM_THREADS;
-      if (it >= 32 * nq) break;
-      const int h = it / nq, dim = d0 + 4 * (it % nq);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int q = 0; q < CS; ++q) {
-        const float wq = wts[q * 32 + h];
-        acc.x += wq * x[u][q].x;
-        acc.y += wq * x[u][q].y;
-        acc.z += wq * x[u][q].z;
-        acc.w += wq * x[u][q].w;
-      }
-      const float L = lsum[h], inv = L > 0.f ? 1.f / L : 0.f;
-      *reinterpret_cast<float4 *>(orow + h * D + dim) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    }
+    const float L = lsum[h], inv = L > 0.f ? 1.f / L : 0.f;
+    *reinterpret_cast<float4 *>(orow + h * D + d0 + dl) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   }
-  cluster.sync();  // every peer has finished reading this CTA's stage
 }
 
 template <int CS>

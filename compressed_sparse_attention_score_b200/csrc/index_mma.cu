@@ -55,7 +55,7 @@ constexpr int SM_STAGES = 0;
 constexpr int SM_B = IM_STAGES * IM_STAGE_BYTES;       // 64 x 64 B query codes
 constexpr int SM_SFB = SM_B + IM_N * 64;                // 512 B scale atom
 constexpr int SM_W = SM_SFB + 512;                      // 64 fp32 head weights
-constexpr int IM_CAND_TILES = 16;                       // candidate lists staged when a CTA has at most this many tiles
+constexpr int IM_CAND_TILES = 8;                        // candidate lists staged when a CTA has at most this many tiles
 constexpr int SM_CAND = SM_W + 256;                     // [IM_CAND_TILES * 128] candidate entry indices
 constexpr int SM_BAR = SM_CAND + IM_CAND_TILES * IM_TILE * 4;   // mbarriers
 constexpr int N_BARS = 2 * IM_STAGES + 2 * IM_ACC + 1;
@@ -625,7 +625,7 @@ int select_clusters(int cs) {
 }
 }  // namespace
 
-// Cluster size: at most IM_CAND_TILES tiles per CTA (8 CTAs for a pool of 16384), up to 16 CTAs
+// Cluster size: at most IM_CAND_TILES tiles per CTA (16 CTAs for a pool of 16384), up to 16 CTAs
 // of about 8 tiles while the rows' CTAs fit two per SM (every CTA quantises the row's query
 // again, so many rows take fewer, longer CTAs), and only as large as lets every row's cluster
 // run at once.
