@@ -760,11 +760,11 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   const bool own_token = p.swa_new && nkw > 0;
   const uint8_t *new_codes = smem + T_NEW;
   float *new_scale = reinterpret_cast<float *>(smem + T_NEW + 512);
-  if (own_token) quantise_new_token(p, row, ring, pos, split == 0 && hg == 0, smem + T_NEW, new_scale, new_scale + 4);
 
   // ---------------------------------------------------------------- loads
   // Producer t: key t % 128, dims 256 (t / 128) .. +255.  The query block's loads go
-  // out first, then the key's index, then its raw bytes, all before any barrier.
+  // out first, then the key's index, then its raw bytes, all before any barrier; this step's
+  // own window token is quantised while they are in flight, and its key loaded after that.
   uint4 qraw[AM_QU];
   uint4 rr[16];  // listed entry: rr[0..7] = 128 code bytes, rr[8] = 16 scale bytes; window: 256 codes
   const int key_in = tid & (AM_TILE - 1), half = (tid >> 7) & 1;
@@ -794,10 +794,11 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
       load_key_half(p, s, true, nullptr, half, rr);
     } else if (j < nk) {
       s = int64_t(ring) * p.R + (lo + (j - nks)) % p.R;
-      const bool own = own_token && j == nk - 1;
-      const float sc = own ? *new_scale : p.scale[s];
-      m = p.tau * sc, pm = sc;
-      load_key_half(p, s, false, own ? new_codes : nullptr, half, rr);
+      if (!(own_token && j == nk - 1)) {
+        const float sc = p.scale[s];
+        m = p.tau * sc, pm = sc;
+        load_key_half(p, s, false, nullptr, half, rr);
+      }
     }
     if (half == 0) {
       slot[key_in] = s;
@@ -805,6 +806,17 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
       pv[key_in] = pm;
     }
     publish_query_max(qraw, qmx);  // after the key loads are out
+  }
+  if (own_token) {
+    quantise_new_token(p, row, ring, pos, split == 0 && hg == 0, smem + T_NEW, new_scale, new_scale + 4);
+    if (producer && j == nk - 1) {
+      const float sc = *new_scale;
+      load_key_half(p, s, false, new_codes, half, rr);
+      if (half == 0) {
+        mu[key_in] = p.tau * sc;
+        pv[key_in] = sc;
+      }
+    }
   }
   if (warp == AM_PRODUCERS / 32) {
     tmem_alloc(tmem_slot, AM_TMEM_COLS);
