@@ -19,8 +19,8 @@
 //   warps 2-9  epilogue, two warpgroups taking alternate tiles: tcgen05.ld of
 //              the 64 head values of its 32 keys, weighted ReLU sum, fp32 score
 //              store.
-// The query heads are quantised to MXFP4 in the prologue (warps 2-5; same codec as
-// the keys).
+// The query heads are quantised to MXFP4 in the prologue (warps 2-9, one 32-value block per
+// thread; same codec as the keys).
 // Every mbarrier wait is time-bounded; on expiry the CTA drains and reports
 // CSA2_ERR_TIMEOUT instead of hanging.
 #include <cooperative_groups.h>
@@ -281,50 +281,47 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     mbar_init(done, 1);
     *abort_flag = 0;
     mbar_init_fence();
-  } else if (warp >= 2 && warp < 6) {
-    // quantise the query heads: threads 2h, 2h+1 own blocks {0,1}, {2,3} of head h.
-    // Dividing by the power-of-two scale 2^e is done as the (exactly equal) product
-    // with 2^-e.
-    const int t = threadIdx.x - 64, h = t >> 1, g0 = 2 * (t & 1);
+  } else if (warp >= 2) {
+    // quantise the query heads: thread 4h + g owns 32-value block g of head h (the 8 epilogue
+    // warps, idle until the first tile).  Dividing by the power-of-two scale 2^e is done as the
+    // (exactly equal) product with 2^-e.
+    const int t = threadIdx.x - 64, h = t >> 2, g = t & 3;
     const uint16_t *qh = a.q_ix + (int64_t(row) * HI + h) * DI;
     uint8_t *brow = smem + SM_B + h * 64;
-    uint32_t sfpart = 0;
-#pragma unroll 1
-    for (int g = g0; g < g0 + 2; ++g) {
-      float v[32];
+    float v[32];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 u = reinterpret_cast<const uint4 *>(qh + 32 * g)[i];
-        const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
+    for (int i = 0; i < 4; ++i) {
+      const uint4 u = reinterpret_cast<const uint4 *>(qh + 32 * g)[i];
+      const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          v[8 * i + 2 * j] = __uint_as_float(ww[j] << 16);
-          v[8 * i + 2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
-        }
+      for (int j = 0; j < 4; ++j) {
+        v[8 * i + 2 * j] = __uint_as_float(ww[j] << 16);
+        v[8 * i + 2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
       }
-      float am = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
-      int ex = -127;
-      uint32_t cw[4] = {0, 0, 0, 0};
-      if (am != 0.f) {
-        ex = e8m0_ceil_exponent(__fdiv_rn(am, 6.0f));
-        const float inv = pow2f(-ex);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) cw[i >> 3] |= e2m1_code(__fmul_rn(v[i], inv)) << (4 * (i & 7));
-      }
-      // 16 bytes = chunk g of this 64-byte row, at its swizzled position
-      *reinterpret_cast<uint4 *>(brow + ((g ^ ((h >> 1) & 3)) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      sfpart |= uint32_t(ex + 127) << (8 * g);
     }
-    const uint32_t sfword = sfpart | __shfl_xor_sync(0xffffffffu, sfpart, 1);
+    float am = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+    int ex = -127;
+    uint32_t cw[4] = {0, 0, 0, 0};
+    if (am != 0.f) {
+      ex = e8m0_ceil_exponent(__fdiv_rn(am, 6.0f));
+      const float inv = pow2f(-ex);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) cw[i >> 3] |= e2m1_code(__fmul_rn(v[i], inv)) << (4 * (i & 7));
+    }
+    // 16 bytes = chunk g of this 64-byte row, at its swizzled position
+    *reinterpret_cast<uint4 *>(brow + ((g ^ ((h >> 1) & 3)) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    uint32_t sfword = uint32_t(ex + 127) << (8 * g);
+    sfword |= __shfl_xor_sync(0xffffffffu, sfword, 1);
+    sfword |= __shfl_xor_sync(0xffffffffu, sfword, 2);
     // scale atom word of row r: lane-row r % 32, column r / 32 (rows 64..127 unused, zero)
     if constexpr (SEL)
-      for (int j = t; j < 512; j += 128) reinterpret_cast<uint32_t *>(smem + SM_HG)[j] = 0;
-    if ((t & 1) == 0) {
+      for (int j = t; j < 512; j += 256) reinterpret_cast<uint32_t *>(smem + SM_HG)[j] = 0;
+    if (g == 0) {
       *reinterpret_cast<uint32_t *>(smem + SM_SFB + (h & 31) * 16 + (h >> 5) * 4) = sfword;
       ws[h] = bf16_to_f32(a.w[int64_t(row) * HI + h]);
-    } else {
+    } else if (g == 1) {
       const int rz = 64 + h;
       *reinterpret_cast<uint32_t *>(smem + SM_SFB + (rz & 31) * 16 + (rz >> 5) * 4) = 0u;
     }

@@ -4,10 +4,11 @@
 // A 128-entry key tile is loaded once (one TMA box of the codes plus the scale words, or
 // cp.async gathers for caches a tensor map cannot describe) and serves all PF_Q queries: per
 // query two K=64 block-scaled FP4 MMAs (tcgen05 kind::mxf4, N = 64 heads) into the query's
-// accumulator; two sets of accumulators alternate between tiles.  Warp roles:
+// accumulator.  Two CTAs share an SM (each holds 256 TMEM columns and a 4-stage ring), so one
+// CTA's tensor-core and load phases fill the other's epilogue gaps.  Warp roles:
 //   warp 0       producer;
 //   warp 1       MMA issuer (one lane);
-//   warps 2-13   one epilogue warpgroup per query: the weighted-ReLU score of each of its 128
+//   warps 2-..   one epilogue warpgroup per query: the weighted-ReLU score of each of its 128
 //                keys per tile (the decode kernel's arithmetic, so both give the same fp32
 //                score); keys the query cannot see are dropped, keys above the query's running
 //                threshold are appended to its candidate list in shared memory.
@@ -30,18 +31,18 @@ namespace csa2 {
 using namespace sm100;
 
 namespace {
-constexpr int PF_Q = 3;                 // query tokens per CTA = epilogue warpgroups
-constexpr int PF_STAGES = 8;
+constexpr int PF_Q = 2;                 // query tokens per CTA = epilogue warpgroups
+constexpr int PF_STAGES = 4;
 constexpr int PF_TILE = 128;            // keys per tile = MMA M
 constexpr int PF_N = 64;                // indexer heads = MMA N
 constexpr int PF_A_BYTES = PF_TILE * 64;
 constexpr int PF_STAGE_BYTES = 9216;    // 8192 codes + 512 scale atom, padded to 1024
 constexpr int PF_WG = 128;              // threads per epilogue warpgroup
 constexpr int PF_THREADS = 64 + PF_Q * PF_WG;
-constexpr int PF_CAP = 4096;            // candidate list per query
+constexpr int PF_CAP = 2048;            // candidate list per query
 constexpr int PF_KMAX = 512;
-constexpr uint32_t PF_TMEM_COLS = 512;
-constexpr int PF_ACC = 2;               // accumulator sets (tiles in flight between MMA and epilogue)
+constexpr uint32_t PF_TMEM_COLS = 256;   // two CTAs per SM share the 512 columns
+constexpr int PF_ACC = 1;               // accumulator sets (the other CTA on the SM fills the gaps)
 constexpr uint32_t PF_COL_SFA = PF_ACC * PF_Q * 64;    // after the accumulator sets
 constexpr uint32_t PF_COL_SFB = PF_COL_SFA + 4 * PF_ACC;
 constexpr uint64_t PF_WAIT_NS = 2000000000ull;
@@ -201,7 +202,7 @@ __device__ uint32_t cut_to_k(uint32_t *keys, int32_t *ents, int n, int k, uint32
 }
 }  // namespace
 
-__global__ void __launch_bounds__(PF_THREADS, 1) prefill_index_kernel(const __grid_constant__ CUtensorMap tmap,
+__global__ void __launch_bounds__(PF_THREADS, 2) prefill_index_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                       PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
