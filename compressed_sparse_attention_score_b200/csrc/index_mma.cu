@@ -477,25 +477,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      // eight independent partial sums (heads h, h+8, ...) keep the FMA chains short
-      float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int h4 = 0; h4 < 8; ++h4) {
-        const float4 wv = w4[h4];
-        part[(4 * h4) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(r0[4 * h4]), 0.f), part[(4 * h4) & 7]);
-        part[(4 * h4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(r0[4 * h4 + 1]), 0.f), part[(4 * h4 + 1) & 7]);
-        part[(4 * h4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(r0[4 * h4 + 2]), 0.f), part[(4 * h4 + 2) & 7]);
-        part[(4 * h4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(r0[4 * h4 + 3]), 0.f), part[(4 * h4 + 3) & 7]);
-      }
-#pragma unroll
-      for (int h4 = 0; h4 < 8; ++h4) {
-        const float4 wv = w4[8 + h4];
-        part[(4 * h4) & 7] = fmaf(wv.x, fmaxf(__uint_as_float(r1[4 * h4]), 0.f), part[(4 * h4) & 7]);
-        part[(4 * h4 + 1) & 7] = fmaf(wv.y, fmaxf(__uint_as_float(r1[4 * h4 + 1]), 0.f), part[(4 * h4 + 1) & 7]);
-        part[(4 * h4 + 2) & 7] = fmaf(wv.z, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f), part[(4 * h4 + 2) & 7]);
-        part[(4 * h4 + 3) & 7] = fmaf(wv.w, fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f), part[(4 * h4 + 3) & 7]);
-      }
-      const float sc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+      const float sc = weighted_relu_score(r0, r1, w4);
       const int pos = (t0 + i) * IM_TILE + e;
       if (pos < a.n_out) {
         const bool ok = n_cur >= 0 && n_cur < nvis && cache_slot(a.c, b, n_cur) >= 0;

@@ -85,16 +85,6 @@ __device__ __forceinline__ int pf_entry_of_row(int m) { return (m & 31) * 4 + (m
 // Named barrier of one epilogue warpgroup (ids 1 .. PF_Q).
 __device__ __forceinline__ void wg_sync(int g) { asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "n"(PF_WG) : "memory"); }
 
-// c0 += a0 * b0 and c1 += a1 * b1, each one fp32 fused multiply-add rounded to nearest (the
-// packed form of two fmaf, bit for bit).
-__device__ __forceinline__ void fma2(float &c0, float &c1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
-      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\tmov.b64 pc, {%0, %1};\n\t"
-      "fma.rn.f32x2 pc, pa, pb, pc;\n\tmov.b64 {%0, %1}, pc;\n\t}"
-      : "+f"(c0), "+f"(c1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
 // The k-th largest key T of list keys[0..n) (n > k) and how many of the keys equal to T belong
 // to the best k (need_eq), by radix selection on 8-bit digits from the top; also whether every
 // key equal to T is kept (all_eq).  Called by the PF_WG threads of warpgroup g (t = their index).
@@ -424,27 +414,7 @@ __global__ void __launch_bounds__(PF_THREADS, 2) prefill_index_kernel(const __gr
         tc_ld_32x32b_x32(taddr + 32, r1);
         tc_wait_ld();
         tc_fence_before();
-        // heads h -> partial h % 8 in head order (the decode kernel's order, so the same score)
-        float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int h4 = 0; h4 < 8; ++h4) {
-          const float4 wv = w4[h4];
-          const int j = (4 * h4) & 7;
-          fma2(part[j], part[j + 1], wv.x, wv.y, fmaxf(__uint_as_float(r0[4 * h4]), 0.f),
-               fmaxf(__uint_as_float(r0[4 * h4 + 1]), 0.f));
-          fma2(part[j + 2], part[j + 3], wv.z, wv.w, fmaxf(__uint_as_float(r0[4 * h4 + 2]), 0.f),
-               fmaxf(__uint_as_float(r0[4 * h4 + 3]), 0.f));
-        }
-#pragma unroll
-        for (int h4 = 0; h4 < 8; ++h4) {
-          const float4 wv = w4[8 + h4];
-          const int j = (4 * h4) & 7;
-          fma2(part[j], part[j + 1], wv.x, wv.y, fmaxf(__uint_as_float(r1[4 * h4]), 0.f),
-               fmaxf(__uint_as_float(r1[4 * h4 + 1]), 0.f));
-          fma2(part[j + 2], part[j + 3], wv.z, wv.w, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f),
-               fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f));
-        }
-        sc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+        sc = weighted_relu_score(r0, r1, w4);  // the decode kernel's arithmetic: the same score
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);

@@ -245,5 +245,43 @@ __device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[1
       : "r"(taddr));
 }
 
+// c0 += a0 * b0 and c1 += a1 * b1, each one fp32 fused multiply-add rounded to nearest (the
+// packed form of two fmaf, bit for bit).
+__device__ __forceinline__ void fma2(float &c0, float &c1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\tmov.b64 pc, {%0, %1};\n\t"
+      "fma.rn.f32x2 pc, pa, pb, pc;\n\tmov.b64 {%0, %1}, pc;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// The indexer score of one key from its 64 head products (r0: heads 0-31, r1: heads 32-63, fp32
+// bits) and the head weights w4 (16 float4): sum_h w_h * relu(d_h), head h accumulated into
+// partial h % 8 in head order, the partials summed as a fixed tree.  Every indexer kernel scores
+// through this function, so all of them produce the same fp32 score for the same key.
+__device__ __forceinline__ float weighted_relu_score(const uint32_t (&r0)[32], const uint32_t (&r1)[32],
+                                                     const float4 *w4) {
+  float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int h4 = 0; h4 < 8; ++h4) {
+    const float4 wv = w4[h4];
+    const int j = (4 * h4) & 7;
+    fma2(part[j], part[j + 1], wv.x, wv.y, fmaxf(__uint_as_float(r0[4 * h4]), 0.f),
+         fmaxf(__uint_as_float(r0[4 * h4 + 1]), 0.f));
+    fma2(part[j + 2], part[j + 3], wv.z, wv.w, fmaxf(__uint_as_float(r0[4 * h4 + 2]), 0.f),
+         fmaxf(__uint_as_float(r0[4 * h4 + 3]), 0.f));
+  }
+#pragma unroll
+  for (int h4 = 0; h4 < 8; ++h4) {
+    const float4 wv = w4[8 + h4];
+    const int j = (4 * h4) & 7;
+    fma2(part[j], part[j + 1], wv.x, wv.y, fmaxf(__uint_as_float(r1[4 * h4]), 0.f),
+         fmaxf(__uint_as_float(r1[4 * h4 + 1]), 0.f));
+    fma2(part[j + 2], part[j + 3], wv.z, wv.w, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f),
+         fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f));
+  }
+  return ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+}
+
 }  // namespace sm100
 }  // namespace csa2
