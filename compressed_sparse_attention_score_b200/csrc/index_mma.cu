@@ -72,6 +72,7 @@ constexpr int SM_CG = SM_HG + 2 * 256 * 4;              // [16][2] every CTA's c
 constexpr int SM_SELW = SM_CG + 16 * 2 * 4;             // selection state (4 words)
 constexpr int SM_WCNT = SM_SELW + 16;                   // per warp: keys above / equal to the threshold
 constexpr size_t IM_SEL_SMEM_BYTES = SM_WCNT + 2 * (IM_THREADS / 32) * 4 + 1024;
+static_assert(IM_EPI_WG >= 2, "the query is quantised by 8 epilogue warps");
 static_assert((IM_SEL_MAX + IM_TILE - 1) / IM_TILE <= 16 * IM_CAND_TILES,
               "a pool of IM_SEL_MAX candidates must fit 16 CTAs of IM_CAND_TILES tiles (the count table holds 16)");
 }  // namespace
@@ -281,8 +282,8 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     mbar_init(done, 1);
     *abort_flag = 0;
     mbar_init_fence();
-  } else if (warp >= 2) {
-    // quantise the query heads: thread 4h + g owns 32-value block g of head h (the 8 epilogue
+  } else if (warp >= 2 && warp < 10) {
+    // quantise the query heads: thread 4h + g owns 32-value block g of head h (8 of the epilogue
     // warps, idle until the first tile).  Dividing by the power-of-two scale 2^e is done as the
     // (exactly equal) product with 2^-e.
     const int t = threadIdx.x - 64, h = t >> 2, g = t & 3;
