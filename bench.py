@@ -949,6 +949,20 @@ def main():
     achieved = wl.scan_bytes() / (scan_ms * 1e-3) / 1e9
     traffic = profiled_traffic(["compressed_sparse_attention_score_b200/csrc/index_mma.cu"],
                                "index_score_hier1m.md")
+    # context for the scan's fraction: a plain read-only stream over as many bytes (torch's sum
+    # reduction over the same 570 MB), timed the same way (L2 flushed, CUDA events)
+    stream_buf = torch.empty(wl.scan_bytes() // 4, dtype=torch.float32, device=dev).fill_(1.0)
+    rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+    stream_buf.sum()
+    for a, b in rev:
+        flush.zero_()
+        a.record(stream)
+        stream_buf.sum()
+        b.record(stream)
+    torch.cuda.synchronize()
+    read_ms = sorted(a.elapsed_time(b) for a, b in rev)[2]
+    read_gbs = wl.scan_bytes() / (read_ms * 1e-3) / 1e9
+    del stream_buf
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded N(0,1) latents and queries)",
@@ -957,7 +971,9 @@ def main():
             "roofline": {"bound": "hbm", "kernel": "csa2 indexer scan (Full layer)", "achieved": achieved,
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "scan_ms": scan_ms,
-                         "entries_scanned_per_s": wl.B * wl.N / (scan_ms * 1e-3)},
+                         "entries_scanned_per_s": wl.B * wl.N / (scan_ms * 1e-3),
+                         "read_stream": {"kernel": "torch sum over the same bytes (context, not the peak)",
+                                         "GBps": read_gbs, "scan_frac_of_it": achieved / read_gbs}},
             "gather": gather,
             "e2e": {"value": units / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,

@@ -1035,8 +1035,9 @@ static int attn_clusters_fit() {
 int attn_dense_segment() { return attn_clusters_fit<16>() > 0 ? 8192 : 4096; }
 
 // Up to 64 query rows: a cluster of CTAs (one per 128-key tile) splits each row's keys and
-// combines the partials through distributed shared memory (a few waves of one-tile CTAs finish
-// sooner than one wave of CTAs that take every tile of a row in turn).  A CTA holds at most 5
+// combines the partials through distributed shared memory; when those one-tile CTAs would need
+// more than one wave, clusters of two CTAs of two or three tiles each (measured on 32 rows of 640
+// keys: 47 us against 53 us for five-CTA clusters and 68 us for three).  A CTA holds at most 5
 // tiles (640 keys), so longer key sets (dense segments) always use clusters of up to 16 CTAs.
 void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
                      bool dense, int e0, int e1, int n_bound, const csa2_cache *c, const uint8_t *codes,
@@ -1054,6 +1055,7 @@ void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, floa
   const int nkeys = (dense ? max(0, e1 - e0) : a.k) + (codes ? window : 0);
   const int tiles = (nkeys + AM_TILE - 1) / AM_TILE;
   int cs = rows * (H / AM_HG) <= 128 ? max(1, min(tiles, 5)) : 1;
+  if (cs == 5 && rows * (H / AM_HG) * 5 > sm_count()) cs = 2;  // one wave of two-CTA clusters beats several of five
   if (cs > 1 && cs == tiles) {  // one tile per CTA: the single-dequant form
     switch (cs) {
       case 2: launch_tile<2>(a, rows, st); return;
