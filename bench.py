@@ -192,19 +192,19 @@ class Hier1M:
         torch.cuda.synchronize()
         assert k.csa2_check(err) == 0
 
-    # kernels launched per step, by call: pack_kv 1; per layer pack_swa 1 and one attention launch that covers
-    # the sparse branch, the SWA branch and their log-sum-exp merge; the Full layer's indexer scan 1 and top-k 1
-    # (its top-512 and pool share one launch); per Reindex layer one launch that scores the pool and selects
+    # kernels launched per step, by call: pack_kv 1; per layer one attention launch that packs the layer's window
+    # token and covers the sparse branch, the SWA branch and their log-sum-exp merge; the Full layer's indexer
+    # scan 1 and top-k 1 (its top-512 and pool share one launch); per Reindex layer one launch that scores the
+    # pool and selects
     def launches_per_step(self):
-        return 1 + 4 + (self.LAYERS - 1) * 3
+        return 1 + 3 + (self.LAYERS - 1) * 2
 
-    # The step in three parts: [pack the new token's entry; pack layer 0's SWA token], [the Full layer's
-    # scan], [its top-k and attention; the four Reindex layers].  The scan stays a separate part so that
-    # CUDA events can time it even when the other two parts are replayed as CUDA graphs.
+    # The step in three parts: [pack the new token's entry], [the Full layer's scan], [its top-k and
+    # attention; the four Reindex layers].  The scan stays a separate part so that CUDA events can time it
+    # even when the other two parts are replayed as CUDA graphs.  Every layer's window token is packed into
+    # its SWA ring inside that layer's attention launch (swa_new).
     def part_pre(self):
-        k = self.k
-        k.csa2_pack_kv(self.new_kv, self.new_ix, self.first_entry, self.cache, err=self.err)
-        k.csa2_pack_swa(self.swa_new[0], self.swa_pos, self.swa_codes[0], self.swa_scale[0], err=self.err)
+        self.k.csa2_pack_kv(self.new_kv, self.new_ix, self.first_entry, self.cache, err=self.err)
 
     def part_scan(self):
         self.k.csa2_index_score(self.q_ix[0], self.w[0], self.q_pos, self.cache, self.N, scores=self.scores,
@@ -214,11 +214,8 @@ class Hier1M:
         k, s = self.k, self.spec
         k.csa2_topk(self.scores, s.k, idx=self.idx[0], k2=s.pool_k, idx2=self.pool)
         for layer in range(self.LAYERS):
-            if layer > 0:
-                k.csa2_pack_swa(self.swa_new[layer], self.swa_pos, self.swa_codes[layer], self.swa_scale[layer],
-                                err=self.err)
             q, q_ix, w = self.q[layer], self.q_ix[layer], self.w[layer]
-            swa = dict(swa_codes=self.swa_codes[layer], swa_scale=self.swa_scale[layer])
+            swa = dict(swa_codes=self.swa_codes[layer], swa_scale=self.swa_scale[layer], swa_new=self.swa_new[layer])
             if layer == 0:
                 k.csa2_sparse_attn("reuse", q, self.q_pos, self.cache, s.tau, self.N, k=s.k, idx_in=self.idx[0],
                                    o=self.o[layer], lse=self.lse[layer], err=self.err, **swa)

@@ -69,7 +69,8 @@ _SIGS = {
                    c_void_p, c_void_p], ctypes.c_int),
     "csa2_sparse_attn": ([ctypes.c_int, c_void_p, c_int32, c_int32, c_void_p, c_float, c_void_p, c_void_p,
                           c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int32, _P, c_void_p, c_void_p, c_int32,
-                          c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p], ctypes.c_int),
+                          c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p],
+                         ctypes.c_int),
     "csa2_swa_attn": ([c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_float,
                        c_void_p, c_void_p, c_void_p, c_void_p], ctypes.c_int),
     "csa2_merge": ([c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p],
@@ -228,8 +229,9 @@ def csa2_topk(scores, k, n_valid=None, idx=None, val=None, k2=0, idx2=None, val2
 
 def csa2_sparse_attn(mode, q, q_pos, cache, softmax_scale, max_entries, k=512, q_ix=None, w=None, pool_k=0,
                      pool_io=None, idx_in=None, idx_out=None, o=None, lse=None, ws=None, err=None, stream=None,
-                     swa_codes=None, swa_scale=None, window=128):
-    """One layer's sparse branch; with swa_codes/swa_scale the SWA window joins the same softmax (merged)."""
+                     swa_codes=None, swa_scale=None, window=128, swa_new=None):
+    """One layer's sparse branch; with swa_codes/swa_scale the SWA window joins the same softmax (merged).
+    swa_new [B][1][512] bf16 (decode): this step's window token, quantised into the ring in the same launch."""
     B, Q = q.shape[0], q.shape[1]
     if o is None:
         o = torch.empty((B, Q, HEADS, MAIN_DIM), dtype=torch.float32, device=q.device)
@@ -242,8 +244,9 @@ def csa2_sparse_attn(mode, q, q_pos, cache, softmax_scale, max_entries, k=512, q
     R = 0 if swa_codes is None else swa_codes.shape[1]
     _ok(_lib.csa2_sparse_attn(MODE[mode], _ptr(q), B, Q, _ptr(q_pos), float(softmax_scale), _ptr(q_ix), _ptr(w),
                               k, pool_k, _ptr(pool_io), _ptr(idx_in), _ptr(idx_out), max_entries, ctypes.byref(d),
-                              _ptr(swa_codes), _ptr(swa_scale), R, window, _ptr(o), _ptr(lse), _ptr(ws),
-                              0 if ws is None else ws.numel(), _ptr(err), _stream(stream)), "csa2_sparse_attn")
+                              _ptr(swa_codes), _ptr(swa_scale), R, window, _ptr(swa_new), _ptr(o), _ptr(lse),
+                              _ptr(ws), 0 if ws is None else ws.numel(), _ptr(err), _stream(stream)),
+        "csa2_sparse_attn")
     return o, lse
 
 

@@ -186,8 +186,8 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
                                          const uint16_t *w, int32_t k, int32_t pool_k, int32_t *pool_io,
                                          const int32_t *idx_in, int32_t *idx_out, int32_t max_entries,
                                          const csa2_cache *cache, const uint8_t *swa_codes, const float *swa_scale,
-                                         int32_t R, int32_t window, float *o, float *lse, void *ws, size_t ws_bytes,
-                                         int32_t *err, csa2_stream_t stream) {
+                                         int32_t R, int32_t window, const uint16_t *swa_new, float *o, float *lse,
+                                         void *ws, size_t ws_bytes, int32_t *err, csa2_stream_t stream) {
   if (B < 0 || Q < 0 || k < 1 || pool_k < 0 || max_entries < 0) return fail(CSA2_ERR_INVALID_ARG, "bad size");
   if (B == 0 || Q == 0) return CSA2_OK;
   if (csa2_status s = check_cache(cache, B)) return s;
@@ -197,6 +197,10 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
   if (swa_codes) {
     if (!swa_scale || window < 1 || window > 128 || R < window) return fail(CSA2_ERR_INVALID_ARG, "need 1 <= window <= 128, window <= R");
     if (!aligned16(swa_codes)) return fail(CSA2_ERR_INVALID_ARG, "swa_codes misaligned");
+  }
+  if (swa_new) {
+    if (!swa_codes || Q != 1) return fail(CSA2_ERR_INVALID_ARG, "swa_new needs the window branch and Q == 1");
+    if (reinterpret_cast<uintptr_t>(swa_new) & 7) return fail(CSA2_ERR_INVALID_ARG, "swa_new misaligned");
   }
   if (int64_t(B) * Q > 65535 * 16) return fail(CSA2_ERR_UNSUPPORTED, "too many query rows per call");
   const int rows = B * Q;
@@ -215,7 +219,7 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
       const int e1 = e0 + seg < max_entries ? e0 + seg : max_entries;
       csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, nullptr, 0, true, e0, e1, max_entries, cache,
                             s == 0 ? swa_codes : nullptr, s == 0 && swa_codes ? swa_scale : nullptr, R, window,
-                            s == 0 ? o : po, s == 0 ? lse : pl, err, stream);
+                            s == 0 ? o : po, s == 0 ? lse : pl, err, stream, s == 0 ? swa_new : nullptr);
       if (s > 0) csa2::launch_merge(o, lse, po, pl, int64_t(rows) * CSA2_HEADS, CSA2_MAIN_DIM, o, lse, stream);
     }
     return launched("csa2_sparse_attn");
@@ -235,7 +239,7 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
       int32_t *sel = idx_out ? idx_out : static_cast<int32_t *>(ws);
       csa2::launch_prefill_index(q_ix, w, B, Q, q_pos, k, max_entries, *cache, sel, err, stream);
       csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, sel, k, false, 0, 0, 0, cache, swa_codes,
-                            swa_codes ? swa_scale : nullptr, R, window, o, lse, err, stream);
+                            swa_codes ? swa_scale : nullptr, R, window, o, lse, err, stream, swa_new);
       return launched("csa2_sparse_attn");
     }
     const int n_out = mode == CSA2_MODE_FULL ? max_entries : pool_k;
@@ -260,7 +264,7 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
     return fail(CSA2_ERR_INVALID_ARG, "bad mode");
   }
   csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, idx, k, false, 0, 0, 0, cache, swa_codes,
-                        swa_codes ? swa_scale : nullptr, R, window, o, lse, err, stream);
+                        swa_codes ? swa_scale : nullptr, R, window, o, lse, err, stream, swa_new);
   return launched("csa2_sparse_attn");
 }
 

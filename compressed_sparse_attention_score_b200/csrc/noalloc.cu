@@ -70,6 +70,7 @@ CSA2_EXPORT csa2_status csa2_sparse_attn_noalloc(csa2_mode mode, const uint16_t 
     }
   }
   return csa2_sparse_attn(mode, q, B, Q, q_pos, softmax_scale, q_ix, w, k, pool_k, pool_io, idx_in, idx_out,
-                          max_entries, cache, swa_codes, swa_scale, R, window, o, lse, ws, need > 0 ? kScratchBytes : 0,
+                          max_entries, cache, swa_codes, swa_scale, R, window, nullptr, o, lse, ws,
+                          need > 0 ? kScratchBytes : 0,
                           err, stream);
 }

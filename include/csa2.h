@@ -259,6 +259,11 @@ csa2_status csa2_index_topk(const uint16_t *q_ix, const uint16_t *w, int32_t B, 
  * window of each query (as csa2_swa_attn: ring [B][R], window <= 128) joins the
  * same softmax, so o / lse are the log-sum-exp merge of the two branches
  * (what csa2_merge of the separate results gives).  swa_codes = NULL: none.
+ * swa_new [B][1][512] bf16 (decode, Q == 1, with the window branch; NULL: none): this step's
+ * token of each sequence for the window, quantised inside the launch exactly as csa2_pack_swa
+ * quantises it, written to ring slot q_pos mod R (codes and scale) and used as the window's last
+ * key -- csa2_pack_swa followed by this call, in one launch ("从V4到V4.1 Flash", SWA 有界重放).
+ * 8-byte aligned.
  * ws: csa2_workspace_size(mode, ...) bytes (may be NULL for REUSE).
  * Device errors: an index outside the visible entries -> CSA2_ERR_INDEX, skipped;
  * FULL or DENSE with a query that sees more than max_entries entries -> CSA2_ERR_SHAPE
@@ -269,9 +274,9 @@ csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int32_t B, int32
                              const uint16_t *w, int32_t k, int32_t pool_k, int32_t *pool_io,
                              const int32_t *idx_in, int32_t *idx_out, int32_t max_entries,
                              const csa2_cache *cache, const uint8_t *swa_codes,
-                             const float *swa_scale, int32_t R, int32_t window, float *o,
-                             float *lse, void *ws, size_t ws_bytes, int32_t *err,
-                             csa2_stream_t stream);
+                             const float *swa_scale, int32_t R, int32_t window,
+                             const uint16_t *swa_new, float *o, float *lse, void *ws,
+                             size_t ws_bytes, int32_t *err, csa2_stream_t stream);
 
 /*
  * Sliding-window branch ("从V4到V4.1 Flash", sections "CSA2 机制下的全局 KV 共享与局部

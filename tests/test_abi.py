@@ -80,12 +80,16 @@ def test_host_side_argument_checks(lib):
     assert lib.csa2_swa_attn(addr, 1, 1, addr, addr, addr, 64, 128, 1.0, addr, addr, None, None) == 1
     c.ratio = 1
     assert lib.csa2_sparse_attn(7, addr, 1, 1, addr, 1.0, None, None, 512, 0, None, None, None, 16,
-                                ctypes.byref(c), None, None, 0, 0, addr, addr, None, 0, None, None) == 1
+                                ctypes.byref(c), None, None, 0, 0, None, addr, addr, None, 0, None, None) == 1
     assert lib.csa2_sparse_attn(2, addr, 1, 1, addr, 1.0, None, None, 1024, 0, None, addr, None, 16,
-                                ctypes.byref(c), None, None, 0, 0, addr, addr, None, 0, None, None) == 3
+                                ctypes.byref(c), None, None, 0, 0, None, addr, addr, None, 0, None, None) == 3
     assert lib.csa2_sparse_attn(0, addr, 1, 1, addr, 1.0, addr, addr, 512, 0, None, None, None, 16,
-                                ctypes.byref(c), None, None, 0, 0, addr, addr, None, 0, None, None) == 1
+                                ctypes.byref(c), None, None, 0, 0, None, addr, addr, None, 0, None, None) == 1
     assert b"workspace" in lib.csa2_last_error_string()
+    # this step's window token needs the window branch and one query per sequence
+    assert lib.csa2_sparse_attn(2, addr, 1, 2, addr, 1.0, None, None, 512, 0, None, addr, None, 16,
+                                ctypes.byref(c), addr, addr, 128, 128, addr, addr, addr, None, 0, None, None) == 1
+    assert b"swa_new" in lib.csa2_last_error_string()
 
 
 def test_zero_work_calls_are_no_ops(lib):
@@ -95,7 +99,7 @@ def test_zero_work_calls_are_no_ops(lib):
     assert lib.csa2_index_score(None, None, 0, 1, None, None, 0, 16, None, None, None, None) == 0
     assert lib.csa2_topk(None, None, 0, 10, 5, None, None, 0, None, None, None) == 0
     assert lib.csa2_sparse_attn(2, None, 0, 1, None, 1.0, None, None, 512, 0, None, None, None, 16,
-                                None, None, None, 0, 0, None, None, None, 0, None, None) == 0
+                                None, None, None, 0, 0, None, None, None, None, 0, None, None) == 0
     assert lib.csa2_swa_attn(None, 0, 1, None, None, None, 128, 128, 1.0, None, None, None, None) == 0
     assert lib.csa2_merge(None, None, None, None, 0, 512, None, None, None) == 0
     # negative sizes are still errors

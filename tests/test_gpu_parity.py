@@ -708,6 +708,39 @@ def test_prefill_fused_ties_and_short_rows():
             assert got[:nvis].tolist() == want and (got[nvis:] == -1).all()
 
 
+# ------------------------------------------------------------------ this step's window token in the attention launch
+@pytest.mark.parametrize("case", ["reuse4", "reuse32", "full1"])
+def test_swa_new_token_in_the_attention_launch(case):
+    """csa2_sparse_attn with swa_new (the step's window token quantised inside the launch) must equal
+    csa2_pack_swa of that token followed by csa2_sparse_attn, bit for bit: the ring's codes and scale
+    and the layer's o and lse.  reuse4: one-tile clusters; reuse32: two-CTA clusters of the general
+    kernel; full1: the Full path (scan, top-k, attention)."""
+    k = K()
+    if case == "full1":
+        spec = W.scaled(W.tiny_full(), [3001], B=1)
+    else:
+        B = 4 if case == "reuse4" else 32
+        spec = W.scaled(W.reuse64k(), [3000 + 37 * b for b in range(B)], B=B)
+    cache = gpu_cache(spec)
+    q, q_ix, w, q_pos = W.query_tensors(spec, 0, DEV)
+    x, pos = W.swa_tokens(spec, 0, DEV)
+    err = _err()
+    ring = [torch.zeros((spec.B, 128, 512), dtype=torch.uint8, device=DEV),
+            torch.zeros((spec.B, 128), dtype=torch.float32, device=DEV)]
+    k.csa2_pack_swa(x[:, :-1].contiguous(), pos[:, :-1].contiguous(), ring[0], ring[1], err=err)
+    ring2 = [t.clone() for t in ring]
+    mode = "full" if case == "full1" else "reuse"
+    kw = dict(q_ix=q_ix, w=w) if mode == "full" else dict(idx_in=W.reuse_indices(spec, DEV))
+    k.csa2_pack_swa(x[:, -1:].contiguous(), pos[:, -1:].contiguous(), ring[0], ring[1], err=err)
+    o1, l1 = k.csa2_sparse_attn(mode, q, q_pos, cache, spec.tau, spec.max_entries, err=err, swa_codes=ring[0],
+                                swa_scale=ring[1], **kw)
+    o2, l2 = k.csa2_sparse_attn(mode, q, q_pos, cache, spec.tau, spec.max_entries, err=err, swa_codes=ring2[0],
+                                swa_scale=ring2[1], swa_new=x[:, -1:].contiguous(), **kw)
+    assert k.csa2_check(err) == 0
+    assert torch.equal(ring[0], ring2[0]) and torch.equal(ring[1], ring2[1])
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
 # ------------------------------------------------------------------ fused Reindex selection
 @pytest.mark.parametrize("B,P,tokens", [(8, 16384, 2 * 20000), (3, 5000, 2 * 9000), (4, 3000, 2 * 4000),
                                         (300, 700, 2 * 1500), (2, 400, 2 * 1000)])
