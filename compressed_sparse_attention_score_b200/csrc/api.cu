@@ -263,6 +263,8 @@ CSA2_EXPORT csa2_status csa2_sparse_attn(csa2_mode mode, const uint16_t *q, int3
   } else {
     return fail(CSA2_ERR_INVALID_ARG, "bad mode");
   }
+  // (a programmatic dependent launch after the selection measured no faster here: 0.390 against
+  // 0.389 ms on the hier1m step, 62 against 53 us on one-query Full decode)
   csa2::launch_attn_mma(q, B, Q, q_pos, softmax_scale, idx, k, false, 0, 0, 0, cache, swa_codes,
                         swa_codes ? swa_scale : nullptr, R, window, o, lse, err, stream, swa_new);
   return launched("csa2_sparse_attn");

@@ -382,6 +382,19 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   const bool producer = tid < AM_PRODUCERS, issuer = tid == AM_PRODUCERS;
   const int row = blockIdx.x, hg = blockIdx.y;   // query row; its sequence b owns SWA ring b
   const int lrow = row, b = row / p.Q, ring = b;
+  // The query block (an input of the call) is loaded first; everything else may be written by
+  // the kernel launched just before this one, so it is read after grid_dep_wait().
+  uint4 qraw[AM_QU];
+  if (producer) {
+    const uint16_t *qrow = p.q + (int64_t(row) * H + hg * AM_HG) * D;
+#pragma unroll
+    for (int u = 0; u < AM_QU; ++u) {
+      const int it = tid + u * AM_PRODUCERS;
+      qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
+    }
+  }
+  grid_dep_launch();
+  grid_dep_wait();
   const int pos = p.q_pos[row];
 
   // ---------------------------------------------------------------- key list
@@ -403,18 +416,9 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   const int ntiles = min(min(tiles_all, tile0 + tps) - tile0, AM_MAXKEYS / AM_TILE);
   if (tid == 0 && (tps > AM_MAXKEYS / AM_TILE || (p.dense && nvis > p.n_bound))) report(p.err, CSA2_ERR_SHAPE);
   const int key0 = tile0 * AM_TILE;  // first key of this CTA; local key j is key key0 + j
-  // the query block's loads go out first; they are converted once the key list is done
+  // the query block (loaded above) is converted once the key list is done
   uint32_t *qmx = reinterpret_cast<uint32_t *>(smem + SM_QS);
   float *qinv = reinterpret_cast<float *>(smem + SM_QS + 8 * AM_QU * 4);
-  uint4 qraw[AM_QU];
-  if (producer) {
-    const uint16_t *qrow = p.q + (int64_t(row) * H + hg * AM_HG) * D;
-#pragma unroll
-    for (int u = 0; u < AM_QU; ++u) {
-      const int it = tid + u * AM_PRODUCERS;
-      qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
-    }
-  }
   // this step's own window token (the row's last key), quantised here and stored by one CTA
   const bool own_token = p.swa_new && nkw > 0;
   uint8_t *new_codes = own_token ? smem + SM_NEW : nullptr;
@@ -743,6 +747,19 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   const int row = blockIdx.x, hg = blockIdx.y;
   const int split = int(cg::this_cluster().block_rank());
   const int lrow = row, b = row / p.Q, ring = b;   // the row's sequence b owns SWA ring b
+  // The query block (an input of the call) is loaded first; everything else may be written by
+  // the kernel launched just before this one, so it is read after grid_dep_wait().
+  uint4 qraw[AM_QU];
+  if (producer) {
+    const uint16_t *qrow = p.q + (int64_t(row) * H + hg * AM_HG) * D;
+#pragma unroll
+    for (int u = 0; u < AM_QU; ++u) {
+      const int it = tid + u * AM_PRODUCERS;
+      qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
+    }
+  }
+  grid_dep_launch();
+  grid_dep_wait();
   const int pos = p.q_pos[row];
   const int nvis = (p.idx || p.dense) ? visible_entries(p.c, b, pos) : 0;
   const int nks = p.dense ? max(0, min(p.e1, nvis) - p.e0) : (p.idx ? p.k : 0);
@@ -765,19 +782,12 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   // Producer t: key t % 128, dims 256 (t / 128) .. +255.  The query block's loads go
   // out first, then the key's index, then its raw bytes, all before any barrier; this step's
   // own window token is quantised while they are in flight, and its key loaded after that.
-  uint4 qraw[AM_QU];
   uint4 rr[16];  // listed entry: rr[0..7] = 128 code bytes, rr[8] = 16 scale bytes; window: 256 codes
   const int key_in = tid & (AM_TILE - 1), half = (tid >> 7) & 1;
   const int j = key0 + key_in;
   bool sparse = false;
   int64_t s = -1;
   if (producer) {
-    const uint16_t *qrow = p.q + (int64_t(row) * H + hg * AM_HG) * D;
-#pragma unroll
-    for (int u = 0; u < AM_QU; ++u) {
-      const int it = tid + u * AM_PRODUCERS;
-      qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
-    }
     float m = 0.f, pm = 0.f;
     if (j < nks) {
       sparse = true;
@@ -952,7 +962,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
 }
 
 template <int CS>
-static void launch_tile(const AttnArgs &a, int rows, cudaStream_t st) {
+static void launch_tile(const AttnArgs &a, int rows, cudaStream_t st, bool pdl) {
   static bool attr[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -965,18 +975,20 @@ static void launch_tile(const AttnArgs &a, int rows, cudaStream_t st) {
   cfg.blockDim = dim3(AM_THREADS);
   cfg.dynamicSmemBytes = T_SMEM;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 1;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = CS;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   cudaLaunchKernelEx(&cfg, attn_tile_kernel<CS>, a);
 }
 
 template <int CS>
-static void launch_cs(const AttnArgs &a, int rows, cudaStream_t st) {
+static void launch_cs(const AttnArgs &a, int rows, cudaStream_t st, bool pdl) {
   static bool attr[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -985,23 +997,28 @@ static void launch_cs(const AttnArgs &a, int rows, cudaStream_t st) {
     cudaFuncSetAttribute(attn_mma_kernel<CS>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(AM_SMEM));
     attr[dev] = true;
   }
-  if constexpr (CS == 1) {
-    attn_mma_kernel<1><<<dim3(rows, H / AM_HG, 1), AM_THREADS, AM_SMEM, st>>>(a);
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(rows, H / AM_HG, CS);
-    cfg.blockDim = dim3(AM_THREADS);
-    cfg.dynamicSmemBytes = AM_SMEM;
-    cfg.stream = st;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = 1;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = CS;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, attn_mma_kernel<CS>, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows, H / AM_HG, CS);
+  cfg.blockDim = dim3(AM_THREADS);
+  cfg.dynamicSmemBytes = AM_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  int n = 0;
+  if (CS > 1) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = 1;
+    at[n].val.clusterDim.y = 1;
+    at[n].val.clusterDim.z = CS;
+    ++n;
   }
+  if (pdl) {
+    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  cudaLaunchKernelEx(&cfg, attn_mma_kernel<CS>, a);
 }
 
 // Clusters of CS attention CTAs the device can hold at once (0: none), per device.
@@ -1042,7 +1059,7 @@ int attn_dense_segment() { return attn_clusters_fit<16>() > 0 ? 8192 : 4096; }
 void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
                      bool dense, int e0, int e1, int n_bound, const csa2_cache *c, const uint8_t *codes,
                      const float *scale, int R, int window, float *o, float *lse, int32_t *err, cudaStream_t st,
-                     const uint16_t *swa_new) {
+                     const uint16_t *swa_new, bool pdl) {
   const int rows = B * Q;
   if (rows == 0) return;
   AttnArgs a{};
@@ -1058,23 +1075,23 @@ void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, floa
   if (cs == 5 && rows * (H / AM_HG) * 5 > sm_count()) cs = 2;  // one wave of two-CTA clusters beats several of five
   if (cs > 1 && cs == tiles) {  // one tile per CTA: the single-dequant form
     switch (cs) {
-      case 2: launch_tile<2>(a, rows, st); return;
-      case 3: launch_tile<3>(a, rows, st); return;
-      case 4: launch_tile<4>(a, rows, st); return;
-      default: launch_tile<5>(a, rows, st); return;
+      case 2: launch_tile<2>(a, rows, st, pdl); return;
+      case 3: launch_tile<3>(a, rows, st, pdl); return;
+      case 4: launch_tile<4>(a, rows, st, pdl); return;
+      default: launch_tile<5>(a, rows, st, pdl); return;
     }
   }
   cs = max(cs, (tiles + 4) / 5);
   if (cs > 5) cs = cs <= 8 ? 8 : (cs <= 12 ? 12 : 16);
   switch (cs) {
-    case 2: launch_cs<2>(a, rows, st); break;
-    case 3: launch_cs<3>(a, rows, st); break;
-    case 4: launch_cs<4>(a, rows, st); break;
-    case 5: launch_cs<5>(a, rows, st); break;
-    case 8: launch_cs<8>(a, rows, st); break;
-    case 12: launch_cs<12>(a, rows, st); break;
-    case 16: launch_cs<16>(a, rows, st); break;
-    default: launch_cs<1>(a, rows, st); break;
+    case 2: launch_cs<2>(a, rows, st, pdl); break;
+    case 3: launch_cs<3>(a, rows, st, pdl); break;
+    case 4: launch_cs<4>(a, rows, st, pdl); break;
+    case 5: launch_cs<5>(a, rows, st, pdl); break;
+    case 8: launch_cs<8>(a, rows, st, pdl); break;
+    case 12: launch_cs<12>(a, rows, st, pdl); break;
+    case 16: launch_cs<16>(a, rows, st, pdl); break;
+    default: launch_cs<1>(a, rows, st, pdl); break;
   }
 }
 

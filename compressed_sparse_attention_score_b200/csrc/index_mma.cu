@@ -237,6 +237,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
   float *ws = reinterpret_cast<float *>(smem + SM_W);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  grid_dep_launch();  // a dependent attention launch may start its prologue
   const int row = blockIdx.y, b = row / a.Q;
   const int nvis = visible_entries(a.c, b, a.q_pos[row]);
   const int n_entries = a.c.num_entries[b];

@@ -66,10 +66,12 @@ void launch_topk_cluster(const float *scores, const int32_t *n_valid, int R, int
                          int k1, int32_t *idx1, float *val1, const int32_t *map, cudaStream_t st);
 // swa_new [B*Q][512] bf16 (decode): each row's own window token, quantised inside the launch,
 // used as the window's last key and stored in the ring (codes / scale must then be writable).
+// pdl: launched as a programmatic dependent of the kernel before it in the stream (only when that
+// kernel belongs to the same library call, so everything else it reads was written before).
 void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
                      bool dense, int e0, int e1, int n_bound, const csa2_cache *c, const uint8_t *codes,
                      const float *scale, int R, int window, float *o, float *lse, int32_t *err, cudaStream_t st,
-                     const uint16_t *swa_new = nullptr);
+                     const uint16_t *swa_new = nullptr, bool pdl = false);
 // Entries per dense-attention launch (one cluster of at most 16 CTAs x 640 keys per row).
 int attn_dense_segment();
 void launch_merge(const float *o1, const float *l1, const float *o2, const float *l2, int64_t rows, int D_,

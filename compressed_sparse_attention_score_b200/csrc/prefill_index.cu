@@ -206,6 +206,7 @@ __global__ void __launch_bounds__(PF_THREADS, 2) prefill_index_kernel(const __gr
   float *ws = reinterpret_cast<float *>(smem + PS_W);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  grid_dep_launch();  // a dependent attention launch may start its prologue
   const int b = blockIdx.y, q0 = blockIdx.x * PF_Q;
   const int nq = min(PF_Q, a.Q - q0);  // query tokens of this CTA
   int nvis_max = 0;

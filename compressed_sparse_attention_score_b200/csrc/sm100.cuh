@@ -245,6 +245,14 @@ __device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[1
       : "r"(taddr));
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization may
+// start while the kernel before it in the stream is still running: grid_dep_wait() returns once
+// that kernel has completed and its memory is visible (a kernel reads nothing the previous one may
+// write before it).  grid_dep_launch() lets such a follower start once every CTA of this kernel has
+// called it (without the call it starts when this kernel exits).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // c0 += a0 * b0 and c1 += a1 * b1, each one fp32 fused multiply-add rounded to nearest (the
 // packed form of two fmaf, bit for bit).
 __device__ __forceinline__ void fma2(float &c0, float &c1, float a0, float a1, float b0, float b1) {

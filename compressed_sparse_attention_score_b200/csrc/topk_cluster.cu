@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -57,6 +58,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
                                                                      const int32_t *__restrict__ map) {
   constexpr int U = 8;        // scalar loads in flight per lane
   constexpr int SAMPLE = 16;  // one group of 32 keys in SAMPLE is sampled
+  sm100::grid_dep_launch();  // a dependent attention launch may start its prologue
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint32_t tk_smem[];
   uint32_t(*ckey)[TK_CAPW] = reinterpret_cast<uint32_t(*)[TK_CAPW]>(tk_smem);        // [32][cap]
