@@ -44,7 +44,8 @@ using namespace sm100;
 namespace {
 constexpr int AM_PRODUCERS = 256;               // warps 0-7 dequantise keys
 constexpr int AM_THREADS = AM_PRODUCERS + 32;   // warp 8 drives the tensor core
-constexpr int AM_HG = 32;          // heads per CTA = MMA N
+constexpr int AM_HG = 32;          // heads per CTA of the one-tile kernel = MMA N
+constexpr int RG = 64;             // heads per CTA of the general kernel (every head of a row)
 constexpr int AM_TILE = 128;       // keys per S^T tile
 constexpr int AM_MAXKEYS = 640;    // 512 listed entries + 128 window tokens
 constexpr int AM_BLOCKS = 8;       // 64-dim blocks of a key tile = operand buffers (one tile)
@@ -52,22 +53,30 @@ constexpr int AM_STAGE = 16384;    // one block: 128 keys x 64 dims fp16
 constexpr uint32_t AM_TMEM_COLS = 256;
 constexpr uint64_t AM_WAIT_NS = 2000000000ull;
 
-constexpr int SM_Q = 0;                              // 8 chunks x [32 heads x 128 B]
-constexpr int SM_P = SM_Q + 8 * 4096;                // P^T [640 keys x 64 B]
-constexpr int SM_STG = SM_P + AM_MAXKEYS * 64;       // one key tile: 8 x 16 KB blocks
+constexpr int AM_MAXCS = 16;      // largest cluster splitting one row's keys
+constexpr int AM_QU = AM_HG * (D / 8) / AM_PRODUCERS;   // 16-byte query chunks per producer thread
+template <int HG>
+__host__ __device__ constexpr int qu_of() { return HG * (D / 8) / AM_PRODUCERS; }
+constexpr uint32_t RG_TMEM_COLS = 512;  // S^T of 5 tiles x 64 heads; O^T (4 x 64) reuses those columns
+// General kernel (RG heads): Q during the first phase, P^T (written after every S^T product has
+// completed) in the same bytes afterwards.
+constexpr int SM_QP_BYTES = (8 * RG * 128 > AM_MAXKEYS * RG * 2) ? 8 * RG * 128 : AM_MAXKEYS * RG * 2;
+constexpr int SM_Q = 0;                              // 8 chunks x [RG heads x 128 B]
+constexpr int SM_P = 0;                              // P^T [640 keys x RG x 2 B], 128-byte swizzle
+constexpr int SM_STG = SM_QP_BYTES;                  // one key tile: 8 x 16 KB blocks
 constexpr int SM_SLOT = SM_STG + AM_BLOCKS * AM_STAGE;
 constexpr int SM_MU = SM_SLOT + AM_MAXKEYS * 8;      // logit multiplier per key
 constexpr int SM_PV = SM_MU + AM_MAXKEYS * 4;        // P multiplier per key
-constexpr int AM_MAXCS = 16;      // largest cluster splitting one row's keys
-constexpr int AM_QU = AM_HG * (D / 8) / AM_PRODUCERS;   // 16-byte query chunks per producer thread
-constexpr int SM_RED = SM_PV + AM_MAXKEYS * 4;       // [4 warps][32 heads]; [CS][32] weights + [32] sums
-constexpr int SM_HM = SM_RED + (AM_MAXCS + 1) * 32 * 4;   // head max [32], head sum [32]
-constexpr int SM_QS = SM_HM + 2 * 32 * 4;            // query prescale: [8 warps][AM_QU] max bits, [32] 2^-s
-constexpr int SM_NEW = SM_QS + (8 * AM_QU + 32) * 4; // this step's window token: 512 codes, scale, [4] maxima
+constexpr int SM_RED = SM_PV + AM_MAXKEYS * 4;       // [8 warps][32 heads]; [CS][RG] weights + [RG] sums
+constexpr int SM_HM = SM_RED + (AM_MAXCS + 1) * RG * 4;   // head max [RG], head sum [RG]
+constexpr int SM_QS = SM_HM + 2 * RG * 4;            // query prescale: [8 warps][QU] max bits, [RG] 2^-s
+constexpr int SM_NEW = SM_QS + (8 * qu_of<RG>() + RG) * 4;  // this step's window token: 512 codes, scale, [4] maxima
 constexpr int SM_BAR = SM_NEW + 512 + 32;
 constexpr int SM_MISC = SM_BAR + 8 * (2 * AM_BLOCKS + 1);
 constexpr int SM_TOTAL = SM_MISC + 16;
 constexpr size_t AM_SMEM = SM_TOTAL + 1024;
+static_assert(AM_SMEM <= 227 * 1024, "general attention kernel exceeds the shared memory of a CTA");
+static_assert(SM_STG % 1024 == 0, "operand buffers need 1 KB alignment");
 }  // namespace
 
 struct AttnArgs {
@@ -109,16 +118,18 @@ __device__ __forceinline__ int mnmaj64(int k, int u) { return (k >> 3) * 512 + (
 // Producer thread tid holds query chunks it = tid + 256 u, i.e. head tid / 64 + 4 u, so the
 // two warps 2c, 2c + 1 share the heads c + 4 u.  Each warp publishes the largest |bf16| bit
 // pattern of each of its AM_QU chunks' heads (|x| orders like its bits).
-__device__ __forceinline__ void publish_query_max(const uint4 (&qraw)[AM_QU], uint32_t *qmx) {
+template <int HG = AM_HG>
+__device__ __forceinline__ void publish_query_max(const uint4 (&qraw)[qu_of<HG>()], uint32_t *qmx) {
+  constexpr int QU = qu_of<HG>();
   const int warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int u = 0; u < AM_QU; ++u) {
+  for (int u = 0; u < QU; ++u) {
     const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
     uint32_t mb = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) mb = max(mb, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
     mb = __reduce_max_sync(0xffffffffu, mb);
-    if ((threadIdx.x & 31) == 0) qmx[warp * AM_QU + u] = mb;
+    if ((threadIdx.x & 31) == 0) qmx[warp * QU + u] = mb;
   }
 }
 // Exponent s of the prescale of a head whose largest |bf16| bit pattern is mb (0 for an all-zero
@@ -128,19 +139,23 @@ __device__ __forceinline__ int query_prescale_exp(uint32_t mb) {
   if (mb == 0 || E >= 255) return 0;
   return min(126, 141 - max(E, 1));
 }
+template <int HG = AM_HG>
 __device__ __forceinline__ uint32_t head_max_bits(const uint32_t *qmx, int h) {
+  constexpr int QU = qu_of<HG>();
   const int c = h & 3, u = h >> 2;
-  return max(qmx[(2 * c) * AM_QU + u], qmx[(2 * c + 1) * AM_QU + u]);
+  return max(qmx[(2 * c) * QU + u], qmx[(2 * c + 1) * QU + u]);
 }
 // Write this producer's query chunks, prescaled, as fp16 into the K-major 128-byte-swizzled
-// Q operand (8 chunks of 64 dims x 32 heads); thread tid < 32 also stores 2^-s of head tid.
-__device__ __forceinline__ void store_query_fp16(const uint4 (&qraw)[AM_QU], const uint32_t *qmx, float *qinv,
+// Q operand (8 chunks of 64 dims x HG heads); thread tid < HG also stores 2^-s of head tid.
+template <int HG = AM_HG>
+__device__ __forceinline__ void store_query_fp16(const uint4 (&qraw)[qu_of<HG>()], const uint32_t *qmx, float *qinv,
                                                  uint8_t *qdst) {
+  constexpr int QU = qu_of<HG>();
   const int tid = threadIdx.x;
 #pragma unroll
-  for (int u = 0; u < AM_QU; ++u) {
+  for (int u = 0; u < QU; ++u) {
     const int it = tid + u * AM_PRODUCERS, h = it / (D / 8), u8 = it % (D / 8);
-    const float sc = pow2f(query_prescale_exp(head_max_bits(qmx, h)));
+    const float sc = pow2f(query_prescale_exp(head_max_bits<HG>(qmx, h)));
     const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
     uint32_t o4[4];
 #pragma unroll
@@ -148,9 +163,10 @@ __device__ __forceinline__ void store_query_fp16(const uint4 (&qraw)[AM_QU], con
       const __half2 hv = __floats2half2_rn(__uint_as_float(w[i] << 16) * sc, __uint_as_float(w[i] & 0xFFFF0000u) * sc);
       o4[i] = *reinterpret_cast<const uint32_t *>(&hv);
     }
-    *reinterpret_cast<uint4 *>(qdst + (u8 / 8) * 4096 + kmaj128(h, u8 % 8)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    *reinterpret_cast<uint4 *>(qdst + (u8 / 8) * (HG * 128) + kmaj128(h, u8 % 8)) =
+        make_uint4(o4[0], o4[1], o4[2], o4[3]);
   }
-  if (tid < 32) qinv[tid] = pow2f(-query_prescale_exp(head_max_bits(qmx, tid)));
+  if (tid < HG) qinv[tid] = pow2f(-query_prescale_exp(head_max_bits<HG>(qmx, tid)));
 }
 
 // Raw bytes of one half of a key (dims 256 half .. +255) into registers: a listed entry's
@@ -271,28 +287,30 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32]) {
 // each owner its slice of O_s and every owner its (m_s, l_s), straight from TMEM into the
 // owners' receive buffers (remote stores, nothing waits on them), then one cluster barrier, and
 // each owner combines its slice locally: o = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s,
-// M = max_s m_s.  The receive buffer (recv: CS x 32 x PER floats, then CS x 64 statistics) is
+// M = max_s m_s.  The receive buffer (recv: CS x HG x PER floats, then CS x 2 HG statistics) is
 // the CTA's key-tile memory, so a first barrier (split: arrive when this CTA's products are
 // complete, wait before the first push) keeps peers from writing into a tile still being read.
-template <int CS>
+template <int CS, int HG = AM_HG>
 __device__ __forceinline__ void combine_partials(const AttnArgs &p, uint32_t tmem, bool aborted, bool has_keys,
                                                  float *recv, float *red, float *hmax, float *hsum, int row, int hg,
                                                  int split) {
   constexpr int PER = ((D + CS - 1) / CS + 3) & ~3;  // dims per owner, a multiple of 4
+  constexpr int NWARP = HG / 8;                      // warps reading TMEM: 4 lane quarters x HG / 32 head groups
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  float *stats = recv + CS * 32 * PER;  // [source][max 32 | sum 32]
+  float *stats = recv + CS * HG * PER;  // [source][max HG | sum HG]
   cg::cluster_group cluster = cg::this_cluster();
-  if (warp < 4 && aborted) {
-    hsum[lane] = 0.f;
-    hmax[lane] = -INFINITY;
+  if (tid < HG && aborted) {
+    hsum[tid] = 0.f;
+    hmax[tid] = -INFINITY;
   }
   cluster_arrive();  // this CTA's tensor-core products are complete
   bool waited = false;
-  if (warp < 4) {
+  if (warp < NWARP) {
+    const int hb = 32 * (warp >> 2);  // this warp's 32 heads
     for (int d = 0; d < 4; ++d) {
       uint32_t r0[16], r1[16];
       if (!aborted && has_keys) {
-        const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + d * AM_HG;
+        const uint32_t ta = tmem + (uint32_t(32 * (warp & 3)) << 16) + d * HG + hb;
         tc_ld_32x32b_x16(ta, r0);
         tc_ld_32x32b_x16(ta + 16, r1);
         tc_wait_ld();
@@ -304,54 +322,54 @@ __device__ __forceinline__ void combine_partials(const AttnArgs &p, uint32_t tme
         cluster_wait();  // every peer's tile memory is free
         waited = true;
       }
-      const int dim = 128 * d + 32 * warp + lane, q = dim / PER;
-      float *dst = cluster.map_shared_rank(recv + split * 32 * PER + (dim - q * PER), q);
+      const int dim = 128 * d + 32 * (warp & 3) + lane, q = dim / PER;
+      float *dst = cluster.map_shared_rank(recv + (split * HG + hb) * PER + (dim - q * PER), q);
 #pragma unroll
       for (int h = 0; h < 16; ++h) {
         dst[h * PER] = __uint_as_float(r0[h]);
         dst[(16 + h) * PER] = __uint_as_float(r1[h]);
       }
     }
-    if (warp == 0) {
-      const float m = hmax[lane], l = hsum[lane];
+    if (tid < HG) {
+      const float m = hmax[tid], l = hsum[tid];
 #pragma unroll
       for (int q = 0; q < CS; ++q) {
-        float *st = cluster.map_shared_rank(stats + split * 64, q);
-        st[lane] = m;
-        st[32 + lane] = l;
+        float *st = cluster.map_shared_rank(stats + split * 2 * HG, q);
+        st[tid] = m;
+        st[HG + tid] = l;
       }
     }
   } else {
     cluster_wait();
   }
   cluster.sync();  // every slice and statistic has arrived; no peer's memory is touched after this
-  float *wts = red;  // [CS][32] combination weights
-  float *lsum = red + CS * 32;
-  if (tid < 32) {
+  float *wts = red;  // [CS][HG] combination weights
+  float *lsum = red + CS * HG;
+  if (tid < HG) {
     float M = -INFINITY;
 #pragma unroll
-    for (int q = 0; q < CS; ++q) M = fmaxf(M, stats[q * 64 + tid]);
+    for (int q = 0; q < CS; ++q) M = fmaxf(M, stats[q * 2 * HG + tid]);
     float L = 0.f;
 #pragma unroll
     for (int q = 0; q < CS; ++q) {
-      const float mq = stats[q * 64 + tid];
+      const float mq = stats[q * 2 * HG + tid];
       const float wq = (M == -INFINITY || mq == -INFINITY) ? 0.f : __expf(mq - M);
-      wts[q * 32 + tid] = wq;
-      L += wq * stats[q * 64 + 32 + tid];
+      wts[q * HG + tid] = wq;
+      L += wq * stats[q * 2 * HG + HG + tid];
     }
     lsum[tid] = L;
-    if (split == 0) p.lse[int64_t(row) * H + hg * AM_HG + tid] = L > 0.f ? M + logf(L) : -INFINITY;
+    if (split == 0) p.lse[int64_t(row) * H + hg * HG + tid] = L > 0.f ? M + logf(L) : -INFINITY;
   }
   __syncthreads();
   const int d0 = min(D, split * PER), nq = (min(D, d0 + PER) - d0) / 4;
-  float *orow = p.o + (int64_t(row) * H + hg * AM_HG) * D;
-  for (int it = tid; it < 32 * nq; it += AM_THREADS) {
+  float *orow = p.o + (int64_t(row) * H + hg * HG) * D;
+  for (int it = tid; it < HG * nq; it += AM_THREADS) {
     const int h = it / nq, dl = 4 * (it % nq);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int q = 0; q < CS; ++q) {
-      const float wq = wts[q * 32 + h];
-      const float4 x = *reinterpret_cast<const float4 *>(recv + (q * 32 + h) * PER + dl);
+      const float wq = wts[q * HG + h];
+      const float4 x = *reinterpret_cast<const float4 *>(recv + (q * HG + h) * PER + dl);
       acc.x += wq * x.x;
       acc.y += wq * x.y;
       acc.z += wq * x.z;
@@ -371,7 +389,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   float *pv = reinterpret_cast<float *>(smem + SM_PV);
   float *red = reinterpret_cast<float *>(smem + SM_RED);
   float *hmax = reinterpret_cast<float *>(smem + SM_HM);
-  float *hsum = hmax + 32;
+  float *hsum = hmax + RG;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM_BAR);  // block written (128 arrivals)
   uint64_t *mma_done = full + AM_BLOCKS;                          // block consumed (tcgen05.commit)
   uint64_t *phase_done = mma_done + AM_BLOCKS;                    // all products of a phase complete
@@ -384,11 +402,12 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   const int lrow = row, b = row / p.Q, ring = b;
   // The query block (an input of the call) is loaded first; everything else may be written by
   // the kernel launched just before this one, so it is read after grid_dep_wait().
-  uint4 qraw[AM_QU];
+  constexpr int QU = qu_of<RG>();
+  uint4 qraw[QU];
   if (producer) {
-    const uint16_t *qrow = p.q + (int64_t(row) * H + hg * AM_HG) * D;
+    const uint16_t *qrow = p.q + (int64_t(row) * H + hg * RG) * D;
 #pragma unroll
-    for (int u = 0; u < AM_QU; ++u) {
+    for (int u = 0; u < QU; ++u) {
       const int it = tid + u * AM_PRODUCERS;
       qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
     }
@@ -418,7 +437,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   const int key0 = tile0 * AM_TILE;  // first key of this CTA; local key j is key key0 + j
   // the query block (loaded above) is converted once the key list is done
   uint32_t *qmx = reinterpret_cast<uint32_t *>(smem + SM_QS);
-  float *qinv = reinterpret_cast<float *>(smem + SM_QS + 8 * AM_QU * 4);
+  float *qinv = reinterpret_cast<float *>(smem + SM_QS + 8 * QU * 4);
   // this step's own window token (the row's last key), quantised here and stored by one CTA
   const bool own_token = p.swa_new && nkw > 0;
   uint8_t *new_codes = own_token ? smem + SM_NEW : nullptr;
@@ -467,9 +486,9 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       pv[jl] = j < nks ? 1.f : (win ? sc[r] : 0.f);
     }
   }
-  if (producer) publish_query_max(qraw, qmx);
+  if (producer) publish_query_max<RG>(qraw, qmx);
   if (warp == AM_PRODUCERS / 32) {
-    tmem_alloc(tmem_slot, AM_TMEM_COLS);
+    tmem_alloc(tmem_slot, RG_TMEM_COLS);
     tmem_relinquish();
   }
   if (issuer) {
@@ -491,7 +510,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
     const bool own = own_token && key0 + jl == nk - 1;
     load_key_half(p, slot[jl], key0 + jl < nks, own ? new_codes : nullptr, half, cur);
   };
-  if (producer) store_query_fp16(qraw, qmx, qinv, smem + SM_Q);
+  if (producer) store_query_fp16<RG>(qraw, qmx, qinv, smem + SM_Q);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -529,17 +548,17 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   if (producer) {
     aborted = !produce_all(0);
   } else if (issuer) {
-    constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, false, false);
+    constexpr uint32_t id = idesc_f16(AM_TILE, RG, false, false);
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) {
       for (int i = 0; i < AM_BLOCKS; ++i) {
         const int blk = (i & 1) * 4 + (i >> 1);
         if (!(ok = mbar_wait_bounded(&full[blk], t & 1, abort_flag, AM_WAIT_NS))) break;
         tc_fence_after();
-        const uint32_t a0 = stg + blk * AM_STAGE, b0 = smem_u32(smem + SM_Q + blk * 4096);
+        const uint32_t a0 = stg + blk * AM_STAGE, b0 = smem_u32(smem + SM_Q + blk * (RG * 128));
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4)
-          tc_mma_f16(tmem + t * AM_HG, smem_desc(a0 + 32 * k4, 16, 1024, LAYOUT_SWIZZLE_128B),
+          tc_mma_f16(tmem + t * RG, smem_desc(a0 + 32 * k4, 16, 1024, LAYOUT_SWIZZLE_128B),
                      smem_desc(b0 + 32 * k4, 16, 1024, LAYOUT_SWIZZLE_128B), id, i > 0 || k4 > 0);
         tc_commit(&mma_done[blk]);
       }
@@ -553,14 +572,17 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   tc_fence_after();
 
   // ---------------------------------------------------------------- phase 2: softmax over all keys
-  if (!aborted && warp < 4) {
+  // The 8 producer warps: warp w reads keys 32 (w % 4) .. + 31 of every tile (its TMEM lanes) for
+  // heads 32 (w / 4) .. + 31; the four warps of each head half reduce through shared memory.
+  if (!aborted && warp < 8) {
+    const int q4 = warp & 3, hb = 32 * (warp >> 2);
     float mx[32];
 #pragma unroll
     for (int h = 0; h < 32; ++h) mx[h] = -INFINITY;
     for (int t = 0; t < ntiles; ++t) {
-      const int key = t * AM_TILE + 32 * warp + lane;
+      const int key = t * AM_TILE + 32 * q4 + lane;
       uint32_t r0[16], r1[16];
-      const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + t * AM_HG;
+      const uint32_t ta = tmem + (uint32_t(32 * q4) << 16) + t * RG + hb;
       tc_ld_32x32b_x16(ta, r0);
       tc_ld_32x32b_x16(ta + 16, r1);
       tc_wait_ld();
@@ -574,18 +596,20 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       }
     }
     red[warp * 32 + lane] = reduce_scatter32<true>(mx);
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (warp == 0)  // the maxima of the prescaled logits, scaled back by 2^-s (exact)
-      hmax[lane] = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane])) * qinv[lane];
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (q4 == 0) {  // the maxima of the prescaled logits, scaled back by 2^-s (exact)
+      const float *rg = red + warp * 32;
+      hmax[hb + lane] = fmaxf(fmaxf(rg[lane], rg[32 + lane]), fmaxf(rg[64 + lane], rg[96 + lane])) * qinv[hb + lane];
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
     float sm[32];  // the head maxima are read from shared memory (a broadcast) as needed
 #pragma unroll
     for (int h = 0; h < 32; ++h) sm[h] = 0.f;
-    const float *m_h = hmax;
+    const float *m_h = hmax + hb, *qi = qinv + hb;
     for (int t = 0; t < ntiles; ++t) {
-      const int key = t * AM_TILE + 32 * warp + lane;
+      const int key = t * AM_TILE + 32 * q4 + lane;
       uint32_t r0[16], r1[16];
-      const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + t * AM_HG;
+      const uint32_t ta = tmem + (uint32_t(32 * q4) << 16) + t * RG + hb;
       tc_ld_32x32b_x16(ta, r0);
       tc_ld_32x32b_x16(ta + 16, r1);
       tc_wait_ld();
@@ -594,8 +618,8 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       uint32_t ph[16];
 #pragma unroll
       for (int h = 0; h < 32; h += 2) {
-        const float x0 = (m * __uint_as_float(h < 16 ? r0[h] : r1[h - 16])) * qinv[h];
-        const float x1 = (m * __uint_as_float(h + 1 < 16 ? r0[h + 1] : r1[h - 15])) * qinv[h + 1];
+        const float x0 = (m * __uint_as_float(h < 16 ? r0[h] : r1[h - 16])) * qi[h];
+        const float x1 = (m * __uint_as_float(h + 1 < 16 ? r0[h + 1] : r1[h - 15])) * qi[h + 1];
         const float e0 = (valid && m_h[h] != -INFINITY) ? __expf(x0 - m_h[h]) : 0.f;
         const float e1 = (valid && m_h[h + 1] != -INFINITY) ? __expf(x1 - m_h[h + 1]) : 0.f;
         sm[h] += e0;
@@ -603,14 +627,18 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
         const __half2 hp = __floats2half2_rn(e0 * pm, e1 * pm);
         ph[h >> 1] = *reinterpret_cast<const uint32_t *>(&hp);
       }
+      // P^T row of this key: RG heads x 2 B = 128 B, 128-byte swizzle (MN-major B operand)
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        *reinterpret_cast<uint4 *>(smem + SM_P + mnmaj64(key, u)) =
+        *reinterpret_cast<uint4 *>(smem + SM_P + kmaj128(key, hb / 8 + u)) =
             make_uint4(ph[4 * u], ph[4 * u + 1], ph[4 * u + 2], ph[4 * u + 3]);
     }
     red[warp * 32 + lane] = reduce_scatter32<false>(sm);
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (warp == 0) hsum[lane] = (red[lane] + red[32 + lane]) + (red[64 + lane] + red[96 + lane]);
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (q4 == 0) {
+      const float *rg = red + warp * 32;
+      hsum[hb + lane] = (rg[lane] + rg[32 + lane]) + (rg[64 + lane] + rg[96 + lane]);
+    }
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -625,7 +653,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   if (!aborted && producer) {
     if (ntiles > 1) aborted = !produce_all(ntiles);
   } else if (!aborted && issuer) {
-    constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, true, true);
+    constexpr uint32_t id = idesc_f16(AM_TILE, RG, true, true);
     const uint32_t pt = smem_u32(smem + SM_P);
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) {
@@ -641,9 +669,9 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
         for (int jc = 0; jc < 2; ++jc)
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4)
-            tc_mma_f16(tmem + d * AM_HG,
+            tc_mma_f16(tmem + d * RG,
                        smem_desc(stg + (2 * d) * AM_STAGE + jc * 8192 + 2048 * k4, 16384, 1024, LAYOUT_SWIZZLE_128B),
-                       smem_desc(pt + (8 * (2 * t + jc) + 2 * k4) * 512, 16, 512, LAYOUT_SWIZZLE_64B), id,
+                       smem_desc(pt + (8 * (2 * t + jc) + 2 * k4) * 1024, 16, 1024, LAYOUT_SWIZZLE_128B), id,
                        t > 0 || jc > 0 || k4 > 0);
         tc_commit(&mma_done[2 * d]);
         tc_commit(&mma_done[2 * d + 1]);
@@ -659,18 +687,19 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
 
   // ---------------------------------------------------------------- phase 4: normalise and store
   if constexpr (CS == 1) {
-    if (warp < 4) {
+    if (warp < 8) {  // warp w: dims 32 (w % 4) + .. of each 128-dim block, heads 32 (w / 4) .. + 31
+      const int q4 = warp & 3, hb = 32 * (warp >> 2);
       float inv[32];
 #pragma unroll
       for (int h = 0; h < 32; ++h) {
-        const float s = aborted ? 0.f : hsum[h];
+        const float s = aborted ? 0.f : hsum[hb + h];
         inv[h] = s > 0.f ? 1.f / s : 0.f;
       }
-      float *orow = p.o + (int64_t(row) * H + hg * AM_HG) * D;
+      float *orow = p.o + (int64_t(row) * H + hg * RG + hb) * D;
       for (int d = 0; d < 4; ++d) {
         uint32_t r0[16], r1[16];
         if (!aborted && nkc > 0) {
-          const uint32_t ta = tmem + (uint32_t(32 * warp) << 16) + d * AM_HG;
+          const uint32_t ta = tmem + (uint32_t(32 * q4) << 16) + d * RG + hb;
           tc_ld_32x32b_x16(ta, r0);
           tc_ld_32x32b_x16(ta + 16, r1);
           tc_wait_ld();
@@ -678,28 +707,28 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) r0[i] = r1[i] = 0u;
         }
-        const int dim = 128 * d + 32 * warp + lane;
+        const int dim = 128 * d + 32 * q4 + lane;
 #pragma unroll
         for (int h = 0; h < 16; ++h) {
           orow[h * D + dim] = __uint_as_float(r0[h]) * inv[h];
           orow[(16 + h) * D + dim] = __uint_as_float(r1[h]) * inv[16 + h];
         }
       }
-      if (warp == 0) {
-        const float s = aborted ? 0.f : hsum[lane];
-        p.lse[int64_t(row) * H + hg * AM_HG + lane] = s > 0.f ? hmax[lane] + logf(s) : -INFINITY;
+      if (q4 == 0) {
+        const float s = aborted ? 0.f : hsum[hb + lane];
+        p.lse[int64_t(row) * H + hg * RG + hb + lane] = s > 0.f ? hmax[hb + lane] + logf(s) : -INFINITY;
       }
     }
   } else {
-    combine_partials<CS>(p, tmem, aborted, nkc > 0, reinterpret_cast<float *>(smem + SM_P), red, hmax, hsum, row, hg,
-                         split);
+    combine_partials<CS, RG>(p, tmem, aborted, nkc > 0, reinterpret_cast<float *>(smem + SM_P), red, hmax, hsum, row,
+                             hg, split);
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == AM_PRODUCERS / 32) {
     tc_fence_after();
-    tmem_dealloc(tmem, AM_TMEM_COLS);
+    tmem_dealloc(tmem, RG_TMEM_COLS);
   }
   if (tid == 0 && aborted) report(p.err, CSA2_ERR_TIMEOUT);
 }
@@ -998,7 +1027,7 @@ static void launch_cs(const AttnArgs &a, int rows, cudaStream_t st, bool pdl) {
     attr[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(rows, H / AM_HG, CS);
+  cfg.gridDim = dim3(rows, H / RG, CS);
   cfg.blockDim = dim3(AM_THREADS);
   cfg.dynamicSmemBytes = AM_SMEM;
   cfg.stream = st;
