@@ -1080,10 +1080,11 @@ static int attn_clusters_fit() {
 
 int attn_dense_segment() { return attn_clusters_fit<16>() > 0 ? 8192 : 4096; }
 
-// Up to 64 query rows: a cluster of CTAs (one per 128-key tile) splits each row's keys and
-// combines the partials through distributed shared memory; when those one-tile CTAs would need
-// more than one wave, clusters of two CTAs of two or three tiles each (measured on 32 rows of 640
-// keys: 47 us against 53 us for five-CTA clusters and 68 us for three).  A CTA holds at most 5
+// Up to 64 query rows: a cluster of CTAs (one per 128-key tile, 32 heads each) splits each row's
+// keys and combines the partials through distributed shared memory; when those one-tile CTAs would
+// need more than one wave, the 64-head general kernel in clusters of three CTAs of one or two
+// tiles (measured on 32 rows of 640 keys: 44 us, against 51 us for two-CTA clusters, 55 us for
+// five and 53 us for the one-tile kernel).  A CTA holds at most 5
 // tiles (640 keys), so longer key sets (dense segments) always use clusters of up to 16 CTAs.
 void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, float tau, const int32_t *idx, int k,
                      bool dense, int e0, int e1, int n_bound, const csa2_cache *c, const uint8_t *codes,
@@ -1101,8 +1102,10 @@ void launch_attn_mma(const uint16_t *q, int B, int Q, const int32_t *q_pos, floa
   const int nkeys = (dense ? max(0, e1 - e0) : a.k) + (codes ? window : 0);
   const int tiles = (nkeys + AM_TILE - 1) / AM_TILE;
   int cs = rows * (H / AM_HG) <= 128 ? max(1, min(tiles, 5)) : 1;
-  if (cs == 5 && rows * (H / AM_HG) * 5 > sm_count()) cs = 2;  // one wave of two-CTA clusters beats several of five
-  if (cs > 1 && cs == tiles) {  // one tile per CTA: the single-dequant form
+  // one-tile CTAs of 32 heads that would need several waves: the 64-head kernel in 3-CTA clusters
+  const bool many = cs == 5 && rows * (H / AM_HG) * 5 > sm_count();
+  if (many) cs = 3;
+  if (!many && cs > 1 && cs == tiles) {  // one tile per CTA: the single-dequant form
     switch (cs) {
       case 2: launch_tile<2>(a, rows, st, pdl); return;
       case 3: launch_tile<3>(a, rows, st, pdl); return;
