@@ -944,8 +944,8 @@ def main():
               "unit": "GB/s", "frac": gather_gbs / peak, "launch_us": gather_ms * 1e3,
               "timing": "isolated launches, L2 flushed before each"}
     achieved = wl.scan_bytes() / (scan_ms * 1e-3) / 1e9
-    traffic = profiled_traffic(["compressed_sparse_attention_score_b200/csrc/index_mma.cu"],
-                               "index_score_hier1m.md")
+    traffic = profiled_traffic(["compressed_sparse_attention_score_b200/csrc/" + f
+                                for f in ("index_mma.cu", "sm100.cuh", "common.cuh")], "index_score_hier1m.md")
     # context for the scan's fraction: a plain read-only stream over as many bytes (torch's sum
     # reduction over the same 570 MB), timed the same way (L2 flushed, CUDA events)
     stream_buf = torch.empty(wl.scan_bytes() // 4, dtype=torch.float32, device=dev).fill_(1.0)
