@@ -230,13 +230,18 @@ __device__ __forceinline__ void dequant_block(const uint4 (&rr)[16], bool sparse
 // (shared), its scale to *new_scale (shared); the CTA given `store` also writes both to the ring
 // slot of position pos, which no CTA of this launch reads (window slots are distinct mod R).
 // Called by every thread of the CTA; contains two __syncthreads.
-__device__ __forceinline__ void quantise_new_token(const AttnArgs &p, int row, int ring, int pos, bool store,
+// The token's bf16 values 4 tid .. 4 tid + 3 (threads < 128), loaded at the start of the launch.
+__device__ __forceinline__ uint2 load_new_token(const AttnArgs &p, int row) {
+  return (p.swa_new && threadIdx.x < 128)
+             ? *reinterpret_cast<const uint2 *>(p.swa_new + int64_t(row) * CSA2_SWA_DIM + 4 * threadIdx.x)
+             : make_uint2(0u, 0u);
+}
+__device__ __forceinline__ void quantise_new_token(const AttnArgs &p, uint2 u, int ring, int pos, bool store,
                                                    uint8_t *new_codes, float *new_scale, float *red) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   float v[4] = {0.f, 0.f, 0.f, 0.f};
   float am = 0.f;
   if (tid < 128) {
-    const uint2 u = *reinterpret_cast<const uint2 *>(p.swa_new + int64_t(row) * CSA2_SWA_DIM + 4 * tid);
     v[0] = __uint_as_float(u.x << 16), v[1] = __uint_as_float(u.x & 0xFFFF0000u);
     v[2] = __uint_as_float(u.y << 16), v[3] = __uint_as_float(u.y & 0xFFFF0000u);
     am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
@@ -295,7 +300,8 @@ __device__ __forceinline__ void combine_partials(const AttnArgs &p, uint32_t tme
                                                  float *recv, float *red, float *hmax, float *hsum, int row, int hg,
                                                  int split) {
   constexpr int PER = ((D + CS - 1) / CS + 3) & ~3;  // dims per owner, a multiple of 4
-  constexpr int NWARP = HG / 8;                      // warps reading TMEM: 4 lane quarters x HG / 32 head groups
+  constexpr int NWARP = 8;                           // warps reading TMEM: 4 lane quarters x 2
+  constexpr int DPW = HG / 16;                       // (head group, 128-dim block) pairs per warp
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float *stats = recv + CS * HG * PER;  // [source][max HG | sum HG]
   cg::cluster_group cluster = cg::this_cluster();
@@ -305,9 +311,10 @@ __device__ __forceinline__ void combine_partials(const AttnArgs &p, uint32_t tme
   }
   cluster_arrive();  // this CTA's tensor-core products are complete
   bool waited = false;
+  static_assert(HG % 32 == 0 && 2 * DPW == 4 * (HG / 32), "the 8 warps share the (head group, block) pairs");
   if (warp < NWARP) {
-    const int hb = 32 * (warp >> 2);  // this warp's 32 heads
-    for (int d = 0; d < 4; ++d) {
+    for (int u = 0; u < DPW; ++u) {
+      const int pi = (warp >> 2) * DPW + u, hb = 32 * (pi >> 2), d = pi & 3;  // 32 heads x 128 dims
       uint32_t r0[16], r1[16];
       if (!aborted && has_keys) {
         const uint32_t ta = tmem + (uint32_t(32 * (warp & 3)) << 16) + d * HG + hb;
@@ -412,6 +419,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
       qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
     }
   }
+  const uint2 tok = load_new_token(p, row);  // this step's window token (an input too)
   grid_dep_launch();
   grid_dep_wait();
   const int pos = p.q_pos[row];
@@ -442,7 +450,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_mma_kernel(AttnArgs p) {
   const bool own_token = p.swa_new && nkw > 0;
   uint8_t *new_codes = own_token ? smem + SM_NEW : nullptr;
   float *new_scale = reinterpret_cast<float *>(smem + SM_NEW + 512);
-  if (own_token) quantise_new_token(p, row, ring, pos, split == 0 && hg == 0, smem + SM_NEW, new_scale, new_scale + 4);
+  if (own_token) quantise_new_token(p, tok, ring, pos, split == 0 && hg == 0, smem + SM_NEW, new_scale, new_scale + 4);
   // The list's index loads go out together (at most three keys per thread), then the slots,
   // then the window tokens' scales.
   constexpr int KPT = (AM_MAXKEYS + AM_THREADS - 1) / AM_THREADS;
@@ -787,8 +795,13 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
       qraw[u] = *reinterpret_cast<const uint4 *>(qrow + (it / (D / 8)) * D + (it % (D / 8)) * 8);
     }
   }
+  const uint2 tok = load_new_token(p, row);  // this step's window token (an input too)
   grid_dep_launch();
   grid_dep_wait();
+  // this thread's listed entry is fetched together with the row's position (not after it)
+  const int key_in = tid & (AM_TILE - 1), half = (tid >> 7) & 1;
+  const int j = split * AM_TILE + key_in;
+  const int n_listed = (producer && p.idx && !p.dense && j < p.k) ? p.idx[int64_t(lrow) * p.k + j] : -1;
   const int pos = p.q_pos[row];
   const int nvis = (p.idx || p.dense) ? visible_entries(p.c, b, pos) : 0;
   const int nks = p.dense ? max(0, min(p.e1, nvis) - p.e0) : (p.idx ? p.k : 0);
@@ -798,7 +811,6 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
     nkw = pos - lo + 1;
   }
   const int nk = nks + nkw;
-  const int key0 = split * AM_TILE;
   if (tid == 0 && p.dense && nvis > p.n_bound) report(p.err, CSA2_ERR_SHAPE);
   uint32_t *qmx = reinterpret_cast<uint32_t *>(smem + T_QS);
   float *qinv = reinterpret_cast<float *>(smem + T_QS + 8 * AM_QU * 4);
@@ -812,15 +824,13 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   // out first, then the key's index, then its raw bytes, all before any barrier; this step's
   // own window token is quantised while they are in flight, and its key loaded after that.
   uint4 rr[16];  // listed entry: rr[0..7] = 128 code bytes, rr[8] = 16 scale bytes; window: 256 codes
-  const int key_in = tid & (AM_TILE - 1), half = (tid >> 7) & 1;
-  const int j = key0 + key_in;
   bool sparse = false;
   int64_t s = -1;
   if (producer) {
     float m = 0.f, pm = 0.f;
     if (j < nks) {
       sparse = true;
-      const int n = p.dense ? p.e0 + j : p.idx[int64_t(lrow) * p.k + j];
+      const int n = p.dense ? p.e0 + j : n_listed;
       if (n != -1) {
         if (n < -1 || n >= nvis) {
           if (half == 0) report(p.err, CSA2_ERR_INDEX);
@@ -846,8 +856,10 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
     }
     publish_query_max(qraw, qmx);  // after the key loads are out
   }
-  if (own_token) {
-    quantise_new_token(p, row, ring, pos, split == 0 && hg == 0, smem + T_NEW, new_scale, new_scale + 4);
+  // Only the CTAs holding this step's own token (the row's last key) quantise it; the first
+  // head group's stores it in the ring.
+  if (own_token && split == (nk - 1) / AM_TILE) {
+    quantise_new_token(p, tok, ring, pos, hg == 0, smem + T_NEW, new_scale, new_scale + 4);
     if (producer && j == nk - 1) {
       const float sc = *new_scale;
       load_key_half(p, s, false, new_codes, half, rr);
@@ -857,6 +869,12 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
       }
     }
   }
+  // Each key half is dequantised into the tile as soon as its bytes are in, before the
+  // prologue barrier (the tile is not otherwise used yet); its blocks are published to the
+  // issuer after the barrier.
+  if (producer)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) dequant_block(rr, sparse, s >= 0, c, key_in, smem + T_KT + (4 * half + c) * 16384);
   if (warp == AM_PRODUCERS / 32) {
     tmem_alloc(tmem_slot, AM_TMEM_COLS);
     tmem_relinquish();
@@ -877,17 +895,10 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   // ---------------------------------------------------------------- phase 1: S^T = K Q^T
   if (producer) {
     store_query_fp16(qraw, qmx, qinv, smem + T_Q);
-    fence_proxy_async_smem();
+    fence_proxy_async_smem();  // the query and this thread's key blocks, written before
     mbar_arrive(qfull);
-    // this thread's four 64-dim blocks of its key, each published as soon as it is written
-    const bool valid = s >= 0;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int blk = 4 * half + c;
-      dequant_block(rr, sparse, valid, c, key_in, smem + T_KT + blk * 16384);
-      fence_proxy_async_smem();
-      mbar_arrive(&full[blk]);
-    }
+    for (int c = 0; c < 4; ++c) mbar_arrive(&full[4 * half + c]);
   } else if (issuer) {
     constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, false, false);
     bool ok = mbar_wait_bounded(qfull, 0, abort_flag, AM_WAIT_NS);

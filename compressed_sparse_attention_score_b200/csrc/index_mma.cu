@@ -254,6 +254,54 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
   // on a global load of an index.
   int32_t *cand_s = reinterpret_cast<int32_t *>(smem + SM_CAND);
   const bool cand_staged = a.cand && ntiles <= IM_CAND_TILES;
+  // Gathered tiles that all fit the ring at once are issued by the epilogue warps, one tile
+  // each, right after the prologue (they are idle until the first product anyway); otherwise
+  // warp 0 issues every tile in turn.
+  static_assert(IM_CAND_TILES <= IM_STAGES && IM_CAND_TILES <= 4 * IM_EPI_WG, "a staged list is one tile per epilogue warp");
+  const bool spread = !a.use_tma && cand_staged;
+  const uint32_t stages = smem_u32(smem + SM_STAGES);
+
+  // Gather path: lane l resolves the slots of tile entries l, l+32, l+64, l+96, the slots
+  // are shuffled to the lanes that copy each 16-byte chunk, and each lane's copies arrive on
+  // the stage's barrier by themselves (cp.async.mbarrier.arrive.noinc).
+  auto load_cand = [&](int tile, int32_t (&cv)[4]) {  // entry index of each position (-1: none)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int pos = tile * IM_TILE + lane + 32 * j;
+      if (tile >= t0 + ntiles) cv[j] = -1;
+      else if (!a.cand) cv[j] = pos;
+      else if (cand_staged) cv[j] = cand_s[pos - t0 * IM_TILE];
+      else cv[j] = pos < a.P ? a.cand[int64_t(row) * a.P + pos] : -1;
+    }
+  };
+  auto resolve = [&](const int32_t (&cv)[4], int64_t (&sl)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = cv[j];
+      if (a.cand && (n < -1 || n >= n_entries)) report(a.err, CSA2_ERR_INDEX);
+      int64_t sv = -1;
+      if (n >= 0 && n < nvis) {
+        sv = cache_slot(a.c, b, n);
+        if (sv < 0) report(a.err, CSA2_ERR_INDEX);
+      }
+      sl[j] = sv;
+    }
+  };
+  auto issue_tile = [&](int s, const int64_t (&cur)[4]) {  // the whole warp
+    const uint32_t st = stages + s * IM_STAGE_BYTES;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {  // 512 chunks of 16 bytes: chunk qd = lane + 32 j
+      const int qd = lane + 32 * j, e = qd >> 2, c = qd & 3, m = row_of_entry(e);
+      // entry e = 8 j + lane / 4 lives in lane e % 32, register j / 4
+      const int64_t slot = __shfl_sync(0xffffffffu, cur[j >> 2], e & 31);
+      if (slot >= 0)
+        cp_async_16(st + m * 64 + ((c ^ ((m >> 1) & 3)) << 4), a.c.ix_codes + slot * CSA2_IX_CODE_BYTES + c * 16);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)  // scale word of entry e = lane + 32 j at atom word e
+      if (cur[j] >= 0) cp_async_4(st + IM_A_BYTES + (lane + 32 * j) * 4, a.c.ix_scales + cur[j] * CSA2_IX_SCALE_BYTES);
+    cp_async_arrive_noinc(&full[s]);
+  };
 
   // ---------------------------------------------------------------- prologue
   if (warp == 0) {
@@ -288,6 +336,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     // warps, idle until the first tile).  Dividing by the power-of-two scale 2^e is done as the
     // (exactly equal) product with 2^-e.
     const int t = threadIdx.x - 64, h = t >> 2, g = t & 3;
+    const uint16_t w_raw = a.w[int64_t(row) * HI + h];  // loaded with the query block, used at the end
     const uint16_t *qh = a.q_ix + (int64_t(row) * HI + h) * DI;
     uint8_t *brow = smem + SM_B + h * 64;
     float v[32];
@@ -322,7 +371,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       for (int j = t; j < 512; j += 256) reinterpret_cast<uint32_t *>(smem + SM_HG)[j] = 0;
     if (g == 0) {
       *reinterpret_cast<uint32_t *>(smem + SM_SFB + (h & 31) * 16 + (h >> 5) * 4) = sfword;
-      ws[h] = bf16_to_f32(a.w[int64_t(row) * HI + h]);
+      ws[h] = bf16_to_f32(w_raw);
     } else if (g == 1) {
       const int rz = 64 + h;
       *reinterpret_cast<uint32_t *>(smem + SM_SFB + (rz & 31) * 16 + (rz >> 5) * 4) = 0u;
@@ -337,7 +386,6 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    const uint32_t stages = smem_u32(smem + SM_STAGES);
     if (a.use_tma) {
       if (lane == 0) {
         for (int i = 0; i < ntiles; ++i) {
@@ -355,34 +403,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
           }
         }
       }
-    } else {
-      // Gather path: lane l resolves the slots of tile entries l, l+32, l+64, l+96 (raw
-      // candidate indices are loaded two tiles ahead), the slots are shuffled to the
-      // lanes that copy each 16-byte chunk, and each lane's copies arrive on the stage's
-      // barrier by themselves (cp.async.mbarrier.arrive.noinc).
-      auto load_cand = [&](int tile, int32_t (&cv)[4]) {  // entry index of each position (-1: none)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int pos = tile * IM_TILE + lane + 32 * j;
-          if (tile >= t0 + ntiles) cv[j] = -1;
-          else if (!a.cand) cv[j] = pos;
-          else if (cand_staged) cv[j] = cand_s[pos - t0 * IM_TILE];
-          else cv[j] = pos < a.P ? a.cand[int64_t(row) * a.P + pos] : -1;
-        }
-      };
-      auto resolve = [&](const int32_t (&cv)[4], int64_t (&sl)[4]) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int n = cv[j];
-          if (a.cand && (n < -1 || n >= n_entries)) report(a.err, CSA2_ERR_INDEX);
-          int64_t sv = -1;
-          if (n >= 0 && n < nvis) {
-            sv = cache_slot(a.c, b, n);
-            if (sv < 0) report(a.err, CSA2_ERR_INDEX);
-          }
-          sl[j] = sv;
-        }
-      };
+    } else if (!spread) {  // gather path, one tile after another (raw candidate indices two tiles ahead)
       int32_t c1[4], c2[4];
       int64_t cur[4], nxt[4];
       load_cand(t0, c1);
@@ -393,19 +414,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
         load_cand(t0 + i + 2, c2);
         resolve(c1, nxt);
         if (!mbar_wait_bounded(&empty[s], ((i / IM_STAGES) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
-        const uint32_t st = stages + s * IM_STAGE_BYTES;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {  // 512 chunks of 16 bytes: chunk qd = lane + 32 j
-          const int qd = lane + 32 * j, e = qd >> 2, c = qd & 3, m = row_of_entry(e);
-          // entry e = 8 j + lane / 4 lives in lane e % 32, register j / 4
-          const int64_t slot = __shfl_sync(0xffffffffu, cur[j >> 2], e & 31);
-          if (slot >= 0)
-            cp_async_16(st + m * 64 + ((c ^ ((m >> 1) & 3)) << 4), a.c.ix_codes + slot * CSA2_IX_CODE_BYTES + c * 16);
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j)  // scale word of entry e = lane + 32 j at atom word e
-          if (cur[j] >= 0) cp_async_4(st + IM_A_BYTES + (lane + 32 * j) * 4, a.c.ix_scales + cur[j] * CSA2_IX_SCALE_BYTES);
-        cp_async_arrive_noinc(&full[s]);
+        issue_tile(s, cur);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           cur[j] = nxt[j];
@@ -462,6 +471,13 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       if (i >= ntiles || pos >= a.P) return -1;
       return cand_staged ? cand_s[pos - t0 * IM_TILE] : a.cand[int64_t(row) * a.P + pos];
     };
+    if (spread && warp - 2 < ntiles) {  // this warp's tile of the gather (every stage is still free)
+      int32_t cv[4];
+      int64_t sl[4];
+      load_cand(t0 + warp - 2, cv);
+      resolve(cv, sl);
+      issue_tile(warp - 2, sl);
+    }
     int64_t n_next = entry_at(wg);
     for (int i = wg; i < ntiles; i += IM_EPI_WG) {
       const int acc = i % IM_ACC;
@@ -489,6 +505,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
           a.scores[int64_t(row) * a.n_out + pos] = ok ? sc : -INFINITY;
       }
     }
+    if (spread) cp_async_wait<0>();  // no copy of this thread is left in flight
     // positions past the visible entries (no key tile was loaded for them)
     if (!a.cand) {
       const int lo = max(t0, t_work) * IM_TILE, hi = min(t1 * IM_TILE, a.n_out);

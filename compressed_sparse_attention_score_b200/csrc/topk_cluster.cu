@@ -218,16 +218,18 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
         if (lane >= o) incl += y;
       }
       int at = cnt + incl - c;
+      while (tm) {  // few keys pass the bound: visit only those
+        const int e = __ffs(tm) - 1;
+        tm &= tm - 1;
+        uint32_t key = kk[0];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        if (tm & (1u << e)) {
-          atomicAdd(&hdst[kk[e] >> 20], 1u);
-          if (at < TK_CAPW) {
-            ckey[warp][at] = kk[e];
-            cidx[warp][at] = j0 + e;
-          }
-          ++at;
+        for (int i = 1; i < 16; ++i) key = e == i ? kk[i] : key;
+        atomicAdd(&hdst[key >> 20], 1u);
+        if (at < TK_CAPW) {
+          ckey[warp][at] = key;
+          cidx[warp][at] = j0 + e;
         }
+        ++at;
       }
       cnt += __shfl_sync(0xffffffffu, incl, 31);
     }
