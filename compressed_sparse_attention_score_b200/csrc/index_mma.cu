@@ -302,6 +302,24 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       if (cur[j] >= 0) cp_async_4(st + IM_A_BYTES + (lane + 32 * j) * 4, a.c.ix_scales + cur[j] * CSA2_IX_SCALE_BYTES);
     cp_async_arrive_noinc(&full[s]);
   };
+  auto issue_tma = [&](int i) {  // one lane: tile i of a whole-group run (its stage is free)
+    const int s = i % IM_STAGES;
+    const uint32_t st = stages + s * IM_STAGE_BYTES;
+    const int64_t slot0 = cache_slot(a.c, b, int64_t(t0 + i) * IM_TILE);
+    if (slot0 >= 0 && (slot0 & (IM_TILE - 1)) == 0 && slot0 + IM_TILE <= a.c.num_slots) {
+      mbar_arrive_expect_tx(&full[s], IM_A_BYTES + 512);
+      tma_load_4d(st, &tmap, 0, 0, 0, int(slot0 / IM_TILE), &full[s]);
+      bulk_load(st + IM_A_BYTES, a.c.ix_scales + slot0 * CSA2_IX_SCALE_BYTES, 512, &full[s]);
+    } else {
+      report(a.err, CSA2_ERR_INDEX);  // a visible tile without a valid page: epilogue masks it
+      mbar_arrive(&full[s]);
+    }
+  };
+  // The first tiles go out before the prologue's end: warp 1 initialises the barriers and
+  // meets the warps that issue them (warp 0 for whole-group runs, the epilogue warps for
+  // staged gathers) on named barrier 1.
+  const int pre_tiles = a.use_tma ? min(ntiles, IM_STAGES) : 0;
+  const int pre_threads = a.use_tma ? 64 : (spread ? 288 : 0);
 
   // ---------------------------------------------------------------- prologue
   if (warp == 0) {
@@ -319,18 +337,26 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       cp_async_commit();
       cp_async_wait<0>();
     }
-  } else if (warp == 1 && lane == 0) {
-    for (int s = 0; s < IM_STAGES; ++s) {
-      mbar_init(&full[s], a.use_tma ? 1 : 32);  // gather path: one cp.async arrival per producer lane
-      mbar_init(&empty[s], 1);
+    if (a.use_tma) {
+      named_bar_sync(1, pre_threads);
+      if (lane == 0)
+        for (int i = 0; i < pre_tiles; ++i) issue_tma(i);
     }
-    for (int i = 0; i < IM_ACC; ++i) {
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int s = 0; s < IM_STAGES; ++s) {
+        mbar_init(&full[s], a.use_tma ? 1 : 32);  // gather path: one cp.async arrival per producer lane
+        mbar_init(&empty[s], 1);
+      }
+      for (int i = 0; i < IM_ACC; ++i) {
+        mbar_init(&acc_full[i], 1);
+        mbar_init(&acc_empty[i], 4);
+      }
+      mbar_init(done, 1);
+      *abort_flag = 0;
+      mbar_init_fence();
     }
-    mbar_init(done, 1);
-    *abort_flag = 0;
-    mbar_init_fence();
+    if (pre_threads) named_bar_sync(1, pre_threads);
   } else if (warp >= 2 && warp < 10) {
     // quantise the query heads: thread 4h + g owns 32-value block g of head h (8 of the epilogue
     // warps, idle until the first tile).  Dividing by the power-of-two scale 2^e is done as the
@@ -338,11 +364,28 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     const int t = threadIdx.x - 64, h = t >> 2, g = t & 3;
     const uint16_t w_raw = a.w[int64_t(row) * HI + h];  // loaded with the query block, used at the end
     const uint16_t *qh = a.q_ix + (int64_t(row) * HI + h) * DI;
+    uint4 qv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qv[i] = reinterpret_cast<const uint4 *>(qh + 32 * g)[i];
+    if (spread) {  // this warp's tile of a staged gather (every stage is still free), read from the list
+      named_bar_sync(1, pre_threads);
+      if (warp - 2 < ntiles) {
+        int32_t cv[4];
+        int64_t sl[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int pos = (t0 + warp - 2) * IM_TILE + lane + 32 * j;
+          cv[j] = pos < a.P ? a.cand[int64_t(row) * a.P + pos] : -1;
+        }
+        resolve(cv, sl);
+        issue_tile(warp - 2, sl);
+      }
+    }
     uint8_t *brow = smem + SM_B + h * 64;
     float v[32];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 u = reinterpret_cast<const uint4 *>(qh + 32 * g)[i];
+      const uint4 u = qv[i];
       const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -388,19 +431,10 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     // ---------------------------------------------------------------- producer
     if (a.use_tma) {
       if (lane == 0) {
-        for (int i = 0; i < ntiles; ++i) {
+        for (int i = pre_tiles; i < ntiles; ++i) {
           const int s = i % IM_STAGES;
           if (!mbar_wait_bounded(&empty[s], ((i / IM_STAGES) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
-          const uint32_t st = stages + s * IM_STAGE_BYTES;
-          const int64_t slot0 = cache_slot(a.c, b, int64_t(t0 + i) * IM_TILE);
-          if (slot0 >= 0 && (slot0 & (IM_TILE - 1)) == 0 && slot0 + IM_TILE <= a.c.num_slots) {
-            mbar_arrive_expect_tx(&full[s], IM_A_BYTES + 512);
-            tma_load_4d(st, &tmap, 0, 0, 0, int(slot0 / IM_TILE), &full[s]);
-            bulk_load(st + IM_A_BYTES, a.c.ix_scales + slot0 * CSA2_IX_SCALE_BYTES, 512, &full[s]);
-          } else {
-            report(a.err, CSA2_ERR_INDEX);  // a visible tile without a valid page: epilogue masks it
-            mbar_arrive(&full[s]);
-          }
+          issue_tma(i);
         }
       }
     } else if (!spread) {  // gather path, one tile after another (raw candidate indices two tiles ahead)
@@ -471,13 +505,6 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       if (i >= ntiles || pos >= a.P) return -1;
       return cand_staged ? cand_s[pos - t0 * IM_TILE] : a.cand[int64_t(row) * a.P + pos];
     };
-    if (spread && warp - 2 < ntiles) {  // this warp's tile of the gather (every stage is still free)
-      int32_t cv[4];
-      int64_t sl[4];
-      load_cand(t0 + warp - 2, cv);
-      resolve(cv, sl);
-      issue_tile(warp - 2, sl);
-    }
     int64_t n_next = entry_at(wg);
     for (int i = wg; i < ntiles; i += IM_EPI_WG) {
       const int acc = i % IM_ACC;

@@ -46,6 +46,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Named barrier `id` over `threads` threads (a multiple of 32; whole warps take part).
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // Wait for the phase with the given parity to complete.  Gives up when *abort is
 // raised by another role or after `limit_ns`, raising *abort itself; returns
 // false when it gave up.
