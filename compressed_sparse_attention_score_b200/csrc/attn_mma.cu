@@ -758,8 +758,8 @@ constexpr int T_RED = T_PV + AM_TILE * 4;
 constexpr int T_HM = T_RED + 8 * 32 * 4;
 constexpr int T_QS = T_HM + 2 * 32 * 4;         // query prescale (as SM_QS)
 constexpr int T_NEW = T_QS + (8 * AM_QU + 32) * 4;   // this step's window token (as SM_NEW)
-constexpr int T_BAR = T_NEW + 512 + 32;         // full[8], qfull, phase_done
-constexpr int T_MISC = T_BAR + 8 * 10;
+constexpr int T_BAR = T_NEW + 512 + 32;         // qfull, phase_done
+constexpr int T_MISC = T_BAR + 8 * 2;
 constexpr size_t T_SMEM = T_MISC + 16 + 1024;
 }  // namespace
 
@@ -773,8 +773,7 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   float *red = reinterpret_cast<float *>(smem + T_RED);
   float *hmax = reinterpret_cast<float *>(smem + T_HM);
   float *hsum = hmax + 32;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + T_BAR);  // 64-dim block b of the tile written (128)
-  uint64_t *qfull = full + 8;                                     // Q written (256)
+  uint64_t *qfull = reinterpret_cast<uint64_t *>(smem + T_BAR);  // Q and the whole tile written (256)
   uint64_t *phase_done = qfull + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + T_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + T_MISC + 4);
@@ -880,7 +879,6 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
     tmem_relinquish();
   }
   if (issuer) {
-    for (int i = 0; i < 8; ++i) mbar_init(&full[i], AM_TILE);
     mbar_init(qfull, AM_PRODUCERS);
     mbar_init(phase_done, 1);
     *abort_flag = 0;
@@ -896,21 +894,18 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
   if (producer) {
     store_query_fp16(qraw, qmx, qinv, smem + T_Q);
     fence_proxy_async_smem();  // the query and this thread's key blocks, written before
-    mbar_arrive(qfull);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) mbar_arrive(&full[4 * half + c]);
+    mbar_arrive(qfull);        // the whole tile and the query are in place once all have arrived
   } else if (issuer) {
     constexpr uint32_t id = idesc_f16(AM_TILE, AM_HG, false, false);
-    bool ok = mbar_wait_bounded(qfull, 0, abort_flag, AM_WAIT_NS);
-    for (int i = 0; i < 8 && ok; ++i) {
-      const int blk = (i & 1) * 4 + (i >> 1);  // both halves' blocks in the order they are written
-      if (!(ok = mbar_wait_bounded(&full[blk], 0, abort_flag, AM_WAIT_NS))) break;
+    if (mbar_wait_bounded(qfull, 0, abort_flag, AM_WAIT_NS)) {
       tc_fence_after();
-      const uint32_t a0 = smem_u32(smem + T_KT + blk * 16384), b0 = smem_u32(smem + T_Q + blk * 4096);
+      for (int blk = 0; blk < 8; ++blk) {
+        const uint32_t a0 = smem_u32(smem + T_KT + blk * 16384), b0 = smem_u32(smem + T_Q + blk * 4096);
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4)
-        tc_mma_f16(tmem, smem_desc(a0 + 32 * k4, 16, 1024, LAYOUT_SWIZZLE_128B),
-                   smem_desc(b0 + 32 * k4, 16, 1024, LAYOUT_SWIZZLE_128B), id, i > 0 || k4 > 0);
+        for (int k4 = 0; k4 < 4; ++k4)
+          tc_mma_f16(tmem, smem_desc(a0 + 32 * k4, 16, 1024, LAYOUT_SWIZZLE_128B),
+                     smem_desc(b0 + 32 * k4, 16, 1024, LAYOUT_SWIZZLE_128B), id, blk > 0 || k4 > 0);
+      }
     }
     tc_commit(phase_done);
   }
