@@ -368,15 +368,15 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
 #pragma unroll
     for (int i = 0; i < 4; ++i) qv[i] = reinterpret_cast<const uint4 *>(qh + 32 * g)[i];
     if (spread) {  // this warp's tile of a staged gather (every stage is still free), read from the list
+      int32_t cv[4];  // loaded together with the query block
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int pos = (t0 + warp - 2) * IM_TILE + lane + 32 * j;
+        cv[j] = (warp - 2 < ntiles && pos < a.P) ? a.cand[int64_t(row) * a.P + pos] : -1;
+      }
       named_bar_sync(1, pre_threads);
       if (warp - 2 < ntiles) {
-        int32_t cv[4];
         int64_t sl[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int pos = (t0 + warp - 2) * IM_TILE + lane + 32 * j;
-          cv[j] = pos < a.P ? a.cand[int64_t(row) * a.P + pos] : -1;
-        }
         resolve(cv, sl);
         issue_tile(warp - 2, sl);
       }
@@ -402,7 +402,10 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       ex = e8m0_ceil_exponent(__fdiv_rn(am, 6.0f));
       const float inv = pow2f(-ex);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) cw[i >> 3] |= e2m1_code(__fmul_rn(v[i], inv)) << (4 * (i & 7));
+      for (int i = 0; i < 32; i += 2) {  // a NaN encodes as 0, as the format's encoder does
+        const float a0 = __fmul_rn(v[i], inv), a1 = __fmul_rn(v[i + 1], inv);
+        cw[i >> 3] |= e2m1x2_code(a0 == a0 ? a0 : 0.f, a1 == a1 ? a1 : 0.f) << (4 * (i & 7));
+      }
     }
     // 16 bytes = chunk g of this 64-byte row, at its swizzled position
     *reinterpret_cast<uint4 *>(brow + ((g ^ ((h >> 1) & 3)) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);

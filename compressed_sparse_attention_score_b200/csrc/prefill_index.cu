@@ -268,7 +268,10 @@ __global__ void __launch_bounds__(PF_THREADS, 2) prefill_index_kernel(const __gr
           ex = e8m0_ceil_exponent(__fdiv_rn(am, 6.0f));
           const float inv = pow2f(-ex);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) cw[i >> 3] |= e2m1_code(__fmul_rn(v[i], inv)) << (4 * (i & 7));
+          for (int i = 0; i < 32; i += 2) {  // a NaN encodes as 0, as the format's encoder does
+            const float a0 = __fmul_rn(v[i], inv), a1 = __fmul_rn(v[i + 1], inv);
+            cw[i >> 3] |= e2m1x2_code(a0 == a0 ? a0 : 0.f, a1 == a1 ? a1 : 0.f) << (4 * (i & 7));
+          }
         }
         *reinterpret_cast<uint4 *>(brow + ((g ^ ((h >> 1) & 3)) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
         sfpart |= uint32_t(ex + 127) << (8 * g);

@@ -231,6 +231,19 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2_f16x2(uint32_t byte) {
   asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(out) : "r"(byte));
   return out;
 }
+// Two fp32 values -> two e2m1 codes in one byte, `lo` in the low nibble (cvt.rn.satfinite puts
+// its first operand in the high nibble): round to nearest even, saturating at +-6.  Checked on
+// the B200 against the encoder written from the format (common.cuh) over ties, saturation,
+// subnormals and a dense range: the same codes, except that a negative value rounding to zero
+// comes out as -0 (code 8, the same value in every product).  NaN is not mapped like the
+// encoder does (to code 0): callers map it to 0 first.
+__device__ __forceinline__ uint32_t e2m1x2_code(float lo, float hi) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 r;\n\tcvt.rn.satfinite.e2m1x2.f32 r, %1, %2;\n\tcvt.u32.u8 %0, r;\n\t}"
+      : "=r"(out)
+      : "f"(hi), "f"(lo));
+  return out;
+}
 // Two E4M3 codes (16 bits, low byte first) -> two fp16 values (exact).
 __device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint32_t two) {
   uint32_t out;
