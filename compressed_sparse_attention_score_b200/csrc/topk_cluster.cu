@@ -338,15 +338,15 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_cluster_kernel(const float
   } else {
   // ---- sampled lower bound on the larger selection's threshold (top 12 key bits)
   const uint32_t target = uint32_t(kbig / SAMPLE) + uint32_t(kbig / (2 * SAMPLE)) + 32;
-  for (int base = wb; base < we; base += 32 * SAMPLE * 4) {
-    float v[4];
+  for (int base = wb; base < we; base += 32 * SAMPLE * 8) {  // 8 loads in flight per lane (one round for a
+    float v[8];                                                // range of up to 4096 scores)
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 8; ++u) {
       const int j = base + 32 * SAMPLE * u + lane;
       v[u] = j < we ? srow[j] : -INFINITY;
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 8; ++u) {
       const uint32_t key = score_key(v[u]);
       if (key != KEY_NEG_INF) atomicAdd(&hs[key >> 20], 1u);
     }
