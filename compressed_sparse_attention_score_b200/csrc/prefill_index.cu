@@ -410,7 +410,7 @@ __global__ void __launch_bounds__(PF_THREADS, 2) prefill_index_kernel(const __gr
       if (ok && !mbar_wait_bounded(&acc_full[buf], (i / PF_ACC) & 1, abort_flag, PF_WAIT_NS)) ok = false;
       ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld is taken by the whole warp or not at all
       float sc = 0.f;
-      if (ok) {
+      if (ok) {  // (uniform in the warp)
         tc_fence_after();
         const uint32_t taddr = tmem + (uint32_t(32 * q4) << 16) + (buf * PF_Q + g) * PF_N;
         uint32_t r0[32], r1[32];
@@ -418,10 +418,13 @@ __global__ void __launch_bounds__(PF_THREADS, 2) prefill_index_kernel(const __gr
         tc_ld_32x32b_x32(taddr + 32, r1);
         tc_wait_ld();
         tc_fence_before();
-        sc = weighted_relu_score(r0, r1, w4);  // the decode kernel's arithmetic: the same score
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);  // the next tile's products may start now
+        sc = weighted_relu_score(r0, r1, w4);         // the decode kernel's arithmetic: the same score
+      } else {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
       // append the keys above the threshold; an entry without a valid page is never a
       // candidate (its error is already reported)
       const int n = i * PF_TILE + e;
