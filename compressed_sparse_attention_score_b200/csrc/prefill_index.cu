@@ -46,12 +46,13 @@ constexpr int PF_ACC = 1;               // accumulator sets (the other CTA on th
 constexpr uint32_t PF_COL_SFA = PF_ACC * PF_Q * 64;    // after the accumulator sets
 constexpr uint32_t PF_COL_SFB = PF_COL_SFA + 4 * PF_ACC;
 constexpr uint64_t PF_WAIT_NS = 2000000000ull;
-static_assert(PF_COL_SFB + 4 * PF_Q <= PF_TMEM_COLS, "accumulators and scale atoms exceed the TMEM allocation");
+static_assert(PF_COL_SFB + 4 <= PF_TMEM_COLS, "accumulators and scale atoms exceed the TMEM allocation");
+static_assert(PF_Q * PF_N <= 256, "the CTA's queries are one MMA's B operand (N <= 256)");
 
 constexpr int PS_STAGES = 0;
 constexpr int PS_B = PF_STAGES * PF_STAGE_BYTES;          // PF_Q x [64 heads x 64 B] query codes
-constexpr int PS_SFB = PS_B + PF_Q * 4096;                // PF_Q x 512 B scale atoms
-constexpr int PS_W = PS_SFB + PF_Q * 512;                 // PF_Q x 64 fp32 head weights
+constexpr int PS_SFB = PS_B + PF_Q * 4096;                // 512 B scale atom of the PF_Q x 64 B rows
+constexpr int PS_W = PS_SFB + 512;                        // PF_Q x 64 fp32 head weights
 constexpr int PS_CKEY = PS_W + PF_Q * 256;                // PF_Q x PF_CAP keys
 constexpr int PS_CENT = PS_CKEY + PF_Q * PF_CAP * 4;      // PF_Q x PF_CAP entries
 constexpr int PS_SCR = PS_CENT + PF_Q * PF_CAP * 4;       // PF_Q x cut scratch: PF_KMAX keys, PF_KMAX entries
@@ -277,13 +278,10 @@ __global__ void __launch_bounds__(PF_THREADS, 2) prefill_index_kernel(const __gr
         sfpart |= uint32_t(ex + 127) << (8 * g);
       }
       const uint32_t sfword = sfpart | __shfl_xor_sync(0xffffffffu, sfpart, 1);
-      uint8_t *sfb = smem + PS_SFB + qi * 512;
-      if ((item & 1) == 0) {
-        *reinterpret_cast<uint32_t *>(sfb + (h & 31) * 16 + (h >> 5) * 4) = sfword;
+      if ((item & 1) == 0) {  // B row 64 qi + h: lane-row r % 32, column r / 32 of the atom
+        const int r = 64 * qi + h;
+        *reinterpret_cast<uint32_t *>(smem + PS_SFB + (r & 31) * 16 + (r >> 5) * 4) = sfword;
         ws[qi * 64 + h] = bf16_to_f32(a.w[(int64_t(b) * a.Q + q0 + min(qi, nq - 1)) * HI + h]);
-      } else {
-        const int rz = 64 + h;
-        *reinterpret_cast<uint32_t *>(sfb + (rz & 31) * 16 + (rz >> 5) * 4) = 0u;
       }
     }
     if (t < PF_Q * 3) reinterpret_cast<uint32_t *>(smem + PS_TCNT)[t] = 0;
@@ -342,17 +340,13 @@ __global__ void __launch_bounds__(PF_THREADS, 2) prefill_index_kernel(const __gr
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t stages = smem_u32(smem + PS_STAGES);
-      uint64_t bd0[PF_Q], bd1[PF_Q];
-#pragma unroll
-      for (int qi = 0; qi < PF_Q; ++qi) {
-        const uint32_t bq = smem_u32(smem + PS_B + qi * 4096);
-        tc_cp_32x128b_warpx4(tmem + PF_COL_SFB + 4 * qi,
-                             smem_desc(smem_u32(smem + PS_SFB + qi * 512), 16, 128, LAYOUT_SWIZZLE_NONE));
-        bd0[qi] = smem_desc(bq, 16, 512, LAYOUT_SWIZZLE_64B);
-        bd1[qi] = smem_desc(bq + 32, 16, 512, LAYOUT_SWIZZLE_64B);
-      }
-      constexpr uint32_t id0 = idesc_mxf4(PF_TILE, PF_N, 0, 0);
-      constexpr uint32_t id1 = idesc_mxf4(PF_TILE, PF_N, 2, 2);
+      // the CTA's queries are one B operand (query qi = rows 64 qi .. 64 qi + 63), one MMA per K half
+      const uint32_t bq = smem_u32(smem + PS_B);
+      tc_cp_32x128b_warpx4(tmem + PF_COL_SFB, smem_desc(smem_u32(smem + PS_SFB), 16, 128, LAYOUT_SWIZZLE_NONE));
+      const uint64_t bd0 = smem_desc(bq, 16, 512, LAYOUT_SWIZZLE_64B);
+      const uint64_t bd1 = smem_desc(bq + 32, 16, 512, LAYOUT_SWIZZLE_64B);
+      constexpr uint32_t id0 = idesc_mxf4(PF_TILE, PF_Q * PF_N, 0, 0);
+      constexpr uint32_t id1 = idesc_mxf4(PF_TILE, PF_Q * PF_N, 2, 2);
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % PF_STAGES, buf = i % PF_ACC;
         if (!mbar_wait_bounded(&full[s], (i / PF_STAGES) & 1, abort_flag, PF_WAIT_NS)) break;
@@ -364,12 +358,9 @@ __global__ void __launch_bounds__(PF_THREADS, 2) prefill_index_kernel(const __gr
         tc_cp_32x128b_warpx4(sfa, smem_desc(st + PF_A_BYTES, 16, 128, LAYOUT_SWIZZLE_NONE));
         const uint64_t a0 = smem_desc(st, 16, 512, LAYOUT_SWIZZLE_64B);
         const uint64_t a1 = smem_desc(st + 32, 16, 512, LAYOUT_SWIZZLE_64B);
-#pragma unroll
-        for (int qi = 0; qi < PF_Q; ++qi) {
-          const uint32_t d = tmem + (buf * PF_Q + qi) * PF_N;
-          tc_mma_mxf4(d, a0, bd0[qi], id0, sfa, tmem + PF_COL_SFB + 4 * qi, false);
-          tc_mma_mxf4(d, a1, bd1[qi], id1, sfa, tmem + PF_COL_SFB + 4 * qi, true);
-        }
+        const uint32_t d = tmem + buf * PF_Q * PF_N;
+        tc_mma_mxf4(d, a0, bd0, id0, sfa, tmem + PF_COL_SFB, false);
+        tc_mma_mxf4(d, a1, bd1, id1, sfa, tmem + PF_COL_SFB, true);
         tc_commit(&empty[s]);
         tc_commit(&acc_full[buf]);
       }
