@@ -66,11 +66,10 @@ constexpr size_t IM_SMEM_BYTES = SM_TOTAL + 1024;       // slack for 1024-byte a
 // counts cross the cluster.
 constexpr int IM_SEL_MAX = REINDEX_SELECT_MAX;          // candidates per row
 constexpr int SM_KEYS = SM_TOTAL;                       // [IM_CAND_TILES * 128] this CTA's keys
-constexpr int SM_HL = SM_KEYS + IM_CAND_TILES * IM_TILE * 4;   // local 256-bin histogram
-constexpr int SM_HG = SM_HL + 256 * 4;                  // [2][256] cluster-wide histograms (peers add here)
+constexpr int SM_HL = SM_KEYS + IM_CAND_TILES * IM_TILE * 4;   // [2][256] local histograms (alternate digits)
+constexpr int SM_HG = SM_HL + 2 * 256 * 4;              // [2][256] cluster-wide histograms (peers add here)
 constexpr int SM_CG = SM_HG + 2 * 256 * 4;              // [16][2] every CTA's counts above / equal
-constexpr int SM_SELW = SM_CG + 16 * 2 * 4;             // selection state (4 words)
-constexpr int SM_WCNT = SM_SELW + 16;                   // per warp: keys above / equal to the threshold
+constexpr int SM_WCNT = SM_CG + 16 * 2 * 4;             // per warp: keys above / equal to the threshold
 constexpr size_t IM_SEL_SMEM_BYTES = SM_WCNT + 2 * (IM_THREADS / 32) * 4 + 1024;
 static_assert(IM_EPI_WG >= 2, "the query is quantised by 8 epilogue warps");
 static_assert((IM_SEL_MAX + IM_TILE - 1) / IM_TILE <= 16 * IM_CAND_TILES,
@@ -108,7 +107,7 @@ __device__ __forceinline__ int entry_of_row(int m) { return (m & 31) * 4 + (m >>
 // the threshold bin holds exactly the keys still needed.  A last exchange of per-CTA counts
 // places each CTA's chosen entries.  Called by every thread of every CTA of the cluster.
 __device__ __forceinline__ void select_cluster(const uint32_t *kl, const int32_t *el, int nl, int k, int32_t *orow,
-                                               uint32_t *hl, uint32_t *hg, int *cg_, uint32_t *selw, int *wcnt) {
+                                               uint32_t *hl, uint32_t *hg, int *cg_, int *wcnt) {
   constexpr int NW = IM_THREADS / 32;
   cg::cluster_group cluster = cg::this_cluster();
   const int cs = int(cluster.num_blocks()), rank = int(cluster.block_rank());
@@ -116,10 +115,12 @@ __device__ __forceinline__ void select_cluster(const uint32_t *kl, const int32_t
   uint32_t prefix = 0;
   int need = k, width = 0;
   bool all = false;
+  // Per digit: local histogram, one block barrier, pushes, one cluster barrier; every warp then
+  // finds the digit itself.  The local and cluster histograms alternate between two copies, each
+  // zeroed a digit ahead, after the last reads of it are ordered by a barrier.
   for (int pass = 0, shift = 24; shift >= 0; ++pass, shift -= 8) {
-    uint32_t *hcur = hg + (pass & 1) * 256;
-    if (t < 256) hl[t] = 0;
-    __syncthreads();
+    uint32_t *hcur = hg + (pass & 1) * 256, *hgn = hg + ((pass + 1) & 1) * 256;
+    uint32_t *hlc = hl + (pass & 1) * 256, *hln = hl + ((pass + 1) & 1) * 256;
     const uint32_t himask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
     for (int i = t; i - lane < nl; i += IM_THREADS) {  // lanes with the same bin add once
       const uint32_t key = i < nl ? kl[i] : KEY_NEG_INF;
@@ -127,55 +128,54 @@ __device__ __forceinline__ void select_cluster(const uint32_t *kl, const int32_t
       const uint32_t am = __ballot_sync(0xffffffffu, act);
       if (act) {
         const uint32_t bin = (key >> shift) & 255u, peers = __match_any_sync(am, bin);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hl[bin], uint32_t(__popc(peers)));
+        if (lane == __ffs(peers) - 1) atomicAdd(&hlc[bin], uint32_t(__popc(peers)));
       }
     }
+    if (t < 256) hln[t] = 0;  // read last by the previous digit's pushes
     __syncthreads();
+    if (t < 256) hgn[t] = 0;  // read last by every warp before this digit's block barrier
     for (int j = t; j < 256 * cs; j += IM_THREADS) {  // into every CTA's copy, this one's included
-      const uint32_t c = hl[j & 255];
+      const uint32_t c = hlc[j & 255];
       if (c) atomicAdd(cluster.map_shared_rank(hcur + (j & 255), j >> 8), c);
     }
-    if (t < 256) hg[((pass + 1) & 1) * 256 + t] = 0;  // the next digit's copy: read last before the previous barrier
     cluster.sync();
-    if (warp == 0) {  // the digit at which the count from the top reaches `need`
-      uint32_t c8[8], sum = 0;
+    // the digit at which the count from the top reaches `need` (the same in every warp and CTA)
+    uint32_t c8[8], sum = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) sum += (c8[j] = hcur[255 - (8 * lane + j)]);
-      uint32_t x = sum;
+    for (int j = 0; j < 8; ++j) sum += (c8[j] = hcur[255 - (8 * lane + j)]);
+    uint32_t x = sum;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      const uint32_t excl = x - sum, total = __shfl_sync(0xffffffffu, x, 31);
-      if (total <= uint32_t(need)) {  // first digit only: at most k valid keys, all chosen
-        if (lane == 0) selw[0] = 0xFFFFFFFFu;
-      } else {
-        const int L = __ffs(__ballot_sync(0xffffffffu, excl < uint32_t(need) && x >= uint32_t(need))) - 1;
-        if (lane == L) {
-          uint32_t cum = excl;
-#pragma unroll 1
-          for (int j = 0; j < 8; ++j) {
-            if (cum + c8[j] >= uint32_t(need)) {
-              selw[0] = uint32_t(255 - (8 * lane + j));
-              selw[1] = uint32_t(need) - cum;
-              selw[2] = c8[j];
-              break;
-            }
-            cum += c8[j];
-          }
-        }
-      }
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    __syncthreads();
-    if (selw[0] == 0xFFFFFFFFu) {
+    const uint32_t excl = x - sum, total = __shfl_sync(0xffffffffu, x, 31);
+    if (total <= uint32_t(need)) {  // first digit only: at most k valid keys, all chosen
       all = true;
       break;
     }
-    prefix |= selw[0] << shift;
-    need = int(selw[1]);
+    const int L = __ffs(__ballot_sync(0xffffffffu, excl < uint32_t(need) && x >= uint32_t(need))) - 1;
+    uint32_t dg = 0, nd = 0, cnt = 0;
+    if (lane == L) {
+      uint32_t cum = excl;
+#pragma unroll 1
+      for (int j = 0; j < 8; ++j) {
+        if (cum + c8[j] >= uint32_t(need)) {
+          dg = uint32_t(255 - (8 * lane + j));
+          nd = uint32_t(need) - cum;
+          cnt = c8[j];
+          break;
+        }
+        cum += c8[j];
+      }
+    }
+    dg = __shfl_sync(0xffffffffu, dg, L);
+    nd = __shfl_sync(0xffffffffu, nd, L);
+    cnt = __shfl_sync(0xffffffffu, cnt, L);
+    prefix |= dg << shift;
+    need = int(nd);
     width = 32 - shift;
-    if (int(selw[2]) == need) break;  // every key of the threshold bin is chosen
+    if (int(cnt) == need) break;  // every key of the threshold bin is chosen
   }
   // keys above / equal to the threshold T, compared on the top `width` bits
   const int sh = 32 - width;
@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     sfword |= __shfl_xor_sync(0xffffffffu, sfword, 2);
     // scale atom word of row r: lane-row r % 32, column r / 32 (rows 64..127 unused, zero)
     if constexpr (SEL)
-      for (int j = t; j < 512; j += 256) reinterpret_cast<uint32_t *>(smem + SM_HG)[j] = 0;
+      for (int j = t; j < 1024; j += 256) reinterpret_cast<uint32_t *>(smem + SM_HL)[j] = 0;  // both pairs
     if (g == 0) {
       *reinterpret_cast<uint32_t *>(smem + SM_SFB + (h & 31) * 16 + (h >> 5) * 4) = sfword;
       ws[h] = bf16_to_f32(w_raw);
@@ -556,7 +556,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     select_cluster(reinterpret_cast<const uint32_t *>(smem + SM_KEYS), cand_s, max(0, min(a.P - t0 * IM_TILE, ntiles * IM_TILE)),
                    a.k, a.sel + int64_t(row) * a.k, reinterpret_cast<uint32_t *>(smem + SM_HL),
                    reinterpret_cast<uint32_t *>(smem + SM_HG), reinterpret_cast<int *>(smem + SM_CG),
-                   reinterpret_cast<uint32_t *>(smem + SM_SELW), reinterpret_cast<int *>(smem + SM_WCNT));
+                   reinterpret_cast<int *>(smem + SM_WCNT));
   }
 }
 
