@@ -935,14 +935,14 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
     for (int h = 0; h < 32; ++h) mx[h] = valid ? x[h] : -INFINITY;
     red[warp * 32 + lane] = reduce_scatter32<true>(mx);
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (warp == 0)
-      hmax[lane] = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane]));
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    // every warp forms the 32 head maxima itself (lane l: head l) and shares them by shuffles
+    const float mh = fmaxf(fmaxf(red[lane], red[32 + lane]), fmaxf(red[64 + lane], red[96 + lane]));
+    if (warp == 0) hmax[lane] = mh;
     float sm[32];
     uint32_t ph[16];
 #pragma unroll
     for (int h = 0; h < 32; h += 2) {
-      const float m0 = hmax[h], m1 = hmax[h + 1];
+      const float m0 = __shfl_sync(0xffffffffu, mh, h), m1 = __shfl_sync(0xffffffffu, mh, h + 1);
       const float e0 = (valid && m0 != -INFINITY) ? __expf(x[h] - m0) : 0.f;
       const float e1 = (valid && m1 != -INFINITY) ? __expf(x[h + 1] - m1) : 0.f;
       sm[h] = e0;
@@ -954,14 +954,13 @@ __global__ void __launch_bounds__(AM_THREADS, 1) attn_tile_kernel(AttnArgs p) {
     for (int u = 0; u < 4; ++u)
       *reinterpret_cast<uint4 *>(smem + T_Q + mnmaj64(key, u)) =
           make_uint4(ph[4 * u], ph[4 * u + 1], ph[4 * u + 2], ph[4 * u + 3]);
-    red[warp * 32 + lane] = reduce_scatter32<false>(sm);
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (warp == 0) hsum[lane] = (red[lane] + red[32 + lane]) + (red[64 + lane] + red[96 + lane]);
+    red[128 + warp * 32 + lane] = reduce_scatter32<false>(sm);  // (the maxima above may still be read)
   }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (!aborted && warp == 0) hsum[lane] = (red[128 + lane] + red[160 + lane]) + (red[192 + lane] + red[224 + lane]);
 
   // ---------------------------------------------------------------- phase 3: O^T = V^T P^T
   if (!aborted && issuer) {
