@@ -746,7 +746,7 @@ def test_swa_new_token_in_the_attention_launch(case):
                                         (300, 700, 2 * 1500), (2, 400, 2 * 1000)])
 def test_reindex_fused_selection(B, P, tokens):
     """Reindex over a pool of at most 16384 candidates scores and selects in one launch (each
-    row's keys in one CTA's shared memory).  Its choice must equal the unfused path's bit for
+    row's keys spread over its cluster's shared memory).  Its choice must equal the unfused path's bit for
     bit: csa2_index_score over the pool, csa2_topk of those scores, mapped through the pool.
     Pools are ascending with -1 pads and entries the query cannot see; some rows score every
     candidate 0 (all tied: the earliest candidates win); P = 400 < k pads the selection; B = 300
