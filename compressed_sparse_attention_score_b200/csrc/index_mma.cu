@@ -12,15 +12,17 @@
 // that tcgen05.cp expects (word w = (m % 32) * 4 + m / 32 = e).  Warp roles:
 //   warp 0     producer: for a run of whole 128-entry groups one TMA box of a
 //              4-D tensor map whose outer strides perform the row permutation
-//              (64-byte swizzle) plus one 512-byte bulk copy of the scales;
-//              for candidate lists, cp.async of each listed entry instead;
+//              (64-byte swizzle) plus one 512-byte bulk copy of the scales, the
+//              first 8 tiles during the prologue; for long candidate lists,
+//              cp.async of each listed entry instead;
 //   warp 1     MMA issuer (one lane): tcgen05.cp of the scale atom to TMEM, two
 //              K=64 MMAs into one of three TMEM accumulators, tcgen05.commit;
 //   warps 2-9  epilogue, two warpgroups taking alternate tiles: tcgen05.ld of
 //              the 64 head values of its 32 keys, weighted ReLU sum, fp32 score
-//              store.
+//              store.  A candidate list of at most 8 tiles is gathered by these
+//              warps, one tile each, in the prologue.
 // The query heads are quantised to MXFP4 in the prologue (warps 2-9, one 32-value block per
-// thread; same codec as the keys).
+// thread; the keys' block format, encoded by cvt.rn.satfinite.e2m1x2).
 // Every mbarrier wait is time-bounded; on expiry the CTA drains and reports
 // CSA2_ERR_TIMEOUT instead of hanging.
 #include <cooperative_groups.h>
