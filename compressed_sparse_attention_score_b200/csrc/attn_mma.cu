@@ -1,9 +1,9 @@
 // K6/K7/K8 (tensor-core form): attention of 64 query heads over a row's selected
 // global-KV entries and/or its sliding window, on tcgen05 (kind::f16).
 //
-// CTA = one query row x 32 heads.  Each key's 512-d vector is both key and value.
-// Keys come from two sources that share one softmax (so a CTA given both returns
-// the log-sum-exp merge of the two branches exactly):
+// Each key's 512-d vector is both key and value.  Keys come from two sources that share
+// one softmax (so a CTA given both returns the log-sum-exp merge of the two branches
+// exactly):
 //   sparse  -- listed main-KV entries (or, dense, every visible entry of a range):
 //              e2m1 x E4M3-per-16 dequantised to fp16 (exact: <= 6 significant
 //              bits, in fp16 range);
@@ -11,24 +11,23 @@
 //              folded into the logit multiplier and into P.
 // The bf16 query heads enter the MMA prescaled by a power of two per head (see
 // store_query_fp16), so they are exact in fp16 whatever their magnitude.
-// Phase 1  S^T[key][head] = K Q^T per 128-key tile (M = 128 keys, N = 32 heads,
-//          K = 512 dims in 64-dim chunks, 128-byte swizzled K-major operands),
-//          all tiles resident in TMEM.
-// Phase 2  exact two-pass softmax over every key of the row, read from TMEM
-//          (per-head max / sum by warp reduce-scatter), P^T written to shared
-//          memory in fp16 (MN-major, 64-byte swizzle).
-// Phase 3  O^T[dim][head] = V^T P^T per 128-dim tile (M = 128 dims, N = 32 heads,
-//          K = keys in 16-key steps), V^T chunks MN-major with 128-byte swizzle,
-//          accumulated in TMEM.
-// Phase 4  O / sum and lse = max + log(sum), coalesced fp32 stores; when a cluster of
-//          CTAs splits the row's keys, the partials (O, max, sum) are combined over
-//          distributed shared memory, each CTA producing one slice of the 512 dims.
-// A tile's raw key bytes (288 B per listed entry, 512 B per window token) are
-// gathered once into shared memory with asynchronous 16-byte copies, all in flight
-// together; both products dequantise from there, so a CTA whose keys fit one tile
-// reads them from memory once.  The dequantising threads fill a 4-deep ring of
-// 16 KB operand buffers while the single issuing thread drives the tensor core;
-// every wait is time-bounded.
+// Two kernels:
+//   attn_tile_kernel  -- one 128-key tile per CTA, 32 heads (a cluster of up to 5 CTAs
+//              per row and head group): the producers load their key halves into
+//              registers and dequantise them into a 128 KB fp16 tile (8 blocks of 64
+//              dims, 128-byte swizzle) that is the K-major A operand of S^T = K Q^T
+//              and the MN-major A operand of O^T = V^T P^T, so every key is read and
+//              dequantised once;
+//   attn_mma_kernel   -- up to 5 tiles per CTA, all 64 heads (many rows, or dense rows
+//              in clusters of up to 16): the same tile as a ring with one mbarrier pair
+//              per 64-dim block, S^T of every tile kept in TMEM for an exact two-pass
+//              softmax, each tile dequantised again for O^T (a CTA with one tile keeps it).
+// Softmax: per-head max and sum by warp reduce-scatter, P^T written to shared memory
+// in fp16 (MN-major).  Output: O / sum and lse = max + log(sum), coalesced fp32
+// stores; when a cluster of CTAs splits the row's keys, each CTA pushes each owner its
+// slice of the partial O (with max and sum) into distributed shared memory, and the
+// owners combine.  A single thread issues the tensor-core work; every wait is
+// time-bounded.
 #include <cooperative_groups.h>
 #include <cuda_fp16.h>
 
