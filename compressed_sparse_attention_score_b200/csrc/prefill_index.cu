@@ -2,10 +2,12 @@
 //
 // CTA = PF_Q consecutive query tokens of one sequence x every key tile any of them sees.
 // A 128-entry key tile is loaded once (one TMA box of the codes plus the scale words, or
-// cp.async gathers for caches a tensor map cannot describe) and serves all PF_Q queries: per
-// query two K=64 block-scaled FP4 MMAs (tcgen05 kind::mxf4, N = 64 heads) into the query's
-// accumulator.  Two CTAs share an SM (each holds 256 TMEM columns and a 4-stage ring), so one
-// CTA's tensor-core and load phases fill the other's epilogue gaps.  Warp roles:
+// cp.async gathers for caches a tensor map cannot describe) and serves all PF_Q queries: their
+// 64 heads each are one B operand (N = 64 PF_Q, one scale atom), two K=64 block-scaled FP4
+// MMAs (tcgen05 kind::mxf4) per tile, query g's accumulator in columns 64 g ..  Two CTAs
+// share an SM (each holds 256 TMEM columns and a 4-stage ring), so one CTA's tensor-core and
+// load phases fill the other's epilogue gaps; the epilogue hands the accumulator back as soon
+// as it has read it.  Warp roles:
 //   warp 0       producer;
 //   warp 1       MMA issuer (one lane);
 //   warps 2-..   one epilogue warpgroup per query: the weighted-ReLU score of each of its 128
