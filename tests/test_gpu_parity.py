@@ -709,15 +709,19 @@ def test_prefill_fused_ties_and_short_rows():
 
 
 # ------------------------------------------------------------------ this step's window token in the attention launch
-@pytest.mark.parametrize("case", ["reuse4", "reuse32", "full1"])
+@pytest.mark.parametrize("case", ["reuse4", "reuse32", "full1", "short4"])
 def test_swa_new_token_in_the_attention_launch(case):
     """csa2_sparse_attn with swa_new (the step's window token quantised inside the launch) must equal
     csa2_pack_swa of that token followed by csa2_sparse_attn, bit for bit: the ring's codes and scale
     and the layer's o and lse.  reuse4: one-tile clusters; reuse32: two-CTA clusters of the general
-    kernel; full1: the Full path (scan, top-k, attention)."""
+    kernel; full1: the Full path (scan, top-k, attention); short4: one-tile clusters of sequences
+    whose window is not yet full, so that the token is the key of a thread in each of the four
+    warp pairs of the window tile (positions 5, 40, 77 and 1000)."""
     k = K()
     if case == "full1":
         spec = W.scaled(W.tiny_full(), [3001], B=1)
+    elif case == "short4":
+        spec = W.scaled(W.reuse64k(), [6, 41, 78, 1001], B=4)
     else:
         B = 4 if case == "reuse4" else 32
         spec = W.scaled(W.reuse64k(), [3000 + 37 * b for b in range(B)], B=B)
