@@ -93,7 +93,86 @@ struct IndexMmaArgs {
   int chunk;  // tiles per CTA
   int k;         // fused selection: top-k of the candidates ...
   int32_t *sel;  // ... written here [rows][k] (entries, ascending; -1 pads)
+  int rows;      // query rows (balanced full scan: at most 32)
+  int grid;      // > 0: balanced full scan over a one-dimensional grid of this many CTAs
+  int spec;      // balanced: CTAs per row of the deal when every row fills the output (0: none)
 };
+
+// Balanced full scan.  Rows of very different lengths (a ragged batch) would leave most of a
+// fixed (split, row) grid idle while the longest rows' few CTAs stream; instead every CTA deals
+// the grid to the rows in proportion to their tiles (the same deal in every warp and CTA: it
+// depends only on the rows' visible entries), at least IM_MIN_TILES tiles per CTA, and the score
+// positions past each row's visible entries are split evenly over all CTAs.  Lane r of a warp
+// holds row r's figures.
+constexpr int IM_MIN_TILES = 8;
+struct Deal {
+  int row, t0, t_end;          // this CTA's row (-1: none) and its tiles [t0, t_end)
+  int tiles, fill;             // lane r: row r's tiles and its positions past them
+  int64_t fill_pre, fill_all;  // lane r: positions past the tiles of rows < r; of every row
+};
+__device__ __forceinline__ Deal deal_rows(const IndexMmaArgs &a, int lane) {
+  int tl = 0;
+  if (lane < a.rows) tl = (min(visible_entries(a.c, lane / a.Q, a.q_pos[lane]), a.n_out) + IM_TILE - 1) / IM_TILE;
+  int total = tl;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+  // CTAs of a row with tiles: ceil(g tiles / total), at least 1, at most one per IM_MIN_TILES tiles;
+  // with g = grid - rows the sum is at most (grid - rows) + rows (and grid >= rows)
+  auto share = [&](int g) {
+    if (tl == 0) return 0;
+    return max(1, min(int((int64_t(g) * tl + total - 1) / total), (tl + IM_MIN_TILES - 1) / IM_MIN_TILES));
+  };
+  int sp = share(a.grid), sum = sp;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (sum > a.grid) sp = share(max(0, a.grid - a.rows));
+  int incl = sp;
+  int64_t fincl = lane < a.rows ? max(0, a.n_out - tl * IM_TILE) : 0;
+  const int fill = int(fincl);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    const int64_t fy = __shfl_up_sync(0xffffffffu, fincl, o);
+    if (lane >= o) incl += y, fincl += fy;
+  }
+  const int c = int(blockIdx.x);
+  const unsigned own = __ballot_sync(0xffffffffu, sp > 0 && c >= incl - sp && c < incl);
+  Deal d;
+  d.row = -1, d.t0 = 0, d.t_end = 0;
+  if (own) {
+    const int r = __ffs(own) - 1;
+    const int spr = __shfl_sync(0xffffffffu, sp, r), tlr = __shfl_sync(0xffffffffu, tl, r);
+    const int part = c - (__shfl_sync(0xffffffffu, incl, r) - spr), ch = (tlr + spr - 1) / spr;
+    d.t0 = min(tlr, part * ch), d.t_end = min(tlr, d.t0 + ch);
+    if (d.t0 < d.t_end) d.row = r;
+  }
+  d.tiles = tl, d.fill = fill;
+  d.fill_pre = fincl - fill, d.fill_all = __shfl_sync(0xffffffffu, fincl, 31);
+  return d;
+}
+// The deal's tail figures kept in shared memory (the candidate-list space, which a full scan
+// does not use) from the prologue to the end of the epilogue: per row the positions past the
+// tiles of the rows before it, its own, its tiles; then the total.
+struct Tails {
+  int64_t pre[32];
+  int n[32], tiles[32];
+  int64_t all;
+};
+__device__ __forceinline__ void keep_tails(Tails *tz, const Deal &d, int lane) {  // one warp
+  tz->pre[lane] = d.fill_pre, tz->n[lane] = d.fill, tz->tiles[lane] = d.tiles;
+  if (lane == 0) tz->all = d.fill_all;
+}
+// This CTA's even share of the positions past the rows' visible tiles, written -inf by the
+// threads t = 0 .. nt-1.
+__device__ __forceinline__ void fill_tails(const IndexMmaArgs &a, const Tails *tz, int t, int nt) {
+  const int64_t G = gridDim.x, c = blockIdx.x;
+  const int64_t lo = tz->all * c / G, hi = tz->all * (c + 1) / G;
+  for (int r = 0; r < a.rows; ++r) {
+    const int64_t pre = tz->pre[r];
+    float *out = a.scores + int64_t(r) * a.n_out + int64_t(tz->tiles[r]) * IM_TILE;  // first position past its tiles
+    for (int64_t i = max(lo, pre) + t; i < min(hi, pre + tz->n[r]); i += nt) out[i - pre] = -INFINITY;
+  }
+}
 
 // A-operand row of tile entry e and the inverse map.
 __device__ __forceinline__ int row_of_entry(int e) { return (e & 3) * 32 + (e >> 2); }
@@ -240,16 +319,50 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   grid_dep_launch();  // a dependent attention launch may start its prologue
-  const int row = blockIdx.y, b = row / a.Q;
+  int row = blockIdx.y, t0 = blockIdx.x * a.chunk, t_end = t0 + a.chunk;
+  // The epilogue warps' query block and head weight go out first.  A balanced scan knows its row
+  // only from the deal, one round trip later: it loads the row it has when every row fills the
+  // output (the deal of equal rows) and loads again only if the deal says otherwise.
+  const int qt = int(threadIdx.x) - 64, qhd = qt >> 2, qg = qt & 3;
+  uint4 qv[4];
+  uint16_t w_raw = 0;
+  auto load_query = [&](int r) {
+    if (warp >= 2) {
+      w_raw = a.w[int64_t(r) * HI + qhd];
+      const uint16_t *qh = a.q_ix + (int64_t(r) * HI + qhd) * DI;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) qv[i] = reinterpret_cast<const uint4 *>(qh + 32 * qg)[i];
+    }
+  };
+  int row_q = row;
+  if constexpr (!SEL) {
+    if (a.grid > 0) row_q = a.spec > 0 ? min(a.rows - 1, int(blockIdx.x) / a.spec) : 0;
+  }
+  load_query(row_q);
+  Tails *tails = reinterpret_cast<Tails *>(smem + SM_CAND);
+  static_assert(sizeof(Tails) <= IM_CAND_TILES * IM_TILE * 4, "the deal's tails fit the candidate-list space");
+  if constexpr (!SEL) {
+    if (a.grid > 0) {  // balanced full scan: this CTA's row and tiles from the deal
+      const Deal d = deal_rows(a, lane);
+      if (warp == 0) keep_tails(tails, d, lane);
+      if (d.row < 0) {  // no tiles: only its share of the tails
+        __syncthreads();
+        fill_tails(a, tails, threadIdx.x, IM_THREADS);
+        return;
+      }
+      row = d.row, t0 = d.t0, t_end = d.t_end;
+      if (row != row_q) load_query(row);
+    }
+  }
+  const int b = row / a.Q;
   const int nvis = visible_entries(a.c, b, a.q_pos[row]);
   const int n_entries = a.c.num_entries[b];
   const int t_all = (a.n_out + IM_TILE - 1) / IM_TILE;
   const int t_work = a.cand ? (a.P + IM_TILE - 1) / IM_TILE : (nvis + IM_TILE - 1) / IM_TILE;
-  const int t0 = blockIdx.x * a.chunk;
-  const int t1 = min(t0 + a.chunk, t_all);
+  const int t1 = min(t_end, t_all);
   const int ntiles = max(0, min(t1, t_work) - t0);
   // a full scan whose output row is shorter than the visible entries would drop the tail
-  if (!a.cand && nvis > a.n_out && blockIdx.x == 0 && threadIdx.x == 0) report(a.err, CSA2_ERR_SHAPE);
+  if (!a.cand && nvis > a.n_out && t0 == 0 && threadIdx.x == 0) report(a.err, CSA2_ERR_SHAPE);
 
   // Candidate lists of at most IM_CAND_TILES tiles are copied to shared memory by warp 0
   // while the other warps run the prologue, so the producer and the epilogue never wait
@@ -363,12 +476,7 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
     // quantise the query heads: thread 4h + g owns 32-value block g of head h (8 of the epilogue
     // warps, idle until the first tile).  Dividing by the power-of-two scale 2^e is done as the
     // (exactly equal) product with 2^-e.
-    const int t = threadIdx.x - 64, h = t >> 2, g = t & 3;
-    const uint16_t w_raw = a.w[int64_t(row) * HI + h];  // loaded with the query block, used at the end
-    const uint16_t *qh = a.q_ix + (int64_t(row) * HI + h) * DI;
-    uint4 qv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) qv[i] = reinterpret_cast<const uint4 *>(qh + 32 * g)[i];
+    const int t = qt, h = qhd, g = qg;  // the query block and w_raw (used at the end) are in flight
     if (spread) {  // this warp's tile of a staged gather (every stage is still free), read from the list
       int32_t cv[4];  // loaded together with the query block
 #pragma unroll
@@ -538,8 +646,12 @@ __global__ void __launch_bounds__(IM_THREADS, 2) index_score_mma_kernel(const __
       }
     }
     if (spread) cp_async_wait<0>();  // no copy of this thread is left in flight
-    // positions past the visible entries (no key tile was loaded for them)
-    if (!a.cand) {
+    // positions past the visible entries (no key tile was loaded for them): in a balanced scan
+    // this CTA's share of every row's, else those of its own range
+    if constexpr (!SEL) {
+      if (a.grid > 0) fill_tails(a, tails, threadIdx.x - 64, 128 * IM_EPI_WG);
+    }
+    if (!a.cand && a.grid == 0) {
       const int lo = max(t0, t_work) * IM_TILE, hi = min(t1 * IM_TILE, a.n_out);
       for (int pos = lo + threadIdx.x - 64; pos < hi; pos += 128 * IM_EPI_WG)
         a.scores[int64_t(row) * a.n_out + pos] = -INFINITY;
@@ -601,14 +713,24 @@ void launch_index_score_mma(const uint16_t *q_ix, const uint16_t *w, int B, int 
   if (n_out == 0 || rows == 0) return;
   const int t_all = (n_out + IM_TILE - 1) / IM_TILE;
   const int want = (2 * sm_count() + rows - 1) / rows;   // about two CTAs per SM in total
-  const int min_tiles = cand ? 4 : 8;                     // short candidate lists: spread them wider
+  const int min_tiles = cand ? 4 : IM_MIN_TILES;          // short candidate lists: spread them wider
   const int splits = max(1, min(min(want, (t_all + min_tiles - 1) / min_tiles), 65535));
   const int chunk = (t_all + splits - 1) / splits;
   CUtensorMap tmap;
   memset(&tmap, 0, sizeof(tmap));
   const bool use_tma = cand == nullptr && make_index_code_map(&tmap, c);
   IndexMmaArgs a{use_tma, q_ix, w, Q, q_pos, cand, P, n_out, c, scores, err, chunk};
+  a.rows = rows;
   set_smem_limit(index_score_mma_kernel<false>, IM_SMEM_BYTES);
+  // A full scan of 2 to 32 rows deals the CTAs to the rows by their visible entries (a ragged
+  // batch keeps every SM streaming); for rows of equal length the deal is the (split, row) grid.
+  // One row keeps that grid, which already spreads it over every CTA, without the deal's round trip.
+  if (cand == nullptr && rows >= 2 && rows <= 32) {
+    a.grid = min(2 * sm_count(), rows * ((t_all + IM_MIN_TILES - 1) / IM_MIN_TILES));
+    a.spec = a.grid % rows == 0 ? a.grid / rows : 0;
+    index_score_mma_kernel<false><<<dim3(a.grid), IM_THREADS, IM_SMEM_BYTES, st>>>(tmap, a);
+    return;
+  }
   index_score_mma_kernel<false><<<dim3((t_all + chunk - 1) / chunk, rows), IM_THREADS, IM_SMEM_BYTES, st>>>(tmap, a);
 }
 
