@@ -146,6 +146,36 @@ def test_index_score_full_and_candidates():
         np.testing.assert_array_equal(got[b, 0, :650], full[b, 0, cn[b, 0, :650]])
 
 
+def test_index_score_full_ragged_rows():
+    """A Full scan of rows of very different lengths deals its CTAs to the rows by their visible
+    tiles and splits the -inf tails over all CTAs: every row's scores must still equal the
+    oracle's, with -inf from its visible entries to the end of a row longer than any sequence
+    (a row that sees nothing is all -inf)."""
+    k = K()
+    lengths = [257, 3001, 20000, 700, 129, 5000, 64]
+    spec = W.scaled(W.tiny_full(), lengths, B=len(lengths), q_len=3)   # 21 query rows
+    cache = gpu_cache(spec)
+    q, q_ix, w, q_pos = W.query_tensors(spec, 0, DEV)
+    q_pos = q_pos.clone()
+    q_pos[3, :] = -1                        # sees no entry
+    q_pos[1, 0] = 999                       # earlier queries of a longer sequence
+    q_pos[2, 1] = 4321
+    n_out = spec.max_entries + 777
+    err = _err()
+    s = k.csa2_index_score(q_ix, w, q_pos, cache, n_out, err=err)
+    assert k.csa2_check(err) == 0
+    assert s.shape[-1] == n_out
+    for b in range(len(lengths)):
+        c = oracle_seq(spec, b, main_rows=[], gen_device=DEV)
+        for qi in range(3):
+            nvis = c.visible(0, int(q_pos[b, qi])) if int(q_pos[b, qi]) >= 0 else 0
+            got = to_np(s[b, qi])
+            assert np.all(np.isneginf(got[nvis:])), (b, qi)
+            if nvis:
+                ref = OC.indexer_scores(to_np(q_ix[b, qi]), to_np(w[b, qi]), c.indexer_values(0, np.arange(nvis)))
+                np.testing.assert_allclose(got[:nvis], ref, rtol=2e-6, atol=2e-6 * np.abs(ref).max())
+
+
 def test_index_score_rejects_bad_candidates():
     k = K()
     spec = W.scaled(W.tiny_full(), [600], B=1)
